@@ -1,0 +1,54 @@
+"""Seeded synthetic inputs shared by the CUDA path's tests, the oracle tests and
+the benchmark.  This module holds no arithmetic of the method itself: it only
+draws tensors.
+
+Recipe (the Swin-shaped synthetic workloads of the FlashSwin evaluation,
+thelatestinai.com/papers/2610.04664, Table S1 and Figure S1 shapes):
+  * Q, K, V, dO: bf16 draws of N(0, 1) on a [B, H, W, heads, d] grid from
+    torch generators seeded 0, 1, 2, 3; optionally Q and K scaled by a constant
+    (the high-resolution stress case sharpens the softmax with a factor 3);
+  * theta: fp32 [heads, 2, d/4], the geometric RoPE schedule
+    100 ** (-2 i / (d / 2)), i = 0 .. d/4 - 1, repeated for both axes and every
+    head (the initialisation the pages call "the standard geometric RoPE
+    schedule", Figure S4), plus N(0, 0.01) noise from a generator seeded 4.
+"""
+from __future__ import annotations
+
+import torch
+
+SEED_Q, SEED_K, SEED_V, SEED_DO, SEED_THETA = 0, 1, 2, 3, 4
+
+
+def _normal(shape, seed: int, device, scale: float = 1.0) -> torch.Tensor:
+    g = torch.Generator(device=device)
+    g.manual_seed(seed)
+    x = torch.randn(shape, generator=g, device=device, dtype=torch.float32)
+    if scale != 1.0:
+        x.mul_(scale)
+    return x.to(torch.bfloat16)
+
+
+def theta_init(heads: int, d: int, device="cpu", noise: float = 0.01, seed: int = SEED_THETA) -> torch.Tensor:
+    q = d // 4
+    i = torch.arange(q, dtype=torch.float64)
+    base = (100.0 ** (-2.0 * i / (d / 2))).to(torch.float32)
+    th = base.repeat(heads, 2, 1).contiguous()
+    if noise:
+        g = torch.Generator(device="cpu")
+        g.manual_seed(seed)
+        th = th + noise * torch.randn(th.shape, generator=g, dtype=torch.float32)
+    return th.to(device)
+
+
+def make_inputs(B: int, H: int, W: int, heads: int, d: int, device="cpu", qk_scale: float = 1.0,
+                with_dout: bool = True) -> dict:
+    shape = (B, H, W, heads, d)
+    out = {
+        "q": _normal(shape, SEED_Q, device, qk_scale),
+        "k": _normal(shape, SEED_K, device, qk_scale),
+        "v": _normal(shape, SEED_V, device),
+        "theta": theta_init(heads, d, device),
+    }
+    if with_dout:
+        out["dout"] = _normal(shape, SEED_DO, device)
+    return out
