@@ -1,0 +1,416 @@
+#!/usr/bin/env python
+"""Benchmark of fused windowed-RoPE attention (forward + backward) on B200.
+
+One step = one pass of the whole hot path over one batch: forward and
+backward at every shift of the workload (the Swin-T stage-1 shape at p=4,
+M=8 runs an unshifted and a shifted block, s=0 and s=4).  Inputs are seeded
+synthetic bf16 N(0,1) tensors of the workload's shape (the pages measure on
+ImageNet at 256x256; no dataset is used).
+
+Prints ONE JSON line (rank 0).  `--impl reference` times the fp64 CPU oracle
+instead, on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "windowed-RoPE attention fwd+bwd TFLOP/s (% BF16 peak), tokens/s, peak GB"
+HEAD_DIM = 32
+
+WORKLOADS = {
+    # Swin-T stage-1 shape at p=4 (64x64 grid at 256x256 input), window 8, unshifted and shifted blocks
+    "swin_t_stage1_p4_m8": dict(B=128, H=64, W=64, heads=3, M=8, shifts=(0, 4), qk_scale=1.0),
+    # FlashSwin-T stage 1 at p=2 (128x128 grid), window 32, shifted block
+    "flashswin_t_stage1_p2_m32": dict(B=128, H=128, W=128, heads=3, M=32, shifts=(16,), qk_scale=1.0),
+    # 512x512 input at p=2, window 64 (4096-token windows), Q and K scaled by 3
+    "highres_p2_m64": dict(B=16, H=256, W=256, heads=3, M=64, shifts=(32,), qk_scale=3.0),
+}
+HEADLINE = "swin_t_stage1_p4_m8"
+
+
+def unmasked_pairs(B, H, W, heads, M, s) -> int:
+    """Number of (query, key) pairs that attend (same window, same shift-region label)."""
+    def sizes(X):
+        if s == 0:
+            return [[M]] * (X // M)
+        out = [[M]] * (X // M - 1)
+        out.append([M - s, s])  # last window row/column: two regions of the shifted grid
+        return out
+    rows, cols = sizes(H), sizes(W)
+    per_image = 0
+    for rr in rows:
+        for cc in cols:
+            per_image += sum((a * b) ** 2 for a in rr for b in cc)
+    return per_image * B * heads
+
+
+def workload_flops(wl) -> tuple[float, float]:
+    """Useful forward and backward FLOPs of one step (fwd 4*d per pair, bwd 10*d per pair)."""
+    pairs = sum(unmasked_pairs(wl["B"], wl["H"], wl["W"], wl["heads"], wl["M"], s) for s in wl["shifts"])
+    return 4.0 * HEAD_DIM * pairs, 10.0 * HEAD_DIM * pairs
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return {"hbm_gbs": float(p["hbm_gbs"]), "bf16_tflops": float(p["bf16_tflops"]),
+                "bf16_tflops_sustained": float(p.get("bf16_tflops_sustained", p["bf16_tflops"])),
+                "source": "measured"}
+    except Exception:
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+class ClockSampler:
+    """nvidia-smi clock/throttle samples during the timed region."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except Exception:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sm, mx, reasons = [], 0.0, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = max(mx, float(parts[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def cpu_baseline(tensors, wl, seconds: float = 12.0):
+    """Times the fp64 oracle (forward + backward) on host cores over a bounded
+    sample of the workload's (batch, window, head) units at its last shift."""
+    import numpy as np
+
+    import oracle
+    B, H, W, heads, M = wl["B"], wl["H"], wl["W"], wl["heads"], wl["M"]
+    s = wl["shifts"][-1]
+    nW = (H // M) * (W // M)
+    n_units = B * nW * heads
+    cores = oracle.default_threads()
+    # units spread over the batch, including windows of the last row/column
+    t0 = time.perf_counter()
+    probe = np.arange(0, min(n_units, 4 * cores))
+    oracle.units(tensors["q"], tensors["k"], tensors["v"], tensors["theta"], M, s, probe, dout=tensors["dout"],
+                 nthreads=cores)
+    dt = max(time.perf_counter() - t0, 1e-6)
+    n = int(min(n_units, max(len(probe), len(probe) * seconds / dt)))
+    ids = np.linspace(0, n_units - 1, n).astype(np.int64)
+    t0 = time.perf_counter()
+    oracle.units(tensors["q"], tensors["k"], tensors["v"], tensors["theta"], M, s, ids, dout=tensors["dout"],
+                 nthreads=cores)
+    dt = time.perf_counter() - t0
+    # useful flops of the sampled units (pairs that attend)
+    pairs_all = unmasked_pairs(B, H, W, heads, M, s)
+    flops = 14.0 * HEAD_DIM * pairs_all * (n / n_units)
+    return {"value": flops / dt / 1e12, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+            "sample": f"{n} of {n_units} (batch, window, head) units at s={s}, fwd+bwd, fp64, {dt:.1f} s",
+            "seconds": dt}
+
+
+def run_reference(args):
+    """The fp64 CPU oracle as the reference arm (rank 0 only)."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    import torch
+
+    from vision_transformer_windowed_b200.inputs import make_inputs
+    wl = WORKLOADS[args.workload]
+    t = make_inputs(wl["B"], wl["H"], wl["W"], wl["heads"], HEAD_DIM, device="cpu", qk_scale=wl["qk_scale"])
+    per_step = max(1.0, args.reference_seconds / max(1, args.steps + args.warmup))
+    for _ in range(args.warmup):
+        cpu_baseline(t, wl, seconds=per_step)
+    vals, secs, last = [], 0.0, None
+    for _ in range(args.steps):
+        last = cpu_baseline(t, wl, seconds=per_step)
+        vals.append(last["value"])
+        secs += last["seconds"]
+    value = statistics.mean(vals)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": secs / args.steps * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": args.workload, **{k: v for k, v in wl.items() if k != "shifts"},
+                   "shifts": list(wl["shifts"]), "d": HEAD_DIM},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": last["cores"], "kind": "oracle",
+                         "sample": last["sample"] + " per step"},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    del torch
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="fswin", choices=["fswin", "reference"])
+    ap.add_argument("--workload", default=HEADLINE, choices=sorted(WORKLOADS))
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extra", action="store_true", help="skip the per-config numbers of the other workloads")
+    ap.add_argument("--reference-seconds", type=float, default=60.0)
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+    if args.impl == "reference":
+        run_reference(args)
+        return
+
+    import torch
+    import torch.distributed as dist
+
+    from vision_transformer_windowed_b200 import _lib, ops
+    from vision_transformer_windowed_b200.inputs import make_inputs
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    _lib.load()
+    peaks = load_peaks()
+
+    def barrier():
+        if world > 1:
+            dist.barrier(device_ids=[local])
+
+    def run_workload(name, steps, warmup, phase=True, clocks=False):
+        wl = WORKLOADS[name]
+        B, H, W, heads, M = wl["B"], wl["H"], wl["W"], wl["heads"], wl["M"]
+        t = make_inputs(B, H, W, heads, HEAD_DIM, device=dev, qk_scale=wl["qk_scale"])
+        q, k, v, th, do = t["q"], t["k"], t["v"], t["theta"], t["dout"]
+        outs = {s: (torch.empty_like(q), torch.empty((B, H, W, heads), device=dev, dtype=torch.float32))
+                for s in wl["shifts"]}
+        grads = {s: (torch.empty_like(q), torch.empty_like(q), torch.empty_like(q), torch.empty_like(th))
+                 for s in wl["shifts"]}
+        ws = ops.alloc_workspace(q, M, wl["shifts"][0])
+
+        def step(evs=None):
+            for si, s in enumerate(wl["shifts"]):
+                o, lse = outs[s]
+                dq, dk, dv, dth = grads[s]
+                if evs is not None:
+                    _lib.fs_set_phase_events([e.cuda_event for e in evs[si][0]])
+                ops.winattn_fwd(q, k, v, th, M, s, o=o, lse=lse)
+                if evs is not None:
+                    _lib.fs_set_phase_events([e.cuda_event for e in evs[si][1]])
+                ops.winattn_bwd(q, k, v, o, do, lse, th, M, s, workspace=ws, dq=dq, dk=dk, dv=dv, dtheta=dth)
+                if world > 1:
+                    dist.all_reduce(dth)  # theta is shared by the whole data-parallel batch
+            if evs is not None:
+                _lib.fs_set_phase_events([])
+
+        for _ in range(warmup):
+            step()
+        torch.cuda.synchronize()
+        torch.cuda.reset_peak_memory_stats(dev)
+        evsets = None
+        if phase:
+            evsets = [[([torch.cuda.Event(enable_timing=True) for _ in range(2)],
+                        [torch.cuda.Event(enable_timing=True) for _ in range(5)]) for _ in wl["shifts"]]
+                      for _ in range(steps)]
+            for stp in evsets:  # torch creates the CUDA event on first record
+                for fe, be in stp:
+                    for e in fe + be:
+                        e.record()
+            torch.cuda.synchronize()
+        sampler = ClockSampler(local) if clocks else None
+        barrier()
+        torch.cuda.synchronize()
+        if sampler:
+            sampler.start()
+            time.sleep(0.4)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for i in range(steps):
+            step(evsets[i] if evsets else None)
+        e1.record()
+        torch.cuda.synchronize()
+        barrier()
+        clk = sampler.stop() if sampler else None
+        ms = e0.elapsed_time(e1) / steps
+        if world > 1:
+            tm = torch.tensor([ms], device=dev)
+            dist.all_reduce(tm, op=dist.ReduceOp.MAX)
+            ms = float(tm.item())
+        assert _lib.fs_device_status() == 0, "a kernel reported a device-side failure"
+        peak_gb = torch.cuda.max_memory_allocated(dev) / 1e9
+        fwd_f, bwd_f = workload_flops(wl)
+        tokens = B * H * W * len(wl["shifts"])
+        res = {"ms": ms, "tflops": (fwd_f + bwd_f) * world / (ms * 1e-3) / 1e12,
+               "tokens_per_s": tokens * world / (ms * 1e-3), "peak_gb": peak_gb,
+               "fwd_flops": fwd_f, "bwd_flops": bwd_f, "clocks": clk, "ws_bytes": ws.numel()}
+        if evsets:
+            names = ["fwd", "bwd_prep", "bwd_main", "bwd_post", "bwd_dtheta"]
+            tot = {n: 0.0 for n in names}
+            for stp in evsets:
+                for fe, be in stp:
+                    tot["fwd"] += fe[0].elapsed_time(fe[1])
+                    for j in range(4):
+                        tot[names[1 + j]] += be[j].elapsed_time(be[j + 1])
+            launches = steps * len(wl["shifts"])
+            res["phase_ms"] = {n: tot[n] / launches for n in names}  # average per launch
+            res["phase_share"] = {n: tot[n] / max(sum(tot.values()), 1e-9) for n in names}
+            res["launches_per_kernel"] = launches
+        res["tensors"] = t
+        return res
+
+    main_res = run_workload(args.workload, args.steps, args.warmup, phase=True, clocks=True)
+    wl = WORKLOADS[args.workload]
+    B, H, W, heads, M = wl["B"], wl["H"], wl["W"], wl["heads"], wl["M"]
+    nshift = len(wl["shifts"])
+
+    # roofline of the dominant kernel (largest share of the step)
+    ph = main_res["phase_ms"]
+    dom = max(ph, key=lambda n: main_res["phase_share"][n])
+    th = B * H * W * heads
+    pairs_per_launch = (main_res["fwd_flops"] / (4.0 * HEAD_DIM)) / nshift
+    algo_bytes = {"fwd": 260, "bwd_prep": 588, "bwd_main": 456, "bwd_post": 512, "bwd_dtheta": 0}
+    hbm_bound = M <= 8
+    if hbm_bound or dom in ("bwd_prep", "bwd_post", "bwd_dtheta"):
+        achieved = algo_bytes[dom] * th / (ph[dom] * 1e-3) / 1e9
+        roof = {"kernel": dom, "bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": achieved / peaks["hbm_gbs"], "traffic": None,
+                "algorithmic_bytes_per_launch": algo_bytes[dom] * th,
+                "peak_note": f"HBM copy bandwidth, {peaks['source']}"}
+    else:
+        fl = (4.0 if dom == "fwd" else 10.0) * HEAD_DIM * pairs_per_launch
+        achieved = fl / (ph[dom] * 1e-3) / 1e12
+        roof = {"kernel": dom, "bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"],
+                "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops"], "traffic": None,
+                "algorithmic_flops_per_launch": fl, "peak_note": f"cuBLAS bf16 burst, {peaks['source']}"}
+    roof["avg_launch_ms"] = ph[dom]
+
+    # end to end through the public API with host buffers (pinned), copies inside the timed region
+    t = main_res["tensors"]
+    host = {k: t[k].cpu().pin_memory() for k in ("q", "k", "v", "dout", "theta")}
+    res_host = {}
+    e2e_steps = max(1, min(args.steps, 5))
+    torch.cuda.synchronize()
+    h2d = sum(x.numel() * x.element_size() for x in host.values())
+    d2h = 0
+
+    def e2e_step():
+        nonlocal d2h
+        d2h = 0
+        dv = {k: x.to(dev, non_blocking=True) for k, x in host.items()}
+        for s in wl["shifts"]:
+            o, lse = ops.winattn_fwd(dv["q"], dv["k"], dv["v"], dv["theta"], M, s)
+            dq, dk, dvv, dth = ops.winattn_bwd(dv["q"], dv["k"], dv["v"], o, dv["dout"], lse, dv["theta"], M, s)
+            if world > 1:
+                dist.all_reduce(dth)
+            for name, x in (("o", o), ("dq", dq), ("dk", dk), ("dv", dvv), ("dtheta", dth)):
+                key = (s, name)
+                if key not in res_host:
+                    res_host[key] = torch.empty(x.shape, dtype=x.dtype, pin_memory=True)
+                res_host[key].copy_(x, non_blocking=True)
+                d2h += x.numel() * x.element_size()
+
+    e2e_step()
+    torch.cuda.synchronize()
+    barrier()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(e2e_steps):
+        e2e_step()
+    b.record()
+    torch.cuda.synchronize()
+    e2e_ms = a.elapsed_time(b) / e2e_steps
+    if world > 1:
+        tm = torch.tensor([e2e_ms], device=dev)
+        dist.all_reduce(tm, op=dist.ReduceOp.MAX)
+        e2e_ms = float(tm.item())
+    fl = main_res["fwd_flops"] + main_res["bwd_flops"]
+    e2e = {"value": fl * world / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s", "ms_per_step": e2e_ms,
+           "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+
+    per_config = {args.workload: {"tflops": main_res["tflops"], "ms_per_step": main_res["ms"],
+                                  "pct_bf16_peak": 100 * main_res["tflops"] / peaks["bf16_tflops"] / world,
+                                  "tokens_per_s": main_res["tokens_per_s"], "peak_gb": main_res["peak_gb"],
+                                  "phase_ms": main_res["phase_ms"]}}
+    del main_res["tensors"], t, host, res_host
+    if not args.no_extra:
+        for name in WORKLOADS:
+            if name == args.workload:
+                continue
+            torch.cuda.empty_cache()
+            r = run_workload(name, max(3, args.steps // 2), 3, phase=True, clocks=False)
+            del r["tensors"]
+            per_config[name] = {"tflops": r["tflops"], "ms_per_step": r["ms"],
+                                "pct_bf16_peak": 100 * r["tflops"] / peaks["bf16_tflops"] / world,
+                                "tokens_per_s": r["tokens_per_s"], "peak_gb": r["peak_gb"],
+                                "phase_ms": r["phase_ms"], "bwd_workspace_gb": r["ws_bytes"] / 1e9}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        tt = make_inputs(B, H, W, heads, HEAD_DIM, device="cpu", qk_scale=wl["qk_scale"])
+        cpu = cpu_baseline(tt, wl)
+        cpu.pop("seconds", None)
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": main_res["tflops"], "unit": "TFLOP/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": main_res["ms"], "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": args.workload, "B_per_gpu": B, "H": H, "W": W, "heads": heads, "d": HEAD_DIM,
+                       "M": M, "shifts": list(wl["shifts"]), "qk_scale": wl["qk_scale"],
+                       "step": "fwd+bwd at every shift", "parallelism": f"dp{world}",
+                       "l2": "inputs larger than L2 (each tensor > 126 MB)"},
+            "pct_bf16_peak": 100 * main_res["tflops"] / peaks["bf16_tflops"] / world,
+            "tokens_per_s": main_res["tokens_per_s"], "peak_gb": main_res["peak_gb"],
+            "gpu_launches": args.steps * nshift * 5,
+            "roofline": roof, "clocks": main_res["clocks"], "e2e": e2e, "cpu_baseline": cpu,
+            "per_config": per_config, "peaks": peaks,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,139 @@
+/*
+ * fswin — fused Swin windowed self-attention with window-local learnable 2D RoPE
+ * on B200 (sm_100a): forward and backward behind a plain C ABI.
+ *
+ * The operation is the one the FlashSwin paper introduces ("FLASHSWIN: Unlocking
+ * Large Windows and Dense Tokens in Swin Vision Transformers with Memory Efficient
+ * Attention"; arxivdaily.com/papers/2610.04664, English abstract; and
+ * thelatestinai.com/papers/2610.04664, Figure 1B and Figure S4): exact softmax
+ * attention inside every M x M window of a cyclically shifted token grid, computed
+ * without materialising the M^2 x M^2 score matrix, with queries and keys rotated
+ * by a window-local 2D RoPE whose inverse frequencies theta are learnable.
+ *
+ * Conventions (readings of the paper where it is silent):
+ *  - tensors q, k, v, o, dout, dq, dk, dv are bf16, contiguous [B, H, W, heads, d]
+ *    (d = 32), 16-byte aligned, in DEVICE memory;
+ *  - theta and dtheta are fp32 [heads, 2, d/4]; axis 0 (x) rotates channel pairs
+ *    (2k, 2k+1) of the first d/2 channels by j * theta[h][0][k], axis 1 (y) the pairs
+ *    of the last d/2 channels by i * theta[h][1][k], where (i, j) is the token's
+ *    row and column inside its window (0 .. M-1, in the rolled frame);
+ *  - the shift takes rolled token (r, c) from original position ((r+s) mod H,
+ *    (c+s) mod W); outputs are written back at original positions;
+ *  - with s > 0 a query attends a key of its window only when both carry the same
+ *    Swin shift-region label, built from the row/column slices [0, H-M),
+ *    [H-M, H-s), [H-s, H); masked scores are -infinity;
+ *  - softmax scale 1/sqrt(d); lse is the natural-log log-sum-exp per query, fp32
+ *    [B, H, W, heads];
+ *  - gradients are those of sum(o * dout).
+ *
+ * Ownership and ordering: the caller owns every buffer.  The library never
+ * allocates device memory and never synchronises; all work is enqueued on the
+ * given stream (a cudaStream_t; NULL is the legacy default stream).
+ *
+ * Errors: invalid arguments return a status and launch nothing.  A kernel whose
+ * internal wait runs past its time limit stops and records FS_ERR_TIMEOUT in a
+ * device status word that fs_device_status() reads (after the stream is
+ * synchronised by the caller).
+ */
+#ifndef FSWIN_H
+#define FSWIN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define FS_API __attribute__((visibility("default")))
+#else
+#define FS_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    FS_OK = 0,
+    FS_ERR_NULL = 1,      /* a required pointer is NULL */
+    FS_ERR_SHAPE = 2,     /* unsupported or inconsistent shape (see fs_winattn_shape) */
+    FS_ERR_ALIGN = 3,     /* a pointer is not 16-byte aligned */
+    FS_ERR_WORKSPACE = 4, /* workspace missing, misaligned or too small */
+    FS_ERR_CUDA = 5,      /* a CUDA runtime/driver call failed */
+    FS_ERR_TIMEOUT = 6,   /* a device-side wait ran out of time */
+    FS_ERR_ARCH = 7       /* the current device is not sm_100 */
+} fs_status;
+
+/*
+ * Problem shape.  Supported: d == 32; M in {4, 8, 16, 32, 64}; H and W multiples
+ * of M; 0 <= s < M with s a multiple of 4; heads >= 1; B >= 0 (B == 0 is a valid
+ * empty problem).  Anything else returns FS_ERR_SHAPE.
+ */
+typedef struct {
+    int B, H, W, heads, d, M, s;
+} fs_winattn_shape;
+
+typedef struct CUstream_st* fs_stream_t; /* same type as cudaStream_t */
+
+/* Returns FS_OK when the shape is supported, without touching the device. */
+FS_API fs_status fs_winattn_check_shape(const fs_winattn_shape* shape);
+
+/*
+ * Forward.  In: q, k, v (bf16 [B,H,W,heads,d]), theta (fp32 [heads,2,d/4]).
+ * Out: o (bf16 [B,H,W,heads,d]) and lse (fp32 [B,H,W,heads]); both overwritten.
+ * Exact softmax attention per window (FlashSwin abstract: "exact softmax
+ * attention without materializing the score matrix").
+ */
+FS_API fs_status fs_winattn_fwd(const fs_winattn_shape* shape, const void* q, const void* k, const void* v,
+                         const float* theta, void* o, float* lse, fs_stream_t stream);
+
+/*
+ * Workspace the backward needs, in bytes.  It depends on B*H*W*heads only, not on
+ * the window size M (memory flat in M, FlashSwin Table S1).
+ */
+FS_API size_t fs_winattn_bwd_workspace_bytes(const fs_winattn_shape* shape);
+
+/*
+ * Backward (recompute-based: the probabilities are rebuilt from lse, never stored).
+ * In: q, k, v, o (the forward output), dout, lse, theta.  Out: dq, dk, dv (bf16
+ * [B,H,W,heads,d]) and dtheta (fp32 [heads,2,d/4]); all overwritten.  workspace:
+ * device scratch of at least fs_winattn_bwd_workspace_bytes(shape) bytes, 256-byte
+ * aligned; its contents on entry are ignored.
+ */
+FS_API fs_status fs_winattn_bwd(const fs_winattn_shape* shape, const void* q, const void* k, const void* v,
+                         const void* o, const void* dout, const float* lse, const float* theta, void* dq,
+                         void* dk, void* dv, float* dtheta, void* workspace, size_t workspace_bytes,
+                         fs_stream_t stream);
+
+/* Human-readable name of a status. */
+FS_API const char* fs_status_string(fs_status status);
+
+/*
+ * Reads and clears the device status word of the current device.  *code receives 0
+ * when no kernel reported a failure, else (status << 24) | where.  Synchronous.
+ */
+FS_API fs_status fs_device_status(unsigned int* code);
+
+/* Time limit of every device-side wait, in nanoseconds (default 10 s). */
+FS_API fs_status fs_set_wait_limit_ns(uint64_t limit_ns);
+
+/*
+ * Self-test of the bounded-wait path: launches one CTA that waits on a barrier no
+ * thread ever arrives on, with the given limit.  Afterwards (stream synchronised)
+ * fs_device_status() reports FS_ERR_TIMEOUT.  The GPU context stays usable.
+ */
+FS_API fs_status fs_selftest_bounded_wait(uint64_t limit_ns, fs_stream_t stream);
+
+/*
+ * Profiling hook.  events: `n` caller-created cudaEvent_t handles (as void*), or
+ * n == 0 to switch the hook off.  While set, fs_winattn_fwd records events[0]
+ * before and events[1] after its kernel (n >= 2), and fs_winattn_bwd records
+ * events[0] before its first kernel and events[1 + i] after its kernel i
+ * (prep, main, post, dtheta reduction; n >= 5), on the call's stream.  The
+ * handles are kept by value; the hook is process-wide and not thread-safe.
+ */
+FS_API fs_status fs_set_phase_events(void* const* events, int n);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FSWIN_H */

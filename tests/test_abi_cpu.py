@@ -1,0 +1,93 @@
+"""Host-side checks of the C ABI: the library loads, exports every entry point
+declared in include/fswin.h, and validates arguments without launching work
+(these calls return before touching any device)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from vision_transformer_windowed_b200 import _lib
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared_functions():
+    text = open(os.path.join(ROOT, "include", "fswin.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(fs_[a-z_0-9]+)\s*\(", text)))
+
+
+def test_library_exports_every_declared_symbol():
+    lib = _lib.load()
+    names = _declared_functions()
+    assert "fs_winattn_fwd" in names and "fs_winattn_bwd" in names
+    for n in names:
+        assert hasattr(lib, n), n
+        assert ctypes.cast(getattr(lib, n), ctypes.c_void_p).value
+
+
+def test_status_strings():
+    for code, name in enumerate(_lib.STATUS_NAMES):
+        assert _lib.status_string(code).startswith(name)
+
+
+GOOD = [(1, 16, 16, 2, 32, 8, 0), (128, 64, 64, 3, 32, 8, 4), (128, 128, 128, 3, 32, 32, 16),
+        (16, 256, 256, 3, 32, 64, 32), (128, 16, 16, 24, 32, 16, 0), (0, 16, 16, 2, 32, 8, 0),
+        (2, 8, 24, 1, 32, 4, 0), (1, 32, 32, 1, 32, 32, 0)]
+BAD = [(1, 16, 16, 2, 64, 8, 0),    # d != 32
+       (1, 16, 16, 2, 32, 12, 0),   # M not supported
+       (1, 20, 16, 2, 32, 8, 0),    # H % M
+       (1, 16, 20, 2, 32, 8, 0),    # W % M
+       (1, 16, 16, 2, 32, 8, 8),    # s >= M
+       (1, 16, 16, 2, 32, 8, 2),    # s % 4
+       (1, 16, 16, 2, 32, 8, -4),   # s < 0
+       (-1, 16, 16, 2, 32, 8, 0),   # B < 0
+       (1, 16, 16, 0, 32, 8, 0),    # heads
+       (1, 4, 4, 1, 32, 8, 0)]      # grid smaller than a window
+
+
+@pytest.mark.parametrize("shape", GOOD)
+def test_supported_shapes(shape):
+    assert _lib.fs_winattn_check_shape(_lib.make_shape(*shape)) == _lib.FS_OK
+
+
+@pytest.mark.parametrize("shape", BAD)
+def test_rejected_shapes(shape):
+    sh = _lib.make_shape(*shape)
+    assert _lib.fs_winattn_check_shape(sh) == _lib.FS_ERR_SHAPE
+    assert _lib.fs_winattn_bwd_workspace_bytes(sh) == 0
+    with pytest.raises(_lib.FswinError) as e:
+        _lib.fs_winattn_fwd(sh, 16, 16, 16, 16, 16, 16, 0)
+    assert e.value.status == _lib.FS_ERR_SHAPE
+
+
+def test_null_and_alignment_rejected_before_launch():
+    sh = _lib.make_shape(1, 16, 16, 2, 32, 8, 0)
+    with pytest.raises(_lib.FswinError) as e:
+        _lib.fs_winattn_fwd(sh, 0, 16, 16, 16, 16, 16, 0)
+    assert e.value.status == _lib.FS_ERR_NULL
+    with pytest.raises(_lib.FswinError) as e:
+        _lib.fs_winattn_fwd(sh, 24, 16, 16, 16, 16, 16, 0)
+    assert e.value.status == _lib.FS_ERR_ALIGN
+    n = _lib.fs_winattn_bwd_workspace_bytes(sh)
+    with pytest.raises(_lib.FswinError) as e:
+        _lib.fs_winattn_bwd(sh, *([256] * 11), 256, n - 1, 0)
+    assert e.value.status == _lib.FS_ERR_WORKSPACE
+    with pytest.raises(_lib.FswinError) as e:
+        _lib.fs_winattn_bwd(sh, *([256] * 11), 128, n, 0)   # misaligned workspace
+    assert e.value.status == _lib.FS_ERR_WORKSPACE
+    with pytest.raises(_lib.FswinError) as e:
+        _lib.fs_winattn_bwd(sh, *([256] * 10), 0, 256, n, 0)  # dtheta NULL
+    assert e.value.status == _lib.FS_ERR_NULL
+
+
+def test_workspace_flat_in_window_size():
+    """Backward scratch depends on the token count only, not on M (memory flat in M)."""
+    a = _lib.fs_winattn_bwd_workspace_bytes(_lib.make_shape(16, 256, 256, 3, 32, 32, 16))
+    b = _lib.fs_winattn_bwd_workspace_bytes(_lib.make_shape(16, 256, 256, 3, 32, 64, 32))
+    c = _lib.fs_winattn_bwd_workspace_bytes(_lib.make_shape(16, 256, 256, 3, 32, 8, 4))
+    assert a == b == c > 0
+    # and linear in the number of tokens
+    d = _lib.fs_winattn_bwd_workspace_bytes(_lib.make_shape(32, 256, 256, 3, 32, 32, 16))
+    assert abs(d - 2 * a) < 4096

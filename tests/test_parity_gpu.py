@@ -1,0 +1,111 @@
+"""GPU parity: the CUDA path (through the C ABI) against the fp64 oracle.
+
+Tolerances (bf16 inputs/outputs, fp32 accumulation):
+  forward outputs (o, lse):   max|err| <= 1e-2 * max|ref| + 2e-3
+  gradients (dq, dk, dv, dθ): max|err| <= 3e-2 * max|ref| + 5e-3
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from vision_transformer_windowed_b200 import _lib, ops
+from vision_transformer_windowed_b200.inputs import make_inputs
+
+FWD_TOL = (1e-2, 2e-3)
+GRAD_TOL = (3e-2, 5e-3)
+
+
+def check(name, got, ref, tol):
+    got = got.detach().float().cpu().numpy() if isinstance(got, torch.Tensor) else np.asarray(got)
+    got = got.astype(np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    assert got.shape == ref.shape, name
+    assert np.isfinite(got).all(), f"{name}: non-finite values"
+    err = np.abs(got - ref).max() if got.size else 0.0
+    bound = tol[0] * (np.abs(ref).max() if ref.size else 0.0) + tol[1]
+    assert err <= bound, f"{name}: max|err| {err:.4g} > {bound:.4g}"
+
+
+@pytest.fixture(autouse=True)
+def _device_status_clean():
+    _lib.fs_set_wait_limit_ns(4_000_000_000)
+    _lib.fs_device_status()  # clear
+    yield
+    torch.cuda.synchronize()
+    assert _lib.fs_device_status() == 0
+
+
+def run_both(B, H, W, h, M, s, qk_scale=1.0):
+    inp = make_inputs(B, H, W, h, 32, qk_scale=qk_scale)
+    dev = {k: v.cuda() for k, v in inp.items()}
+    o, lse = ops.winattn_fwd(dev["q"], dev["k"], dev["v"], dev["theta"], M, s)
+    dq, dk, dv, dth = ops.winattn_bwd(dev["q"], dev["k"], dev["v"], o, dev["dout"], lse, dev["theta"], M, s)
+    torch.cuda.synchronize()
+    ref = oracle.full(inp["q"], inp["k"], inp["v"], inp["theta"], M, s, dout=inp["dout"])
+    return {"o": o, "lse": lse, "dq": dq, "dk": dk, "dv": dv, "dtheta": dth}, ref
+
+
+SMALL = [  # (B, H, W, heads, M, s)
+    (1, 16, 16, 2, 8, 0),     # the tiny configuration: 4 windows of 64 tokens
+    (2, 16, 16, 3, 8, 4),     # shifted, 4x4 boxes
+    (1, 8, 24, 1, 8, 4),      # 3 windows: ragged last tile
+    (1, 8, 12, 2, 4, 0),      # 16-token windows, ragged
+    (1, 32, 32, 2, 16, 8),
+    (1, 32, 48, 1, 16, 4),
+    (1, 64, 64, 1, 32, 16),   # FlashSwin-T stage-1 window, shifted
+    (2, 32, 32, 2, 32, 0),    # one window per image
+    (1, 64, 64, 1, 64, 32),   # 4096-token window
+    (1, 64, 96, 1, 32, 12),
+]
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("cfg", SMALL)
+def test_fwd_bwd_parity(cfg):
+    got, ref = run_both(*cfg)
+    check("o", got["o"], ref["o"], FWD_TOL)
+    check("lse", got["lse"], ref["lse"], FWD_TOL)
+    for key in ("dq", "dk", "dv", "dtheta"):
+        check(key, got[key], ref[key], GRAD_TOL)
+
+
+@pytest.mark.gpu
+def test_sharp_softmax_parity():
+    """Q, K scaled by 3 (the high-resolution stress recipe) sharpen the softmax."""
+    got, ref = run_both(1, 64, 64, 1, 32, 16, qk_scale=3.0)
+    check("o", got["o"], ref["o"], FWD_TOL)
+    check("lse", got["lse"], ref["lse"], FWD_TOL)
+    for key in ("dq", "dk", "dv", "dtheta"):
+        check(key, got[key], ref[key], GRAD_TOL)
+
+
+@pytest.mark.gpu
+def test_empty_batch():
+    inp = make_inputs(0, 16, 16, 2, 32)
+    dev = {k: v.cuda() for k, v in inp.items()}
+    o, lse = ops.winattn_fwd(dev["q"], dev["k"], dev["v"], dev["theta"], 8, 0)
+    dth = torch.full_like(dev["theta"], 7.0)
+    ops.winattn_bwd(dev["q"], dev["k"], dev["v"], o, dev["dout"], lse, dev["theta"], 8, 0, dtheta=dth)
+    torch.cuda.synchronize()
+    assert o.numel() == 0 and (dth == 0).all()
+
+
+@pytest.mark.gpu
+def test_forward_is_deterministic():
+    inp = make_inputs(2, 32, 32, 2, 32)
+    dev = {k: v.cuda() for k, v in inp.items()}
+    o1, l1 = ops.winattn_fwd(dev["q"], dev["k"], dev["v"], dev["theta"], 16, 8)
+    o2, l2 = ops.winattn_fwd(dev["q"], dev["k"], dev["v"], dev["theta"], 16, 8)
+    assert torch.equal(o1, o2) and torch.equal(l1, l2)
+
+
+@pytest.mark.gpu
+def test_bounded_wait_reports_timeout_and_context_survives():
+    stream = torch.cuda.current_stream().cuda_stream
+    _lib.fs_selftest_bounded_wait(50_000_000, stream)
+    torch.cuda.synchronize()
+    code = _lib.fs_device_status()
+    assert code >> 24 == _lib.FS_ERR_TIMEOUT and (code & 0xFFFFFF) == 0xABC
+    got, ref = run_both(1, 16, 16, 2, 8, 0)  # the context is still usable
+    check("o", got["o"], ref["o"], FWD_TOL)

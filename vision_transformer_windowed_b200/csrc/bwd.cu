@@ -1,0 +1,740 @@
+// Backward of fused shifted-window attention with window-local 2D RoPE.
+//
+// Recompute-based (the probabilities are rebuilt from the forward's
+// log-sum-exp, never stored), in four launches on the caller's stream:
+//   1. prep:   per token row, rotate q and k (RoPE) into swizzled bf16 tile
+//              images, copy dO into a tile image, D = rowsum(dO * O), lse in
+//              log2 units, and zero the fp32 dQ accumulator;
+//   2. main:   persistent, warp-specialised tcgen05 kernel; a work item is one
+//              128-key tile, iterating over the query tiles it attends to:
+//                S^T = K' Q'^T, dP^T = V dO^T            (TMEM)
+//                P^T = exp2(S^T * c - lse2), dS^T = P^T (dP^T - D)
+//                dV += P^T dO, dK' += dS^T Q'            (TMEM accumulators)
+//                dQ' = dS K'  -> bulk reduce-add into the fp32 accumulator
+//   3. post:   per token row, undo the rotation of dQ' and dK', write dq and
+//              dk, and the per-tile partial sums of d theta;
+//   4. reduce: fixed-order sum of the partials into dtheta (deterministic).
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "geometry.cuh"
+#include "kernels.cuh"
+#include "ptx.cuh"
+#include "schedule.cuh"
+
+namespace fswin {
+
+namespace bwdk {
+
+// ------------------------------------------------------------------ workspace
+struct WsLayout {
+    size_t qimg, kimg, doimg, lse2, dvec, dqacc, dkimg, part, total;
+};
+
+__host__ __device__ inline size_t round256(size_t x) { return (x + 255) & ~size_t(255); }
+
+__host__ __device__ inline WsLayout ws_layout(const Geo& g) {
+    const size_t ht = static_cast<size_t>(g.heads) * static_cast<size_t>(g.tiles);
+    WsLayout L;
+    size_t o = 0;
+    L.qimg = o;  o += round256(ht * kTileBytes);
+    L.kimg = o;  o += round256(ht * kTileBytes);
+    L.doimg = o; o += round256(ht * kTileBytes);
+    L.lse2 = o;  o += round256(ht * kTile * 4);
+    L.dvec = o;  o += round256(ht * kTile * 4);
+    L.dqacc = o; o += round256(ht * kTile * kHeadDim * 4);
+    L.dkimg = o; o += round256(ht * kTile * kHeadDim * 4);
+    L.part = o;  o += round256(ht * 16 * 4);
+    L.total = o;
+    return L;
+}
+
+struct PrepParams {
+    Geo g;
+    const uint4 *q, *k, *o, *dout;
+    const float *lse, *theta;
+    uint8_t* ws;
+    WsLayout L;
+};
+
+struct PostParams {
+    Geo g;
+    const uint4 *q, *k;
+    const float* theta;
+    uint4 *dq, *dk;
+    const uint8_t* ws;
+    WsLayout L;
+    float scale;
+};
+
+// cos/sin of pos * theta[h][ax][k] for pos < M, in shared memory: [2][64][8].
+__device__ __forceinline__ void build_table(float2* tab, const float* theta_h, int M) {
+    for (int e = threadIdx.x; e < 2 * M * 8; e += blockDim.x) {
+        const int ax = e / (M * 8), rem = e - ax * M * 8, pos = rem >> 3, k = rem & 7;
+        float sn, cs;
+        sincosf(static_cast<float>(pos) * theta_h[ax * 8 + k], &sn, &cs);
+        tab[(ax * 64 + pos) * 8 + k] = make_float2(cs, sn);
+    }
+}
+
+// Rotate (inv = false) or un-rotate (inv = true) 32 channel values of a token
+// at in-window position (i, j).
+__device__ __forceinline__ void rope32(float (&x)[32], int i, int j, const float2* tab, bool inv) {
+#pragma unroll
+    for (int ax = 0; ax < 2; ++ax) {
+        const float2* t = tab + (ax * 64 + (ax ? i : j)) * 8;
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+            const float2 cs = t[k];
+            const float sn = inv ? -cs.y : cs.y;
+            const float a = x[ax * 16 + 2 * k], b = x[ax * 16 + 2 * k + 1];
+            x[ax * 16 + 2 * k] = a * cs.x - b * sn;
+            x[ax * 16 + 2 * k + 1] = a * sn + b * cs.x;
+        }
+    }
+}
+
+__device__ __forceinline__ void load_row_bf16(const uint4* src, float (&x)[32]) {
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+        const uint4 v = src[c];
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            x[8 * c + 2 * e] = bf16lo_to_f32(w[e]);
+            x[8 * c + 2 * e + 1] = bf16hi_to_f32(w[e]);
+        }
+    }
+}
+
+__device__ __forceinline__ uint32_t pack2(float lo, float hi, bool fp16) {
+    return fp16 ? pack_f16x2(lo, hi) : pack_bf16x2(lo, hi);
+}
+
+__device__ __forceinline__ uint4 pack_chunk(const float (&x)[32], int c, bool fp16 = false) {
+    return make_uint4(pack2(x[8 * c], x[8 * c + 1], fp16), pack2(x[8 * c + 2], x[8 * c + 3], fp16),
+                      pack2(x[8 * c + 4], x[8 * c + 5], fp16), pack2(x[8 * c + 6], x[8 * c + 7], fp16));
+}
+
+// Row r of a 64-byte-swizzled 16-bit tile image (bf16, or fp16 for the
+// rotated Q' and K', see the forward kernel).
+__device__ __forceinline__ void store_row_swz(uint8_t* tile, int r, const float (&x)[32], bool fp16 = false) {
+    uint8_t* row = tile + r * kRowBytes;
+    const int sw = (r >> 1) & 3;
+#pragma unroll
+    for (int c = 0; c < 4; ++c) *reinterpret_cast<uint4*>(row + ((c ^ sw) << 4)) = pack_chunk(x, c, fp16);
+}
+
+// ------------------------------------------------------------------ 1. prep
+__global__ void __launch_bounds__(128) prep_kernel(const PrepParams p) {
+    __shared__ float2 tab[2 * 64 * 8];
+    const Geo& g = p.g;
+    const long long ht = blockIdx.x;
+    const int h = static_cast<int>(ht / g.tiles);
+    const long long T = ht - static_cast<long long>(h) * g.tiles;
+    build_table(tab, p.theta + h * 16, g.M);
+    __syncthreads();
+    const int r = threadIdx.x;
+    const Slot sl = slot_of(g, T, r);
+    float q[32], k[32], dO[32], o[32];
+    float D = 0.f, lse2 = INFINITY;
+    if (sl.box.valid) {
+        const long long tok = ((static_cast<long long>(sl.box.b) * g.H + sl.row) * g.W + sl.col) * g.heads + h;
+        load_row_bf16(p.q + tok * 4, q);
+        load_row_bf16(p.k + tok * 4, k);
+        load_row_bf16(p.dout + tok * 4, dO);
+        load_row_bf16(p.o + tok * 4, o);
+        float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int e = 0; e < 32; ++e) acc[e & 3] = fmaf(dO[e], o[e], acc[e & 3]);
+        D = (acc[0] + acc[1]) + (acc[2] + acc[3]);
+        lse2 = p.lse[tok] * 1.4426950408889634f;
+        rope32(q, sl.i, sl.j, tab, false);
+        rope32(k, sl.i, sl.j, tab, false);
+    } else {
+#pragma unroll
+        for (int e = 0; e < 32; ++e) q[e] = k[e] = dO[e] = 0.f;
+    }
+    store_row_swz(p.ws + p.L.qimg + ht * kTileBytes, r, q, true);
+    store_row_swz(p.ws + p.L.kimg + ht * kTileBytes, r, k, true);
+    store_row_swz(p.ws + p.L.doimg + ht * kTileBytes, r, dO);
+    reinterpret_cast<float*>(p.ws + p.L.lse2)[ht * kTile + r] = lse2;
+    reinterpret_cast<float*>(p.ws + p.L.dvec)[ht * kTile + r] = D;
+    uint4* acc = reinterpret_cast<uint4*>(p.ws + p.L.dqacc + (ht * kTile + r) * kHeadDim * 4);
+#pragma unroll
+    for (int c = 0; c < 8; ++c) acc[c] = make_uint4(0, 0, 0, 0);
+}
+
+// ------------------------------------------------------------------ 2. main
+constexpr int kThreads = 448;
+constexpr int kQStages = 3;
+constexpr int kWarpTma = 12, kWarpMma = 13;  // warps 0-7: P/dS, 8-11: epilogue
+
+constexpr int kQStageBytes = 2 * kTileBytes + 2 * kTile * 4;  // Q', dO, lse2, D
+constexpr int kKVOff = 0;                                      // 2 slots x (K', V)
+constexpr int kQOff = kKVOff + 2 * 2 * kTileBytes;
+constexpr int kDSOff = kQOff + kQStages * kQStageBytes;        // dS, MN-major 128B swizzle
+constexpr int kDQStOff = kDSOff + 4 * kTileBytes;              // 2 x fp32 [128][32]
+constexpr int kDKStOff = kDQStOff + 2 * 4 * kTile * kHeadDim;  // fp32 [128][32]
+constexpr int kDVStOff = kDKStOff + 4 * kTile * kHeadDim;      // bf16 tile
+constexpr int kBarOff = kDVStOff + kTileBytes;
+constexpr int kSmemBytes = kBarOff + 1024 + 1024;
+
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kColS = 0, kColDP = 128, kColP = 256, kColDS = 320, kColDQ = 384, kColDV = 416, kColDK = 448;
+
+struct Bars {
+    uint64_t kv_full[2], kv_empty[2];
+    uint64_t q_full[kQStages], q_empty[kQStages];
+    uint64_t s_full, p_full, mma2_done;
+    uint64_t dq_full, dq_free, dkv_full, dkv_free;
+    uint64_t done;
+    uint32_t tmem_base;
+    int abort_flag;
+};
+
+struct MainParams {
+    Geo g;
+    uint8_t* ws;
+    WsLayout L;
+    unsigned int* status;
+    unsigned long long limit_ns;
+    long long items;
+    float scale;
+};
+
+using Item = BwdItem;
+__device__ __forceinline__ Item item_of(const Geo& g, long long it) { return bwd_item(g, it); }
+__device__ __forceinline__ bool q_active(const Geo& g, const Item& I, int n) { return bwd_active(g, I, n); }
+
+__global__ void __launch_bounds__(kThreads, 1)
+    main_kernel(const __grid_constant__ CUtensorMap map_v, const __grid_constant__ CUtensorMap map_dv,
+                const MainParams prm) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    Bars* bars = reinterpret_cast<Bars*>(smem + kBarOff);
+    const Geo& g = prm.g;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const size_t tiles = static_cast<size_t>(g.tiles);
+
+    if (tid == 0) {
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&bars->kv_full[i], 1);
+            mbar_init(&bars->kv_empty[i], 1);
+        }
+        for (int i = 0; i < kQStages; ++i) {
+            mbar_init(&bars->q_full[i], 1);
+            mbar_init(&bars->q_empty[i], 1);
+        }
+        mbar_init(&bars->s_full, 1);
+        mbar_init(&bars->p_full, 8);
+        mbar_init(&bars->mma2_done, 1);
+        mbar_init(&bars->dq_full, 1);
+        mbar_init(&bars->dq_free, 4);
+        mbar_init(&bars->dkv_full, 1);
+        mbar_init(&bars->dkv_free, 4);
+        mbar_init(&bars->done, 1);
+        bars->abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 0) {
+        tmem_alloc(&bars->tmem_base, kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = bars->tmem_base;
+    const Ctl ctl{prm.status, &bars->abort_flag, prm.limit_ns};
+    const uint8_t* ws = prm.ws;
+
+    if (warp == kWarpTma) {
+        // ------------------------------------------------------------ producer
+        if (lane == 0) {
+            prefetch_tmap(&map_v);
+            int it = 0;
+            uint32_t qc = 0;
+            bool ok = true;
+            for (long long item = blockIdx.x; item < prm.items && ok; item += gridDim.x, ++it) {
+                const Item I = item_of(g, item);
+                const int ks = it & 1;
+                if (!mbar_wait(&bars->kv_empty[ks], ((it >> 1) & 1) ^ 1, ctl, 0x1101)) break;
+                uint8_t* kv = smem + kKVOff + ks * 2 * kTileBytes;
+                const size_t hu = static_cast<size_t>(I.h) * tiles + static_cast<size_t>(I.u);
+                mbar_arrive_expect_tx(&bars->kv_full[ks], 2 * kTileBytes);
+                bulk_load(kv, ws + prm.L.kimg + hu * kTileBytes, kTileBytes, &bars->kv_full[ks]);
+                for (int i = 0; i < g.bpt; ++i) {
+                    const Box bx = box_of(g, I.u * g.bpt + i);
+                    tma_load_5d(kv + kTileBytes + i * g.BT * kRowBytes, &map_v, &bars->kv_full[ks], 0, I.h, bx.col0,
+                                bx.row0, bx.b);
+                }
+                for (int n = 0; n < I.nq; ++n) {
+                    if (!q_active(g, I, n)) continue;
+                    const int st = qc % kQStages;
+                    const uint32_t ph = (qc / kQStages) & 1;
+                    ++qc;
+                    if (!mbar_wait(&bars->q_empty[st], ph ^ 1, ctl, 0x1102)) { ok = false; break; }
+                    uint8_t* qs = smem + kQOff + st * kQStageBytes;
+                    const size_t hv = static_cast<size_t>(I.h) * tiles + static_cast<size_t>(I.q0 + n);
+                    mbar_arrive_expect_tx(&bars->q_full[st], kQStageBytes);
+                    bulk_load(qs, ws + prm.L.qimg + hv * kTileBytes, kTileBytes, &bars->q_full[st]);
+                    bulk_load(qs + kTileBytes, ws + prm.L.doimg + hv * kTileBytes, kTileBytes, &bars->q_full[st]);
+                    bulk_load(qs + 2 * kTileBytes, ws + prm.L.lse2 + hv * kTile * 4, kTile * 4, &bars->q_full[st]);
+                    bulk_load(qs + 2 * kTileBytes + kTile * 4, ws + prm.L.dvec + hv * kTile * 4, kTile * 4,
+                              &bars->q_full[st]);
+                }
+            }
+        }
+    } else if (warp == kWarpMma) {
+        // ------------------------------------------------------------ MMA issue
+        if (lane == 0) {
+            // operand types: Q', K', dS in fp16; V, dO, P in bf16
+            const uint32_t id_s = make_idesc(kTile, kTile, false, false, true);
+            const uint32_t id_dp = make_idesc(kTile, kTile, false, false, false);
+            const uint32_t id_kv = make_idesc(kTile, kHeadDim, false, true, false);
+            const uint32_t id_dk = make_idesc(kTile, kHeadDim, false, true, true);
+            const uint32_t id_dq = make_idesc(kTile, kHeadDim, true, true, true);
+            const uint32_t ds_addr = smem_u32(smem + kDSOff);
+            // state of the step whose second half is pending
+            bool have_prev = false;
+            int prev_st = 0, prev_ks = 0;
+            bool prev_first = false, prev_last = false;
+            int prev_item_idx = -1;
+            uint32_t pph = 0, dqph = 0, dkvph = 0;
+            bool ok = true;
+            // Step j issues S(j), dP(j) as soon as the softmax of step j-1 has read
+            // S and dP, then the second half of step j-1: dV, dK and dQ.
+            int it = 0;
+            uint32_t qc = 0;
+            long long nsteps_done = 0;
+            for (long long item = blockIdx.x; item < prm.items && ok; item += gridDim.x, ++it) {
+                const Item I = item_of(g, item);
+                const int ks = it & 1;
+                if (!mbar_wait(&bars->kv_full[ks], (it >> 1) & 1, ctl, 0x1302)) break;
+                const uint32_t kaddr = smem_u32(smem + kKVOff + ks * 2 * kTileBytes);
+                // count active query tiles to know the last step of the item
+                int last_n = -1;
+                for (int n = 0; n < I.nq; ++n)
+                    if (q_active(g, I, n)) last_n = n;
+                bool first = true;
+                for (int n = 0; n < I.nq && ok; ++n) {
+                    if (!q_active(g, I, n)) continue;
+                    const int st = qc % kQStages;
+                    const uint32_t ph = (qc / kQStages) & 1;
+                    ++qc;
+                    if (!mbar_wait(&bars->q_full[st], ph, ctl, 0x1303)) { ok = false; break; }
+                    if (have_prev) {
+                        if (!mbar_wait(&bars->p_full, pph, ctl, 0x1304)) { ok = false; break; }
+                        pph ^= 1;
+                    }
+                    tc_fence_after();
+                    const uint32_t qaddr = smem_u32(smem + kQOff + st * kQStageBytes);
+                    // S^T = K' Q'^T and dP^T = V dO^T
+#pragma unroll
+                    for (int k = 0; k < kHeadDim / 16; ++k)
+                        umma_ss(tmem + kColS, make_sdesc(kaddr + 32 * k, 16, 512, kSw64),
+                                make_sdesc(qaddr + 32 * k, 16, 512, kSw64), id_s, k > 0);
+#pragma unroll
+                    for (int k = 0; k < kHeadDim / 16; ++k)
+                        umma_ss(tmem + kColDP, make_sdesc(kaddr + kTileBytes + 32 * k, 16, 512, kSw64),
+                                make_sdesc(qaddr + kTileBytes + 32 * k, 16, 512, kSw64), id_dp, k > 0);
+                    umma_commit(&bars->s_full);
+                    if (have_prev) {
+                        // second half of the previous step
+                        const uint32_t pk = smem_u32(smem + kKVOff + prev_ks * 2 * kTileBytes);
+                        const uint32_t pq = smem_u32(smem + kQOff + prev_st * kQStageBytes);
+                        if (prev_first && prev_item_idx > 0) {
+                            if (!mbar_wait(&bars->dkv_free, dkvph, ctl, 0x1305)) { ok = false; break; }
+                            dkvph ^= 1;
+                            tc_fence_after();
+                        }
+#pragma unroll
+                        for (int k = 0; k < kTile / 16; ++k)
+                            umma_ts(tmem + kColDV, tmem + kColP + 8 * k,
+                                    make_sdesc(pq + kTileBytes + 1024 * k, 8192, 512, kSw64), id_kv,
+                                    (!prev_first || k > 0) ? 1u : 0u);
+#pragma unroll
+                        for (int k = 0; k < kTile / 16; ++k)
+                            umma_ts(tmem + kColDK, tmem + kColDS + 8 * k, make_sdesc(pq + 1024 * k, 8192, 512, kSw64),
+                                    id_dk, (!prev_first || k > 0) ? 1u : 0u);
+                        if (nsteps_done > 0) {
+                            if (!mbar_wait(&bars->dq_free, dqph, ctl, 0x1306)) { ok = false; break; }
+                            dqph ^= 1;
+                            tc_fence_after();
+                        }
+#pragma unroll
+                        for (int k = 0; k < kTile / 16; ++k)
+                            umma_ss(tmem + kColDQ, make_sdesc(ds_addr + 2048 * k, 16384, 1024, kSw128),
+                                    make_sdesc(pk + 1024 * k, 8192, 512, kSw64), id_dq, k > 0);
+                        umma_commit(&bars->mma2_done);
+                        umma_commit(&bars->dq_full);
+                        umma_commit(&bars->q_empty[prev_st]);
+                        if (prev_last) {
+                            umma_commit(&bars->dkv_full);
+                            umma_commit(&bars->kv_empty[prev_ks]);
+                        }
+                        ++nsteps_done;
+                    }
+                    have_prev = true;
+                    prev_st = st;
+                    prev_ks = ks;
+                    prev_first = first;
+                    prev_last = (n == last_n);
+                    prev_item_idx = it;
+                    first = false;
+                }
+            }
+            if (ok && have_prev) {
+                const uint32_t pk = smem_u32(smem + kKVOff + prev_ks * 2 * kTileBytes);
+                const uint32_t pq = smem_u32(smem + kQOff + prev_st * kQStageBytes);
+                bool ok2 = mbar_wait(&bars->p_full, pph, ctl, 0x1307);
+                pph ^= 1;
+                if (ok2 && prev_first && prev_item_idx > 0) {
+                    ok2 = mbar_wait(&bars->dkv_free, dkvph, ctl, 0x1308);
+                    dkvph ^= 1;
+                }
+                if (ok2) {
+                    tc_fence_after();
+#pragma unroll
+                    for (int k = 0; k < kTile / 16; ++k)
+                        umma_ts(tmem + kColDV, tmem + kColP + 8 * k,
+                                make_sdesc(pq + kTileBytes + 1024 * k, 8192, 512, kSw64), id_kv,
+                                (!prev_first || k > 0) ? 1u : 0u);
+#pragma unroll
+                    for (int k = 0; k < kTile / 16; ++k)
+                        umma_ts(tmem + kColDK, tmem + kColDS + 8 * k, make_sdesc(pq + 1024 * k, 8192, 512, kSw64),
+                                id_dk, (!prev_first || k > 0) ? 1u : 0u);
+                    if (nsteps_done > 0) {
+                        ok2 = mbar_wait(&bars->dq_free, dqph, ctl, 0x1309);
+                        dqph ^= 1;
+                        tc_fence_after();
+                    }
+                    if (ok2) {
+#pragma unroll
+                        for (int k = 0; k < kTile / 16; ++k)
+                            umma_ss(tmem + kColDQ, make_sdesc(ds_addr + 2048 * k, 16384, 1024, kSw128),
+                                    make_sdesc(pk + 1024 * k, 8192, 512, kSw64), id_dq, k > 0);
+                        umma_commit(&bars->mma2_done);
+                        umma_commit(&bars->dq_full);
+                        umma_commit(&bars->q_empty[prev_st]);
+                        umma_commit(&bars->dkv_full);
+                        umma_commit(&bars->kv_empty[prev_ks]);
+                    }
+                }
+            }
+            umma_commit(&bars->done);
+            mbar_wait(&bars->done, 0, ctl, 0x13ff);
+        }
+        __syncwarp();
+    } else if (warp < 8) {
+        // ------------------------------------------------------------ P^T, dS^T (thread = key row)
+        const int hw = warp >> 2;  // query half: columns [64 hw, 64 hw + 64)
+        const int quarter = warp & 3;
+        const int r = quarter * 32 + lane;
+        const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
+        const float sl2 = g.scale_log2;
+        uint8_t* ds = smem + kDSOff;
+        uint32_t sph = 0, mph = 0;
+        uint32_t qc = 0;
+        bool started = false, ok = true;
+        for (long long item = blockIdx.x; item < prm.items && ok; item += gridDim.x) {
+            const Item I = item_of(g, item);
+            const long long keyseg = seg_of(slot_of(g, I.u, r).box);
+            for (int n = 0; n < I.nq; ++n) {
+                if (!q_active(g, I, n)) continue;
+                const int st = qc % kQStages;
+                ++qc;
+                const float* lse2 = reinterpret_cast<const float*>(smem + kQOff + st * kQStageBytes + 2 * kTileBytes);
+                const float* dvec = lse2 + kTile;
+                const uint32_t allow = allow_mask(g, keyseg, I.q0 + n);
+                const bool full = allow == ((1u << g.bpt) - 1u);
+                if (!mbar_wait(&bars->s_full, sph, ctl, 0x1401)) { ok = false; break; }
+                sph ^= 1;
+                tc_fence_after();
+#pragma unroll
+                for (int c = 0; c < 2; ++c) {
+                    const int col0 = 64 * hw + 32 * c;
+                    uint32_t sv[32], pv[32];
+                    tmem_ld32(tmem + lane_off + kColS + col0, sv);
+                    tmem_ld32(tmem + lane_off + kColDP + col0, pv);
+                    tmem_wait_ld();
+                    float p[32], dsv[32];
+#pragma unroll
+                    for (int e4 = 0; e4 < 8; ++e4) {
+                        const float4 L4 = *reinterpret_cast<const float4*>(lse2 + col0 + 4 * e4);
+                        const float4 D4 = *reinterpret_cast<const float4*>(dvec + col0 + 4 * e4);
+                        const float Ls[4] = {L4.x, L4.y, L4.z, L4.w}, Ds[4] = {D4.x, D4.y, D4.z, D4.w};
+#pragma unroll
+                        for (int e1 = 0; e1 < 4; ++e1) {
+                            const int e = 4 * e4 + e1;
+                            p[e] = ex2_approx(fmaf(__uint_as_float(sv[e]), sl2, -Ls[e1]));
+                            dsv[e] = p[e] * (__uint_as_float(pv[e]) - Ds[e1]);
+                        }
+                    }
+                    if (!full) {
+#pragma unroll
+                        for (int e = 0; e < 32; ++e) {
+                            const int qb = (col0 + e) / g.BT;
+                            if (!((allow >> qb) & 1u)) {
+                                p[e] = 0.f;
+                                dsv[e] = 0.f;
+                            }
+                        }
+                    }
+                    if (c == 0 && started) {
+                        if (!mbar_wait(&bars->mma2_done, mph, ctl, 0x1402)) { ok = false; break; }
+                        mph ^= 1;
+                        tc_fence_after();
+                    }
+                    uint32_t wp[16], wd[16];
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) {
+                        wp[e] = pack_bf16x2(p[2 * e], p[2 * e + 1]);
+                        wd[e] = pack_f16x2(dsv[2 * e], dsv[2 * e + 1]);
+                    }
+                    tmem_st16(tmem + lane_off + kColP + col0 / 2, wp);
+                    tmem_st16(tmem + lane_off + kColDS + col0 / 2, wd);
+                    // dS (queries along M, keys along K) as an MN-major operand
+                    uint8_t* base = ds + hw * 16384 + (r >> 3) * 1024 + (r & 7) * 128;
+#pragma unroll
+                    for (int q4 = 0; q4 < 4; ++q4) {
+                        const int cc = 4 * c + q4;
+                        *reinterpret_cast<uint4*>(base + ((cc ^ (r & 7)) << 4)) =
+                            make_uint4(wd[4 * q4], wd[4 * q4 + 1], wd[4 * q4 + 2], wd[4 * q4 + 3]);
+                    }
+                }
+                if (!ok) break;
+                tmem_wait_st();
+                fence_proxy_async_smem();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&bars->p_full);
+                started = true;
+            }
+        }
+    } else {
+        // ------------------------------------------------------------ dQ / dK / dV epilogue (warps 8-11)
+        const int quarter = warp & 3;
+        const int r = quarter * 32 + lane;
+        const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
+        const bool leader = (quarter == 0 && lane == 0);
+        float* dqst = reinterpret_cast<float*>(smem + kDQStOff);
+        float* dkst = reinterpret_cast<float*>(smem + kDKStOff);
+        uint8_t* dvst = smem + kDVStOff;
+        uint32_t dqph = 0, dkvph = 0;
+        long long j = 0;
+        bool ok = true;
+        for (long long item = blockIdx.x; item < prm.items && ok; item += gridDim.x) {
+            const Item I = item_of(g, item);
+            for (int n = 0; n < I.nq; ++n) {
+                if (!q_active(g, I, n)) continue;
+                if (!mbar_wait(&bars->dq_full, dqph, ctl, 0x1501)) { ok = false; break; }
+                dqph ^= 1;
+                tc_fence_after();
+                uint32_t v[32];
+                tmem_ld32(tmem + lane_off + kColDQ, v);
+                tmem_wait_ld();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&bars->dq_free);
+                float* buf = dqst + (j & 1) * kTile * kHeadDim;
+                if (leader) bulk_wait_read_but1();
+                named_bar_sync(1, 128);
+                float4* rowp = reinterpret_cast<float4*>(buf + r * kHeadDim);
+#pragma unroll
+                for (int c0 = 0; c0 < 8; ++c0) {
+                    const int c = (c0 + lane) & 7;
+                    rowp[c] = make_float4(__uint_as_float(v[4 * c]) * prm.scale, __uint_as_float(v[4 * c + 1]) * prm.scale,
+                                          __uint_as_float(v[4 * c + 2]) * prm.scale,
+                                          __uint_as_float(v[4 * c + 3]) * prm.scale);
+                }
+                fence_proxy_async_smem();
+                named_bar_sync(1, 128);
+                if (leader) {
+                    const size_t hv = static_cast<size_t>(I.h) * tiles + static_cast<size_t>(I.q0 + n);
+                    bulk_reduce_add_f32(prm.ws + prm.L.dqacc + hv * kTile * kHeadDim * 4, buf, kTile * kHeadDim * 4);
+                    bulk_commit();
+                }
+                ++j;
+            }
+            if (!ok) break;
+            // item end: dV and dK' accumulators
+            if (!mbar_wait(&bars->dkv_full, dkvph, ctl, 0x1502)) break;
+            dkvph ^= 1;
+            tc_fence_after();
+            uint32_t vv[32], kk[32];
+            tmem_ld32(tmem + lane_off + kColDV, vv);
+            tmem_ld32(tmem + lane_off + kColDK, kk);
+            tmem_wait_ld();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bars->dkv_free);
+            if (leader) bulk_wait_read_all();
+            named_bar_sync(1, 128);
+            {
+                float4* rowp = reinterpret_cast<float4*>(dkst + r * kHeadDim);
+#pragma unroll
+                for (int c0 = 0; c0 < 8; ++c0) {
+                    const int c = (c0 + lane) & 7;
+                    rowp[c] = make_float4(__uint_as_float(kk[4 * c]) * prm.scale, __uint_as_float(kk[4 * c + 1]) * prm.scale,
+                                          __uint_as_float(kk[4 * c + 2]) * prm.scale,
+                                          __uint_as_float(kk[4 * c + 3]) * prm.scale);
+                }
+                float x[32];
+#pragma unroll
+                for (int e = 0; e < 32; ++e) x[e] = __uint_as_float(vv[e]);
+                store_row_swz(dvst, r, x);
+            }
+            fence_proxy_async_smem();
+            named_bar_sync(1, 128);
+            if (leader) {
+                const size_t hu = static_cast<size_t>(I.h) * tiles + static_cast<size_t>(I.u);
+                bulk_store(prm.ws + prm.L.dkimg + hu * kTile * kHeadDim * 4, dkst, kTile * kHeadDim * 4);
+                for (int i = 0; i < g.bpt; ++i) {
+                    const Box bx = box_of(g, I.u * g.bpt + i);
+                    if (bx.valid) tma_store_5d(&map_dv, dvst + i * g.BT * kRowBytes, 0, I.h, bx.col0, bx.row0, bx.b);
+                }
+                bulk_commit();
+            }
+        }
+        if (leader) bulk_wait_all();
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 0) tmem_dealloc(tmem, kTmemCols);
+}
+
+// ------------------------------------------------------------------ 3. post
+__global__ void __launch_bounds__(128) post_kernel(const PostParams p) {
+    __shared__ float2 tab[2 * 64 * 8];
+    __shared__ float red[4][16];
+    const Geo& g = p.g;
+    const long long ht = blockIdx.x;
+    const int h = static_cast<int>(ht / g.tiles);
+    const long long T = ht - static_cast<long long>(h) * g.tiles;
+    build_table(tab, p.theta + h * 16, g.M);
+    __syncthreads();
+    const int r = threadIdx.x, lane = r & 31, warp = r >> 5;
+    const Slot sl = slot_of(g, T, r);
+    float part[16];
+#pragma unroll
+    for (int e = 0; e < 16; ++e) part[e] = 0.f;
+    if (sl.box.valid) {
+        const long long tok = ((static_cast<long long>(sl.box.b) * g.H + sl.row) * g.W + sl.col) * g.heads + h;
+        float dq[32], dk[32], q[32], k[32];
+        const float4* aq = reinterpret_cast<const float4*>(p.ws + p.L.dqacc + (ht * kTile + r) * kHeadDim * 4);
+        const float4* ak = reinterpret_cast<const float4*>(p.ws + p.L.dkimg + (ht * kTile + r) * kHeadDim * 4);
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+            const float4 a = aq[c], b = ak[c];
+            dq[4 * c] = a.x; dq[4 * c + 1] = a.y; dq[4 * c + 2] = a.z; dq[4 * c + 3] = a.w;
+            dk[4 * c] = b.x; dk[4 * c + 1] = b.y; dk[4 * c + 2] = b.z; dk[4 * c + 3] = b.w;
+        }
+        rope32(dq, sl.i, sl.j, tab, true);
+        rope32(dk, sl.i, sl.j, tab, true);
+        load_row_bf16(p.q + tok * 4, q);
+        load_row_bf16(p.k + tok * 4, k);
+#pragma unroll
+        for (int ax = 0; ax < 2; ++ax) {
+            const float pos = static_cast<float>(ax ? sl.i : sl.j);
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk) {
+                const int a = ax * 16 + 2 * kk, b = a + 1;
+                const float w = (dq[b] * q[a] - dq[a] * q[b]) + (dk[b] * k[a] - dk[a] * k[b]);
+                part[ax * 8 + kk] = pos * w;
+            }
+        }
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+            p.dq[tok * 4 + c] = pack_chunk(dq, c);
+            p.dk[tok * 4 + c] = pack_chunk(dk, c);
+        }
+    }
+#pragma unroll
+    for (int e = 0; e < 16; ++e) {
+        float v = part[e];
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+        if (lane == 0) red[warp][e] = v;
+    }
+    __syncthreads();
+    if (r < 16) {
+        const float s = (red[0][r] + red[1][r]) + (red[2][r] + red[3][r]);
+        reinterpret_cast<float*>(const_cast<uint8_t*>(p.ws) + p.L.part)[ht * 16 + r] = s;
+    }
+}
+
+// ------------------------------------------------------------------ 4. reduce
+__global__ void __launch_bounds__(256) dtheta_kernel(const float* part, long long tiles, float* dtheta) {
+    __shared__ float acc[16][17];
+    const int h = blockIdx.x;
+    const int comp = threadIdx.x & 15, grp = threadIdx.x >> 4;
+    float s = 0.f;
+    for (long long T = grp; T < tiles; T += 16) s += part[(static_cast<long long>(h) * tiles + T) * 16 + comp];
+    acc[grp][comp] = s;
+    __syncthreads();
+    if (threadIdx.x < 16) {
+        float t = 0.f;
+        for (int i = 0; i < 16; ++i) t += acc[i][threadIdx.x];
+        dtheta[h * 16 + threadIdx.x] = t;
+    }
+}
+
+}  // namespace bwdk
+
+size_t bwd_workspace_bytes(const Geo& g) { return bwdk::ws_layout(g).total; }
+
+long long bwd_items(const Geo& g) { return bwd_item_count(g); }
+
+
+cudaError_t launch_bwd(const Geo& g, const BwdPtrs& p, const CUtensorMap& mv, const CUtensorMap& mdv,
+                       unsigned int* status, unsigned long long limit_ns, int num_sms, cudaStream_t stream,
+                       cudaEvent_t const* events) {
+    using namespace bwdk;
+    const WsLayout L = ws_layout(g);
+    const long long ht = static_cast<long long>(g.heads) * g.tiles;
+    const float scale = static_cast<float>(1.0 / 5.656854249492380195);  // 1/sqrt(32)
+    cudaError_t e = cudaSuccess;
+    auto mark = [&](int i) {
+        if (events && e == cudaSuccess) e = cudaEventRecord(events[i], stream);
+    };
+    static bool attr_set = false;
+    if (!attr_set) {
+        e = cudaFuncSetAttribute(main_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+        if (e != cudaSuccess) return e;
+        attr_set = true;
+    }
+    mark(0);
+    PrepParams pp{g, static_cast<const uint4*>(p.q), static_cast<const uint4*>(p.k), static_cast<const uint4*>(p.o),
+                  static_cast<const uint4*>(p.dout), p.lse, p.theta, p.ws, L};
+    prep_kernel<<<static_cast<unsigned>(ht), 128, 0, stream>>>(pp);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    mark(1);
+
+    MainParams mp;
+    mp.g = g;
+    mp.ws = p.ws;
+    mp.L = L;
+    mp.status = status;
+    mp.limit_ns = limit_ns;
+    mp.items = bwd_items(g);
+    mp.scale = scale;
+    const long long grid = mp.items < num_sms ? mp.items : num_sms;
+    main_kernel<<<static_cast<unsigned>(grid), kThreads, kSmemBytes, stream>>>(mv, mdv, mp);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    mark(2);
+
+    PostParams qp{g, static_cast<const uint4*>(p.q), static_cast<const uint4*>(p.k), p.theta,
+                  static_cast<uint4*>(p.dq), static_cast<uint4*>(p.dk), p.ws, L, scale};
+    post_kernel<<<static_cast<unsigned>(ht), 128, 0, stream>>>(qp);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    mark(3);
+    dtheta_kernel<<<g.heads, 256, 0, stream>>>(reinterpret_cast<const float*>(p.ws + L.part), g.tiles, p.dtheta);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    mark(4);
+    return e;
+}
+
+}  // namespace fswin

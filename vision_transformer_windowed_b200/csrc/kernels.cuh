@@ -1,0 +1,35 @@
+// Host-side launch entry points of the kernels, shared by api.cu.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cstddef>
+#include <cstdint>
+
+#include "geometry.cuh"
+
+namespace fswin {
+
+long long fwd_items(const Geo& g);
+cudaError_t launch_fwd(const Geo& g, const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+                       const CUtensorMap& mo, const float* theta, float* lse, unsigned int* status,
+                       unsigned long long limit_ns, int num_sms, cudaStream_t stream, cudaEvent_t const* events);
+
+struct BwdPtrs {
+    const void *q, *k, *v, *o, *dout;
+    const float *lse, *theta;
+    void *dq, *dk, *dv;
+    float* dtheta;
+    uint8_t* ws;
+};
+
+long long bwd_items(const Geo& g);
+size_t bwd_workspace_bytes(const Geo& g);
+// events: NULL, or 5 events recorded before the first and after each of the
+// four launches.
+cudaError_t launch_bwd(const Geo& g, const BwdPtrs& p, const CUtensorMap& mv, const CUtensorMap& mdv,
+                       unsigned int* status, unsigned long long limit_ns, int num_sms, cudaStream_t stream,
+                       cudaEvent_t const* events);
+
+}  // namespace fswin

@@ -1,0 +1,113 @@
+"""Torch-facing wrappers of the C ABI: they allocate outputs with PyTorch, pass
+raw device pointers and the current CUDA stream, and nothing else.  Every step
+of the attention runs in the CUDA kernels of libfswin.so.
+
+Method: FlashSwin ("FLASHSWIN: Unlocking Large Windows and Dense Tokens in Swin
+Vision Transformers with Memory Efficient Attention", thelatestinai.com/papers/
+2610.04664, Figure 1B): exact windowed softmax attention with window-local
+learnable 2D RoPE, the fused FlashAttention-style kernel replacing Swin's
+materialised score matrix.
+"""
+from __future__ import annotations
+
+import torch
+
+from . import _lib
+
+HEAD_DIM = 32
+
+
+def _shape(q: torch.Tensor, M: int, s: int) -> _lib.Shape:
+    if q.dim() != 5:
+        raise ValueError("expected a [B, H, W, heads, d] tensor")
+    B, H, W, heads, d = q.shape
+    return _lib.make_shape(B, H, W, heads, d, M, s)
+
+
+def _check_tensor(name: str, t: torch.Tensor, shape, dtype) -> None:
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def _stream(device) -> int:
+    return torch.cuda.current_stream(device).cuda_stream
+
+
+def winattn_fwd(q, k, v, theta, M: int, s: int, o=None, lse=None):
+    """O, LSE = fused windowed-RoPE attention forward (bf16 in/out, fp32 LSE)."""
+    sh = _shape(q, M, s)
+    B, H, W, heads, d = q.shape
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        _check_tensor(name, t, q.shape, torch.bfloat16)
+    _check_tensor("theta", theta, (heads, 2, d // 4), torch.float32)
+    if o is None:
+        o = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, H, W, heads), device=q.device, dtype=torch.float32)
+    _check_tensor("o", o, q.shape, torch.bfloat16)
+    _check_tensor("lse", lse, (B, H, W, heads), torch.float32)
+    _lib.fs_winattn_fwd(sh, q.data_ptr(), k.data_ptr(), v.data_ptr(), theta.data_ptr(), o.data_ptr(),
+                        lse.data_ptr(), _stream(q.device))
+    return o, lse
+
+
+def bwd_workspace_bytes(B: int, H: int, W: int, heads: int, M: int, s: int, d: int = HEAD_DIM) -> int:
+    return _lib.fs_winattn_bwd_workspace_bytes(_lib.make_shape(B, H, W, heads, d, M, s))
+
+
+def alloc_workspace(q: torch.Tensor, M: int, s: int) -> torch.Tensor:
+    n = _lib.fs_winattn_bwd_workspace_bytes(_shape(q, M, s))
+    return torch.empty(max(n, 256), device=q.device, dtype=torch.uint8)
+
+
+def winattn_bwd(q, k, v, o, dout, lse, theta, M: int, s: int, workspace=None, dq=None, dk=None, dv=None,
+                dtheta=None):
+    """dQ, dK, dV, dtheta of sum(O * dout) (recompute-based backward)."""
+    sh = _shape(q, M, s)
+    B, H, W, heads, d = q.shape
+    for name, t in (("q", q), ("k", k), ("v", v), ("o", o), ("dout", dout)):
+        _check_tensor(name, t, q.shape, torch.bfloat16)
+    _check_tensor("lse", lse, (B, H, W, heads), torch.float32)
+    _check_tensor("theta", theta, (heads, 2, d // 4), torch.float32)
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(q) if dk is None else dk
+    dv = torch.empty_like(q) if dv is None else dv
+    dtheta = torch.empty_like(theta) if dtheta is None else dtheta
+    if workspace is None:
+        workspace = alloc_workspace(q, M, s)
+    _lib.fs_winattn_bwd(sh, q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), dout.data_ptr(), lse.data_ptr(),
+                        theta.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), dtheta.data_ptr(),
+                        workspace.data_ptr(), workspace.numel(), _stream(q.device))
+    return dq, dk, dv, dtheta
+
+
+class WindowAttentionRoPE(torch.autograd.Function):
+    """Autograd wrapper: forward and backward both run in libfswin.so.
+
+    theta are the inverse frequencies; with the log parameterisation of the
+    paper (theta = exp(omega), thelatestinai.com/papers/2610.04664, Figure S4)
+    autograd through ``torch.exp`` gives d omega = theta * d theta.
+    """
+
+    @staticmethod
+    def forward(ctx, q, k, v, theta, M: int, s: int):
+        o, lse = winattn_fwd(q, k, v, theta, M, s)
+        ctx.save_for_backward(q, k, v, o, lse, theta)
+        ctx.M, ctx.s = M, s
+        return o
+
+    @staticmethod
+    def backward(ctx, dout):
+        q, k, v, o, lse, theta = ctx.saved_tensors
+        dq, dk, dv, dth = winattn_bwd(q, k, v, o, dout.contiguous(), lse, theta, ctx.M, ctx.s)
+        return dq, dk, dv, dth, None, None
+
+
+def window_attention(q, k, v, theta, M: int, s: int):
+    return WindowAttentionRoPE.apply(q, k, v, theta, M, s)
