@@ -192,8 +192,11 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-extra", action="store_true", help="skip the per-config numbers of the other workloads")
     ap.add_argument("--reference-seconds", type=float, default=60.0)
+    ap.add_argument("--batch", type=int, default=0, help="override the workload's batch (profiling runs only)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
+    if args.batch > 0:
+        WORKLOADS[args.workload] = dict(WORKLOADS[args.workload], B=args.batch)
     if args.impl == "reference":
         run_reference(args)
         return

@@ -11,7 +11,7 @@ CSRC = os.path.join(HERE, "csrc")
 BUILD = os.path.join(HERE, "_build")
 LIB = os.path.join(BUILD, "libfswin.so")
 SOURCES = ["api.cu", "fwd.cu", "bwd.cu"]
-HEADERS = ["geometry.cuh", "kernels.cuh", "ptx.cuh", "schedule.cuh"]
+HEADERS = ["dgeo.cuh", "geometry.cuh", "kernels.cuh", "ptx.cuh", "schedule.cuh", "tile_io.cuh"]
 
 
 def nvcc_path() -> str:

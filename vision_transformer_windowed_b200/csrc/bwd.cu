@@ -21,6 +21,8 @@
 #include "kernels.cuh"
 #include "ptx.cuh"
 #include "schedule.cuh"
+#include "tile_io.cuh"
+#include "dgeo.cuh"
 
 namespace fswin {
 
@@ -204,12 +206,12 @@ struct MainParams {
 };
 
 using Item = BwdItem;
-__device__ __forceinline__ Item item_of(const Geo& g, long long it) { return bwd_item(g, it); }
+__device__ __forceinline__ Item item_of(const Geo& g, long long it) { return d_bwd_item(g, it); }
 __device__ __forceinline__ bool q_active(const Geo& g, const Item& I, int n) { return bwd_active(g, I, n); }
 
 __global__ void __launch_bounds__(kThreads, 1)
     main_kernel(const __grid_constant__ CUtensorMap map_v, const __grid_constant__ CUtensorMap map_dv,
-                const MainParams prm) {
+                const __grid_constant__ MainParams prm) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     Bars* bars = reinterpret_cast<Bars*>(smem + kBarOff);
@@ -263,11 +265,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const size_t hu = static_cast<size_t>(I.h) * tiles + static_cast<size_t>(I.u);
                 mbar_arrive_expect_tx(&bars->kv_full[ks], 2 * kTileBytes);
                 bulk_load(kv, ws + prm.L.kimg + hu * kTileBytes, kTileBytes, &bars->kv_full[ks]);
-                for (int i = 0; i < g.bpt; ++i) {
-                    const Box bx = box_of(g, I.u * g.bpt + i);
-                    tma_load_5d(kv + kTileBytes + i * g.BT * kRowBytes, &map_v, &bars->kv_full[ks], 0, I.h, bx.col0,
-                                bx.row0, bx.b);
-                }
+                tile_tma(g, &map_v, kv + kTileBytes, &bars->kv_full[ks], I.u, I.h, false);
                 for (int n = 0; n < I.nq; ++n) {
                     if (!q_active(g, I, n)) continue;
                     const int st = qc % kQStages;
@@ -439,58 +437,53 @@ __global__ void __launch_bounds__(kThreads, 1)
         bool started = false, ok = true;
         for (long long item = blockIdx.x; item < prm.items && ok; item += gridDim.x) {
             const Item I = item_of(g, item);
-            const long long keyseg = seg_of(slot_of(g, I.u, r).box);
+            const uint32_t keyseg = seg_at(d_tile_segs(g, I.u, I.win), r >> g.lBT);
             for (int n = 0; n < I.nq; ++n) {
                 if (!q_active(g, I, n)) continue;
                 const int st = qc % kQStages;
                 ++qc;
                 const float* lse2 = reinterpret_cast<const float*>(smem + kQOff + st * kQStageBytes + 2 * kTileBytes);
                 const float* dvec = lse2 + kTile;
-                const uint32_t allow = allow_mask(g, keyseg, I.q0 + n);
-                const bool full = allow == ((1u << g.bpt) - 1u);
+                // bit c: query columns [16 c, 16 c + 16) attend this key row
+                const uint32_t a16 = d_allow16(g, keyseg, I.q0 + n, I.win);
+                const bool full = ((a16 >> (4 * hw)) & 0xFu) == 0xFu;
                 if (!mbar_wait(&bars->s_full, sph, ctl, 0x1401)) { ok = false; break; }
                 sph ^= 1;
                 tc_fence_after();
-#pragma unroll
-                for (int c = 0; c < 2; ++c) {
+#pragma unroll 1
+                for (int c = 0; c < 2; ++c) {  // rolled: keeps live ranges (registers) short
                     const int col0 = 64 * hw + 32 * c;
                     uint32_t sv[32], pv[32];
                     tmem_ld32(tmem + lane_off + kColS + col0, sv);
                     tmem_ld32(tmem + lane_off + kColDP + col0, pv);
                     tmem_wait_ld();
-                    float p[32], dsv[32];
+                    const bool ok0 = full || ((a16 >> (col0 >> 4)) & 1u);
+                    const bool ok1 = full || ((a16 >> ((col0 >> 4) + 1)) & 1u);
+                    uint32_t wp[16], wd[16];
 #pragma unroll
                     for (int e4 = 0; e4 < 8; ++e4) {
-                        const float4 L4 = *reinterpret_cast<const float4*>(lse2 + col0 + 4 * e4);
+                        float4 L4 = *reinterpret_cast<const float4*>(lse2 + col0 + 4 * e4);
                         const float4 D4 = *reinterpret_cast<const float4*>(dvec + col0 + 4 * e4);
-                        const float Ls[4] = {L4.x, L4.y, L4.z, L4.w}, Ds[4] = {D4.x, D4.y, D4.z, D4.w};
-#pragma unroll
-                        for (int e1 = 0; e1 < 4; ++e1) {
-                            const int e = 4 * e4 + e1;
-                            p[e] = ex2_approx(fmaf(__uint_as_float(sv[e]), sl2, -Ls[e1]));
-                            dsv[e] = p[e] * (__uint_as_float(pv[e]) - Ds[e1]);
-                        }
-                    }
-                    if (!full) {
-#pragma unroll
-                        for (int e = 0; e < 32; ++e) {
-                            const int qb = (col0 + e) / g.BT;
-                            if (!((allow >> qb) & 1u)) {
-                                p[e] = 0.f;
-                                dsv[e] = 0.f;
-                            }
-                        }
+                        if (!(e4 < 4 ? ok0 : ok1)) L4 = make_float4(INFINITY, INFINITY, INFINITY, INFINITY);
+                        const int e = 4 * e4;
+                        float t0, t1, t2, t3;
+                        ffma2(t0, t1, __uint_as_float(sv[e]), __uint_as_float(sv[e + 1]), sl2, sl2, -L4.x, -L4.y);
+                        ffma2(t2, t3, __uint_as_float(sv[e + 2]), __uint_as_float(sv[e + 3]), sl2, sl2, -L4.z, -L4.w);
+                        const float p0 = ex2_approx(t0), p1 = ex2_approx(t1), p2 = ex2_approx(t2), p3 = ex2_approx(t3);
+                        float d0, d1, d2, d3;
+                        fadd2(d0, d1, __uint_as_float(pv[e]), __uint_as_float(pv[e + 1]), -D4.x, -D4.y);
+                        fadd2(d2, d3, __uint_as_float(pv[e + 2]), __uint_as_float(pv[e + 3]), -D4.z, -D4.w);
+                        fmul2(d0, d1, d0, d1, p0, p1);
+                        fmul2(d2, d3, d2, d3, p2, p3);
+                        wp[2 * e4] = pack_bf16x2(p0, p1);
+                        wp[2 * e4 + 1] = pack_bf16x2(p2, p3);
+                        wd[2 * e4] = pack_f16x2(d0, d1);
+                        wd[2 * e4 + 1] = pack_f16x2(d2, d3);
                     }
                     if (c == 0 && started) {
                         if (!mbar_wait(&bars->mma2_done, mph, ctl, 0x1402)) { ok = false; break; }
                         mph ^= 1;
                         tc_fence_after();
-                    }
-                    uint32_t wp[16], wd[16];
-#pragma unroll
-                    for (int e = 0; e < 16; ++e) {
-                        wp[e] = pack_bf16x2(p[2 * e], p[2 * e + 1]);
-                        wd[e] = pack_f16x2(dsv[2 * e], dsv[2 * e + 1]);
                     }
                     tmem_st16(tmem + lane_off + kColP + col0 / 2, wp);
                     tmem_st16(tmem + lane_off + kColDS + col0 / 2, wd);
@@ -540,11 +533,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                 float* buf = dqst + (j & 1) * kTile * kHeadDim;
                 if (leader) bulk_wait_read_but1();
                 named_bar_sync(1, 128);
+                // fp32 tile image, chunk c of row r at chunk position c ^ (r & 7)
                 float4* rowp = reinterpret_cast<float4*>(buf + r * kHeadDim);
 #pragma unroll
-                for (int c0 = 0; c0 < 8; ++c0) {
-                    const int c = (c0 + lane) & 7;
-                    rowp[c] = make_float4(__uint_as_float(v[4 * c]) * prm.scale, __uint_as_float(v[4 * c + 1]) * prm.scale,
+                for (int c = 0; c < 8; ++c) {
+                    rowp[c ^ (r & 7)] = make_float4(__uint_as_float(v[4 * c]) * prm.scale, __uint_as_float(v[4 * c + 1]) * prm.scale,
                                           __uint_as_float(v[4 * c + 2]) * prm.scale,
                                           __uint_as_float(v[4 * c + 3]) * prm.scale);
                 }
@@ -574,9 +567,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             {
                 float4* rowp = reinterpret_cast<float4*>(dkst + r * kHeadDim);
 #pragma unroll
-                for (int c0 = 0; c0 < 8; ++c0) {
-                    const int c = (c0 + lane) & 7;
-                    rowp[c] = make_float4(__uint_as_float(kk[4 * c]) * prm.scale, __uint_as_float(kk[4 * c + 1]) * prm.scale,
+                for (int c = 0; c < 8; ++c) {
+                    rowp[c ^ (r & 7)] = make_float4(__uint_as_float(kk[4 * c]) * prm.scale, __uint_as_float(kk[4 * c + 1]) * prm.scale,
                                           __uint_as_float(kk[4 * c + 2]) * prm.scale,
                                           __uint_as_float(kk[4 * c + 3]) * prm.scale);
                 }
@@ -590,10 +582,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (leader) {
                 const size_t hu = static_cast<size_t>(I.h) * tiles + static_cast<size_t>(I.u);
                 bulk_store(prm.ws + prm.L.dkimg + hu * kTile * kHeadDim * 4, dkst, kTile * kHeadDim * 4);
-                for (int i = 0; i < g.bpt; ++i) {
-                    const Box bx = box_of(g, I.u * g.bpt + i);
-                    if (bx.valid) tma_store_5d(&map_dv, dvst + i * g.BT * kRowBytes, 0, I.h, bx.col0, bx.row0, bx.b);
-                }
+                tile_tma(g, &map_dv, dvst, nullptr, I.u, I.h, true);
                 bulk_commit();
             }
         }
@@ -628,7 +617,7 @@ __global__ void __launch_bounds__(128) post_kernel(const PostParams p) {
         const float4* ak = reinterpret_cast<const float4*>(p.ws + p.L.dkimg + (ht * kTile + r) * kHeadDim * 4);
 #pragma unroll
         for (int c = 0; c < 8; ++c) {
-            const float4 a = aq[c], b = ak[c];
+            const float4 a = aq[c ^ (r & 7)], b = ak[c ^ (r & 7)];  // swizzled fp32 tile images
             dq[4 * c] = a.x; dq[4 * c + 1] = a.y; dq[4 * c + 2] = a.z; dq[4 * c + 3] = a.w;
             dk[4 * c] = b.x; dk[4 * c + 1] = b.y; dk[4 * c + 2] = b.z; dk[4 * c + 3] = b.w;
         }

@@ -4,9 +4,10 @@
 // 128-row query tiles (A and B) that share one stream of key/value tiles:
 //   warps 0-3  softmax for tile A (thread = query row = TMEM lane)
 //   warps 4-7  softmax for tile B
-//   warps 8-11 RoPE: rotate Q and K tiles in shared memory as they land
-//   warp 12    TMA producer (window boxes at shifted addresses, no gather copy)
-//   warp 13    tcgen05 MMA issuer: S = Q'K'^T and O_tile = P V into TMEM
+//   warp 8     RoPE: rotate Q and K tiles in shared memory as they land
+//   warp 9     TMA producer (window boxes at shifted addresses, no gather copy)
+//   warps 10-11 tcgen05 MMA issuers, one per query tile (they never wait on each
+//              other): S = Q'K'^T and O_tile = P V into TMEM
 // The online softmax keeps O in registers and folds in each P V tile product,
 // rescaling only when the running maximum grows by more than 2^8 (exact: the
 // final normalisation uses the same maximum as the sum).
@@ -17,14 +18,17 @@
 #include "kernels.cuh"
 #include "ptx.cuh"
 #include "schedule.cuh"
+#include "tile_io.cuh"
+#include "dgeo.cuh"
 
 namespace fswin {
 
 namespace fwdk {
 
-constexpr int kThreads = 448;
+// 12 warps: 3 per SM sub-partition, so each thread may hold up to 168 registers.
+constexpr int kThreads = 384;
 constexpr int kStages = 6;
-constexpr int kWarpRot = 8, kWarpTma = 12, kWarpMma = 13;
+constexpr int kWarpRot = 8, kRotWarps = 1, kWarpTma = 9, kWarpMma = 10;  // MMA: warps 10 (tile A), 11 (tile B)
 
 // shared-memory layout (offsets from a 1024-byte aligned base)
 constexpr int kQOff = 0;                                   // 2 slots x 2 tiles
@@ -43,7 +47,7 @@ __device__ __forceinline__ uint32_t col_o(int T) { return T * 256 + 192; }
 struct Bars {
     uint64_t q_full[2], q_ready[2], q_empty[2];
     uint64_t kv_full[kStages], kv_ready[kStages], kv_empty[kStages];
-    uint64_t s_full[2], p_full[2], o_full[2];
+    uint64_t s_full[2], s_free[2], p_full[2], o_full[2];
     uint64_t done;
     uint32_t tmem_base;
     int abort_flag;
@@ -58,66 +62,70 @@ struct Params {
     long long items;
 };
 
-using Item = FwdItem;
-__device__ __forceinline__ Item item_of(const Geo& g, long long it) { return fwd_item(g, it); }
-__device__ __forceinline__ bool active(const Geo& g, const Item& I, int T, int u) { return fwd_active(g, I, T, u); }
-
-__device__ __forceinline__ void load_tile_boxes(const Geo& g, const CUtensorMap* map, uint8_t* dst, uint64_t* bar,
-                                                long long tile, int h) {
-    for (int i = 0; i < g.bpt; ++i) {
-        const Box bx = box_of(g, tile * g.bpt + i);
-        tma_load_5d(dst + i * g.BT * kRowBytes, map, bar, 0, h, bx.col0, bx.row0, bx.b);
-    }
-}
-
 // Rotate token row r of a swizzled (64-byte swizzle) tile in place: bf16 in,
 // fp16 out (the rotated operands of S = Q'K'^T are held in fp16, whose 11-bit
 // significand keeps their rounding well below the bf16 rounding of the inputs).
-__device__ __forceinline__ void rope_row(uint8_t* tile, int r, int pi, int pj, const float2* tab) {
+// All loads first, then the arithmetic, then all stores: the row and the table
+// are both in shared memory, so interleaving would serialise every chunk.
+__device__ __noinline__ void rope_row(uint8_t* __restrict__ tile, int r, int pi, int pj,
+                                      const float2* __restrict__ tab) {
     uint8_t* row = tile + r * kRowBytes;
     const int sw = (r >> 1) & 3;
+    uint4 v[4];
+    float4 t[8];  // (cos, sin) of the 16 channel pairs
+#pragma unroll
+    for (int c = 0; c < 4; ++c) v[c] = *reinterpret_cast<const uint4*>(row + ((c ^ sw) << 4));
+    const float4* tx = reinterpret_cast<const float4*>(tab + pj * 8);
+    const float4* ty = reinterpret_cast<const float4*>(tab + (64 + pi) * 8);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        t[q] = tx[q];
+        t[4 + q] = ty[q];
+    }
 #pragma unroll
     for (int c = 0; c < 4; ++c) {
-        uint4* p = reinterpret_cast<uint4*>(row + ((c ^ sw) << 4));
-        uint4 v = *p;
-        const int ax = c >> 1;
-        const float2* t = tab + (ax * 64 + (ax ? pi : pj)) * 8 + (c & 1) * 4;
-        uint32_t w[4] = {v.x, v.y, v.z, v.w};
+        uint32_t w[4] = {v[c].x, v[c].y, v[c].z, v[c].w};
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
+            const int pr = 4 * c + e;  // channel pair 0..15 (0-7: x axis, 8-15: y axis)
+            const float4 tt = t[pr >> 1];
+            const float cs = (pr & 1) ? tt.z : tt.x, sn = (pr & 1) ? tt.w : tt.y;
             const float a = bf16lo_to_f32(w[e]), b = bf16hi_to_f32(w[e]);
-            const float2 cs = t[e];
-            w[e] = pack_f16x2(a * cs.x - b * cs.y, a * cs.y + b * cs.x);
+            w[e] = pack_f16x2(a * cs - b * sn, a * sn + b * cs);
         }
-        *p = make_uint4(w[0], w[1], w[2], w[3]);
+        v[c] = make_uint4(w[0], w[1], w[2], w[3]);
     }
+#pragma unroll
+    for (int c = 0; c < 4; ++c) *reinterpret_cast<uint4*>(row + ((c ^ sw) << 4)) = v[c];
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
     fwd_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
                const __grid_constant__ CUtensorMap map_v, const __grid_constant__ CUtensorMap map_o,
-               const Params prm) {
+               const __grid_constant__ Params prm) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     Bars* bars = reinterpret_cast<Bars*>(smem + kBarOff);
     const Geo& g = prm.g;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
+    FS_TRACE_INIT();
     if (tid == 0) {
         for (int i = 0; i < 2; ++i) {
             mbar_init(&bars->q_full[i], 1);
-            mbar_init(&bars->q_ready[i], 4);
-            mbar_init(&bars->q_empty[i], 1);
+            mbar_init(&bars->q_ready[i], kRotWarps);
+            mbar_init(&bars->q_empty[i], 2);  // one commit per MMA-issuing thread
             mbar_init(&bars->s_full[i], 1);
             mbar_init(&bars->p_full[i], 4);
+            mbar_init(&bars->s_free[i], 4);
             mbar_init(&bars->o_full[i], 1);
         }
         for (int i = 0; i < kStages; ++i) {
             mbar_init(&bars->kv_full[i], 1);
-            mbar_init(&bars->kv_ready[i], 4);
-            mbar_init(&bars->kv_empty[i], 1);
+            mbar_init(&bars->kv_ready[i], kRotWarps);
+            mbar_init(&bars->kv_empty[i], 2);  // one arrival per MMA-issuing thread
         }
-        mbar_init(&bars->done, 1);
+        mbar_init(&bars->done, 2);
         bars->abort_flag = 0;
         fence_mbar_init();
     }
@@ -139,132 +147,158 @@ __global__ void __launch_bounds__(kThreads, 1)
             prefetch_tmap(&map_v);
             int it = 0;
             uint32_t kvc = 0;
-            for (long long item = blockIdx.x; item < prm.items; item += gridDim.x, ++it) {
-                const Item I = item_of(g, item);
+            bool ok = true;
+            for (long long item = blockIdx.x; item < prm.items && ok; item += gridDim.x, ++it) {
+                const FwdItem I = d_fwd_item(g, item);
                 const int qi = it & 1;
                 if (!mbar_wait(&bars->q_empty[qi], ((it >> 1) & 1) ^ 1, ctl, 0x101)) break;
                 uint8_t* qs = smem + kQOff + qi * 2 * kTileBytes;
                 mbar_arrive_expect_tx(&bars->q_full[qi], (I.tB >= 0 ? 2 : 1) * kTileBytes);
-                load_tile_boxes(g, &map_q, qs, &bars->q_full[qi], I.tA, I.h);
-                if (I.tB >= 0) load_tile_boxes(g, &map_q, qs + kTileBytes, &bars->q_full[qi], I.tB, I.h);
-                bool ok = true;
-                for (int u = 0; u < I.nkv && ok; ++u) {
-                    if (!active(g, I, 0, u) && !active(g, I, 1, u)) continue;
+                tile_tma(g, &map_q, qs, &bars->q_full[qi], I.tA, I.h, false);
+                if (I.tB >= 0) tile_tma(g, &map_q, qs + kTileBytes, &bars->q_full[qi], I.tB, I.h, false);
+                const uint32_t used = I.act[0] | I.act[1];
+                for (int u = 0; u < I.nkv; ++u) {
+                    if (!((used >> u) & 1u)) continue;
                     const int st = kvc % kStages;
                     const uint32_t ph = (kvc / kStages) & 1;
                     ++kvc;
                     if (!mbar_wait(&bars->kv_empty[st], ph ^ 1, ctl, 0x102)) { ok = false; break; }
                     uint8_t* ks = smem + kKVOff + st * 2 * kTileBytes;
                     mbar_arrive_expect_tx(&bars->kv_full[st], 2 * kTileBytes);
-                    load_tile_boxes(g, &map_k, ks, &bars->kv_full[st], I.kv0 + u, I.h);
-                    load_tile_boxes(g, &map_v, ks + kTileBytes, &bars->kv_full[st], I.kv0 + u, I.h);
+                    tile_tma(g, &map_k, ks, &bars->kv_full[st], I.kv0 + u, I.h, false);
+                    tile_tma(g, &map_v, ks + kTileBytes, &bars->kv_full[st], I.kv0 + u, I.h, false);
                 }
-                if (!ok) break;
             }
         }
-    } else if (warp >= kWarpRot && warp < kWarpRot + 4) {
+    } else if (warp >= kWarpRot && warp < kWarpRot + kRotWarps) {
         // ------------------------------------------------------------ RoPE
-        const int r = tid - kWarpRot * 32;
+        const int r0 = tid - kWarpRot * 32;  // rows r0, r0 + 32, ... of every tile
+        constexpr int kRotThreads = kRotWarps * 32;
         int it = 0;
         uint32_t kvc = 0;
         bool ok = true;
+        int tab_head = -1, tab_buf = 1;
         for (long long item = blockIdx.x; item < prm.items && ok; item += gridDim.x, ++it) {
-            const Item I = item_of(g, item);
-            float2* tab = reinterpret_cast<float2*>(smem + kTabOff) + (it & 1) * (2 * 64 * 8);
-            const float* th = prm.theta + I.h * 16;
-            for (int e = r; e < 2 * g.M * 8; e += 128) {
-                const int ax = e / (g.M * 8), rem = e - ax * g.M * 8, pos = rem >> 3, k = rem & 7;
-                float sn, cs;
-                sincosf(static_cast<float>(pos) * th[ax * 8 + k], &sn, &cs);
-                tab[(ax * 64 + pos) * 8 + k] = make_float2(cs, sn);
+            const FwdItem I = d_fwd_item(g, item);
+            // cos/sin table of the item's head, rebuilt only when the head changes
+            // (double-buffered; the barrier orders it against the previous rotations)
+            if (I.h != tab_head) {
+                tab_buf ^= 1;
+                tab_head = I.h;
+                float2* tw = reinterpret_cast<float2*>(smem + kTabOff) + tab_buf * (2 * 64 * 8);
+                const float* th = prm.theta + I.h * 16;
+                for (int e = r0; e < 2 * g.M * 8; e += kRotThreads) {
+                    const int ax = e / (g.M * 8), rem = e - ax * g.M * 8, pos = rem >> 3, k = rem & 7;
+                    float sn, cs;
+                    sincosf(static_cast<float>(pos) * th[ax * 8 + k], &sn, &cs);
+                    tw[(ax * 64 + pos) * 8 + k] = make_float2(cs, sn);
+                }
+                named_bar_sync(1, kRotThreads);
             }
-            named_bar_sync(1, 128);
+            const float2* tab = reinterpret_cast<const float2*>(smem + kTabOff) + tab_buf * (2 * 64 * 8);
             const int qi = it & 1;
             if (!mbar_wait(&bars->q_full[qi], (it >> 1) & 1, ctl, 0x201)) break;
             uint8_t* qs = smem + kQOff + qi * 2 * kTileBytes;
-            {
-                const Slot sa = slot_of(g, I.tA, r);
-                rope_row(qs, r, sa.i, sa.j, tab);
+#pragma unroll 1
+            for (int h2 = 0; h2 < kTile / kRotThreads; ++h2) {
+                const int r = r0 + h2 * kRotThreads;
+                int pi, pj;
+                tile_row_pos(g, I.tA, r, &pi, &pj);
+                rope_row(qs, r, pi, pj, tab);
                 if (I.tB >= 0) {
-                    const Slot sb = slot_of(g, I.tB, r);
-                    rope_row(qs + kTileBytes, r, sb.i, sb.j, tab);
+                    tile_row_pos(g, I.tB, r, &pi, &pj);
+                    rope_row(qs + kTileBytes, r, pi, pj, tab);
                 }
             }
             fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0) mbar_arrive(&bars->q_ready[qi]);
+            const uint32_t used = I.act[0] | I.act[1];
             for (int u = 0; u < I.nkv; ++u) {
-                if (!active(g, I, 0, u) && !active(g, I, 1, u)) continue;
+                if (!((used >> u) & 1u)) continue;
                 const int st = kvc % kStages;
                 const uint32_t ph = (kvc / kStages) & 1;
                 ++kvc;
                 if (!mbar_wait(&bars->kv_full[st], ph, ctl, 0x202)) { ok = false; break; }
-                const Slot sk = slot_of(g, I.kv0 + u, r);
-                rope_row(smem + kKVOff + st * 2 * kTileBytes, r, sk.i, sk.j, tab);
+#pragma unroll 1
+                for (int h2 = 0; h2 < kTile / kRotThreads; ++h2) {
+                    const int r = r0 + h2 * kRotThreads;
+                    int pi, pj;
+                    tile_row_pos(g, I.kv0 + u, r, &pi, &pj);
+                    rope_row(smem + kKVOff + st * 2 * kTileBytes, r, pi, pj, tab);
+                }
                 fence_proxy_async_smem();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&bars->kv_ready[st]);
             }
         }
-    } else if (warp == kWarpMma) {
-        // ------------------------------------------------------------ MMA issue
+    } else if (warp == kWarpMma || warp == kWarpMma + 1) {
+        // ------------------------------------------------------------ MMA issue, one thread per query tile
         if (lane == 0) {
+            const int T = warp - kWarpMma;
             const uint32_t idesc_qk = make_idesc(kTile, kTile, false, false, true);  // fp16 Q', K'
             const uint32_t idesc_pv = make_idesc_bf16(kTile, kHeadDim, false, true);
+            // Shared-memory descriptors built once; per MMA only an offset (in 16-byte
+            // units) is added to the start-address field.
+            const uint64_t dq0 = make_sdesc(smem_u32(smem + kQOff + T * kTileBytes), 16, 512, kSw64);
+            const uint64_t dk0 = make_sdesc(smem_u32(smem + kKVOff), 16, 512, kSw64);
+            const uint64_t dv0 = make_sdesc(smem_u32(smem + kKVOff + kTileBytes), 8192, 512, kSw64);
+            constexpr uint32_t kStep = (2 * kTileBytes) >> 4;  // next Q slot / next K,V stage
+            const uint32_t t_s = tmem + col_s(T), t_p = tmem + col_p(T), t_o = tmem + col_o(T);
             int it = 0;
-            uint32_t kvc = 0;
-            uint32_t pph[2] = {0, 0};
+            uint32_t kvc = 0, pph = 0, sfph = 0;
             bool ok = true;
-            auto issue_pv = [&](int T, int st) {
-                const uint32_t vaddr = smem_u32(smem + kKVOff + st * 2 * kTileBytes + kTileBytes);
+            auto issue_pv = [&](int st) {
+                const uint64_t dv = dv0 + static_cast<uint64_t>(st) * kStep;
 #pragma unroll
-                for (int k = 0; k < kTile / 16; ++k)
-                    umma_ts(tmem + col_o(T), tmem + col_p(T) + 8 * k, make_sdesc(vaddr + 1024 * k, 8192, 512, kSw64),
-                            idesc_pv, k > 0);
+                for (int k = 0; k < kTile / 16; ++k) umma_ts(t_o, t_p + 8 * k, dv + 64 * k, idesc_pv, k > 0);
                 umma_commit(&bars->o_full[T]);
+                umma_commit(&bars->kv_empty[st]);
             };
             for (long long item = blockIdx.x; item < prm.items && ok; item += gridDim.x, ++it) {
-                const Item I = item_of(g, item);
+                const FwdItem I = d_fwd_item(g, item);
                 const int qi = it & 1;
                 if (!mbar_wait(&bars->q_ready[qi], (it >> 1) & 1, ctl, 0x301)) break;
-                tc_fence_after();
-                const uint32_t qaddr = smem_u32(smem + kQOff + qi * 2 * kTileBytes);
-                int pend[2] = {-1, -1};
-                int readers[kStages];
+                const uint64_t dq = dq0 + static_cast<uint64_t>(qi) * kStep;
+                const uint32_t mine = I.act[T], used = I.act[0] | I.act[1];
+                int pend = -1;
                 for (int u = 0; u < I.nkv && ok; ++u) {
-                    const bool aA = active(g, I, 0, u), aB = active(g, I, 1, u);
-                    if (!aA && !aB) continue;
+                    if (!((used >> u) & 1u)) continue;
                     const int st = kvc % kStages;
                     const uint32_t ph = (kvc / kStages) & 1;
                     ++kvc;
                     if (!mbar_wait(&bars->kv_ready[st], ph, ctl, 0x302)) { ok = false; break; }
-                    tc_fence_after();
-                    readers[st] = (aA ? 1 : 0) + (aB ? 1 : 0);
-                    const uint32_t kaddr = smem_u32(smem + kKVOff + st * 2 * kTileBytes);
-                    for (int T = 0; T < 2; ++T) {
-                        if (!(T ? aB : aA)) continue;
-                        if (pend[T] >= 0) {
-                            if (!mbar_wait(&bars->p_full[T], pph[T], ctl, 0x303 + T)) { ok = false; break; }
-                            pph[T] ^= 1;
-                            tc_fence_after();
-                            issue_pv(T, pend[T]);
-                            if (--readers[pend[T]] == 0) umma_commit(&bars->kv_empty[pend[T]]);
-                        }
-#pragma unroll
-                        for (int k = 0; k < kHeadDim / 16; ++k)
-                            umma_ss(tmem + col_s(T), make_sdesc(qaddr + T * kTileBytes + 32 * k, 16, 512, kSw64),
-                                    make_sdesc(kaddr + 32 * k, 16, 512, kSw64), idesc_qk, k > 0);
-                        umma_commit(&bars->s_full[T]);
-                        pend[T] = st;
+                    if (!((mine >> u) & 1u)) {  // only the other query tile reads this stage
+                        mbar_arrive(&bars->kv_empty[st]);
+                        continue;
                     }
-                }
-                for (int T = 0; T < 2 && ok; ++T) {
-                    if (pend[T] < 0) continue;
-                    if (!mbar_wait(&bars->p_full[T], pph[T], ctl, 0x305 + T)) { ok = false; break; }
-                    pph[T] ^= 1;
                     tc_fence_after();
-                    issue_pv(T, pend[T]);
-                    if (--readers[pend[T]] == 0) umma_commit(&bars->kv_empty[pend[T]]);
+                    // the next S = Q K^T as soon as the softmax has read the previous S,
+                    // then P V of the previous tile once its P is in TMEM
+                    if (pend >= 0) {
+                        if (!mbar_wait(&bars->s_free[T], sfph, ctl, 0x307 + T)) { ok = false; break; }
+                        sfph ^= 1;
+                        tc_fence_after();
+                    }
+                    const uint64_t dk = dk0 + static_cast<uint64_t>(st) * kStep;
+                    umma_ss(t_s, dq, dk, idesc_qk, 0u);
+                    umma_ss(t_s, dq + 2, dk + 2, idesc_qk, 1u);  // second 16-channel step: +32 bytes
+                    umma_commit(&bars->s_full[T]);
+                    if (pend >= 0) {
+                        if (!mbar_wait(&bars->p_full[T], pph, ctl, 0x303 + T)) { ok = false; break; }
+                        pph ^= 1;
+                        tc_fence_after();
+                        issue_pv(pend);
+                    }
+                    pend = st;
+                }
+                if (ok && pend >= 0) {
+                    if (!mbar_wait(&bars->s_free[T], sfph, ctl, 0x309 + T)) break;
+                    sfph ^= 1;
+                    if (!mbar_wait(&bars->p_full[T], pph, ctl, 0x305 + T)) break;
+                    pph ^= 1;
+                    tc_fence_after();
+                    issue_pv(pend);
                 }
                 umma_commit(&bars->q_empty[qi]);
             }
@@ -286,29 +320,30 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint32_t sph = 0, oph = 0;
         bool ok = true;
         for (long long item = blockIdx.x; item < prm.items && ok; item += gridDim.x) {
-            const Item I = item_of(g, item);
+            const FwdItem I = d_fwd_item(g, item);
             if (T == 1 && I.tB < 0) continue;
             const long long X = T ? I.tB : I.tA;
-            const Slot me = slot_of(g, X, r);
-            const long long myseg = seg_of(me.box);
+            const Win wq = I.paired ? d_tile_win(g, X) : I.win;
+            const uint32_t myseg = seg_at(d_tile_segs(g, X, wq), r >> g.lBT);
+            const uint32_t myact = T ? I.act[1] : I.act[0];
             float o[32];
 #pragma unroll
             for (int e = 0; e < 32; ++e) o[e] = 0.f;
             float m = -INFINITY, l = 0.f;
             bool first = true;
             for (int u = 0; u < I.nkv; ++u) {
-                if (!active(g, I, T, u)) continue;
-                const uint32_t allow = allow_mask(g, myseg, I.kv0 + u);
-                const bool full = allow == ((1u << g.bpt) - 1u);
+                if (!((myact >> u) & 1u)) continue;
+                const uint32_t a16 = d_allow16(g, myseg, I.kv0 + u, wq);
+                const bool full = a16 == 0xFFu;
                 if (!mbar_wait(&bars->s_full[T], sph, ctl, 0x401 + T)) { ok = false; break; }
                 sph ^= 1;
                 tc_fence_after();
-                // pass 1: row maximum of the raw scores
+                // pass 1: row maximum of the attended raw scores
                 float mx8[8];
 #pragma unroll
                 for (int e = 0; e < 8; ++e) mx8[e] = -INFINITY;
-#pragma unroll
-                for (int c = 0; c < 4; ++c) {
+#pragma unroll 1
+                for (int c = 0; c < 4; ++c) {  // rolled: keeps live ranges (registers) short
                     uint32_t v[32];
                     tmem_ld32(t_s + 32 * c, v);
                     tmem_wait_ld();
@@ -316,10 +351,11 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                         for (int e = 0; e < 32; ++e) mx8[e & 7] = fmaxf(mx8[e & 7], __uint_as_float(v[e]));
                     } else {
+                        const bool ok0 = (a16 >> (2 * c)) & 1u, ok1 = (a16 >> (2 * c + 1)) & 1u;
 #pragma unroll
                         for (int e = 0; e < 32; ++e) {
-                            const int kb = (32 * c + e) / g.BT;
-                            if ((allow >> kb) & 1u) mx8[e & 7] = fmaxf(mx8[e & 7], __uint_as_float(v[e]));
+                            const float x = (e < 16 ? ok0 : ok1) ? __uint_as_float(v[e]) : -INFINITY;
+                            mx8[e & 7] = fmaxf(mx8[e & 7], x);
                         }
                     }
                 }
@@ -334,38 +370,43 @@ __global__ void __launch_bounds__(kThreads, 1)
                     tmem_ld32(t_o, v);
                     tmem_wait_ld();
 #pragma unroll
-                    for (int e = 0; e < 32; ++e) o[e] += __uint_as_float(v[e]);
+                    for (int e = 0; e < 32; e += 2)
+                        fadd2(o[e], o[e + 1], o[e], o[e + 1], __uint_as_float(v[e]), __uint_as_float(v[e + 1]));
                 }
                 if (m_tile > m + 8.f) {
                     const float alpha = ex2_approx(m - m_tile);
 #pragma unroll
-                    for (int e = 0; e < 32; ++e) o[e] *= alpha;
+                    for (int e = 0; e < 32; e += 2) fmul2(o[e], o[e + 1], o[e], o[e + 1], alpha, alpha);
                     l *= alpha;
                     m = m_tile;
                 }
                 const float mu = (m == -INFINITY) ? 0.f : m;
                 // pass 2: probabilities, row sum, bf16 P into TMEM
+                // A masked 16-column group gets the addend -inf: its scores map to
+                // exp2(-inf) = 0 with no extra instruction.
                 float l4[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
+#pragma unroll 1
                 for (int c = 0; c < 4; ++c) {
                     uint32_t v[32];
                     tmem_ld32(t_s + 32 * c, v);
                     tmem_wait_ld();
-                    float p[32];
-#pragma unroll
-                    for (int e = 0; e < 32; ++e) p[e] = ex2_approx(fmaf(__uint_as_float(v[e]), sl2, -mu));
-                    if (!full) {
-#pragma unroll
-                        for (int e = 0; e < 32; ++e) {
-                            const int kb = (32 * c + e) / g.BT;
-                            if (!((allow >> kb) & 1u)) p[e] = 0.f;
-                        }
+                    if (c == 3) {  // S fully read: the next S = Q K^T may overwrite it
+                        tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(&bars->s_free[T]);
                     }
+                    const float add0 = ((a16 >> (2 * c)) & 1u) ? -mu : -INFINITY;
+                    const float add1 = ((a16 >> (2 * c + 1)) & 1u) ? -mu : -INFINITY;
                     uint32_t w[16];
 #pragma unroll
                     for (int e = 0; e < 16; ++e) {
-                        l4[e & 3] += p[2 * e] + p[2 * e + 1];
-                        w[e] = pack_bf16x2(p[2 * e], p[2 * e + 1]);
+                        const float ad = e < 8 ? add0 : add1;
+                        float t0, t1;
+                        ffma2(t0, t1, __uint_as_float(v[2 * e]), __uint_as_float(v[2 * e + 1]), sl2, sl2, ad, ad);
+                        const float p0 = ex2_approx(t0), p1 = ex2_approx(t1);
+                        const int a = (e & 1) * 2;
+                        fadd2(l4[a], l4[a + 1], l4[a], l4[a + 1], p0, p1);
+                        w[e] = pack_bf16x2(p0, p1);
                     }
                     tmem_st16(t_p + 16 * c, w);
                 }
@@ -385,7 +426,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tmem_ld32(t_o, v);
                 tmem_wait_ld();
 #pragma unroll
-                for (int e = 0; e < 32; ++e) o[e] += __uint_as_float(v[e]);
+                for (int e = 0; e < 32; e += 2)
+                        fadd2(o[e], o[e + 1], o[e], o[e + 1], __uint_as_float(v[e]), __uint_as_float(v[e + 1]));
             }
             const float inv = 1.f / l;
             // epilogue: O row into the staging tile (64-byte swizzle), then TMA stores
@@ -407,12 +449,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             fence_proxy_async_smem();
             named_bar_sync(2 + T, 128);
             if (leader) {
-                for (int i = 0; i < g.bpt; ++i) {
-                    const Box bx = box_of(g, X * g.bpt + i);
-                    if (bx.valid) tma_store_5d(&map_o, ost + i * g.BT * kRowBytes, 0, I.h, bx.col0, bx.row0, bx.b);
-                }
+                tile_tma(g, &map_o, ost, nullptr, X, I.h, true);
                 bulk_commit();
             }
+            const Slot me = d_slot_of(g, X, r);
             if (me.box.valid) {
                 const float lse2 = m + lg2_approx(l);
                 const long long tok =

@@ -9,6 +9,9 @@
 // tile when windows are smaller (several windows per tile, separated by a
 // block-diagonal mask).  Two tokens attend to each other iff they share the
 // window and the shift-region label (the Swin shifted-window rule).
+//
+// Every extent below is a power of two, so the per-row and per-tile helpers
+// use shifts and masks; integer division only happens once per window.
 #pragma once
 
 #include <cstdint>
@@ -17,7 +20,7 @@ namespace fswin {
 
 constexpr int kTile = 128;                  // token rows per tile
 constexpr int kHeadDim = 32;                // supported head dimension
-constexpr int kRowBytes = kHeadDim * 2;     // one bf16 token row
+constexpr int kRowBytes = kHeadDim * 2;     // one 16-bit token row
 constexpr int kTileBytes = kTile * kRowBytes;
 
 struct Geo {
@@ -28,10 +31,18 @@ struct Geo {
     int nbc, nbw;       // boxes per window row, per window
     int bpt;            // boxes per tile
     int tpw;            // tiles per window (N >= 128), else 0
+    int wpt;            // windows per tile (N < 128), else 0
+    int lbh, lbw, lBT, lnbc, lnbw, lbpt, ltpw, lwpt;  // log2 of the above
     long long wins;     // windows in the batch
     long long tiles;    // tiles per head
     float scale_log2;   // log2(e) / sqrt(d)
 };
+
+__host__ __device__ inline int ilog2_exact(int x) {
+    int l = 0;
+    while ((1 << l) < x) ++l;
+    return l;
+}
 
 // Builds the geometry of a problem.  Returns 0 on success, 2 for an
 // unsupported shape (the FS_ERR_SHAPE code of the C ABI).
@@ -66,6 +77,15 @@ inline int geo_init(Geo* g, int B, int H, int W, int heads, int d, int M, int s)
     x.nbw = (M / x.bh) * (M / x.bw);
     x.bpt = kTile / x.BT;
     x.tpw = x.N >= kTile ? x.N / kTile : 0;
+    x.wpt = x.N < kTile ? kTile / x.N : 0;
+    x.lbh = ilog2_exact(x.bh);
+    x.lbw = ilog2_exact(x.bw);
+    x.lBT = ilog2_exact(x.BT);
+    x.lnbc = ilog2_exact(x.nbc);
+    x.lnbw = ilog2_exact(x.nbw);
+    x.lbpt = ilog2_exact(x.bpt);
+    x.ltpw = x.tpw ? ilog2_exact(x.tpw) : 0;
+    x.lwpt = x.wpt ? ilog2_exact(x.wpt) : 0;
     x.wins = static_cast<long long>(B) * x.nW;
     x.tiles = (x.wins * x.N + kTile - 1) / kTile;
     x.scale_log2 = 1.4426950408889634f / 5.656854249492380195f;  // log2(e) / sqrt(32)
@@ -77,9 +97,113 @@ __host__ __device__ inline int region_of(int X, int M, int s, int x) {
     return x < X - M ? 0 : (x < X - s ? 1 : 2);
 }
 
+// A window of the batch in the rolled frame.
+struct Win {
+    long long gw;
+    int b, wr, wc;
+    bool valid;
+};
+
+__host__ __device__ inline Win win_of(const Geo& g, long long gw) {
+    Win w;
+    w.gw = gw;
+    w.valid = gw < g.wins;
+    w.b = static_cast<int>(gw / g.nW);  // >= B for padding windows: TMA then zero-fills
+    const int r = static_cast<int>(gw - static_cast<long long>(w.b) * g.nW);
+    w.wr = r / g.nWw;
+    w.wc = r - w.wr * g.nWw;
+    return w;
+}
+
+// Box x (0 .. bpt-1) of a tile: its window and its index k inside the window.
+__host__ __device__ inline void tile_box(const Geo& g, long long tile, int x, long long* gw, int* k) {
+    if (g.tpw) {
+        *gw = tile >> g.ltpw;
+        *k = (static_cast<int>(tile & (g.tpw - 1)) << g.lbpt) + x;
+    } else {
+        *gw = (tile << g.lwpt) + (x >> g.lnbw);
+        *k = x & (g.nbw - 1);
+    }
+}
+
+// Rolled coordinates of the first token of box k of window w.
+__host__ __device__ inline int box_r(const Geo& g, const Win& w, int k) { return w.wr * g.M + ((k >> g.lnbc) << g.lbh); }
+__host__ __device__ inline int box_c(const Geo& g, const Win& w, int k) {
+    return w.wc * g.M + ((k & (g.nbc - 1)) << g.lbw);
+}
+
+__host__ __device__ inline int box_label(const Geo& g, const Win& w, int k) {
+    if (!g.s) return 0;
+    return 3 * region_of(g.H, g.M, g.s, box_r(g, w, k)) + region_of(g.W, g.M, g.s, box_c(g, w, k));
+}
+
+// Original (un-rolled) coordinates of the first token of box k of window w.
+__host__ __device__ inline void box_origin(const Geo& g, const Win& w, int k, int* row0, int* col0) {
+    int r = box_r(g, w, k) + g.s, c = box_c(g, w, k) + g.s;
+    if (r >= g.H) r -= g.H;
+    if (c >= g.W) c -= g.W;
+    *row0 = r;
+    *col0 = c;
+}
+
+// In-window position (i = row, j = column) of token slot p of a tile.
+__host__ __device__ inline void tile_row_pos(const Geo& g, long long tile, int p, int* i, int* j) {
+    const int k = g.tpw ? (static_cast<int>(tile & (g.tpw - 1)) << g.lbpt) + (p >> g.lBT) : (p & (g.N - 1)) >> g.lBT;
+    const int q = p & (g.BT - 1);
+    *i = ((k >> g.lnbc) << g.lbh) + (q >> g.lbw);
+    *j = ((k & (g.nbc - 1)) << g.lbw) + (q & (g.bw - 1));
+}
+
+// Segment byte of every box of a tile: (window index inside the tile << 4) |
+// region label.  Two tokens of one group attend iff their boxes' bytes match.
+// `w0` is the tile's (first) window, computed by the caller with win_of.
+__host__ __device__ inline uint64_t tile_segs(const Geo& g, long long tile, const Win& w0) {
+    uint64_t out = 0;
+    if (g.tpw) {
+        if (!g.s) return 0;
+        const int k0 = static_cast<int>(tile & (g.tpw - 1)) << g.lbpt;
+        for (int x = 0; x < g.bpt; ++x) out |= static_cast<uint64_t>(box_label(g, w0, k0 + x)) << (8 * x);
+        return out;
+    }
+    Win w = w0;
+    for (int x = 0; x < g.bpt; ++x) {
+        const int widx = x >> g.lnbw, k = x & (g.nbw - 1);
+        if (k == 0 && widx > 0) w = win_of(g, w0.gw + widx);
+        out |= static_cast<uint64_t>((widx << 4) | box_label(g, w, k)) << (8 * x);
+    }
+    return out;
+}
+
+// First window of a tile.
+__host__ __device__ inline Win tile_win(const Geo& g, long long tile) {
+    return win_of(g, g.tpw ? (tile >> g.ltpw) : (tile << g.lwpt));
+}
+
+__host__ __device__ inline uint32_t seg_at(uint64_t segs, int box) { return static_cast<uint32_t>(segs >> (8 * box)) & 0xFFu; }
+
+// Does some token of tile a attend some token of tile b (same group)?
+__host__ __device__ inline bool segs_meet(const Geo& g, uint64_t a, uint64_t b) {
+    for (int x = 0; x < g.bpt; ++x)
+        for (int y = 0; y < g.bpt; ++y)
+            if (seg_at(a, x) == seg_at(b, y)) return true;
+    return false;
+}
+
+// Bit c (0..7): may a token with segment byte `my` attend the 16 tokens in
+// slots [16 c, 16 c + 16) of a tile with segment bytes `segs`?  (Boxes hold
+// >= 16 tokens, so a 16-slot group never spans two boxes.)
+__host__ __device__ inline uint32_t allow16(const Geo& g, uint32_t my, uint64_t segs) {
+    uint32_t m = 0;
+    for (int c = 0; c < 8; ++c)
+        if (seg_at(segs, (c << 4) >> g.lBT) == my) m |= 1u << c;
+    return m;
+}
+
+// ----------------------------------------------------------------- slow path
+// Full description of a box / token slot (used once per work item at most).
 struct Box {
-    int b;            // image (>= B for padding boxes: TMA then zero-fills)
-    int row0, col0;   // original (un-rolled) coordinates of the first token
+    int b;            // image (>= B for padding boxes)
+    int row0, col0;   // original coordinates of the first token
     int i0, j0;       // in-window coordinates of the first token
     long long gw;     // window index within the batch
     int label;        // shift-region label (0 when s == 0)
@@ -88,33 +212,20 @@ struct Box {
 
 __host__ __device__ inline Box box_of(const Geo& g, long long gbox) {
     Box x;
-    x.gw = gbox / g.nbw;
-    const int k = static_cast<int>(gbox - x.gw * g.nbw);
-    x.valid = x.gw < g.wins;
-    x.b = static_cast<int>(x.gw / g.nW);
-    const int w = static_cast<int>(x.gw - static_cast<long long>(x.b) * g.nW);
-    const int wr = w / g.nWw, wc = w - (w / g.nWw) * g.nWw;
-    const int br = k / g.nbc, bc = k - br * g.nbc;
-    x.i0 = br * g.bh;
-    x.j0 = bc * g.bw;
-    const int r = wr * g.M + x.i0, c = wc * g.M + x.j0;
-    x.label = g.s ? 3 * region_of(g.H, g.M, g.s, r) + region_of(g.W, g.M, g.s, c) : 0;
-    x.row0 = (r + g.s) % g.H;
-    x.col0 = (c + g.s) % g.W;
+    long long gw;
+    int k;
+    tile_box(g, gbox >> g.lbpt, static_cast<int>(gbox & (g.bpt - 1)), &gw, &k);
+    const Win w = win_of(g, gw);
+    x.gw = gw;
+    x.valid = w.valid;
+    x.b = w.b;
+    x.i0 = (k >> g.lnbc) << g.lbh;
+    x.j0 = (k & (g.nbc - 1)) << g.lbw;
+    x.label = box_label(g, w, k);
+    box_origin(g, w, k, &x.row0, &x.col0);
     return x;
 }
 
-// Segment key: tokens attend iff their segment keys are equal.
-__host__ __device__ inline long long seg_of(const Box& x) { return x.gw * 9 + x.label; }
-
-// Bit set of the region labels present in a tile.
-__host__ __device__ inline uint32_t tile_labels(const Geo& g, long long tile) {
-    uint32_t m = 0;
-    for (int i = 0; i < g.bpt; ++i) m |= 1u << box_of(g, tile * g.bpt + i).label;
-    return m;
-}
-
-// Token slot p (0..127) of a tile: its box and the in-box offset.
 struct Slot {
     Box box;
     int i, j;        // in-window coordinates (RoPE positions: y = i, x = j)
@@ -123,22 +234,13 @@ struct Slot {
 
 __host__ __device__ inline Slot slot_of(const Geo& g, long long tile, int p) {
     Slot s;
-    s.box = box_of(g, tile * g.bpt + p / g.BT);
-    const int q = p % g.BT, bi = q / g.bw, bj = q - (q / g.bw) * g.bw;
+    s.box = box_of(g, tile * g.bpt + (p >> g.lBT));
+    const int q = p & (g.BT - 1), bi = q >> g.lbw, bj = q & (g.bw - 1);
     s.i = s.box.i0 + bi;
     s.j = s.box.j0 + bj;
     s.row = s.box.row0 + bi;
     s.col = s.box.col0 + bj;
     return s;
-}
-
-// For a query (or key) box segment `seg` and the boxes of another tile,
-// the bit set of that tile's boxes whose tokens it may attend.
-__host__ __device__ inline uint32_t allow_mask(const Geo& g, long long seg, long long other_tile) {
-    uint32_t m = 0;
-    for (int i = 0; i < g.bpt; ++i)
-        if (seg_of(box_of(g, other_tile * g.bpt + i)) == seg) m |= 1u << i;
-    return m;
 }
 
 }  // namespace fswin

@@ -33,8 +33,23 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t tx
     asm volatile("mbarrier.arrive.expect_tx.release.cta.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(tx)
                  : "memory");
 }
+// try_wait with a suspend-time hint: a thread whose phase is not complete is
+// suspended (it does not spin on the issue slots) until the phase completes or
+// about 1 ms passes.
+#ifndef FSWIN_WAIT_HINT_NS
+#define FSWIN_WAIT_HINT_NS 1000000u
+#endif
 __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
     uint32_t ok;
+#if FSWIN_WAIT_HINT_NS > 0
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity), "r"(FSWIN_WAIT_HINT_NS)
+        : "memory");
+#else
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
         "mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2;\n\t"
@@ -42,6 +57,7 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
         : "=r"(ok)
         : "r"(smem_u32(bar)), "r"(parity)
         : "memory");
+#endif
     return ok != 0;
 }
 
@@ -56,23 +72,28 @@ struct Ctl {
 
 enum : unsigned int { kErrTimeout = 6u };
 
+// Slow path of mbar_wait, kept out of line so that the many wait sites of a
+// warp-specialised kernel stay small in the instruction cache.
+static __device__ __noinline__ bool mbar_wait_slow(uint64_t* bar, uint32_t parity, unsigned int* status,
+                                            volatile int* abort_flag, uint64_t limit_ns, unsigned int where) {
+    const uint64_t t0 = globaltimer_ns();
+    for (;;) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if (*abort_flag) return false;
+        if (globaltimer_ns() - t0 > limit_ns) {
+            atomicCAS(status, 0u, (kErrTimeout << 24) | (where & 0xFFFFFFu));
+            *abort_flag = 1;
+            __threadfence_block();
+            return false;
+        }
+    }
+}
+
 // Returns true when the phase with the given parity has completed; false when
 // the wait ran out of time or another role of this CTA aborted.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const Ctl& ctl, unsigned int where) {
     if (mbar_try_wait(bar, parity)) return true;
-    const uint64_t t0 = globaltimer_ns();
-    for (uint32_t it = 1;; ++it) {
-        if (mbar_try_wait(bar, parity)) return true;
-        if ((it & 255u) == 0) {
-            if (*ctl.abort_flag) return false;
-            if (globaltimer_ns() - t0 > ctl.limit_ns) {
-                atomicCAS(ctl.status, 0u, (kErrTimeout << 24) | (where & 0xFFFFFFu));
-                *ctl.abort_flag = 1;
-                __threadfence_block();
-                return false;
-            }
-        }
-    }
+    return mbar_wait_slow(bar, parity, ctl.status, ctl.abort_flag, ctl.limit_ns, where);
 }
 
 // ---------------------------------------------------------------- fences
@@ -250,6 +271,27 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
     return r;
 }
+// Packed two-lane fp32 arithmetic (one instruction for two values).
+__device__ __forceinline__ void ffma2(float& dx, float& dy, float ax, float ay, float bx, float by, float cx,
+                                      float cy) {
+    asm("{\n\t.reg .b64 a, b, c, d;\n\tmov.b64 a, {%2, %3};\n\tmov.b64 b, {%4, %5};\n\tmov.b64 c, {%6, %7};\n\t"
+        "fma.rn.f32x2 d, a, b, c;\n\tmov.b64 {%0, %1}, d;\n\t}"
+        : "=f"(dx), "=f"(dy)
+        : "f"(ax), "f"(ay), "f"(bx), "f"(by), "f"(cx), "f"(cy));
+}
+__device__ __forceinline__ void fadd2(float& dx, float& dy, float ax, float ay, float bx, float by) {
+    asm("{\n\t.reg .b64 a, b, d;\n\tmov.b64 a, {%2, %3};\n\tmov.b64 b, {%4, %5};\n\t"
+        "add.rn.f32x2 d, a, b;\n\tmov.b64 {%0, %1}, d;\n\t}"
+        : "=f"(dx), "=f"(dy)
+        : "f"(ax), "f"(ay), "f"(bx), "f"(by));
+}
+__device__ __forceinline__ void fmul2(float& dx, float& dy, float ax, float ay, float bx, float by) {
+    asm("{\n\t.reg .b64 a, b, d;\n\tmov.b64 a, {%2, %3};\n\tmov.b64 b, {%4, %5};\n\t"
+        "mul.rn.f32x2 d, a, b;\n\tmov.b64 {%0, %1}, d;\n\t}"
+        : "=f"(dx), "=f"(dy)
+        : "f"(ax), "f"(ay), "f"(bx), "f"(by));
+}
+
 // Packs two floats into f16x2 with `lo` in the low half (round to nearest even).
 __device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
     uint32_t r;
@@ -258,5 +300,41 @@ __device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
 }
 __device__ __forceinline__ float bf16lo_to_f32(uint32_t v) { return __uint_as_float(v << 16); }
 __device__ __forceinline__ float bf16hi_to_f32(uint32_t v) { return __uint_as_float(v & 0xFFFF0000u); }
+
+// ---------------------------------------------------------------- tracing
+// Builds with -DFSWIN_TRACE record (SM clock, warp, event) for CTA 0 into a
+// device buffer, to inspect the pipeline timeline; other builds compile the
+// hook to nothing.
+#ifdef FSWIN_TRACE
+struct TraceBuf {
+    unsigned long long* ev;  // [cap][2]
+    unsigned int* n;
+    unsigned int cap;
+};
+static __device__ TraceBuf g_trace;  // one per translation unit
+// Per-warp event counters in shared memory: one region of cap/32 events per warp.
+__device__ __forceinline__ unsigned int* trace_counters() {
+    __shared__ unsigned int ctr[32];
+    return ctr;
+}
+__device__ __forceinline__ void trace_init() {
+    if (threadIdx.x < 32) trace_counters()[threadIdx.x] = 0;
+}
+__device__ __forceinline__ void trace(unsigned int ev) {
+    const unsigned long long t = clock64();
+    if (blockIdx.x != 0 || g_trace.ev == nullptr) return;
+    const unsigned int w = threadIdx.x >> 5, per = g_trace.cap / 32;
+    const unsigned int i = atomicAdd(&trace_counters()[w], 1u);
+    if (i < per) {
+        g_trace.ev[2 * (w * per + i)] = t;
+        g_trace.ev[2 * (w * per + i) + 1] = (static_cast<unsigned long long>(w) << 32) | ev;
+    }
+}
+#define FS_TRACE(ev) ::fswin::trace(ev)
+#define FS_TRACE_INIT() ::fswin::trace_init()
+#else
+#define FS_TRACE(ev) ((void)0)
+#define FS_TRACE_INIT() ((void)0)
+#endif
 
 }  // namespace fswin
