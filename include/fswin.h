@@ -123,6 +123,29 @@ FS_API fs_status fs_set_wait_limit_ns(uint64_t limit_ns);
 FS_API fs_status fs_selftest_bounded_wait(uint64_t limit_ns, fs_stream_t stream);
 
 /*
+ * Backward that allocates nothing and takes no workspace (the paper has no
+ * counterpart; this is a convenience of this library).  For callers that cannot
+ * allocate device memory when they call the backward, for example code that
+ * runs inside a memory pool that is already fully handed out, or a runtime that
+ * forbids cudaMalloc after start-up.  The scratch is one array inside the
+ * library, fs_winattn_bwd_noalloc_max_bytes() bytes (64 MiB) on every GPU that
+ * loads the library, held until the process exits.  Problems whose
+ * fs_winattn_bwd_workspace_bytes() exceeds that size return FS_ERR_WORKSPACE and
+ * launch nothing.  Arguments and results are those of fs_winattn_bwd.
+ *
+ * The first call on a device looks up the array's device address (once per
+ * device); make that first call before any stream capture.  All calls on a
+ * device share the array: calls whose kernels may overlap on the GPU (other
+ * streams or host threads without ordering between them) race on it.
+ */
+FS_API fs_status fs_winattn_bwd_noalloc(const fs_winattn_shape* shape, const void* q, const void* k, const void* v,
+                                        const void* o, const void* dout, const float* lse, const float* theta,
+                                        void* dq, void* dk, void* dv, float* dtheta, fs_stream_t stream);
+
+/* Size of the scratch array fs_winattn_bwd_noalloc uses, in bytes. */
+FS_API size_t fs_winattn_bwd_noalloc_max_bytes(void);
+
+/*
  * Profiling hook.  events: `n` caller-created cudaEvent_t handles (as void*), or
  * n == 0 to switch the hook off.  While set, fs_winattn_fwd records events[0]
  * before and events[1] after its kernel (n >= 2), and fs_winattn_bwd records

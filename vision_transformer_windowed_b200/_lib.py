@@ -65,6 +65,10 @@ def load(build_if_missing: bool = True):
         lib.fs_selftest_bounded_wait.restype = st
         lib.fs_set_phase_events.argtypes = [ctypes.POINTER(ctypes.c_void_p), ctypes.c_int]
         lib.fs_set_phase_events.restype = st
+        lib.fs_winattn_bwd_noalloc.argtypes = [P] + [vp] * 12
+        lib.fs_winattn_bwd_noalloc.restype = st
+        lib.fs_winattn_bwd_noalloc_max_bytes.argtypes = []
+        lib.fs_winattn_bwd_noalloc_max_bytes.restype = ctypes.c_size_t
         _lib = lib
         return lib
 
@@ -98,6 +102,18 @@ def fs_winattn_bwd(shape: Shape, q: int, k: int, v: int, o: int, dout: int, lse:
                    dv: int, dtheta: int, workspace: int, workspace_bytes: int, stream: int) -> None:
     _check(load().fs_winattn_bwd(ctypes.byref(shape), q, k, v, o, dout, lse, theta, dq, dk, dv, dtheta, workspace,
                                  workspace_bytes, stream), "fs_winattn_bwd")
+
+
+def fs_winattn_bwd_noalloc(shape: Shape, q: int, k: int, v: int, o: int, dout: int, lse: int, theta: int, dq: int,
+                           dk: int, dv: int, dtheta: int, stream: int) -> None:
+    """Backward without a caller workspace: for callers that cannot allocate
+    device memory at that point; uses the library's own fixed scratch array."""
+    _check(load().fs_winattn_bwd_noalloc(ctypes.byref(shape), q, k, v, o, dout, lse, theta, dq, dk, dv, dtheta,
+                                         stream), "fs_winattn_bwd_noalloc")
+
+
+def fs_winattn_bwd_noalloc_max_bytes() -> int:
+    return int(load().fs_winattn_bwd_noalloc_max_bytes())
 
 
 def fs_device_status() -> int:
