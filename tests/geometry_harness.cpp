@@ -9,7 +9,30 @@
 
 using namespace fswin;
 
+// Division by invariant integers against the hardware divide: small and large
+// divisors, numerators near multiples of the divisor and near 2^31.
+static int check_fastdiv() {
+    unsigned long long bad = 0, n_checked = 0;
+    const uint32_t ds[] = {1u, 2u, 3u, 5u, 7u, 9u, 16u, 48u, 64u, 100u, 255u, 256u, 1000u, 4096u, 6553u, 65535u,
+                           65536u, 123457u, 1u << 20, (1u << 20) + 1u, 33554431u, 1u << 30, (1u << 31) - 1u, 1u << 31};
+    for (uint32_t d : ds) {
+        const FastDiv f = make_fastdiv(d);
+        for (uint32_t k = 0; k < 2000; ++k) {
+            const uint32_t cand[] = {k, k * d, k * d - 1u, k * d + 1u, 0x7FFFFFFFu - k, 0x80000000u - k,
+                                     static_cast<uint32_t>((k * 2654435761ull) & 0x7FFFFFFFu)};
+            for (uint32_t n : cand) {
+                if (n > 0x80000000u) continue;
+                ++n_checked;
+                if (fdiv(f, n) != n / d) ++bad;
+            }
+        }
+    }
+    std::printf("D %llu %llu\n", n_checked, bad);
+    return bad ? 1 : 0;
+}
+
 int main(int argc, char** argv) {
+    if (argc == 2 && argv[1][0] == 'D') return check_fastdiv();
     if (argc != 8) return 1;
     int a[7];
     for (int i = 0; i < 7; ++i) a[i] = std::atoi(argv[i + 1]);
@@ -31,12 +54,8 @@ int main(int argc, char** argv) {
     }
     for (long long it = 0; it < fwd_item_count(g); ++it) {
         const FwdItem I = fwd_item(g, it);
-        for (int T = 0; T < 2; ++T) {
-            const long long qt = T ? I.tB : I.tA;
-            if (qt < 0) continue;
-            for (int u = 0; u < I.nkv; ++u)
-                if (fwd_active(g, I, T, u)) std::printf("F %lld %d %lld %lld\n", it, I.h, qt, I.kv0 + u);
-        }
+        for (int u = 0; u < I.nkv; ++u)
+            if ((I.act >> u) & 1u) std::printf("F %lld %d %lld %lld\n", it, I.h, I.X, I.kv0 + u);
     }
     for (long long it = 0; it < bwd_item_count(g); ++it) {
         const BwdItem I = bwd_item(g, it);

@@ -111,3 +111,10 @@ def test_geometry_and_schedule(harness, shape):
             if l[0] == "B" and int(l.split()[2]) == h:
                 kitems[int(l.split()[3])].add(int(l.split()[1]))
         assert all(len(x) == 1 for x in kitems.values()) and len(kitems) == tiles
+
+
+def test_invariant_division_matches_hardware_divide(harness):
+    """The 32-bit division by set-up constants used for window and item indices."""
+    out = subprocess.run([harness, "D"], capture_output=True, text=True)
+    tag, checked, bad = out.stdout.split()
+    assert tag == "D" and int(checked) > 100000 and int(bad) == 0 and out.returncode == 0

@@ -11,12 +11,41 @@
 // window and the shift-region label (the Swin shifted-window rule).
 //
 // Every extent below is a power of two, so the per-row and per-tile helpers
-// use shifts and masks; integer division only happens once per window.
+// use shifts and masks.  The few divisions by other set-up constants (windows
+// per image, tiles per head) use 32-bit division by invariant integers.
 #pragma once
 
 #include <cstdint>
 
 namespace fswin {
+
+// Unsigned 32-bit division by a divisor fixed at set-up: one multiply-high, a
+// subtract, an add and two shifts (T. Granlund and P. L. Montgomery, "Division
+// by invariant integers using multiplication", PLDI 1994, section 4: the
+// multiplier m' = floor(2^32 (2^l - d) / d) + 1 with l = ceil(log2 d)).
+struct FastDiv {
+    uint32_t d, m, s1, s2;
+};
+
+inline FastDiv make_fastdiv(uint32_t d) {  // 1 <= d <= 2^31
+    FastDiv f;
+    f.d = d;
+    int l = 0;
+    while ((1ull << l) < d) ++l;
+    f.m = static_cast<uint32_t>(((1ull << 32) * ((1ull << l) - d)) / d + 1);
+    f.s1 = l > 0 ? 1u : 0u;
+    f.s2 = l > 0 ? static_cast<uint32_t>(l - 1) : 0u;
+    return f;
+}
+
+__host__ __device__ inline uint32_t fdiv(const FastDiv& f, uint32_t n) {
+#ifdef __CUDA_ARCH__
+    const uint32_t t = __umulhi(f.m, n);
+#else
+    const uint32_t t = static_cast<uint32_t>((static_cast<uint64_t>(f.m) * n) >> 32);
+#endif
+    return (t + ((n - t) >> f.s1)) >> f.s2;
+}
 
 constexpr int kTile = 128;                  // token rows per tile
 constexpr int kHeadDim = 32;                // supported head dimension
@@ -36,6 +65,7 @@ struct Geo {
     long long wins;     // windows in the batch
     long long tiles;    // tiles per head
     float scale_log2;   // log2(e) / sqrt(d)
+    FastDiv fd_nW, fd_nWw, fd_tiles;  // window, tile and item indices fit 32 bits
 };
 
 __host__ __device__ inline int ilog2_exact(int x) {
@@ -52,7 +82,9 @@ inline int geo_init(Geo* g, int B, int H, int W, int heads, int d, int M, int s)
     if (B < 0 || heads < 1 || H < M || W < M || H % M || W % M) return 2;
     if (s < 0 || s >= M || s % 4) return 2;
     if (H > (1 << 24) || W > (1 << 24) || heads > 4096) return 2;
-    if (static_cast<long long>(B) * H * W * heads > (1ll << 40)) return 2;
+    // token, window, tile and work-item indices of one head stay below 2^31
+    if (static_cast<long long>(B) * H * W > (1ll << 31)) return 2;
+    if (static_cast<long long>(B) * H * W * heads > (1ll << 37)) return 2;
     int a = M, b = s;  // box side: gcd(M, s), or M without shift
     while (b) {
         const int t = a % b;
@@ -89,6 +121,9 @@ inline int geo_init(Geo* g, int B, int H, int W, int heads, int d, int M, int s)
     x.wins = static_cast<long long>(B) * x.nW;
     x.tiles = (x.wins * x.N + kTile - 1) / kTile;
     x.scale_log2 = 1.4426950408889634f / 5.656854249492380195f;  // log2(e) / sqrt(32)
+    x.fd_nW = make_fastdiv(static_cast<uint32_t>(x.nW));
+    x.fd_nWw = make_fastdiv(static_cast<uint32_t>(x.nWw));
+    x.fd_tiles = make_fastdiv(static_cast<uint32_t>(x.tiles > 0 ? x.tiles : 1));
     *g = x;
     return 0;
 }
@@ -108,10 +143,11 @@ __host__ __device__ inline Win win_of(const Geo& g, long long gw) {
     Win w;
     w.gw = gw;
     w.valid = gw < g.wins;
-    w.b = static_cast<int>(gw / g.nW);  // >= B for padding windows: TMA then zero-fills
-    const int r = static_cast<int>(gw - static_cast<long long>(w.b) * g.nW);
-    w.wr = r / g.nWw;
-    w.wc = r - w.wr * g.nWw;
+    const uint32_t g32 = static_cast<uint32_t>(gw);
+    w.b = static_cast<int>(fdiv(g.fd_nW, g32));  // >= B for padding windows: TMA then zero-fills
+    const uint32_t r = g32 - static_cast<uint32_t>(w.b) * g.nW;
+    w.wr = static_cast<int>(fdiv(g.fd_nWw, r));
+    w.wc = static_cast<int>(r) - w.wr * g.nWw;
     return w;
 }
 
