@@ -13,6 +13,7 @@ instead, on a bounded sample of the same workload.
 from __future__ import annotations
 
 import argparse
+import hashlib
 import json
 import os
 import statistics
@@ -51,6 +52,32 @@ def unmasked_pairs(B, H, W, heads, M, s) -> int:
         for cc in cols:
             per_image += sum((a * b) ** 2 for a in rr for b in cc)
     return per_image * B * heads
+
+
+def kernel_sources_sha256() -> str:
+    """Hash of the CUDA sources; stored DRAM traffic is valid only for the build it was captured on."""
+    root = os.path.join(os.path.dirname(os.path.abspath(__file__)), "vision_transformer_windowed_b200", "csrc")
+    h = hashlib.sha256()
+    for f in sorted(os.listdir(root)):
+        if f.endswith((".cu", ".cuh")):
+            h.update(f.encode())
+            with open(os.path.join(root, f), "rb") as fh:
+                h.update(fh.read())
+    return h.hexdigest()
+
+
+def measured_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch of `kernel` from the committed ncu capture, or None when
+    there is none for this workload or the kernel sources changed since."""
+    path = os.path.join(os.path.dirname(os.path.abspath(__file__)), "profiles", "traffic.json")
+    try:
+        with open(path) as fh:
+            rec = json.load(fh).get(kernel)
+    except (OSError, ValueError):
+        return None
+    if not rec or rec.get("workload") != workload or rec.get("sources_sha256") != kernel_sources_sha256():
+        return None
+    return rec["bytes_per_launch"]
 
 
 def workload_flops(wl) -> tuple[float, float]:
@@ -328,6 +355,7 @@ def main():
                 "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops"], "traffic": None,
                 "algorithmic_flops_per_launch": fl, "peak_note": f"cuBLAS bf16 burst, {peaks['source']}"}
     roof["avg_launch_ms"] = ph[dom]
+    roof["traffic"] = measured_traffic(dom, args.workload)
 
     # end to end through the public API with host buffers (pinned), copies inside the timed region
     t = main_res["tensors"]

@@ -2,9 +2,9 @@
 //
 // Recompute-based (the probabilities are rebuilt from the forward's
 // log-sum-exp, never stored), in four launches on the caller's stream:
-//   1. prep:   per token row, rotate q and k (RoPE) into swizzled bf16 tile
-//              images, copy dO into a tile image, D = rowsum(dO * O), lse in
-//              log2 units, and zero the fp32 dQ accumulator;
+//   1. prep:   per token row, rotate q and k (RoPE) into swizzled fp16 tile
+//              images, copy dO into a bf16 tile image, D = rowsum(dO * O),
+//              lse in log2 units, and zero the fp32 dQ accumulator;
 //   2. main:   persistent, warp-specialised tcgen05 kernel; a work item is one
 //              128-key tile, iterating over the query tiles it attends to:
 //                S^T = K' Q'^T, dP^T = V dO^T            (TMEM)
