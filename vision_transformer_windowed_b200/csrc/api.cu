@@ -188,15 +188,18 @@ fs_status fs_winattn_bwd(const fs_winattn_shape* shape, const void* q, const voi
     if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) || workspace_bytes < bwd_workspace_bytes(g))
         return FS_ERR_WORKSPACE;
     if ((st = device_state(&status, &sms)) != FS_OK) return st;
-    CUtensorMap mv, mdv;
-    if (encode_box_map(&mv, v, g) || encode_box_map(&mdv, dv, g)) return FS_ERR_CUDA;
+    BwdMaps maps;
+    if (encode_box_map(&maps.q, q, g) || encode_box_map(&maps.k, k, g) || encode_box_map(&maps.v, v, g) ||
+        encode_box_map(&maps.o, o, g) || encode_box_map(&maps.dout, dout, g) || encode_box_map(&maps.dq, dq, g) ||
+        encode_box_map(&maps.dk, dk, g) || encode_box_map(&maps.dv, dv, g))
+        return FS_ERR_CUDA;
     unsigned long long lim;
     {
         std::lock_guard<std::mutex> lk(g_mu);
         lim = g_limit_ns;
     }
     BwdPtrs p{q, k, v, o, dout, lse, theta, dq, dk, dv, dtheta, static_cast<uint8_t*>(workspace)};
-    cudaError_t e = launch_bwd(g, p, mv, mdv, status, lim, sms, reinterpret_cast<cudaStream_t>(stream),
+    cudaError_t e = launch_bwd(g, p, maps, status, lim, sms, reinterpret_cast<cudaStream_t>(stream),
                                g_phase_n >= 5 ? g_phase_events : nullptr);
     return e == cudaSuccess ? FS_OK : FS_ERR_CUDA;
 }

@@ -65,7 +65,7 @@ struct Geo {
     long long wins;     // windows in the batch
     long long tiles;    // tiles per head
     float scale_log2;   // log2(e) / sqrt(d)
-    FastDiv fd_nW, fd_nWw, fd_tiles;  // window, tile and item indices fit 32 bits
+    FastDiv fd_nW, fd_nWw, fd_tiles, fd_heads;  // window, tile and item indices fit 32 bits
 };
 
 __host__ __device__ inline int ilog2_exact(int x) {
@@ -124,6 +124,7 @@ inline int geo_init(Geo* g, int B, int H, int W, int heads, int d, int M, int s)
     x.fd_nW = make_fastdiv(static_cast<uint32_t>(x.nW));
     x.fd_nWw = make_fastdiv(static_cast<uint32_t>(x.nWw));
     x.fd_tiles = make_fastdiv(static_cast<uint32_t>(x.tiles > 0 ? x.tiles : 1));
+    x.fd_heads = make_fastdiv(static_cast<uint32_t>(heads));
     *g = x;
     return 0;
 }

@@ -24,12 +24,17 @@ struct BwdPtrs {
     uint8_t* ws;
 };
 
+// TMA maps (window boxes) of the backward's token tensors.
+struct BwdMaps {
+    CUtensorMap q, k, v, o, dout, dq, dk, dv;
+};
+
 long long bwd_items(const Geo& g);
 size_t bwd_workspace_bytes(const Geo& g);
 // events: NULL, or 5 events recorded before the first and after each of the
-// four launches.
-cudaError_t launch_bwd(const Geo& g, const BwdPtrs& p, const CUtensorMap& mv, const CUtensorMap& mdv,
-                       unsigned int* status, unsigned long long limit_ns, int num_sms, cudaStream_t stream,
-                       cudaEvent_t const* events);
+// four launches (prep, main, post, d theta; windows of fewer than 128 tokens
+// run one kernel in the place of the first three).
+cudaError_t launch_bwd(const Geo& g, const BwdPtrs& p, const BwdMaps& maps, unsigned int* status,
+                       unsigned long long limit_ns, int num_sms, cudaStream_t stream, cudaEvent_t const* events);
 
 }  // namespace fswin
