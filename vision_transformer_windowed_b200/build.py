@@ -10,8 +10,8 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 BUILD = os.path.join(HERE, "_build")
 LIB = os.path.join(BUILD, "libfswin.so")
-SOURCES = ["api.cu", "fwd.cu", "bwd.cu", "noalloc.cu"]
-HEADERS = ["dgeo.cuh", "geometry.cuh", "kernels.cuh", "ptx.cuh", "schedule.cuh", "tile_io.cuh"]
+SOURCES = ["api.cu", "fwd.cu", "bwd.cu", "small.cu", "noalloc.cu"]
+HEADERS = ["dgeo.cuh", "geometry.cuh", "kernels.cuh", "ptx.cuh", "rows.cuh", "schedule.cuh", "tile_io.cuh"]
 
 
 def nvcc_path() -> str:

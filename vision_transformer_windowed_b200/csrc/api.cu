@@ -152,7 +152,8 @@ fs_status fs_winattn_fwd(const fs_winattn_shape* shape, const void* q, const voi
         std::lock_guard<std::mutex> lk(g_mu);
         lim = g_limit_ns;
     }
-    cudaError_t e = launch_fwd(g, mq, mk, mv, mo, theta, lse, status, lim, sms, reinterpret_cast<cudaStream_t>(stream),
+    cudaError_t e = launch_fwd(g, mq, mk, mv, mo, q, k, v, o, theta, lse, status, lim, sms,
+                               reinterpret_cast<cudaStream_t>(stream),
                                g_phase_n >= 2 ? g_phase_events : nullptr);
     return e == cudaSuccess ? FS_OK : FS_ERR_CUDA;
 }

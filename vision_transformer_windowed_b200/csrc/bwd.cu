@@ -15,7 +15,6 @@
 //              dk, and the per-tile partial sums of d theta;
 //   4. reduce: fixed-order sum of the partials into dtheta (deterministic).
 #include <cuda.h>
-#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
 #include "geometry.cuh"
@@ -24,6 +23,7 @@
 #include "schedule.cuh"
 #include "tile_io.cuh"
 #include "dgeo.cuh"
+#include "rows.cuh"
 
 namespace fswin {
 
@@ -108,24 +108,6 @@ __device__ __forceinline__ void load_row_bf16(const uint4* src, float (&x)[32]) 
             x[8 * c + 2 * e + 1] = bf16hi_to_f32(w[e]);
         }
     }
-}
-
-__device__ __forceinline__ uint32_t pack2(float lo, float hi, bool fp16) {
-    return fp16 ? pack_f16x2(lo, hi) : pack_bf16x2(lo, hi);
-}
-
-__device__ __forceinline__ uint4 pack_chunk(const float (&x)[32], int c, bool fp16 = false) {
-    return make_uint4(pack2(x[8 * c], x[8 * c + 1], fp16), pack2(x[8 * c + 2], x[8 * c + 3], fp16),
-                      pack2(x[8 * c + 4], x[8 * c + 5], fp16), pack2(x[8 * c + 6], x[8 * c + 7], fp16));
-}
-
-// Row r of a 64-byte-swizzled 16-bit tile image (bf16, or fp16 for the
-// rotated Q' and K', see the forward kernel).
-__device__ __forceinline__ void store_row_swz(uint8_t* tile, int r, const float (&x)[32], bool fp16 = false) {
-    uint8_t* row = tile + r * kRowBytes;
-    const int sw = (r >> 1) & 3;
-#pragma unroll
-    for (int c = 0; c < 4; ++c) *reinterpret_cast<uint4*>(row + ((c ^ sw) << 4)) = pack_chunk(x, c, fp16);
 }
 
 // ------------------------------------------------------------------ 1. prep
@@ -674,491 +656,6 @@ __global__ void __launch_bounds__(256) dtheta_kernel(const float* part, long lon
 }
 
 
-// ------------------------------------------------------------------ 5. small windows
-// Windows of fewer than 128 tokens (M = 4, 8) lie whole inside one 128-slot
-// tile, so every gradient of a tile's tokens comes from that tile alone.  One
-// persistent kernel then does the whole backward of a tile on chip, with no
-// workspace round trip: only the 16 d theta partials of the tile leave it.
-//   warps 0-3: thread = slot row.  Loads its own q, k, v, dO, o rows with
-//              16-byte async copies one work item ahead (a window box of a
-//              shifted grid is as small as 4 x 4 tokens, too small for TMA box
-//              copies to keep up); D, lse and the RoPE of its q and k rows; the
-//              row of P^T and dS^T of its key; the epilogue of its token, whose
-//              dq, dk, dv rows it stores directly.
-//   warp 4:    MMA issuer: S^T = K' Q'^T, dP^T = V dO^T; then dV = P^T dO,
-//              dK' = dS^T Q', dQ' = dS K'.
-// Two CTAs share an SM (256 TMEM columns each).  Work items are (tile, head),
-// heads innermost when their RoPE tables fit, so the heads of a token, which
-// are adjacent in memory, are read close together in time.
-namespace small {
-
-constexpr int kThreads = 160;
-constexpr int kWarpMma = 4;
-constexpr int kSlotBytes = 4 * kTileBytes;        // q, k, v, dO tiles of one item
-constexpr int kSlotOff = 0;                        // 2 slots
-constexpr int kOOff = 2 * kSlotBytes;              // o tile
-constexpr int kDSOff = kOOff + kTileBytes;         // dS (queries along M), MN-major 128-byte swizzle
-constexpr int kVecOff = kDSOff + 4 * kTileBytes;   // lse2[128], D[128]
-constexpr int kTabHeads = 4;                       // resident cos/sin tables
-constexpr int kTabPerHead = 2 * 8 * 8;             // [axis][pair][position < 8] float2
-constexpr int kTabOff = kVecOff + 2 * kTile * 4;
-constexpr int kBarOff = kTabOff + kTabHeads * kTabPerHead * 8;
-constexpr int kSmemBytes = kBarOff + 256 + 1024;   // + alignment of the base
-constexpr uint32_t kTmemCols = 256;
-// TMEM columns: S^T [0,128), dP^T [128,256); P^T (bf16) over S^T [0,64), dS^T
-// (fp16) over dP^T [128,192); the products over columns already consumed.
-constexpr uint32_t kColS = 0, kColDP = 128, kColP = 0, kColDS = 128;
-constexpr uint32_t kColDV = 64, kColDQ = 96, kColDK = 192;
-
-struct Bars {
-    uint64_t in_ready, s_full, p_ready, mma2_done, tmem_free, grp, done;
-    uint32_t tmem_base;
-    int abort_flag;
-};
-static_assert(sizeof(Bars) <= 256, "barrier block overflows its slot");
-
-struct Params {
-    Geo g;
-    const uint8_t *q, *k, *v, *o, *dout;  // bf16 [B, H, W, heads, 32]
-    uint8_t *dq, *dk, *dv;
-    const float *lse, *theta;
-    float* part;  // [heads][tiles][16]
-    unsigned int* status;
-    unsigned long long limit_ns;
-    long long items;
-    float scale;
-    bool head_minor;
-};
-
-// Item -> (tile, head): heads innermost when all tables are resident.
-__device__ __forceinline__ void small_item(const Params& p, long long it, long long* X, int* h) {
-    const uint32_t i32 = static_cast<uint32_t>(it);
-    if (p.head_minor) {
-        const uint32_t x = fdiv(p.g.fd_heads, i32);
-        *X = x;
-        *h = static_cast<int>(i32 - x * static_cast<uint32_t>(p.g.heads));
-    } else {
-        const uint32_t hh = fdiv(p.g.fd_tiles, i32);
-        *h = static_cast<int>(hh);
-        *X = it - static_cast<long long>(hh) * p.g.tiles;
-    }
-}
-
-// Row r of a 64-byte-swizzled 16-bit tile (bf16, or fp16) as 32 floats.
-__device__ __forceinline__ void load_row_swz(const uint8_t* tile, int r, float (&x)[32], bool fp16) {
-    const uint8_t* row = tile + r * kRowBytes;
-    const int sw = (r >> 1) & 3;
-#pragma unroll
-    for (int c = 0; c < 4; ++c) {
-        const uint4 v = *reinterpret_cast<const uint4*>(row + ((c ^ sw) << 4));
-        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            if (fp16) {
-                const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&w[e]));
-                x[8 * c + 2 * e] = f.x;
-                x[8 * c + 2 * e + 1] = f.y;
-            } else {
-                x[8 * c + 2 * e] = bf16lo_to_f32(w[e]);
-                x[8 * c + 2 * e + 1] = bf16hi_to_f32(w[e]);
-            }
-        }
-    }
-}
-
-// Rotation by the compact table of one head ([axis][pair][position], M <= 8).
-__device__ __forceinline__ void rope32_small(float (&x)[32], int i, int j, const float2* tab, bool inv) {
-#pragma unroll
-    for (int ax = 0; ax < 2; ++ax) {
-        const int pos = ax ? i : j;
-#pragma unroll
-        for (int k = 0; k < 8; ++k) {
-            const float2 cs = tab[(ax * 8 + k) * 8 + pos];
-            const float sn = inv ? -cs.y : cs.y;
-            const float a = x[ax * 16 + 2 * k], b = x[ax * 16 + 2 * k + 1];
-            x[ax * 16 + 2 * k] = a * cs.x - b * sn;
-            x[ax * 16 + 2 * k + 1] = a * sn + b * cs.x;
-        }
-    }
-}
-
-__device__ void build_small_table(float2* tab, const float* theta_h, int M, int tid, int nthreads) {
-    for (int e = tid; e < 16 * M; e += nthreads) {
-        const int ap = e / M, pos = e - ap * M;  // ap = axis * 8 + pair
-        float sn, cs;
-        sincosf(static_cast<float>(pos) * theta_h[ap], &sn, &cs);
-        tab[ap * 8 + pos] = make_float2(cs, sn);
-    }
-}
-
-// Token of slot r of tile X (false for padding windows): in-window position
-// and flat index of the [B, H, W, heads] grid at head h.
-__device__ __forceinline__ bool slot_token(const Geo& g, long long X, int r, int h, int* pi, int* pj,
-                                           long long* tok) {
-    Win w = tile_win(g, X);
-    const int widx = r >> (g.lnbw + g.lBT);  // window of the slot inside the tile
-    if (widx) w = win_of(g, w.gw + widx);
-    tile_row_pos(g, X, r, pi, pj);
-    int row = w.wr * g.M + *pi + g.s, col = w.wc * g.M + *pj + g.s;
-    if (row >= g.H) row -= g.H;
-    if (col >= g.W) col -= g.W;
-    *tok = ((static_cast<long long>(w.b) * g.H + row) * g.W + col) * g.heads + h;
-    return w.valid;
-}
-
-__global__ void __launch_bounds__(kThreads, 2) small_kernel(const __grid_constant__ Params prm) {
-    extern __shared__ uint8_t smem_raw[];
-    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    Bars* bars = reinterpret_cast<Bars*>(smem + kBarOff);
-    const Geo& g = prm.g;
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-
-    if (tid == 0) {
-        mbar_init(&bars->in_ready, 1);
-        mbar_init(&bars->s_full, 1);
-        mbar_init(&bars->p_ready, 4);
-        mbar_init(&bars->mma2_done, 1);
-        mbar_init(&bars->tmem_free, 4);
-        mbar_init(&bars->grp, 4);
-        mbar_init(&bars->done, 1);
-        bars->abort_flag = 0;
-        fence_mbar_init();
-    }
-    if (warp == 0) {
-        tmem_alloc(&bars->tmem_base, kTmemCols);
-        tmem_relinquish();
-    }
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-    const uint32_t tmem = bars->tmem_base;
-    const Ctl ctl{prm.status, &bars->abort_flag, prm.limit_ns};
-    // this CTA's items: blockIdx.x + j * gridDim.x, j < n
-    const long long n = prm.items > blockIdx.x ? (prm.items - 1 - blockIdx.x) / gridDim.x + 1 : 0;
-    auto item_at = [&](long long j) { return static_cast<long long>(blockIdx.x) + j * gridDim.x; };
-
-    if (warp == kWarpMma) {
-        // ------------------------------------------------------------ MMA issue
-        if (lane == 0) {
-            const uint32_t id_s = make_idesc(kTile, kTile, false, false, true);     // fp16 K', Q'
-            const uint32_t id_dp = make_idesc(kTile, kTile, false, false, false);   // bf16 V, dO
-            const uint32_t id_dv = make_idesc(kTile, kHeadDim, false, true, false); // P^T (TMEM) x dO
-            const uint32_t id_dk = make_idesc(kTile, kHeadDim, false, true, true);  // dS^T (TMEM) x Q'
-            const uint32_t id_dq = make_idesc(kTile, kHeadDim, true, true, true);   // dS (smem) x K'
-            const uint32_t ds_addr = smem_u32(smem + kDSOff);
-            for (long long j = 0; j < n; ++j) {
-                const uint32_t ph = static_cast<uint32_t>(j & 1);
-                if (!mbar_wait(&bars->in_ready, ph, ctl, 0x2201)) break;
-                if (j > 0 && !mbar_wait(&bars->tmem_free, ph ^ 1, ctl, 0x2202)) break;
-                tc_fence_after();
-                const uint32_t qa = smem_u32(smem + kSlotOff + (j & 1) * kSlotBytes);
-                const uint32_t ka = qa + kTileBytes, va = qa + 2 * kTileBytes, da = qa + 3 * kTileBytes;
-#pragma unroll
-                for (int k = 0; k < kHeadDim / 16; ++k)
-                    umma_ss(tmem + kColS, make_sdesc(ka + 32 * k, 16, 512, kSw64),
-                            make_sdesc(qa + 32 * k, 16, 512, kSw64), id_s, k > 0);
-#pragma unroll
-                for (int k = 0; k < kHeadDim / 16; ++k)
-                    umma_ss(tmem + kColDP, make_sdesc(va + 32 * k, 16, 512, kSw64),
-                            make_sdesc(da + 32 * k, 16, 512, kSw64), id_dp, k > 0);
-                umma_commit(&bars->s_full);
-                if (!mbar_wait(&bars->p_ready, ph, ctl, 0x2203)) break;
-                tc_fence_after();
-#pragma unroll
-                for (int k = 0; k < kTile / 16; ++k)
-                    umma_ts(tmem + kColDV, tmem + kColP + 8 * k, make_sdesc(da + 1024 * k, 8192, 512, kSw64), id_dv,
-                            k > 0);
-#pragma unroll
-                for (int k = 0; k < kTile / 16; ++k)
-                    umma_ts(tmem + kColDK, tmem + kColDS + 8 * k, make_sdesc(qa + 1024 * k, 8192, 512, kSw64), id_dk,
-                            k > 0);
-#pragma unroll
-                for (int k = 0; k < kTile / 16; ++k)
-                    umma_ss(tmem + kColDQ, make_sdesc(ds_addr + 2048 * k, 16384, 1024, kSw128),
-                            make_sdesc(ka + 1024 * k, 8192, 512, kSw64), id_dq, k > 0);
-                umma_commit(&bars->mma2_done);
-            }
-            umma_commit(&bars->done);
-            mbar_wait(&bars->done, 0, ctl, 0x22ff);
-        }
-        __syncwarp();
-    } else {
-        // ------------------------------------------------------------ rows (warps 0-3)
-        const int r = tid;
-        const uint32_t trow = tmem + (static_cast<uint32_t>(warp * 32) << 16);
-        const float sl2 = g.scale_log2;
-        float* lse2v = reinterpret_cast<float*>(smem + kVecOff);
-        float* dvec = lse2v + kTile;
-        float2* tabs = reinterpret_cast<float2*>(smem + kTabOff);
-        uint8_t* ds = smem + kDSOff;
-        uint32_t gph = 0;
-        bool ok = true;
-        // Waits are warp-uniform, so that no warp-collective TMEM access runs on
-        // a partial warp; the group barrier is an mbarrier with a bounded wait.
-        auto wwait = [&](uint64_t* bar, uint32_t ph, unsigned int where) -> bool {
-            return __all_sync(0xFFFFFFFFu, mbar_wait(bar, ph, ctl, where));
-        };
-        auto group_sync = [&](unsigned int where) -> bool {
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&bars->grp);
-            const bool passed = wwait(&bars->grp, gph, where);
-            gph ^= 1;
-            return passed;
-        };
-        // This row's token in item j (invalid for padding windows), and the
-        // item's 16-column masks for this row.
-        struct RowTok {
-            long long X, tok;
-            int h, pi, pj;
-            bool valid;
-        };
-        auto row_tok = [&](long long j) {
-            RowTok t;
-            small_item(prm, item_at(j), &t.X, &t.h);
-            t.valid = slot_token(g, t.X, r, t.h, &t.pi, &t.pj, &t.tok);
-            return t;
-        };
-        auto row_mask = [&](const RowTok& t) {
-            const uint64_t segs = d_tile_segs(g, t.X, d_tile_win(g, t.X));
-            return allow16(g, seg_at(segs, r >> g.lBT), segs);  // bit c: columns [16c, 16c+16)
-        };
-        // Copies of the warp's 32 token rows, coalesced: each instruction moves
-        // 8 whole 64-byte rows (lane = row 8i + lane/4, 16-byte chunk lane%4).
-        // Padding rows are zero filled.
-        auto copy_rows = [&](const RowTok& t, const uint8_t* const* src, uint8_t* const* tile, int ntensors) {
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const int sl_lane = 8 * i + (lane >> 2), c = lane & 3;
-                const long long tok = __shfl_sync(0xFFFFFFFFu, t.tok, sl_lane);
-                const bool valid = __shfl_sync(0xFFFFFFFFu, t.valid ? 1 : 0, sl_lane) != 0;
-                const int row = warp * 32 + sl_lane;
-                const uint32_t off = row * kRowBytes + ((c ^ ((row >> 1) & 3)) << 4);
-                for (int x = 0; x < ntensors; ++x)
-                    cp_async16(smem_u32(tile[x] + off), valid ? src[x] + tok * kRowBytes + 16 * c : src[x],
-                               valid ? 16u : 0u);
-            }
-        };
-        auto copy_slot = [&](long long j, const RowTok& t) {
-            uint8_t* sl = smem + kSlotOff + (j & 1) * kSlotBytes;
-            const uint8_t* src[4] = {prm.q, prm.k, prm.v, prm.dout};
-            uint8_t* dst[4] = {sl, sl + kTileBytes, sl + 2 * kTileBytes, sl + 3 * kTileBytes};
-            copy_rows(t, src, dst, 4);
-        };
-        auto copy_o = [&](const RowTok& t) {
-            const uint8_t* src[1] = {prm.o};
-            uint8_t* dst[1] = {smem + kOOff};
-            copy_rows(t, src, dst, 1);
-        };
-        // Commit groups: at the start of item j the newest group holds item
-        // j+1's q, k, v, dO and everything older (item j's slot, o) is waited for.
-        RowTok cur = n > 0 ? row_tok(0) : RowTok{};
-        if (n > 0) {
-            copy_slot(0, cur);
-            copy_o(cur);
-        }
-        cp_async_commit();
-        if (n > 1) copy_slot(1, row_tok(1));
-        cp_async_commit();
-        int tab_head = -1;
-        if (prm.head_minor) {  // every head's table, once
-            for (int hh = 0; hh < g.heads; ++hh)
-                build_small_table(tabs + hh * kTabPerHead, prm.theta + hh * 16, g.M, r, kTile);
-            ok = group_sync(0x2301);
-        }
-        float lse_cur = (n > 0 && cur.valid) ? __ldg(prm.lse + cur.tok) : 0.f;
-        uint32_t a16 = n > 0 ? row_mask(cur) : 0u;
-        for (long long j = 0; j < n && ok; ++j) {
-            const uint32_t ph = static_cast<uint32_t>(j & 1);
-            const float2* tab = tabs;
-            if (prm.head_minor) {
-                tab = tabs + cur.h * kTabPerHead;
-            } else if (cur.h != tab_head) {
-                if (!group_sync(0x2302)) break;  // no row still rotates with the old table
-                build_small_table(tabs, prm.theta + cur.h * 16, g.M, r, kTile);
-                if (!group_sync(0x2303)) break;
-                tab_head = cur.h;
-            }
-            uint8_t* sl = smem + kSlotOff + (j & 1) * kSlotBytes;
-            cp_async_wait<1>();
-            __syncwarp();  // rows copied by other lanes of the warp
-            // D = dO . O of this row's token; then the next item's o rows
-            float D = 0.f;
-            {
-                float a[32], b[32];
-                load_row_swz(smem + kOOff, r, a, false);
-                load_row_swz(sl + 3 * kTileBytes, r, b, false);
-#pragma unroll
-                for (int e = 0; e < 32; ++e) D = fmaf(a[e], b[e], D);
-            }
-            __syncwarp();  // every lane has read its o row
-            RowTok nxt{};
-            if (j + 1 < n) {
-                nxt = row_tok(j + 1);
-                copy_o(nxt);
-            }
-            cp_async_commit();
-            lse2v[r] = cur.valid ? lse_cur * 1.4426950408889634f : INFINITY;  // padding: no probability
-            dvec[r] = D;
-            // RoPE of this row's q and k, bf16 in, fp16 out, in place
-            {
-                float x[32];
-                load_row_swz(sl, r, x, false);
-                rope32_small(x, cur.pi, cur.pj, tab, false);
-                store_row_swz(sl, r, x, true);
-                load_row_swz(sl + kTileBytes, r, x, false);
-                rope32_small(x, cur.pi, cur.pj, tab, false);
-                store_row_swz(sl + kTileBytes, r, x, true);
-            }
-            fence_proxy_async_smem();
-            if (!group_sync(0x2306)) break;
-            if (r == 0) mbar_arrive(&bars->in_ready);
-            const float lse_nxt = (j + 1 < n && nxt.valid) ? __ldg(prm.lse + nxt.tok) : 0.f;
-            // row of P^T and dS^T of this key, 32 query columns at a time
-            if (!wwait(&bars->s_full, ph, 0x2307)) break;
-            tc_fence_after();
-#pragma unroll 1
-            for (int c = 0; c < 4; ++c) {
-                uint32_t sv[32], pv[32];
-                tmem_ld32(trow + kColS + 32 * c, sv);
-                tmem_ld32(trow + kColDP + 32 * c, pv);
-                tmem_wait_ld();
-                const bool ok0 = (a16 >> (2 * c)) & 1u, ok1 = (a16 >> (2 * c + 1)) & 1u;
-                uint32_t wp[16], wd[16];
-#pragma unroll
-                for (int e4 = 0; e4 < 8; ++e4) {
-                    float4 L4 = *reinterpret_cast<const float4*>(lse2v + 32 * c + 4 * e4);
-                    const float4 D4 = *reinterpret_cast<const float4*>(dvec + 32 * c + 4 * e4);
-                    if (!(e4 < 4 ? ok0 : ok1)) L4 = make_float4(INFINITY, INFINITY, INFINITY, INFINITY);
-                    const int e = 4 * e4;
-                    float t0, t1, t2, t3;
-                    ffma2(t0, t1, __uint_as_float(sv[e]), __uint_as_float(sv[e + 1]), sl2, sl2, -L4.x, -L4.y);
-                    ffma2(t2, t3, __uint_as_float(sv[e + 2]), __uint_as_float(sv[e + 3]), sl2, sl2, -L4.z, -L4.w);
-                    const float p0 = ex2_approx(t0), p1 = ex2_approx(t1), p2 = ex2_approx(t2), p3 = ex2_approx(t3);
-                    float d0, d1, d2, d3;
-                    fadd2(d0, d1, __uint_as_float(pv[e]), __uint_as_float(pv[e + 1]), -D4.x, -D4.y);
-                    fadd2(d2, d3, __uint_as_float(pv[e + 2]), __uint_as_float(pv[e + 3]), -D4.z, -D4.w);
-                    fmul2(d0, d1, d0, d1, p0, p1);
-                    fmul2(d2, d3, d2, d3, p2, p3);
-                    wp[2 * e4] = pack_bf16x2(p0, p1);
-                    wp[2 * e4 + 1] = pack_bf16x2(p2, p3);
-                    wd[2 * e4] = pack_f16x2(d0, d1);
-                    wd[2 * e4 + 1] = pack_f16x2(d2, d3);
-                }
-                // over columns of S^T and dP^T already read
-                tmem_st16(trow + kColP + 16 * c, wp);
-                tmem_st16(trow + kColDS + 16 * c, wd);
-                // dS (queries along M, keys along K) as an MN-major operand
-                uint8_t* base = ds + (c >> 1) * 16384 + (r >> 3) * 1024 + (r & 7) * 128;
-#pragma unroll
-                for (int q4 = 0; q4 < 4; ++q4) {
-                    const int cc = 4 * (c & 1) + q4;
-                    *reinterpret_cast<uint4*>(base + ((cc ^ (r & 7)) << 4)) =
-                        make_uint4(wd[4 * q4], wd[4 * q4 + 1], wd[4 * q4 + 2], wd[4 * q4 + 3]);
-                }
-            }
-            tmem_wait_st();
-            fence_proxy_async_smem();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&bars->p_ready);
-            // the next item's masks while the MMAs run
-            const uint32_t a16_nxt = j + 1 < n ? row_mask(nxt) : 0u;
-            // epilogue of this row's token: dq, dk (un-rotated), dv, d theta terms
-            if (!wwait(&bars->mma2_done, ph, 0x2308)) break;
-            tc_fence_after();
-            float part[16];
-#pragma unroll
-            for (int e = 0; e < 16; ++e) part[e] = 0.f;
-#pragma unroll 1
-            for (int which = 0; which < 2; ++which) {  // 0: q side, 1: k side
-                uint32_t t[32];
-                tmem_ld32(trow + (which ? kColDK : kColDQ), t);
-                tmem_wait_ld();
-                float dx[32], x[32];
-#pragma unroll
-                for (int e = 0; e < 32; ++e) dx[e] = __uint_as_float(t[e]) * prm.scale;
-                uint8_t* tile = sl + which * kTileBytes;
-                load_row_swz(tile, r, x, true);  // rotated q' or k' (fp16)
-                // d theta: the pair's cross product is the same before and after the rotation
-#pragma unroll
-                for (int ax = 0; ax < 2; ++ax) {
-                    const float pos = static_cast<float>(ax ? cur.pi : cur.pj);
-#pragma unroll
-                    for (int k = 0; k < 8; ++k) {
-                        const int a = ax * 16 + 2 * k, b = a + 1;
-                        part[ax * 8 + k] = fmaf(pos, dx[b] * x[a] - dx[a] * x[b], part[ax * 8 + k]);
-                    }
-                }
-                rope32_small(dx, cur.pi, cur.pj, tab, true);
-                store_row_swz(tile, r, dx);  // dq or dk (bf16), staged over q' or k'
-            }
-            {
-                uint32_t t[32];
-                tmem_ld32(trow + kColDV, t);
-                tmem_wait_ld();
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&bars->tmem_free);
-                float x[32];
-#pragma unroll
-                for (int e = 0; e < 32; ++e) x[e] = __uint_as_float(t[e]);
-                store_row_swz(sl + 2 * kTileBytes, r, x);  // dv, staged over v
-            }
-            __syncwarp();
-            // coalesced stores of the warp's 32 rows of dq, dk, dv (8 rows per instruction)
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const int sl_lane = 8 * i + (lane >> 2), c = lane & 3;
-                const long long tok = __shfl_sync(0xFFFFFFFFu, cur.tok, sl_lane);
-                const bool valid = __shfl_sync(0xFFFFFFFFu, cur.valid ? 1 : 0, sl_lane) != 0;
-                const int row = warp * 32 + sl_lane;
-                const uint32_t off = row * kRowBytes + ((c ^ ((row >> 1) & 3)) << 4);
-                if (valid) {
-                    const long long go = tok * kRowBytes + 16 * c;
-                    *reinterpret_cast<uint4*>(prm.dq + go) = *reinterpret_cast<const uint4*>(sl + off);
-                    *reinterpret_cast<uint4*>(prm.dk + go) = *reinterpret_cast<const uint4*>(sl + kTileBytes + off);
-                    *reinterpret_cast<uint4*>(prm.dv + go) = *reinterpret_cast<const uint4*>(sl + 2 * kTileBytes + off);
-                }
-            }
-            __syncwarp();  // the staged rows are read: the slot takes item j+2's rows
-            if (j + 2 < n) copy_slot(j + 2, row_tok(j + 2));
-            cp_async_commit();
-            // this warp's 16 d theta partials of the tile (summed in a fixed order
-            // later): a butterfly that halves the values at each step, so that
-            // lane pair (2c, 2c+1) ends with the warp sum of component c
-            if (!cur.valid) {
-#pragma unroll
-                for (int e = 0; e < 16; ++e) part[e] = 0.f;
-            }
-#pragma unroll
-            for (int half = 8, bit = 16; half >= 1; half >>= 1, bit >>= 1) {
-                const bool upper = (lane & bit) != 0;
-#pragma unroll
-                for (int e = 0; e < half; ++e) {
-                    const float send = upper ? part[e] : part[e + half];
-                    const float keep = upper ? part[e + half] : part[e];
-                    part[e] = keep + __shfl_xor_sync(0xFFFFFFFFu, send, bit);
-                }
-            }
-            part[0] += __shfl_xor_sync(0xFFFFFFFFu, part[0], 1);
-            // component held by this lane: bits 4..1 of the lane, most significant first
-            const int comp = ((lane >> 4) & 1) * 8 + ((lane >> 3) & 1) * 4 + ((lane >> 2) & 1) * 2 + ((lane >> 1) & 1);
-            if ((lane & 1) == 0)
-                prm.part[((static_cast<long long>(cur.h) * g.tiles + cur.X) * 4 + warp) * 16 + comp] = part[0];
-            cur = nxt;
-            lse_cur = lse_nxt;
-            a16 = a16_nxt;
-        }
-        cp_async_wait<0>();
-    }
-
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-    if (warp == 0) tmem_dealloc(tmem, kTmemCols);
-}
-
-}  // namespace small
 
 }  // namespace bwdk
 
@@ -1179,39 +676,14 @@ cudaError_t launch_bwd(const Geo& g, const BwdPtrs& p, const BwdMaps& maps, unsi
     };
     if (g.N < kTile) {
         // windows inside one tile: the whole backward of a tile in one kernel
-        static bool small_attr = false;
-        if (!small_attr) {
-            e = cudaFuncSetAttribute(small::small_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     small::kSmemBytes);
-            if (e != cudaSuccess) return e;
-            small_attr = true;
-        }
+        float* part = reinterpret_cast<float*>(p.ws + L.part);
         mark(0);
         mark(1);
-        small::Params sp;
-        sp.g = g;
-        sp.q = static_cast<const uint8_t*>(p.q);
-        sp.k = static_cast<const uint8_t*>(p.k);
-        sp.v = static_cast<const uint8_t*>(p.v);
-        sp.o = static_cast<const uint8_t*>(p.o);
-        sp.dout = static_cast<const uint8_t*>(p.dout);
-        sp.dq = static_cast<uint8_t*>(p.dq);
-        sp.dk = static_cast<uint8_t*>(p.dk);
-        sp.dv = static_cast<uint8_t*>(p.dv);
-        sp.lse = p.lse;
-        sp.theta = p.theta;
-        sp.part = reinterpret_cast<float*>(p.ws + L.part);
-        sp.status = status;
-        sp.limit_ns = limit_ns;
-        sp.items = ht;
-        sp.scale = scale;
-        sp.head_minor = g.heads <= small::kTabHeads;
-        const long long grid = ht < 2ll * num_sms ? ht : 2ll * num_sms;
-        small::small_kernel<<<static_cast<unsigned>(grid), small::kThreads, small::kSmemBytes, stream>>>(sp);
-        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        e = launch_small_bwd(g, p, part, status, limit_ns, num_sms, stream);
+        if (e != cudaSuccess) return e;
         mark(2);
         mark(3);
-        dtheta_kernel<<<g.heads, 256, 0, stream>>>(sp.part, g.tiles * 4, p.dtheta);
+        dtheta_kernel<<<g.heads, 256, 0, stream>>>(part, g.tiles * 4, p.dtheta);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
         mark(4);
         return e;

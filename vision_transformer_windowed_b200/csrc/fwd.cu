@@ -496,7 +496,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 long long fwd_items(const Geo& g) { return fwd_item_count(g); }
 
 cudaError_t launch_fwd(const Geo& g, const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
-                       const CUtensorMap& mo, const float* theta, float* lse, unsigned int* status,
+                       const CUtensorMap& mo, const void* q, const void* k, const void* v, void* o,
+                       const float* theta, float* lse, unsigned int* status,
                        unsigned long long limit_ns, int num_sms, cudaStream_t stream, cudaEvent_t const* events) {
     fwdk::Params prm;
     prm.g = g;
@@ -506,6 +507,15 @@ cudaError_t launch_fwd(const Geo& g, const CUtensorMap& mq, const CUtensorMap& m
     prm.limit_ns = limit_ns;
     prm.items = fwd_items(g);
     if (prm.items == 0) return cudaSuccess;
+    if (g.N < kTile) {  // windows inside one tile
+        if (events) {
+            cudaError_t e = cudaEventRecord(events[0], stream);
+            if (e != cudaSuccess) return e;
+        }
+        cudaError_t e = launch_small_fwd(g, q, k, v, theta, o, lse, status, limit_ns, num_sms, stream);
+        if (e == cudaSuccess && events) e = cudaEventRecord(events[1], stream);
+        return e;
+    }
     static bool attr_set = false;
     if (!attr_set) {
         cudaError_t e = cudaFuncSetAttribute(fwdk::fwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,

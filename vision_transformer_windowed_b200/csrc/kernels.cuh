@@ -13,7 +13,8 @@ namespace fswin {
 
 long long fwd_items(const Geo& g);
 cudaError_t launch_fwd(const Geo& g, const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
-                       const CUtensorMap& mo, const float* theta, float* lse, unsigned int* status,
+                       const CUtensorMap& mo, const void* q, const void* k, const void* v, void* o,
+                       const float* theta, float* lse, unsigned int* status,
                        unsigned long long limit_ns, int num_sms, cudaStream_t stream, cudaEvent_t const* events);
 
 struct BwdPtrs {
@@ -36,5 +37,14 @@ size_t bwd_workspace_bytes(const Geo& g);
 // run one kernel in the place of the first three).
 cudaError_t launch_bwd(const Geo& g, const BwdPtrs& p, const BwdMaps& maps, unsigned int* status,
                        unsigned long long limit_ns, int num_sms, cudaStream_t stream, cudaEvent_t const* events);
+
+// Windows of fewer than 128 tokens (the tile holds whole windows): the whole
+// backward of a tile in one kernel (d theta partials, 4 x 16 per (head, tile),
+// into `part`), and the forward.
+cudaError_t launch_small_bwd(const Geo& g, const BwdPtrs& p, float* part, unsigned int* status,
+                             unsigned long long limit_ns, int num_sms, cudaStream_t stream);
+cudaError_t launch_small_fwd(const Geo& g, const void* q, const void* k, const void* v, const float* theta, void* o,
+                             float* lse, unsigned int* status, unsigned long long limit_ns, int num_sms,
+                             cudaStream_t stream);
 
 }  // namespace fswin
