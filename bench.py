@@ -340,7 +340,13 @@ def main():
     dom = max(ph, key=lambda n: main_res["phase_share"][n])
     th = B * H * W * heads
     pairs_per_launch = (main_res["fwd_flops"] / (4.0 * HEAD_DIM)) / nshift
-    algo_bytes = {"fwd": 260, "bwd_prep": 588, "bwd_main": 456, "bwd_post": 512, "bwd_dtheta": 0}
+    # bytes each kernel must move per token-head row: windows inside one tile run the whole
+    # backward as one kernel (Q, K, V, O, dO read, dQ, dK, dV written, LSE and D: 520 B);
+    # larger windows run prep / main / post with workspace round trips
+    if M * M < 128:
+        algo_bytes = {"fwd": 260, "bwd_prep": 0, "bwd_main": 520, "bwd_post": 0, "bwd_dtheta": 0}
+    else:
+        algo_bytes = {"fwd": 260, "bwd_prep": 588, "bwd_main": 456, "bwd_post": 512, "bwd_dtheta": 0}
     hbm_bound = M <= 8
     if hbm_bound or dom in ("bwd_prep", "bwd_post", "bwd_dtheta"):
         achieved = algo_bytes[dom] * th / (ph[dom] * 1e-3) / 1e9
