@@ -88,6 +88,7 @@ def test_workspace_flat_in_window_size():
     b = _lib.fs_winattn_bwd_workspace_bytes(_lib.make_shape(16, 256, 256, 3, 32, 64, 32))
     c = _lib.fs_winattn_bwd_workspace_bytes(_lib.make_shape(16, 256, 256, 3, 32, 8, 4))
     assert a == b == c > 0
-    # and linear in the number of tokens
+    # and linear in the number of tokens, up to a fixed per-head part (the d theta
+    # reduction's second level: heads x 64 x 16 floats)
     d = _lib.fs_winattn_bwd_workspace_bytes(_lib.make_shape(32, 256, 256, 3, 32, 32, 16))
-    assert abs(d - 2 * a) < 4096
+    assert abs(d - 2 * a) <= 3 * 64 * 16 * 4 + 4096

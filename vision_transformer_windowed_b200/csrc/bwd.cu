@@ -31,7 +31,7 @@ namespace bwdk {
 
 // ------------------------------------------------------------------ workspace
 struct WsLayout {
-    size_t qimg, kimg, doimg, lse2, dvec, dqacc, dkimg, part, total;
+    size_t qimg, kimg, doimg, lse2, dvec, dqacc, dkimg, part, part2, total;
 };
 
 __host__ __device__ inline size_t round256(size_t x) { return (x + 255) & ~size_t(255); }
@@ -48,6 +48,7 @@ __host__ __device__ inline WsLayout ws_layout(const Geo& g) {
     L.dqacc = o; o += round256(ht * kTile * kHeadDim * 4);
     L.dkimg = o; o += round256(ht * kTile * kHeadDim * 4);
     L.part = o;  o += round256(ht * 4 * 16 * 4);  // up to 4 x 16 partials per (head, tile)
+    L.part2 = o; o += round256(static_cast<size_t>(g.heads) * 64 * 16 * 4);  // level-1 d theta sums
     L.total = o;
     return L;
 }
@@ -639,23 +640,37 @@ __global__ void __launch_bounds__(128) post_kernel(const PostParams p) {
 }
 
 // ------------------------------------------------------------------ 4. reduce
-// part: [heads][per_head][16] partial sums; dtheta[h] = their sum, in a fixed order.
-__global__ void __launch_bounds__(256) dtheta_kernel(const float* part, long long per_head, float* dtheta) {
+// In two launches, each in a fixed order (deterministic d theta):
+//   level 1, grid (kSplit, heads): block b of head h sums its contiguous share
+//            of the head's [per_head][16] partials into out[h][b][16];
+//   level 2, grid (1, heads): the kSplit level-1 sums of each head.
+constexpr int kSplit = 64;
+
+__global__ void __launch_bounds__(256) dtheta_kernel(const float* part, long long per_head, float* out) {
     __shared__ float acc[16][17];
-    const int h = blockIdx.x;
+    const int h = blockIdx.y, b = blockIdx.x, nb = gridDim.x;
+    const long long lo = per_head * b / nb, hi = per_head * (b + 1) / nb;
     const int comp = threadIdx.x & 15, grp = threadIdx.x >> 4;
     float s = 0.f;
-    for (long long T = grp; T < per_head; T += 16) s += part[(static_cast<long long>(h) * per_head + T) * 16 + comp];
+    for (long long T = lo + grp; T < hi; T += 16) s += part[(static_cast<long long>(h) * per_head + T) * 16 + comp];
     acc[grp][comp] = s;
     __syncthreads();
     if (threadIdx.x < 16) {
         float t = 0.f;
         for (int i = 0; i < 16; ++i) t += acc[i][threadIdx.x];
-        dtheta[h * 16 + threadIdx.x] = t;
+        out[(static_cast<long long>(h) * nb + b) * 16 + threadIdx.x] = t;
     }
 }
 
-
+// part: [heads][per_head][16]; dtheta: [heads][16]; scratch: heads * kSplit * 16 floats
+cudaError_t launch_dtheta(const float* part, long long per_head, int heads, float* scratch, float* dtheta,
+                          cudaStream_t stream) {
+    dtheta_kernel<<<dim3(kSplit, heads), 256, 0, stream>>>(part, per_head, scratch);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    dtheta_kernel<<<dim3(1, heads), 256, 0, stream>>>(scratch, kSplit, dtheta);
+    return cudaGetLastError();
+}
 
 }  // namespace bwdk
 
@@ -683,8 +698,9 @@ cudaError_t launch_bwd(const Geo& g, const BwdPtrs& p, const BwdMaps& maps, unsi
         if (e != cudaSuccess) return e;
         mark(2);
         mark(3);
-        dtheta_kernel<<<g.heads, 256, 0, stream>>>(part, g.tiles * 4, p.dtheta);
-        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        if ((e = launch_dtheta(part, g.tiles * 4, g.heads, reinterpret_cast<float*>(p.ws + L.part2), p.dtheta,
+                               stream)) != cudaSuccess)
+            return e;
         mark(4);
         return e;
     }
@@ -719,8 +735,9 @@ cudaError_t launch_bwd(const Geo& g, const BwdPtrs& p, const BwdMaps& maps, unsi
     post_kernel<<<static_cast<unsigned>(ht), 128, 0, stream>>>(qp);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     mark(3);
-    dtheta_kernel<<<g.heads, 256, 0, stream>>>(reinterpret_cast<const float*>(p.ws + L.part), g.tiles, p.dtheta);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    if ((e = launch_dtheta(reinterpret_cast<const float*>(p.ws + L.part), g.tiles, g.heads,
+                           reinterpret_cast<float*>(p.ws + L.part2), p.dtheta, stream)) != cudaSuccess)
+        return e;
     mark(4);
     return e;
 }

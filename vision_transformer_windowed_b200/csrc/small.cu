@@ -307,6 +307,16 @@ __global__ void __launch_bounds__(kThreads, 2) small_kernel(const __grid_constan
             tc_fence_after();
 #pragma unroll 1
             for (int c = 0; c < 4; ++c) {
+                uint8_t* base = ds + (c >> 1) * 16384 + (r >> 3) * 1024 + (r & 7) * 128;
+                if (!__any_sync(0xFFFFFFFFu, ((a16 >> (2 * c)) & 3u) != 0u)) {  // P, dS = 0 for the whole warp
+                    const uint32_t z[16] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
+                    tmem_st16(trow + kColP + 16 * c, z);
+                    tmem_st16(trow + kColDS + 16 * c, z);
+#pragma unroll
+                    for (int q4 = 0; q4 < 4; ++q4)
+                        *reinterpret_cast<uint4*>(base + (((4 * (c & 1) + q4) ^ (r & 7)) << 4)) = make_uint4(0, 0, 0, 0);
+                    continue;
+                }
                 uint32_t sv[32], pv[32];
                 tmem_ld32(trow + kColS + 32 * c, sv);
                 tmem_ld32(trow + kColDP + 32 * c, pv);
@@ -337,7 +347,6 @@ __global__ void __launch_bounds__(kThreads, 2) small_kernel(const __grid_constan
                 tmem_st16(trow + kColP + 16 * c, wp);
                 tmem_st16(trow + kColDS + 16 * c, wd);
                 // dS (queries along M, keys along K) as an MN-major operand
-                uint8_t* base = ds + (c >> 1) * 16384 + (r >> 3) * 1024 + (r & 7) * 128;
 #pragma unroll
                 for (int q4 = 0; q4 < 4; ++q4) {
                     const int cc = 4 * (c & 1) + q4;
@@ -643,12 +652,16 @@ __global__ void __launch_bounds__(kThreads, 4) fwd_kernel(const __grid_constant_
             float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll 1
             for (int c = 0; c < 4; ++c) {
+                const uint32_t grp2 = (a16 >> (2 * c)) & 3u;  // this row's 16-column groups of the chunk
+                if (!__any_sync(0xFFFFFFFFu, grp2 != 0u)) continue;  // no row of the warp attends them
                 uint32_t v[32];
                 tmem_ld32(trow + kColS + 32 * c, v);
                 tmem_wait_ld();
+                if (grp2 != 3u) {
 #pragma unroll
-                for (int e = 0; e < 32; ++e)
-                    if (!((a16 >> (2 * c + (e >> 4))) & 1u)) v[e] = __float_as_uint(-INFINITY);
+                    for (int e = 0; e < 32; ++e)
+                        if (!((grp2 >> (e >> 4)) & 1u)) v[e] = __float_as_uint(-INFINITY);
+                }
 #pragma unroll
                 for (int e = 0; e < 32; e += 2)
                     mx4[(e >> 1) & 3] = fmax3(mx4[(e >> 1) & 3], __uint_as_float(v[e]), __uint_as_float(v[e + 1]));
@@ -657,6 +670,11 @@ __global__ void __launch_bounds__(kThreads, 4) fwd_kernel(const __grid_constant_
             float l4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll 1
             for (int c = 0; c < 4; ++c) {
+                if (!__any_sync(0xFFFFFFFFu, ((a16 >> (2 * c)) & 3u) != 0u)) {  // P = 0 for the whole warp
+                    const uint32_t z[16] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
+                    tmem_st16(trow + kColP + 16 * c, z);
+                    continue;
+                }
                 uint32_t v[32];
                 tmem_ld32(trow + kColS + 32 * c, v);
                 tmem_wait_ld();
