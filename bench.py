@@ -231,7 +231,7 @@ def main():
     import torch
     import torch.distributed as dist
 
-    from vision_transformer_windowed_b200 import _lib, ops
+    from vision_transformer_windowed_b200 import _lib, dp, ops
     from vision_transformer_windowed_b200.inputs import make_inputs
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -252,7 +252,7 @@ def main():
     def run_workload(name, steps, warmup, phase=True, clocks=False):
         wl = WORKLOADS[name]
         B, H, W, heads, M = wl["B"], wl["H"], wl["W"], wl["heads"], wl["M"]
-        t = make_inputs(B, H, W, heads, HEAD_DIM, device=dev, qk_scale=wl["qk_scale"])
+        t = dp.rank_inputs(B, H, W, heads, HEAD_DIM, rank, dev, qk_scale=wl["qk_scale"])
         q, k, v, th, do = t["q"], t["k"], t["v"], t["theta"], t["dout"]
         outs = {s: (torch.empty_like(q), torch.empty((B, H, W, heads), device=dev, dtype=torch.float32))
                 for s in wl["shifts"]}
@@ -270,8 +270,7 @@ def main():
                 if evs is not None:
                     _lib.fs_set_phase_events([e.cuda_event for e in evs[si][1]])
                 ops.winattn_bwd(q, k, v, o, do, lse, th, M, s, workspace=ws, dq=dq, dk=dk, dv=dv, dtheta=dth)
-                if world > 1:
-                    dist.all_reduce(dth)  # theta is shared by the whole data-parallel batch
+                dp.allreduce_dtheta(dth)  # theta is shared by the whole data-parallel batch
             if evs is not None:
                 _lib.fs_set_phase_events([])
 
@@ -303,11 +302,7 @@ def main():
         torch.cuda.synchronize()
         barrier()
         clk = sampler.stop() if sampler else None
-        ms = e0.elapsed_time(e1) / steps
-        if world > 1:
-            tm = torch.tensor([ms], device=dev)
-            dist.all_reduce(tm, op=dist.ReduceOp.MAX)
-            ms = float(tm.item())
+        ms = dp.max_over_ranks(e0.elapsed_time(e1) / steps, dev)
         assert _lib.fs_device_status() == 0, "a kernel reported a device-side failure"
         peak_gb = torch.cuda.max_memory_allocated(dev) / 1e9
         fwd_f, bwd_f = workload_flops(wl)
@@ -379,8 +374,7 @@ def main():
         for s in wl["shifts"]:
             o, lse = ops.winattn_fwd(dv["q"], dv["k"], dv["v"], dv["theta"], M, s)
             dq, dk, dvv, dth = ops.winattn_bwd(dv["q"], dv["k"], dv["v"], o, dv["dout"], lse, dv["theta"], M, s)
-            if world > 1:
-                dist.all_reduce(dth)
+            dp.allreduce_dtheta(dth)
             for name, x in (("o", o), ("dq", dq), ("dk", dk), ("dv", dvv), ("dtheta", dth)):
                 key = (s, name)
                 if key not in res_host:
@@ -397,11 +391,7 @@ def main():
         e2e_step()
     b.record()
     torch.cuda.synchronize()
-    e2e_ms = a.elapsed_time(b) / e2e_steps
-    if world > 1:
-        tm = torch.tensor([e2e_ms], device=dev)
-        dist.all_reduce(tm, op=dist.ReduceOp.MAX)
-        e2e_ms = float(tm.item())
+    e2e_ms = dp.max_over_ranks(a.elapsed_time(b) / e2e_steps, dev)
     fl = main_res["fwd_flops"] + main_res["bwd_flops"]
     e2e = {"value": fl * world / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s", "ms_per_step": e2e_ms,
            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}

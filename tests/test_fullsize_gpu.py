@@ -1,0 +1,92 @@
+"""GPU parity at the full sizes of the workloads, on sampled windows.
+
+The whole problem runs on the GPU exactly as the benchmark runs it; the fp64
+oracle then computes a sample of (image, window, head) units one by one, and
+the sampled tokens of O, LSE, dQ, dK, dV are compared.  The sample always
+holds windows of the last window row and column (the only ones the shift mask
+cuts) and of the first.  dθ sums over every token, so it is checked through a
+property that holds at any size: with dO zero outside the sampled units, the
+other units contribute nothing, and dθ equals the sum of the sampled units'
+shares.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from vision_transformer_windowed_b200 import ops
+from vision_transformer_windowed_b200.inputs import make_inputs
+
+FWD_TOL = (1e-2, 2e-3)
+GRAD_TOL = (3e-2, 5e-3)
+
+# (name, B, H, W, heads, M, s, qk_scale): the benchmark workloads and the
+# FlashSwin-T stage shapes at 256 x 256 input with patch 2
+FULL = [
+    ("swin_t_stage1_p4_m8_s0", 128, 64, 64, 3, 8, 0, 1.0),
+    ("swin_t_stage1_p4_m8_s4", 128, 64, 64, 3, 8, 4, 1.0),
+    ("flashswin_t_stage1_p2_m32", 128, 128, 128, 3, 32, 16, 1.0),
+    ("flashswin_t_stage2_p2_m32_s0", 128, 64, 64, 6, 32, 0, 1.0),
+    ("flashswin_t_stage3_p2_m32_s16", 128, 32, 32, 12, 32, 16, 1.0),
+    ("flashswin_t_stage4_p2_m16", 128, 16, 16, 24, 16, 0, 1.0),
+    ("highres_p2_m64", 16, 256, 256, 3, 64, 32, 3.0),
+]
+
+
+def _check(name, got, ref, tol):
+    got = np.asarray(got, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    assert got.shape == ref.shape, name
+    assert np.isfinite(got).all(), f"{name}: non-finite values"
+    err = np.abs(got - ref).max()
+    bound = tol[0] * np.abs(ref).max() + tol[1]
+    assert err <= bound, f"{name}: max|err| {err:.4g} > {bound:.4g}"
+
+
+def _sample_units(B, H, W, heads, M, n_random=6, seed=7):
+    nWh, nWw = H // M, W // M
+    nW = nWh * nWw
+    picks = {(0, 0, 0), (B - 1, nWh - 1, nWw - 1), (0, nWh - 1, 0), (0, 0, nWw - 1), (B // 2, nWh - 1, nWw // 2)}
+    rng = np.random.default_rng(seed)
+    for _ in range(n_random):
+        picks.add((int(rng.integers(B)), int(rng.integers(nWh)), int(rng.integers(nWw))))
+    units = []
+    for b, wr, wc in sorted(picks):
+        for h in range(heads) if heads <= 3 else (0, heads // 2, heads - 1):
+            units.append((b * nW + wr * nWw + wc) * heads + h)
+    return np.array(sorted(set(units)), dtype=np.int64)
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("cfg", FULL, ids=[c[0] for c in FULL])
+def test_full_size_sampled_windows(cfg):
+    name, B, H, W, heads, M, s, qk = cfg
+    inp = make_inputs(B, H, W, heads, 32, qk_scale=qk)
+    units = _sample_units(B, H, W, heads, M)
+    pos = [oracle.unit_token_positions(H, W, M, s, int(u), heads) for u in units]
+    # dO kept on the sampled units' tokens only
+    keep = torch.zeros((B, H, W, heads), dtype=torch.bool)
+    for b, rows, cols, h in pos:
+        keep[b, torch.from_numpy(rows), torch.from_numpy(cols), h] = True
+    dout = torch.where(keep[..., None], inp["dout"], torch.zeros((), dtype=inp["dout"].dtype))
+
+    dev = {k: v.cuda() for k, v in inp.items() if k != "dout"}
+    o, lse = ops.winattn_fwd(dev["q"], dev["k"], dev["v"], dev["theta"], M, s)
+    dq, dk, dv, dth = ops.winattn_bwd(dev["q"], dev["k"], dev["v"], o, dout.cuda(), lse, dev["theta"], M, s)
+    torch.cuda.synchronize()
+
+    ref = oracle.units(inp["q"], inp["k"], inp["v"], inp["theta"], M, s, units, dout=dout)
+    idx = lambda t, b, rows, cols, h: t[b, torch.from_numpy(rows), torch.from_numpy(cols), h]
+    got = {k: [] for k in ("o", "lse", "dq", "dk", "dv")}
+    for b, rows, cols, h in pos:
+        for key, t in (("o", o), ("lse", lse), ("dq", dq), ("dk", dk), ("dv", dv)):
+            got[key].append(idx(t, b, rows, cols, h).float().cpu().numpy())
+    _check(f"{name} o", np.stack(got["o"]), ref["o"], FWD_TOL)
+    _check(f"{name} lse", np.stack(got["lse"]), ref["lse"], FWD_TOL)
+    for key in ("dq", "dk", "dv"):
+        _check(f"{name} {key}", np.stack(got[key]), ref[key], GRAD_TOL)
+    # dθ: only the sampled units carry dO, so the total is their sum
+    want = np.zeros((heads, 2, 8))
+    for u, share in zip(units, ref["dtheta"]):
+        want[int(u) % heads] += share
+    _check(f"{name} dtheta", dth.float().cpu().numpy(), want, GRAD_TOL)

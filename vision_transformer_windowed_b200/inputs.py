@@ -41,14 +41,17 @@ def theta_init(heads: int, d: int, device="cpu", noise: float = 0.01, seed: int 
 
 
 def make_inputs(B: int, H: int, W: int, heads: int, d: int, device="cpu", qk_scale: float = 1.0,
-                with_dout: bool = True) -> dict:
+                with_dout: bool = True, shard: int = 0) -> dict:
+    """`shard` > 0 draws other images (seeds offset by 16 * shard) with the same
+    theta: the per-process batch of a data-parallel run."""
     shape = (B, H, W, heads, d)
+    off = 16 * shard
     out = {
-        "q": _normal(shape, SEED_Q, device, qk_scale),
-        "k": _normal(shape, SEED_K, device, qk_scale),
-        "v": _normal(shape, SEED_V, device),
+        "q": _normal(shape, SEED_Q + off, device, qk_scale),
+        "k": _normal(shape, SEED_K + off, device, qk_scale),
+        "v": _normal(shape, SEED_V + off, device),
         "theta": theta_init(heads, d, device),
     }
     if with_dout:
-        out["dout"] = _normal(shape, SEED_DO, device)
+        out["dout"] = _normal(shape, SEED_DO + off, device)
     return out
