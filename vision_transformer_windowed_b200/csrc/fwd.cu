@@ -47,15 +47,19 @@ __device__ __forceinline__ int ost_off(int w) { return w * kWorkerBytes + kQByte
 __device__ __forceinline__ int tab_off(int w) { return w * kWorkerBytes + kQBytes + kKVBytes + kTileBytes; }
 
 // TMEM columns per worker: S [128 cols], P (bf16) [64], O tile [32]
+// TMEM columns per worker: two S buffers of 128 columns, used by alternate
+// tiles.  A tile's P (bf16) is written over the first 64 columns of its S
+// buffer as the softmax consumes them, and the tile's P V product goes to
+// columns 64-95 of the same buffer (consumed before P V is issued), so the next
+// tile's S = Q K^T, in the other buffer, runs while this tile's softmax does.
 constexpr uint32_t kTmemCols = 512;
-__device__ __forceinline__ uint32_t col_s(int w) { return w * 256; }
-__device__ __forceinline__ uint32_t col_p(int w) { return w * 256 + 128; }
-__device__ __forceinline__ uint32_t col_o(int w) { return w * 256 + 192; }
+__device__ __forceinline__ uint32_t col_s(int w, uint32_t b) { return w * 256 + b * 128; }
+constexpr uint32_t kColP = 0, kColO = 64;  // within an S buffer
 
 struct WorkerBars {
     uint64_t q_full[2], q_ready[2], q_empty[2];
     uint64_t kv_full[kStages], kv_ready[kStages], kv_empty[kStages];
-    uint64_t s_full, s_free, p_full, o_full, done;
+    uint64_t s_full[2], s_empty[2], p_full, o_full, done;  // s_empty[b]: buffer b's P V product read
     uint64_t grp;  // the worker's four softmax warps (a bounded group barrier)
 };
 struct Bars {
@@ -144,8 +148,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                 mbar_init(&b.kv_ready[i], 4);
                 mbar_init(&b.kv_empty[i], 1);
             }
-            mbar_init(&b.s_full, 1);
-            mbar_init(&b.s_free, 4);
+            for (int i = 0; i < 2; ++i) {
+                mbar_init(&b.s_full[i], 1);
+                mbar_init(&b.s_empty[i], 4);
+            }
             mbar_init(&b.p_full, 4);
             mbar_init(&b.o_full, 1);
             mbar_init(&b.done, 1);
@@ -207,14 +213,15 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint64_t dk0 = make_sdesc(smem_u32(smem + kv_off(wk)), 16, 512, kSw64);
             const uint64_t dv0 = make_sdesc(smem_u32(smem + kv_off(wk) + kTileBytes), 8192, 512, kSw64);
             constexpr uint32_t kQStep = kTileBytes >> 4, kKVStep = (2 * kTileBytes) >> 4;
-            const uint32_t t_s = tmem + col_s(wk), t_p = tmem + col_p(wk), t_o = tmem + col_o(wk);
             int it = 0;
-            uint32_t kvc = 0, pph = 0, sfph = 0;
+            uint32_t kvc = 0, pph = 0, tc = 0;  // tc: tiles of this worker so far (S buffer tc & 1)
             bool ok = true;
-            auto issue_pv = [&](int st) {
+            auto issue_pv = [&](int st, uint32_t b) {
                 const uint64_t dv = dv0 + static_cast<uint64_t>(st) * kKVStep;
+                const uint32_t t_b = tmem + col_s(wk, b);
 #pragma unroll
-                for (int k = 0; k < kTile / 16; ++k) umma_ts(t_o, t_p + 8 * k, dv + 64 * k, idesc_pv, k > 0);
+                for (int k = 0; k < kTile / 16; ++k)
+                    umma_ts(t_b + kColO, t_b + kColP + 8 * k, dv + 64 * k, idesc_pv, k > 0);
                 umma_commit(&B.o_full);
                 umma_commit(&B.kv_empty[st]);
             };
@@ -230,33 +237,31 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const uint32_t ph = (kvc / kStages) & 1;
                     ++kvc;
                     if (!mbar_wait(&B.kv_ready[st], ph, ctl, 0x302)) { ok = false; break; }
+                    // S buffer b is free once the softmax has read the P V product of
+                    // the tile two back (which also means that tile's P V is done)
+                    const uint32_t b = tc & 1u;
+                    if (tc >= 2 && !mbar_wait(&B.s_empty[b], ((tc >> 1) & 1u) ^ 1u, ctl, 0x303)) { ok = false; break; }
                     tc_fence_after();
-                    // the next S = Q K^T as soon as the softmax has read the previous S,
-                    // then P V of the previous tile once its P is in TMEM
-                    if (pend >= 0) {
-                        if (!mbar_wait(&B.s_free, sfph, ctl, 0x303)) { ok = false; break; }
-                        sfph ^= 1;
-                        tc_fence_after();
-                    }
+                    const uint32_t t_s = tmem + col_s(wk, b);
                     const uint64_t dk = dk0 + static_cast<uint64_t>(st) * kKVStep;
                     umma_ss(t_s, dq, dk, idesc_qk, 0u);
                     umma_ss(t_s, dq + 2, dk + 2, idesc_qk, 1u);  // second 16-channel step: +32 bytes
-                    umma_commit(&B.s_full);
+                    umma_commit(&B.s_full[b]);
+                    // then P V of the previous tile once its P is in TMEM
                     if (pend >= 0) {
                         if (!mbar_wait(&B.p_full, pph, ctl, 0x304)) { ok = false; break; }
                         pph ^= 1;
                         tc_fence_after();
-                        issue_pv(pend);
+                        issue_pv(pend, b ^ 1u);
                     }
                     pend = st;
+                    ++tc;
                 }
                 if (ok && pend >= 0) {
-                    if (!mbar_wait(&B.s_free, sfph, ctl, 0x305)) break;
-                    sfph ^= 1;
                     if (!mbar_wait(&B.p_full, pph, ctl, 0x306)) break;
                     pph ^= 1;
                     tc_fence_after();
-                    issue_pv(pend);
+                    issue_pv(pend, (tc - 1) & 1u);
                 }
                 umma_commit(&B.q_empty[qi]);
             }
@@ -269,13 +274,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int quarter = warp & 3;
         const int r = quarter * 32 + lane;
         const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
-        const uint32_t t_s = tmem + lane_off + col_s(wk), t_p = tmem + lane_off + col_p(wk),
-                       t_o = tmem + lane_off + col_o(wk);
+        const uint32_t t_row = tmem + lane_off;  // this warp's TMEM lanes
+        uint32_t tcs = 0;                         // tiles of this worker so far (S buffer tcs & 1)
         uint8_t* ost = smem + ost_off(wk);
         float2* tab = reinterpret_cast<float2*>(smem + tab_off(wk));
         const bool leader = (quarter == 0 && lane == 0);
         const float sl2 = g.scale_log2;
-        uint32_t sph = 0, oph = 0, gph = 0, kvc_rot = 0;
+        uint32_t oph = 0, gph = 0, kvc_rot = 0;
         int tab_head = -1;
         bool ok = true;
         // Waits are made warp-uniform: a lane that gave up takes its warp out
@@ -348,8 +353,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (!rotate_next()) { ok = false; break; }
                 const uint32_t a16 = d_allow16(g, myseg, I.kv0 + u, I.win);
                 const bool full = a16 == 0xFFu;
-                if (!wwait(&B.s_full, sph, 0x403)) { ok = false; break; }
-                sph ^= 1;
+                const uint32_t b = tcs & 1u;
+                const uint32_t t_s = t_row + col_s(wk, b);
+                if (!wwait(&B.s_full[b], (tcs >> 1) & 1u, 0x403)) { ok = false; break; }
                 tc_fence_after();
                 // pass 1: row maximum of the attended raw scores
                 float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
@@ -369,13 +375,16 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 const float mx = fmaxf(fmax3(mx4[0], mx4[1], mx4[2]), mx4[3]);
                 const float m_tile = mx * sl2;
-                if (!first) {
+                if (!first) {  // the previous tile's P V product, in the other S buffer
                     if (!wwait(&B.o_full, oph, 0x404)) { ok = false; break; }
                     oph ^= 1;
                     tc_fence_after();
                     uint32_t v[32];
-                    tmem_ld32(t_o, v);
+                    tmem_ld32(t_row + col_s(wk, b ^ 1u) + kColO, v);
                     tmem_wait_ld();
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&B.s_empty[b ^ 1u]);
 #pragma unroll
                     for (int e = 0; e < 32; e += 2)
                         fadd2(o[e], o[e + 1], o[e], o[e + 1], __uint_as_float(v[e]), __uint_as_float(v[e + 1]));
@@ -396,11 +405,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                     uint32_t v[32];
                     tmem_ld32(t_s + 32 * c, v);
                     tmem_wait_ld();
-                    if (c == 3) {  // S fully read: the next S = Q K^T may overwrite it
-                        tc_fence_before();
-                        __syncwarp();
-                        if (lane == 0) mbar_arrive(&B.s_free);
-                    }
                     const float add0 = ((a16 >> (2 * c)) & 1u) ? -mu : -INFINITY;
                     const float add1 = ((a16 >> (2 * c + 1)) & 1u) ? -mu : -INFINITY;
                     uint32_t w[16];
@@ -414,7 +418,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         fadd2(l4[a], l4[a + 1], l4[a], l4[a + 1], p0, p1);
                         w[e] = pack_bf16x2(p0, p1);
                     }
-                    tmem_st16(t_p + 16 * c, w);
+                    tmem_st16(t_s + kColP + 16 * c, w);  // over columns of S already read
                 }
                 l += (l4[0] + l4[1]) + (l4[2] + l4[3]);
                 tmem_wait_st();
@@ -422,6 +426,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&B.p_full);
                 first = false;
+                ++tcs;
             }
             if (!ok) break;
             const long long X = I.X;
@@ -435,9 +440,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             oph ^= 1;
             tc_fence_after();
             {
+                const uint32_t bl = (tcs - 1) & 1u;  // the item's last tile
                 uint32_t v[32];
-                tmem_ld32(t_o, v);
+                tmem_ld32(t_row + col_s(wk, bl) + kColO, v);
                 tmem_wait_ld();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&B.s_empty[bl]);
 #pragma unroll
                 for (int e = 0; e < 32; e += 2)
                     fadd2(o[e], o[e + 1], o[e], o[e + 1], __uint_as_float(v[e]), __uint_as_float(v[e + 1]));
