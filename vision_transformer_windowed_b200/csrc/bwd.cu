@@ -152,6 +152,19 @@ __global__ void __launch_bounds__(128) prep_kernel(const PrepParams p) {
 }
 
 // ------------------------------------------------------------------ 2. main
+// A work item is one 128-key tile u and the query tiles of its window that
+// attend it; a step is one (u, query tile) pair, done in two half-steps of 64
+// queries.  Per half-step h (counter hc, TMEM buffer b = hc & 1):
+//   MMA warp:      S^T_h = K' Q'_h^T and dP^T_h = V dO_h^T (N = 64) into buffer b
+//   compute warps: P^T = exp2(S^T c - lse2), dS^T = P^T (dP^T - D) into the
+//                  buffer's P^T, dS^T columns, and dS into shared memory
+//   MMA warp:      dV += P^T dO_h, dK' += dS^T Q'_h; after both halves
+//                  dQ' = dS K' (a double-buffered accumulator); then the
+//                  S^T, dP^T of the half-step two ahead into the same buffer
+// so the compute warps work on one buffer while the tensor core fills the
+// other and never wait for the previous gradients.
+//   epilogue warps: dQ' of each step to the fp32 accumulator (bulk
+//                   reduce-add), dK' and dV of each item.
 constexpr int kThreads = 448;
 constexpr int kQStages = 3;
 constexpr int kWarpTma = 12, kWarpMma = 13;  // warps 0-7: P/dS, 8-11: epilogue
@@ -159,25 +172,36 @@ constexpr int kWarpTma = 12, kWarpMma = 13;  // warps 0-7: P/dS, 8-11: epilogue
 constexpr int kQStageBytes = 2 * kTileBytes + 2 * kTile * 4;  // Q', dO, lse2, D
 constexpr int kKVOff = 0;                                      // 2 slots x (K', V)
 constexpr int kQOff = kKVOff + 2 * 2 * kTileBytes;
-constexpr int kDSOff = kQOff + kQStages * kQStageBytes;        // dS, MN-major 128B swizzle
-constexpr int kDQStOff = kDSOff + 4 * kTileBytes;              // 2 x fp32 [128][32]
+constexpr int kDSOff = kQOff + kQStages * kQStageBytes;        // 2 x dS, MN-major 128B swizzle
+constexpr int kDSBytes = 4 * kTileBytes;
+constexpr int kDQStOff = kDSOff + 2 * kDSBytes;                // 2 x fp32 [128][32]
 constexpr int kDKStOff = kDQStOff + 2 * 4 * kTile * kHeadDim;  // fp32 [128][32]
 constexpr int kDVStOff = kDKStOff + 4 * kTile * kHeadDim;      // bf16 tile
 constexpr int kBarOff = kDVStOff + kTileBytes;
 constexpr int kSmemBytes = kBarOff + 1024 + 1024;
+static_assert(kDSOff % 1024 == 0, "128-byte swizzled operand must be 1024-byte aligned");
 
+// TMEM columns (all 512): half-step buffer b: S^T at 128 b, dP^T at 128 b + 64
+// (64 columns each); its P^T (bf16) at 256 + 64 b and dS^T (fp16) at
+// 256 + 64 b + 32 (32 columns each, 8 per K step of 16 queries), apart from
+// S^T and dP^T, so that the next S^T, dP^T of the buffer never overwrite what
+// pending gradient MMAs read; dQ' accumulators at 384 + 32 c (step parity c);
+// dV at 448, dK' at 480.
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColS = 0, kColDP = 128, kColP = 256, kColDS = 320, kColDQ = 384, kColDV = 416, kColDK = 448;
+constexpr uint32_t kColDQ = 384, kColDV = 448, kColDK = 480;
+__device__ __forceinline__ uint32_t col_buf(uint32_t b) { return 128u * b; }
+__device__ __forceinline__ uint32_t col_pb(uint32_t b) { return 256u + 64u * b; }
 
 struct Bars {
     uint64_t kv_full[2], kv_empty[2];
     uint64_t q_full[kQStages], q_empty[kQStages];
-    uint64_t s_full, p_full, mma2_done;
-    uint64_t dq_full, dq_free, dkv_full, dkv_free;
+    uint64_t s_full[2], p_full[2];
+    uint64_t dq_full[2], dq_free[2], dkv_full, dkv_free;
     uint64_t done;
     uint32_t tmem_base;
     int abort_flag;
 };
+static_assert(sizeof(Bars) <= 1024, "barrier block overflows its slot");
 
 struct MainParams {
     Geo g;
@@ -207,16 +231,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int i = 0; i < 2; ++i) {
             mbar_init(&bars->kv_full[i], 1);
             mbar_init(&bars->kv_empty[i], 1);
+            mbar_init(&bars->s_full[i], 1);
+            mbar_init(&bars->p_full[i], 8);
+            mbar_init(&bars->dq_full[i], 1);
+            mbar_init(&bars->dq_free[i], 4);
         }
         for (int i = 0; i < kQStages; ++i) {
             mbar_init(&bars->q_full[i], 1);
             mbar_init(&bars->q_empty[i], 1);
         }
-        mbar_init(&bars->s_full, 1);
-        mbar_init(&bars->p_full, 8);
-        mbar_init(&bars->mma2_done, 1);
-        mbar_init(&bars->dq_full, 1);
-        mbar_init(&bars->dq_free, 4);
         mbar_init(&bars->dkv_full, 1);
         mbar_init(&bars->dkv_free, 4);
         mbar_init(&bars->done, 1);
@@ -271,138 +294,147 @@ __global__ void __launch_bounds__(kThreads, 1)
         // ------------------------------------------------------------ MMA issue
         if (lane == 0) {
             // operand types: Q', K', dS in fp16; V, dO, P in bf16
-            const uint32_t id_s = make_idesc(kTile, kTile, false, false, true);
-            const uint32_t id_dp = make_idesc(kTile, kTile, false, false, false);
-            const uint32_t id_kv = make_idesc(kTile, kHeadDim, false, true, false);
+            const uint32_t id_s = make_idesc(kTile, 64, false, false, true);
+            const uint32_t id_dp = make_idesc(kTile, 64, false, false, false);
+            const uint32_t id_dv = make_idesc(kTile, kHeadDim, false, true, false);
             const uint32_t id_dk = make_idesc(kTile, kHeadDim, false, true, true);
             const uint32_t id_dq = make_idesc(kTile, kHeadDim, true, true, true);
-            const uint32_t ds_addr = smem_u32(smem + kDSOff);
-            // state of the step whose second half is pending
-            bool have_prev = false;
-            int prev_st = 0, prev_ks = 0;
-            bool prev_first = false, prev_last = false;
-            int prev_item_idx = -1;
-            uint32_t pph = 0, dqph = 0, dkvph = 0;
+            // cursor over this CTA's steps: items and their attending query tiles
+            struct Step {
+                bool valid, first, last;
+                int it, ks, st;
+                uint32_t qph;
+            };
+            long long c_item = blockIdx.x;
+            int c_it = 0, c_n = -1;
+            uint32_t c_qc = 0;
+            bool c_loaded = false;
+            Item CI{};
+            auto next_step = [&]() -> Step {
+                Step s{};
+                while (c_item < prm.items) {
+                    if (!c_loaded) {
+                        CI = item_of(g, c_item);
+                        c_loaded = true;
+                        c_n = -1;
+                    }
+                    int n = c_n + 1;
+                    while (n < CI.nq && !q_active(g, CI, n)) ++n;
+                    if (n < CI.nq) {
+                        int n2 = n + 1;
+                        while (n2 < CI.nq && !q_active(g, CI, n2)) ++n2;
+                        s.valid = true;
+                        s.first = c_n < 0;
+                        s.last = n2 >= CI.nq;
+                        s.it = c_it;
+                        s.ks = c_it & 1;
+                        s.st = static_cast<int>(c_qc % kQStages);
+                        s.qph = (c_qc / kQStages) & 1;
+                        ++c_qc;
+                        c_n = n;
+                        return s;
+                    }
+                    c_loaded = false;  // item done
+                    c_item += gridDim.x;
+                    ++c_it;
+                }
+                return s;
+            };
+            auto wait_inputs = [&](const Step& s) -> bool {
+                if (s.first && !mbar_wait(&bars->kv_full[s.ks], (s.it >> 1) & 1, ctl, 0x1302)) return false;
+                return mbar_wait(&bars->q_full[s.st], s.qph, ctl, 0x1303);
+            };
+            // S^T_h = K' Q'_h^T and dP^T_h = V dO_h^T into buffer b
+            auto issue_sdp = [&](const Step& s, int h, uint32_t b) {
+                const uint32_t ka = smem_u32(smem + kKVOff + s.ks * 2 * kTileBytes), va = ka + kTileBytes;
+                const uint32_t qa = smem_u32(smem + kQOff + s.st * kQStageBytes) + 4096u * h;  // rows 64h..
+                const uint32_t da = qa + kTileBytes;
+                const uint32_t t_b = tmem + col_buf(b);
+#pragma unroll
+                for (int k = 0; k < kHeadDim / 16; ++k)
+                    umma_ss(t_b, make_sdesc(ka + 32 * k, 16, 512, kSw64), make_sdesc(qa + 32 * k, 16, 512, kSw64), id_s,
+                            k > 0);
+#pragma unroll
+                for (int k = 0; k < kHeadDim / 16; ++k)
+                    umma_ss(t_b + 64, make_sdesc(va + 32 * k, 16, 512, kSw64), make_sdesc(da + 32 * k, 16, 512, kSw64),
+                            id_dp, k > 0);
+                umma_commit(&bars->s_full[b]);
+            };
+            // dV += P^T_h dO_h, dK' += dS^T_h Q'_h (the item's first half-step starts them)
+            auto issue_grads = [&](const Step& s, int h, uint32_t b) {
+                const uint32_t qa = smem_u32(smem + kQOff + s.st * kQStageBytes), da = qa + kTileBytes;
+                const uint32_t t_p = tmem + col_pb(b);
+                const bool acc = !(s.first && h == 0);
+#pragma unroll
+                for (int k = 0; k < 4; ++k)
+                    umma_ts(tmem + kColDV, t_p + 8 * k, make_sdesc(da + 1024 * (4 * h + k), 8192, 512, kSw64), id_dv,
+                            (acc || k > 0) ? 1u : 0u);
+#pragma unroll
+                for (int k = 0; k < 4; ++k)
+                    umma_ts(tmem + kColDK, t_p + 32 + 8 * k, make_sdesc(qa + 1024 * (4 * h + k), 8192, 512, kSw64),
+                            id_dk, (acc || k > 0) ? 1u : 0u);
+            };
+            // dQ' = dS K' of a step into accumulator c
+            auto issue_dq = [&](const Step& s, uint32_t c) {
+                const uint32_t ka = smem_u32(smem + kKVOff + s.ks * 2 * kTileBytes);
+                const uint32_t dsa = smem_u32(smem + kDSOff + c * kDSBytes);
+#pragma unroll
+                for (int k = 0; k < kTile / 16; ++k)
+                    umma_ss(tmem + kColDQ + 32 * c, make_sdesc(dsa + 2048 * k, 16384, 1024, kSw128),
+                            make_sdesc(ka + 1024 * k, 8192, 512, kSw64), id_dq, k > 0);
+                umma_commit(&bars->dq_full[c]);
+            };
             bool ok = true;
-            // Step j issues S(j), dP(j) as soon as the softmax of step j-1 has read
-            // S and dP, then the second half of step j-1: dV, dK and dQ.
-            int it = 0;
-            uint32_t qc = 0;
-            long long nsteps_done = 0;
-            for (long long item = blockIdx.x; item < prm.items && ok; item += gridDim.x, ++it) {
-                const Item I = item_of(g, item);
-                const int ks = it & 1;
-                if (!mbar_wait(&bars->kv_full[ks], (it >> 1) & 1, ctl, 0x1302)) break;
-                const uint32_t kaddr = smem_u32(smem + kKVOff + ks * 2 * kTileBytes);
-                // count active query tiles to know the last step of the item
-                int last_n = -1;
-                for (int n = 0; n < I.nq; ++n)
-                    if (q_active(g, I, n)) last_n = n;
-                bool first = true;
-                for (int n = 0; n < I.nq && ok; ++n) {
-                    if (!q_active(g, I, n)) continue;
-                    const int st = qc % kQStages;
-                    const uint32_t ph = (qc / kQStages) & 1;
-                    ++qc;
-                    if (!mbar_wait(&bars->q_full[st], ph, ctl, 0x1303)) { ok = false; break; }
-                    if (have_prev) {
-                        if (!mbar_wait(&bars->p_full, pph, ctl, 0x1304)) { ok = false; break; }
-                        pph ^= 1;
-                    }
+            Step cur = next_step();
+            if (cur.valid) {
+                ok = wait_inputs(cur);
+                if (ok) {
                     tc_fence_after();
-                    const uint32_t qaddr = smem_u32(smem + kQOff + st * kQStageBytes);
-                    // S^T = K' Q'^T and dP^T = V dO^T
-#pragma unroll
-                    for (int k = 0; k < kHeadDim / 16; ++k)
-                        umma_ss(tmem + kColS, make_sdesc(kaddr + 32 * k, 16, 512, kSw64),
-                                make_sdesc(qaddr + 32 * k, 16, 512, kSw64), id_s, k > 0);
-#pragma unroll
-                    for (int k = 0; k < kHeadDim / 16; ++k)
-                        umma_ss(tmem + kColDP, make_sdesc(kaddr + kTileBytes + 32 * k, 16, 512, kSw64),
-                                make_sdesc(qaddr + kTileBytes + 32 * k, 16, 512, kSw64), id_dp, k > 0);
-                    umma_commit(&bars->s_full);
-                    if (have_prev) {
-                        // second half of the previous step
-                        const uint32_t pk = smem_u32(smem + kKVOff + prev_ks * 2 * kTileBytes);
-                        const uint32_t pq = smem_u32(smem + kQOff + prev_st * kQStageBytes);
-                        if (prev_first && prev_item_idx > 0) {
-                            if (!mbar_wait(&bars->dkv_free, dkvph, ctl, 0x1305)) { ok = false; break; }
-                            dkvph ^= 1;
-                            tc_fence_after();
-                        }
-#pragma unroll
-                        for (int k = 0; k < kTile / 16; ++k)
-                            umma_ts(tmem + kColDV, tmem + kColP + 8 * k,
-                                    make_sdesc(pq + kTileBytes + 1024 * k, 8192, 512, kSw64), id_kv,
-                                    (!prev_first || k > 0) ? 1u : 0u);
-#pragma unroll
-                        for (int k = 0; k < kTile / 16; ++k)
-                            umma_ts(tmem + kColDK, tmem + kColDS + 8 * k, make_sdesc(pq + 1024 * k, 8192, 512, kSw64),
-                                    id_dk, (!prev_first || k > 0) ? 1u : 0u);
-                        if (nsteps_done > 0) {
-                            if (!mbar_wait(&bars->dq_free, dqph, ctl, 0x1306)) { ok = false; break; }
-                            dqph ^= 1;
-                            tc_fence_after();
-                        }
-#pragma unroll
-                        for (int k = 0; k < kTile / 16; ++k)
-                            umma_ss(tmem + kColDQ, make_sdesc(ds_addr + 2048 * k, 16384, 1024, kSw128),
-                                    make_sdesc(pk + 1024 * k, 8192, 512, kSw64), id_dq, k > 0);
-                        umma_commit(&bars->mma2_done);
-                        umma_commit(&bars->dq_full);
-                        umma_commit(&bars->q_empty[prev_st]);
-                        if (prev_last) {
-                            umma_commit(&bars->dkv_full);
-                            umma_commit(&bars->kv_empty[prev_ks]);
-                        }
-                        ++nsteps_done;
-                    }
-                    have_prev = true;
-                    prev_st = st;
-                    prev_ks = ks;
-                    prev_first = first;
-                    prev_last = (n == last_n);
-                    prev_item_idx = it;
-                    first = false;
+                    issue_sdp(cur, 0, 0);
+                    issue_sdp(cur, 1, 1);
                 }
             }
-            if (ok && have_prev) {
-                const uint32_t pk = smem_u32(smem + kKVOff + prev_ks * 2 * kTileBytes);
-                const uint32_t pq = smem_u32(smem + kQOff + prev_st * kQStageBytes);
-                bool ok2 = mbar_wait(&bars->p_full, pph, ctl, 0x1307);
-                pph ^= 1;
-                if (ok2 && prev_first && prev_item_idx > 0) {
-                    ok2 = mbar_wait(&bars->dkv_free, dkvph, ctl, 0x1308);
-                    dkvph ^= 1;
-                }
-                if (ok2) {
+            uint32_t hc = 0, dkvph = 0;
+            long long j = 0;  // steps done
+            while (ok && cur.valid) {
+                const Step nxt = next_step();
+                bool nxt_ready = false;
+                for (int h = 0; h < 2; ++h, ++hc) {
+                    const uint32_t b = hc & 1u;
+                    if (!mbar_wait(&bars->p_full[b], (hc >> 1) & 1u, ctl, 0x1304)) { ok = false; break; }
+                    if (h == 0 && cur.first && cur.it > 0) {  // the epilogue has read the previous item's dV, dK'
+                        if (!mbar_wait(&bars->dkv_free, dkvph, ctl, 0x1305)) { ok = false; break; }
+                        dkvph ^= 1;
+                    }
                     tc_fence_after();
-#pragma unroll
-                    for (int k = 0; k < kTile / 16; ++k)
-                        umma_ts(tmem + kColDV, tmem + kColP + 8 * k,
-                                make_sdesc(pq + kTileBytes + 1024 * k, 8192, 512, kSw64), id_kv,
-                                (!prev_first || k > 0) ? 1u : 0u);
-#pragma unroll
-                    for (int k = 0; k < kTile / 16; ++k)
-                        umma_ts(tmem + kColDK, tmem + kColDS + 8 * k, make_sdesc(pq + 1024 * k, 8192, 512, kSw64),
-                                id_dk, (!prev_first || k > 0) ? 1u : 0u);
-                    if (nsteps_done > 0) {
-                        ok2 = mbar_wait(&bars->dq_free, dqph, ctl, 0x1309);
-                        dqph ^= 1;
+                    issue_grads(cur, h, b);
+                    if (h == 1) {
+                        const uint32_t c = static_cast<uint32_t>(j & 1);
+                        if (j >= 2 && !mbar_wait(&bars->dq_free[c], ((j >> 1) & 1) ^ 1, ctl, 0x1306)) {
+                            ok = false;
+                            break;
+                        }
                         tc_fence_after();
+                        issue_dq(cur, c);
+                        umma_commit(&bars->q_empty[cur.st]);
+                        if (cur.last) {
+                            umma_commit(&bars->dkv_full);
+                            umma_commit(&bars->kv_empty[cur.ks]);
+                        }
+                        ++j;
                     }
-                    if (ok2) {
-#pragma unroll
-                        for (int k = 0; k < kTile / 16; ++k)
-                            umma_ss(tmem + kColDQ, make_sdesc(ds_addr + 2048 * k, 16384, 1024, kSw128),
-                                    make_sdesc(pk + 1024 * k, 8192, 512, kSw64), id_dq, k > 0);
-                        umma_commit(&bars->mma2_done);
-                        umma_commit(&bars->dq_full);
-                        umma_commit(&bars->q_empty[prev_st]);
-                        umma_commit(&bars->dkv_full);
-                        umma_commit(&bars->kv_empty[prev_ks]);
+                    // the half-step two ahead into the same S^T, dP^T buffer (the
+                    // gradients read P^T, dS^T from their own columns)
+                    if (nxt.valid) {
+                        if (!nxt_ready) {
+                            if (!wait_inputs(nxt)) { ok = false; break; }
+                            nxt_ready = true;
+                            tc_fence_after();
+                        }
+                        issue_sdp(nxt, h, b);
                     }
                 }
+                cur = nxt;
             }
             umma_commit(&bars->done);
             mbar_wait(&bars->done, 0, ctl, 0x13ff);
@@ -410,83 +442,91 @@ __global__ void __launch_bounds__(kThreads, 1)
         __syncwarp();
     } else if (warp < 8) {
         // ------------------------------------------------------------ P^T, dS^T (thread = key row)
-        const int hw = warp >> 2;  // query half: columns [64 hw, 64 hw + 64)
+        const int cw = warp >> 2;  // 32-column chunk of the 64-query half-step
         const int quarter = warp & 3;
         const int r = quarter * 32 + lane;
         const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
         const float sl2 = g.scale_log2;
-        uint8_t* ds = smem + kDSOff;
-        uint32_t sph = 0, mph = 0;
-        uint32_t qc = 0;
-        bool started = false, ok = true;
+        uint32_t hc = 0, qc = 0;
+        long long j = 0;
+        bool ok = true;
         for (long long item = blockIdx.x; item < prm.items && ok; item += gridDim.x) {
             const Item I = item_of(g, item);
             const uint32_t keyseg = seg_at(d_tile_segs(g, I.u, I.win), r >> g.lBT);
-            for (int n = 0; n < I.nq; ++n) {
+            for (int n = 0; n < I.nq && ok; ++n) {
                 if (!q_active(g, I, n)) continue;
                 const int st = qc % kQStages;
                 ++qc;
                 const float* lse2 = reinterpret_cast<const float*>(smem + kQOff + st * kQStageBytes + 2 * kTileBytes);
                 const float* dvec = lse2 + kTile;
+                uint8_t* ds = smem + kDSOff + (j & 1) * kDSBytes;
                 // bit c: query columns [16 c, 16 c + 16) attend this key row
                 const uint32_t a16 = d_allow16(g, keyseg, I.q0 + n, I.win);
-                const bool full = ((a16 >> (4 * hw)) & 0xFu) == 0xFu;
-                if (!mbar_wait(&bars->s_full, sph, ctl, 0x1401)) { ok = false; break; }
-                sph ^= 1;
-                tc_fence_after();
-#pragma unroll 1
-                for (int c = 0; c < 2; ++c) {  // rolled: keeps live ranges (registers) short
-                    const int col0 = 64 * hw + 32 * c;
-                    uint32_t sv[32], pv[32];
-                    tmem_ld32(tmem + lane_off + kColS + col0, sv);
-                    tmem_ld32(tmem + lane_off + kColDP + col0, pv);
-                    tmem_wait_ld();
-                    const bool ok0 = full || ((a16 >> (col0 >> 4)) & 1u);
-                    const bool ok1 = full || ((a16 >> ((col0 >> 4) + 1)) & 1u);
-                    uint32_t wp[16], wd[16];
+                for (int h = 0; h < 2; ++h, ++hc) {
+                    const uint32_t b = hc & 1u;
+                    const int col0 = 64 * h + 32 * cw;  // this thread's 32 query columns
+                    const uint32_t tc = tmem + lane_off + col_buf(b) + 32 * cw;  // S^T chunk; dP^T chunk at +64
+                    const uint32_t tp = tmem + lane_off + col_pb(b) + 16 * cw;   // P^T chunk; dS^T chunk at +32
+                    uint8_t* base = ds + h * 16384 + (r >> 3) * 1024 + (r & 7) * 128;
+                    if (!__all_sync(0xFFFFFFFFu, mbar_wait(&bars->s_full[b], (hc >> 1) & 1u, ctl, 0x1401))) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t grp2 = (a16 >> (col0 >> 4)) & 3u;
+                    if (!__any_sync(0xFFFFFFFFu, grp2 != 0u)) {  // no key row of the warp attends these queries
+                        const uint32_t z[16] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
+                        tmem_st16(tp, z);
+                        tmem_st16(tp + 32, z);
 #pragma unroll
-                    for (int e4 = 0; e4 < 8; ++e4) {
-                        float4 L4 = *reinterpret_cast<const float4*>(lse2 + col0 + 4 * e4);
-                        const float4 D4 = *reinterpret_cast<const float4*>(dvec + col0 + 4 * e4);
-                        if (!(e4 < 4 ? ok0 : ok1)) L4 = make_float4(INFINITY, INFINITY, INFINITY, INFINITY);
-                        const int e = 4 * e4;
-                        float t0, t1, t2, t3;
-                        ffma2(t0, t1, __uint_as_float(sv[e]), __uint_as_float(sv[e + 1]), sl2, sl2, -L4.x, -L4.y);
-                        ffma2(t2, t3, __uint_as_float(sv[e + 2]), __uint_as_float(sv[e + 3]), sl2, sl2, -L4.z, -L4.w);
-                        const float p0 = ex2_approx(t0), p1 = ex2_approx(t1), p2 = ex2_approx(t2), p3 = ex2_approx(t3);
-                        float d0, d1, d2, d3;
-                        fadd2(d0, d1, __uint_as_float(pv[e]), __uint_as_float(pv[e + 1]), -D4.x, -D4.y);
-                        fadd2(d2, d3, __uint_as_float(pv[e + 2]), __uint_as_float(pv[e + 3]), -D4.z, -D4.w);
-                        fmul2(d0, d1, d0, d1, p0, p1);
-                        fmul2(d2, d3, d2, d3, p2, p3);
-                        wp[2 * e4] = pack_bf16x2(p0, p1);
-                        wp[2 * e4 + 1] = pack_bf16x2(p2, p3);
-                        wd[2 * e4] = pack_f16x2(d0, d1);
-                        wd[2 * e4 + 1] = pack_f16x2(d2, d3);
-                    }
-                    if (c == 0 && started) {
-                        if (!mbar_wait(&bars->mma2_done, mph, ctl, 0x1402)) { ok = false; break; }
-                        mph ^= 1;
-                        tc_fence_after();
-                    }
-                    tmem_st16(tmem + lane_off + kColP + col0 / 2, wp);
-                    tmem_st16(tmem + lane_off + kColDS + col0 / 2, wd);
-                    // dS (queries along M, keys along K) as an MN-major operand
-                    uint8_t* base = ds + hw * 16384 + (r >> 3) * 1024 + (r & 7) * 128;
+                        for (int q4 = 0; q4 < 4; ++q4)
+                            *reinterpret_cast<uint4*>(base + (((4 * cw + q4) ^ (r & 7)) << 4)) = make_uint4(0, 0, 0, 0);
+                    } else {
+                        uint32_t sv[32], pv[32];
+                        tmem_ld32(tc, sv);
+                        tmem_ld32(tc + 64, pv);
+                        tmem_wait_ld();
+                        const bool ok0 = grp2 & 1u, ok1 = (grp2 >> 1) & 1u;
+                        uint32_t wp[16], wd[16];
 #pragma unroll
-                    for (int q4 = 0; q4 < 4; ++q4) {
-                        const int cc = 4 * c + q4;
-                        *reinterpret_cast<uint4*>(base + ((cc ^ (r & 7)) << 4)) =
-                            make_uint4(wd[4 * q4], wd[4 * q4 + 1], wd[4 * q4 + 2], wd[4 * q4 + 3]);
+                        for (int e4 = 0; e4 < 8; ++e4) {
+                            float4 L4 = *reinterpret_cast<const float4*>(lse2 + col0 + 4 * e4);
+                            const float4 D4 = *reinterpret_cast<const float4*>(dvec + col0 + 4 * e4);
+                            if (!(e4 < 4 ? ok0 : ok1)) L4 = make_float4(INFINITY, INFINITY, INFINITY, INFINITY);
+                            const int e = 4 * e4;
+                            float t0, t1, t2, t3;
+                            ffma2(t0, t1, __uint_as_float(sv[e]), __uint_as_float(sv[e + 1]), sl2, sl2, -L4.x, -L4.y);
+                            ffma2(t2, t3, __uint_as_float(sv[e + 2]), __uint_as_float(sv[e + 3]), sl2, sl2, -L4.z,
+                                  -L4.w);
+                            const float p0 = ex2_approx(t0), p1 = ex2_approx(t1), p2 = ex2_approx(t2),
+                                        p3 = ex2_approx(t3);
+                            float d0, d1, d2, d3;
+                            fadd2(d0, d1, __uint_as_float(pv[e]), __uint_as_float(pv[e + 1]), -D4.x, -D4.y);
+                            fadd2(d2, d3, __uint_as_float(pv[e + 2]), __uint_as_float(pv[e + 3]), -D4.z, -D4.w);
+                            fmul2(d0, d1, d0, d1, p0, p1);
+                            fmul2(d2, d3, d2, d3, p2, p3);
+                            wp[2 * e4] = pack_bf16x2(p0, p1);
+                            wp[2 * e4 + 1] = pack_bf16x2(p2, p3);
+                            wd[2 * e4] = pack_f16x2(d0, d1);
+                            wd[2 * e4 + 1] = pack_f16x2(d2, d3);
+                        }
+                        tmem_st16(tp, wp);
+                        tmem_st16(tp + 32, wd);
+                        // dS (queries along M, keys along K) as an MN-major operand of dQ'
+#pragma unroll
+                        for (int q4 = 0; q4 < 4; ++q4) {
+                            const int cc = 4 * cw + q4;
+                            *reinterpret_cast<uint4*>(base + ((cc ^ (r & 7)) << 4)) =
+                                make_uint4(wd[4 * q4], wd[4 * q4 + 1], wd[4 * q4 + 2], wd[4 * q4 + 3]);
+                        }
                     }
+                    tmem_wait_st();
+                    fence_proxy_async_smem();
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&bars->p_full[b]);
                 }
-                if (!ok) break;
-                tmem_wait_st();
-                fence_proxy_async_smem();
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&bars->p_full);
-                started = true;
+                ++j;
             }
         }
     } else {
@@ -498,22 +538,22 @@ __global__ void __launch_bounds__(kThreads, 1)
         float* dqst = reinterpret_cast<float*>(smem + kDQStOff);
         float* dkst = reinterpret_cast<float*>(smem + kDKStOff);
         uint8_t* dvst = smem + kDVStOff;
-        uint32_t dqph = 0, dkvph = 0;
+        uint32_t dkvph = 0;
         long long j = 0;
         bool ok = true;
         for (long long item = blockIdx.x; item < prm.items && ok; item += gridDim.x) {
             const Item I = item_of(g, item);
             for (int n = 0; n < I.nq; ++n) {
                 if (!q_active(g, I, n)) continue;
-                if (!mbar_wait(&bars->dq_full, dqph, ctl, 0x1501)) { ok = false; break; }
-                dqph ^= 1;
+                const uint32_t c = static_cast<uint32_t>(j & 1);  // the step's dQ' accumulator
+                if (!mbar_wait(&bars->dq_full[c], (j >> 1) & 1, ctl, 0x1501)) { ok = false; break; }
                 tc_fence_after();
                 uint32_t v[32];
-                tmem_ld32(tmem + lane_off + kColDQ, v);
+                tmem_ld32(tmem + lane_off + kColDQ + 32 * c, v);
                 tmem_wait_ld();
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&bars->dq_free);
+                if (lane == 0) mbar_arrive(&bars->dq_free[c]);
                 float* buf = dqst + (j & 1) * kTile * kHeadDim;
                 if (leader) bulk_wait_read_but1();
                 named_bar_sync(1, 128);
