@@ -344,44 +344,45 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (s.first && !mbar_wait(&bars->kv_full[s.ks], (s.it >> 1) & 1, ctl, 0x1302)) return false;
                 return mbar_wait(&bars->q_full[s.st], s.qph, ctl, 0x1303);
             };
+            // Shared-memory descriptors built once per layout; per MMA only an offset
+            // in 16-byte units is added to the start-address field (14 bits: every
+            // offset of this kernel stays below 256 KiB).
+            const uint32_t sbase = smem_u32(smem);
+            const uint64_t dK0 = make_sdesc(sbase, 16, 512, kSw64);       // K-major, 64-byte rows
+            const uint64_t dMN0 = make_sdesc(sbase, 8192, 512, kSw64);    // MN-major, 64-byte rows
+            const uint64_t dDS0 = make_sdesc(sbase, 16384, 1024, kSw128); // dS, MN-major, 128-byte rows
+            auto u16 = [](uint32_t bytes) { return static_cast<uint64_t>(bytes >> 4); };
             // S^T_h = K' Q'_h^T and dP^T_h = V dO_h^T into buffer b
             auto issue_sdp = [&](const Step& s, int h, uint32_t b) {
-                const uint32_t ka = smem_u32(smem + kKVOff + s.ks * 2 * kTileBytes), va = ka + kTileBytes;
-                const uint32_t qa = smem_u32(smem + kQOff + s.st * kQStageBytes) + 4096u * h;  // rows 64h..
-                const uint32_t da = qa + kTileBytes;
+                const uint64_t ko = u16(kKVOff + s.ks * 2 * kTileBytes), vo = ko + u16(kTileBytes);
+                const uint64_t qo = u16(kQOff + s.st * kQStageBytes + 4096u * h), dof = qo + u16(kTileBytes);
                 const uint32_t t_b = tmem + col_buf(b);
 #pragma unroll
-                for (int k = 0; k < kHeadDim / 16; ++k)
-                    umma_ss(t_b, make_sdesc(ka + 32 * k, 16, 512, kSw64), make_sdesc(qa + 32 * k, 16, 512, kSw64), id_s,
-                            k > 0);
+                for (int k = 0; k < kHeadDim / 16; ++k) umma_ss(t_b, dK0 + ko + 2 * k, dK0 + qo + 2 * k, id_s, k > 0);
 #pragma unroll
                 for (int k = 0; k < kHeadDim / 16; ++k)
-                    umma_ss(t_b + 64, make_sdesc(va + 32 * k, 16, 512, kSw64), make_sdesc(da + 32 * k, 16, 512, kSw64),
-                            id_dp, k > 0);
+                    umma_ss(t_b + 64, dK0 + vo + 2 * k, dK0 + dof + 2 * k, id_dp, k > 0);
                 umma_commit(&bars->s_full[b]);
             };
             // dV += P^T_h dO_h, dK' += dS^T_h Q'_h (the item's first half-step starts them)
             auto issue_grads = [&](const Step& s, int h, uint32_t b) {
-                const uint32_t qa = smem_u32(smem + kQOff + s.st * kQStageBytes), da = qa + kTileBytes;
+                const uint64_t qo = u16(kQOff + s.st * kQStageBytes + 4096u * h), dof = qo + u16(kTileBytes);
                 const uint32_t t_p = tmem + col_pb(b);
-                const bool acc = !(s.first && h == 0);
+                const uint32_t acc = (s.first && h == 0) ? 0u : 1u;
 #pragma unroll
                 for (int k = 0; k < 4; ++k)
-                    umma_ts(tmem + kColDV, t_p + 8 * k, make_sdesc(da + 1024 * (4 * h + k), 8192, 512, kSw64), id_dv,
-                            (acc || k > 0) ? 1u : 0u);
+                    umma_ts(tmem + kColDV, t_p + 8 * k, dMN0 + dof + 64 * k, id_dv, k > 0 ? 1u : acc);
 #pragma unroll
                 for (int k = 0; k < 4; ++k)
-                    umma_ts(tmem + kColDK, t_p + 32 + 8 * k, make_sdesc(qa + 1024 * (4 * h + k), 8192, 512, kSw64),
-                            id_dk, (acc || k > 0) ? 1u : 0u);
+                    umma_ts(tmem + kColDK, t_p + 32 + 8 * k, dMN0 + qo + 64 * k, id_dk, k > 0 ? 1u : acc);
             };
             // dQ' = dS K' of a step into accumulator c
             auto issue_dq = [&](const Step& s, uint32_t c) {
-                const uint32_t ka = smem_u32(smem + kKVOff + s.ks * 2 * kTileBytes);
-                const uint32_t dsa = smem_u32(smem + kDSOff + c * kDSBytes);
+                const uint64_t ko = u16(kKVOff + s.ks * 2 * kTileBytes);
+                const uint64_t so = u16(kDSOff + c * kDSBytes);
 #pragma unroll
                 for (int k = 0; k < kTile / 16; ++k)
-                    umma_ss(tmem + kColDQ + 32 * c, make_sdesc(dsa + 2048 * k, 16384, 1024, kSw128),
-                            make_sdesc(ka + 1024 * k, 8192, 512, kSw64), id_dq, k > 0);
+                    umma_ss(tmem + kColDQ + 32 * c, dDS0 + so + 128 * k, dMN0 + ko + 64 * k, id_dq, k > 0);
                 umma_commit(&bars->dq_full[c]);
             };
             bool ok = true;

@@ -21,6 +21,5 @@ static __device__ __noinline__ uint64_t d_tile_segs(const Geo& g, long long tile
 static __device__ __noinline__ uint32_t d_allow16(const Geo& g, uint32_t my, long long tile, const Win& w) {
     return allow16(g, my, tile_segs(g, tile, w));
 }
-static __device__ __noinline__ Slot d_slot_of(const Geo& g, long long tile, int p) { return slot_of(g, tile, p); }
 
 }  // namespace fswin
