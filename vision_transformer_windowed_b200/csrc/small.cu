@@ -134,37 +134,35 @@ __global__ void __launch_bounds__(kThreads, 2) small_kernel(const __grid_constan
             const uint32_t id_dv = make_idesc(kTile, kHeadDim, false, true, false); // P^T (TMEM) x dO
             const uint32_t id_dk = make_idesc(kTile, kHeadDim, false, true, true);  // dS^T (TMEM) x Q'
             const uint32_t id_dq = make_idesc(kTile, kHeadDim, true, true, true);   // dS (smem) x K'
-            const uint32_t ds_addr = smem_u32(smem + kDSOff);
+            // descriptors built once; per MMA only an offset in 16-byte units is added
+            const uint32_t sbase = smem_u32(smem);
+            const uint64_t dK0 = make_sdesc(sbase, 16, 512, kSw64);        // K-major, 64-byte rows
+            const uint64_t dMN0 = make_sdesc(sbase, 8192, 512, kSw64);     // MN-major, 64-byte rows
+            const uint64_t dDS = make_sdesc(sbase + kDSOff, 16384, 1024, kSw128);
             for (long long j = 0; j < n; ++j) {
                 const uint32_t ph = static_cast<uint32_t>(j & 1);
                 if (!mbar_wait(&bars->in_ready, ph, ctl, 0x2201)) break;
                 if (j > 0 && !mbar_wait(&bars->tmem_free, ph ^ 1, ctl, 0x2202)) break;
                 tc_fence_after();
-                const uint32_t qa = smem_u32(smem + kSlotOff + (j & 1) * kSlotBytes);
-                const uint32_t ka = qa + kTileBytes, va = qa + 2 * kTileBytes, da = qa + 3 * kTileBytes;
+                const uint64_t qo = static_cast<uint64_t>((kSlotOff + (j & 1) * kSlotBytes) >> 4);
+                const uint64_t ko = qo + (kTileBytes >> 4), vo = qo + (2 * kTileBytes >> 4), dof = qo + (3 * kTileBytes >> 4);
+#pragma unroll
+                for (int k = 0; k < kHeadDim / 16; ++k) umma_ss(tmem + kColS, dK0 + ko + 2 * k, dK0 + qo + 2 * k, id_s, k > 0);
 #pragma unroll
                 for (int k = 0; k < kHeadDim / 16; ++k)
-                    umma_ss(tmem + kColS, make_sdesc(ka + 32 * k, 16, 512, kSw64),
-                            make_sdesc(qa + 32 * k, 16, 512, kSw64), id_s, k > 0);
-#pragma unroll
-                for (int k = 0; k < kHeadDim / 16; ++k)
-                    umma_ss(tmem + kColDP, make_sdesc(va + 32 * k, 16, 512, kSw64),
-                            make_sdesc(da + 32 * k, 16, 512, kSw64), id_dp, k > 0);
+                    umma_ss(tmem + kColDP, dK0 + vo + 2 * k, dK0 + dof + 2 * k, id_dp, k > 0);
                 umma_commit(&bars->s_full);
                 if (!mbar_wait(&bars->p_ready, ph, ctl, 0x2203)) break;
                 tc_fence_after();
 #pragma unroll
                 for (int k = 0; k < kTile / 16; ++k)
-                    umma_ts(tmem + kColDV, tmem + kColP + 8 * k, make_sdesc(da + 1024 * k, 8192, 512, kSw64), id_dv,
-                            k > 0);
+                    umma_ts(tmem + kColDV, tmem + kColP + 8 * k, dMN0 + dof + 64 * k, id_dv, k > 0);
 #pragma unroll
                 for (int k = 0; k < kTile / 16; ++k)
-                    umma_ts(tmem + kColDK, tmem + kColDS + 8 * k, make_sdesc(qa + 1024 * k, 8192, 512, kSw64), id_dk,
-                            k > 0);
+                    umma_ts(tmem + kColDK, tmem + kColDS + 8 * k, dMN0 + qo + 64 * k, id_dk, k > 0);
 #pragma unroll
                 for (int k = 0; k < kTile / 16; ++k)
-                    umma_ss(tmem + kColDQ, make_sdesc(ds_addr + 2048 * k, 16384, 1024, kSw128),
-                            make_sdesc(ka + 1024 * k, 8192, 512, kSw64), id_dq, k > 0);
+                    umma_ss(tmem + kColDQ, dDS + 128 * k, dMN0 + ko + 64 * k, id_dq, k > 0);
                 umma_commit(&bars->mma2_done);
             }
             umma_commit(&bars->done);
@@ -532,24 +530,24 @@ __global__ void __launch_bounds__(kThreads, 4) fwd_kernel(const __grid_constant_
         if (lane == 0) {
             const uint32_t id_s = make_idesc(kTile, kTile, false, false, true);  // fp16 Q', K'
             const uint32_t id_pv = make_idesc_bf16(kTile, kHeadDim, false, true);  // P (TMEM) x V
+            // descriptors built once; per MMA only an offset in 16-byte units is added
+            const uint32_t sbase = smem_u32(smem);
+            const uint64_t dK0 = make_sdesc(sbase, 16, 512, kSw64);     // K-major, 64-byte rows
+            const uint64_t dMN0 = make_sdesc(sbase, 8192, 512, kSw64);  // MN-major, 64-byte rows
             for (long long j = 0; j < n; ++j) {
                 const uint32_t ph = static_cast<uint32_t>(j & 1);
                 if (!mbar_wait(&bars->in_ready, ph, ctl, 0x3201)) break;
                 if (j > 0 && !mbar_wait(&bars->tmem_free, ph ^ 1, ctl, 0x3202)) break;
                 tc_fence_after();
-                const uint32_t qa = smem_u32(smem + kSlotOff + (j & 1) * kSlotBytes);
-                const uint32_t ka = qa + kTileBytes, va = qa + 2 * kTileBytes;
+                const uint64_t qo = static_cast<uint64_t>((kSlotOff + (j & 1) * kSlotBytes) >> 4);
+                const uint64_t ko = qo + (kTileBytes >> 4), vo = qo + (2 * kTileBytes >> 4);
 #pragma unroll
-                for (int k = 0; k < kHeadDim / 16; ++k)
-                    umma_ss(tmem + kColS, make_sdesc(qa + 32 * k, 16, 512, kSw64),
-                            make_sdesc(ka + 32 * k, 16, 512, kSw64), id_s, k > 0);
+                for (int k = 0; k < kHeadDim / 16; ++k) umma_ss(tmem + kColS, dK0 + qo + 2 * k, dK0 + ko + 2 * k, id_s, k > 0);
                 umma_commit(&bars->s_full);
                 if (!mbar_wait(&bars->p_ready, ph, ctl, 0x3203)) break;
                 tc_fence_after();
 #pragma unroll
-                for (int k = 0; k < kTile / 16; ++k)
-                    umma_ts(tmem + kColO, tmem + kColP + 8 * k, make_sdesc(va + 1024 * k, 8192, 512, kSw64), id_pv,
-                            k > 0);
+                for (int k = 0; k < kTile / 16; ++k) umma_ts(tmem + kColO, tmem + kColP + 8 * k, dMN0 + vo + 64 * k, id_pv, k > 0);
                 umma_commit(&bars->o_full);
             }
             umma_commit(&bars->done);
