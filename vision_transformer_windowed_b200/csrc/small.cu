@@ -123,8 +123,12 @@ __global__ void __launch_bounds__(kThreads, 2) small_kernel(const __grid_constan
     const uint32_t tmem = bars->tmem_base;
     const Ctl ctl{prm.status, &bars->abort_flag, prm.limit_ns};
     // this CTA's items: blockIdx.x + j * gridDim.x, j < n
-    const long long n = prm.items > blockIdx.x ? (prm.items - 1 - blockIdx.x) / gridDim.x + 1 : 0;
-    auto item_at = [&](long long j) { return static_cast<long long>(blockIdx.x) + j * gridDim.x; };
+    // this CTA's items: a contiguous run, so that consecutive items are the
+    // heads of one tile (heads innermost) and share the tile's geometry
+    const long long per = (prm.items + gridDim.x - 1) / gridDim.x;
+    const long long first = static_cast<long long>(blockIdx.x) * per;
+    const long long n = prm.items > first ? (prm.items - first < per ? prm.items - first : per) : 0;
+    auto item_at = [&](long long j) { return first + j; };
 
     if (warp == kWarpMma) {
         // ------------------------------------------------------------ MMA issue
@@ -199,15 +203,31 @@ __global__ void __launch_bounds__(kThreads, 2) small_kernel(const __grid_constan
             int h, pi, pj;
             bool valid;
         };
+        // geometry of this row in the last tile seen (shared by the tile's heads)
+        long long geo_X = -1, geo_tok0 = 0;
+        int geo_pi = 0, geo_pj = 0;
+        bool geo_valid = false;
+        uint32_t geo_a16 = 0;
+        auto geo_for = [&](long long X) {
+            if (X == geo_X) return;
+            geo_X = X;
+            geo_valid = slot_token(g, X, r, 0, &geo_pi, &geo_pj, &geo_tok0);  // token of head 0
+            const uint64_t segs = d_tile_segs(g, X, d_tile_win(g, X));
+            geo_a16 = allow16(g, seg_at(segs, r >> g.lBT), segs);  // bit c: columns [16c, 16c+16)
+        };
         auto row_tok = [&](long long j) {
             RowTok t;
             small_item(g, prm.head_minor, item_at(j), &t.X, &t.h);
-            t.valid = slot_token(g, t.X, r, t.h, &t.pi, &t.pj, &t.tok);
+            geo_for(t.X);
+            t.valid = geo_valid;
+            t.tok = geo_tok0 + t.h;  // heads are innermost in the token layout
+            t.pi = geo_pi;
+            t.pj = geo_pj;
             return t;
         };
         auto row_mask = [&](const RowTok& t) {
-            const uint64_t segs = d_tile_segs(g, t.X, d_tile_win(g, t.X));
-            return allow16(g, seg_at(segs, r >> g.lBT), segs);  // bit c: columns [16c, 16c+16)
+            geo_for(t.X);
+            return geo_a16;
         };
         // Copies of the warp's 32 token rows, coalesced: each instruction moves
         // 8 whole 64-byte rows (lane = row 8i + lane/4, 16-byte chunk lane%4).
@@ -522,8 +542,12 @@ __global__ void __launch_bounds__(kThreads, 4) fwd_kernel(const __grid_constant_
     tc_fence_after();
     const uint32_t tmem = bars->tmem_base;
     const Ctl ctl{prm.status, &bars->abort_flag, prm.limit_ns};
-    const long long n = prm.items > blockIdx.x ? (prm.items - 1 - blockIdx.x) / gridDim.x + 1 : 0;
-    auto item_at = [&](long long j) { return static_cast<long long>(blockIdx.x) + j * gridDim.x; };
+    // this CTA's items: a contiguous run, so that consecutive items are the
+    // heads of one tile (heads innermost) and share the tile's geometry
+    const long long per = (prm.items + gridDim.x - 1) / gridDim.x;
+    const long long first = static_cast<long long>(blockIdx.x) * per;
+    const long long n = prm.items > first ? (prm.items - first < per ? prm.items - first : per) : 0;
+    auto item_at = [&](long long j) { return first + j; };
 
     if (warp == kWarpMma) {
         // ------------------------------------------------------------ MMA issue
@@ -577,15 +601,31 @@ __global__ void __launch_bounds__(kThreads, 4) fwd_kernel(const __grid_constant_
             int h, pi, pj;
             bool valid;
         };
+        // geometry of this row in the last tile seen (shared by the tile's heads)
+        long long geo_X = -1, geo_tok0 = 0;
+        int geo_pi = 0, geo_pj = 0;
+        bool geo_valid = false;
+        uint32_t geo_a16 = 0;
+        auto geo_for = [&](long long X) {
+            if (X == geo_X) return;
+            geo_X = X;
+            geo_valid = slot_token(g, X, r, 0, &geo_pi, &geo_pj, &geo_tok0);  // token of head 0
+            const uint64_t segs = d_tile_segs(g, X, d_tile_win(g, X));
+            geo_a16 = allow16(g, seg_at(segs, r >> g.lBT), segs);  // bit c: columns [16c, 16c+16)
+        };
         auto row_tok = [&](long long j) {
             RowTok t;
             small_item(g, prm.head_minor, item_at(j), &t.X, &t.h);
-            t.valid = slot_token(g, t.X, r, t.h, &t.pi, &t.pj, &t.tok);
+            geo_for(t.X);
+            t.valid = geo_valid;
+            t.tok = geo_tok0 + t.h;  // heads are innermost in the token layout
+            t.pi = geo_pi;
+            t.pj = geo_pj;
             return t;
         };
         auto row_mask = [&](const RowTok& t) {
-            const uint64_t segs = d_tile_segs(g, t.X, d_tile_win(g, t.X));
-            return allow16(g, seg_at(segs, r >> g.lBT), segs);  // bit c: columns [16c, 16c+16)
+            geo_for(t.X);
+            return geo_a16;
         };
         // coalesced copies of the warp's 32 rows of q, k, v (8 rows per instruction)
         auto copy_slot = [&](long long j, const RowTok& t) {
