@@ -62,8 +62,9 @@ __device__ __forceinline__ void rope32_small(float (&x)[32], int i, int j, const
             const float2 cs = tab[(ax * 8 + k) * 8 + pos];
             const float sn = inv ? -cs.y : cs.y;
             const float a = x[ax * 16 + 2 * k], b = x[ax * 16 + 2 * k + 1];
-            x[ax * 16 + 2 * k] = a * cs.x - b * sn;
-            x[ax * 16 + 2 * k + 1] = a * sn + b * cs.x;
+            float t0, t1;
+            fmul2(t0, t1, a, b, cs.x, cs.x);  // (a cos, b cos), then + (-b sin, a sin)
+            ffma2(x[ax * 16 + 2 * k], x[ax * 16 + 2 * k + 1], -b, a, sn, sn, t0, t1);
         }
     }
 }

@@ -294,8 +294,13 @@ __global__ void __launch_bounds__(kThreads, 2) small_kernel(const __grid_constan
                 float a[32], b[32];
                 load_row_swz(smem + kOOff, r, a, false);
                 load_row_swz(sl + 3 * kTileBytes, r, b, false);
+                float d4[4] = {0.f, 0.f, 0.f, 0.f};  // four independent partial sums
 #pragma unroll
-                for (int e = 0; e < 32; ++e) D = fmaf(a[e], b[e], D);
+                for (int e = 0; e < 32; e += 4) {
+                    ffma2(d4[0], d4[1], a[e], a[e + 1], b[e], b[e + 1], d4[0], d4[1]);
+                    ffma2(d4[2], d4[3], a[e + 2], a[e + 3], b[e + 2], b[e + 3], d4[2], d4[3]);
+                }
+                D = (d4[0] + d4[1]) + (d4[2] + d4[3]);
             }
             __syncwarp();  // every lane has read its o row
             RowTok nxt{};
@@ -392,7 +397,8 @@ __global__ void __launch_bounds__(kThreads, 2) small_kernel(const __grid_constan
                 tmem_wait_ld();
                 float dx[32], x[32];
 #pragma unroll
-                for (int e = 0; e < 32; ++e) dx[e] = __uint_as_float(t[e]) * prm.scale;
+                for (int e = 0; e < 32; e += 2)
+                    fmul2(dx[e], dx[e + 1], __uint_as_float(t[e]), __uint_as_float(t[e + 1]), prm.scale, prm.scale);
                 uint8_t* tile = sl + which * kTileBytes;
                 load_row_swz(tile, r, x, true);  // rotated q' or k' (fp16)
                 // d theta: the pair's cross product is the same before and after the rotation
