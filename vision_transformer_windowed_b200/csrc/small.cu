@@ -59,8 +59,8 @@ __device__ __forceinline__ void small_item(const Geo& g, bool head_minor, long l
 // are adjacent in memory, are read close together in time.
 namespace bwd {
 
-constexpr int kThreads = 160;
-constexpr int kWarpMma = 4;
+constexpr int kThreads = 192;
+constexpr int kWarpMma = 4, kWarpMover = 5;
 constexpr int kSlotBytes = 4 * kTileBytes;        // q, k, v, dO tiles of one item
 constexpr int kSlotOff = 0;                        // 2 slots
 constexpr int kOOff = 2 * kSlotBytes;              // o tile
@@ -77,6 +77,7 @@ constexpr uint32_t kColDV = 64, kColDQ = 96, kColDK = 192;
 
 struct Bars {
     uint64_t in_ready, s_full, p_ready, mma2_done, tmem_free, grp, done;
+    uint64_t slot_full[2], o_full, o_free, staged;  // row copies and stores (mover warp)
     uint32_t tmem_base;
     int abort_flag;
 };
@@ -110,6 +111,11 @@ __global__ void __launch_bounds__(kThreads, 2) small_kernel(const __grid_constan
         mbar_init(&bars->tmem_free, 4);
         mbar_init(&bars->grp, 4);
         mbar_init(&bars->done, 1);
+        mbar_init(&bars->slot_full[0], 32);  // one cp.async arrival per mover lane
+        mbar_init(&bars->slot_full[1], 32);
+        mbar_init(&bars->o_full, 32);
+        mbar_init(&bars->o_free, 4);
+        mbar_init(&bars->staged, 4);
         bars->abort_flag = 0;
         fence_mbar_init();
     }
@@ -173,6 +179,92 @@ __global__ void __launch_bounds__(kThreads, 2) small_kernel(const __grid_constan
             mbar_wait(&bars->done, 0, ctl, 0x22ff);
         }
         __syncwarp();
+    } else if (warp == kWarpMover) {
+        // ------------------------------------------------------------ row copies and result stores
+        // Lane l moves 16-byte chunk l % 4 of row 8 i + l / 4 of each group of 32
+        // rows: every instruction moves 8 whole 64-byte rows.  Copies arrive on an
+        // mbarrier when they land (one arrival per lane); padding rows are zero
+        // filled on load and skipped on store.
+        bool ok = true;
+        auto mwait = [&](uint64_t* bar, uint32_t ph, unsigned int where) -> bool {
+            return __all_sync(0xFFFFFFFFu, mbar_wait(bar, ph, ctl, where));
+        };
+        // token (head 0) of rows lane + 32 q of the last tile seen
+        long long mv_X = -1, mv_tok0[4] = {0, 0, 0, 0};
+        bool mv_valid[4] = {false, false, false, false};
+        auto geo4 = [&](long long j, int* h) {
+            long long X;
+            small_item(g, prm.head_minor, item_at(j), &X, h);
+            if (X == mv_X) return;
+            mv_X = X;
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                int pi, pj;
+                mv_valid[q] = slot_token(g, X, lane + 32 * q, 0, &pi, &pj, &mv_tok0[q]);
+            }
+        };
+        // load (into the tiles) or store (from them) the rows of item j
+        auto move = [&](long long j, const uint8_t* const* gsrc, uint8_t* const* gdst, uint8_t* const* tiles, int nt,
+                        bool load) {
+            int h;
+            geo4(j, &h);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const int sl_lane = 8 * i + (lane >> 2), c = lane & 3;
+                    const long long tok = __shfl_sync(0xFFFFFFFFu, mv_tok0[q] + h, sl_lane);
+                    const bool valid = __shfl_sync(0xFFFFFFFFu, mv_valid[q] ? 1 : 0, sl_lane) != 0;
+                    const int row = 32 * q + sl_lane;
+                    const uint32_t off = row * kRowBytes + ((c ^ ((row >> 1) & 3)) << 4);
+                    const long long go = tok * kRowBytes + 16 * c;
+                    for (int x = 0; x < nt; ++x) {
+                        if (load)
+                            cp_async16(smem_u32(tiles[x] + off), valid ? gsrc[x] + go : gsrc[x], valid ? 16u : 0u);
+                        else if (valid)
+                            *reinterpret_cast<uint4*>(gdst[x] + go) = *reinterpret_cast<const uint4*>(tiles[x] + off);
+                    }
+                }
+            }
+        };
+        const uint8_t* qkvd[4] = {prm.q, prm.k, prm.v, prm.dout};
+        const uint8_t* osrc[1] = {prm.o};
+        uint8_t* grads[3] = {prm.dq, prm.dk, prm.dv};
+        uint8_t* otile[1] = {smem + kOOff};
+        auto slot_tiles = [&](long long j, uint8_t** t) {
+            uint8_t* sl = smem + kSlotOff + (j & 1) * kSlotBytes;
+            for (int x = 0; x < 4; ++x) t[x] = sl + x * kTileBytes;
+        };
+        uint8_t* st[4];
+        if (n > 0) {
+            slot_tiles(0, st);
+            move(0, qkvd, nullptr, st, 4, true);
+            cp_async_mbar_arrive(&bars->slot_full[0]);
+            move(0, osrc, nullptr, otile, 1, true);
+            cp_async_mbar_arrive(&bars->o_full);
+        }
+        if (n > 1) {
+            slot_tiles(1, st);
+            move(1, qkvd, nullptr, st, 4, true);
+            cp_async_mbar_arrive(&bars->slot_full[1]);
+        }
+        for (long long j = 0; j < n && ok; ++j) {
+            const uint32_t ph = static_cast<uint32_t>(j & 1);
+            if (j + 1 < n) {  // the next item's o rows once the rows have read this item's
+                if (!mwait(&bars->o_free, ph, 0x2401)) break;
+                move(j + 1, osrc, nullptr, otile, 1, true);
+                cp_async_mbar_arrive(&bars->o_full);
+            }
+            if (!mwait(&bars->staged, ph, 0x2402)) break;  // dq, dk, dv staged over the slot's q, k, v
+            slot_tiles(j, st);
+            move(j, nullptr, grads, st, 3, false);
+            __syncwarp();  // every lane has read the staged rows: the slot takes item j+2's rows
+            if (j + 2 < n) {
+                move(j + 2, qkvd, nullptr, st, 4, true);
+                cp_async_mbar_arrive(&bars->slot_full[j & 1]);
+            }
+        }
+        cp_async_wait<0>();
     } else {
         // ------------------------------------------------------------ rows (warps 0-3)
         const int r = tid;
@@ -229,43 +321,7 @@ __global__ void __launch_bounds__(kThreads, 2) small_kernel(const __grid_constan
             geo_for(t.X);
             return geo_a16;
         };
-        // Copies of the warp's 32 token rows, coalesced: each instruction moves
-        // 8 whole 64-byte rows (lane = row 8i + lane/4, 16-byte chunk lane%4).
-        // Padding rows are zero filled.
-        auto copy_rows = [&](const RowTok& t, const uint8_t* const* src, uint8_t* const* tile, int ntensors) {
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const int sl_lane = 8 * i + (lane >> 2), c = lane & 3;
-                const long long tok = __shfl_sync(0xFFFFFFFFu, t.tok, sl_lane);
-                const bool valid = __shfl_sync(0xFFFFFFFFu, t.valid ? 1 : 0, sl_lane) != 0;
-                const int row = warp * 32 + sl_lane;
-                const uint32_t off = row * kRowBytes + ((c ^ ((row >> 1) & 3)) << 4);
-                for (int x = 0; x < ntensors; ++x)
-                    cp_async16(smem_u32(tile[x] + off), valid ? src[x] + tok * kRowBytes + 16 * c : src[x],
-                               valid ? 16u : 0u);
-            }
-        };
-        auto copy_slot = [&](long long j, const RowTok& t) {
-            uint8_t* sl = smem + kSlotOff + (j & 1) * kSlotBytes;
-            const uint8_t* src[4] = {prm.q, prm.k, prm.v, prm.dout};
-            uint8_t* dst[4] = {sl, sl + kTileBytes, sl + 2 * kTileBytes, sl + 3 * kTileBytes};
-            copy_rows(t, src, dst, 4);
-        };
-        auto copy_o = [&](const RowTok& t) {
-            const uint8_t* src[1] = {prm.o};
-            uint8_t* dst[1] = {smem + kOOff};
-            copy_rows(t, src, dst, 1);
-        };
-        // Commit groups: at the start of item j the newest group holds item
-        // j+1's q, k, v, dO and everything older (item j's slot, o) is waited for.
         RowTok cur = n > 0 ? row_tok(0) : RowTok{};
-        if (n > 0) {
-            copy_slot(0, cur);
-            copy_o(cur);
-        }
-        cp_async_commit();
-        if (n > 1) copy_slot(1, row_tok(1));
-        cp_async_commit();
         int tab_head = -1;
         if (prm.head_minor) {  // every head's table, once
             for (int hh = 0; hh < g.heads; ++hh)
@@ -286,8 +342,9 @@ __global__ void __launch_bounds__(kThreads, 2) small_kernel(const __grid_constan
                 tab_head = cur.h;
             }
             uint8_t* sl = smem + kSlotOff + (j & 1) * kSlotBytes;
-            cp_async_wait<1>();
-            __syncwarp();  // rows copied by other lanes of the warp
+            if (!wwait(&bars->slot_full[j & 1], static_cast<uint32_t>((j >> 1) & 1), 0x2304) ||
+                !wwait(&bars->o_full, ph, 0x2305))
+                break;
             // D = dO . O of this row's token; then the next item's o rows
             float D = 0.f;
             {
@@ -302,13 +359,9 @@ __global__ void __launch_bounds__(kThreads, 2) small_kernel(const __grid_constan
                 }
                 D = (d4[0] + d4[1]) + (d4[2] + d4[3]);
             }
-            __syncwarp();  // every lane has read its o row
-            RowTok nxt{};
-            if (j + 1 < n) {
-                nxt = row_tok(j + 1);
-                copy_o(nxt);
-            }
-            cp_async_commit();
+            __syncwarp();  // every lane has read its o row: the mover may load the next item's
+            if (lane == 0) mbar_arrive(&bars->o_free);
+            const RowTok nxt = j + 1 < n ? row_tok(j + 1) : RowTok{};
             lse2v[r] = cur.valid ? lse_cur * 1.4426950408889634f : INFINITY;  // padding: no probability
             dvec[r] = D;
             // RoPE of this row's q and k, bf16 in, fp16 out, in place
@@ -427,24 +480,7 @@ __global__ void __launch_bounds__(kThreads, 2) small_kernel(const __grid_constan
                 store_row_swz(sl + 2 * kTileBytes, r, x);  // dv, staged over v
             }
             __syncwarp();
-            // coalesced stores of the warp's 32 rows of dq, dk, dv (8 rows per instruction)
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const int sl_lane = 8 * i + (lane >> 2), c = lane & 3;
-                const long long tok = __shfl_sync(0xFFFFFFFFu, cur.tok, sl_lane);
-                const bool valid = __shfl_sync(0xFFFFFFFFu, cur.valid ? 1 : 0, sl_lane) != 0;
-                const int row = warp * 32 + sl_lane;
-                const uint32_t off = row * kRowBytes + ((c ^ ((row >> 1) & 3)) << 4);
-                if (valid) {
-                    const long long go = tok * kRowBytes + 16 * c;
-                    *reinterpret_cast<uint4*>(prm.dq + go) = *reinterpret_cast<const uint4*>(sl + off);
-                    *reinterpret_cast<uint4*>(prm.dk + go) = *reinterpret_cast<const uint4*>(sl + kTileBytes + off);
-                    *reinterpret_cast<uint4*>(prm.dv + go) = *reinterpret_cast<const uint4*>(sl + 2 * kTileBytes + off);
-                }
-            }
-            __syncwarp();  // the staged rows are read: the slot takes item j+2's rows
-            if (j + 2 < n) copy_slot(j + 2, row_tok(j + 2));
-            cp_async_commit();
+            if (lane == 0) mbar_arrive(&bars->staged);  // the mover stores them
             // this warp's 16 d theta partials of the tile (summed in a fixed order
             // later): a butterfly that halves the values at each step, so that
             // lane pair (2c, 2c+1) ends with the warp sum of component c
@@ -471,7 +507,6 @@ __global__ void __launch_bounds__(kThreads, 2) small_kernel(const __grid_constan
             lse_cur = lse_nxt;
             a16 = a16_nxt;
         }
-        cp_async_wait<0>();
     }
 
     tc_fence_before();
