@@ -337,11 +337,13 @@ def main():
     pairs_per_launch = (main_res["fwd_flops"] / (4.0 * HEAD_DIM)) / nshift
     # bytes each kernel must move per token-head row: windows inside one tile run the whole
     # backward as one kernel (Q, K, V, O, dO read, dQ, dK, dV written, LSE and D: 520 B);
-    # larger windows run prep / main / post with workspace round trips
+    # larger windows run prep / main / post with workspace round trips (prep: q, k, o, dO, lse in,
+    # q', k' images, lse2, D and the zeroed dQ' accumulator out; main: the images, dO, v, lse2, D in,
+    # dk, dv out; post: the dQ' accumulator and q in, dq out)
     if M * M < 128:
         algo_bytes = {"fwd": 260, "bwd_prep": 0, "bwd_main": 520, "bwd_post": 0, "bwd_dtheta": 0}
     else:
-        algo_bytes = {"fwd": 260, "bwd_prep": 588, "bwd_main": 456, "bwd_post": 512, "bwd_dtheta": 0}
+        algo_bytes = {"fwd": 260, "bwd_prep": 524, "bwd_main": 392, "bwd_post": 256, "bwd_dtheta": 0}
     hbm_bound = M <= 8
     if hbm_bound or dom in ("bwd_prep", "bwd_post", "bwd_dtheta"):
         achieved = algo_bytes[dom] * th / (ph[dom] * 1e-3) / 1e9

@@ -3,16 +3,18 @@
 // Recompute-based (the probabilities are rebuilt from the forward's
 // log-sum-exp, never stored), in four launches on the caller's stream:
 //   1. prep:   per token row, rotate q and k (RoPE) into swizzled fp16 tile
-//              images, copy dO into a bf16 tile image, D = rowsum(dO * O),
-//              lse in log2 units, and zero the fp32 dQ accumulator;
+//              images, D = rowsum(dO * O), lse in log2 units, and zero the
+//              fp32 dQ accumulator;
 //   2. main:   persistent, warp-specialised tcgen05 kernel; a work item is one
 //              128-key tile, iterating over the query tiles it attends to:
 //                S^T = K' Q'^T, dP^T = V dO^T            (TMEM)
 //                P^T = exp2(S^T * c - lse2), dS^T = P^T (dP^T - D)
 //                dV += P^T dO, dK' += dS^T Q'            (TMEM accumulators)
 //                dQ' = dS K'  -> bulk reduce-add into the fp32 accumulator
-//   3. post:   per token row, undo the rotation of dQ' and dK', write dq and
-//              dk, and the per-tile partial sums of d theta;
+//              and, per item, dk (dK' un-rotated) and dv, with the key side
+//              of d theta;
+//   3. post:   per token row, undo the rotation of dQ', write dq, and the
+//              query side of d theta;
 //   4. reduce: fixed-order sum of the partials into dtheta (deterministic).
 #include <cuda.h>
 #include <cuda_runtime.h>
@@ -31,7 +33,7 @@ namespace bwdk {
 
 // ------------------------------------------------------------------ workspace
 struct WsLayout {
-    size_t qimg, kimg, doimg, lse2, dvec, dqacc, dkimg, part, part2, total;
+    size_t qimg, kimg, lse2, dvec, dqacc, part, part2, total;
 };
 
 __host__ __device__ inline size_t round256(size_t x) { return (x + 255) & ~size_t(255); }
@@ -42,12 +44,10 @@ __host__ __device__ inline WsLayout ws_layout(const Geo& g) {
     size_t o = 0;
     L.qimg = o;  o += round256(ht * kTileBytes);
     L.kimg = o;  o += round256(ht * kTileBytes);
-    L.doimg = o; o += round256(ht * kTileBytes);
     L.lse2 = o;  o += round256(ht * kTile * 4);
     L.dvec = o;  o += round256(ht * kTile * 4);
     L.dqacc = o; o += round256(ht * kTile * kHeadDim * 4);
-    L.dkimg = o; o += round256(ht * kTile * kHeadDim * 4);
-    L.part = o;  o += round256(ht * 4 * 16 * 4);  // up to 4 x 16 partials per (head, tile)
+    L.part = o;  o += round256(ht * 8 * 16 * 4);  // up to 8 x 16 partials per (head, tile)
     L.part2 = o; o += round256(static_cast<size_t>(g.heads) * 64 * 16 * 4);  // level-1 d theta sums
     L.total = o;
     return L;
@@ -63,17 +63,18 @@ struct PrepParams {
 
 struct PostParams {
     Geo g;
-    const uint4 *q, *k;
+    const uint4* q;
     const float* theta;
-    uint4 *dq, *dk;
+    uint4* dq;
     const uint8_t* ws;
     WsLayout L;
     float scale;
 };
 
-// cos/sin of pos * theta[h][ax][k] for pos < M, in shared memory: [2][64][8].
-__device__ __forceinline__ void build_table(float2* tab, const float* theta_h, int M) {
-    for (int e = threadIdx.x; e < 2 * M * 8; e += blockDim.x) {
+// cos/sin of pos * theta[h][ax][k] for pos < M, in shared memory: [2][64][8],
+// built by threads t < nt.
+__device__ __forceinline__ void build_table(float2* tab, const float* theta_h, int M, int t, int nt) {
+    for (int e = t; e < 2 * M * 8; e += nt) {
         const int ax = e / (M * 8), rem = e - ax * M * 8, pos = rem >> 3, k = rem & 7;
         float sn, cs;
         sincosf(static_cast<float>(pos) * theta_h[ax * 8 + k], &sn, &cs);
@@ -118,7 +119,7 @@ __global__ void __launch_bounds__(128) prep_kernel(const PrepParams p) {
     const long long ht = blockIdx.x;
     const int h = static_cast<int>(ht / g.tiles);
     const long long T = ht - static_cast<long long>(h) * g.tiles;
-    build_table(tab, p.theta + h * 16, g.M);
+    build_table(tab, p.theta + h * 16, g.M, threadIdx.x, blockDim.x);
     __syncthreads();
     const int r = threadIdx.x;
     const Slot sl = slot_of(g, T, r);
@@ -143,7 +144,6 @@ __global__ void __launch_bounds__(128) prep_kernel(const PrepParams p) {
     }
     store_row_swz(p.ws + p.L.qimg + ht * kTileBytes, r, q, true);
     store_row_swz(p.ws + p.L.kimg + ht * kTileBytes, r, k, true);
-    store_row_swz(p.ws + p.L.doimg + ht * kTileBytes, r, dO);
     reinterpret_cast<float*>(p.ws + p.L.lse2)[ht * kTile + r] = lse2;
     reinterpret_cast<float*>(p.ws + p.L.dvec)[ht * kTile + r] = D;
     uint4* acc = reinterpret_cast<uint4*>(p.ws + p.L.dqacc + (ht * kTile + r) * kHeadDim * 4);
@@ -175,8 +175,9 @@ constexpr int kQOff = kKVOff + 2 * 2 * kTileBytes;
 constexpr int kDSOff = kQOff + kQStages * kQStageBytes;        // 2 x dS, MN-major 128B swizzle
 constexpr int kDSBytes = 4 * kTileBytes;
 constexpr int kDQStOff = kDSOff + 2 * kDSBytes;                // 2 x fp32 [128][32]
-constexpr int kDKStOff = kDQStOff + 2 * 4 * kTile * kHeadDim;  // fp32 [128][32]
-constexpr int kDVStOff = kDKStOff + 4 * kTile * kHeadDim;      // bf16 tile
+constexpr int kDKStOff = kDQStOff + 2 * 4 * kTile * kHeadDim;  // bf16 tile
+constexpr int kTabOff = kDKStOff + kTileBytes;                  // cos / sin [2][64][8]
+constexpr int kDVStOff = kTabOff + 2 * 64 * 8 * 8;              // bf16 tile
 constexpr int kBarOff = kDVStOff + kTileBytes;
 constexpr int kSmemBytes = kBarOff + 1024 + 1024;
 static_assert(kDSOff % 1024 == 0, "128-byte swizzled operand must be 1024-byte aligned");
@@ -207,6 +208,8 @@ struct MainParams {
     Geo g;
     uint8_t* ws;
     WsLayout L;
+    const float* theta;
+    float* part;  // [heads][tiles][8][16] d theta partials
     unsigned int* status;
     unsigned long long limit_ns;
     long long items;
@@ -219,6 +222,7 @@ __device__ __forceinline__ bool q_active(const Geo& g, const Item& I, int n) { r
 
 __global__ void __launch_bounds__(kThreads, 1)
     main_kernel(const __grid_constant__ CUtensorMap map_v, const __grid_constant__ CUtensorMap map_dv,
+                const __grid_constant__ CUtensorMap map_do, const __grid_constant__ CUtensorMap map_dk,
                 const __grid_constant__ MainParams prm) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -230,7 +234,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (tid == 0) {
         for (int i = 0; i < 2; ++i) {
             mbar_init(&bars->kv_full[i], 1);
-            mbar_init(&bars->kv_empty[i], 1);
+            mbar_init(&bars->kv_empty[i], 5);  // the item's last MMAs, and each epilogue warp's read of its k' rows
             mbar_init(&bars->s_full[i], 1);
             mbar_init(&bars->p_full[i], 8);
             mbar_init(&bars->dq_full[i], 1);
@@ -261,6 +265,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // ------------------------------------------------------------ producer
         if (lane == 0) {
             prefetch_tmap(&map_v);
+            prefetch_tmap(&map_do);
             int it = 0;
             uint32_t qc = 0;
             bool ok = true;
@@ -283,7 +288,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const size_t hv = static_cast<size_t>(I.h) * tiles + static_cast<size_t>(I.q0 + n);
                     mbar_arrive_expect_tx(&bars->q_full[st], kQStageBytes);
                     bulk_load(qs, ws + prm.L.qimg + hv * kTileBytes, kTileBytes, &bars->q_full[st]);
-                    bulk_load(qs + kTileBytes, ws + prm.L.doimg + hv * kTileBytes, kTileBytes, &bars->q_full[st]);
+                    tile_tma(g, &map_do, qs + kTileBytes, &bars->q_full[st], I.q0 + n, I.h, false);
                     bulk_load(qs + 2 * kTileBytes, ws + prm.L.lse2 + hv * kTile * 4, kTile * 4, &bars->q_full[st]);
                     bulk_load(qs + 2 * kTileBytes + kTile * 4, ws + prm.L.dvec + hv * kTile * 4, kTile * 4,
                               &bars->q_full[st]);
@@ -537,12 +542,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
         const bool leader = (quarter == 0 && lane == 0);
         float* dqst = reinterpret_cast<float*>(smem + kDQStOff);
-        float* dkst = reinterpret_cast<float*>(smem + kDKStOff);
+        uint8_t* dkst = smem + kDKStOff;
         uint8_t* dvst = smem + kDVStOff;
+        float2* tab = reinterpret_cast<float2*>(smem + kTabOff);
         uint32_t dkvph = 0;
         long long j = 0;
+        int it = 0, tab_h = -1;
         bool ok = true;
-        for (long long item = blockIdx.x; item < prm.items && ok; item += gridDim.x) {
+        for (long long item = blockIdx.x; item < prm.items && ok; item += gridDim.x, ++it) {
             const Item I = item_of(g, item);
             for (int n = 0; n < I.nq; ++n) {
                 if (!q_active(g, I, n)) continue;
@@ -576,39 +583,83 @@ __global__ void __launch_bounds__(kThreads, 1)
                 ++j;
             }
             if (!ok) break;
-            // item end: dV and dK' accumulators
+            // item end: dV and dK' accumulators.  dk is un-rotated here, and the
+            // key side of d theta taken with the item's rotated k' rows, which stay
+            // in its K', V slot until every row has read them.
             if (!mbar_wait(&bars->dkv_full, dkvph, ctl, 0x1502)) break;
             dkvph ^= 1;
             tc_fence_after();
-            uint32_t vv[32], kk[32];
-            tmem_ld32(tmem + lane_off + kColDV, vv);
-            tmem_ld32(tmem + lane_off + kColDK, kk);
-            tmem_wait_ld();
-            tc_fence_before();
+            uint32_t dvp[16];  // dv, bf16 pairs
+            float dk[32];
+            {
+                uint32_t vv[32], kk[32];
+                tmem_ld32(tmem + lane_off + kColDV, vv);
+                tmem_ld32(tmem + lane_off + kColDK, kk);
+                tmem_wait_ld();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&bars->dkv_free);
+#pragma unroll
+                for (int e = 0; e < 16; ++e) dvp[e] = pack_bf16x2(__uint_as_float(vv[2 * e]), __uint_as_float(vv[2 * e + 1]));
+#pragma unroll
+                for (int e = 0; e < 32; e += 2)
+                    fmul2(dk[e], dk[e + 1], __uint_as_float(kk[e]), __uint_as_float(kk[e + 1]), prm.scale, prm.scale);
+            }
+            const int ks = it & 1;
+            if (!mbar_wait(&bars->kv_full[ks], (it >> 1) & 1, ctl, 0x1503)) break;
+            const Slot sl = slot_of(g, I.u, r);
+            float part[16];
+            {
+                // k' (fp16) pairs of this row, read one pair at a time
+                const uint8_t* krow = smem + kKVOff + ks * 2 * kTileBytes + r * kRowBytes;
+                const int sw = (r >> 1) & 3;
+#pragma unroll
+                for (int ax = 0; ax < 2; ++ax) {
+                    const float pos = sl.box.valid ? static_cast<float>(ax ? sl.i : sl.j) : 0.f;
+#pragma unroll
+                    for (int k = 0; k < 8; ++k) {  // the pair's cross product is the same in both frames
+                        const int a = ax * 16 + 2 * k, b = a + 1;
+                        const float2 kp = __half22float2(
+                            *reinterpret_cast<const __half2*>(krow + (((a >> 3) ^ sw) << 4) + (a & 7) * 2));
+                        part[ax * 8 + k] = pos * (dk[b] * kp.x - dk[a] * kp.y);
+                    }
+                }
+            }
             __syncwarp();
-            if (lane == 0) mbar_arrive(&bars->dkv_free);
+            if (lane == 0) mbar_arrive(&bars->kv_empty[ks]);
+            if (I.h != tab_h) {  // every row is past its last use of the previous table
+                build_table(tab, prm.theta + I.h * 16, g.M, r, 128);
+                named_bar_sync(1, 128);
+                tab_h = I.h;
+            }
+            rope32(dk, sl.i, sl.j, tab, true);
             if (leader) bulk_wait_read_all();
             named_bar_sync(1, 128);
+            store_row_swz(dkst, r, dk);
             {
-                float4* rowp = reinterpret_cast<float4*>(dkst + r * kHeadDim);
+                uint8_t* row = dvst + r * kRowBytes;
+                const int sw = (r >> 1) & 3;
 #pragma unroll
-                for (int c = 0; c < 8; ++c) {
-                    rowp[c ^ (r & 7)] = make_float4(__uint_as_float(kk[4 * c]) * prm.scale, __uint_as_float(kk[4 * c + 1]) * prm.scale,
-                                          __uint_as_float(kk[4 * c + 2]) * prm.scale,
-                                          __uint_as_float(kk[4 * c + 3]) * prm.scale);
-                }
-                float x[32];
-#pragma unroll
-                for (int e = 0; e < 32; ++e) x[e] = __uint_as_float(vv[e]);
-                store_row_swz(dvst, r, x);
+                for (int c = 0; c < 4; ++c)
+                    *reinterpret_cast<uint4*>(row + ((c ^ sw) << 4)) =
+                        make_uint4(dvp[4 * c], dvp[4 * c + 1], dvp[4 * c + 2], dvp[4 * c + 3]);
             }
             fence_proxy_async_smem();
             named_bar_sync(1, 128);
             if (leader) {
-                const size_t hu = static_cast<size_t>(I.h) * tiles + static_cast<size_t>(I.u);
-                bulk_store(prm.ws + prm.L.dkimg + hu * kTile * kHeadDim * 4, dkst, kTile * kHeadDim * 4);
                 tile_tma(g, &map_dv, dvst, nullptr, I.u, I.h, true);
+                tile_tma(g, &map_dk, dkst, nullptr, I.u, I.h, true);
                 bulk_commit();
+            }
+            // this warp's 16 key-side partials of the tile, group 4 + quarter
+            // (the query side, from the post kernel, takes groups 0-3)
+            float* out = prm.part + ((static_cast<long long>(I.h) * g.tiles + I.u) * 8 + 4 + quarter) * 16;
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+                float v = part[e];
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+                if (lane == e) out[e] = v;
             }
         }
         if (leader) bulk_wait_all();
@@ -621,14 +672,16 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 // ------------------------------------------------------------------ 3. post
+// dq of each token row (dQ' un-rotated) and the query side of d theta: per
+// warp, 16 partials of the tile in groups 0-3 (the main kernel's epilogue
+// writes the key side in groups 4-7).
 __global__ void __launch_bounds__(128) post_kernel(const PostParams p) {
     __shared__ float2 tab[2 * 64 * 8];
-    __shared__ float red[4][16];
     const Geo& g = p.g;
     const long long ht = blockIdx.x;
     const int h = static_cast<int>(ht / g.tiles);
     const long long T = ht - static_cast<long long>(h) * g.tiles;
-    build_table(tab, p.theta + h * 16, g.M);
+    build_table(tab, p.theta + h * 16, g.M, threadIdx.x, blockDim.x);
     __syncthreads();
     const int r = threadIdx.x, lane = r & 31, warp = r >> 5;
     const Slot sl = slot_of(g, T, r);
@@ -637,46 +690,34 @@ __global__ void __launch_bounds__(128) post_kernel(const PostParams p) {
     for (int e = 0; e < 16; ++e) part[e] = 0.f;
     if (sl.box.valid) {
         const long long tok = ((static_cast<long long>(sl.box.b) * g.H + sl.row) * g.W + sl.col) * g.heads + h;
-        float dq[32], dk[32], q[32], k[32];
+        float dq[32], q[32];
         const float4* aq = reinterpret_cast<const float4*>(p.ws + p.L.dqacc + (ht * kTile + r) * kHeadDim * 4);
-        const float4* ak = reinterpret_cast<const float4*>(p.ws + p.L.dkimg + (ht * kTile + r) * kHeadDim * 4);
 #pragma unroll
         for (int c = 0; c < 8; ++c) {
-            const float4 a = aq[c ^ (r & 7)], b = ak[c ^ (r & 7)];  // swizzled fp32 tile images
+            const float4 a = aq[c ^ (r & 7)];  // swizzled fp32 tile image
             dq[4 * c] = a.x; dq[4 * c + 1] = a.y; dq[4 * c + 2] = a.z; dq[4 * c + 3] = a.w;
-            dk[4 * c] = b.x; dk[4 * c + 1] = b.y; dk[4 * c + 2] = b.z; dk[4 * c + 3] = b.w;
         }
         rope32(dq, sl.i, sl.j, tab, true);
-        rope32(dk, sl.i, sl.j, tab, true);
         load_row_bf16(p.q + tok * 4, q);
-        load_row_bf16(p.k + tok * 4, k);
 #pragma unroll
         for (int ax = 0; ax < 2; ++ax) {
             const float pos = static_cast<float>(ax ? sl.i : sl.j);
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk) {
                 const int a = ax * 16 + 2 * kk, b = a + 1;
-                const float w = (dq[b] * q[a] - dq[a] * q[b]) + (dk[b] * k[a] - dk[a] * k[b]);
-                part[ax * 8 + kk] = pos * w;
+                part[ax * 8 + kk] = pos * (dq[b] * q[a] - dq[a] * q[b]);
             }
         }
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-            p.dq[tok * 4 + c] = pack_chunk(dq, c);
-            p.dk[tok * 4 + c] = pack_chunk(dk, c);
-        }
+        for (int c = 0; c < 4; ++c) p.dq[tok * 4 + c] = pack_chunk(dq, c);
     }
+    float* out = reinterpret_cast<float*>(const_cast<uint8_t*>(p.ws) + p.L.part) + (ht * 8 + warp) * 16;
 #pragma unroll
     for (int e = 0; e < 16; ++e) {
         float v = part[e];
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-        if (lane == 0) red[warp][e] = v;
-    }
-    __syncthreads();
-    if (r < 16) {
-        const float s = (red[0][r] + red[1][r]) + (red[2][r] + red[3][r]);
-        reinterpret_cast<float*>(const_cast<uint8_t*>(p.ws) + p.L.part)[ht * 16 + r] = s;
+        if (lane == e) out[e] = v;
     }
 }
 
@@ -766,17 +807,18 @@ cudaError_t launch_bwd(const Geo& g, const BwdPtrs& p, const BwdMaps& maps, unsi
     mp.limit_ns = limit_ns;
     mp.items = bwd_items(g);
     mp.scale = scale;
+    mp.theta = p.theta;
+    mp.part = reinterpret_cast<float*>(p.ws + L.part);
     const long long grid = mp.items < num_sms ? mp.items : num_sms;
-    main_kernel<<<static_cast<unsigned>(grid), kThreads, kSmemBytes, stream>>>(maps.v, maps.dv, mp);
+    main_kernel<<<static_cast<unsigned>(grid), kThreads, kSmemBytes, stream>>>(maps.v, maps.dv, maps.dout, maps.dk, mp);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     mark(2);
 
-    PostParams qp{g, static_cast<const uint4*>(p.q), static_cast<const uint4*>(p.k), p.theta,
-                  static_cast<uint4*>(p.dq), static_cast<uint4*>(p.dk), p.ws, L, scale};
+    PostParams qp{g, static_cast<const uint4*>(p.q), p.theta, static_cast<uint4*>(p.dq), p.ws, L, scale};
     post_kernel<<<static_cast<unsigned>(ht), 128, 0, stream>>>(qp);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     mark(3);
-    if ((e = launch_dtheta(reinterpret_cast<const float*>(p.ws + L.part), g.tiles, g.heads,
+    if ((e = launch_dtheta(reinterpret_cast<const float*>(p.ws + L.part), g.tiles * 8, g.heads,
                            reinterpret_cast<float*>(p.ws + L.part2), p.dtheta, stream)) != cudaSuccess)
         return e;
     mark(4);
