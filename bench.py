@@ -16,6 +16,7 @@ import argparse
 import hashlib
 import json
 import os
+import re
 import statistics
 import subprocess
 import sys
@@ -54,15 +55,36 @@ def unmasked_pairs(B, H, W, heads, M, s) -> int:
     return per_image * B * heads
 
 
-def kernel_sources_sha256() -> str:
-    """Hash of the CUDA sources; stored DRAM traffic is valid only for the build it was captured on."""
-    root = os.path.join(os.path.dirname(os.path.abspath(__file__)), "vision_transformer_windowed_b200", "csrc")
+def _include_closure(root: str, tu: str) -> list:
+    """The translation unit and the local headers it includes, directly or not."""
+    seen, todo = set(), [tu]
+    while todo:
+        f = todo.pop()
+        path = os.path.join(root, f)
+        if f in seen or not os.path.exists(path):
+            continue
+        seen.add(f)
+        with open(path) as fh:
+            for line in fh:
+                m = re.match(r'\s*#include "([^"/]+)"', line)
+                if m:
+                    todo.append(m.group(1))
+    return sorted(seen)
+
+
+def kernel_sources_sha256(tu: str) -> str:
+    """Hash of a kernel's sources (its translation unit, the local headers it includes)
+    and of the build script; stored DRAM traffic is valid only for the build it was
+    captured on."""
+    pkg = os.path.join(os.path.dirname(os.path.abspath(__file__)), "vision_transformer_windowed_b200")
+    root = os.path.join(pkg, "csrc")
     h = hashlib.sha256()
-    for f in sorted(os.listdir(root)):
-        if f.endswith((".cu", ".cuh")):
-            h.update(f.encode())
-            with open(os.path.join(root, f), "rb") as fh:
-                h.update(fh.read())
+    for f in _include_closure(root, tu):
+        h.update(f.encode())
+        with open(os.path.join(root, f), "rb") as fh:
+            h.update(fh.read())
+    with open(os.path.join(pkg, "build.py"), "rb") as fh:
+        h.update(fh.read())
     return h.hexdigest()
 
 
@@ -75,7 +97,7 @@ def measured_traffic(kernel: str, workload: str):
             rec = json.load(fh).get(kernel)
     except (OSError, ValueError):
         return None
-    if not rec or rec.get("workload") != workload or rec.get("sources_sha256") != kernel_sources_sha256():
+    if not rec or rec.get("workload") != workload or rec.get("sources_sha256") != kernel_sources_sha256(rec["source"]):
         return None
     return rec["bytes_per_launch"]
 

@@ -116,9 +116,11 @@ __device__ __forceinline__ void load_row_bf16(const uint4* src, float (&x)[32]) 
 __global__ void __launch_bounds__(128) prep_kernel(const PrepParams p) {
     __shared__ float2 tab[2 * 64 * 8];
     const Geo& g = p.g;
-    const long long ht = blockIdx.x;
-    const int h = static_cast<int>(ht / g.tiles);
-    const long long T = ht - static_cast<long long>(h) * g.tiles;
+    // blocks take the heads of a tile in turn (a token's heads share memory
+    // lines); ht indexes the workspace images, [head][tile]
+    const long long T = blockIdx.x / g.heads;
+    const int h = static_cast<int>(blockIdx.x - T * g.heads);
+    const long long ht = static_cast<long long>(h) * g.tiles + T;
     build_table(tab, p.theta + h * 16, g.M, threadIdx.x, blockDim.x);
     __syncthreads();
     const int r = threadIdx.x;
@@ -678,9 +680,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 __global__ void __launch_bounds__(128) post_kernel(const PostParams p) {
     __shared__ float2 tab[2 * 64 * 8];
     const Geo& g = p.g;
-    const long long ht = blockIdx.x;
-    const int h = static_cast<int>(ht / g.tiles);
-    const long long T = ht - static_cast<long long>(h) * g.tiles;
+    const long long T = blockIdx.x / g.heads;  // heads of a tile in turn, as in prep
+    const int h = static_cast<int>(blockIdx.x - T * g.heads);
+    const long long ht = static_cast<long long>(h) * g.tiles + T;
     build_table(tab, p.theta + h * 16, g.M, threadIdx.x, blockDim.x);
     __syncthreads();
     const int r = threadIdx.x, lane = r & 31, warp = r >> 5;
