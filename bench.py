@@ -35,6 +35,11 @@ WORKLOADS = {
     "flashswin_t_stage1_p2_m32": dict(B=128, H=128, W=128, heads=3, M=32, shifts=(16,), qk_scale=1.0),
     # 512x512 input at p=2, window 64 (4096-token windows), Q and K scaled by 3
     "highres_p2_m64": dict(B=16, H=256, W=256, heads=3, M=64, shifts=(32,), qk_scale=3.0),
+    # inference forward (no LSE written) at the shape of FlashSwin's inference-throughput figure:
+    # p=4 (64x64 grid at 256x256 input), batch 128, windows 8 to 32, unshifted and shifted blocks
+    "swin_t_stage1_p4_infer_m8": dict(B=128, H=64, W=64, heads=3, M=8, shifts=(0, 4), qk_scale=1.0, infer=True),
+    "swin_t_stage1_p4_infer_m16": dict(B=128, H=64, W=64, heads=3, M=16, shifts=(0, 8), qk_scale=1.0, infer=True),
+    "swin_t_stage1_p4_infer_m32": dict(B=128, H=64, W=64, heads=3, M=32, shifts=(0, 16), qk_scale=1.0, infer=True),
 }
 HEADLINE = "swin_t_stage1_p4_m8"
 
@@ -237,7 +242,7 @@ def main():
     ap.add_argument("--steps", type=int, default=10)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="fswin", choices=["fswin", "reference"])
-    ap.add_argument("--workload", default=HEADLINE, choices=sorted(WORKLOADS))
+    ap.add_argument("--workload", default=HEADLINE, choices=sorted(n for n in WORKLOADS if not WORKLOADS[n].get("infer")))
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-extra", action="store_true", help="skip the per-config numbers of the other workloads")
     ap.add_argument("--reference-seconds", type=float, default=60.0)
@@ -276,13 +281,22 @@ def main():
         B, H, W, heads, M = wl["B"], wl["H"], wl["W"], wl["heads"], wl["M"]
         t = dp.rank_inputs(B, H, W, heads, HEAD_DIM, rank, dev, qk_scale=wl["qk_scale"])
         q, k, v, th, do = t["q"], t["k"], t["v"], t["theta"], t["dout"]
-        outs = {s: (torch.empty_like(q), torch.empty((B, H, W, heads), device=dev, dtype=torch.float32))
+        infer = wl.get("infer", False)
+        outs = {s: (torch.empty_like(q), None if infer else torch.empty((B, H, W, heads), device=dev, dtype=torch.float32))
                 for s in wl["shifts"]}
-        grads = {s: (torch.empty_like(q), torch.empty_like(q), torch.empty_like(q), torch.empty_like(th))
-                 for s in wl["shifts"]}
-        ws = ops.alloc_workspace(q, M, wl["shifts"][0])
+        grads = {} if infer else {s: (torch.empty_like(q), torch.empty_like(q), torch.empty_like(q), torch.empty_like(th))
+                                  for s in wl["shifts"]}
+        ws = torch.empty(0, dtype=torch.uint8) if infer else ops.alloc_workspace(q, M, wl["shifts"][0])
 
         def step(evs=None):
+            if infer:  # forward only, O only
+                for si, s in enumerate(wl["shifts"]):
+                    if evs is not None:
+                        _lib.fs_set_phase_events([e.cuda_event for e in evs[si][0]])
+                    ops.winattn_fwd(q, k, v, th, M, s, o=outs[s][0], need_lse=False)
+                if evs is not None:
+                    _lib.fs_set_phase_events([])
+                return
             for si, s in enumerate(wl["shifts"]):
                 o, lse = outs[s]
                 dq, dk, dv, dth = grads[s]
@@ -328,6 +342,8 @@ def main():
         assert _lib.fs_device_status() == 0, "a kernel reported a device-side failure"
         peak_gb = torch.cuda.max_memory_allocated(dev) / 1e9
         fwd_f, bwd_f = workload_flops(wl)
+        if infer:
+            bwd_f = 0.0
         tokens = B * H * W * len(wl["shifts"])
         res = {"ms": ms, "tflops": (fwd_f + bwd_f) * world / (ms * 1e-3) / 1e12,
                "tokens_per_s": tokens * world / (ms * 1e-3), "peak_gb": peak_gb,
@@ -338,8 +354,13 @@ def main():
             for stp in evsets:
                 for fe, be in stp:
                     tot["fwd"] += fe[0].elapsed_time(fe[1])
+                    if infer:
+                        continue
                     for j in range(4):
                         tot[names[1 + j]] += be[j].elapsed_time(be[j + 1])
+            if infer:
+                names = ["fwd"]
+                tot = {"fwd": tot["fwd"]}
             launches = steps * len(wl["shifts"])
             res["phase_ms"] = {n: tot[n] / launches for n in names}  # average per launch
             res["phase_share"] = {n: tot[n] / max(sum(tot.values()), 1e-9) for n in names}
@@ -436,6 +457,9 @@ def main():
                                 "pct_bf16_peak": 100 * r["tflops"] / peaks["bf16_tflops"] / world,
                                 "tokens_per_s": r["tokens_per_s"], "peak_gb": r["peak_gb"],
                                 "phase_ms": r["phase_ms"], "bwd_workspace_gb": r["ws_bytes"] / 1e9}
+            if WORKLOADS[name].get("infer"):
+                per_config[name]["step"] = "inference forward (no LSE) at every shift"
+                del per_config[name]["bwd_workspace_gb"]
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

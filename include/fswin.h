@@ -78,7 +78,10 @@ FS_API fs_status fs_winattn_check_shape(const fs_winattn_shape* shape);
 
 /*
  * Forward.  In: q, k, v (bf16 [B,H,W,heads,d]), theta (fp32 [heads,2,d/4]).
- * Out: o (bf16 [B,H,W,heads,d]) and lse (fp32 [B,H,W,heads]); both overwritten.
+ * Out: o (bf16 [B,H,W,heads,d]) and lse (fp32 [B,H,W,heads], natural log);
+ * both overwritten.  lse may be NULL: an inference forward that writes o only
+ * (the workload of FlashSwin's inference-throughput figure, thelatestinai.com
+ * Fig. S1); the backward needs lse, so a training forward passes it.
  * Exact softmax attention per window (FlashSwin abstract: "exact softmax
  * attention without materializing the score matrix").
  */

@@ -6,6 +6,7 @@ import os
 import re
 
 import pytest
+import torch
 
 from vision_transformer_windowed_b200 import _lib
 
@@ -92,3 +93,13 @@ def test_workspace_flat_in_window_size():
     # reduction's second level: heads x 64 x 16 floats)
     d = _lib.fs_winattn_bwd_workspace_bytes(_lib.make_shape(32, 256, 256, 3, 32, 32, 16))
     assert abs(d - 2 * a) <= 3 * 64 * 16 * 4 + 4096
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="would launch on the placeholder pointers")
+def test_inference_forward_takes_a_null_lse():
+    """lse may be NULL (inference forward): the call passes argument checking and,
+    with no GPU here, stops at the device check."""
+    sh = _lib.make_shape(1, 16, 16, 2, 32, 8, 0)
+    with pytest.raises(_lib.FswinError) as e:
+        _lib.fs_winattn_fwd(sh, 16, 16, 16, 16, 16, 0, 0)
+    assert e.value.status not in (_lib.FS_ERR_NULL, _lib.FS_ERR_ALIGN, _lib.FS_ERR_SHAPE)

@@ -136,7 +136,7 @@ fs_status fs_winattn_fwd(const fs_winattn_shape* shape, const void* q, const voi
     fs_status st = make_geo(shape, &g);
     if (st != FS_OK) return st;
     if (g.B == 0) return FS_OK;
-    if (!q || !k || !v || !theta || !o || !lse) return FS_ERR_NULL;
+    if (!q || !k || !v || !theta || !o) return FS_ERR_NULL;  // lse may be NULL (inference)
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) ||
         (reinterpret_cast<uintptr_t>(theta) & 3u) || (reinterpret_cast<uintptr_t>(lse) & 3u))
         return FS_ERR_ALIGN;

@@ -72,7 +72,7 @@ static_assert(sizeof(Bars) <= 2048, "barrier block overflows its shared-memory s
 struct Params {
     Geo g;
     const float* theta;  // [heads][2][8]
-    float* lse;          // [B,H,W,heads]
+    float* lse;          // [B,H,W,heads], or null (inference: not written)
     unsigned int* status;
     unsigned long long limit_ns;
     long long items;
@@ -480,7 +480,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const int widx = r >> (g.lnbw + g.lBT);  // window of the row inside the tile
                 if (widx) w = win_of(g, wq.gw + widx);
             }
-            if (w.valid) {
+            if (w.valid && prm.lse != nullptr) {  // no lse: inference
                 int pi, pj;
                 tile_row_pos(g, X, r, &pi, &pj);
                 int row = w.wr * g.M + pi + g.s, col = w.wc * g.M + pj + g.s;

@@ -794,7 +794,8 @@ __global__ void __launch_bounds__(kThreads, 4) fwd_kernel(const __grid_constant_
                 for (int e = 0; e < 32; ++e) x[e] = __uint_as_float(t[e]) * inv;
                 store_row_swz(sl, r, x);
             }
-            if (cur.valid) prm.lse[cur.tok] = (m + lg2_approx(l)) * 0.69314718055994530942f;
+            if (cur.valid && prm.lse != nullptr)  // no lse: inference
+                prm.lse[cur.tok] = (m + lg2_approx(l)) * 0.69314718055994530942f;
             __syncwarp();
             // coalesced stores of the warp's 32 rows of O (8 rows per instruction)
 #pragma unroll

@@ -39,8 +39,10 @@ def _stream(device) -> int:
     return torch.cuda.current_stream(device).cuda_stream
 
 
-def winattn_fwd(q, k, v, theta, M: int, s: int, o=None, lse=None):
-    """O, LSE = fused windowed-RoPE attention forward (bf16 in/out, fp32 LSE)."""
+def winattn_fwd(q, k, v, theta, M: int, s: int, o=None, lse=None, need_lse: bool = True):
+    """O, LSE = fused windowed-RoPE attention forward (bf16 in/out, fp32 LSE).
+
+    need_lse=False (and no lse buffer): inference forward, O only; LSE is returned as None."""
     sh = _shape(q, M, s)
     B, H, W, heads, d = q.shape
     for name, t in (("q", q), ("k", k), ("v", v)):
@@ -48,12 +50,13 @@ def winattn_fwd(q, k, v, theta, M: int, s: int, o=None, lse=None):
     _check_tensor("theta", theta, (heads, 2, d // 4), torch.float32)
     if o is None:
         o = torch.empty_like(q)
-    if lse is None:
+    if lse is None and need_lse:
         lse = torch.empty((B, H, W, heads), device=q.device, dtype=torch.float32)
     _check_tensor("o", o, q.shape, torch.bfloat16)
-    _check_tensor("lse", lse, (B, H, W, heads), torch.float32)
+    if lse is not None:
+        _check_tensor("lse", lse, (B, H, W, heads), torch.float32)
     _lib.fs_winattn_fwd(sh, q.data_ptr(), k.data_ptr(), v.data_ptr(), theta.data_ptr(), o.data_ptr(),
-                        lse.data_ptr(), _stream(q.device))
+                        lse.data_ptr() if lse is not None else 0, _stream(q.device))
     return o, lse
 
 
