@@ -57,6 +57,9 @@ SMALL = [  # (B, H, W, heads, M, s)
     (2, 32, 32, 2, 32, 0),    # one window per image
     (1, 64, 64, 1, 64, 32),   # 4096-token window
     (1, 64, 96, 1, 32, 12),
+    (1, 16, 16, 6, 8, 4),     # windows inside a tile with more heads than resident RoPE tables
+    (1, 32, 32, 12, 32, 16),  # FlashSwin-T stage 3: one shifted window per image, 12 heads
+    (1, 16, 16, 24, 16, 0),   # stage 4: the window is the grid, 24 heads
 ]
 
 
@@ -109,3 +112,44 @@ def test_bounded_wait_reports_timeout_and_context_survives():
     assert code >> 24 == _lib.FS_ERR_TIMEOUT and (code & 0xFFFFFF) == 0xABC
     got, ref = run_both(1, 16, 16, 2, 8, 0)  # the context is still usable
     check("o", got["o"], ref["o"], FWD_TOL)
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("cfg", [(2, 16, 16, 3, 8, 4), (1, 64, 64, 2, 32, 16)])
+def test_backward_is_deterministic(cfg):
+    """Two runs on the same inputs: every output bit for bit, except at M >= 16 dq,
+    whose per-tile sums are reduce-added by several CTAs in any order, and d theta,
+    whose query-side terms are taken from that dq (they agree to rounding)."""
+    B, H, W, h, M, s = cfg
+    inp = make_inputs(B, H, W, h, 32)
+    dev = {k: v.cuda() for k, v in inp.items()}
+    o, lse = ops.winattn_fwd(dev["q"], dev["k"], dev["v"], dev["theta"], M, s)
+    a = ops.winattn_bwd(dev["q"], dev["k"], dev["v"], o, dev["dout"], lse, dev["theta"], M, s)
+    b = ops.winattn_bwd(dev["q"], dev["k"], dev["v"], o, dev["dout"], lse, dev["theta"], M, s)
+    torch.cuda.synchronize()
+    names = ("dq", "dk", "dv", "dtheta")
+    exact = names if M * M < 128 else ("dk", "dv")
+    for name, x, y in zip(names, a, b):
+        if name in exact:
+            assert torch.equal(x, y), name
+        else:
+            check(name, x, y.float().cpu().numpy(), (1e-3, 1e-6))
+
+
+@pytest.mark.gpu
+def test_side_stream_gives_the_default_stream_results():
+    """Work is enqueued on the caller's current stream."""
+    inp = make_inputs(2, 32, 32, 2, 32)
+    dev = {k: v.cuda() for k, v in inp.items()}
+    o0, l0 = ops.winattn_fwd(dev["q"], dev["k"], dev["v"], dev["theta"], 8, 4)
+    g0 = ops.winattn_bwd(dev["q"], dev["k"], dev["v"], o0, dev["dout"], l0, dev["theta"], 8, 4)
+    torch.cuda.synchronize()
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        o1, l1 = ops.winattn_fwd(dev["q"], dev["k"], dev["v"], dev["theta"], 8, 4)
+        g1 = ops.winattn_bwd(dev["q"], dev["k"], dev["v"], o1, dev["dout"], l1, dev["theta"], 8, 4)
+    side.synchronize()
+    assert torch.equal(o0, o1) and torch.equal(l0, l1)
+    for x, y in zip(g0, g1):
+        assert torch.equal(x, y)
