@@ -27,8 +27,11 @@ FULL = [
     ("swin_t_stage1_p4_m8_s4", 128, 64, 64, 3, 8, 4, 1.0),
     ("flashswin_t_stage1_p2_m32", 128, 128, 128, 3, 32, 16, 1.0),
     ("flashswin_t_stage2_p2_m32_s0", 128, 64, 64, 6, 32, 0, 1.0),
+    ("flashswin_t_stage2_p2_m32_s16", 128, 64, 64, 6, 32, 16, 1.0),
+    ("flashswin_t_stage3_p2_m32_s0", 128, 32, 32, 12, 32, 0, 1.0),
     ("flashswin_t_stage3_p2_m32_s16", 128, 32, 32, 12, 32, 16, 1.0),
     ("flashswin_t_stage4_p2_m16", 128, 16, 16, 24, 16, 0, 1.0),
+    ("highres_p2_m32", 16, 256, 256, 3, 32, 16, 3.0),
     ("highres_p2_m64", 16, 256, 256, 3, 64, 32, 3.0),
 ]
 
