@@ -15,7 +15,9 @@
 //              of d theta;
 //   3. post:   per token row, undo the rotation of dQ', write dq, and the
 //              query side of d theta;
-//   4. reduce: fixed-order sum of the partials into dtheta (deterministic).
+//   4. reduce: fixed-order sum of the partials into dtheta (it adds no
+//              run-to-run variation; the query-side partials carry that of
+//              dQ', whose reduce-adds land in any order).
 #include <cuda.h>
 #include <cuda_runtime.h>
 
@@ -166,7 +168,8 @@ __global__ void __launch_bounds__(128) prep_kernel(const PrepParams p) {
 // so the compute warps work on one buffer while the tensor core fills the
 // other and never wait for the previous gradients.
 //   epilogue warps: dQ' of each step to the fp32 accumulator (bulk
-//                   reduce-add), dK' and dV of each item.
+//                   reduce-add); at the end of each item dk (dK' un-rotated),
+//                   the key side of d theta, and dv (TMA stores).
 constexpr int kThreads = 448;
 constexpr int kQStages = 3;
 constexpr int kWarpTma = 12, kWarpMma = 13;  // warps 0-7: P/dS, 8-11: epilogue

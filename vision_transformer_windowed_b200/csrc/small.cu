@@ -3,10 +3,10 @@
 // head) and all of its attention stays inside the tile.
 //
 // At these sizes a window box of a shifted grid is as small as 4 x 4 tokens,
-// too small for TMA box copies to keep up, so each row thread of these
-// kernels moves token rows itself: coalesced 16-byte cp.async copies (8 whole
-// 64-byte rows per warp instruction) issued one work item ahead, and
-// coalesced 16-byte stores of the results.  Work items are (tile, head) with
+// too small for TMA box copies to keep up, so threads move token rows
+// themselves (the forward's row warps, the backward's mover warp): coalesced
+// 16-byte cp.async copies (8 whole 64-byte rows per warp instruction) issued
+// one work item ahead, and coalesced 16-byte stores of the results.  Work items are (tile, head) with
 // heads innermost while every head's RoPE table fits in shared memory, so the
 // heads of a token, which are adjacent in memory, are read close together.
 #include <cuda.h>
@@ -40,20 +40,21 @@ __device__ __forceinline__ void small_item(const Geo& g, bool head_minor, long l
 }
 
 // ------------------------------------------------------------------ backward
-// The whole backward of a tile on chip, with no workspace round trip: only
-// 4 x 16 d theta partials per tile leave it.
 // Windows of fewer than 128 tokens (M = 4, 8) lie whole inside one 128-slot
 // tile, so every gradient of a tile's tokens comes from that tile alone.  One
 // persistent kernel then does the whole backward of a tile on chip, with no
-// workspace round trip: only the 16 d theta partials of the tile leave it.
-//   warps 0-3: thread = slot row.  Loads its own q, k, v, dO, o rows with
-//              16-byte async copies one work item ahead (a window box of a
-//              shifted grid is as small as 4 x 4 tokens, too small for TMA box
-//              copies to keep up); D, lse and the RoPE of its q and k rows; the
-//              row of P^T and dS^T of its key; the epilogue of its token, whose
-//              dq, dk, dv rows it stores directly.
+// workspace round trip: only 4 x 16 d theta partials per tile leave it.
+//   warps 0-3: thread = slot row.  D, lse and the RoPE of its q and k rows;
+//              the row of P^T and dS^T of its key; the epilogue of its token
+//              (dq, dk un-rotated, dv, the d theta terms), staged over the
+//              slot's q, k, v rows.
 //   warp 4:    MMA issuer: S^T = K' Q'^T, dP^T = V dO^T; then dV = P^T dO,
 //              dK' = dS^T Q', dQ' = dS K'.
+//   warp 5:    mover: the q, k, v, dO rows of each item (and its o rows) with
+//              16-byte async copies one item ahead, completing on mbarriers (a
+//              window box of a shifted grid is as small as 4 x 4 tokens, too
+//              small for TMA box copies to keep up), and the stores of the
+//              staged dq, dk, dv rows.
 // Two CTAs share an SM (256 TMEM columns each).  Work items are (tile, head),
 // heads innermost when their RoPE tables fit, so the heads of a token, which
 // are adjacent in memory, are read close together in time.
