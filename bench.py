@@ -174,33 +174,37 @@ class ClockSampler:
 
 def cpu_baseline(tensors, wl, seconds: float = 12.0):
     """Times the fp64 oracle (forward + backward) on host cores over a bounded
-    sample of the workload's (batch, window, head) units at its last shift."""
+    sample of the workload's (batch, window, head) units at every shift of the
+    step (all of them when they fit in the time budget)."""
     import numpy as np
 
     import oracle
     B, H, W, heads, M = wl["B"], wl["H"], wl["W"], wl["heads"], wl["M"]
-    s = wl["shifts"][-1]
     nW = (H // M) * (W // M)
     n_units = B * nW * heads
     cores = oracle.default_threads()
-    # units spread over the batch, including windows of the last row/column
-    t0 = time.perf_counter()
-    probe = np.arange(0, min(n_units, 4 * cores))
-    oracle.units(tensors["q"], tensors["k"], tensors["v"], tensors["theta"], M, s, probe, dout=tensors["dout"],
-                 nthreads=cores)
-    dt = max(time.perf_counter() - t0, 1e-6)
-    n = int(min(n_units, max(len(probe), len(probe) * seconds / dt)))
-    ids = np.linspace(0, n_units - 1, n).astype(np.int64)
-    t0 = time.perf_counter()
-    oracle.units(tensors["q"], tensors["k"], tensors["v"], tensors["theta"], M, s, ids, dout=tensors["dout"],
-                 nthreads=cores)
-    dt = time.perf_counter() - t0
-    # useful flops of the sampled units (pairs that attend)
-    pairs_all = unmasked_pairs(B, H, W, heads, M, s)
-    flops = 14.0 * HEAD_DIM * pairs_all * (n / n_units)
-    return {"value": flops / dt / 1e12, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
-            "sample": f"{n} of {n_units} (batch, window, head) units at s={s}, fwd+bwd, fp64, {dt:.1f} s",
-            "seconds": dt}
+    flops, total_dt, parts = 0.0, 0.0, []
+    for s in wl["shifts"]:
+        # units spread over the batch, including windows of the last row/column
+        t0 = time.perf_counter()
+        probe = np.arange(0, min(n_units, 4 * cores))
+        oracle.units(tensors["q"], tensors["k"], tensors["v"], tensors["theta"], M, s, probe, dout=tensors["dout"],
+                     nthreads=cores)
+        dt = max(time.perf_counter() - t0, 1e-6)
+        budget = seconds / len(wl["shifts"])
+        n = int(min(n_units, max(len(probe), len(probe) * budget / dt)))
+        ids = np.linspace(0, n_units - 1, n).astype(np.int64)
+        t0 = time.perf_counter()
+        oracle.units(tensors["q"], tensors["k"], tensors["v"], tensors["theta"], M, s, ids, dout=tensors["dout"],
+                     nthreads=cores)
+        dt = time.perf_counter() - t0
+        # useful flops of the sampled units (pairs that attend)
+        flops += 14.0 * HEAD_DIM * unmasked_pairs(B, H, W, heads, M, s) * (n / n_units)
+        total_dt += dt
+        parts.append(f"{n} of {n_units} at s={s}")
+    return {"value": flops / total_dt / 1e12, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+            "sample": f"(batch, window, head) units: {', '.join(parts)}; fwd+bwd, fp64, {total_dt:.1f} s",
+            "seconds": total_dt}
 
 
 def run_reference(args):
