@@ -1,0 +1,53 @@
+"""fp64 oracle of the window-attention block of a Swin layer (test infrastructure).
+
+TEST INFRASTRUCTURE ONLY, like the rest of ``oracle``: the product package
+never imports it.
+
+The block around FlashSwin's attention (thelatestinai.com/papers/2610.04664,
+Figure 1B: the attention module of each FlashSwin block) is the Swin layer's
+qkv linear map, the windowed RoPE attention per head, and the output linear
+map.  Written out as that definition:
+
+    qkv = x W_qkv^T + b_qkv          x [B, H, W, C], W_qkv [3C, C], C = heads * d
+    q, k, v = qkv split in (3, heads, d) along the channels
+    o = windowed-RoPE attention of (q, k, v) per head, as in ``oracle.full``
+    y = o W_o^T + b_o                o flattened to [B, H, W, C], W_o [C, C]
+
+The projections are fp64 matrix products (a library primitive); the attention
+is the C oracle.  The shift needs no separate handling: the projections act
+token by token, so they commute with the cyclic roll of the windows.
+"""
+from __future__ import annotations
+
+import numpy as np
+
+from . import full
+
+
+def _f64(a):
+    try:
+        import torch
+        if isinstance(a, torch.Tensor):
+            return a.detach().cpu().to(torch.float64).numpy()
+    except ImportError:  # pragma: no cover
+        pass
+    return np.asarray(a, dtype=np.float64)
+
+
+def project_qkv(x, w_qkv, b_qkv, heads: int):
+    """q, k, v [B, H, W, heads, d] (float64) of the block's input x."""
+    x, w, b = _f64(x), _f64(w_qkv), _f64(b_qkv)
+    B, H, W, C = x.shape
+    d = C // heads
+    qkv = x @ w.T + b  # [B, H, W, 3C]
+    qkv = qkv.reshape(B, H, W, 3, heads, d)
+    return qkv[..., 0, :, :], qkv[..., 1, :, :], qkv[..., 2, :, :]
+
+
+def block_forward(x, w_qkv, b_qkv, w_o, b_o, theta, M: int, s: int, heads: int, nthreads: int | None = None):
+    """y [B, H, W, C] (float64) of the attention block; also returns the attention output o."""
+    q, k, v = project_qkv(x, w_qkv, b_qkv, heads)
+    o = full(q, k, v, theta, M, s, nthreads=nthreads)["o"]  # [B, H, W, heads, d]
+    B, H, W = o.shape[:3]
+    of = o.reshape(B, H, W, -1)
+    return of @ _f64(w_o).T + _f64(b_o), o

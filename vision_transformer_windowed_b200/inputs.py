@@ -11,12 +11,19 @@ thelatestinai.com/papers/2610.04664, Table S1 and Figure S1 shapes):
     100 ** (-2 i / (d / 2)), i = 0 .. d/4 - 1, repeated for both axes and every
     head (the initialisation the pages call "the standard geometric RoPE
     schedule", Figure S4), plus N(0, 0.01) noise from a generator seeded 4.
+
+For the attention block with its projections (Figure 1B): x bf16 N(0, 1) on a
+[B, H, W, C] grid (seed 5), C = heads * d; W_qkv [3C, C] and W_o [C, C] bf16
+N(0, 1/C), the variance of a linear layer's initialisation, so that q, k, v
+are near N(0, 1) like the attention workloads' (seeds 6 and 8); b_qkv and b_o
+fp32 N(0, 0.02^2) (seeds 7 and 9); theta as above.
 """
 from __future__ import annotations
 
 import torch
 
 SEED_Q, SEED_K, SEED_V, SEED_DO, SEED_THETA = 0, 1, 2, 3, 4
+SEED_X, SEED_WQKV, SEED_BQKV, SEED_WO, SEED_BO = 5, 6, 7, 8, 9
 
 
 def _normal(shape, seed: int, device, scale: float = 1.0) -> torch.Tensor:
@@ -55,3 +62,22 @@ def make_inputs(B: int, H: int, W: int, heads: int, d: int, device="cpu", qk_sca
     if with_dout:
         out["dout"] = _normal(shape, SEED_DO + off, device)
     return out
+
+
+def make_block_inputs(B: int, H: int, W: int, heads: int, d: int, device="cpu") -> dict:
+    """Inputs of the attention block: x, w_qkv, b_qkv, w_o, b_o, theta."""
+    C = heads * d
+
+    def draw(shape, seed, std, dtype):
+        g = torch.Generator(device=device)
+        g.manual_seed(seed)
+        return (torch.randn(shape, generator=g, device=device, dtype=torch.float32) * std).to(dtype)
+
+    return {
+        "x": draw((B, H, W, C), SEED_X, 1.0, torch.bfloat16),
+        "w_qkv": draw((3 * C, C), SEED_WQKV, C ** -0.5, torch.bfloat16),
+        "b_qkv": draw((3 * C,), SEED_BQKV, 0.02, torch.float32),
+        "w_o": draw((C, C), SEED_WO, C ** -0.5, torch.bfloat16),
+        "b_o": draw((C,), SEED_BO, 0.02, torch.float32),
+        "theta": theta_init(heads, d, device),
+    }
