@@ -89,6 +89,25 @@ FS_API fs_status fs_winattn_fwd(const fs_winattn_shape* shape, const void* q, co
                          const float* theta, void* o, float* lse, fs_stream_t stream);
 
 /*
+ * Forward of the whole window-attention block of a Swin layer, for inference
+ * (the attention module of a FlashSwin block, thelatestinai.com 2610.04664,
+ * Figure 1B, with its two linear maps):
+ *   qkv = x W_qkv^T + b_qkv, split in (3, heads, d) along the channels;
+ *   o = fs_winattn_fwd's attention of (q, k, v) with theta, M, s;
+ *   y = o W_o^T + b_o, o taken as [B,H,W,C].
+ * In: x bf16 [B,H,W,C] with C = heads * d; w_qkv bf16 [3C, C] (output channels
+ * q of every head, then k, then v); b_qkv fp32 [3C]; w_o bf16 [C, C]; b_o
+ * fp32 [C]; theta fp32 [heads,2,d/4].  Out: y bf16 [B,H,W,C], overwritten.
+ * q, k, v and o never reach device memory.  Supported: the shapes of
+ * fs_winattn_check_shape with M*M < 128 (windows inside one 128-token tile)
+ * and heads <= 3; anything else returns FS_ERR_SHAPE.  x, w_qkv, w_o, y
+ * 16-byte aligned (FS_ERR_ALIGN); no pointer may be NULL (FS_ERR_NULL).
+ */
+FS_API fs_status fs_winattn_block_fwd(const fs_winattn_shape* shape, const void* x, const void* w_qkv,
+                               const float* b_qkv, const void* w_o, const float* b_o, const float* theta,
+                               void* y, fs_stream_t stream);
+
+/*
  * Workspace the backward needs, in bytes.  It depends on B*H*W*heads only, not on
  * the window size M (memory flat in M, FlashSwin Table S1).
  */

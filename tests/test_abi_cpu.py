@@ -103,3 +103,16 @@ def test_inference_forward_takes_a_null_lse():
     with pytest.raises(_lib.FswinError) as e:
         _lib.fs_winattn_fwd(sh, 16, 16, 16, 16, 16, 0, 0)
     assert e.value.status not in (_lib.FS_ERR_NULL, _lib.FS_ERR_ALIGN, _lib.FS_ERR_SHAPE)
+
+
+def test_block_forward_rejects_before_launch():
+    """Windows inside one tile and at most three heads; NULL and misaligned pointers."""
+    def call(shape, *ptrs):
+        with pytest.raises(_lib.FswinError) as e:
+            _lib.fs_winattn_block_fwd(_lib.make_shape(*shape), *ptrs, 0)
+        return e.value.status
+    ok = [16] * 7
+    assert call((1, 32, 32, 3, 32, 16, 0), *ok) == _lib.FS_ERR_SHAPE   # 256-token windows
+    assert call((1, 16, 16, 4, 32, 8, 0), *ok) == _lib.FS_ERR_SHAPE    # four heads
+    assert call((1, 16, 16, 3, 32, 8, 0), 0, *ok[1:]) == _lib.FS_ERR_NULL
+    assert call((1, 16, 16, 3, 32, 8, 0), 24, *ok[1:]) == _lib.FS_ERR_ALIGN

@@ -51,6 +51,8 @@ def load(build_if_missing: bool = True):
         lib.fs_winattn_check_shape.restype = st
         lib.fs_winattn_fwd.argtypes = [P, vp, vp, vp, vp, vp, vp, vp]
         lib.fs_winattn_fwd.restype = st
+        lib.fs_winattn_block_fwd.argtypes = [P] + [vp] * 7 + [vp]
+        lib.fs_winattn_block_fwd.restype = st
         lib.fs_winattn_bwd_workspace_bytes.argtypes = [P]
         lib.fs_winattn_bwd_workspace_bytes.restype = ctypes.c_size_t
         lib.fs_winattn_bwd.argtypes = [P] + [vp] * 12 + [ctypes.c_size_t, vp]
@@ -92,6 +94,12 @@ def fs_winattn_check_shape(shape: Shape) -> int:
 
 def fs_winattn_fwd(shape: Shape, q: int, k: int, v: int, theta: int, o: int, lse: int, stream: int) -> None:
     _check(load().fs_winattn_fwd(ctypes.byref(shape), q, k, v, theta, o, lse, stream), "fs_winattn_fwd")
+
+
+def fs_winattn_block_fwd(shape: Shape, x: int, w_qkv: int, b_qkv: int, w_o: int, b_o: int, theta: int, y: int,
+                         stream: int) -> None:
+    _check(load().fs_winattn_block_fwd(ctypes.byref(shape), x, w_qkv, b_qkv, w_o, b_o, theta, y, stream),
+           "fs_winattn_block_fwd")
 
 
 def fs_winattn_bwd_workspace_bytes(shape: Shape) -> int:

@@ -158,6 +158,32 @@ fs_status fs_winattn_fwd(const fs_winattn_shape* shape, const void* q, const voi
     return e == cudaSuccess ? FS_OK : FS_ERR_CUDA;
 }
 
+fs_status fs_winattn_block_fwd(const fs_winattn_shape* shape, const void* x, const void* w_qkv,
+                               const float* b_qkv, const void* w_o, const float* b_o, const float* theta,
+                               void* y, fs_stream_t stream) {
+    Geo g;
+    fs_status st = make_geo(shape, &g);
+    if (st != FS_OK) return st;
+    if (g.N >= kTile || g.heads > 3) return FS_ERR_SHAPE;  // windows inside one tile, C <= 96
+    if (g.B == 0) return FS_OK;
+    if (!x || !w_qkv || !b_qkv || !w_o || !b_o || !theta || !y) return FS_ERR_NULL;
+    if (!aligned16(x) || !aligned16(w_qkv) || !aligned16(w_o) || !aligned16(y) ||
+        (reinterpret_cast<uintptr_t>(b_qkv) & 3u) || (reinterpret_cast<uintptr_t>(b_o) & 3u) ||
+        (reinterpret_cast<uintptr_t>(theta) & 3u))
+        return FS_ERR_ALIGN;
+    unsigned int* status = nullptr;
+    int sms = 0;
+    if ((st = device_state(&status, &sms)) != FS_OK) return st;
+    unsigned long long lim;
+    {
+        std::lock_guard<std::mutex> lk(g_mu);
+        lim = g_limit_ns;
+    }
+    const BlockPtrs p{x, w_qkv, w_o, b_qkv, b_o, theta, y};
+    const cudaError_t e = launch_block_fwd(g, p, status, lim, sms, reinterpret_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? FS_OK : FS_ERR_CUDA;
+}
+
 size_t fs_winattn_bwd_workspace_bytes(const fs_winattn_shape* shape) {
     Geo g;
     if (make_geo(shape, &g) != FS_OK) return 0;

@@ -1,0 +1,460 @@
+// Forward of the whole window-attention block of a Swin layer (inference) for
+// windows of fewer than 128 tokens (M = 4, 8) and at most three heads:
+//   qkv = x W_qkv^T + b_qkv, o_h = windowed RoPE attention of head h,
+//   y = o W_o^T + b_o
+// (the attention module of a FlashSwin block, thelatestinai.com 2610.04664,
+// Figure 1B).  One persistent kernel: a work item is one 128-slot tile with
+// all of its heads, so x is read and y written once per token, and q, k, v
+// and o never leave the chip.
+//   warps 0-3 (rows): thread = slot row = TMEM lane.  Per head: the biases
+//       and the RoPE of its q, k row (TMEM -> fp16 q', k' and bf16 v tiles),
+//       the softmax of its query row, O / l into the head's o tile; per item
+//       y + b_o into the staging tiles (the o tiles, once read).
+//   warp 4 (MMA): per head q|k|v = x [W_q,h; W_k,h; W_v,h]^T (N = 96, issued
+//       while the previous head's softmax runs), S = Q'K'^T, O_h = P V; per
+//       item Y = sum_h O_h W_o[:, 32h:32h+32]^T.
+//   warp 5 (mover): the item's x rows one item ahead (16-byte cp.async), then
+//       its y rows out.
+// The weights and biases stay in shared memory for the whole launch.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "dgeo.cuh"
+#include "geometry.cuh"
+#include "kernels.cuh"
+#include "ptx.cuh"
+#include "rows.cuh"
+
+namespace fswin {
+
+namespace blockk {
+
+constexpr int kMaxHeads = 3;
+constexpr int kThreads = 192;
+constexpr int kWarpMma = 4, kWarpMover = 5;
+constexpr int kQkvRows = 3 * kHeadDim;  // q, k, v rows of one head in a W_qkv chunk tile
+
+// Shared memory (offsets from a 1024-byte aligned base).  A weight "chunk" is
+// the 32 input channels [32c, 32c + 32) of every output row, 64-byte rows,
+// 64-byte swizzle (the K-major operand layout of the MMAs); the W_qkv chunk
+// rows are ordered head by head, q, k, v rows of a head together.
+constexpr int kWqkvChunk = kMaxHeads * kQkvRows * kRowBytes;  // 18 KB
+constexpr int kWqkvOff = 0;
+constexpr int kWoChunk = kMaxHeads * kHeadDim * kRowBytes;    // 6 KB
+constexpr int kWoOff = kWqkvOff + kMaxHeads * kWqkvChunk;
+constexpr int kXBytes = kMaxHeads * kTileBytes;               // the x chunks of one item
+constexpr int kXOff = kWoOff + kMaxHeads * kWoChunk;          // 2 item buffers
+constexpr int kHeadOff = kXOff + 2 * kXBytes;                 // q' (fp16), k' (fp16), v (bf16) tiles of a head
+constexpr int kOOff = kHeadOff + 3 * kTileBytes;              // o tiles of the heads; then y staging
+constexpr int kBiasOff = kOOff + kMaxHeads * kTileBytes;      // b_qkv [3C], b_o [C] (fp32)
+constexpr int kTabPerHead = 2 * 8 * 8;                        // [axis][pair][position < 8] float2
+constexpr int kTabOff = kBiasOff + 4 * kMaxHeads * kHeadDim * 4;
+constexpr int kBarOff = kTabOff + kMaxHeads * kTabPerHead * 8;
+constexpr int kSmemBytes = kBarOff + 256 + 1024;  // + alignment of the base
+static_assert(kXOff % 1024 == 0 && kHeadOff % 1024 == 0 && kOOff % 1024 == 0, "tile alignment");
+static_assert(kWoOff % 1024 == 0 && kWqkvChunk % 1024 == 0 && kWoChunk % 512 == 0, "weight tile alignment");
+
+// TMEM columns: q|k|v of a head [0, 96) (then Y [0, C)), O_h [96, 128),
+// S [128, 256) with P (bf16) written over its consumed columns.
+constexpr uint32_t kTmemCols = 256;
+constexpr uint32_t kColQKV = 0, kColY = 0, kColO = 96, kColS = 128;
+
+struct Bars {
+    uint64_t x_full[2], x_free[2];  // per item parity: x rows landed (32 mover lanes); last q|k|v MMAs done
+    uint64_t qkv_full, in_ready, s_full, p_ready, o_full;  // per head
+    uint64_t o_ready, y_full, y_free, staged, y_done;      // per item
+    uint64_t grp, done;
+    uint32_t tmem_base;
+    int abort_flag;
+};
+static_assert(sizeof(Bars) <= 256, "barrier block overflows its slot");
+
+struct Params {
+    Geo g;
+    const uint8_t* x;  // bf16 [B, H, W, C]
+    const uint8_t *w_qkv, *w_o;  // bf16 [3C, C], [C, C]
+    const float *b_qkv, *b_o, *theta;
+    uint8_t* y;  // bf16 [B, H, W, C]
+    unsigned int* status;
+    unsigned long long limit_ns;
+    long long items;  // tiles
+};
+
+__global__ void __launch_bounds__(kThreads, 1) block_kernel(const __grid_constant__ Params prm) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    Bars* bars = reinterpret_cast<Bars*>(smem + kBarOff);
+    const Geo& g = prm.g;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int heads = g.heads, C = heads * kHeadDim;
+    float* bias = reinterpret_cast<float*>(smem + kBiasOff);  // b_qkv [3C], then b_o at [3 * 96]
+    float2* tabs = reinterpret_cast<float2*>(smem + kTabOff);
+
+    if (tid == 0) {
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&bars->x_full[i], 32);  // one arrival per mover lane, once its copies have landed
+            mbar_init(&bars->x_free[i], 1);
+        }
+        mbar_init(&bars->qkv_full, 1);
+        mbar_init(&bars->in_ready, 1);
+        mbar_init(&bars->s_full, 1);
+        mbar_init(&bars->p_ready, 4);
+        mbar_init(&bars->o_full, 1);
+        mbar_init(&bars->o_ready, 4);
+        mbar_init(&bars->y_full, 1);
+        mbar_init(&bars->y_free, 4);
+        mbar_init(&bars->staged, 4);
+        mbar_init(&bars->y_done, 1);
+        mbar_init(&bars->grp, 4);
+        mbar_init(&bars->done, 1);
+        bars->abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 0) {
+        tmem_alloc(&bars->tmem_base, kTmemCols);
+        tmem_relinquish();
+    }
+    // weights (64-byte swizzled chunk tiles), biases and RoPE tables, once
+    for (int i = tid; i < heads * 3 * C * 4; i += kThreads) {
+        const int p = i & 3, rest = i >> 2;
+        const int n = rest % (3 * C), c = rest / (3 * C);  // tile row n: head n / 96, then q, k, v rows
+        const int hh = n / kQkvRows, part = (n % kQkvRows) / kHeadDim, e = n % kHeadDim;
+        const size_t src = static_cast<size_t>(part * C + hh * kHeadDim + e) * C + 32 * c + 8 * p;
+        *reinterpret_cast<uint4*>(smem + kWqkvOff + c * kWqkvChunk + n * kRowBytes + ((p ^ ((n >> 1) & 3)) << 4)) =
+            *reinterpret_cast<const uint4*>(prm.w_qkv + 2 * src);
+    }
+    for (int i = tid; i < heads * C * 4; i += kThreads) {
+        const int p = i & 3, rest = i >> 2;
+        const int n = rest % C, c = rest / C;
+        const size_t src = static_cast<size_t>(n) * C + 32 * c + 8 * p;
+        *reinterpret_cast<uint4*>(smem + kWoOff + c * kWoChunk + n * kRowBytes + ((p ^ ((n >> 1) & 3)) << 4)) =
+            *reinterpret_cast<const uint4*>(prm.w_o + 2 * src);
+    }
+    for (int i = tid; i < 3 * C; i += kThreads) bias[i] = prm.b_qkv[i];
+    for (int i = tid; i < C; i += kThreads) bias[3 * kMaxHeads * kHeadDim + i] = prm.b_o[i];
+    for (int hh = 0; hh < heads; ++hh) build_small_table(tabs + hh * kTabPerHead, prm.theta + hh * 16, g.M, tid, kThreads);
+    fence_proxy_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = bars->tmem_base;
+    const Ctl ctl{prm.status, &bars->abort_flag, prm.limit_ns};
+    // this CTA's items (tiles): a contiguous run
+    const long long per = (prm.items + gridDim.x - 1) / gridDim.x;
+    const long long first = static_cast<long long>(blockIdx.x) * per;
+    const long long n = prm.items > first ? (prm.items - first < per ? prm.items - first : per) : 0;
+
+    if (warp == kWarpMma) {
+        // ------------------------------------------------------------ MMA issue
+        if (lane == 0) {
+            const uint32_t id_qkv = make_idesc(kTile, kQkvRows, false, false, false);  // bf16 x, W_qkv
+            const uint32_t id_s = make_idesc(kTile, kTile, false, false, true);         // fp16 Q', K'
+            const uint32_t id_pv = make_idesc(kTile, kHeadDim, false, true, false);     // P (TMEM) x V, bf16
+            const uint32_t id_y = make_idesc(kTile, C, false, false, false);            // bf16 O, W_o
+            const uint32_t sbase = smem_u32(smem);
+            const uint64_t dK0 = make_sdesc(sbase, 16, 512, kSw64);     // K-major, 64-byte rows
+            const uint64_t dMN0 = make_sdesc(sbase, 8192, 512, kSw64);  // MN-major, 64-byte rows
+            auto u16 = [](int bytes) { return static_cast<uint64_t>(bytes >> 4); };
+            const uint64_t qo = u16(kHeadOff), ko = u16(kHeadOff + kTileBytes), vo = u16(kHeadOff + 2 * kTileBytes);
+            // q|k|v of head h for item j: x (its chunk tiles) times the head's 96 W_qkv rows
+            auto issue_qkv = [&](long long j, int h) {
+                const uint64_t xo = u16(kXOff + static_cast<int>(j & 1) * kXBytes);
+                for (int c = 0; c < heads; ++c)
+#pragma unroll
+                    for (int ks = 0; ks < 2; ++ks)
+                        umma_ss(tmem + kColQKV, dK0 + xo + u16(c * kTileBytes) + 2 * ks,
+                                dK0 + u16(kWqkvOff + c * kWqkvChunk + h * kQkvRows * kRowBytes) + 2 * ks, id_qkv,
+                                (c | ks) != 0);
+                umma_commit(&bars->qkv_full);
+            };
+            uint32_t hc = 0;
+            bool ok = true;
+            for (long long j = 0; j < n && ok; ++j) {
+                const int par = static_cast<int>(j & 1);
+                if (!mbar_wait(&bars->x_full[par], static_cast<uint32_t>((j >> 1) & 1), ctl, 0x5201)) break;
+                // the rows have read the previous item's Y, which q|k|v overwrite
+                if (j > 0 && !mbar_wait(&bars->y_free, static_cast<uint32_t>((j - 1) & 1), ctl, 0x5202)) break;
+                tc_fence_after();
+                issue_qkv(j, 0);
+                for (int h = 0; h < heads; ++h, ++hc) {
+                    const uint32_t ph = hc & 1u;
+                    // the rows have read this head's q|k|v and written its q', k', v tiles
+                    if (!mbar_wait(&bars->in_ready, ph, ctl, 0x5203)) { ok = false; break; }
+                    tc_fence_after();
+#pragma unroll
+                    for (int ks = 0; ks < kHeadDim / 16; ++ks)
+                        umma_ss(tmem + kColS, dK0 + qo + 2 * ks, dK0 + ko + 2 * ks, id_s, ks > 0);
+                    umma_commit(&bars->s_full);
+                    if (h + 1 < heads)
+                        issue_qkv(j, h + 1);  // during this head's softmax
+                    else
+                        umma_commit(&bars->x_free[par]);  // every MMA that reads the item's x is issued
+                    if (!mbar_wait(&bars->p_ready, ph, ctl, 0x5204)) { ok = false; break; }
+                    tc_fence_after();
+#pragma unroll
+                    for (int k = 0; k < kTile / 16; ++k)
+                        umma_ts(tmem + kColO, tmem + kColS + 8 * k, dMN0 + vo + 64 * k, id_pv, k > 0);
+                    umma_commit(&bars->o_full);
+                }
+                if (!ok) break;
+                // Y = sum over heads of O_h W_o[:, 32h:32h+32]^T, once every o tile is written
+                if (!mbar_wait(&bars->o_ready, static_cast<uint32_t>(j & 1), ctl, 0x5205)) break;
+                tc_fence_after();
+                for (int h = 0; h < heads; ++h)
+#pragma unroll
+                    for (int ks = 0; ks < 2; ++ks)
+                        umma_ss(tmem + kColY, dK0 + u16(kOOff + h * kTileBytes) + 2 * ks,
+                                dK0 + u16(kWoOff + h * kWoChunk) + 2 * ks, id_y, (h | ks) != 0);
+                umma_commit(&bars->y_full);
+            }
+            umma_commit(&bars->done);
+            mbar_wait(&bars->done, 0, ctl, 0x52ff);
+        }
+        __syncwarp();
+    } else if (warp == kWarpMover) {
+        // ------------------------------------------------------------ x rows in, y rows out
+        // Lane l moves 16-byte chunk l % 4 of row 8 i + l / 4 of each group of 32
+        // rows: every instruction moves 8 whole 64-byte rows of one chunk tile.
+        auto mwait = [&](uint64_t* bar, uint32_t ph, unsigned int where) -> bool {
+            return __all_sync(0xFFFFFFFFu, mbar_wait(bar, ph, ctl, where));
+        };
+        long long mv_X = -1, mv_t[4] = {0, 0, 0, 0};  // token (B, H, W index) of rows lane + 32 q
+        bool mv_valid[4] = {false, false, false, false};
+        auto geo = [&](long long X) {
+            if (X == mv_X) return;
+            mv_X = X;
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                int pi, pj;
+                long long tok0;
+                mv_valid[q] = slot_token(g, X, lane + 32 * q, 0, &pi, &pj, &tok0);
+                mv_t[q] = tok0 / heads;
+            }
+        };
+        auto move = [&](long long j, bool load) {
+            geo(first + j);
+            uint8_t* xb = smem + kXOff + static_cast<int>(j & 1) * kXBytes;
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const int sl_lane = 8 * i + (lane >> 2), cp = lane & 3;
+                    const long long t = __shfl_sync(0xFFFFFFFFu, mv_t[q], sl_lane);
+                    const bool valid = __shfl_sync(0xFFFFFFFFu, mv_valid[q] ? 1 : 0, sl_lane) != 0;
+                    const int row = 32 * q + sl_lane;
+                    const uint32_t off = row * kRowBytes + ((cp ^ ((row >> 1) & 3)) << 4);
+                    const long long go = t * C * 2 + 16 * cp;
+                    for (int c = 0; c < heads; ++c) {
+                        if (load)
+                            cp_async16(smem_u32(xb + c * kTileBytes + off), valid ? prm.x + go + 64 * c : prm.x,
+                                       valid ? 16u : 0u);
+                        else if (valid)
+                            *reinterpret_cast<uint4*>(prm.y + go + 64 * c) =
+                                *reinterpret_cast<const uint4*>(smem + kOOff + c * kTileBytes + off);
+                    }
+                }
+            }
+        };
+        // Each lane waits for its own copies and fences them for the tensor
+        // core (the async proxy) before it arrives.
+        auto load = [&](long long j) {
+            move(j, true);
+            cp_async_commit();
+            cp_async_wait<0>();
+            fence_proxy_async_smem();
+            mbar_arrive(&bars->x_full[j & 1]);
+        };
+        if (n > 0) load(0);
+        if (n > 1) load(1);
+        for (long long j = 0; j < n; ++j) {
+            if (j + 2 < n) {  // item j+2's x once item j's q|k|v MMAs are done with the buffer
+                if (!mwait(&bars->x_free[j & 1], static_cast<uint32_t>((j >> 1) & 1), 0x5401)) break;
+                load(j + 2);
+            }
+            if (!mwait(&bars->staged, static_cast<uint32_t>(j & 1), 0x5402)) break;
+            move(j, false);
+            __syncwarp();  // every lane has read the staged rows: the rows may write o tiles again
+            if (lane == 0) mbar_arrive(&bars->y_done);
+        }
+        cp_async_wait<0>();
+    } else {
+        // ------------------------------------------------------------ rows (warps 0-3)
+        const int r = tid;
+        const uint32_t trow = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+        const float sl2 = g.scale_log2;
+        uint8_t* qt = smem + kHeadOff;
+        uint8_t* kt = qt + kTileBytes;
+        uint8_t* vt = qt + 2 * kTileBytes;
+        uint32_t gph = 0, hc = 0;
+        bool ok = true;
+        auto wwait = [&](uint64_t* bar, uint32_t ph, unsigned int where) -> bool {
+            return __all_sync(0xFFFFFFFFu, mbar_wait(bar, ph, ctl, where));
+        };
+        auto group_sync = [&](unsigned int where) -> bool {
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bars->grp);
+            const bool passed = wwait(&bars->grp, gph, where);
+            gph ^= 1;
+            return passed;
+        };
+        for (long long j = 0; j < n && ok; ++j) {
+            const long long X = first + j;
+            int pi, pj;
+            long long tok0;
+            slot_token(g, X, r, 0, &pi, &pj, &tok0);
+            const uint64_t segs = d_tile_segs(g, X, d_tile_win(g, X));
+            const uint32_t a16 = allow16(g, seg_at(segs, r >> g.lBT), segs);  // bit c: columns [16c, 16c+16)
+            for (int h = 0; h < heads && ok; ++h, ++hc) {
+                const uint32_t ph = hc & 1u;
+                const float2* tab = tabs + h * kTabPerHead;
+                // q, k, v of this row and head: + biases, RoPE of q and k, into the head's tiles
+                if (!wwait(&bars->qkv_full, ph, 0x5301)) { ok = false; break; }
+                tc_fence_after();
+#pragma unroll 1
+                for (int part = 0; part < 3; ++part) {
+                    uint32_t t[32];
+                    tmem_ld32(trow + kColQKV + 32 * part, t);
+                    tmem_wait_ld();
+                    const float* b = bias + part * C + h * kHeadDim;
+                    float x[32];
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) x[e] = __uint_as_float(t[e]) + b[e];
+                    if (part < 2) rope32_small(x, pi, pj, tab, false);
+                    store_row_swz(part == 0 ? qt : (part == 1 ? kt : vt), r, x, part < 2);  // q', k' fp16; v bf16
+                }
+                tc_fence_before();
+                fence_proxy_async_smem();
+                if (!group_sync(0x5302)) { ok = false; break; }
+                if (r == 0) mbar_arrive(&bars->in_ready);
+                // softmax of this query row: the maximum, then probabilities and their sum
+                if (!wwait(&bars->s_full, ph, 0x5303)) { ok = false; break; }
+                tc_fence_after();
+                float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll 1
+                for (int c = 0; c < 4; ++c) {
+                    const uint32_t grp2 = (a16 >> (2 * c)) & 3u;  // this row's 16-column groups of the chunk
+                    if (!__any_sync(0xFFFFFFFFu, grp2 != 0u)) continue;  // no row of the warp attends them
+                    uint32_t v[32];
+                    tmem_ld32(trow + kColS + 32 * c, v);
+                    tmem_wait_ld();
+                    if (grp2 != 3u) {
+#pragma unroll
+                        for (int e = 0; e < 32; ++e)
+                            if (!((grp2 >> (e >> 4)) & 1u)) v[e] = __float_as_uint(-INFINITY);
+                    }
+#pragma unroll
+                    for (int e = 0; e < 32; e += 2)
+                        mx4[(e >> 1) & 3] = fmax3(mx4[(e >> 1) & 3], __uint_as_float(v[e]), __uint_as_float(v[e + 1]));
+                }
+                const float m = fmaxf(fmax3(mx4[0], mx4[1], mx4[2]), mx4[3]) * sl2;  // a row always attends itself
+                float l4[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 1
+                for (int c = 0; c < 4; ++c) {
+                    if (!__any_sync(0xFFFFFFFFu, ((a16 >> (2 * c)) & 3u) != 0u)) {  // P = 0 for the whole warp
+                        const uint32_t z[16] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
+                        tmem_st16(trow + kColS + 16 * c, z);
+                        continue;
+                    }
+                    uint32_t v[32];
+                    tmem_ld32(trow + kColS + 32 * c, v);
+                    tmem_wait_ld();
+                    const float add0 = ((a16 >> (2 * c)) & 1u) ? -m : -INFINITY;
+                    const float add1 = ((a16 >> (2 * c + 1)) & 1u) ? -m : -INFINITY;
+                    uint32_t w[16];
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) {
+                        const float ad = e < 8 ? add0 : add1;
+                        float t0, t1;
+                        ffma2(t0, t1, __uint_as_float(v[2 * e]), __uint_as_float(v[2 * e + 1]), sl2, sl2, ad, ad);
+                        const float p0 = ex2_approx(t0), p1 = ex2_approx(t1);
+                        const int a = (e & 1) * 2;
+                        fadd2(l4[a], l4[a + 1], l4[a], l4[a + 1], p0, p1);
+                        w[e] = pack_bf16x2(p0, p1);
+                    }
+                    tmem_st16(trow + kColS + 16 * c, w);  // P over columns of S already read
+                }
+                const float l = (l4[0] + l4[1]) + (l4[2] + l4[3]);
+                tmem_wait_st();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&bars->p_ready);
+                // O_h / l into the head's o tile
+                if (!wwait(&bars->o_full, ph, 0x5304)) { ok = false; break; }
+                tc_fence_after();
+                uint32_t t[32];
+                tmem_ld32(trow + kColO, t);
+                tmem_wait_ld();
+                tc_fence_before();
+                // the previous item's y rows, staged over the o tiles, are stored
+                if (h == 0 && j > 0 && !wwait(&bars->y_done, static_cast<uint32_t>((j - 1) & 1), 0x5305)) {
+                    ok = false;
+                    break;
+                }
+                const float inv = 1.f / l;
+                float x[32];
+#pragma unroll
+                for (int e = 0; e < 32; ++e) x[e] = __uint_as_float(t[e]) * inv;
+                store_row_swz(smem + kOOff + h * kTileBytes, r, x);
+            }
+            if (!ok) break;
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bars->o_ready);
+            // y = Y + b_o into the staging tiles (the o tiles, read by the finished Y MMAs)
+            if (!wwait(&bars->y_full, static_cast<uint32_t>(j & 1), 0x5306)) break;
+            tc_fence_after();
+            for (int c = 0; c < heads; ++c) {
+                uint32_t t[32];
+                tmem_ld32(trow + kColY + 32 * c, t);
+                tmem_wait_ld();
+                const float* b = bias + 3 * kMaxHeads * kHeadDim + 32 * c;
+                float x[32];
+#pragma unroll
+                for (int e = 0; e < 32; ++e) x[e] = __uint_as_float(t[e]) + b[e];
+                store_row_swz(smem + kOOff + c * kTileBytes, r, x);
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) {
+                mbar_arrive(&bars->y_free);
+                mbar_arrive(&bars->staged);  // the mover stores them
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 0) tmem_dealloc(tmem, kTmemCols);
+}
+
+}  // namespace blockk
+
+cudaError_t launch_block_fwd(const Geo& g, const BlockPtrs& p, unsigned int* status, unsigned long long limit_ns,
+                             int num_sms, cudaStream_t stream) {
+    using namespace blockk;
+    static bool attr_set = false;
+    if (!attr_set) {
+        const cudaError_t e = cudaFuncSetAttribute(block_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+        if (e != cudaSuccess) return e;
+        attr_set = true;
+    }
+    Params prm;
+    prm.g = g;
+    prm.x = static_cast<const uint8_t*>(p.x);
+    prm.w_qkv = static_cast<const uint8_t*>(p.w_qkv);
+    prm.w_o = static_cast<const uint8_t*>(p.w_o);
+    prm.b_qkv = p.b_qkv;
+    prm.b_o = p.b_o;
+    prm.theta = p.theta;
+    prm.y = static_cast<uint8_t*>(p.y);
+    prm.status = status;
+    prm.limit_ns = limit_ns;
+    prm.items = g.tiles;
+    const long long grid = prm.items < num_sms ? prm.items : num_sms;
+    if (grid <= 0) return cudaSuccess;
+    block_kernel<<<static_cast<unsigned>(grid), kThreads, kSmemBytes, stream>>>(prm);
+    return cudaGetLastError();
+}
+
+}  // namespace fswin

@@ -47,4 +47,14 @@ cudaError_t launch_small_fwd(const Geo& g, const void* q, const void* k, const v
                              float* lse, unsigned int* status, unsigned long long limit_ns, int num_sms,
                              cudaStream_t stream);
 
+// The attention block with its projections (inference), windows of fewer than
+// 128 tokens, at most three heads: y = attention(x W_qkv^T + b_qkv) W_o^T + b_o.
+struct BlockPtrs {
+    const void *x, *w_qkv, *w_o;  // bf16 [B,H,W,C], [3C,C], [C,C]
+    const float *b_qkv, *b_o, *theta;
+    void* y;  // bf16 [B,H,W,C]
+};
+cudaError_t launch_block_fwd(const Geo& g, const BlockPtrs& p, unsigned int* status, unsigned long long limit_ns,
+                             int num_sms, cudaStream_t stream);
+
 }  // namespace fswin

@@ -60,6 +60,26 @@ def winattn_fwd(q, k, v, theta, M: int, s: int, o=None, lse=None, need_lse: bool
     return o, lse
 
 
+def winattn_block_fwd(x, w_qkv, b_qkv, w_o, b_o, theta, M: int, s: int, heads: int, y=None):
+    """y = windowed-RoPE attention of (x W_qkv^T + b_qkv) per head, then W_o, b_o
+    (the attention block of a Swin layer, inference; M*M < 128, heads <= 3)."""
+    B, H, W, C = x.shape
+    d = C // heads
+    sh = _lib.make_shape(B, H, W, heads, d, M, s)
+    _check_tensor("x", x, (B, H, W, C), torch.bfloat16)
+    _check_tensor("w_qkv", w_qkv, (3 * C, C), torch.bfloat16)
+    _check_tensor("b_qkv", b_qkv, (3 * C,), torch.float32)
+    _check_tensor("w_o", w_o, (C, C), torch.bfloat16)
+    _check_tensor("b_o", b_o, (C,), torch.float32)
+    _check_tensor("theta", theta, (heads, 2, d // 4), torch.float32)
+    if y is None:
+        y = torch.empty_like(x)
+    _check_tensor("y", y, (B, H, W, C), torch.bfloat16)
+    _lib.fs_winattn_block_fwd(sh, x.data_ptr(), w_qkv.data_ptr(), b_qkv.data_ptr(), w_o.data_ptr(), b_o.data_ptr(),
+                              theta.data_ptr(), y.data_ptr(), _stream(x.device))
+    return y
+
+
 def bwd_workspace_bytes(B: int, H: int, W: int, heads: int, M: int, s: int, d: int = HEAD_DIM) -> int:
     return _lib.fs_winattn_bwd_workspace_bytes(_lib.make_shape(B, H, W, heads, d, M, s))
 
