@@ -43,6 +43,12 @@ WORKLOADS = {
 }
 HEADLINE = "swin_t_stage1_p4_m8"
 
+# the window-attention block of a Swin layer with its qkv and output projections (inference),
+# Swin-T stage 1 at p=4: C = 96 channels in 3 heads, window 8, unshifted and shifted blocks
+BLOCK_WORKLOADS = {
+    "swin_t_stage1_p4_block_infer_m8": dict(B=128, H=64, W=64, heads=3, M=8, shifts=(0, 4)),
+}
+
 
 def unmasked_pairs(B, H, W, heads, M, s) -> int:
     """Number of (query, key) pairs that attend (same window, same shift-region label)."""
@@ -111,6 +117,15 @@ def workload_flops(wl) -> tuple[float, float]:
     """Useful forward and backward FLOPs of one step (fwd 4*d per pair, bwd 10*d per pair)."""
     pairs = sum(unmasked_pairs(wl["B"], wl["H"], wl["W"], wl["heads"], wl["M"], s) for s in wl["shifts"])
     return 4.0 * HEAD_DIM * pairs, 10.0 * HEAD_DIM * pairs
+
+
+def block_flops(wl) -> float:
+    """Useful FLOPs of one block step: the two projections (2 * 4 C^2 per token) and the
+    attention forward (4 d per attending pair), at every shift."""
+    C = wl["heads"] * HEAD_DIM
+    tokens = wl["B"] * wl["H"] * wl["W"]
+    pairs = sum(unmasked_pairs(wl["B"], wl["H"], wl["W"], wl["heads"], wl["M"], s) for s in wl["shifts"])
+    return 2.0 * 4 * C * C * tokens * len(wl["shifts"]) + 4.0 * HEAD_DIM * pairs
 
 
 def load_peaks():
@@ -205,6 +220,59 @@ def cpu_baseline(tensors, wl, seconds: float = 12.0):
     return {"value": flops / total_dt / 1e12, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
             "sample": f"(batch, window, head) units: {', '.join(parts)}; fwd+bwd, fp64, {total_dt:.1f} s",
             "seconds": total_dt}
+
+
+def run_block(wl, dev, rank, steps, warmup, peaks):
+    """The fused attention block (one kernel) and, for comparison, the same block unfused:
+    cuBLAS projections around this library's inference attention forward."""
+    import torch
+
+    from vision_transformer_windowed_b200 import dp, ops
+    from vision_transformer_windowed_b200.inputs import make_block_inputs
+    B, H, W, heads, M = wl["B"], wl["H"], wl["W"], wl["heads"], wl["M"]
+    C = heads * HEAD_DIM
+    t = make_block_inputs(B, H, W, heads, HEAD_DIM, device=dev)
+    x, wqkv, bqkv, wo, bo, th = t["x"], t["w_qkv"], t["b_qkv"], t["w_o"], t["b_o"], t["theta"]
+    y = torch.empty_like(x)
+    bqkv16, bo16 = bqkv.to(torch.bfloat16), bo.to(torch.bfloat16)
+
+    def fused():
+        for s in wl["shifts"]:
+            ops.winattn_block_fwd(x, wqkv, bqkv, wo, bo, th, M, s, heads, y=y)
+
+    def unfused():
+        for s in wl["shifts"]:
+            qkv = torch.nn.functional.linear(x, wqkv, bqkv16).view(B, H, W, 3, heads, HEAD_DIM)
+            q, k, v = (qkv[..., i, :, :].contiguous() for i in range(3))
+            o, _ = ops.winattn_fwd(q, k, v, th, M, s, need_lse=False)
+            y.copy_(torch.nn.functional.linear(o.view(B, H, W, C), wo, bo16))
+
+    def timed(fn):
+        for _ in range(warmup):
+            fn()
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        for _ in range(steps):
+            fn()
+        b.record()
+        torch.cuda.synchronize()
+        return dp.max_over_ranks(a.elapsed_time(b) / steps, dev)
+
+    ms = timed(fused)
+    ms_unfused = timed(unfused)
+    import torch.distributed as dist
+    world = dist.get_world_size() if dist.is_initialized() else 1
+    fl = block_flops(wl)
+    tokens = B * H * W * len(wl["shifts"])
+    gbs = tokens * 2 * C * 2 / (ms * 1e-3) / 1e9  # x read and y written once per token
+    return {"tflops": fl * world / (ms * 1e-3) / 1e12, "ms_per_step": ms,
+            "pct_bf16_peak": 100 * fl / (ms * 1e-3) / 1e12 / peaks["bf16_tflops"],
+            "tokens_per_s": tokens * world / (ms * 1e-3),
+            "hbm_gbs": gbs, "hbm_frac": gbs / peaks["hbm_gbs"],
+            "unfused_ms_per_step": ms_unfused,
+            "step": "attention block with qkv and output projections, inference, at every shift",
+            "unfused": "cuBLAS bf16 projections around the inference attention forward"}
 
 
 def run_reference(args):
@@ -464,6 +532,11 @@ def main():
             if WORKLOADS[name].get("infer"):
                 per_config[name]["step"] = "inference forward (no LSE) at every shift"
                 del per_config[name]["bwd_workspace_gb"]
+
+    if not args.no_extra:
+        for name, wl_b in BLOCK_WORKLOADS.items():
+            torch.cuda.empty_cache()
+            per_config[name] = run_block(wl_b, dev, rank, max(3, args.steps // 2), 3, peaks)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
