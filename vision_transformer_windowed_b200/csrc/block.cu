@@ -5,17 +5,23 @@
 // (the attention module of a FlashSwin block, thelatestinai.com 2610.04664,
 // Figure 1B).  One persistent kernel: a work item is one 128-slot tile with
 // all of its heads, so x is read and y written once per token, and q, k, v
-// and o never leave the chip.
-//   warps 0-3 (rows): thread = slot row = TMEM lane.  Per head: the biases
-//       and the RoPE of its q, k row (TMEM -> fp16 q', k' and bf16 v tiles),
-//       the softmax of its query row, O / l into the head's o tile; per item
-//       y + b_o into the staging tiles (the o tiles, once read).
-//   warp 4 (MMA): per head q|k|v = x [W_q,h; W_k,h; W_v,h]^T (N = 96, issued
-//       while the previous head's softmax runs), S = Q'K'^T, O_h = P V; per
-//       item Y = sum_h O_h W_o[:, 32h:32h+32]^T.
-//   warp 5 (mover): the item's x rows one item ahead (16-byte cp.async), then
-//       its y rows out.
-// The weights and biases stay in shared memory for the whole launch.
+// and o never leave the chip.  A CTA runs two items at a time (pipelines
+// p = 0, 1: alternate items of its run), each with its own 256 TMEM columns,
+// x buffer, head tiles, o tiles and barriers:
+//   warps 4p .. 4p+3 (rows of pipeline p): thread = slot row = TMEM lane.
+//       Per head: the biases and the RoPE of its q, k row (TMEM -> fp16 q',
+//       k' and bf16 v tiles), the softmax of its query row, O / l into the
+//       head's o tile; per item y + b_o into the staging tiles (the o tiles,
+//       once read).
+//   warp 8 (MMA): for either pipeline, whenever its next step is ready: per
+//       head q|k|v = x [W_q,h; W_k,h; W_v,h]^T (N = 96, issued while the
+//       previous head's softmax runs), S = Q'K'^T, O_h = P V; per item
+//       Y = sum_h O_h W_o[:, 32h:32h+32]^T.
+//   warp 9 (mover): x rows in (16-byte cp.async) as soon as a pipeline's x
+//       buffer is free, y rows out as soon as they are staged.
+// The MMA and mover warps poll the two pipelines' barriers without blocking,
+// within the usual time limit.  The weights and biases stay in shared memory
+// for the whole launch.
 #include <cuda.h>
 #include <cuda_runtime.h>
 
@@ -30,8 +36,9 @@ namespace fswin {
 namespace blockk {
 
 constexpr int kMaxHeads = 3;
-constexpr int kThreads = 192;
-constexpr int kWarpMma = 4, kWarpMover = 5;
+constexpr int kPipes = 2;
+constexpr int kThreads = 320;
+constexpr int kWarpMma = 8, kWarpMover = 9;
 constexpr int kQkvRows = 3 * kHeadDim;  // q, k, v rows of one head in a W_qkv chunk tile
 
 // Shared memory (offsets from a 1024-byte aligned base).  A weight "chunk" is
@@ -42,32 +49,39 @@ constexpr int kWqkvChunk = kMaxHeads * kQkvRows * kRowBytes;  // 18 KB
 constexpr int kWqkvOff = 0;
 constexpr int kWoChunk = kMaxHeads * kHeadDim * kRowBytes;    // 6 KB
 constexpr int kWoOff = kWqkvOff + kMaxHeads * kWqkvChunk;
-constexpr int kXBytes = kMaxHeads * kTileBytes;               // the x chunks of one item
-constexpr int kXOff = kWoOff + kMaxHeads * kWoChunk;          // 2 item buffers
-constexpr int kHeadOff = kXOff + 2 * kXBytes;                 // q' (fp16), k' (fp16), v (bf16) tiles of a head
-constexpr int kOOff = kHeadOff + 3 * kTileBytes;              // o tiles of the heads; then y staging
-constexpr int kBiasOff = kOOff + kMaxHeads * kTileBytes;      // b_qkv [3C], b_o [C] (fp32)
+// per pipeline: the x chunks of its item, a head's q' (fp16), k' (fp16), v
+// (bf16) tiles, the heads' o tiles (then the y staging)
+constexpr int kXBytes = kMaxHeads * kTileBytes;
+constexpr int kPipeBytes = kXBytes + 3 * kTileBytes + kMaxHeads * kTileBytes;
+constexpr int kPipeOff = kWoOff + kMaxHeads * kWoChunk;
+constexpr int kPX = 0, kPHead = kXBytes, kPO = kXBytes + 3 * kTileBytes;
+constexpr int kBiasOff = kPipeOff + kPipes * kPipeBytes;      // b_qkv [3C], b_o [C] (fp32)
 constexpr int kTabPerHead = 2 * 8 * 8;                        // [axis][pair][position < 8] float2
 constexpr int kTabOff = kBiasOff + 4 * kMaxHeads * kHeadDim * 4;
 constexpr int kBarOff = kTabOff + kMaxHeads * kTabPerHead * 8;
-constexpr int kSmemBytes = kBarOff + 256 + 1024;  // + alignment of the base
-static_assert(kXOff % 1024 == 0 && kHeadOff % 1024 == 0 && kOOff % 1024 == 0, "tile alignment");
+constexpr int kSmemBytes = kBarOff + 512 + 1024;  // + alignment of the base
+static_assert(kPipeOff % 1024 == 0 && kPipeBytes % 1024 == 0, "tile alignment");
 static_assert(kWoOff % 1024 == 0 && kWqkvChunk % 1024 == 0 && kWoChunk % 512 == 0, "weight tile alignment");
+static_assert(kSmemBytes <= 232448, "more shared memory than a CTA may have");
 
-// TMEM columns: q|k|v of a head [0, 96) (then Y [0, C)), O_h [96, 128),
-// S [128, 256) with P (bf16) written over its consumed columns.
-constexpr uint32_t kTmemCols = 256;
+// TMEM columns of pipeline p, from 256 p: q|k|v of a head [0, 96) (then Y
+// [0, C)), O_h [96, 128), S [128, 256) with P (bf16) over its consumed columns.
+constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColQKV = 0, kColY = 0, kColO = 96, kColS = 128;
 
-struct Bars {
-    uint64_t x_full[2], x_free[2];  // per item parity: x rows landed (32 mover lanes); last q|k|v MMAs done
+struct PipeBars {
+    uint64_t x_full, x_free;                               // per item: x landed (32 mover lanes); last q|k|v MMAs done
     uint64_t qkv_full, in_ready, s_full, p_ready, o_full;  // per head
     uint64_t o_ready, y_full, y_free, staged, y_done;      // per item
-    uint64_t grp, done;
+    uint64_t grp;                                          // the pipeline's four row warps
+};
+struct Bars {
+    PipeBars pp[kPipes];
+    uint64_t done;
     uint32_t tmem_base;
     int abort_flag;
 };
-static_assert(sizeof(Bars) <= 256, "barrier block overflows its slot");
+static_assert(sizeof(Bars) <= 512, "barrier block overflows its slot");
 
 struct Params {
     Geo g;
@@ -91,21 +105,22 @@ __global__ void __launch_bounds__(kThreads, 1) block_kernel(const __grid_constan
     float2* tabs = reinterpret_cast<float2*>(smem + kTabOff);
 
     if (tid == 0) {
-        for (int i = 0; i < 2; ++i) {
-            mbar_init(&bars->x_full[i], 32);  // one arrival per mover lane, once its copies have landed
-            mbar_init(&bars->x_free[i], 1);
+        for (int p = 0; p < kPipes; ++p) {
+            PipeBars& B = bars->pp[p];
+            mbar_init(&B.x_full, 32);  // one arrival per mover lane, once its copies have landed
+            mbar_init(&B.x_free, 1);
+            mbar_init(&B.qkv_full, 1);
+            mbar_init(&B.in_ready, 1);
+            mbar_init(&B.s_full, 1);
+            mbar_init(&B.p_ready, 4);
+            mbar_init(&B.o_full, 1);
+            mbar_init(&B.o_ready, 4);
+            mbar_init(&B.y_full, 1);
+            mbar_init(&B.y_free, 4);
+            mbar_init(&B.staged, 4);
+            mbar_init(&B.y_done, 1);
+            mbar_init(&B.grp, 4);
         }
-        mbar_init(&bars->qkv_full, 1);
-        mbar_init(&bars->in_ready, 1);
-        mbar_init(&bars->s_full, 1);
-        mbar_init(&bars->p_ready, 4);
-        mbar_init(&bars->o_full, 1);
-        mbar_init(&bars->o_ready, 4);
-        mbar_init(&bars->y_full, 1);
-        mbar_init(&bars->y_free, 4);
-        mbar_init(&bars->staged, 4);
-        mbar_init(&bars->y_done, 1);
-        mbar_init(&bars->grp, 4);
         mbar_init(&bars->done, 1);
         bars->abort_flag = 0;
         fence_mbar_init();
@@ -116,18 +131,18 @@ __global__ void __launch_bounds__(kThreads, 1) block_kernel(const __grid_constan
     }
     // weights (64-byte swizzled chunk tiles), biases and RoPE tables, once
     for (int i = tid; i < heads * 3 * C * 4; i += kThreads) {
-        const int p = i & 3, rest = i >> 2;
+        const int q16 = i & 3, rest = i >> 2;
         const int n = rest % (3 * C), c = rest / (3 * C);  // tile row n: head n / 96, then q, k, v rows
         const int hh = n / kQkvRows, part = (n % kQkvRows) / kHeadDim, e = n % kHeadDim;
-        const size_t src = static_cast<size_t>(part * C + hh * kHeadDim + e) * C + 32 * c + 8 * p;
-        *reinterpret_cast<uint4*>(smem + kWqkvOff + c * kWqkvChunk + n * kRowBytes + ((p ^ ((n >> 1) & 3)) << 4)) =
+        const size_t src = static_cast<size_t>(part * C + hh * kHeadDim + e) * C + 32 * c + 8 * q16;
+        *reinterpret_cast<uint4*>(smem + kWqkvOff + c * kWqkvChunk + n * kRowBytes + ((q16 ^ ((n >> 1) & 3)) << 4)) =
             *reinterpret_cast<const uint4*>(prm.w_qkv + 2 * src);
     }
     for (int i = tid; i < heads * C * 4; i += kThreads) {
-        const int p = i & 3, rest = i >> 2;
+        const int q16 = i & 3, rest = i >> 2;
         const int n = rest % C, c = rest / C;
-        const size_t src = static_cast<size_t>(n) * C + 32 * c + 8 * p;
-        *reinterpret_cast<uint4*>(smem + kWoOff + c * kWoChunk + n * kRowBytes + ((p ^ ((n >> 1) & 3)) << 4)) =
+        const size_t src = static_cast<size_t>(n) * C + 32 * c + 8 * q16;
+        *reinterpret_cast<uint4*>(smem + kWoOff + c * kWoChunk + n * kRowBytes + ((q16 ^ ((n >> 1) & 3)) << 4)) =
             *reinterpret_cast<const uint4*>(prm.w_o + 2 * src);
     }
     for (int i = tid; i < 3 * C; i += kThreads) bias[i] = prm.b_qkv[i];
@@ -139,10 +154,32 @@ __global__ void __launch_bounds__(kThreads, 1) block_kernel(const __grid_constan
     tc_fence_after();
     const uint32_t tmem = bars->tmem_base;
     const Ctl ctl{prm.status, &bars->abort_flag, prm.limit_ns};
-    // this CTA's items (tiles): a contiguous run
+    // this CTA's items (tiles): a contiguous run; pipeline p takes its items p, p + 2, ...
     const long long per = (prm.items + gridDim.x - 1) / gridDim.x;
     const long long first = static_cast<long long>(blockIdx.x) * per;
     const long long n = prm.items > first ? (prm.items - first < per ? prm.items - first : per) : 0;
+    auto pipe_base = [&](int p) { return smem + kPipeOff + p * kPipeBytes; };
+    // Polling with a time limit (MMA and mover warps): call after each round
+    // without progress; false once the limit is spent or another role aborted.
+    uint64_t t_idle = 0;
+    int idle_rounds = 0;
+    auto idle_ok = [&](bool progressed, unsigned int where) -> bool {
+        if (progressed) {
+            t_idle = 0;
+            idle_rounds = 0;
+            return true;
+        }
+        if (++idle_rounds < 64) return true;
+        idle_rounds = 0;
+        if (*ctl.abort_flag) return false;
+        const uint64_t now = globaltimer_ns();
+        if (t_idle == 0) t_idle = now;
+        if (now - t_idle <= ctl.limit_ns) return true;
+        atomicCAS(ctl.status, 0u, (kErrTimeout << 24) | (where & 0xFFFFFFu));
+        *ctl.abort_flag = 1;
+        __threadfence_block();
+        return false;
+    };
 
     if (warp == kWarpMma) {
         // ------------------------------------------------------------ MMA issue
@@ -155,57 +192,81 @@ __global__ void __launch_bounds__(kThreads, 1) block_kernel(const __grid_constan
             const uint64_t dK0 = make_sdesc(sbase, 16, 512, kSw64);     // K-major, 64-byte rows
             const uint64_t dMN0 = make_sdesc(sbase, 8192, 512, kSw64);  // MN-major, 64-byte rows
             auto u16 = [](int bytes) { return static_cast<uint64_t>(bytes >> 4); };
-            const uint64_t qo = u16(kHeadOff), ko = u16(kHeadOff + kTileBytes), vo = u16(kHeadOff + 2 * kTileBytes);
-            // q|k|v of head h for item j: x (its chunk tiles) times the head's 96 W_qkv rows
-            auto issue_qkv = [&](long long j, int h) {
-                const uint64_t xo = u16(kXOff + static_cast<int>(j & 1) * kXBytes);
+            // q|k|v of head h of pipeline p's item: x (its chunk tiles) times the head's 96 W_qkv rows
+            auto issue_qkv = [&](int p, int h) {
+                const int pb = kPipeOff + p * kPipeBytes;
                 for (int c = 0; c < heads; ++c)
 #pragma unroll
                     for (int ks = 0; ks < 2; ++ks)
-                        umma_ss(tmem + kColQKV, dK0 + xo + u16(c * kTileBytes) + 2 * ks,
+                        umma_ss(tmem + 256 * p + kColQKV, dK0 + u16(pb + kPX + c * kTileBytes) + 2 * ks,
                                 dK0 + u16(kWqkvOff + c * kWqkvChunk + h * kQkvRows * kRowBytes) + 2 * ks, id_qkv,
                                 (c | ks) != 0);
-                umma_commit(&bars->qkv_full);
+                umma_commit(&bars->pp[p].qkv_full);
             };
-            uint32_t hc = 0;
+            struct State {
+                long long jj;  // the pipeline's item (pipeline-local index)
+                int h, step;   // head; 0: item start, 1: S, 2: P V, 3: Y
+                uint32_t hc;   // heads done (phase of the per-head barriers)
+                bool done;
+            };
+            State st[kPipes];
+            for (int p = 0; p < kPipes; ++p) st[p] = State{0, 0, 0, 0u, p >= n};
             bool ok = true;
-            for (long long j = 0; j < n && ok; ++j) {
-                const int par = static_cast<int>(j & 1);
-                if (!mbar_wait(&bars->x_full[par], static_cast<uint32_t>((j >> 1) & 1), ctl, 0x5201)) break;
-                // the rows have read the previous item's Y, which q|k|v overwrite
-                if (j > 0 && !mbar_wait(&bars->y_free, static_cast<uint32_t>((j - 1) & 1), ctl, 0x5202)) break;
-                tc_fence_after();
-                issue_qkv(j, 0);
-                for (int h = 0; h < heads; ++h, ++hc) {
-                    const uint32_t ph = hc & 1u;
-                    // the rows have read this head's q|k|v and written its q', k', v tiles
-                    if (!mbar_wait(&bars->in_ready, ph, ctl, 0x5203)) { ok = false; break; }
-                    tc_fence_after();
+            while (ok && !(st[0].done && st[1].done)) {
+                bool prog = false;
+                for (int p = 0; p < kPipes; ++p) {
+                    State& S = st[p];
+                    if (S.done) continue;
+                    PipeBars& B = bars->pp[p];
+                    const uint32_t tb = tmem + 256 * p;
+                    const int pb = kPipeOff + p * kPipeBytes;
+                    if (S.step == 0) {  // the item's x landed; the rows have read the previous Y
+                        if (!mbar_test(&B.x_full, static_cast<uint32_t>(S.jj & 1))) continue;
+                        if (S.jj > 0 && !mbar_test(&B.y_free, static_cast<uint32_t>((S.jj - 1) & 1))) continue;
+                        tc_fence_after();
+                        issue_qkv(p, 0);
+                        S.h = 0;
+                        S.step = 1;
+                    } else if (S.step == 1) {  // the rows have read q|k|v and written q', k', v
+                        if (!mbar_test(&B.in_ready, S.hc & 1u)) continue;
+                        tc_fence_after();
 #pragma unroll
-                    for (int ks = 0; ks < kHeadDim / 16; ++ks)
-                        umma_ss(tmem + kColS, dK0 + qo + 2 * ks, dK0 + ko + 2 * ks, id_s, ks > 0);
-                    umma_commit(&bars->s_full);
-                    if (h + 1 < heads)
-                        issue_qkv(j, h + 1);  // during this head's softmax
-                    else
-                        umma_commit(&bars->x_free[par]);  // every MMA that reads the item's x is issued
-                    if (!mbar_wait(&bars->p_ready, ph, ctl, 0x5204)) { ok = false; break; }
-                    tc_fence_after();
+                        for (int ks = 0; ks < kHeadDim / 16; ++ks)
+                            umma_ss(tb + kColS, dK0 + u16(pb + kPHead) + 2 * ks,
+                                    dK0 + u16(pb + kPHead + kTileBytes) + 2 * ks, id_s, ks > 0);
+                        umma_commit(&B.s_full);
+                        if (S.h + 1 < heads)
+                            issue_qkv(p, S.h + 1);  // during this head's softmax
+                        else
+                            umma_commit(&B.x_free);  // every MMA that reads the item's x is issued
+                        S.step = 2;
+                    } else if (S.step == 2) {  // P written
+                        if (!mbar_test(&B.p_ready, S.hc & 1u)) continue;
+                        tc_fence_after();
 #pragma unroll
-                    for (int k = 0; k < kTile / 16; ++k)
-                        umma_ts(tmem + kColO, tmem + kColS + 8 * k, dMN0 + vo + 64 * k, id_pv, k > 0);
-                    umma_commit(&bars->o_full);
+                        for (int k = 0; k < kTile / 16; ++k)
+                            umma_ts(tb + kColO, tb + kColS + 8 * k, dMN0 + u16(pb + kPHead + 2 * kTileBytes) + 64 * k,
+                                    id_pv, k > 0);
+                        umma_commit(&B.o_full);
+                        ++S.hc;
+                        ++S.h;
+                        S.step = S.h < heads ? 1 : 3;
+                    } else {  // every o tile written: Y
+                        if (!mbar_test(&B.o_ready, static_cast<uint32_t>(S.jj & 1))) continue;
+                        tc_fence_after();
+                        for (int h = 0; h < heads; ++h)
+#pragma unroll
+                            for (int ks = 0; ks < 2; ++ks)
+                                umma_ss(tb + kColY, dK0 + u16(pb + kPO + h * kTileBytes) + 2 * ks,
+                                        dK0 + u16(kWoOff + h * kWoChunk) + 2 * ks, id_y, (h | ks) != 0);
+                        umma_commit(&B.y_full);
+                        ++S.jj;
+                        S.step = 0;
+                        S.done = p + 2 * S.jj >= n;
+                    }
+                    prog = true;
                 }
-                if (!ok) break;
-                // Y = sum over heads of O_h W_o[:, 32h:32h+32]^T, once every o tile is written
-                if (!mbar_wait(&bars->o_ready, static_cast<uint32_t>(j & 1), ctl, 0x5205)) break;
-                tc_fence_after();
-                for (int h = 0; h < heads; ++h)
-#pragma unroll
-                    for (int ks = 0; ks < 2; ++ks)
-                        umma_ss(tmem + kColY, dK0 + u16(kOOff + h * kTileBytes) + 2 * ks,
-                                dK0 + u16(kWoOff + h * kWoChunk) + 2 * ks, id_y, (h | ks) != 0);
-                umma_commit(&bars->y_full);
+                ok = idle_ok(prog, 0x5201);
             }
             umma_commit(&bars->done);
             mbar_wait(&bars->done, 0, ctl, 0x52ff);
@@ -215,9 +276,6 @@ __global__ void __launch_bounds__(kThreads, 1) block_kernel(const __grid_constan
         // ------------------------------------------------------------ x rows in, y rows out
         // Lane l moves 16-byte chunk l % 4 of row 8 i + l / 4 of each group of 32
         // rows: every instruction moves 8 whole 64-byte rows of one chunk tile.
-        auto mwait = [&](uint64_t* bar, uint32_t ph, unsigned int where) -> bool {
-            return __all_sync(0xFFFFFFFFu, mbar_wait(bar, ph, ctl, where));
-        };
         long long mv_X = -1, mv_t[4] = {0, 0, 0, 0};  // token (B, H, W index) of rows lane + 32 q
         bool mv_valid[4] = {false, false, false, false};
         auto geo = [&](long long X) {
@@ -231,9 +289,10 @@ __global__ void __launch_bounds__(kThreads, 1) block_kernel(const __grid_constan
                 mv_t[q] = tok0 / heads;
             }
         };
-        auto move = [&](long long j, bool load) {
+        // item j of the run through pipeline p's x buffer (load) or o tiles (store)
+        auto move = [&](long long j, int p, bool load) {
             geo(first + j);
-            uint8_t* xb = smem + kXOff + static_cast<int>(j & 1) * kXBytes;
+            uint8_t* pb = pipe_base(p);
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
 #pragma unroll
@@ -246,43 +305,72 @@ __global__ void __launch_bounds__(kThreads, 1) block_kernel(const __grid_constan
                     const long long go = t * C * 2 + 16 * cp;
                     for (int c = 0; c < heads; ++c) {
                         if (load)
-                            cp_async16(smem_u32(xb + c * kTileBytes + off), valid ? prm.x + go + 64 * c : prm.x,
+                            cp_async16(smem_u32(pb + kPX + c * kTileBytes + off), valid ? prm.x + go + 64 * c : prm.x,
                                        valid ? 16u : 0u);
                         else if (valid)
                             *reinterpret_cast<uint4*>(prm.y + go + 64 * c) =
-                                *reinterpret_cast<const uint4*>(smem + kOOff + c * kTileBytes + off);
+                                *reinterpret_cast<const uint4*>(pb + kPO + c * kTileBytes + off);
                     }
                 }
             }
         };
-        // Each lane waits for its own copies and fences them for the tensor
-        // core (the async proxy) before it arrives.
-        auto load = [&](long long j) {
-            move(j, true);
+        // each lane waits for its own copies and fences them for the tensor core
+        // (the async proxy) before it arrives
+        auto load = [&](long long j, int p) {
+            move(j, p, true);
             cp_async_commit();
             cp_async_wait<0>();
             fence_proxy_async_smem();
-            mbar_arrive(&bars->x_full[j & 1]);
+            mbar_arrive(&bars->pp[p].x_full);
         };
-        if (n > 0) load(0);
-        if (n > 1) load(1);
-        for (long long j = 0; j < n; ++j) {
-            if (j + 2 < n) {  // item j+2's x once item j's q|k|v MMAs are done with the buffer
-                if (!mwait(&bars->x_free[j & 1], static_cast<uint32_t>((j >> 1) & 1), 0x5401)) break;
-                load(j + 2);
+        long long ld[kPipes], stj[kPipes];  // next item (pipeline-local) to load, to store
+        for (int p = 0; p < kPipes; ++p) {
+            ld[p] = 0;
+            stj[p] = 0;
+            if (p < n) {
+                load(p, p);
+                ld[p] = 1;
             }
-            if (!mwait(&bars->staged, static_cast<uint32_t>(j & 1), 0x5402)) break;
-            move(j, false);
-            __syncwarp();  // every lane has read the staged rows: the rows may write o tiles again
-            if (lane == 0) mbar_arrive(&bars->y_done);
+        }
+        bool ok = true;
+        while (ok) {
+            bool prog = false, left = false;
+            for (int p = 0; p < kPipes; ++p) {
+                PipeBars& B = bars->pp[p];
+                const long long jl = p + 2 * ld[p];  // x of the next item once the previous one's is consumed
+                if (jl < n) {
+                    left = true;
+                    if (__all_sync(0xFFFFFFFFu, mbar_test(&B.x_free, static_cast<uint32_t>((ld[p] - 1) & 1)))) {
+                        load(jl, p);
+                        ++ld[p];
+                        prog = true;
+                    }
+                }
+                const long long js = p + 2 * stj[p];
+                if (js < n) {
+                    left = true;
+                    if (__all_sync(0xFFFFFFFFu, mbar_test(&B.staged, static_cast<uint32_t>(stj[p] & 1)))) {
+                        move(js, p, false);
+                        __syncwarp();  // every lane has read the staged rows
+                        if (lane == 0) mbar_arrive(&B.y_done);
+                        ++stj[p];
+                        prog = true;
+                    }
+                }
+            }
+            if (!left) break;
+            ok = __all_sync(0xFFFFFFFFu, idle_ok(prog, 0x5401));
         }
         cp_async_wait<0>();
     } else {
-        // ------------------------------------------------------------ rows (warps 0-3)
-        const int r = tid;
-        const uint32_t trow = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+        // ------------------------------------------------------------ rows (warps 0-7)
+        const int p = warp >> 2, wq = warp & 3;
+        const int r = wq * 32 + lane;
+        PipeBars& B = bars->pp[p];
+        uint8_t* pb = pipe_base(p);
+        const uint32_t trow = tmem + 256 * p + (static_cast<uint32_t>(wq * 32) << 16);
         const float sl2 = g.scale_log2;
-        uint8_t* qt = smem + kHeadOff;
+        uint8_t* qt = pb + kPHead;
         uint8_t* kt = qt + kTileBytes;
         uint8_t* vt = qt + 2 * kTileBytes;
         uint32_t gph = 0, hc = 0;
@@ -292,13 +380,13 @@ __global__ void __launch_bounds__(kThreads, 1) block_kernel(const __grid_constan
         };
         auto group_sync = [&](unsigned int where) -> bool {
             __syncwarp();
-            if (lane == 0) mbar_arrive(&bars->grp);
-            const bool passed = wwait(&bars->grp, gph, where);
+            if (lane == 0) mbar_arrive(&B.grp);
+            const bool passed = wwait(&B.grp, gph, where);
             gph ^= 1;
             return passed;
         };
-        for (long long j = 0; j < n && ok; ++j) {
-            const long long X = first + j;
+        for (long long jj = 0; p + 2 * jj < n && ok; ++jj) {
+            const long long X = first + p + 2 * jj;
             int pi, pj;
             long long tok0;
             slot_token(g, X, r, 0, &pi, &pj, &tok0);
@@ -308,7 +396,7 @@ __global__ void __launch_bounds__(kThreads, 1) block_kernel(const __grid_constan
                 const uint32_t ph = hc & 1u;
                 const float2* tab = tabs + h * kTabPerHead;
                 // q, k, v of this row and head: + biases, RoPE of q and k, into the head's tiles
-                if (!wwait(&bars->qkv_full, ph, 0x5301)) { ok = false; break; }
+                if (!wwait(&B.qkv_full, ph, 0x5301)) { ok = false; break; }
                 tc_fence_after();
 #pragma unroll 1
                 for (int part = 0; part < 3; ++part) {
@@ -325,9 +413,9 @@ __global__ void __launch_bounds__(kThreads, 1) block_kernel(const __grid_constan
                 tc_fence_before();
                 fence_proxy_async_smem();
                 if (!group_sync(0x5302)) { ok = false; break; }
-                if (r == 0) mbar_arrive(&bars->in_ready);
+                if (r == 0) mbar_arrive(&B.in_ready);
                 // softmax of this query row: the maximum, then probabilities and their sum
-                if (!wwait(&bars->s_full, ph, 0x5303)) { ok = false; break; }
+                if (!wwait(&B.s_full, ph, 0x5303)) { ok = false; break; }
                 tc_fence_after();
                 float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll 1
@@ -377,16 +465,16 @@ __global__ void __launch_bounds__(kThreads, 1) block_kernel(const __grid_constan
                 tmem_wait_st();
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&bars->p_ready);
+                if (lane == 0) mbar_arrive(&B.p_ready);
                 // O_h / l into the head's o tile
-                if (!wwait(&bars->o_full, ph, 0x5304)) { ok = false; break; }
+                if (!wwait(&B.o_full, ph, 0x5304)) { ok = false; break; }
                 tc_fence_after();
                 uint32_t t[32];
                 tmem_ld32(trow + kColO, t);
                 tmem_wait_ld();
                 tc_fence_before();
-                // the previous item's y rows, staged over the o tiles, are stored
-                if (h == 0 && j > 0 && !wwait(&bars->y_done, static_cast<uint32_t>((j - 1) & 1), 0x5305)) {
+                // the pipeline's previous y rows, staged over the o tiles, are stored
+                if (h == 0 && jj > 0 && !wwait(&B.y_done, static_cast<uint32_t>((jj - 1) & 1), 0x5305)) {
                     ok = false;
                     break;
                 }
@@ -394,14 +482,14 @@ __global__ void __launch_bounds__(kThreads, 1) block_kernel(const __grid_constan
                 float x[32];
 #pragma unroll
                 for (int e = 0; e < 32; ++e) x[e] = __uint_as_float(t[e]) * inv;
-                store_row_swz(smem + kOOff + h * kTileBytes, r, x);
+                store_row_swz(pb + kPO + h * kTileBytes, r, x);
             }
             if (!ok) break;
             fence_proxy_async_smem();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&bars->o_ready);
+            if (lane == 0) mbar_arrive(&B.o_ready);
             // y = Y + b_o into the staging tiles (the o tiles, read by the finished Y MMAs)
-            if (!wwait(&bars->y_full, static_cast<uint32_t>(j & 1), 0x5306)) break;
+            if (!wwait(&B.y_full, static_cast<uint32_t>(jj & 1), 0x5306)) break;
             tc_fence_after();
             for (int c = 0; c < heads; ++c) {
                 uint32_t t[32];
@@ -411,13 +499,13 @@ __global__ void __launch_bounds__(kThreads, 1) block_kernel(const __grid_constan
                 float x[32];
 #pragma unroll
                 for (int e = 0; e < 32; ++e) x[e] = __uint_as_float(t[e]) + b[e];
-                store_row_swz(smem + kOOff + c * kTileBytes, r, x);
+                store_row_swz(pb + kPO + c * kTileBytes, r, x);
             }
             tc_fence_before();
             __syncwarp();
             if (lane == 0) {
-                mbar_arrive(&bars->y_free);
-                mbar_arrive(&bars->staged);  // the mover stores them
+                mbar_arrive(&B.y_free);
+                mbar_arrive(&B.staged);  // the mover stores them
             }
         }
     }
