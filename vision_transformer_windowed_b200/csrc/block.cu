@@ -17,10 +17,10 @@
 //       head q|k|v = x [W_q,h; W_k,h; W_v,h]^T (N = 96, issued while the
 //       previous head's softmax runs), S = Q'K'^T, O_h = P V; per item
 //       Y = sum_h O_h W_o[:, 32h:32h+32]^T.
-//   warp 9 (mover): x rows in (16-byte cp.async) as soon as a pipeline's x
-//       buffer is free, y rows out as soon as they are staged.
-// The MMA and mover warps poll the two pipelines' barriers without blocking,
-// within the usual time limit.  The weights and biases stay in shared memory
+//   warp 9 + p (mover of pipeline p): x rows in (16-byte cp.async) as soon as
+//       the pipeline's x buffer is free, y rows out as soon as they are staged.
+// The MMA warp polls the two pipelines' barriers without blocking, within the
+// usual time limit.  The weights and biases stay in shared memory
 // for the whole launch.
 #include <cuda.h>
 #include <cuda_runtime.h>
@@ -37,8 +37,8 @@ namespace blockk {
 
 constexpr int kMaxHeads = 3;
 constexpr int kPipes = 2;
-constexpr int kThreads = 320;
-constexpr int kWarpMma = 8, kWarpMover = 9;
+constexpr int kThreads = 352;
+constexpr int kWarpMma = 8, kWarpMover = 9;  // movers: warps 9 and 10
 constexpr int kQkvRows = 3 * kHeadDim;  // q, k, v rows of one head in a W_qkv chunk tile
 
 // Shared memory (offsets from a 1024-byte aligned base).  A weight "chunk" is
@@ -272,10 +272,16 @@ __global__ void __launch_bounds__(kThreads, 1) block_kernel(const __grid_constan
             mbar_wait(&bars->done, 0, ctl, 0x52ff);
         }
         __syncwarp();
-    } else if (warp == kWarpMover) {
-        // ------------------------------------------------------------ x rows in, y rows out
+    } else if (warp >= kWarpMover) {
+        // ------------------------------------------------------------ x rows in, y rows out (pipeline p)
         // Lane l moves 16-byte chunk l % 4 of row 8 i + l / 4 of each group of 32
         // rows: every instruction moves 8 whole 64-byte rows of one chunk tile.
+        const int p = warp - kWarpMover;
+        PipeBars& B = bars->pp[p];
+        uint8_t* pb = pipe_base(p);
+        auto mwait = [&](uint64_t* bar, uint32_t ph, unsigned int where) -> bool {
+            return __all_sync(0xFFFFFFFFu, mbar_wait(bar, ph, ctl, where));
+        };
         long long mv_X = -1, mv_t[4] = {0, 0, 0, 0};  // token (B, H, W index) of rows lane + 32 q
         bool mv_valid[4] = {false, false, false, false};
         auto geo = [&](long long X) {
@@ -289,10 +295,11 @@ __global__ void __launch_bounds__(kThreads, 1) block_kernel(const __grid_constan
                 mv_t[q] = tok0 / heads;
             }
         };
-        // item j of the run through pipeline p's x buffer (load) or o tiles (store)
-        auto move = [&](long long j, int p, bool load) {
+        // x rows of item j into the pipeline's x buffer; each lane waits for its
+        // own copies and fences them for the tensor core (the async proxy)
+        // before it arrives
+        auto load = [&](long long j) {
             geo(first + j);
-            uint8_t* pb = pipe_base(p);
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
 #pragma unroll
@@ -303,63 +310,57 @@ __global__ void __launch_bounds__(kThreads, 1) block_kernel(const __grid_constan
                     const int row = 32 * q + sl_lane;
                     const uint32_t off = row * kRowBytes + ((cp ^ ((row >> 1) & 3)) << 4);
                     const long long go = t * C * 2 + 16 * cp;
-                    for (int c = 0; c < heads; ++c) {
-                        if (load)
-                            cp_async16(smem_u32(pb + kPX + c * kTileBytes + off), valid ? prm.x + go + 64 * c : prm.x,
-                                       valid ? 16u : 0u);
-                        else if (valid)
-                            *reinterpret_cast<uint4*>(prm.y + go + 64 * c) =
-                                *reinterpret_cast<const uint4*>(pb + kPO + c * kTileBytes + off);
-                    }
+                    for (int c = 0; c < heads; ++c)
+                        cp_async16(smem_u32(pb + kPX + c * kTileBytes + off), valid ? prm.x + go + 64 * c : prm.x,
+                                   valid ? 16u : 0u);
                 }
             }
-        };
-        // each lane waits for its own copies and fences them for the tensor core
-        // (the async proxy) before it arrives
-        auto load = [&](long long j, int p) {
-            move(j, p, true);
             cp_async_commit();
             cp_async_wait<0>();
             fence_proxy_async_smem();
-            mbar_arrive(&bars->pp[p].x_full);
+            mbar_arrive(&B.x_full);
         };
-        long long ld[kPipes], stj[kPipes];  // next item (pipeline-local) to load, to store
-        for (int p = 0; p < kPipes; ++p) {
-            ld[p] = 0;
-            stj[p] = 0;
-            if (p < n) {
-                load(p, p);
-                ld[p] = 1;
-            }
-        }
-        bool ok = true;
-        while (ok) {
-            bool prog = false, left = false;
-            for (int p = 0; p < kPipes; ++p) {
-                PipeBars& B = bars->pp[p];
-                const long long jl = p + 2 * ld[p];  // x of the next item once the previous one's is consumed
-                if (jl < n) {
-                    left = true;
-                    if (__all_sync(0xFFFFFFFFu, mbar_test(&B.x_free, static_cast<uint32_t>((ld[p] - 1) & 1)))) {
-                        load(jl, p);
-                        ++ld[p];
-                        prog = true;
-                    }
+        // y rows of item j from the staging tiles: per group of 32 rows, all
+        // shared loads first, then the global stores
+        auto store = [&](long long j) {
+            geo(first + j);
+            const uint32_t s0 = smem_u32(pb + kPO);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                uint4 v[4][kMaxHeads];
+                long long go[4];
+                bool valid[4];
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const int sl_lane = 8 * i + (lane >> 2), cp = lane & 3;
+                    go[i] = __shfl_sync(0xFFFFFFFFu, mv_t[q], sl_lane) * C * 2 + 16 * cp;
+                    valid[i] = __shfl_sync(0xFFFFFFFFu, mv_valid[q] ? 1 : 0, sl_lane) != 0;
+                    const int row = 32 * q + sl_lane;
+                    const uint32_t off = row * kRowBytes + ((cp ^ ((row >> 1) & 3)) << 4);
+#pragma unroll
+                    for (int c = 0; c < kMaxHeads; ++c)
+                        if (c < heads) v[i][c] = ld_shared_v4(s0 + c * kTileBytes + off);
                 }
-                const long long js = p + 2 * stj[p];
-                if (js < n) {
-                    left = true;
-                    if (__all_sync(0xFFFFFFFFu, mbar_test(&B.staged, static_cast<uint32_t>(stj[p] & 1)))) {
-                        move(js, p, false);
-                        __syncwarp();  // every lane has read the staged rows
-                        if (lane == 0) mbar_arrive(&B.y_done);
-                        ++stj[p];
-                        prog = true;
+#pragma unroll
+                for (int i = 0; i < 4; ++i)
+                    if (valid[i]) {
+#pragma unroll
+                        for (int c = 0; c < kMaxHeads; ++c)
+                            if (c < heads) st_global_v4(prm.y + go[i] + 64 * c, v[i][c]);
                     }
-                }
             }
-            if (!left) break;
-            ok = __all_sync(0xFFFFFFFFu, idle_ok(prog, 0x5401));
+        };
+        const long long count = p < n ? (n - p + 1) / 2 : 0;  // the pipeline's items: p, p + 2, ...
+        if (count > 0) load(p);
+        for (long long jj = 0; jj < count; ++jj) {
+            if (jj + 1 < count) {  // the next item's x once this item's q|k|v MMAs are done with the buffer
+                if (!mwait(&B.x_free, static_cast<uint32_t>(jj & 1), 0x5401)) break;
+                load(p + 2 * (jj + 1));
+            }
+            if (!mwait(&B.staged, static_cast<uint32_t>(jj & 1), 0x5402)) break;
+            store(p + 2 * jj);
+            __syncwarp();  // every lane has read the staged rows
+            if (lane == 0) mbar_arrive(&B.y_done);
         }
         cp_async_wait<0>();
     } else {
