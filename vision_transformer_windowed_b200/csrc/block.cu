@@ -202,6 +202,9 @@ __global__ void __launch_bounds__(kThreads, 1) block_kernel(const __grid_constan
                                 dK0 + u16(kWqkvOff + c * kWqkvChunk + h * kQkvRows * kRowBytes) + 2 * ks, id_qkv,
                                 (c | ks) != 0);
                 umma_commit(&bars->pp[p].qkv_full);
+                // the last head's q|k|v is the last MMA that reads the item's x:
+                // the mover may refill the buffer once it completes
+                if (h == heads - 1) umma_commit(&bars->pp[p].x_free);
             };
             struct State {
                 long long jj;  // the pipeline's item (pipeline-local index)
@@ -235,10 +238,7 @@ __global__ void __launch_bounds__(kThreads, 1) block_kernel(const __grid_constan
                             umma_ss(tb + kColS, dK0 + u16(pb + kPHead) + 2 * ks,
                                     dK0 + u16(pb + kPHead + kTileBytes) + 2 * ks, id_s, ks > 0);
                         umma_commit(&B.s_full);
-                        if (S.h + 1 < heads)
-                            issue_qkv(p, S.h + 1);  // during this head's softmax
-                        else
-                            umma_commit(&B.x_free);  // every MMA that reads the item's x is issued
+                        if (S.h + 1 < heads) issue_qkv(p, S.h + 1);  // during this head's softmax
                         S.step = 2;
                     } else if (S.step == 2) {  // P written
                         if (!mbar_test(&B.p_ready, S.hc & 1u)) continue;
