@@ -130,7 +130,10 @@ def full(q, k, v, theta, M: int, s: int, dout=None, nthreads: int | None = None)
     q, k, v, dout: [B, H, W, heads, d] (bf16 torch tensors or bit arrays are
     upcast exactly; float arrays are used as is).  theta: [heads, 2, d/4].
     Returns float64 arrays at original token positions: o, lse [B,H,W,heads]
-    and, with dout, dq, dk, dv and dtheta [heads, 2, d/4].
+    and, with dout, dq, dk, dv and dtheta [heads, 2, d/4].  H or W that is not
+    a multiple of M is padded with zero tokens up to the next multiple (the
+    Swin layer's padding); the windows, the shift and its mask then refer to
+    the padded grid.
     """
     qa, qi = _as_input(q)
     ka, ki = _as_input(k)
@@ -160,8 +163,10 @@ def full(q, k, v, theta, M: int, s: int, dout=None, nthreads: int | None = None)
 def units(q, k, v, theta, M: int, s: int, unit_ids, dout=None, nthreads: int | None = None) -> dict:
     """Forward (and backward with ``dout``) for selected (batch, window, head) units.
 
-    unit = (b * nW + w) * heads + h, windows w = wr * (W/M) + wc in the rolled
-    frame.  Outputs are per unit in window-local token order t = i*M + j:
+    unit = (b * nW + w) * heads + h, windows w = wr * (Wp/M) + wc in the rolled
+    frame of the padded grid (Hp, Wp = H, W rounded up to multiples of M).
+    Outputs are per unit in window-local token order t = i*M + j, padded tokens
+    included:
     o, dq, dk, dv [n, M*M, d]; lse [n, M*M]; dtheta [n, 2, d/4] (the unit's share).
     """
     qa, qi = _as_input(q)
@@ -193,13 +198,17 @@ def units(q, k, v, theta, M: int, s: int, unit_ids, dout=None, nthreads: int | N
 
 
 def unit_token_positions(H: int, W: int, M: int, s: int, unit: int, heads: int):
-    """Original (b, row, col, head) of every token of a unit, in window-local order."""
-    nWw = W // M
-    nW = (H // M) * nWw
+    """Original (b, row, col, head) of every token of a unit, in window-local order.
+
+    Positions of padded tokens (grids that are not multiples of M) have
+    row >= H or col >= W."""
+    Hp, Wp = -(-H // M) * M, -(-W // M) * M
+    nWw = Wp // M
+    nW = (Hp // M) * nWw
     b, rem = divmod(unit, nW * heads)
     w, h = divmod(rem, heads)
     wr, wc = divmod(w, nWw)
     t = np.arange(M * M)
-    rows = (wr * M + t // M + s) % H
-    cols = (wc * M + t % M + s) % W
+    rows = (wr * M + t // M + s) % Hp
+    cols = (wc * M + t % M + s) % Wp
     return b, rows, cols, h

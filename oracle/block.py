@@ -15,7 +15,10 @@ map.  Written out as that definition:
 
 The projections are fp64 matrix products (a library primitive); the attention
 is the C oracle.  The shift needs no separate handling: the projections act
-token by token, so they commute with the cyclic roll of the windows.
+token by token, so they commute with the cyclic roll of the windows.  A grid
+that is not a multiple of M is padded as a Swin layer pads it: x gets zero
+tokens up to the next multiple of M before the qkv map (so padded q, k, v
+equal the bias), attention runs on the padded grid, and y is cropped.
 """
 from __future__ import annotations
 
@@ -46,8 +49,12 @@ def project_qkv(x, w_qkv, b_qkv, heads: int):
 
 def block_forward(x, w_qkv, b_qkv, w_o, b_o, theta, M: int, s: int, heads: int, nthreads: int | None = None):
     """y [B, H, W, C] (float64) of the attention block; also returns the attention output o."""
-    q, k, v = project_qkv(x, w_qkv, b_qkv, heads)
-    o = full(q, k, v, theta, M, s, nthreads=nthreads)["o"]  # [B, H, W, heads, d]
-    B, H, W = o.shape[:3]
+    x = _f64(x)
+    B, H, W, C = x.shape
+    Hp, Wp = -(-H // M) * M, -(-W // M) * M
+    xp = np.zeros((B, Hp, Wp, C))
+    xp[:, :H, :W] = x
+    q, k, v = project_qkv(xp, w_qkv, b_qkv, heads)
+    o = full(q, k, v, theta, M, s, nthreads=nthreads)["o"][:, :H, :W]  # [B, H, W, heads, d]
     of = o.reshape(B, H, W, -1)
     return of @ _f64(w_o).T + _f64(b_o), o

@@ -27,7 +27,13 @@
  *  - with s > 0, query and key attend only when their region labels agree:
  *    label = 3*l(r) + l(c), l(x) = 0 for x < X-M, 1 for x < X-s, 2 otherwise;
  *    masked scores are -infinity (never an additive constant);
- *  - log-sum-exp is the natural logarithm.
+ *  - log-sum-exp is the natural logarithm;
+ *  - a grid whose H or W is not a multiple of M is first padded at the bottom
+ *    and right to Hp = ceil(H/M)*M, Wp = ceil(W/M)*M with zero tokens (zero q,
+ *    k, v and upstream gradient), as a Swin layer pads its input before the
+ *    shift; the roll, the windows and the region labels then refer to the
+ *    padded grid, padded tokens take part in the softmax like any other token,
+ *    and only the H x W real positions are written back.
  *
  * Gradients are those of L = sum(O * dO) for the upstream gradient dO.
  */
@@ -77,7 +83,7 @@ int fso_check_shape(const fso_shape* sh) {
     if (!sh) return 1;
     if (sh->B < 0 || sh->H <= 0 || sh->W <= 0 || sh->heads <= 0 || sh->d <= 0 || sh->M <= 0) return 2;
     if (sh->d % 4) return 2;
-    if (sh->H % sh->M || sh->W % sh->M) return 2;
+    if (sh->H < sh->M || sh->W < sh->M) return 2;
     if (sh->s < 0 || sh->s >= sh->M) return 2;
     return 0;
 }
@@ -111,13 +117,17 @@ typedef struct {
     int status;
 } fso_job;
 
+/* Padded grid extent: X rounded up to a multiple of M. */
+static int fso_padded(int X, int M) { return (X + M - 1) / M * M; }
+
 /* One (batch, window, head) unit.  Outputs are in window-local token order
- * t = i*M + j. */
+ * t = i*M + j (padded tokens included). */
 static int fso_one_unit(const fso_job* jb, int64_t unit, double* o, double* lse, double* dq, double* dk,
                         double* dv, double* dth) {
     const fso_shape* sh = jb->sh;
     const int H = sh->H, W = sh->W, heads = sh->heads, d = sh->d, M = sh->M, s = sh->s;
-    const int nWw = W / M, nW = (H / M) * nWw, N = M * M;
+    const int Hp = fso_padded(H, M), Wp = fso_padded(W, M);
+    const int nWw = Wp / M, nW = (Hp / M) * nWw, N = M * M;
     const int64_t b = unit / ((int64_t)nW * heads);
     const int64_t rem = unit % ((int64_t)nW * heads);
     const int w = (int)(rem / heads), h = (int)(rem % heads);
@@ -139,17 +149,19 @@ static int fso_one_unit(const fso_job* jb, int64_t unit, double* o, double* lse,
     for (int t = 0; t < N; ++t) {
         int i = t / M, j = t % M;
         int r = wr * M + i, c = wc * M + j;
-        int ro = (r + s) % H, co = (c + s) % W;
-        int64_t base = ((((int64_t)b * H + ro) * W + co) * heads + h) * d;
-        for (int e = 0; e < d; ++e) {
-            qr[(size_t)t * d + e] = fso_load(jb->q, base + e);
-            kr[(size_t)t * d + e] = fso_load(jb->k, base + e);
-            vv[(size_t)t * d + e] = fso_load(jb->v, base + e);
-            if (bwd) go[(size_t)t * d + e] = fso_load(jb->dout, base + e);
+        int ro = (r + s) % Hp, co = (c + s) % Wp;
+        if (ro < H && co < W) { /* a padded token keeps the zeros of calloc */
+            int64_t base = ((((int64_t)b * H + ro) * W + co) * heads + h) * d;
+            for (int e = 0; e < d; ++e) {
+                qr[(size_t)t * d + e] = fso_load(jb->q, base + e);
+                kr[(size_t)t * d + e] = fso_load(jb->k, base + e);
+                vv[(size_t)t * d + e] = fso_load(jb->v, base + e);
+                if (bwd) go[(size_t)t * d + e] = fso_load(jb->dout, base + e);
+            }
         }
         rope_rotate(qr + (size_t)t * d, d, j, i, th, 0);
         rope_rotate(kr + (size_t)t * d, d, j, i, th, 0);
-        lab[t] = 3 * fso_axis_region(H, M, s, r) + fso_axis_region(W, M, s, c);
+        lab[t] = 3 * fso_axis_region(Hp, M, s, r) + fso_axis_region(Wp, M, s, c);
     }
 
     /* Steps 3-5, one query row at a time. */
@@ -236,8 +248,8 @@ static void* fso_worker(void* arg) {
 
 /*
  * Forward (and, when dout and dq/dk/dv/dth are all non-NULL, backward) for a list
- * of units.  unit = (b*nW + w)*heads + h with windows w = wr*(W/M) + wc in the
- * rolled frame.  Per unit outputs, window-local token order t = i*M + j:
+ * of units.  unit = (b*nW + w)*heads + h with windows w = wr*(Wp/M) + wc in the
+ * rolled frame of the padded grid.  Per unit outputs, window-local token order t = i*M + j:
  *   o, dq, dk, dv: [n_units][M*M][d];  lse: [n_units][M*M];
  *   dth: [n_units][2][d/4], this unit's share of d theta for its head.
  */
@@ -266,7 +278,8 @@ int fso_units(const fso_shape* sh, fso_in q, fso_in k, fso_in v, fso_in dout, co
 }
 
 /*
- * Whole-tensor forward/backward.  Outputs at original token positions:
+ * Whole-tensor forward/backward.  Outputs at original token positions (padded
+ * tokens are dropped):
  *   o, dq, dk, dv: [B][H][W][heads][d];  lse: [B][H][W][heads];
  *   dtheta: [heads][2][d/4], summed over units in increasing unit order.
  * Backward outputs may be NULL (forward only).
@@ -276,7 +289,8 @@ int fso_full(const fso_shape* sh, fso_in q, fso_in k, fso_in v, fso_in dout, con
     int st = fso_check_shape(sh);
     if (st) return st;
     const int H = sh->H, W = sh->W, heads = sh->heads, d = sh->d, M = sh->M, s = sh->s;
-    const int nWw = W / M, nW = (H / M) * nWw, N = M * M, qq = d / 4;
+    const int Hp = fso_padded(H, M), Wp = fso_padded(W, M);
+    const int nWw = Wp / M, nW = (Hp / M) * nWw, N = M * M, qq = d / 4;
     const int64_t n_units = (int64_t)sh->B * nW * heads;
     const int bwd = dout.p != NULL && dq && dk && dv && dtheta;
     int64_t* units = (int64_t*)malloc(sizeof(int64_t) * (size_t)(n_units > 0 ? n_units : 1));
@@ -302,7 +316,8 @@ int fso_full(const fso_shape* sh, fso_in q, fso_in k, fso_in v, fso_in dout, con
         int w = (int)(rem / heads), h = (int)(rem % heads);
         int wr = w / nWw, wc = w % nWw;
         for (int t = 0; t < N; ++t) {
-            int ro = (wr * M + t / M + s) % H, co = (wc * M + t % M + s) % W;
+            int ro = (wr * M + t / M + s) % Hp, co = (wc * M + t % M + s) % Wp;
+            if (ro >= H || co >= W) continue;
             int64_t tok = (((int64_t)b * H + ro) * W + co) * heads + h;
             lse[tok] = ul[(size_t)n * N + t];
             for (int e = 0; e < d; ++e) {

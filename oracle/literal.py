@@ -5,6 +5,9 @@ pin the C oracle: it shares no arithmetic with it.  The cyclic shift is
 ``torch.roll``, windows come from a reshape, RoPE is a multiplication of
 channel pairs viewed as complex numbers, the shift mask is built with the Swin
 slice rule, softmax is ``torch.softmax`` and the gradients come from autograd.
+A grid that is not a multiple of M is zero-padded with
+``torch.nn.functional.pad`` before the roll and cropped after it, as a Swin
+layer does.
 
 Method: "FLASHSWIN ..." (arxivdaily.com/papers/2610.04664, English abstract:
 exact softmax attention inside each M x M window, window-local learnable 2D
@@ -16,6 +19,7 @@ from __future__ import annotations
 import math
 
 import torch
+import torch.nn.functional as F
 
 
 def region_labels(H: int, W: int, M: int, s: int) -> torch.Tensor:
@@ -63,7 +67,9 @@ def rope(x: torch.Tensor, theta: torch.Tensor, pos_i: torch.Tensor, pos_j: torch
 
 def forward(q, k, v, theta, M: int, s: int):
     """Returns (o [B,H,W,h,d], lse [B,H,W,h]) in float64."""
-    B, H, W, h, d = q.shape
+    B, H0, W0, h, d = q.shape
+    H, W = -(-H0 // M) * M, -(-W0 // M) * M
+    q, k, v = (F.pad(t, (0, 0, 0, 0, 0, W - W0, 0, H - H0)) for t in (q, k, v))
     shifted = [torch.roll(t, shifts=(-s, -s), dims=(1, 2)) for t in (q, k, v)]
     qw, kw, vw = (_windows(t, M) for t in shifted)
     t = torch.arange(M * M)
@@ -78,7 +84,7 @@ def forward(q, k, v, theta, M: int, s: int):
     o = torch.softmax(scores, dim=-1) @ vw
     o = torch.roll(_unwindows(o, H, W, M), shifts=(s, s), dims=(1, 2))
     lse = torch.roll(_unwindows(lse[..., None], H, W, M)[..., 0], shifts=(s, s), dims=(1, 2))
-    return o, lse
+    return o[:, :H0, :W0], lse[:, :H0, :W0]
 
 
 def forward_backward(q, k, v, theta, M: int, s: int, dout):
