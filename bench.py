@@ -40,6 +40,10 @@ WORKLOADS = {
     "swin_t_stage1_p4_infer_m8": dict(B=128, H=64, W=64, heads=3, M=8, shifts=(0, 4), qk_scale=1.0, infer=True),
     "swin_t_stage1_p4_infer_m16": dict(B=128, H=64, W=64, heads=3, M=16, shifts=(0, 8), qk_scale=1.0, infer=True),
     "swin_t_stage1_p4_infer_m32": dict(B=128, H=64, W=64, heads=3, M=32, shifts=(0, 16), qk_scale=1.0, infer=True),
+    # an 800 x 1333 detection input at p=4: a 200 x 334 grid, not a multiple of the window, worked on
+    # padded with zero tokens (200 x 336 at window 8; 224 x 352 at window 32), batch 16
+    "swin_t_det_stage1_p4_m8": dict(B=16, H=200, W=334, heads=3, M=8, shifts=(0, 4), qk_scale=1.0),
+    "flashswin_t_det_stage1_p4_m32": dict(B=16, H=200, W=334, heads=3, M=32, shifts=(0, 16), qk_scale=1.0),
 }
 HEADLINE = "swin_t_stage1_p4_m8"
 
@@ -51,7 +55,10 @@ BLOCK_WORKLOADS = {
 
 
 def unmasked_pairs(B, H, W, heads, M, s) -> int:
-    """Number of (query, key) pairs that attend (same window, same shift-region label)."""
+    """Number of (query, key) pairs that attend (same window, same shift-region label), on the
+    grid padded to multiples of M (padded tokens attend like the others)."""
+    H, W = -(-H // M) * M, -(-W // M) * M
+
     def sizes(X):
         if s == 0:
             return [[M]] * (X // M)

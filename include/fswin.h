@@ -17,11 +17,16 @@
  *    (2k, 2k+1) of the first d/2 channels by j * theta[h][0][k], axis 1 (y) the pairs
  *    of the last d/2 channels by i * theta[h][1][k], where (i, j) is the token's
  *    row and column inside its window (0 .. M-1, in the rolled frame);
- *  - the shift takes rolled token (r, c) from original position ((r+s) mod H,
- *    (c+s) mod W); outputs are written back at original positions;
+ *  - H or W that is not a multiple of M is padded at the bottom and right to
+ *    Hp = ceil(H/M)*M, Wp = ceil(W/M)*M with zero tokens, as a Swin layer pads its
+ *    input before the shift; everything below then refers to the padded grid
+ *    (Hp = H, Wp = W for multiples), padded tokens take part in the softmax, and
+ *    only the H x W real tokens are read or written;
+ *  - the shift takes rolled token (r, c) from original position ((r+s) mod Hp,
+ *    (c+s) mod Wp); outputs are written back at original positions;
  *  - with s > 0 a query attends a key of its window only when both carry the same
- *    Swin shift-region label, built from the row/column slices [0, H-M),
- *    [H-M, H-s), [H-s, H); masked scores are -infinity;
+ *    Swin shift-region label, built from the row/column slices [0, Hp-M),
+ *    [Hp-M, Hp-s), [Hp-s, Hp); masked scores are -infinity;
  *  - softmax scale 1/sqrt(d); lse is the natural-log log-sum-exp per query, fp32
  *    [B, H, W, heads];
  *  - gradients are those of sum(o * dout).
@@ -63,9 +68,11 @@ typedef enum {
 } fs_status;
 
 /*
- * Problem shape.  Supported: d == 32; M in {4, 8, 16, 32, 64}; H and W multiples
- * of M; 0 <= s < M with s a multiple of 4; heads >= 1; B >= 0 (B == 0 is a valid
- * empty problem).  Anything else returns FS_ERR_SHAPE.
+ * Problem shape.  Supported: d == 32; M in {4, 8, 16, 32, 64}; H >= M and W >= M
+ * (not necessarily multiples of M: the grid is then padded, see above; a grid
+ * smaller than the window is the caller's to clamp, as Swin clamps the window);
+ * 0 <= s < M with s a multiple of 4; heads >= 1; B >= 0 (B == 0 is a valid empty
+ * problem).  Anything else returns FS_ERR_SHAPE.
  */
 typedef struct {
     int B, H, W, heads, d, M, s;
@@ -82,8 +89,8 @@ FS_API fs_status fs_winattn_check_shape(const fs_winattn_shape* shape);
  * both overwritten.  lse may be NULL: an inference forward that writes o only
  * (the workload of FlashSwin's inference-throughput figure, thelatestinai.com
  * Fig. S1); the backward needs lse, so a training forward passes it.
- * Exact softmax attention per window (FlashSwin abstract: "exact softmax
- * attention without materializing the score matrix").
+ * Exact softmax attention per window, with no score matrix in device memory
+ * (the FlashSwin abstract).
  */
 FS_API fs_status fs_winattn_fwd(const fs_winattn_shape* shape, const void* q, const void* k, const void* v,
                          const float* theta, void* o, float* lse, fs_stream_t stream);
@@ -100,7 +107,9 @@ FS_API fs_status fs_winattn_fwd(const fs_winattn_shape* shape, const void* q, co
  * fp32 [C]; theta fp32 [heads,2,d/4].  Out: y bf16 [B,H,W,C], overwritten.
  * q, k, v and o never reach device memory.  Supported: the shapes of
  * fs_winattn_check_shape with M*M < 128 (windows inside one 128-token tile)
- * and heads <= 3; anything else returns FS_ERR_SHAPE.  x, w_qkv, w_o, y
+ * and heads <= 3; anything else returns FS_ERR_SHAPE.  On a padded grid (H or W
+ * not a multiple of M) the padded tokens of x are zero, as the Swin layer pads x
+ * before its qkv map, so their q, k, v equal the bias.  x, w_qkv, w_o, y
  * 16-byte aligned (FS_ERR_ALIGN); no pointer may be NULL (FS_ERR_NULL).
  */
 FS_API fs_status fs_winattn_block_fwd(const fs_winattn_shape* shape, const void* x, const void* w_qkv,
@@ -108,8 +117,9 @@ FS_API fs_status fs_winattn_block_fwd(const fs_winattn_shape* shape, const void*
                                void* y, fs_stream_t stream);
 
 /*
- * Workspace the backward needs, in bytes.  It depends on B*H*W*heads only, not on
- * the window size M (memory flat in M, FlashSwin Table S1).
+ * Workspace the backward needs, in bytes.  It depends on the token count of the
+ * padded grid, B*Hp*Wp*heads, only: for H and W multiples of M it does not depend
+ * on the window size (memory flat in M, FlashSwin Table S1).
  */
 FS_API size_t fs_winattn_bwd_workspace_bytes(const fs_winattn_shape* shape);
 

@@ -41,12 +41,12 @@ int main(int argc, char** argv) {
         std::printf("REJECT\n");
         return 0;
     }
-    std::printf("G %d %d %d %lld %d %d %d\n", g.N, g.BT, g.bpt, g.tiles, g.tpw, g.bh, g.bw);
+    std::printf("G %d %d %d %lld %d %d %d %d %d\n", g.N, g.BT, g.bpt, g.tiles, g.tpw, g.bh, g.bw, g.Hp, g.Wp);
     for (long long t = 0; t < g.tiles; ++t)
         for (int p = 0; p < kTile; ++p) {
             const Slot s = slot_of(g, t, p);
-            std::printf("S %lld %d %d %d %d %d %d %lld %d\n", t * kTile + p, s.box.b, s.row, s.col, s.i, s.j,
-                        s.box.label, s.box.gw, s.box.valid ? 1 : 0);
+            std::printf("S %lld %d %d %d %d %d %d %lld %d %d\n", t * kTile + p, s.box.b, s.row, s.col, s.i, s.j,
+                        s.box.label, s.box.gw, s.box.valid ? 1 : 0, s.valid ? 1 : 0);
         }
     for (long long b = 0; b < g.tiles * g.bpt; ++b) {
         const Box x = box_of(g, b);

@@ -35,11 +35,14 @@ def test_status_strings():
 
 GOOD = [(1, 16, 16, 2, 32, 8, 0), (128, 64, 64, 3, 32, 8, 4), (128, 128, 128, 3, 32, 32, 16),
         (16, 256, 256, 3, 32, 64, 32), (128, 16, 16, 24, 32, 16, 0), (0, 16, 16, 2, 32, 8, 0),
-        (2, 8, 24, 1, 32, 4, 0), (1, 32, 32, 1, 32, 32, 0)]
+        (2, 8, 24, 1, 32, 4, 0), (1, 32, 32, 1, 32, 32, 0),
+        # H or W not a multiple of M: padded to the next multiple
+        (1, 20, 16, 2, 32, 8, 0), (1, 16, 20, 2, 32, 8, 4), (2, 200, 334, 3, 32, 8, 4),
+        (1, 33, 17, 1, 32, 16, 8), (1, 65, 100, 1, 32, 64, 32)]
 BAD = [(1, 16, 16, 2, 64, 8, 0),    # d != 32
        (1, 16, 16, 2, 32, 12, 0),   # M not supported
-       (1, 20, 16, 2, 32, 8, 0),    # H % M
-       (1, 16, 20, 2, 32, 8, 0),    # W % M
+       (1, 7, 16, 2, 32, 8, 0),     # H < M
+       (1, 16, 15, 2, 32, 16, 0),   # W < M
        (1, 16, 16, 2, 32, 8, 8),    # s >= M
        (1, 16, 16, 2, 32, 8, 2),    # s % 4
        (1, 16, 16, 2, 32, 8, -4),   # s < 0
@@ -93,6 +96,15 @@ def test_workspace_flat_in_window_size():
     # reduction's second level: heads x 64 x 16 floats)
     d = _lib.fs_winattn_bwd_workspace_bytes(_lib.make_shape(32, 256, 256, 3, 32, 32, 16))
     assert abs(d - 2 * a) <= 3 * 64 * 16 * 4 + 4096
+
+
+def test_padded_grid_workspace_is_that_of_the_padded_grid():
+    """A grid that is not a multiple of M is worked on padded: the backward
+    scratch is that of the padded grid."""
+    ws = _lib.fs_winattn_bwd_workspace_bytes
+    assert ws(_lib.make_shape(2, 200, 334, 3, 32, 8, 4)) == ws(_lib.make_shape(2, 200, 336, 3, 32, 8, 4))
+    assert ws(_lib.make_shape(1, 33, 17, 1, 32, 16, 8)) == ws(_lib.make_shape(1, 48, 32, 1, 32, 16, 8))
+    assert ws(_lib.make_shape(1, 20, 16, 2, 32, 8, 0)) == ws(_lib.make_shape(1, 24, 16, 2, 32, 8, 0))
 
 
 @pytest.mark.skipif(torch.cuda.is_available(), reason="would launch on the placeholder pointers")

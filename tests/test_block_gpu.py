@@ -18,6 +18,8 @@ CASES = [  # (B, H, W, heads, M, s)
     (1, 8, 12, 1, 4, 0),    # 16-token windows, one head
     (3, 32, 32, 3, 8, 4),   # more tiles than one CTA's first item
     (1, 16, 16, 2, 4, 0),
+    (1, 20, 13, 3, 8, 4),   # grid padded to 24 x 16: padded tokens carry the bias
+    (2, 10, 6, 2, 4, 0),
 ]
 
 

@@ -7,7 +7,8 @@ holds windows of the last window row and column (the only ones the shift mask
 cuts) and of the first.  dθ sums over every token, so it is checked through a
 property that holds at any size: with dO zero outside the sampled units, the
 other units contribute nothing, and dθ equals the sum of the sampled units'
-shares.
+shares.  Grids that are not multiples of M (a detection-sized input) are
+compared at their real tokens; the padded ones exist only inside the kernels.
 """
 import numpy as np
 import pytest
@@ -33,6 +34,9 @@ FULL = [
     ("flashswin_t_stage4_p2_m16", 128, 16, 16, 24, 16, 0, 1.0),
     ("highres_p2_m32", 16, 256, 256, 3, 32, 16, 3.0),
     ("highres_p2_m64", 16, 256, 256, 3, 64, 32, 3.0),
+    # an 800 x 1333 detection input at p=4: a 200 x 334 grid, padded per window size
+    ("swin_t_det_stage1_p4_m8_s4", 16, 200, 334, 3, 8, 4, 1.0),
+    ("flashswin_t_det_stage1_p4_m32_s16", 16, 200, 334, 3, 32, 16, 1.0),
 ]
 
 
@@ -47,7 +51,7 @@ def _check(name, got, ref, tol):
 
 
 def _sample_units(B, H, W, heads, M, n_random=6, seed=7):
-    nWh, nWw = H // M, W // M
+    nWh, nWw = -(-H // M), -(-W // M)  # windows of the padded grid
     nW = nWh * nWw
     picks = {(0, 0, 0), (B - 1, nWh - 1, nWw - 1), (0, nWh - 1, 0), (0, 0, nWw - 1), (B // 2, nWh - 1, nWw // 2)}
     rng = np.random.default_rng(seed)
@@ -66,10 +70,14 @@ def test_full_size_sampled_windows(cfg):
     name, B, H, W, heads, M, s, qk = cfg
     inp = make_inputs(B, H, W, heads, 32, qk_scale=qk)
     units = _sample_units(B, H, W, heads, M)
-    pos = [oracle.unit_token_positions(H, W, M, s, int(u), heads) for u in units]
+    pos = []
+    for u in units:  # real tokens of each unit, and their window-local slots
+        b, rows, cols, h = oracle.unit_token_positions(H, W, M, s, int(u), heads)
+        real = (rows < H) & (cols < W)
+        pos.append((b, rows[real], cols[real], h, real))
     # dO kept on the sampled units' tokens only
     keep = torch.zeros((B, H, W, heads), dtype=torch.bool)
-    for b, rows, cols, h in pos:
+    for b, rows, cols, h, _ in pos:
         keep[b, torch.from_numpy(rows), torch.from_numpy(cols), h] = True
     dout = torch.where(keep[..., None], inp["dout"], torch.zeros((), dtype=inp["dout"].dtype))
 
@@ -81,15 +89,18 @@ def test_full_size_sampled_windows(cfg):
     ref = oracle.units(inp["q"], inp["k"], inp["v"], inp["theta"], M, s, units, dout=dout)
     idx = lambda t, b, rows, cols, h: t[b, torch.from_numpy(rows), torch.from_numpy(cols), h]
     got = {k: [] for k in ("o", "lse", "dq", "dk", "dv")}
-    for b, rows, cols, h in pos:
+    want = {k: [] for k in got}
+    for n, (b, rows, cols, h, real) in enumerate(pos):
         for key, t in (("o", o), ("lse", lse), ("dq", dq), ("dk", dk), ("dv", dv)):
             got[key].append(idx(t, b, rows, cols, h).float().cpu().numpy())
-    _check(f"{name} o", np.stack(got["o"]), ref["o"], FWD_TOL)
-    _check(f"{name} lse", np.stack(got["lse"]), ref["lse"], FWD_TOL)
+            want[key].append(ref[key][n][real])
+    cat = np.concatenate
+    _check(f"{name} o", cat(got["o"]), cat(want["o"]), FWD_TOL)
+    _check(f"{name} lse", cat(got["lse"]), cat(want["lse"]), FWD_TOL)
     for key in ("dq", "dk", "dv"):
-        _check(f"{name} {key}", np.stack(got[key]), ref[key], GRAD_TOL)
+        _check(f"{name} {key}", cat(got[key]), cat(want[key]), GRAD_TOL)
     # dθ: only the sampled units carry dO, so the total is their sum
-    want = np.zeros((heads, 2, 8))
+    want_th = np.zeros((heads, 2, 8))
     for u, share in zip(units, ref["dtheta"]):
-        want[int(u) % heads] += share
-    _check(f"{name} dtheta", dth.float().cpu().numpy(), want, GRAD_TOL)
+        want_th[int(u) % heads] += share
+    _check(f"{name} dtheta", dth.float().cpu().numpy(), want_th, GRAD_TOL)

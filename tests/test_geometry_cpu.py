@@ -3,9 +3,12 @@
 The kernels' own headers (geometry.cuh, schedule.cuh) are compiled for the host
 with g++ and their output is checked against the oracle's definition of the
 shifted windows (roll by -s, M x M windows, Swin region labels):
-  * token slots cover every token exactly once (padding slots only at the end);
+  * token slots cover every token of the grid, padded to multiples of M when
+    H or W is not one, exactly once (slots of padding windows only at the end),
+    and mark as real exactly the H x W tokens in memory;
   * in-window positions, labels and windows agree with the oracle's definition;
-  * TMA boxes never straddle the wrap of the cyclic shift and stay in bounds;
+  * TMA boxes never straddle the wrap of the cyclic shift and stay inside the
+    padded grid;
   * forward items visit exactly the (query tile, key tile) pairs that hold at
     least one attending token pair, every query tile once per head;
   * backward items visit the same pairs, every key tile once per head.
@@ -49,6 +52,14 @@ SHAPES = [  # (B, H, W, heads, d, M, s)
     (1, 64, 64, 1, 32, 64, 32),
     (1, 128, 64, 1, 32, 64, 0),
     (1, 64, 96, 1, 32, 32, 12),
+    # H or W not a multiple of M: the grid is padded
+    (1, 12, 20, 2, 32, 8, 4),
+    (2, 20, 13, 2, 32, 8, 0),
+    (1, 10, 6, 1, 32, 4, 0),
+    (1, 40, 36, 1, 32, 16, 8),
+    (1, 33, 20, 1, 32, 16, 4),
+    (1, 70, 50, 1, 32, 32, 16),
+    (1, 100, 70, 1, 32, 64, 32),
 ]
 
 
@@ -57,29 +68,34 @@ def test_geometry_and_schedule(harness, shape):
     B, H, W, heads, d, M, s = shape
     lines = run(harness, shape)
     g = lines[0].split()
-    N, BT, bpt, tiles, tpw, bh, bw = map(int, g[1:])
+    N, BT, bpt, tiles, tpw, bh, bw, Hp, Wp = map(int, g[1:])
+    assert (Hp, Wp) == (-(-H // M) * M, -(-W // M) * M)
     slots = np.array([list(map(int, l.split()[1:])) for l in lines if l[0] == "S"], dtype=np.int64)
     assert slots.shape[0] == tiles * 128
-    valid = slots[:, 8] == 1
-    ntok = B * H * W
+    valid = slots[:, 8] == 1          # slot of a real window (padded positions included)
+    ntok = B * Hp * Wp
     assert valid.sum() == ntok
     assert valid[:ntok].all() and not valid[ntok:].any()
     v = slots[valid]
     b, row, col, i, j, lab, gw = (v[:, k] for k in range(1, 8))
-    tok = (b * H + row) * W + col
+    assert (row >= 0).all() and (row < Hp).all() and (col >= 0).all() and (col < Wp).all()
+    tok = (b * Hp + row) * Wp + col
     assert np.unique(tok).size == ntok
-    r, c = (row - s) % H, (col - s) % W
+    real = (row < H) & (col < W)
+    assert (v[:, 9] == real).all() and (slots[~valid][:, 9] == 0).all()
+    assert real.sum() == B * H * W
+    r, c = (row - s) % Hp, (col - s) % Wp
     assert (i == r % M).all() and (j == c % M).all()
-    labels = oracle.labels(H, W, M, s)
+    labels = oracle.labels(Hp, Wp, M, s)
     assert (lab == labels[r, c]).all()
-    nW = (H // M) * (W // M)
-    assert (gw == b * nW + (r // M) * (W // M) + c // M).all()
+    nW = (Hp // M) * (Wp // M)
+    assert (gw == b * nW + (r // M) * (Wp // M) + c // M).all()
 
     boxes = np.array([list(map(int, l.split()[1:])) for l in lines if l[0] == "X"], dtype=np.int64)
     bv = boxes[boxes[:, 4] == 1]
     # columns: box id, image, first row, first column, valid
-    assert (bv[:, 2] >= 0).all() and (bv[:, 2] + bh <= H).all()
-    assert (bv[:, 3] >= 0).all() and (bv[:, 3] + bw <= W).all()
+    assert (bv[:, 2] >= 0).all() and (bv[:, 2] + bh <= Hp).all()
+    assert (bv[:, 3] >= 0).all() and (bv[:, 3] + bw <= Wp).all()
     assert (bv[:, 1] < B).all()
     assert (boxes[boxes[:, 4] == 0][:, 1] >= B).all()  # padding boxes fall outside the tensor
 

@@ -22,6 +22,8 @@ CASES = [  # (B, H, W, heads, M, s): both kernel families, shifted and not, ragg
     (1, 32, 48, 1, 16, 4),
     (1, 64, 64, 1, 32, 16),
     (1, 64, 64, 1, 64, 32),
+    (1, 20, 13, 2, 8, 4),     # padded grids
+    (1, 33, 20, 1, 16, 4),
 ]
 
 

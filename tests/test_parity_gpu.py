@@ -73,6 +73,30 @@ def test_fwd_bwd_parity(cfg):
         check(key, got[key], ref[key], GRAD_TOL)
 
 
+# H or W not a multiple of M: the grid is padded with zero tokens (the Swin
+# layer's padding), boxes run partly or wholly past the tokens in memory
+PADDED = [  # (B, H, W, heads, M, s)
+    (1, 20, 13, 2, 8, 4),     # windows inside a tile, shifted, both axes padded
+    (2, 12, 18, 3, 8, 0),
+    (1, 10, 6, 1, 4, 0),      # 16-token windows
+    (1, 50, 83, 3, 8, 4),     # a detection-sized stage-2 grid (400 x 664 image / 8)
+    (1, 40, 36, 2, 16, 8),    # one tile per window
+    (1, 33, 20, 1, 16, 4),    # 1 real row in the last window row
+    (1, 70, 50, 1, 32, 16),   # several tiles per window
+    (1, 100, 70, 1, 64, 32),  # 4096-token windows
+]
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("cfg", PADDED)
+def test_padded_grid_parity(cfg):
+    got, ref = run_both(*cfg)
+    check("o", got["o"], ref["o"], FWD_TOL)
+    check("lse", got["lse"], ref["lse"], FWD_TOL)
+    for key in ("dq", "dk", "dv", "dtheta"):
+        check(key, got[key], ref[key], GRAD_TOL)
+
+
 @pytest.mark.gpu
 def test_sharp_softmax_parity():
     """Q, K scaled by 3 (the high-resolution stress recipe) sharpen the softmax."""

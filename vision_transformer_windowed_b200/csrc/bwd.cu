@@ -129,7 +129,7 @@ __global__ void __launch_bounds__(128) prep_kernel(const PrepParams p) {
     const Slot sl = slot_of(g, T, r);
     float q[32], k[32], dO[32], o[32];
     float D = 0.f, lse2 = INFINITY;
-    if (sl.box.valid) {
+    if (sl.valid) {
         const long long tok = ((static_cast<long long>(sl.box.b) * g.H + sl.row) * g.W + sl.col) * g.heads + h;
         load_row_bf16(p.q + tok * 4, q);
         load_row_bf16(p.k + tok * 4, k);
@@ -693,7 +693,7 @@ __global__ void __launch_bounds__(128) post_kernel(const PostParams p) {
     float part[16];
 #pragma unroll
     for (int e = 0; e < 16; ++e) part[e] = 0.f;
-    if (sl.box.valid) {
+    if (sl.valid) {
         const long long tok = ((static_cast<long long>(sl.box.b) * g.H + sl.row) * g.W + sl.col) * g.heads + h;
         float dq[32], q[32];
         const float4* aq = reinterpret_cast<const float4*>(p.ws + p.L.dqacc + (ht * kTile + r) * kHeadDim * 4);

@@ -484,11 +484,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                 int pi, pj;
                 tile_row_pos(g, X, r, &pi, &pj);
                 int row = w.wr * g.M + pi + g.s, col = w.wc * g.M + pj + g.s;
-                if (row >= g.H) row -= g.H;
-                if (col >= g.W) col -= g.W;
-                const float lse2 = m + lg2_approx(l);
-                const long long tok = ((static_cast<long long>(w.b) * g.H + row) * g.W + col) * g.heads + h;
-                prm.lse[tok] = lse2 * 0.69314718055994530942f;
+                if (row >= g.Hp) row -= g.Hp;
+                if (col >= g.Wp) col -= g.Wp;
+                if (row < g.H && col < g.W) {  // not a padded position
+                    const float lse2 = m + lg2_approx(l);
+                    const long long tok = ((static_cast<long long>(w.b) * g.H + row) * g.W + col) * g.heads + h;
+                    prm.lse[tok] = lse2 * 0.69314718055994530942f;
+                }
             }
         }
         if (leader) bulk_wait_all();

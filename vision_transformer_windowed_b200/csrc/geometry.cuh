@@ -10,6 +10,12 @@
 // block-diagonal mask).  Two tokens attend to each other iff they share the
 // window and the shift-region label (the Swin shifted-window rule).
 //
+// A grid whose H or W is not a multiple of M is padded at the bottom and right
+// to Hp x Wp (the next multiples of M) with zero tokens, as a Swin layer pads
+// its input: windows, the roll and the region labels refer to the padded grid,
+// padded tokens take part in the softmax, and only real positions are read
+// from or written to memory.
+//
 // Every extent below is a power of two, so the per-row and per-tile helpers
 // use shifts and masks.  The few divisions by other set-up constants (windows
 // per image, tiles per head) use 32-bit division by invariant integers.
@@ -53,7 +59,8 @@ constexpr int kRowBytes = kHeadDim * 2;     // one 16-bit token row
 constexpr int kTileBytes = kTile * kRowBytes;
 
 struct Geo {
-    int B, H, W, heads, M, s;
+    int B, H, W, heads, M, s;   // H, W: the tokens in memory
+    int Hp, Wp;         // the grid padded to multiples of M
     int nWw, nW;        // windows per image row, per image
     int N;              // tokens per window
     int bh, bw, BT;     // box rows, box cols, tokens per box
@@ -79,12 +86,13 @@ __host__ __device__ inline int ilog2_exact(int x) {
 inline int geo_init(Geo* g, int B, int H, int W, int heads, int d, int M, int s) {
     if (d != kHeadDim) return 2;
     if (!(M == 4 || M == 8 || M == 16 || M == 32 || M == 64)) return 2;
-    if (B < 0 || heads < 1 || H < M || W < M || H % M || W % M) return 2;
+    if (B < 0 || heads < 1 || H < M || W < M) return 2;
     if (s < 0 || s >= M || s % 4) return 2;
     if (H > (1 << 24) || W > (1 << 24) || heads > 4096) return 2;
+    const int Hp = (H + M - 1) / M * M, Wp = (W + M - 1) / M * M;
     // token, window, tile and work-item indices of one head stay below 2^31
-    if (static_cast<long long>(B) * H * W > (1ll << 31)) return 2;
-    if (static_cast<long long>(B) * H * W * heads > (1ll << 37)) return 2;
+    if (static_cast<long long>(B) * Hp * Wp > (1ll << 31)) return 2;
+    if (static_cast<long long>(B) * Hp * Wp * heads > (1ll << 37)) return 2;
     int a = M, b = s;  // box side: gcd(M, s), or M without shift
     while (b) {
         const int t = a % b;
@@ -96,11 +104,13 @@ inline int geo_init(Geo* g, int B, int H, int W, int heads, int d, int M, int s)
     x.B = B;
     x.H = H;
     x.W = W;
+    x.Hp = Hp;
+    x.Wp = Wp;
     x.heads = heads;
     x.M = M;
     x.s = s;
-    x.nWw = W / M;
-    x.nW = (H / M) * (W / M);
+    x.nWw = Wp / M;
+    x.nW = (Hp / M) * (Wp / M);
     x.N = M * M;
     x.bw = side < kTile ? side : kTile;
     x.bh = side < kTile / x.bw ? side : kTile / x.bw;
@@ -171,14 +181,17 @@ __host__ __device__ inline int box_c(const Geo& g, const Win& w, int k) {
 
 __host__ __device__ inline int box_label(const Geo& g, const Win& w, int k) {
     if (!g.s) return 0;
-    return 3 * region_of(g.H, g.M, g.s, box_r(g, w, k)) + region_of(g.W, g.M, g.s, box_c(g, w, k));
+    return 3 * region_of(g.Hp, g.M, g.s, box_r(g, w, k)) + region_of(g.Wp, g.M, g.s, box_c(g, w, k));
 }
 
-// Original (un-rolled) coordinates of the first token of box k of window w.
+// Original (un-rolled) coordinates of the first token of box k of window w, in
+// the padded grid: the box lies wholly or partly outside the H x W tokens in
+// memory when row0 + bh > H or col0 + bw > W (a box never straddles the wrap:
+// Hp - s and Wp - s are multiples of the box side).
 __host__ __device__ inline void box_origin(const Geo& g, const Win& w, int k, int* row0, int* col0) {
     int r = box_r(g, w, k) + g.s, c = box_c(g, w, k) + g.s;
-    if (r >= g.H) r -= g.H;
-    if (c >= g.W) c -= g.W;
+    if (r >= g.Hp) r -= g.Hp;
+    if (c >= g.Wp) c -= g.Wp;
     *row0 = r;
     *col0 = c;
 }
@@ -266,7 +279,8 @@ __host__ __device__ inline Box box_of(const Geo& g, long long gbox) {
 struct Slot {
     Box box;
     int i, j;        // in-window coordinates (RoPE positions: y = i, x = j)
-    int row, col;    // original coordinates
+    int row, col;    // original coordinates (in the padded grid)
+    bool valid;      // a real token: a real window and row < H, col < W
 };
 
 __host__ __device__ inline Slot slot_of(const Geo& g, long long tile, int p) {
@@ -277,6 +291,7 @@ __host__ __device__ inline Slot slot_of(const Geo& g, long long tile, int p) {
     s.j = s.box.j0 + bj;
     s.row = s.box.row0 + bi;
     s.col = s.box.col0 + bj;
+    s.valid = s.box.valid && s.row < g.H && s.col < g.W;
     return s;
 }
 

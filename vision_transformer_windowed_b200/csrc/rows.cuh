@@ -78,8 +78,9 @@ __device__ __forceinline__ void build_small_table(float2* tab, const float* thet
     }
 }
 
-// Token of slot r of tile X (false for padding windows): in-window position
-// and flat index of the [B, H, W, heads] grid at head h.
+// Token of slot r of tile X: in-window position and flat index of the
+// [B, H, W, heads] tokens at head h.  False (and *tok meaningless) for the
+// slots of padding windows and for padded positions of the grid.
 __device__ __forceinline__ bool slot_token(const Geo& g, long long X, int r, int h, int* pi, int* pj,
                                            long long* tok) {
     Win w = tile_win(g, X);
@@ -87,10 +88,10 @@ __device__ __forceinline__ bool slot_token(const Geo& g, long long X, int r, int
     if (widx) w = win_of(g, w.gw + widx);
     tile_row_pos(g, X, r, pi, pj);
     int row = w.wr * g.M + *pi + g.s, col = w.wc * g.M + *pj + g.s;
-    if (row >= g.H) row -= g.H;
-    if (col >= g.W) col -= g.W;
+    if (row >= g.Hp) row -= g.Hp;
+    if (col >= g.Wp) col -= g.Wp;
     *tok = ((static_cast<long long>(w.b) * g.H + row) * g.W + col) * g.heads + h;
-    return w.valid;
+    return w.valid && row < g.H && col < g.W;
 }
 
 }  // namespace fswin

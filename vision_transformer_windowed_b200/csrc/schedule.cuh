@@ -36,7 +36,7 @@ __host__ __device__ inline FwdItem fwd_item(const Geo& g, long long it) {
         I.nkv = g.tpw;
         I.win = win_of(g, gw);
         I.act = low_bits(g.tpw);
-        if (g.s && (I.win.wr == g.H / g.M - 1 || I.win.wc == g.nWw - 1)) {
+        if (g.s && (I.win.wr == g.Hp / g.M - 1 || I.win.wc == g.nWw - 1)) {
             const uint64_t sx = tile_segs(g, I.X, I.win);
             I.act = 0;
             for (int u = 0; u < g.tpw; ++u)
@@ -80,7 +80,7 @@ __host__ __device__ inline BwdItem bwd_item(const Geo& g, long long it) {
         I.paired = false;
         I.win = win_of(g, gw);
         I.act = low_bits(g.tpw);
-        if (g.s && (I.win.wr == g.H / g.M - 1 || I.win.wc == g.nWw - 1)) {
+        if (g.s && (I.win.wr == g.Hp / g.M - 1 || I.win.wc == g.nWw - 1)) {
             const uint64_t su = tile_segs(g, I.u, I.win);
             I.act = 0;
             for (int n = 0; n < g.tpw; ++n)

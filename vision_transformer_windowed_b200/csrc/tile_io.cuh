@@ -10,6 +10,9 @@ namespace fswin {
 
 // TMA loads (or, when `store`, stores of the boxes of real windows) of every
 // box of a tile; the smem tile holds the boxes back to back, 64-byte swizzled.
+// The tensor maps span the H x W tokens in memory: a load reads zeros at the
+// padded positions of a box, a store leaves them out, and boxes wholly in the
+// padding are not stored at all.
 static __device__ __noinline__ void tile_tma(const Geo& g, const CUtensorMap* map, uint8_t* smem_tile, uint64_t* bar,
                                       long long tile, int h, bool store) {
     Win w = tile_win(g, tile);
@@ -23,7 +26,7 @@ static __device__ __noinline__ void tile_tma(const Geo& g, const CUtensorMap* ma
         uint8_t* p = smem_tile + x * g.BT * kRowBytes;
         if (!store)
             tma_load_5d(p, map, bar, 0, h, c0, r0, w.b);
-        else if (w.valid)
+        else if (w.valid && r0 < g.H && c0 < g.W)
             tma_store_5d(map, p, 0, h, c0, r0, w.b);
     }
 }
