@@ -33,7 +33,8 @@ WORKLOADS = {
     "swin_t_stage1_p4_m8": dict(B=128, H=64, W=64, heads=3, M=8, shifts=(0, 4), qk_scale=1.0),
     # FlashSwin-T stage 1 at p=2 (128x128 grid), window 32, shifted block
     "flashswin_t_stage1_p2_m32": dict(B=128, H=128, W=128, heads=3, M=32, shifts=(16,), qk_scale=1.0),
-    # 512x512 input at p=2, window 64 (4096-token windows), Q and K scaled by 3
+    # 512x512 input at p=2, windows 32 and 64 (4096-token windows), Q and K scaled by 3
+    "highres_p2_m32": dict(B=16, H=256, W=256, heads=3, M=32, shifts=(16,), qk_scale=3.0),
     "highres_p2_m64": dict(B=16, H=256, W=256, heads=3, M=64, shifts=(32,), qk_scale=3.0),
     # inference forward (no LSE written) at the shape of FlashSwin's inference-throughput figure:
     # p=4 (64x64 grid at 256x256 input), batch 128, windows 8 to 32, unshifted and shifted blocks
@@ -46,6 +47,7 @@ WORKLOADS = {
     "flashswin_t_det_stage1_p4_m32": dict(B=16, H=200, W=334, heads=3, M=32, shifts=(0, 16), qk_scale=1.0),
 }
 HEADLINE = "swin_t_stage1_p4_m8"
+SPEC_BF16_TFLOPS = 2250.0  # NVIDIA's dense bf16 figure for one B200: a spec value, not a measurement
 
 # the window-attention block of a Swin layer with its qkv and output projections (inference),
 # Swin-T stage 1 at p=4: C = 96 channels in 3 heads, window 8, unshifted and shifted blocks
@@ -202,10 +204,10 @@ def cpu_baseline(tensors, wl, seconds: float = 12.0):
 
     import oracle
     B, H, W, heads, M = wl["B"], wl["H"], wl["W"], wl["heads"], wl["M"]
-    nW = (H // M) * (W // M)
+    nW = -(-H // M) * -(-W // M)  # windows of the grid padded to multiples of M
     n_units = B * nW * heads
     cores = oracle.default_threads()
-    flops, total_dt, parts = 0.0, 0.0, []
+    flops, total_dt, parts, done, full_s = 0.0, 0.0, [], 0, 0.0
     for s in wl["shifts"]:
         # units spread over the batch, including windows of the last row/column
         t0 = time.perf_counter()
@@ -223,10 +225,38 @@ def cpu_baseline(tensors, wl, seconds: float = 12.0):
         # useful flops of the sampled units (pairs that attend)
         flops += 14.0 * HEAD_DIM * unmasked_pairs(B, H, W, heads, M, s) * (n / n_units)
         total_dt += dt
+        done += n
+        full_s += dt * n_units / n
         parts.append(f"{n} of {n_units} at s={s}")
     return {"value": flops / total_dt / 1e12, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
             "sample": f"(batch, window, head) units: {', '.join(parts)}; fwd+bwd, fp64, {total_dt:.1f} s",
+            "units_per_s": done / total_dt,
+            "full_step_s_extrapolated": full_s,  # equal to the measured time when every unit was sampled
             "seconds": total_dt}
+
+
+def config_entry(wl, r, peaks, world) -> dict:
+    """Per-workload figures: fwd+bwd and forward-alone throughput, the no-recompute count of
+    the backward (8 d per pair instead of 10 d), % of the measured and of the spec bf16 peak,
+    the forward's algorithmic HBM rate, peak memory and the backward workspace."""
+    nshift = len(wl["shifts"])
+    fwd_ms = r["phase_ms"]["fwd"] * nshift  # per step
+    rows = wl["B"] * wl["H"] * wl["W"] * wl["heads"]
+    infer = wl.get("infer", False)
+    e = {"tflops": r["tflops"], "ms_per_step": r["ms"],
+         "pct_bf16_peak": 100 * r["tflops"] / peaks["bf16_tflops"] / world,
+         "pct_bf16_spec": 100 * r["tflops"] / SPEC_BF16_TFLOPS / world,
+         "fwd_tflops": r["fwd_flops"] * world / (fwd_ms * 1e-3) / 1e12,
+         "tokens_per_s": r["tokens_per_s"], "peak_gb": r["peak_gb"], "phase_ms": r["phase_ms"]}
+    e["fwd_pct_bf16_peak"] = 100 * e["fwd_tflops"] / peaks["bf16_tflops"] / world
+    # q, k, v read and o written (bf16), plus the fp32 lse of a training forward
+    e["fwd_gbs"] = (256 if infer else 260) * rows * nshift / (fwd_ms * 1e-3) / 1e9
+    if infer:
+        e["step"] = "inference forward (no LSE) at every shift"
+    else:
+        e["tflops_no_recompute"] = (r["fwd_flops"] + 0.8 * r["bwd_flops"]) * world / (r["ms"] * 1e-3) / 1e12
+        e["bwd_workspace_gb"] = r["ws_bytes"] / 1e9
+    return e
 
 
 def run_block(wl, dev, rank, steps, warmup, peaks):
@@ -520,10 +550,7 @@ def main():
     e2e = {"value": fl * world / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s", "ms_per_step": e2e_ms,
            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
 
-    per_config = {args.workload: {"tflops": main_res["tflops"], "ms_per_step": main_res["ms"],
-                                  "pct_bf16_peak": 100 * main_res["tflops"] / peaks["bf16_tflops"] / world,
-                                  "tokens_per_s": main_res["tokens_per_s"], "peak_gb": main_res["peak_gb"],
-                                  "phase_ms": main_res["phase_ms"]}}
+    per_config = {args.workload: config_entry(wl, main_res, peaks, world)}
     del main_res["tensors"], t, host, res_host
     if not args.no_extra:
         for name in WORKLOADS:
@@ -532,13 +559,7 @@ def main():
             torch.cuda.empty_cache()
             r = run_workload(name, max(3, args.steps // 2), 3, phase=True, clocks=False)
             del r["tensors"]
-            per_config[name] = {"tflops": r["tflops"], "ms_per_step": r["ms"],
-                                "pct_bf16_peak": 100 * r["tflops"] / peaks["bf16_tflops"] / world,
-                                "tokens_per_s": r["tokens_per_s"], "peak_gb": r["peak_gb"],
-                                "phase_ms": r["phase_ms"], "bwd_workspace_gb": r["ws_bytes"] / 1e9}
-            if WORKLOADS[name].get("infer"):
-                per_config[name]["step"] = "inference forward (no LSE) at every shift"
-                del per_config[name]["bwd_workspace_gb"]
+            per_config[name] = config_entry(WORKLOADS[name], r, peaks, world)
 
     if not args.no_extra:
         for name, wl_b in BLOCK_WORKLOADS.items():
@@ -568,6 +589,12 @@ def main():
             "roofline": roof, "clocks": main_res["clocks"], "e2e": e2e, "cpu_baseline": cpu,
             "per_config": per_config, "peaks": peaks,
         }
+        a, b = per_config.get("highres_p2_m32"), per_config.get("highres_p2_m64")
+        if a and b:  # memory flat in M: the same tokens at windows 32 and 64
+            line["flat_in_m"] = {"workloads": ["highres_p2_m32", "highres_p2_m64"],
+                                 "peak_gb": [a["peak_gb"], b["peak_gb"]],
+                                 "peak_diff_mb": abs(a["peak_gb"] - b["peak_gb"]) * 1e3,
+                                 "bwd_workspace_gb": [a["bwd_workspace_gb"], b["bwd_workspace_gb"]]}
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.destroy_process_group()
