@@ -12,16 +12,14 @@
 //       Per head: the biases and the RoPE of its q, k row (TMEM -> fp16 q',
 //       k' and bf16 v tiles), the softmax of its query row, O / l into the
 //       head's o tile; per item y + b_o into the staging tiles (the o tiles,
-//       once read).
-//   warp 8 (MMA): for either pipeline, whenever its next step is ready: per
-//       head q|k|v = x [W_q,h; W_k,h; W_v,h]^T (N = 96, issued while the
-//       previous head's softmax runs), S = Q'K'^T, O_h = P V; per item
-//       Y = sum_h O_h W_o[:, 32h:32h+32]^T.
-//   warp 9 + p (mover of pipeline p): x rows in (16-byte cp.async) as soon as
+//       once read).  Row 0 of the pipeline also issues its MMAs, each as
+//       soon as the rows' barrier before it passes: per head
+//       q|k|v = x [W_q,h; W_k,h; W_v,h]^T (N = 96; the next head's right after
+//       this head's S, so that it runs during the softmax), S = Q'K'^T,
+//       O_h = P V; per item Y = sum_h O_h W_o[:, 32h:32h+32]^T.
+//   warp 8 + p (mover of pipeline p): x rows in (16-byte cp.async) as soon as
 //       the pipeline's x buffer is free, y rows out as soon as they are staged.
-// The MMA warp polls the two pipelines' barriers without blocking, within the
-// usual time limit.  The weights and biases stay in shared memory
-// for the whole launch.
+// The weights and biases stay in shared memory for the whole launch.
 #include <cuda.h>
 #include <cuda_runtime.h>
 
@@ -37,8 +35,8 @@ namespace blockk {
 
 constexpr int kMaxHeads = 3;
 constexpr int kPipes = 2;
-constexpr int kThreads = 352;
-constexpr int kWarpMma = 8, kWarpMover = 9;  // movers: warps 9 and 10
+constexpr int kThreads = 320;
+constexpr int kWarpMover = 8;  // movers: warps 8 and 9
 constexpr int kQkvRows = 3 * kHeadDim;  // q, k, v rows of one head in a W_qkv chunk tile
 
 // Shared memory (offsets from a 1024-byte aligned base).  A weight "chunk" is
@@ -70,8 +68,8 @@ constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColQKV = 0, kColY = 0, kColO = 96, kColS = 128;
 
 struct PipeBars {
-    uint64_t x_full, x_free;                               // per item: x landed (32 mover lanes); last q|k|v MMAs done
-    uint64_t qkv_full, in_ready, s_full, p_ready, o_full;  // per head
+    uint64_t x_full, x_free;                     // per item: x landed (32 mover lanes); last q|k|v MMAs done
+    uint64_t qkv_full, s_full, p_ready, o_full;  // per head
     uint64_t o_ready, y_full, y_free, staged, y_done;      // per item
     uint64_t grp;                                          // the pipeline's four row warps
 };
@@ -110,7 +108,6 @@ __global__ void __launch_bounds__(kThreads, 1) block_kernel(const __grid_constan
             mbar_init(&B.x_full, 32);  // one arrival per mover lane, once its copies have landed
             mbar_init(&B.x_free, 1);
             mbar_init(&B.qkv_full, 1);
-            mbar_init(&B.in_ready, 1);
             mbar_init(&B.s_full, 1);
             mbar_init(&B.p_ready, 4);
             mbar_init(&B.o_full, 1);
@@ -121,7 +118,7 @@ __global__ void __launch_bounds__(kThreads, 1) block_kernel(const __grid_constan
             mbar_init(&B.y_done, 1);
             mbar_init(&B.grp, 4);
         }
-        mbar_init(&bars->done, 1);
+        mbar_init(&bars->done, kPipes);  // each pipeline's MMA-issuing thread
         bars->abort_flag = 0;
         fence_mbar_init();
     }
@@ -159,120 +156,7 @@ __global__ void __launch_bounds__(kThreads, 1) block_kernel(const __grid_constan
     const long long first = static_cast<long long>(blockIdx.x) * per;
     const long long n = prm.items > first ? (prm.items - first < per ? prm.items - first : per) : 0;
     auto pipe_base = [&](int p) { return smem + kPipeOff + p * kPipeBytes; };
-    // Polling with a time limit (MMA and mover warps): call after each round
-    // without progress; false once the limit is spent or another role aborted.
-    uint64_t t_idle = 0;
-    int idle_rounds = 0;
-    auto idle_ok = [&](bool progressed, unsigned int where) -> bool {
-        if (progressed) {
-            t_idle = 0;
-            idle_rounds = 0;
-            return true;
-        }
-        if (++idle_rounds < 64) return true;
-        idle_rounds = 0;
-        if (*ctl.abort_flag) return false;
-        const uint64_t now = globaltimer_ns();
-        if (t_idle == 0) t_idle = now;
-        if (now - t_idle <= ctl.limit_ns) return true;
-        atomicCAS(ctl.status, 0u, (kErrTimeout << 24) | (where & 0xFFFFFFu));
-        *ctl.abort_flag = 1;
-        __threadfence_block();
-        return false;
-    };
-
-    if (warp == kWarpMma) {
-        // ------------------------------------------------------------ MMA issue
-        if (lane == 0) {
-            const uint32_t id_qkv = make_idesc(kTile, kQkvRows, false, false, false);  // bf16 x, W_qkv
-            const uint32_t id_s = make_idesc(kTile, kTile, false, false, true);         // fp16 Q', K'
-            const uint32_t id_pv = make_idesc(kTile, kHeadDim, false, true, false);     // P (TMEM) x V, bf16
-            const uint32_t id_y = make_idesc(kTile, C, false, false, false);            // bf16 O, W_o
-            const uint32_t sbase = smem_u32(smem);
-            const uint64_t dK0 = make_sdesc(sbase, 16, 512, kSw64);     // K-major, 64-byte rows
-            const uint64_t dMN0 = make_sdesc(sbase, 8192, 512, kSw64);  // MN-major, 64-byte rows
-            auto u16 = [](int bytes) { return static_cast<uint64_t>(bytes >> 4); };
-            // q|k|v of head h of pipeline p's item: x (its chunk tiles) times the head's 96 W_qkv rows
-            auto issue_qkv = [&](int p, int h) {
-                const int pb = kPipeOff + p * kPipeBytes;
-                for (int c = 0; c < heads; ++c)
-#pragma unroll
-                    for (int ks = 0; ks < 2; ++ks)
-                        umma_ss(tmem + 256 * p + kColQKV, dK0 + u16(pb + kPX + c * kTileBytes) + 2 * ks,
-                                dK0 + u16(kWqkvOff + c * kWqkvChunk + h * kQkvRows * kRowBytes) + 2 * ks, id_qkv,
-                                (c | ks) != 0);
-                umma_commit(&bars->pp[p].qkv_full);
-                // the last head's q|k|v is the last MMA that reads the item's x:
-                // the mover may refill the buffer once it completes
-                if (h == heads - 1) umma_commit(&bars->pp[p].x_free);
-            };
-            struct State {
-                long long jj;  // the pipeline's item (pipeline-local index)
-                int h, step;   // head; 0: item start, 1: S, 2: P V, 3: Y
-                uint32_t hc;   // heads done (phase of the per-head barriers)
-                bool done;
-            };
-            State st[kPipes];
-            for (int p = 0; p < kPipes; ++p) st[p] = State{0, 0, 0, 0u, p >= n};
-            bool ok = true;
-            while (ok && !(st[0].done && st[1].done)) {
-                bool prog = false;
-                for (int p = 0; p < kPipes; ++p) {
-                    State& S = st[p];
-                    if (S.done) continue;
-                    PipeBars& B = bars->pp[p];
-                    const uint32_t tb = tmem + 256 * p;
-                    const int pb = kPipeOff + p * kPipeBytes;
-                    if (S.step == 0) {  // the item's x landed; the rows have read the previous Y
-                        if (!mbar_test(&B.x_full, static_cast<uint32_t>(S.jj & 1))) continue;
-                        if (S.jj > 0 && !mbar_test(&B.y_free, static_cast<uint32_t>((S.jj - 1) & 1))) continue;
-                        tc_fence_after();
-                        issue_qkv(p, 0);
-                        S.h = 0;
-                        S.step = 1;
-                    } else if (S.step == 1) {  // the rows have read q|k|v and written q', k', v
-                        if (!mbar_test(&B.in_ready, S.hc & 1u)) continue;
-                        tc_fence_after();
-#pragma unroll
-                        for (int ks = 0; ks < kHeadDim / 16; ++ks)
-                            umma_ss(tb + kColS, dK0 + u16(pb + kPHead) + 2 * ks,
-                                    dK0 + u16(pb + kPHead + kTileBytes) + 2 * ks, id_s, ks > 0);
-                        umma_commit(&B.s_full);
-                        if (S.h + 1 < heads) issue_qkv(p, S.h + 1);  // during this head's softmax
-                        S.step = 2;
-                    } else if (S.step == 2) {  // P written
-                        if (!mbar_test(&B.p_ready, S.hc & 1u)) continue;
-                        tc_fence_after();
-#pragma unroll
-                        for (int k = 0; k < kTile / 16; ++k)
-                            umma_ts(tb + kColO, tb + kColS + 8 * k, dMN0 + u16(pb + kPHead + 2 * kTileBytes) + 64 * k,
-                                    id_pv, k > 0);
-                        umma_commit(&B.o_full);
-                        ++S.hc;
-                        ++S.h;
-                        S.step = S.h < heads ? 1 : 3;
-                    } else {  // every o tile written: Y
-                        if (!mbar_test(&B.o_ready, static_cast<uint32_t>(S.jj & 1))) continue;
-                        tc_fence_after();
-                        for (int h = 0; h < heads; ++h)
-#pragma unroll
-                            for (int ks = 0; ks < 2; ++ks)
-                                umma_ss(tb + kColY, dK0 + u16(pb + kPO + h * kTileBytes) + 2 * ks,
-                                        dK0 + u16(kWoOff + h * kWoChunk) + 2 * ks, id_y, (h | ks) != 0);
-                        umma_commit(&B.y_full);
-                        ++S.jj;
-                        S.step = 0;
-                        S.done = p + 2 * S.jj >= n;
-                    }
-                    prog = true;
-                }
-                ok = idle_ok(prog, 0x5201);
-            }
-            umma_commit(&bars->done);
-            mbar_wait(&bars->done, 0, ctl, 0x52ff);
-        }
-        __syncwarp();
-    } else if (warp >= kWarpMover) {
+    if (warp >= kWarpMover) {
         // ------------------------------------------------------------ x rows in, y rows out (pipeline p)
         // Lane l moves 16-byte chunk l % 4 of row 8 i + l / 4 of each group of 32
         // rows: every instruction moves 8 whole 64-byte rows of one chunk tile.
@@ -376,6 +260,33 @@ __global__ void __launch_bounds__(kThreads, 1) block_kernel(const __grid_constan
         uint8_t* vt = qt + 2 * kTileBytes;
         uint32_t gph = 0, hc = 0;
         bool ok = true;
+        // thread 0 of the pipeline issues its MMAs: per head q|k|v (the next
+        // head's right after this head's S), S = Q'K'^T once every row is
+        // rotated, O_h = P V once every warp has written P; per item Y
+        const bool issuer = r == 0;
+        const uint32_t id_qkv = make_idesc(kTile, kQkvRows, false, false, false);  // bf16 x, W_qkv
+        const uint32_t id_s = make_idesc(kTile, kTile, false, false, true);         // fp16 Q', K'
+        const uint32_t id_pv = make_idesc(kTile, kHeadDim, false, true, false);     // P (TMEM) x V, bf16
+        const uint32_t id_y = make_idesc(kTile, C, false, false, false);            // bf16 O, W_o
+        const uint32_t sbase = smem_u32(smem);
+        const uint64_t dK0 = make_sdesc(sbase, 16, 512, kSw64);     // K-major, 64-byte rows
+        const uint64_t dMN0 = make_sdesc(sbase, 8192, 512, kSw64);  // MN-major, 64-byte rows
+        auto u16 = [](int bytes) { return static_cast<uint64_t>(bytes >> 4); };
+        const uint32_t tb = tmem + 256 * p;
+        const int pbo = kPipeOff + p * kPipeBytes;
+        // q|k|v of head h: x (its chunk tiles) times the head's 96 W_qkv rows
+        auto issue_qkv = [&](int h) {
+            for (int c = 0; c < heads; ++c)
+#pragma unroll
+                for (int ks = 0; ks < 2; ++ks)
+                    umma_ss(tb + kColQKV, dK0 + u16(pbo + kPX + c * kTileBytes) + 2 * ks,
+                            dK0 + u16(kWqkvOff + c * kWqkvChunk + h * kQkvRows * kRowBytes) + 2 * ks, id_qkv,
+                            (c | ks) != 0);
+            umma_commit(&B.qkv_full);
+            // the last head's q|k|v is the last MMA that reads the item's x:
+            // the mover may refill the buffer once it completes
+            if (h == heads - 1) umma_commit(&B.x_free);
+        };
         auto wwait = [&](uint64_t* bar, uint32_t ph, unsigned int where) -> bool {
             return __all_sync(0xFFFFFFFFu, mbar_wait(bar, ph, ctl, where));
         };
@@ -393,6 +304,15 @@ __global__ void __launch_bounds__(kThreads, 1) block_kernel(const __grid_constan
             slot_token(g, X, r, 0, &pi, &pj, &tok0);
             const uint64_t segs = d_tile_segs(g, X, d_tile_win(g, X));
             const uint32_t a16 = allow16(g, seg_at(segs, r >> g.lBT), segs);  // bit c: columns [16c, 16c+16)
+            if (issuer) {  // the item's x landed; every row has read the previous Y
+                if (!mbar_wait(&B.x_full, static_cast<uint32_t>(jj & 1), ctl, 0x5201) ||
+                    (jj > 0 && !mbar_wait(&B.y_free, static_cast<uint32_t>((jj - 1) & 1), ctl, 0x5202))) {
+                    ok = false;
+                } else {
+                    tc_fence_after();
+                    issue_qkv(0);
+                }
+            }
             for (int h = 0; h < heads && ok; ++h, ++hc) {
                 const uint32_t ph = hc & 1u;
                 const float2* tab = tabs + h * kTabPerHead;
@@ -413,8 +333,16 @@ __global__ void __launch_bounds__(kThreads, 1) block_kernel(const __grid_constan
                 }
                 tc_fence_before();
                 fence_proxy_async_smem();
-                if (!group_sync(0x5302)) { ok = false; break; }
-                if (r == 0) mbar_arrive(&B.in_ready);
+                if (!group_sync(0x5302)) { ok = false; break; }  // every row's q', k', v written, its q|k|v read
+                if (issuer) {
+                    tc_fence_after();
+#pragma unroll
+                    for (int ks = 0; ks < kHeadDim / 16; ++ks)
+                        umma_ss(tb + kColS, dK0 + u16(pbo + kPHead) + 2 * ks,
+                                dK0 + u16(pbo + kPHead + kTileBytes) + 2 * ks, id_s, ks > 0);
+                    umma_commit(&B.s_full);
+                    if (h + 1 < heads) issue_qkv(h + 1);  // during this head's softmax
+                }
                 // softmax of this query row: the maximum, then probabilities and their sum
                 if (!wwait(&B.s_full, ph, 0x5303)) { ok = false; break; }
                 tc_fence_after();
@@ -467,6 +395,14 @@ __global__ void __launch_bounds__(kThreads, 1) block_kernel(const __grid_constan
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&B.p_ready);
+                if (issuer && mbar_wait(&B.p_ready, ph, ctl, 0x5203)) {  // every warp's P written
+                    tc_fence_after();
+#pragma unroll
+                    for (int k = 0; k < kTile / 16; ++k)
+                        umma_ts(tb + kColO, tb + kColS + 8 * k, dMN0 + u16(pbo + kPHead + 2 * kTileBytes) + 64 * k,
+                                id_pv, k > 0);
+                    umma_commit(&B.o_full);
+                }
                 // O_h / l into the head's o tile
                 if (!wwait(&B.o_full, ph, 0x5304)) { ok = false; break; }
                 tc_fence_after();
@@ -489,6 +425,15 @@ __global__ void __launch_bounds__(kThreads, 1) block_kernel(const __grid_constan
             fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0) mbar_arrive(&B.o_ready);
+            if (issuer && mbar_wait(&B.o_ready, static_cast<uint32_t>(jj & 1), ctl, 0x5204)) {  // every o tile written
+                tc_fence_after();
+                for (int h = 0; h < heads; ++h)
+#pragma unroll
+                    for (int ks = 0; ks < 2; ++ks)
+                        umma_ss(tb + kColY, dK0 + u16(pbo + kPO + h * kTileBytes) + 2 * ks,
+                                dK0 + u16(kWoOff + h * kWoChunk) + 2 * ks, id_y, (h | ks) != 0);
+                umma_commit(&B.y_full);
+            }
             // y = Y + b_o into the staging tiles (the o tiles, read by the finished Y MMAs)
             if (!wwait(&B.y_full, static_cast<uint32_t>(jj & 1), 0x5306)) break;
             tc_fence_after();
@@ -508,6 +453,10 @@ __global__ void __launch_bounds__(kThreads, 1) block_kernel(const __grid_constan
                 mbar_arrive(&B.y_free);
                 mbar_arrive(&B.staged);  // the mover stores them
             }
+        }
+        if (issuer) {  // every MMA issued here has completed before the columns are freed
+            umma_commit(&bars->done);
+            mbar_wait(&bars->done, 0, ctl, 0x52ff);
         }
     }
 

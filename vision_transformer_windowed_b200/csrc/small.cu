@@ -47,10 +47,11 @@ __device__ __forceinline__ void small_item(const Geo& g, bool head_minor, long l
 //   warps 0-3: thread = slot row.  D, lse and the RoPE of its q and k rows;
 //              the row of P^T and dS^T of its key; the epilogue of its token
 //              (dq, dk un-rotated, dv, the d theta terms), staged over the
-//              slot's q, k, v rows.
-//   warp 4:    MMA issuer: S^T = K' Q'^T, dP^T = V dO^T; then dV = P^T dO,
-//              dK' = dS^T Q', dQ' = dS K'.
-//   warp 5:    mover: the q, k, v, dO rows of each item (and its o rows) with
+//              slot's q, k, v rows.  Thread 0 also issues the MMAs:
+//              S^T = K' Q'^T, dP^T = V dO^T right after the barrier that ends
+//              the rotation, then dV = P^T dO, dK' = dS^T Q', dQ' = dS K' once
+//              every warp has written P^T, dS^T and dS.
+//   warp 4:    mover: the q, k, v, dO rows of each item (and its o rows) with
 //              16-byte async copies one item ahead, completing on mbarriers (a
 //              window box of a shifted grid is as small as 4 x 4 tokens, too
 //              small for TMA box copies to keep up), and the stores of the
@@ -60,8 +61,8 @@ __device__ __forceinline__ void small_item(const Geo& g, bool head_minor, long l
 // are adjacent in memory, are read close together in time.
 namespace bwd {
 
-constexpr int kThreads = 192;
-constexpr int kWarpMma = 4, kWarpMover = 5;
+constexpr int kThreads = 160;
+constexpr int kWarpMover = 4;
 constexpr int kSlotBytes = 4 * kTileBytes;        // q, k, v, dO tiles of one item
 constexpr int kSlotOff = 0;                        // 2 slots
 constexpr int kOOff = 2 * kSlotBytes;              // o tile
@@ -77,7 +78,7 @@ constexpr uint32_t kColS = 0, kColDP = 128, kColP = 0, kColDS = 128;
 constexpr uint32_t kColDV = 64, kColDQ = 96, kColDK = 192;
 
 struct Bars {
-    uint64_t in_ready, s_full, p_ready, mma2_done, tmem_free, grp, done;
+    uint64_t s_full, p_ready, mma2_done, grp, done;
     uint64_t slot_full[2], o_full, o_free, staged;  // row copies and stores (mover warp)
     uint32_t tmem_base;
     int abort_flag;
@@ -105,11 +106,9 @@ __global__ void __launch_bounds__(kThreads, 2) small_kernel(const __grid_constan
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
     if (tid == 0) {
-        mbar_init(&bars->in_ready, 1);
         mbar_init(&bars->s_full, 1);
         mbar_init(&bars->p_ready, 4);
         mbar_init(&bars->mma2_done, 1);
-        mbar_init(&bars->tmem_free, 4);
         mbar_init(&bars->grp, 4);
         mbar_init(&bars->done, 1);
         mbar_init(&bars->slot_full[0], 32);  // one cp.async arrival per mover lane
@@ -137,50 +136,7 @@ __global__ void __launch_bounds__(kThreads, 2) small_kernel(const __grid_constan
     const long long n = prm.items > first ? (prm.items - first < per ? prm.items - first : per) : 0;
     auto item_at = [&](long long j) { return first + j; };
 
-    if (warp == kWarpMma) {
-        // ------------------------------------------------------------ MMA issue
-        if (lane == 0) {
-            const uint32_t id_s = make_idesc(kTile, kTile, false, false, true);     // fp16 K', Q'
-            const uint32_t id_dp = make_idesc(kTile, kTile, false, false, false);   // bf16 V, dO
-            const uint32_t id_dv = make_idesc(kTile, kHeadDim, false, true, false); // P^T (TMEM) x dO
-            const uint32_t id_dk = make_idesc(kTile, kHeadDim, false, true, true);  // dS^T (TMEM) x Q'
-            const uint32_t id_dq = make_idesc(kTile, kHeadDim, true, true, true);   // dS (smem) x K'
-            // descriptors built once; per MMA only an offset in 16-byte units is added
-            const uint32_t sbase = smem_u32(smem);
-            const uint64_t dK0 = make_sdesc(sbase, 16, 512, kSw64);        // K-major, 64-byte rows
-            const uint64_t dMN0 = make_sdesc(sbase, 8192, 512, kSw64);     // MN-major, 64-byte rows
-            const uint64_t dDS = make_sdesc(sbase + kDSOff, 16384, 1024, kSw128);
-            for (long long j = 0; j < n; ++j) {
-                const uint32_t ph = static_cast<uint32_t>(j & 1);
-                if (!mbar_wait(&bars->in_ready, ph, ctl, 0x2201)) break;
-                if (j > 0 && !mbar_wait(&bars->tmem_free, ph ^ 1, ctl, 0x2202)) break;
-                tc_fence_after();
-                const uint64_t qo = static_cast<uint64_t>((kSlotOff + (j & 1) * kSlotBytes) >> 4);
-                const uint64_t ko = qo + (kTileBytes >> 4), vo = qo + (2 * kTileBytes >> 4), dof = qo + (3 * kTileBytes >> 4);
-#pragma unroll
-                for (int k = 0; k < kHeadDim / 16; ++k) umma_ss(tmem + kColS, dK0 + ko + 2 * k, dK0 + qo + 2 * k, id_s, k > 0);
-#pragma unroll
-                for (int k = 0; k < kHeadDim / 16; ++k)
-                    umma_ss(tmem + kColDP, dK0 + vo + 2 * k, dK0 + dof + 2 * k, id_dp, k > 0);
-                umma_commit(&bars->s_full);
-                if (!mbar_wait(&bars->p_ready, ph, ctl, 0x2203)) break;
-                tc_fence_after();
-#pragma unroll
-                for (int k = 0; k < kTile / 16; ++k)
-                    umma_ts(tmem + kColDV, tmem + kColP + 8 * k, dMN0 + dof + 64 * k, id_dv, k > 0);
-#pragma unroll
-                for (int k = 0; k < kTile / 16; ++k)
-                    umma_ts(tmem + kColDK, tmem + kColDS + 8 * k, dMN0 + qo + 64 * k, id_dk, k > 0);
-#pragma unroll
-                for (int k = 0; k < kTile / 16; ++k)
-                    umma_ss(tmem + kColDQ, dDS + 128 * k, dMN0 + ko + 64 * k, id_dq, k > 0);
-                umma_commit(&bars->mma2_done);
-            }
-            umma_commit(&bars->done);
-            mbar_wait(&bars->done, 0, ctl, 0x22ff);
-        }
-        __syncwarp();
-    } else if (warp == kWarpMover) {
+    if (warp == kWarpMover) {
         // ------------------------------------------------------------ row copies and result stores
         // Lane l moves 16-byte chunk l % 4 of row 8 i + l / 4 of each group of 32
         // rows: every instruction moves 8 whole 64-byte rows.  Copies arrive on an
@@ -268,6 +224,17 @@ __global__ void __launch_bounds__(kThreads, 2) small_kernel(const __grid_constan
         cp_async_wait<0>();
     } else {
         // ------------------------------------------------------------ rows (warps 0-3)
+        // thread 0 also issues the MMAs: S^T, dP^T once every row is rotated,
+        // the gradients once every warp has written P^T, dS^T and dS
+        const uint32_t id_s = make_idesc(kTile, kTile, false, false, true);     // fp16 K', Q'
+        const uint32_t id_dp = make_idesc(kTile, kTile, false, false, false);   // bf16 V, dO
+        const uint32_t id_dv = make_idesc(kTile, kHeadDim, false, true, false); // P^T (TMEM) x dO
+        const uint32_t id_dk = make_idesc(kTile, kHeadDim, false, true, true);  // dS^T (TMEM) x Q'
+        const uint32_t id_dq = make_idesc(kTile, kHeadDim, true, true, true);   // dS (smem) x K'
+        const uint32_t sbase = smem_u32(smem);
+        const uint64_t dK0 = make_sdesc(sbase, 16, 512, kSw64);        // K-major, 64-byte rows
+        const uint64_t dMN0 = make_sdesc(sbase, 8192, 512, kSw64);     // MN-major, 64-byte rows
+        const uint64_t dDS = make_sdesc(sbase + kDSOff, 16384, 1024, kSw128);
         const int r = tid;
         const uint32_t trow = tmem + (static_cast<uint32_t>(warp * 32) << 16);
         const float sl2 = g.scale_log2;
@@ -376,8 +343,18 @@ __global__ void __launch_bounds__(kThreads, 2) small_kernel(const __grid_constan
                 store_row_swz(sl + kTileBytes, r, x, true);
             }
             fence_proxy_async_smem();
-            if (!group_sync(0x2306)) break;
-            if (r == 0) mbar_arrive(&bars->in_ready);
+            if (!group_sync(0x2306)) break;  // every row rotated; the previous item's products read by every warp
+            if (r == 0) {
+                tc_fence_after();
+                const uint64_t qo = static_cast<uint64_t>((kSlotOff + (j & 1) * kSlotBytes) >> 4);
+                const uint64_t ko = qo + (kTileBytes >> 4), vo = qo + (2 * kTileBytes >> 4), dof = qo + (3 * kTileBytes >> 4);
+#pragma unroll
+                for (int k = 0; k < kHeadDim / 16; ++k) umma_ss(tmem + kColS, dK0 + ko + 2 * k, dK0 + qo + 2 * k, id_s, k > 0);
+#pragma unroll
+                for (int k = 0; k < kHeadDim / 16; ++k)
+                    umma_ss(tmem + kColDP, dK0 + vo + 2 * k, dK0 + dof + 2 * k, id_dp, k > 0);
+                umma_commit(&bars->s_full);
+            }
             const float lse_nxt = (j + 1 < n && nxt.valid) ? __ldg(prm.lse + nxt.tok) : 0.f;
             // row of P^T and dS^T of this key, 32 query columns at a time
             if (!wwait(&bars->s_full, ph, 0x2307)) break;
@@ -436,6 +413,21 @@ __global__ void __launch_bounds__(kThreads, 2) small_kernel(const __grid_constan
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&bars->p_ready);
+            if (r == 0 && mbar_wait(&bars->p_ready, ph, ctl, 0x2203)) {  // every warp's P^T, dS^T and dS written
+                tc_fence_after();
+                const uint64_t qo = static_cast<uint64_t>((kSlotOff + (j & 1) * kSlotBytes) >> 4);
+                const uint64_t ko = qo + (kTileBytes >> 4), dof = qo + (3 * kTileBytes >> 4);
+#pragma unroll
+                for (int k = 0; k < kTile / 16; ++k)
+                    umma_ts(tmem + kColDV, tmem + kColP + 8 * k, dMN0 + dof + 64 * k, id_dv, k > 0);
+#pragma unroll
+                for (int k = 0; k < kTile / 16; ++k)
+                    umma_ts(tmem + kColDK, tmem + kColDS + 8 * k, dMN0 + qo + 64 * k, id_dk, k > 0);
+#pragma unroll
+                for (int k = 0; k < kTile / 16; ++k)
+                    umma_ss(tmem + kColDQ, dDS + 128 * k, dMN0 + ko + 64 * k, id_dq, k > 0);
+                umma_commit(&bars->mma2_done);
+            }
             // the next item's masks while the MMAs run
             const uint32_t a16_nxt = j + 1 < n ? row_mask(nxt) : 0u;
             // epilogue of this row's token: dq, dk (un-rotated), dv, d theta terms
@@ -472,9 +464,8 @@ __global__ void __launch_bounds__(kThreads, 2) small_kernel(const __grid_constan
                 uint32_t t[32];
                 tmem_ld32(trow + kColDV, t);
                 tmem_wait_ld();
-                tc_fence_before();
+                tc_fence_before();  // ordered before the next item's MMAs by its group barrier
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&bars->tmem_free);
                 float x[32];
 #pragma unroll
                 for (int e = 0; e < 32; ++e) x[e] = __uint_as_float(t[e]);
@@ -508,6 +499,10 @@ __global__ void __launch_bounds__(kThreads, 2) small_kernel(const __grid_constan
             lse_cur = lse_nxt;
             a16 = a16_nxt;
         }
+        if (r == 0) {  // every MMA issued here has completed before the columns are freed
+            umma_commit(&bars->done);
+            mbar_wait(&bars->done, 0, ctl, 0x22ff);
+        }
     }
 
     tc_fence_before();
@@ -524,12 +519,13 @@ __global__ void __launch_bounds__(kThreads, 2) small_kernel(const __grid_constan
 // rescale.  TMEM: S [0,128), P (bf16) over S [0,64), O over S [64,96): 128
 // columns, so up to four CTAs share an SM.
 //   warps 0-3: thread = slot row: copies, RoPE of its q and k rows, the
-//              softmax of its query, the epilogue (O / l, log-sum-exp)
-//   warp 4:    MMA issuer: S = Q'K'^T, then O = P V
+//              softmax of its query, the epilogue (O / l, log-sum-exp);
+//              thread 0 also issues S = Q'K'^T right after the barrier that
+//              ends the rotation, and O = P V once every warp has written P
+//              (no separate MMA warp: each hand-off to one cost a wake-up)
 namespace fwd {
 
-constexpr int kThreads = 160;
-constexpr int kWarpMma = 4;
+constexpr int kThreads = 128;
 constexpr int kSlotBytes = 3 * kTileBytes;  // q, k, v tiles of one item
 constexpr int kSlotOff = 0;                  // 2 slots
 constexpr int kTabOff = 2 * kSlotBytes;
@@ -539,7 +535,7 @@ constexpr uint32_t kTmemCols = 128;
 constexpr uint32_t kColS = 0, kColP = 0, kColO = 64;
 
 struct Bars {
-    uint64_t in_ready, s_full, p_ready, o_full, tmem_free, grp, done;
+    uint64_t s_full, p_ready, o_full, grp, done;
     uint32_t tmem_base;
     int abort_flag;
 };
@@ -565,11 +561,9 @@ __global__ void __launch_bounds__(kThreads, 4) fwd_kernel(const __grid_constant_
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
     if (tid == 0) {
-        mbar_init(&bars->in_ready, 1);
         mbar_init(&bars->s_full, 1);
         mbar_init(&bars->p_ready, 4);
         mbar_init(&bars->o_full, 1);
-        mbar_init(&bars->tmem_free, 4);
         mbar_init(&bars->grp, 4);
         mbar_init(&bars->done, 1);
         bars->abort_flag = 0;
@@ -591,36 +585,14 @@ __global__ void __launch_bounds__(kThreads, 4) fwd_kernel(const __grid_constant_
     const long long n = prm.items > first ? (prm.items - first < per ? prm.items - first : per) : 0;
     auto item_at = [&](long long j) { return first + j; };
 
-    if (warp == kWarpMma) {
-        // ------------------------------------------------------------ MMA issue
-        if (lane == 0) {
-            const uint32_t id_s = make_idesc(kTile, kTile, false, false, true);  // fp16 Q', K'
-            const uint32_t id_pv = make_idesc_bf16(kTile, kHeadDim, false, true);  // P (TMEM) x V
-            // descriptors built once; per MMA only an offset in 16-byte units is added
-            const uint32_t sbase = smem_u32(smem);
-            const uint64_t dK0 = make_sdesc(sbase, 16, 512, kSw64);     // K-major, 64-byte rows
-            const uint64_t dMN0 = make_sdesc(sbase, 8192, 512, kSw64);  // MN-major, 64-byte rows
-            for (long long j = 0; j < n; ++j) {
-                const uint32_t ph = static_cast<uint32_t>(j & 1);
-                if (!mbar_wait(&bars->in_ready, ph, ctl, 0x3201)) break;
-                if (j > 0 && !mbar_wait(&bars->tmem_free, ph ^ 1, ctl, 0x3202)) break;
-                tc_fence_after();
-                const uint64_t qo = static_cast<uint64_t>((kSlotOff + (j & 1) * kSlotBytes) >> 4);
-                const uint64_t ko = qo + (kTileBytes >> 4), vo = qo + (2 * kTileBytes >> 4);
-#pragma unroll
-                for (int k = 0; k < kHeadDim / 16; ++k) umma_ss(tmem + kColS, dK0 + qo + 2 * k, dK0 + ko + 2 * k, id_s, k > 0);
-                umma_commit(&bars->s_full);
-                if (!mbar_wait(&bars->p_ready, ph, ctl, 0x3203)) break;
-                tc_fence_after();
-#pragma unroll
-                for (int k = 0; k < kTile / 16; ++k) umma_ts(tmem + kColO, tmem + kColP + 8 * k, dMN0 + vo + 64 * k, id_pv, k > 0);
-                umma_commit(&bars->o_full);
-            }
-            umma_commit(&bars->done);
-            mbar_wait(&bars->done, 0, ctl, 0x32ff);
-        }
-        __syncwarp();
-    } else {
+    {
+        // thread 0 also issues the MMAs (S = Q'K'^T once the four warps have
+        // rotated their rows, O = P V once they have written P)
+        const uint32_t id_s = make_idesc(kTile, kTile, false, false, true);     // fp16 Q', K'
+        const uint32_t id_pv = make_idesc_bf16(kTile, kHeadDim, false, true);  // P (TMEM) x V
+        const uint32_t sbase = smem_u32(smem);
+        const uint64_t dK0 = make_sdesc(sbase, 16, 512, kSw64);     // K-major, 64-byte rows
+        const uint64_t dMN0 = make_sdesc(sbase, 8192, 512, kSw64);  // MN-major, 64-byte rows
         // ------------------------------------------------------------ rows (warps 0-3)
         const int r = tid;
         const uint32_t trow = tmem + (static_cast<uint32_t>(warp * 32) << 16);
@@ -723,8 +695,15 @@ __global__ void __launch_bounds__(kThreads, 4) fwd_kernel(const __grid_constant_
                 store_row_swz(sl + kTileBytes, r, x, true);
             }
             fence_proxy_async_smem();
-            if (!group_sync(0x3304)) break;
-            if (r == 0) mbar_arrive(&bars->in_ready);
+            if (!group_sync(0x3304)) break;  // every row rotated; the previous item's O read by every warp
+            if (r == 0) {
+                tc_fence_after();
+                const uint64_t qo = static_cast<uint64_t>((kSlotOff + (j & 1) * kSlotBytes) >> 4);
+                const uint64_t ko = qo + (kTileBytes >> 4);
+#pragma unroll
+                for (int k = 0; k < kHeadDim / 16; ++k) umma_ss(tmem + kColS, dK0 + qo + 2 * k, dK0 + ko + 2 * k, id_s, k > 0);
+                umma_commit(&bars->s_full);
+            }
             const RowTok nxt = j + 1 < n ? row_tok(j + 1) : RowTok{};
             // softmax of this query row: the maximum, then probabilities and their sum
             if (!wwait(&bars->s_full, ph, 0x3305)) break;
@@ -778,6 +757,13 @@ __global__ void __launch_bounds__(kThreads, 4) fwd_kernel(const __grid_constant_
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&bars->p_ready);
+            if (r == 0 && mbar_wait(&bars->p_ready, ph, ctl, 0x3203)) {  // every warp's P written
+                tc_fence_after();
+                const uint64_t vo = static_cast<uint64_t>((kSlotOff + (j & 1) * kSlotBytes + 2 * kTileBytes) >> 4);
+#pragma unroll
+                for (int k = 0; k < kTile / 16; ++k) umma_ts(tmem + kColO, tmem + kColP + 8 * k, dMN0 + vo + 64 * k, id_pv, k > 0);
+                umma_commit(&bars->o_full);
+            }
             const uint32_t a16_nxt = j + 1 < n ? row_mask(nxt) : 0u;
             // epilogue: O / l into the staging rows (over q'), log-sum-exp
             if (!wwait(&bars->o_full, ph, 0x3306)) break;
@@ -786,9 +772,8 @@ __global__ void __launch_bounds__(kThreads, 4) fwd_kernel(const __grid_constant_
                 uint32_t t[32];
                 tmem_ld32(trow + kColO, t);
                 tmem_wait_ld();
-                tc_fence_before();
+                tc_fence_before();  // ordered before the next item's S by its group barrier
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&bars->tmem_free);
                 const float inv = 1.f / l;
                 float x[32];
 #pragma unroll
@@ -816,6 +801,10 @@ __global__ void __launch_bounds__(kThreads, 4) fwd_kernel(const __grid_constant_
             a16 = a16_nxt;
         }
         cp_async_wait<0>();
+        if (r == 0) {  // every MMA issued here has completed before the columns are freed
+            umma_commit(&bars->done);
+            mbar_wait(&bars->done, 0, ctl, 0x32ff);
+        }
     }
 
     tc_fence_before();
