@@ -1,0 +1,61 @@
+"""CPU checks of the benchmark's host logic: the count of attending pairs the
+flop figures rest on, the per-workload figures, and the CPU-baseline leg."""
+import numpy as np
+import pytest
+
+import oracle
+
+import bench
+from vision_transformer_windowed_b200.inputs import make_inputs
+
+
+def _brute_pairs(B, H, W, heads, M, s):
+    """(query, key) pairs of one window with equal region labels, counted token
+    by token on the grid padded to multiples of M, times B and heads."""
+    Hp, Wp = -(-H // M) * M, -(-W // M) * M
+    lab = oracle.labels(Hp, Wp, M, s)
+    n = 0
+    for wr in range(Hp // M):
+        for wc in range(Wp // M):
+            cell = lab[wr * M:(wr + 1) * M, wc * M:(wc + 1) * M].ravel()
+            _, counts = np.unique(cell, return_counts=True)
+            n += int((counts ** 2).sum())
+    return n * B * heads
+
+
+@pytest.mark.parametrize("shape", [(2, 16, 16, 3, 8, 0), (2, 16, 16, 3, 8, 4), (1, 64, 64, 1, 32, 16),
+                                   (1, 20, 13, 2, 8, 4), (1, 40, 36, 1, 16, 8), (3, 24, 40, 2, 8, 0)])
+def test_unmasked_pairs_match_brute_force(shape):
+    assert bench.unmasked_pairs(*shape) == _brute_pairs(*shape)
+
+
+def test_workload_flops_count_every_shift():
+    wl = dict(B=2, H=16, W=16, heads=3, M=8, shifts=(0, 4), qk_scale=1.0)
+    pairs = sum(_brute_pairs(2, 16, 16, 3, 8, s) for s in (0, 4))
+    fwd, bwd = bench.workload_flops(wl)
+    assert fwd == 4 * 32 * pairs and bwd == 10 * 32 * pairs
+
+
+def test_config_entry_figures():
+    wl = dict(B=1, H=16, W=16, heads=2, M=8, shifts=(0, 4), qk_scale=1.0)
+    fwd_f, bwd_f = bench.workload_flops(wl)
+    r = {"ms": 2.0, "tflops": (fwd_f + bwd_f) / 2e-3 / 1e12, "tokens_per_s": 1.0, "peak_gb": 0.5,
+         "phase_ms": {"fwd": 0.25}, "fwd_flops": fwd_f, "bwd_flops": bwd_f, "ws_bytes": 1000}
+    peaks = {"bf16_tflops": 1000.0}
+    e = bench.config_entry(wl, r, peaks, 1)
+    assert e["fwd_tflops"] == pytest.approx(fwd_f / 0.5e-3 / 1e12)  # two forward calls of 0.25 ms
+    assert e["tflops_no_recompute"] == pytest.approx((fwd_f + 0.8 * bwd_f) / 2e-3 / 1e12)
+    assert e["pct_bf16_spec"] == pytest.approx(100 * r["tflops"] / bench.SPEC_BF16_TFLOPS)
+    assert e["fwd_gbs"] == pytest.approx(260 * 16 * 16 * 2 * 2 / 0.5e-3 / 1e9)
+    assert e["bwd_workspace_gb"] == pytest.approx(1e-6)
+
+
+def test_cpu_baseline_samples_every_unit_of_a_small_workload():
+    wl = dict(B=1, H=20, W=13, heads=2, M=8, shifts=(0, 4), qk_scale=1.0)  # padded: 3 x 2 windows
+    t = make_inputs(1, 20, 13, 2, 32)
+    res = bench.cpu_baseline(t, wl, seconds=2.0)
+    n_units = 1 * 3 * 2 * 2
+    assert res["kind"] == "oracle" and res["value"] > 0 and res["cores"] >= 1
+    assert f"{n_units} of {n_units} at s=0" in res["sample"] and f"{n_units} of {n_units} at s=4" in res["sample"]
+    assert res["units_per_s"] == pytest.approx(2 * n_units / res["seconds"])
+    assert res["full_step_s_extrapolated"] == pytest.approx(res["seconds"])
