@@ -583,9 +583,9 @@ def main():
                        "l2": "inputs larger than L2 (each tensor > 126 MB)"},
             "pct_bf16_peak": 100 * main_res["tflops"] / peaks["bf16_tflops"] / world,
             "tokens_per_s": main_res["tokens_per_s"], "peak_gb": main_res["peak_gb"],
-            # per shift: the forward, then the one-tile backward and the two-level d theta sum
-            # (windows inside one tile) or prep, main, post and the d theta sum
-            "gpu_launches": args.steps * nshift * (1 + (3 if M * M < 128 else 5)),
+            # per shift: the forward, then the one-tile backward and the d theta sum (windows
+            # inside one tile) or prep, main, post and the d theta sum
+            "gpu_launches": args.steps * nshift * (1 + (2 if M * M < 128 else 4)),
             "roofline": roof, "clocks": main_res["clocks"], "e2e": e2e, "cpu_baseline": cpu,
             "per_config": per_config, "peaks": peaks,
         }

@@ -35,7 +35,7 @@ namespace bwdk {
 
 // ------------------------------------------------------------------ workspace
 struct WsLayout {
-    size_t qimg, kimg, lse2, dvec, dqacc, part, part2, total;
+    size_t qimg, kimg, lse2, dvec, dqacc, part, part2, cnt, total;
 };
 
 __host__ __device__ inline size_t round256(size_t x) { return (x + 255) & ~size_t(255); }
@@ -51,6 +51,7 @@ __host__ __device__ inline WsLayout ws_layout(const Geo& g) {
     L.dqacc = o; o += round256(ht * kTile * kHeadDim * 4);
     L.part = o;  o += round256(ht * 8 * 16 * 4);  // up to 8 x 16 partials per (head, tile)
     L.part2 = o; o += round256(static_cast<size_t>(g.heads) * 64 * 16 * 4);  // level-1 d theta sums
+    L.cnt = o;   o += round256(static_cast<size_t>(g.heads) * 4);            // level-1 blocks done, per head
     L.total = o;
     return L;
 }
@@ -123,6 +124,8 @@ __global__ void __launch_bounds__(128) prep_kernel(const PrepParams p) {
     const long long T = blockIdx.x / g.heads;
     const int h = static_cast<int>(blockIdx.x - T * g.heads);
     const long long ht = static_cast<long long>(h) * g.tiles + T;
+    if (blockIdx.x == 0)  // the d theta reduction's counters, for its launch after this one
+        for (int i = threadIdx.x; i < g.heads; i += blockDim.x) reinterpret_cast<unsigned int*>(p.ws + p.L.cnt)[i] = 0u;
     build_table(tab, p.theta + h * 16, g.M, threadIdx.x, blockDim.x);
     __syncthreads();
     const int r = threadIdx.x;
@@ -727,19 +730,21 @@ __global__ void __launch_bounds__(128) post_kernel(const PostParams p) {
 }
 
 // ------------------------------------------------------------------ 4. reduce
-// In two launches, each in a fixed order (deterministic d theta):
-//   level 1, grid (kSplit, heads): block b of head h sums its contiguous share
-//            of the head's [per_head][16] partials into out[h][b][16];
-//   level 2, grid (1, heads): the kSplit level-1 sums of each head.
+// One launch, grid (kSplit, heads), in a fixed order (deterministic d theta):
+//   level 1: block b of head h sums its contiguous share of the head's
+//            [per_head][16] partials into scratch[h][b][16];
+//   level 2: the head's last block to finish (a per-head counter, zeroed by
+//            the kernel before this one) sums the kSplit level-1 sums.
 constexpr int kSplit = 64;
 
-__global__ void __launch_bounds__(256) dtheta_kernel(const float* part, long long per_head, float* out) {
-    __shared__ float acc[16][17];
-    const int h = blockIdx.y, b = blockIdx.x, nb = gridDim.x;
+// Rows [per_head b / nb, per_head (b + 1) / nb) of head h's [per_head][16]
+// partials: 16 groups of strided rows, then the 16 group sums, into out[h][b].
+__device__ __forceinline__ void sum_rows(const float* part, long long per_head, int h, int b, int nb, float* out,
+                                         float (&acc)[16][17]) {
     const long long lo = per_head * b / nb, hi = per_head * (b + 1) / nb;
     const int comp = threadIdx.x & 15, grp = threadIdx.x >> 4;
     float s = 0.f;
-    for (long long T = lo + grp; T < hi; T += 16) s += part[(static_cast<long long>(h) * per_head + T) * 16 + comp];
+    for (long long T = lo + grp; T < hi; T += 16) s += __ldcg(part + (static_cast<long long>(h) * per_head + T) * 16 + comp);
     acc[grp][comp] = s;
     __syncthreads();
     if (threadIdx.x < 16) {
@@ -749,13 +754,26 @@ __global__ void __launch_bounds__(256) dtheta_kernel(const float* part, long lon
     }
 }
 
-// part: [heads][per_head][16]; dtheta: [heads][16]; scratch: heads * kSplit * 16 floats
-cudaError_t launch_dtheta(const float* part, long long per_head, int heads, float* scratch, float* dtheta,
-                          cudaStream_t stream) {
-    dtheta_kernel<<<dim3(kSplit, heads), 256, 0, stream>>>(part, per_head, scratch);
-    cudaError_t e = cudaGetLastError();
-    if (e != cudaSuccess) return e;
-    dtheta_kernel<<<dim3(1, heads), 256, 0, stream>>>(scratch, kSplit, dtheta);
+__global__ void __launch_bounds__(256) dtheta_kernel(const float* part, long long per_head, float* scratch,
+                                                     unsigned int* cnt, float* out) {
+    __shared__ float acc[16][17];
+    __shared__ bool last;
+    const int h = blockIdx.y, b = blockIdx.x, nb = gridDim.x;
+    sum_rows(part, per_head, h, b, nb, scratch, acc);
+    if (threadIdx.x < 16) __threadfence();  // this block's sums visible before it is counted
+    __syncthreads();
+    if (threadIdx.x == 0) last = atomicAdd(cnt + h, 1u) == static_cast<unsigned int>(nb - 1);
+    __syncthreads();
+    if (!last) return;
+    __threadfence();
+    sum_rows(scratch, nb, h, 0, 1, out, acc);
+}
+
+// part: [heads][per_head][16]; dtheta: [heads][16]; scratch: heads * kSplit * 16 floats; cnt: heads
+// counters that are zero when the launch starts
+cudaError_t launch_dtheta(const float* part, long long per_head, int heads, float* scratch, unsigned int* cnt,
+                          float* dtheta, cudaStream_t stream) {
+    dtheta_kernel<<<dim3(kSplit, heads), 256, 0, stream>>>(part, per_head, scratch, cnt, dtheta);
     return cudaGetLastError();
 }
 
@@ -781,11 +799,13 @@ cudaError_t launch_bwd(const Geo& g, const BwdPtrs& p, const BwdMaps& maps, unsi
         float* part = reinterpret_cast<float*>(p.ws + L.part);
         mark(0);
         mark(1);
-        e = launch_small_bwd(g, p, part, status, limit_ns, num_sms, stream);
+        e = launch_small_bwd(g, p, part, reinterpret_cast<unsigned int*>(p.ws + L.cnt), status, limit_ns, num_sms,
+                             stream);
         if (e != cudaSuccess) return e;
         mark(2);
         mark(3);
-        if ((e = launch_dtheta(part, g.tiles * 4, g.heads, reinterpret_cast<float*>(p.ws + L.part2), p.dtheta,
+        if ((e = launch_dtheta(part, g.tiles * 4, g.heads, reinterpret_cast<float*>(p.ws + L.part2),
+                               reinterpret_cast<unsigned int*>(p.ws + L.cnt), p.dtheta,
                                stream)) != cudaSuccess)
             return e;
         mark(4);
@@ -824,7 +844,8 @@ cudaError_t launch_bwd(const Geo& g, const BwdPtrs& p, const BwdMaps& maps, unsi
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     mark(3);
     if ((e = launch_dtheta(reinterpret_cast<const float*>(p.ws + L.part), g.tiles * 8, g.heads,
-                           reinterpret_cast<float*>(p.ws + L.part2), p.dtheta, stream)) != cudaSuccess)
+                           reinterpret_cast<float*>(p.ws + L.part2), reinterpret_cast<unsigned int*>(p.ws + L.cnt),
+                           p.dtheta, stream)) != cudaSuccess)
         return e;
     mark(4);
     return e;

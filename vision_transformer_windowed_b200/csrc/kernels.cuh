@@ -41,8 +41,8 @@ cudaError_t launch_bwd(const Geo& g, const BwdPtrs& p, const BwdMaps& maps, unsi
 // Windows of fewer than 128 tokens (the tile holds whole windows): the whole
 // backward of a tile in one kernel (d theta partials, 4 x 16 per (head, tile),
 // into `part`), and the forward.
-cudaError_t launch_small_bwd(const Geo& g, const BwdPtrs& p, float* part, unsigned int* status,
-                             unsigned long long limit_ns, int num_sms, cudaStream_t stream);
+cudaError_t launch_small_bwd(const Geo& g, const BwdPtrs& p, float* part, unsigned int* dtheta_cnt,
+                             unsigned int* status, unsigned long long limit_ns, int num_sms, cudaStream_t stream);
 cudaError_t launch_small_fwd(const Geo& g, const void* q, const void* k, const void* v, const float* theta, void* o,
                              float* lse, unsigned int* status, unsigned long long limit_ns, int num_sms,
                              cudaStream_t stream);

@@ -91,6 +91,7 @@ struct Params {
     uint8_t *dq, *dk, *dv;
     const float *lse, *theta;
     float* part;  // [heads][tiles][16]
+    unsigned int* dtheta_cnt;  // zeroed here for the d theta reduction launched next
     unsigned int* status;
     unsigned long long limit_ns;
     long long items;
@@ -105,6 +106,8 @@ __global__ void __launch_bounds__(kThreads, 2) small_kernel(const __grid_constan
     const Geo& g = prm.g;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
+    if (blockIdx.x == 0)  // the d theta reduction's counters, for its launch after this one
+        for (int i = tid; i < g.heads; i += kThreads) prm.dtheta_cnt[i] = 0u;
     if (tid == 0) {
         mbar_init(&bars->s_full, 1);
         mbar_init(&bars->p_ready, 4);
@@ -817,8 +820,8 @@ __global__ void __launch_bounds__(kThreads, 4) fwd_kernel(const __grid_constant_
 
 }  // namespace smallk
 
-cudaError_t launch_small_bwd(const Geo& g, const BwdPtrs& p, float* part, unsigned int* status,
-                             unsigned long long limit_ns, int num_sms, cudaStream_t stream) {
+cudaError_t launch_small_bwd(const Geo& g, const BwdPtrs& p, float* part, unsigned int* dtheta_cnt,
+                             unsigned int* status, unsigned long long limit_ns, int num_sms, cudaStream_t stream) {
     using namespace smallk;
     static bool attr_set = false;
     if (!attr_set) {
@@ -840,6 +843,7 @@ cudaError_t launch_small_bwd(const Geo& g, const BwdPtrs& p, float* part, unsign
     sp.lse = p.lse;
     sp.theta = p.theta;
     sp.part = part;
+    sp.dtheta_cnt = dtheta_cnt;
     sp.status = status;
     sp.limit_ns = limit_ns;
     sp.items = static_cast<long long>(g.heads) * g.tiles;
