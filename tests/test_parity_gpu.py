@@ -98,9 +98,12 @@ def test_padded_grid_parity(cfg):
 
 
 @pytest.mark.gpu
-def test_sharp_softmax_parity():
-    """Q, K scaled by 3 (the high-resolution stress recipe) sharpen the softmax."""
-    got, ref = run_both(1, 64, 64, 1, 32, 16, qk_scale=3.0)
+@pytest.mark.parametrize("cfg", [(1, 64, 64, 1, 32, 16), (2, 16, 16, 3, 8, 4), (1, 8, 12, 2, 4, 0),
+                                 (1, 20, 13, 2, 8, 4), (1, 33, 20, 1, 16, 4)])
+def test_sharp_softmax_parity(cfg):
+    """Q, K scaled by 3 (the high-resolution stress recipe) sharpen the softmax:
+    both kernel families, and padded grids."""
+    got, ref = run_both(*cfg, qk_scale=3.0)
     check("o", got["o"], ref["o"], FWD_TOL)
     check("lse", got["lse"], ref["lse"], FWD_TOL)
     for key in ("dq", "dk", "dv", "dtheta"):

@@ -35,7 +35,7 @@ def test_oversized_problem_is_rejected_without_launch():
 
 
 @pytest.mark.gpu
-@pytest.mark.parametrize("cfg", [(2, 32, 32, 2, 16, 8), (1, 16, 16, 2, 8, 4)])
+@pytest.mark.parametrize("cfg", [(2, 32, 32, 2, 16, 8), (1, 16, 16, 2, 8, 4), (1, 20, 13, 2, 8, 4), (1, 33, 20, 1, 16, 4)])
 def test_noalloc_matches_workspace_entry_point_twice(cfg):
     B, H, W, h, M, s = cfg
     inp = make_inputs(B, H, W, h, 32)
