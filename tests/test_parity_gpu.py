@@ -180,3 +180,32 @@ def test_side_stream_gives_the_default_stream_results():
     assert torch.equal(o0, o1) and torch.equal(l0, l1)
     for x, y in zip(g0, g1):
         assert torch.equal(x, y)
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("cfg", [(2, 16, 16, 3, 8, 4), (1, 64, 64, 2, 32, 16)])
+def test_backward_ignores_stale_workspace_contents(cfg):
+    """The caller's workspace may hold anything: a zeroed one, one with every
+    byte 0xFF, and that one again as the previous call left it give the same
+    gradients.  (The d theta reduction's per-head counters live there and are
+    reset by the kernel that runs before it.)  dk, dv are bit-identical; dθ too
+    at M = 8, and at M >= 16 within the last bits its query-side terms take from
+    the unordered dQ' reduce-add."""
+    B, H, W, h, M, s = cfg
+    inp = make_inputs(B, H, W, h, 32)
+    dev = {k: v.cuda() for k, v in inp.items()}
+    o, lse = ops.winattn_fwd(dev["q"], dev["k"], dev["v"], dev["theta"], M, s)
+
+    def bwd(ws):
+        r = ops.winattn_bwd(dev["q"], dev["k"], dev["v"], o, dev["dout"], lse, dev["theta"], M, s, workspace=ws)
+        torch.cuda.synchronize()
+        return [t.clone() for t in r]
+
+    ref = bwd(ops.alloc_workspace(dev["q"], M, s).fill_(0))
+    ws = ops.alloc_workspace(dev["q"], M, s).fill_(0xFF)
+    for got in (bwd(ws), bwd(ws)):
+        assert torch.equal(got[1], ref[1]) and torch.equal(got[2], ref[2])  # dk, dv
+        if M * M < 128:
+            assert torch.equal(got[3], ref[3])
+        else:
+            assert torch.allclose(got[3], ref[3], rtol=1e-5, atol=1e-5)
