@@ -35,6 +35,10 @@
  * allocates device memory and never synchronises; all work is enqueued on the
  * given stream (a cudaStream_t; NULL is the legacy default stream).
  *
+ * Per-device state (the device status word's address, the kernels' shared-memory
+ * opt-in) is set up on the first call on each device and kept for the life of the
+ * process, so the library must not be used on a device after cudaDeviceReset.
+ *
  * Errors: invalid arguments return a status and launch nothing.  A kernel whose
  * internal wait runs past its time limit stops and records FS_ERR_TIMEOUT in a
  * device status word that fs_device_status() reads (after the stream is
@@ -169,6 +173,9 @@ FS_API fs_status fs_selftest_bounded_wait(uint64_t limit_ns, fs_stream_t stream)
  * device); make that first call before any stream capture.  All calls on a
  * device share the array: calls whose kernels may overlap on the GPU (other
  * streams or host threads without ordering between them) race on it.
+ * The address is kept for the life of the process: do not use this entry point
+ * (or any other of this library, whose device status word is looked up the same
+ * way) on a device after cudaDeviceReset.
  */
 FS_API fs_status fs_winattn_bwd_noalloc(const fs_winattn_shape* shape, const void* q, const void* k, const void* v,
                                         const void* o, const void* dout, const float* lse, const float* theta,

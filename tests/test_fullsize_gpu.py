@@ -21,12 +21,18 @@ from vision_transformer_windowed_b200.inputs import make_inputs
 FWD_TOL = (1e-2, 2e-3)
 GRAD_TOL = (3e-2, 5e-3)
 
-# (name, B, H, W, heads, M, s, qk_scale): the benchmark workloads and the
-# FlashSwin-T stage shapes at 256 x 256 input with patch 2
+# (name, B, H, W, heads, M, s, qk_scale[, dout_scale]): the benchmark workloads
+# and the FlashSwin-T stage shapes at 256 x 256 input with patch 2; with a
+# dout_scale (a power of two) the GPU gets dO times it, and its gradients,
+# divided by it, are compared with the oracle's at scale 1 (upstream gradients
+# at the magnitudes of bf16 training, judged at their unit scale)
 FULL = [
     ("swin_t_stage1_p4_m8_s0", 128, 64, 64, 3, 8, 0, 1.0),
     ("swin_t_stage1_p4_m8_s4", 128, 64, 64, 3, 8, 4, 1.0),
+    ("swin_t_stage1_p4_m8_s4_dout2^-20", 128, 64, 64, 3, 8, 4, 1.0, 2.0 ** -20),
+    ("flashswin_t_stage1_p2_m32_s0", 128, 128, 128, 3, 32, 0, 1.0),
     ("flashswin_t_stage1_p2_m32", 128, 128, 128, 3, 32, 16, 1.0),
+    ("flashswin_t_stage1_p2_m32_dout2^-20", 128, 128, 128, 3, 32, 16, 1.0, 2.0 ** -20),
     ("flashswin_t_stage2_p2_m32_s0", 128, 64, 64, 6, 32, 0, 1.0),
     ("flashswin_t_stage2_p2_m32_s16", 128, 64, 64, 6, 32, 16, 1.0),
     ("flashswin_t_stage3_p2_m32_s0", 128, 32, 32, 12, 32, 0, 1.0),
@@ -67,7 +73,8 @@ def _sample_units(B, H, W, heads, M, n_random=6, seed=7):
 @pytest.mark.gpu
 @pytest.mark.parametrize("cfg", FULL, ids=[c[0] for c in FULL])
 def test_full_size_sampled_windows(cfg):
-    name, B, H, W, heads, M, s, qk = cfg
+    name, B, H, W, heads, M, s, qk = cfg[:8]
+    dscale = cfg[8] if len(cfg) > 8 else 1.0
     inp = make_inputs(B, H, W, heads, 32, qk_scale=qk)
     units = _sample_units(B, H, W, heads, M)
     pos = []
@@ -83,8 +90,10 @@ def test_full_size_sampled_windows(cfg):
 
     dev = {k: v.cuda() for k, v in inp.items() if k != "dout"}
     o, lse = ops.winattn_fwd(dev["q"], dev["k"], dev["v"], dev["theta"], M, s)
-    dq, dk, dv, dth = ops.winattn_bwd(dev["q"], dev["k"], dev["v"], o, dout.cuda(), lse, dev["theta"], M, s)
+    dq, dk, dv, dth = ops.winattn_bwd(dev["q"], dev["k"], dev["v"], o, dout.cuda() * dscale, lse, dev["theta"], M, s)
     torch.cuda.synchronize()
+    if dscale != 1.0:
+        dq, dk, dv, dth = (t.double() / dscale for t in (dq, dk, dv, dth))
 
     ref = oracle.units(inp["q"], inp["k"], inp["v"], inp["theta"], M, s, units, dout=dout)
     idx = lambda t, b, rows, cols, h: t[b, torch.from_numpy(rows), torch.from_numpy(cols), h]

@@ -36,12 +36,20 @@ def _device_status_clean():
     assert _lib.fs_device_status() == 0
 
 
-def run_both(B, H, W, h, M, s, qk_scale=1.0):
+def run_both(B, H, W, h, M, s, qk_scale=1.0, dout_scale=1.0):
+    """The CUDA path and the oracle on the same seeded inputs.  With dout_scale
+    (a power of two) the CUDA path gets dO * dout_scale, its gradients are
+    divided by dout_scale (both exact in binary floating point), and the oracle
+    runs at scale 1: the comparison is then judged at the gradients' unit scale,
+    so the absolute term of the tolerance cannot hide an underflow."""
     inp = make_inputs(B, H, W, h, 32, qk_scale=qk_scale)
     dev = {k: v.cuda() for k, v in inp.items()}
     o, lse = ops.winattn_fwd(dev["q"], dev["k"], dev["v"], dev["theta"], M, s)
-    dq, dk, dv, dth = ops.winattn_bwd(dev["q"], dev["k"], dev["v"], o, dev["dout"], lse, dev["theta"], M, s)
+    dout = dev["dout"] * dout_scale if dout_scale != 1.0 else dev["dout"]
+    dq, dk, dv, dth = ops.winattn_bwd(dev["q"], dev["k"], dev["v"], o, dout, lse, dev["theta"], M, s)
     torch.cuda.synchronize()
+    if dout_scale != 1.0:
+        dq, dk, dv, dth = (t.double() / dout_scale for t in (dq, dk, dv, dth))
     ref = oracle.full(inp["q"], inp["k"], inp["v"], inp["theta"], M, s, dout=inp["dout"])
     return {"o": o, "lse": lse, "dq": dq, "dk": dk, "dv": dv, "dtheta": dth}, ref
 
@@ -108,6 +116,79 @@ def test_sharp_softmax_parity(cfg):
     check("lse", got["lse"], ref["lse"], FWD_TOL)
     for key in ("dq", "dk", "dv", "dtheta"):
         check(key, got[key], ref[key], GRAD_TOL)
+
+
+# Upstream gradients at the magnitudes of bf16 training (no loss scaling), and
+# large ones: both kernel families, shifted, padded, and a sharpened softmax.
+# dS = P o (dP - D) is held in fp16 for the dQ' and dK' products; unscaled, the
+# small ones would land in fp16's subnormals or flush to zero, the large ones
+# overflow.
+GRAD_MAGNITUDE = [  # (B, H, W, heads, M, s, qk_scale)
+    (2, 16, 16, 3, 8, 4, 1.0),
+    (1, 8, 12, 2, 4, 0, 1.0),
+    (1, 20, 13, 2, 8, 4, 1.0),    # padded
+    (1, 32, 48, 1, 16, 4, 1.0),
+    (1, 64, 64, 1, 32, 16, 1.0),
+    (1, 70, 50, 1, 32, 16, 1.0),  # padded, several tiles per window
+    (1, 64, 64, 1, 64, 32, 1.0),
+    (2, 16, 16, 3, 8, 4, 3.0),    # sharpened softmax: P near 1
+    (1, 64, 64, 1, 32, 16, 3.0),
+]
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("dout_scale", [2.0 ** -20, 2.0 ** -8, 2.0 ** 12], ids=["2^-20", "2^-8", "2^12"])
+@pytest.mark.parametrize("cfg", GRAD_MAGNITUDE)
+def test_gradient_magnitude_parity(cfg, dout_scale):
+    *shape, qk = cfg
+    got, ref = run_both(*shape, qk_scale=qk, dout_scale=dout_scale)
+    for key in ("dq", "dk", "dv", "dtheta"):
+        check(key, got[key], ref[key], GRAD_TOL)
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("cfg", [(2, 16, 16, 3, 8, 4), (1, 64, 64, 1, 32, 16), (1, 64, 64, 1, 64, 32)])
+def test_gradient_scale_with_uneven_v(cfg):
+    """v rows 2^24 apart in magnitude inside a window (the top half of the grid
+    scaled down), with dO at 2^-20: the scaling of dS must bound dP - D by the
+    largest v row that any output row mixes, not by the key rows of a tile."""
+    B, H, W, h, M, s = cfg
+    inp = make_inputs(B, H, W, h, 32)
+    rows = torch.arange(H).view(1, H, 1, 1, 1)
+    inp["v"] = torch.where(rows < H // 2, inp["v"] * 2.0 ** -24, inp["v"])
+    dev = {k: v.cuda() for k, v in inp.items()}
+    o, lse = ops.winattn_fwd(dev["q"], dev["k"], dev["v"], dev["theta"], M, s)
+    scale = 2.0 ** -20
+    got = ops.winattn_bwd(dev["q"], dev["k"], dev["v"], o, dev["dout"] * scale, lse, dev["theta"], M, s)
+    torch.cuda.synchronize()
+    ref = oracle.full(inp["q"], inp["k"], inp["v"], inp["theta"], M, s, dout=inp["dout"])
+    for key, t in zip(("dq", "dk", "dv", "dtheta"), got):
+        check(key, t.double() / scale, ref[key], GRAD_TOL)
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("cfg", [(1, 16, 16, 2, 8, 4), (1, 64, 64, 1, 32, 16), (1, 20, 13, 2, 8, 4),
+                                 (1, 64, 64, 1, 64, 32)])
+def test_large_qk_forward_parity(cfg):
+    """q, k elements in the thousands (N(0, 1) draws times 1000; the rotated
+    operands stay inside fp16's range, |q'|, |k'| < 65504), logits of order 1e6.
+    With k = q every query's own key leads all others by about 1e6 in the logit,
+    far above the ~1e3 that the fp16 rounding of q', k' moves a logit of that
+    size, so the near one-hot softmax picks the same key on both sides.  (With
+    independent q and k, rows whose two best logits lie within that rounding of
+    each other may pick different keys in any bf16/fp16 attention: such a row is
+    ill-conditioned, not computed wrongly.)"""
+    B, H, W, h, M, s = cfg
+    inp = make_inputs(B, H, W, h, 32, with_dout=False)
+    inp["q"] = (inp["q"].float() * 1000.0).to(torch.bfloat16)
+    inp["k"] = inp["q"].clone()
+    dev = {k: v.cuda() for k, v in inp.items()}
+    o, lse = ops.winattn_fwd(dev["q"], dev["k"], dev["v"], dev["theta"], M, s)
+    torch.cuda.synchronize()
+    ref = oracle.full(inp["q"], inp["k"], inp["v"], inp["theta"], M, s)
+    assert float(inp["q"].float().abs().max()) > 1000.0 and float(ref["lse"].max()) > 1e6
+    check("o", o, ref["o"], FWD_TOL)
+    check("lse", lse, ref["lse"], FWD_TOL)
 
 
 @pytest.mark.gpu

@@ -109,6 +109,12 @@ __global__ void zero_f32_kernel(float* p, int n) {
 
 }  // namespace
 
+int fswin::device_ready() {
+    unsigned int* status = nullptr;
+    int sms = 0;
+    return static_cast<int>(device_state(&status, &sms));
+}
+
 extern "C" {
 
 fs_status fs_winattn_check_shape(const fs_winattn_shape* shape) {

@@ -471,12 +471,8 @@ __global__ void __launch_bounds__(kThreads, 1) block_kernel(const __grid_constan
 cudaError_t launch_block_fwd(const Geo& g, const BlockPtrs& p, unsigned int* status, unsigned long long limit_ns,
                              int num_sms, cudaStream_t stream) {
     using namespace blockk;
-    static bool attr_set = false;
-    if (!attr_set) {
-        const cudaError_t e = cudaFuncSetAttribute(block_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
-        if (e != cudaSuccess) return e;
-        attr_set = true;
-    }
+    static SmemOptIn optin;
+    if (cudaError_t e = optin.ensure(reinterpret_cast<const void*>(block_kernel), kSmemBytes)) return e;
     Params prm;
     prm.g = g;
     prm.x = static_cast<const uint8_t*>(p.x);

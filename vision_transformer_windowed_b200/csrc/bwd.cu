@@ -1,10 +1,13 @@
 // Backward of fused shifted-window attention with window-local 2D RoPE.
 //
 // Recompute-based (the probabilities are rebuilt from the forward's
-// log-sum-exp, never stored), in four launches on the caller's stream:
+// log-sum-exp, never stored), in five launches on the caller's stream:
 //   1. prep:   per token row, rotate q and k (RoPE) into swizzled fp16 tile
 //              images, D = rowsum(dO * O), lse in log2 units, and zero the
-//              fp32 dQ accumulator;
+//              fp32 dQ accumulator; per tile, the largest |dO row| and |v row|;
+//      scale:  per window, the gradient scaling 2^e from those maxima (see
+//              grad_scale_exp in rows.cuh): lse2 -= e, so that the main kernel's
+//              probabilities, dS and dV carry 2^e;
 //   2. main:   persistent, warp-specialised tcgen05 kernel; a work item is one
 //              128-key tile, iterating over the query tiles it attends to:
 //                S^T = K' Q'^T, dP^T = V dO^T            (TMEM)
@@ -12,7 +15,7 @@
 //                dV += P^T dO, dK' += dS^T Q'            (TMEM accumulators)
 //                dQ' = dS K'  -> bulk reduce-add into the fp32 accumulator
 //              and, per item, dk (dK' un-rotated) and dv, with the key side
-//              of d theta;
+//              of d theta (2^-e undoes the scaling of dQ', dK', dV);
 //   3. post:   per token row, undo the rotation of dQ', write dq, and the
 //              query side of d theta;
 //   4. reduce: fixed-order sum of the partials into dtheta (it adds no
@@ -35,7 +38,7 @@ namespace bwdk {
 
 // ------------------------------------------------------------------ workspace
 struct WsLayout {
-    size_t qimg, kimg, lse2, dvec, dqacc, part, part2, cnt, total;
+    size_t qimg, kimg, lse2, dvec, dqacc, nrm, wexp, part, part2, cnt, total;
 };
 
 __host__ __device__ inline size_t round256(size_t x) { return (x + 255) & ~size_t(255); }
@@ -49,6 +52,8 @@ __host__ __device__ inline WsLayout ws_layout(const Geo& g) {
     L.lse2 = o;  o += round256(ht * kTile * 4);
     L.dvec = o;  o += round256(ht * kTile * 4);
     L.dqacc = o; o += round256(ht * kTile * kHeadDim * 4);
+    L.nrm = o;   o += round256(ht * 8);  // per (head, tile): max |dO row|^2, max |v row|^2
+    L.wexp = o;  o += round256(ht * 4);  // per (head, tile): e of the tile's window
     L.part = o;  o += round256(ht * 8 * 16 * 4);  // up to 8 x 16 partials per (head, tile)
     L.part2 = o; o += round256(static_cast<size_t>(g.heads) * 64 * 16 * 4);  // level-1 d theta sums
     L.cnt = o;   o += round256(static_cast<size_t>(g.heads) * 4);            // level-1 blocks done, per head
@@ -58,14 +63,14 @@ __host__ __device__ inline WsLayout ws_layout(const Geo& g) {
 
 struct PrepParams {
     Geo g;
-    const uint4 *q, *k, *o, *dout;
+    const uint4 *q, *k, *v, *o, *dout;
     const float *lse, *theta;
     uint8_t* ws;
     WsLayout L;
 };
 
 struct PostParams {
-    Geo g;
+    Geo g;  // windows of >= 128 tokens
     const uint4* q;
     const float* theta;
     uint4* dq;
@@ -118,6 +123,7 @@ __device__ __forceinline__ void load_row_bf16(const uint4* src, float (&x)[32]) 
 // ------------------------------------------------------------------ 1. prep
 __global__ void __launch_bounds__(128) prep_kernel(const PrepParams p) {
     __shared__ float2 tab[2 * 64 * 8];
+    __shared__ float2 nrm_w[4];
     const Geo& g = p.g;
     // blocks take the heads of a tile in turn (a token's heads share memory
     // lines); ht indexes the workspace images, [head][tile]
@@ -131,17 +137,27 @@ __global__ void __launch_bounds__(128) prep_kernel(const PrepParams p) {
     const int r = threadIdx.x;
     const Slot sl = slot_of(g, T, r);
     float q[32], k[32], dO[32], o[32];
-    float D = 0.f, lse2 = INFINITY;
+    float D = 0.f, lse2 = INFINITY, ndo = 0.f, nv = 0.f;
     if (sl.valid) {
         const long long tok = ((static_cast<long long>(sl.box.b) * g.H + sl.row) * g.W + sl.col) * g.heads + h;
         load_row_bf16(p.q + tok * 4, q);
         load_row_bf16(p.k + tok * 4, k);
         load_row_bf16(p.dout + tok * 4, dO);
         load_row_bf16(p.o + tok * 4, o);
-        float acc[4] = {0.f, 0.f, 0.f, 0.f};
+        float acc[4] = {0.f, 0.f, 0.f, 0.f}, n4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-        for (int e = 0; e < 32; ++e) acc[e & 3] = fmaf(dO[e], o[e], acc[e & 3]);
+        for (int e = 0; e < 32; ++e) {
+            acc[e & 3] = fmaf(dO[e], o[e], acc[e & 3]);
+            n4[e & 3] = fmaf(dO[e], dO[e], n4[e & 3]);
+        }
         D = (acc[0] + acc[1]) + (acc[2] + acc[3]);
+        ndo = (n4[0] + n4[1]) + (n4[2] + n4[3]);
+        load_row_bf16(p.v + tok * 4, o);  // o is done with: v's row
+#pragma unroll
+        for (int e = 0; e < 4; ++e) n4[e] = 0.f;
+#pragma unroll
+        for (int e = 0; e < 32; ++e) n4[e & 3] = fmaf(o[e], o[e], n4[e & 3]);
+        nv = (n4[0] + n4[1]) + (n4[2] + n4[3]);
         lse2 = p.lse[tok] * 1.4426950408889634f;
         rope32(q, sl.i, sl.j, tab, false);
         rope32(k, sl.i, sl.j, tab, false);
@@ -156,6 +172,43 @@ __global__ void __launch_bounds__(128) prep_kernel(const PrepParams p) {
     uint4* acc = reinterpret_cast<uint4*>(p.ws + p.L.dqacc + (ht * kTile + r) * kHeadDim * 4);
 #pragma unroll
     for (int c = 0; c < 8; ++c) acc[c] = make_uint4(0, 0, 0, 0);
+    // the tile's largest squared norms of dO and v rows
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        ndo = fmaxf(ndo, __shfl_xor_sync(0xFFFFFFFFu, ndo, o));
+        nv = fmaxf(nv, __shfl_xor_sync(0xFFFFFFFFu, nv, o));
+    }
+    if ((r & 31) == 0) nrm_w[r >> 5] = make_float2(ndo, nv);
+    __syncthreads();
+    if (r == 0)
+        reinterpret_cast<float2*>(p.ws + p.L.nrm)[ht] =
+            make_float2(fmaxf(fmaxf(nrm_w[0].x, nrm_w[1].x), fmaxf(nrm_w[2].x, nrm_w[3].x)),
+                        fmaxf(fmaxf(nrm_w[0].y, nrm_w[1].y), fmaxf(nrm_w[2].y, nrm_w[3].y)));
+}
+
+// ------------------------------------------------------------------ 1b. scale
+// One block per (head, window) of >= 128 tokens: the gradient scaling exponent
+// e of the window from its tiles' largest |dO row|^2 and |v row|^2 (every row
+// of the window: a key tile's products reach all of the window's queries, and
+// D_t = dO_t . O_t mixes all of its v rows), lse2 -= e for the window's rows,
+// and e kept for each of its tiles (per tile, so that the workspace does not
+// depend on the window size).
+__global__ void __launch_bounds__(128) scale_kernel(const Geo g, uint8_t* ws, const WsLayout L) {
+    const long long hw = blockIdx.x;  // head-major: h * wins + window
+    const int h = static_cast<int>(hw / g.wins);
+    const long long w = hw - static_cast<long long>(h) * g.wins;
+    const size_t t0 = static_cast<size_t>(h) * g.tiles + static_cast<size_t>(w) * g.tpw;
+    const float2* nrm = reinterpret_cast<const float2*>(ws + L.nrm) + t0;
+    float a = 0.f, b = 0.f;
+    for (int i = 0; i < g.tpw; ++i) {
+        const float2 t = nrm[i];
+        a = fmaxf(a, t.x);
+        b = fmaxf(b, t.y);
+    }
+    const int e = grad_scale_exp(a, b);
+    float* lse2 = reinterpret_cast<float*>(ws + L.lse2) + t0 * kTile;
+    for (int i = threadIdx.x; i < g.tpw * kTile; i += blockDim.x) lse2[i] -= static_cast<float>(e);
+    for (int i = threadIdx.x; i < g.tpw; i += blockDim.x) reinterpret_cast<int*>(ws + L.wexp)[t0 + i] = e;
 }
 
 // ------------------------------------------------------------------ 2. main
@@ -559,6 +612,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         bool ok = true;
         for (long long item = blockIdx.x; item < prm.items && ok; item += gridDim.x, ++it) {
             const Item I = item_of(g, item);
+            // dQ' goes to the accumulator with its 2^e (the post kernel undoes it);
+            // dK' and dV get 2^-e at the end of the item
+
             for (int n = 0; n < I.nq; ++n) {
                 if (!q_active(g, I, n)) continue;
                 const uint32_t c = static_cast<uint32_t>(j & 1);  // the step's dQ' accumulator
@@ -571,15 +627,16 @@ __global__ void __launch_bounds__(kThreads, 1)
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&bars->dq_free[c]);
                 float* buf = dqst + (j & 1) * kTile * kHeadDim;
+                const float sc = prm.scale;
                 if (leader) bulk_wait_read_but1();
                 named_bar_sync(1, 128);
                 // fp32 tile image, chunk c of row r at chunk position c ^ (r & 7)
                 float4* rowp = reinterpret_cast<float4*>(buf + r * kHeadDim);
 #pragma unroll
                 for (int c = 0; c < 8; ++c) {
-                    rowp[c ^ (r & 7)] = make_float4(__uint_as_float(v[4 * c]) * prm.scale, __uint_as_float(v[4 * c + 1]) * prm.scale,
-                                          __uint_as_float(v[4 * c + 2]) * prm.scale,
-                                          __uint_as_float(v[4 * c + 3]) * prm.scale);
+                    rowp[c ^ (r & 7)] = make_float4(__uint_as_float(v[4 * c]) * sc, __uint_as_float(v[4 * c + 1]) * sc,
+                                                    __uint_as_float(v[4 * c + 2]) * sc,
+                                                    __uint_as_float(v[4 * c + 3]) * sc);
                 }
                 fence_proxy_async_smem();
                 named_bar_sync(1, 128);
@@ -594,12 +651,16 @@ __global__ void __launch_bounds__(kThreads, 1)
             // item end: dV and dK' accumulators.  dk is un-rotated here, and the
             // key side of d theta taken with the item's rotated k' rows, which stay
             // in its K', V slot until every row has read them.
+            // the window's gradient scaling 2^e undone
+            const float down = exp2i(-__ldcg(reinterpret_cast<const int*>(prm.ws + prm.L.wexp) +
+                                             static_cast<long long>(I.h) * g.tiles + I.u));
             if (!mbar_wait(&bars->dkv_full, dkvph, ctl, 0x1502)) break;
             dkvph ^= 1;
             tc_fence_after();
             uint32_t dvp[16];  // dv, bf16 pairs
             float dk[32];
             {
+                const float sc = prm.scale * down;
                 uint32_t vv[32], kk[32];
                 tmem_ld32(tmem + lane_off + kColDV, vv);
                 tmem_ld32(tmem + lane_off + kColDK, kk);
@@ -608,10 +669,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&bars->dkv_free);
 #pragma unroll
-                for (int e = 0; e < 16; ++e) dvp[e] = pack_bf16x2(__uint_as_float(vv[2 * e]), __uint_as_float(vv[2 * e + 1]));
+                for (int e = 0; e < 16; ++e)
+                    dvp[e] = pack_bf16x2(__uint_as_float(vv[2 * e]) * down, __uint_as_float(vv[2 * e + 1]) * down);
 #pragma unroll
                 for (int e = 0; e < 32; e += 2)
-                    fmul2(dk[e], dk[e + 1], __uint_as_float(kk[e]), __uint_as_float(kk[e + 1]), prm.scale, prm.scale);
+                    fmul2(dk[e], dk[e + 1], __uint_as_float(kk[e]), __uint_as_float(kk[e + 1]), sc, sc);
             }
             const int ks = it & 1;
             if (!mbar_wait(&bars->kv_full[ks], (it >> 1) & 1, ctl, 0x1503)) break;
@@ -700,10 +762,12 @@ __global__ void __launch_bounds__(128) post_kernel(const PostParams p) {
         const long long tok = ((static_cast<long long>(sl.box.b) * g.H + sl.row) * g.W + sl.col) * g.heads + h;
         float dq[32], q[32];
         const float4* aq = reinterpret_cast<const float4*>(p.ws + p.L.dqacc + (ht * kTile + r) * kHeadDim * 4);
+        // the window's gradient scaling 2^e, still in the accumulated dQ'
+        const float down = exp2i(-reinterpret_cast<const int*>(p.ws + p.L.wexp)[ht]);
 #pragma unroll
         for (int c = 0; c < 8; ++c) {
             const float4 a = aq[c ^ (r & 7)];  // swizzled fp32 tile image
-            dq[4 * c] = a.x; dq[4 * c + 1] = a.y; dq[4 * c + 2] = a.z; dq[4 * c + 3] = a.w;
+            dq[4 * c] = a.x * down; dq[4 * c + 1] = a.y * down; dq[4 * c + 2] = a.z * down; dq[4 * c + 3] = a.w * down;
         }
         rope32(dq, sl.i, sl.j, tab, true);
         load_row_bf16(p.q + tok * 4, q);
@@ -811,16 +875,22 @@ cudaError_t launch_bwd(const Geo& g, const BwdPtrs& p, const BwdMaps& maps, unsi
         mark(4);
         return e;
     }
-    static bool attr_set = false;
-    if (!attr_set) {
-        e = cudaFuncSetAttribute(main_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
-        if (e != cudaSuccess) return e;
-        attr_set = true;
-    }
+    static SmemOptIn optin;
+    if ((e = optin.ensure(reinterpret_cast<const void*>(main_kernel), kSmemBytes)) != cudaSuccess) return e;
     mark(0);
-    PrepParams pp{g, static_cast<const uint4*>(p.q), static_cast<const uint4*>(p.k), static_cast<const uint4*>(p.o),
-                  static_cast<const uint4*>(p.dout), p.lse, p.theta, p.ws, L};
+    PrepParams pp{g,
+                  static_cast<const uint4*>(p.q),
+                  static_cast<const uint4*>(p.k),
+                  static_cast<const uint4*>(p.v),
+                  static_cast<const uint4*>(p.o),
+                  static_cast<const uint4*>(p.dout),
+                  p.lse,
+                  p.theta,
+                  p.ws,
+                  L};
     prep_kernel<<<static_cast<unsigned>(ht), 128, 0, stream>>>(pp);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    scale_kernel<<<static_cast<unsigned>(g.heads * g.wins), 128, 0, stream>>>(g, p.ws, L);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     mark(1);
 

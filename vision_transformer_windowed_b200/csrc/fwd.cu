@@ -527,13 +527,9 @@ cudaError_t launch_fwd(const Geo& g, const CUtensorMap& mq, const CUtensorMap& m
         if (e == cudaSuccess && events) e = cudaEventRecord(events[1], stream);
         return e;
     }
-    static bool attr_set = false;
-    if (!attr_set) {
-        cudaError_t e = cudaFuncSetAttribute(fwdk::fwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             fwdk::kSmemBytes);
-        if (e != cudaSuccess) return e;
-        attr_set = true;
-    }
+    static SmemOptIn optin;
+    if (cudaError_t e = optin.ensure(reinterpret_cast<const void*>(fwdk::fwd_kernel), fwdk::kSmemBytes))
+        return e;
     const long long pairs = (prm.items + 1) / 2;  // each CTA runs two workers
     const long long grid = pairs < num_sms ? pairs : num_sms;
     if (events) {

@@ -6,10 +6,42 @@
 
 #include <cstddef>
 #include <cstdint>
+#include <mutex>
 
 #include "geometry.cuh"
 
 namespace fswin {
+
+// Opts a kernel into more than the default 48 KB of dynamic shared memory.  The
+// attribute is per device, so it is set once for every device the kernel is
+// launched on (the first launch there, with that device current), under a lock
+// because several host threads may launch at once.
+class SmemOptIn {
+   public:
+    cudaError_t ensure(const void* func, int bytes) {
+        int dev = 0;
+        cudaError_t e = cudaGetDevice(&dev);
+        if (e != cudaSuccess) return e;
+        if (dev < 0 || dev >= kDevices)
+            return cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+        std::lock_guard<std::mutex> lk(mu_);
+        if (!done_[dev]) {
+            e = cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+            if (e != cudaSuccess) return e;
+            done_[dev] = true;
+        }
+        return cudaSuccess;
+    }
+
+   private:
+    static constexpr int kDevices = 64;
+    std::mutex mu_;
+    bool done_[kDevices] = {};
+};
+
+// Checks that the current device can run the kernels (sm_100) and sets up the
+// library's per-device state; returns an fs_status code (0 when usable).
+int device_ready();
 
 long long fwd_items(const Geo& g);
 cudaError_t launch_fwd(const Geo& g, const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,

@@ -60,6 +60,9 @@ fs_status fs_winattn_bwd_noalloc(const fs_winattn_shape* shape, const void* q, c
     fs_status st = fs_winattn_check_shape(shape);
     if (st != FS_OK) return st;
     if (fs_winattn_bwd_workspace_bytes(shape) > kNoAllocScratchBytes) return FS_ERR_WORKSPACE;
+    // the device check first: on another architecture the symbol lookup below
+    // would fail with a CUDA error instead of FS_ERR_ARCH
+    if ((st = static_cast<fs_status>(fswin::device_ready())) != FS_OK) return st;
     void* scratch = nullptr;
     if ((st = scratch_address(&scratch)) != FS_OK) return st;
     return fs_winattn_bwd(shape, q, k, v, o, dout, lse, theta, dq, dk, dv, dtheta, scratch, kNoAllocScratchBytes,

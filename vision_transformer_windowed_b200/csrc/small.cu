@@ -80,6 +80,7 @@ constexpr uint32_t kColDV = 64, kColDQ = 96, kColDK = 192;
 struct Bars {
     uint64_t s_full, p_ready, mma2_done, grp, done;
     uint64_t slot_full[2], o_full, o_free, staged;  // row copies and stores (mover warp)
+    float2 nrm[2][4];  // per item parity, per row warp: max |dO row|^2, max |v row|^2 (gradient scaling)
     uint32_t tmem_base;
     int abort_flag;
 };
@@ -316,24 +317,31 @@ __global__ void __launch_bounds__(kThreads, 2) small_kernel(const __grid_constan
             if (!wwait(&bars->slot_full[j & 1], static_cast<uint32_t>((j >> 1) & 1), 0x2304) ||
                 !wwait(&bars->o_full, ph, 0x2305))
                 break;
-            // D = dO . O of this row's token; then the next item's o rows
+            // D = dO . O of this row's token, and the squared norms of its dO and
+            // v rows (the bound of the gradient scaling below); then the next
+            // item's o rows
             float D = 0.f;
             {
                 float a[32], b[32];
                 load_row_swz(smem + kOOff, r, a, false);
                 load_row_swz(sl + 3 * kTileBytes, r, b, false);
                 float d4[4] = {0.f, 0.f, 0.f, 0.f};  // four independent partial sums
+                float n4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
                 for (int e = 0; e < 32; e += 4) {
                     ffma2(d4[0], d4[1], a[e], a[e + 1], b[e], b[e + 1], d4[0], d4[1]);
                     ffma2(d4[2], d4[3], a[e + 2], a[e + 3], b[e + 2], b[e + 3], d4[2], d4[3]);
+                    ffma2(n4[0], n4[1], b[e], b[e + 1], b[e], b[e + 1], n4[0], n4[1]);
+                    ffma2(n4[2], n4[3], b[e + 2], b[e + 3], b[e + 2], b[e + 3], n4[2], n4[3]);
                 }
                 D = (d4[0] + d4[1]) + (d4[2] + d4[3]);
+                const float ndo = warp_max_nonneg((n4[0] + n4[1]) + (n4[2] + n4[3]));
+                const float nv = warp_max_nonneg(row_norm2(sl + 2 * kTileBytes, r));
+                if (lane == 0) bars->nrm[ph][warp] = make_float2(ndo, nv);
             }
             __syncwarp();  // every lane has read its o row: the mover may load the next item's
             if (lane == 0) mbar_arrive(&bars->o_free);
             const RowTok nxt = j + 1 < n ? row_tok(j + 1) : RowTok{};
-            lse2v[r] = cur.valid ? lse_cur * 1.4426950408889634f : INFINITY;  // padding: no probability
             dvec[r] = D;
             // RoPE of this row's q and k, bf16 in, fp16 out, in place
             {
@@ -358,6 +366,13 @@ __global__ void __launch_bounds__(kThreads, 2) small_kernel(const __grid_constan
                     umma_ss(tmem + kColDP, dK0 + vo + 2 * k, dK0 + dof + 2 * k, id_dp, k > 0);
                 umma_commit(&bars->s_full);
             }
+            // the tile's gradient scaling 2^e (GradScale in rows.cuh): lse2 - e makes the
+            // probabilities 2^e P; every row's shifted lse2 is in place after the barrier,
+            // which passes while the tensor core computes S^T and dP^T
+            const int gexp = grad_scale_exp4(bars->nrm[ph]);
+            lse2v[r] = cur.valid ? lse_cur * 1.4426950408889634f - static_cast<float>(gexp)
+                                 : INFINITY;  // padding: no probability
+            if (!group_sync(0x2309)) break;
             const float lse_nxt = (j + 1 < n && nxt.valid) ? __ldg(prm.lse + nxt.tok) : 0.f;
             // row of P^T and dS^T of this key, 32 query columns at a time
             if (!wwait(&bars->s_full, ph, 0x2307)) break;
@@ -445,9 +460,12 @@ __global__ void __launch_bounds__(kThreads, 2) small_kernel(const __grid_constan
                 tmem_ld32(trow + (which ? kColDK : kColDQ), t);
                 tmem_wait_ld();
                 float dx[32], x[32];
+                // softmax scale, and the 2^e scaling undone (the exponent again from the
+                // item's norms, which stay in place until item j + 2)
+                const float sc = prm.scale * exp2i(-grad_scale_exp4(bars->nrm[ph]));
 #pragma unroll
                 for (int e = 0; e < 32; e += 2)
-                    fmul2(dx[e], dx[e + 1], __uint_as_float(t[e]), __uint_as_float(t[e + 1]), prm.scale, prm.scale);
+                    fmul2(dx[e], dx[e + 1], __uint_as_float(t[e]), __uint_as_float(t[e + 1]), sc, sc);
                 uint8_t* tile = sl + which * kTileBytes;
                 load_row_swz(tile, r, x, true);  // rotated q' or k' (fp16)
                 // d theta: the pair's cross product is the same before and after the rotation
@@ -470,8 +488,9 @@ __global__ void __launch_bounds__(kThreads, 2) small_kernel(const __grid_constan
                 tc_fence_before();  // ordered before the next item's MMAs by its group barrier
                 __syncwarp();
                 float x[32];
+                const float down = exp2i(-grad_scale_exp4(bars->nrm[ph]));
 #pragma unroll
-                for (int e = 0; e < 32; ++e) x[e] = __uint_as_float(t[e]);
+                for (int e = 0; e < 32; ++e) x[e] = __uint_as_float(t[e]) * down;
                 store_row_swz(sl + 2 * kTileBytes, r, x);  // dv, staged over v
             }
             __syncwarp();
@@ -823,13 +842,8 @@ __global__ void __launch_bounds__(kThreads, 4) fwd_kernel(const __grid_constant_
 cudaError_t launch_small_bwd(const Geo& g, const BwdPtrs& p, float* part, unsigned int* dtheta_cnt,
                              unsigned int* status, unsigned long long limit_ns, int num_sms, cudaStream_t stream) {
     using namespace smallk;
-    static bool attr_set = false;
-    if (!attr_set) {
-        const cudaError_t e =
-            cudaFuncSetAttribute(bwd::small_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bwd::kSmemBytes);
-        if (e != cudaSuccess) return e;
-        attr_set = true;
-    }
+    static SmemOptIn optin;
+    if (cudaError_t e = optin.ensure(reinterpret_cast<const void*>(bwd::small_kernel), bwd::kSmemBytes)) return e;
     bwd::Params sp;
     sp.g = g;
     sp.q = static_cast<const uint8_t*>(p.q);
@@ -858,13 +872,8 @@ cudaError_t launch_small_fwd(const Geo& g, const void* q, const void* k, const v
                              float* lse, unsigned int* status, unsigned long long limit_ns, int num_sms,
                              cudaStream_t stream) {
     using namespace smallk;
-    static bool attr_set = false;
-    if (!attr_set) {
-        const cudaError_t e =
-            cudaFuncSetAttribute(fwd::fwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, fwd::kSmemBytes);
-        if (e != cudaSuccess) return e;
-        attr_set = true;
-    }
+    static SmemOptIn optin;
+    if (cudaError_t e = optin.ensure(reinterpret_cast<const void*>(fwd::fwd_kernel), fwd::kSmemBytes)) return e;
     fwd::Params fp;
     fp.g = g;
     fp.q = static_cast<const uint8_t*>(q);
