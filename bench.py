@@ -2,10 +2,13 @@
 """Benchmark of fused windowed-RoPE attention (forward + backward) on B200.
 
 One step = one pass of the whole hot path over one batch: forward and
-backward at every shift of the workload (the Swin-T stage-1 shape at p=4,
-M=8 runs an unshifted and a shifted block, s=0 and s=4).  Inputs are seeded
-synthetic bf16 N(0,1) tensors of the workload's shape (the pages measure on
-ImageNet at 256x256; no dataset is used).
+backward of every attention block of the workload.  The headline workload is
+the attention of all four FlashSwin-T stages at 256 x 256 input with patch 2
+(grids 128/64/32/16, heads 3/6/12/24, windows 32/32/32/16, batch 128), one
+unshifted and one shifted block per stage (both unshifted at stage 4, whose
+window is the whole grid).  Inputs are seeded synthetic bf16 N(0,1) tensors
+of the workload's shapes (the pages measure on ImageNet at 256x256; no
+dataset is used).
 
 Prints ONE JSON line (rank 0).  `--impl reference` times the fp64 CPU oracle
 instead, on a bounded sample of the same workload.
@@ -29,6 +32,15 @@ METRIC = "windowed-RoPE attention fwd+bwd TFLOP/s (% BF16 peak), tokens/s, peak 
 HEAD_DIM = 32
 
 WORKLOADS = {
+    # the attention of all four FlashSwin-T stages at 256x256 input, p=2, batch 128: grids 128/64/32/16,
+    # heads 3/6/12/24, windows 32/32/32/16; an unshifted and a shifted (s = M/2) block per stage, both
+    # unshifted at stage 4 (the window clamped to the grid)
+    "flashswin_t_p2_4stage": dict(stages=[
+        dict(B=128, H=128, W=128, heads=3, M=32, shifts=(0, 16)),
+        dict(B=128, H=64, W=64, heads=6, M=32, shifts=(0, 16)),
+        dict(B=128, H=32, W=32, heads=12, M=32, shifts=(0, 16)),
+        dict(B=128, H=16, W=16, heads=24, M=16, shifts=(0, 0)),
+    ], qk_scale=1.0),
     # Swin-T stage-1 shape at p=4 (64x64 grid at 256x256 input), window 8, unshifted and shifted blocks
     "swin_t_stage1_p4_m8": dict(B=128, H=64, W=64, heads=3, M=8, shifts=(0, 4), qk_scale=1.0),
     # FlashSwin-T stage 1 at p=2 (128x128 grid), window 32, shifted block
@@ -46,7 +58,7 @@ WORKLOADS = {
     "swin_t_det_stage1_p4_m8": dict(B=16, H=200, W=334, heads=3, M=8, shifts=(0, 4), qk_scale=1.0),
     "flashswin_t_det_stage1_p4_m32": dict(B=16, H=200, W=334, heads=3, M=32, shifts=(0, 16), qk_scale=1.0),
 }
-HEADLINE = "swin_t_stage1_p4_m8"
+HEADLINE = "flashswin_t_p2_4stage"
 SPEC_BF16_TFLOPS = 2250.0  # NVIDIA's dense bf16 figure for one B200: a spec value, not a measurement
 
 # the window-attention block of a Swin layer with its qkv and output projections (inference),
@@ -122,10 +134,95 @@ def measured_traffic(kernel: str, workload: str):
     return rec["bytes_per_launch"]
 
 
+def stages_of(wl) -> list:
+    """A workload as a list of stages: one grid shape each, with the shifts of its blocks."""
+    if "stages" in wl:
+        return [dict(st, qk_scale=st.get("qk_scale", wl.get("qk_scale", 1.0)), infer=wl.get("infer", False))
+                for st in wl["stages"]]
+    return [wl]
+
+
+def blocks_of(wl) -> list:
+    """(stage, shift) of every attention block of one step, in the order the step runs them."""
+    return [(st, s) for st in stages_of(wl) for s in st["shifts"]]
+
+
 def workload_flops(wl) -> tuple[float, float]:
     """Useful forward and backward FLOPs of one step (fwd 4*d per pair, bwd 10*d per pair)."""
-    pairs = sum(unmasked_pairs(wl["B"], wl["H"], wl["W"], wl["heads"], wl["M"], s) for s in wl["shifts"])
+    pairs = sum(unmasked_pairs(st["B"], st["H"], st["W"], st["heads"], st["M"], s) for st, s in blocks_of(wl))
     return 4.0 * HEAD_DIM * pairs, 10.0 * HEAD_DIM * pairs
+
+
+def workload_tokens(wl) -> int:
+    """Token positions the step's blocks process (B * H * W per block)."""
+    return sum(st["B"] * st["H"] * st["W"] for st, _ in blocks_of(wl))
+
+
+PHASES = ["fwd", "bwd_prep", "bwd_main", "bwd_post", "bwd_dtheta"]
+
+
+def phase_work(st, s) -> dict:
+    """Algorithmic work of one block per kernel phase: flops of its products and the bytes it must
+    move.  Windows inside one tile run the whole backward as one kernel (Q, K, V, O, dO read, dQ, dK,
+    dV written, LSE and D: 520 B per token-head row, recorded as bwd_main); larger windows run prep /
+    main / post with workspace round trips (prep: q, k, v, o, dO, lse in, q', k' images, lse2, D and
+    the zeroed dQ' accumulator out, 588 B, and the per-window scale pass over lse2, 8 B, timed with
+    it; main: the images, dO, v, lse2, D in, dk, dv out, 392 B; post: the dQ' accumulator and q in, dq
+    out, 256 B)."""
+    B, H, W, heads, M = st["B"], st["H"], st["W"], st["heads"], st["M"]
+    rows = B * H * W * heads
+    pairs = unmasked_pairs(B, H, W, heads, M, s)
+    small = M * M < 128
+    nbytes = {"fwd": (256 if st.get("infer") else 260) * rows, "bwd_prep": 0 if small else 596 * rows,
+              "bwd_main": (520 if small else 392) * rows, "bwd_post": 0 if small else 256 * rows,
+              "bwd_dtheta": 0}
+    flops = {"fwd": 4.0 * HEAD_DIM * pairs, "bwd_main": 10.0 * HEAD_DIM * pairs}
+    return {"bytes": nbytes, "flops": flops, "hbm_bound": small}
+
+
+def mufu_ceiling_tflops(flops_per_exp: float, sm_mhz: float, sms: int = 148) -> float:
+    """The ceiling one MUFU exp2 per score element puts on a kernel: 16 exp2 per clock per SM
+    (the CUDA guide's throughput table for compute capability 10.0) times the SM count and clock,
+    times the flops counted per element (4 d forward, 10 d backward)."""
+    return flops_per_exp * 16 * sms * sm_mhz * 1e6 / 1e12
+
+
+def roofline(wl, res, peaks, sm_mhz=None) -> dict:
+    """Roofline of the step's dominant kernel (largest share of the step's kernel time): its
+    algorithmic work over all launches of one step divided by its measured time per step.  Windows
+    inside one tile, and the row passes of the larger-window backward, are bound by HBM (reported in
+    GB/s against the measured copy bandwidth); the larger-window attention kernels by the tensor
+    cores (TFLOP/s against the measured cuBLAS bf16 peak, the sustained figure since the kernel runs
+    inside a long step), with the MUFU ceiling beside it."""
+    blocks = blocks_of(wl)
+    work = [phase_work(st, s) for st, s in blocks]
+    ph = res["phase_ms_per_step"]
+    dom = max(ph, key=lambda n: ph[n])
+    hbm = all(w["hbm_bound"] for w in work) or dom in ("bwd_prep", "bwd_post", "bwd_dtheta")
+    t = ph[dom] * 1e-3
+    if hbm:
+        nb = sum(w["bytes"][dom] for w in work)
+        achieved = nb / t / 1e9
+        roof = {"kernel": dom, "bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": achieved / peaks["hbm_gbs"], "traffic": None,
+                "algorithmic_bytes_per_step": nb, "peak_note": f"HBM copy bandwidth, {peaks['source']}"}
+    else:
+        fl = sum(w["flops"].get(dom, 0.0) for w in work)
+        achieved = fl / t / 1e12
+        peak = peaks["bf16_tflops_sustained"]
+        roof = {"kernel": dom, "bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                "frac": achieved / peak, "frac_of_burst": achieved / peaks["bf16_tflops"], "traffic": None,
+                "algorithmic_flops_per_step": fl,
+                "peak_note": f"cuBLAS bf16 sustained (burst {peaks['bf16_tflops']:.1f}), {peaks['source']}"}
+        per_exp = (4.0 if dom == "fwd" else 10.0) * HEAD_DIM
+        mhz = sm_mhz or 1965.0
+        roof["mufu_ceiling_tflops"] = mufu_ceiling_tflops(per_exp, mhz)
+        roof["mufu_note"] = (f"one MUFU exp2 per score element: 16/clk/SM x 148 SMs x {mhz:.0f} MHz x "
+                             f"{per_exp:.0f} flops per element")
+    roof["launches_per_step"] = len(blocks)
+    roof["avg_launch_ms"] = ph[dom] / len(blocks)
+    roof["ms_per_step"] = ph[dom]
+    return roof
 
 
 def block_flops(wl) -> float:
@@ -198,36 +295,41 @@ class ClockSampler:
 
 def cpu_baseline(tensors, wl, seconds: float = 12.0):
     """Times the fp64 oracle (forward + backward) on host cores over a bounded
-    sample of the workload's (batch, window, head) units at every shift of the
-    step (all of them when they fit in the time budget)."""
+    sample of the workload's (batch, window, head) units in every block of the
+    step (all of them when they fit in the time budget).  `tensors`: one dict of
+    inputs per stage of the workload (a single dict for a one-stage workload)."""
     import numpy as np
 
     import oracle
-    B, H, W, heads, M = wl["B"], wl["H"], wl["W"], wl["heads"], wl["M"]
-    nW = -(-H // M) * -(-W // M)  # windows of the grid padded to multiples of M
-    n_units = B * nW * heads
+    stages = stages_of(wl)
+    if isinstance(tensors, dict):
+        tensors = [tensors]
     cores = oracle.default_threads()
+    nblocks = sum(len(st["shifts"]) for st in stages)
     flops, total_dt, parts, done, full_s = 0.0, 0.0, [], 0, 0.0
-    for s in wl["shifts"]:
-        # units spread over the batch, including windows of the last row/column
-        t0 = time.perf_counter()
-        probe = np.arange(0, min(n_units, 4 * cores))
-        oracle.units(tensors["q"], tensors["k"], tensors["v"], tensors["theta"], M, s, probe, dout=tensors["dout"],
-                     nthreads=cores)
-        dt = max(time.perf_counter() - t0, 1e-6)
-        budget = seconds / len(wl["shifts"])
-        n = int(min(n_units, max(len(probe), len(probe) * budget / dt)))
-        ids = np.linspace(0, n_units - 1, n).astype(np.int64)
-        t0 = time.perf_counter()
-        oracle.units(tensors["q"], tensors["k"], tensors["v"], tensors["theta"], M, s, ids, dout=tensors["dout"],
-                     nthreads=cores)
-        dt = time.perf_counter() - t0
-        # useful flops of the sampled units (pairs that attend)
-        flops += 14.0 * HEAD_DIM * unmasked_pairs(B, H, W, heads, M, s) * (n / n_units)
-        total_dt += dt
-        done += n
-        full_s += dt * n_units / n
-        parts.append(f"{n} of {n_units} at s={s}")
+    for st, t in zip(stages, tensors):
+        B, H, W, heads, M = st["B"], st["H"], st["W"], st["heads"], st["M"]
+        nW = -(-H // M) * -(-W // M)  # windows of the grid padded to multiples of M
+        n_units = B * nW * heads
+        for s in st["shifts"]:
+            # units spread over the batch, including windows of the last row/column
+            t0 = time.perf_counter()
+            probe = np.arange(0, min(n_units, 4 * cores))
+            oracle.units(t["q"], t["k"], t["v"], t["theta"], M, s, probe, dout=t["dout"], nthreads=cores)
+            dt = max(time.perf_counter() - t0, 1e-6)
+            budget = seconds / nblocks
+            n = int(min(n_units, max(len(probe), len(probe) * budget / dt)))
+            ids = np.linspace(0, n_units - 1, n).astype(np.int64)
+            t0 = time.perf_counter()
+            oracle.units(t["q"], t["k"], t["v"], t["theta"], M, s, ids, dout=t["dout"], nthreads=cores)
+            dt = time.perf_counter() - t0
+            # useful flops of the sampled units (pairs that attend)
+            flops += 14.0 * HEAD_DIM * unmasked_pairs(B, H, W, heads, M, s) * (n / n_units)
+            total_dt += dt
+            done += n
+            full_s += dt * n_units / n
+            where = f"{H}x{W}/M={M} " if len(stages) > 1 else ""
+            parts.append(f"{n} of {n_units} at {where}s={s}")
     return {"value": flops / total_dt / 1e12, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
             "sample": f"(batch, window, head) units: {', '.join(parts)}; fwd+bwd, fp64, {total_dt:.1f} s",
             "units_per_s": done / total_dt,
@@ -239,9 +341,8 @@ def config_entry(wl, r, peaks, world) -> dict:
     """Per-workload figures: fwd+bwd and forward-alone throughput, the no-recompute count of
     the backward (8 d per pair instead of 10 d), % of the measured and of the spec bf16 peak,
     the forward's algorithmic HBM rate, peak memory and the backward workspace."""
-    nshift = len(wl["shifts"])
-    fwd_ms = r["phase_ms"]["fwd"] * nshift  # per step
-    rows = wl["B"] * wl["H"] * wl["W"] * wl["heads"]
+    blocks = blocks_of(wl)
+    fwd_ms = r["phase_ms"]["fwd"] * len(blocks)  # per step
     infer = wl.get("infer", False)
     e = {"tflops": r["tflops"], "ms_per_step": r["ms"],
          "pct_bf16_peak": 100 * r["tflops"] / peaks["bf16_tflops"] / world,
@@ -250,12 +351,15 @@ def config_entry(wl, r, peaks, world) -> dict:
          "tokens_per_s": r["tokens_per_s"], "peak_gb": r["peak_gb"], "phase_ms": r["phase_ms"]}
     e["fwd_pct_bf16_peak"] = 100 * e["fwd_tflops"] / peaks["bf16_tflops"] / world
     # q, k, v read and o written (bf16), plus the fp32 lse of a training forward
-    e["fwd_gbs"] = (256 if infer else 260) * rows * nshift / (fwd_ms * 1e-3) / 1e9
+    rows = sum(st["B"] * st["H"] * st["W"] * st["heads"] for st, _ in blocks)
+    e["fwd_gbs"] = (256 if infer else 260) * rows / (fwd_ms * 1e-3) / 1e9
     if infer:
         e["step"] = "inference forward (no LSE) at every shift"
     else:
         e["tflops_no_recompute"] = (r["fwd_flops"] + 0.8 * r["bwd_flops"]) * world / (r["ms"] * 1e-3) / 1e12
         e["bwd_workspace_gb"] = r["ws_bytes"] / 1e9
+    if "phase_ms_per_step" in r:
+        e["roofline"] = roofline(wl, r, peaks)
     return e
 
 
@@ -312,6 +416,21 @@ def run_block(wl, dev, rank, steps, warmup, peaks):
             "unfused": "cuBLAS bf16 projections around the inference attention forward"}
 
 
+def workload_config(name, wl, world) -> dict:
+    """The `config` object of the JSON line: the workload's name and shapes."""
+    def shape(st):
+        return {"B_per_gpu": st["B"], "H": st["H"], "W": st["W"], "heads": st["heads"], "M": st["M"],
+                "shifts": list(st["shifts"])}
+    cfg = {"workload": name, "d": HEAD_DIM}
+    if "stages" in wl:
+        cfg["stages"] = [shape(st) for st in stages_of(wl)]
+    else:
+        cfg.update(shape(wl))
+    cfg.update({"qk_scale": wl.get("qk_scale", 1.0), "step": "fwd+bwd of every block",
+                "parallelism": f"dp{world}"})
+    return cfg
+
+
 def run_reference(args):
     """The fp64 CPU oracle as the reference arm (rank 0 only)."""
     rank = int(os.environ.get("RANK", "0"))
@@ -321,7 +440,8 @@ def run_reference(args):
 
     from vision_transformer_windowed_b200.inputs import make_inputs
     wl = WORKLOADS[args.workload]
-    t = make_inputs(wl["B"], wl["H"], wl["W"], wl["heads"], HEAD_DIM, device="cpu", qk_scale=wl["qk_scale"])
+    t = [make_inputs(st["B"], st["H"], st["W"], st["heads"], HEAD_DIM, device="cpu", qk_scale=st["qk_scale"])
+         for st in stages_of(wl)]
     per_step = max(1.0, args.reference_seconds / max(1, args.steps + args.warmup))
     for _ in range(args.warmup):
         cpu_baseline(t, wl, seconds=per_step)
@@ -335,8 +455,7 @@ def run_reference(args):
         "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": secs / args.steps * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": args.workload, **{k: v for k, v in wl.items() if k != "shifts"},
-                   "shifts": list(wl["shifts"]), "d": HEAD_DIM},
+        "config": workload_config(args.workload, wl, 1),
         "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": last["cores"], "kind": "oracle",
                          "sample": last["sample"] + " per step"},
         "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -359,7 +478,11 @@ def main():
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     if args.batch > 0:
-        WORKLOADS[args.workload] = dict(WORKLOADS[args.workload], B=args.batch)
+        wl0 = WORKLOADS[args.workload]
+        if "stages" in wl0:
+            WORKLOADS[args.workload] = dict(wl0, stages=[dict(st, B=args.batch) for st in wl0["stages"]])
+        else:
+            WORKLOADS[args.workload] = dict(wl0, B=args.batch)
     if args.impl == "reference":
         run_reference(args)
         return
@@ -387,38 +510,44 @@ def main():
 
     def run_workload(name, steps, warmup, phase=True, clocks=False):
         wl = WORKLOADS[name]
-        B, H, W, heads, M = wl["B"], wl["H"], wl["W"], wl["heads"], wl["M"]
-        t = dp.rank_inputs(B, H, W, heads, HEAD_DIM, rank, dev, qk_scale=wl["qk_scale"])
-        q, k, v, th, do = t["q"], t["k"], t["v"], t["theta"], t["dout"]
         infer = wl.get("infer", False)
-        outs = {s: (torch.empty_like(q), None if infer else torch.empty((B, H, W, heads), device=dev, dtype=torch.float32))
-                for s in wl["shifts"]}
-        grads = {} if infer else {s: (torch.empty_like(q), torch.empty_like(q), torch.empty_like(q), torch.empty_like(th))
-                                  for s in wl["shifts"]}
-        ws = torch.empty(0, dtype=torch.uint8) if infer else ops.alloc_workspace(q, M, wl["shifts"][0])
+        # per stage: inputs, a backward workspace, and the outputs of each of its blocks
+        data = []
+        for st in stages_of(wl):
+            B, H, W, heads, M = st["B"], st["H"], st["W"], st["heads"], st["M"]
+            t = dp.rank_inputs(B, H, W, heads, HEAD_DIM, rank, dev, qk_scale=st["qk_scale"])
+            blocks = []
+            for s in st["shifts"]:
+                o = torch.empty_like(t["q"])
+                lse = None if infer else torch.empty((B, H, W, heads), device=dev, dtype=torch.float32)
+                g = None if infer else (torch.empty_like(t["q"]), torch.empty_like(t["q"]), torch.empty_like(t["q"]),
+                                        torch.empty_like(t["theta"]))
+                blocks.append((s, o, lse, g))
+            ws = torch.empty(0, dtype=torch.uint8) if infer else ops.alloc_workspace(t["q"], M, st["shifts"][0])
+            data.append((st, t, blocks, ws))
 
         def step(evs=None):
-            if infer:  # forward only, O only
-                for si, s in enumerate(wl["shifts"]):
+            i = 0
+            for st, t, blocks, ws in data:
+                M = st["M"]
+                q, k, v, th, do = t["q"], t["k"], t["v"], t["theta"], t["dout"]
+                for s, o, lse, g in blocks:
                     if evs is not None:
-                        _lib.fs_set_phase_events([e.cuda_event for e in evs[si][0]])
-                    ops.winattn_fwd(q, k, v, th, M, s, o=outs[s][0], need_lse=False)
-                if evs is not None:
-                    _lib.fs_set_phase_events([])
-                return
-            for si, s in enumerate(wl["shifts"]):
-                o, lse = outs[s]
-                dq, dk, dv, dth = grads[s]
-                if evs is not None:
-                    _lib.fs_set_phase_events([e.cuda_event for e in evs[si][0]])
-                ops.winattn_fwd(q, k, v, th, M, s, o=o, lse=lse)
-                if evs is not None:
-                    _lib.fs_set_phase_events([e.cuda_event for e in evs[si][1]])
-                ops.winattn_bwd(q, k, v, o, do, lse, th, M, s, workspace=ws, dq=dq, dk=dk, dv=dv, dtheta=dth)
-                dp.allreduce_dtheta(dth)  # theta is shared by the whole data-parallel batch
+                        _lib.fs_set_phase_events([e.cuda_event for e in evs[i][0]])
+                    if infer:  # forward only, O only
+                        ops.winattn_fwd(q, k, v, th, M, s, o=o, need_lse=False)
+                    else:
+                        ops.winattn_fwd(q, k, v, th, M, s, o=o, lse=lse)
+                        if evs is not None:
+                            _lib.fs_set_phase_events([e.cuda_event for e in evs[i][1]])
+                        dq, dk, dv, dth = g
+                        ops.winattn_bwd(q, k, v, o, do, lse, th, M, s, workspace=ws, dq=dq, dk=dk, dv=dv, dtheta=dth)
+                        dp.allreduce_dtheta(dth)  # theta is shared by the whole data-parallel batch
+                    i += 1
             if evs is not None:
                 _lib.fs_set_phase_events([])
 
+        nblocks = len(blocks_of(wl))
         for _ in range(warmup):
             step()
         torch.cuda.synchronize()
@@ -426,7 +555,7 @@ def main():
         evsets = None
         if phase:
             evsets = [[([torch.cuda.Event(enable_timing=True) for _ in range(2)],
-                        [torch.cuda.Event(enable_timing=True) for _ in range(5)]) for _ in wl["shifts"]]
+                        [torch.cuda.Event(enable_timing=True) for _ in range(5)]) for _ in range(nblocks)]
                       for _ in range(steps)]
             for stp in evsets:  # torch creates the CUDA event on first record
                 for fe, be in stp:
@@ -453,88 +582,61 @@ def main():
         fwd_f, bwd_f = workload_flops(wl)
         if infer:
             bwd_f = 0.0
-        tokens = B * H * W * len(wl["shifts"])
+        tokens = workload_tokens(wl)
         res = {"ms": ms, "tflops": (fwd_f + bwd_f) * world / (ms * 1e-3) / 1e12,
                "tokens_per_s": tokens * world / (ms * 1e-3), "peak_gb": peak_gb,
-               "fwd_flops": fwd_f, "bwd_flops": bwd_f, "clocks": clk, "ws_bytes": ws.numel()}
+               "fwd_flops": fwd_f, "bwd_flops": bwd_f, "clocks": clk,
+               "ws_bytes": sum(x[3].numel() for x in data)}
         if evsets:
-            names = ["fwd", "bwd_prep", "bwd_main", "bwd_post", "bwd_dtheta"]
-            tot = {n: 0.0 for n in names}
+            tot = {n: 0.0 for n in PHASES}
             for stp in evsets:
                 for fe, be in stp:
                     tot["fwd"] += fe[0].elapsed_time(fe[1])
                     if infer:
                         continue
                     for j in range(4):
-                        tot[names[1 + j]] += be[j].elapsed_time(be[j + 1])
-            if infer:
-                names = ["fwd"]
-                tot = {"fwd": tot["fwd"]}
-            launches = steps * len(wl["shifts"])
+                        tot[PHASES[1 + j]] += be[j].elapsed_time(be[j + 1])
+            names = ["fwd"] if infer else PHASES
+            tot = {n: tot[n] for n in names}
+            launches = steps * nblocks
             res["phase_ms"] = {n: tot[n] / launches for n in names}  # average per launch
+            res["phase_ms_per_step"] = {n: tot[n] / steps for n in names}
             res["phase_share"] = {n: tot[n] / max(sum(tot.values()), 1e-9) for n in names}
             res["launches_per_kernel"] = launches
-        res["tensors"] = t
+        res["data"] = data
         return res
 
     main_res = run_workload(args.workload, args.steps, args.warmup, phase=True, clocks=True)
     wl = WORKLOADS[args.workload]
-    B, H, W, heads, M = wl["B"], wl["H"], wl["W"], wl["heads"], wl["M"]
-    nshift = len(wl["shifts"])
-
-    # roofline of the dominant kernel (largest share of the step)
-    ph = main_res["phase_ms"]
-    dom = max(ph, key=lambda n: main_res["phase_share"][n])
-    th = B * H * W * heads
-    pairs_per_launch = (main_res["fwd_flops"] / (4.0 * HEAD_DIM)) / nshift
-    # bytes each kernel must move per token-head row: windows inside one tile run the whole
-    # backward as one kernel (Q, K, V, O, dO read, dQ, dK, dV written, LSE and D: 520 B);
-    # larger windows run prep / main / post with workspace round trips (prep: q, k, o, dO, lse in,
-    # q', k' images, lse2, D and the zeroed dQ' accumulator out; main: the images, dO, v, lse2, D in,
-    # dk, dv out; post: the dQ' accumulator and q in, dq out)
-    if M * M < 128:
-        algo_bytes = {"fwd": 260, "bwd_prep": 0, "bwd_main": 520, "bwd_post": 0, "bwd_dtheta": 0}
-    else:
-        algo_bytes = {"fwd": 260, "bwd_prep": 524, "bwd_main": 392, "bwd_post": 256, "bwd_dtheta": 0}
-    hbm_bound = M <= 8
-    if hbm_bound or dom in ("bwd_prep", "bwd_post", "bwd_dtheta"):
-        achieved = algo_bytes[dom] * th / (ph[dom] * 1e-3) / 1e9
-        roof = {"kernel": dom, "bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                "frac": achieved / peaks["hbm_gbs"], "traffic": None,
-                "algorithmic_bytes_per_launch": algo_bytes[dom] * th,
-                "peak_note": f"HBM copy bandwidth, {peaks['source']}"}
-    else:
-        fl = (4.0 if dom == "fwd" else 10.0) * HEAD_DIM * pairs_per_launch
-        achieved = fl / (ph[dom] * 1e-3) / 1e12
-        roof = {"kernel": dom, "bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"],
-                "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops"], "traffic": None,
-                "algorithmic_flops_per_launch": fl, "peak_note": f"cuBLAS bf16 burst, {peaks['source']}"}
-    roof["avg_launch_ms"] = ph[dom]
-    roof["traffic"] = measured_traffic(dom, args.workload)
+    blocks = blocks_of(wl)
+    sm_mhz = main_res["clocks"]["sm_mhz"] if main_res["clocks"] else None
+    roof = roofline(wl, main_res, peaks, sm_mhz)
+    roof["traffic"] = measured_traffic(roof["kernel"], args.workload)
 
     # end to end through the public API with host buffers (pinned), copies inside the timed region
-    t = main_res["tensors"]
-    host = {k: t[k].cpu().pin_memory() for k in ("q", "k", "v", "dout", "theta")}
+    host = [{k: t[k].cpu().pin_memory() for k in ("q", "k", "v", "dout", "theta")} for _, t, _, _ in main_res["data"]]
     res_host = {}
     e2e_steps = max(1, min(args.steps, 5))
     torch.cuda.synchronize()
-    h2d = sum(x.numel() * x.element_size() for x in host.values())
+    h2d = sum(x.numel() * x.element_size() for hs in host for x in hs.values())
     d2h = 0
 
     def e2e_step():
         nonlocal d2h
         d2h = 0
-        dv = {k: x.to(dev, non_blocking=True) for k, x in host.items()}
-        for s in wl["shifts"]:
-            o, lse = ops.winattn_fwd(dv["q"], dv["k"], dv["v"], dv["theta"], M, s)
-            dq, dk, dvv, dth = ops.winattn_bwd(dv["q"], dv["k"], dv["v"], o, dv["dout"], lse, dv["theta"], M, s)
-            dp.allreduce_dtheta(dth)
-            for name, x in (("o", o), ("dq", dq), ("dk", dk), ("dv", dvv), ("dtheta", dth)):
-                key = (s, name)
-                if key not in res_host:
-                    res_host[key] = torch.empty(x.shape, dtype=x.dtype, pin_memory=True)
-                res_host[key].copy_(x, non_blocking=True)
-                d2h += x.numel() * x.element_size()
+        for si, (st, hs) in enumerate(zip(stages_of(wl), host)):
+            M = st["M"]
+            dv = {k: x.to(dev, non_blocking=True) for k, x in hs.items()}
+            for bi, s in enumerate(st["shifts"]):
+                o, lse = ops.winattn_fwd(dv["q"], dv["k"], dv["v"], dv["theta"], M, s)
+                dq, dk, dvv, dth = ops.winattn_bwd(dv["q"], dv["k"], dv["v"], o, dv["dout"], lse, dv["theta"], M, s)
+                dp.allreduce_dtheta(dth)
+                for name, x in (("o", o), ("dq", dq), ("dk", dk), ("dv", dvv), ("dtheta", dth)):
+                    key = (si, bi, name)
+                    if key not in res_host:
+                        res_host[key] = torch.empty(x.shape, dtype=x.dtype, pin_memory=True)
+                    res_host[key].copy_(x, non_blocking=True)
+                    d2h += x.numel() * x.element_size()
 
     e2e_step()
     torch.cuda.synchronize()
@@ -551,14 +653,14 @@ def main():
            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
 
     per_config = {args.workload: config_entry(wl, main_res, peaks, world)}
-    del main_res["tensors"], t, host, res_host
+    del main_res["data"], host, res_host
     if not args.no_extra:
         for name in WORKLOADS:
             if name == args.workload:
                 continue
             torch.cuda.empty_cache()
             r = run_workload(name, max(3, args.steps // 2), 3, phase=True, clocks=False)
-            del r["tensors"]
+            del r["data"]
             per_config[name] = config_entry(WORKLOADS[name], r, peaks, world)
 
     if not args.no_extra:
@@ -568,24 +670,24 @@ def main():
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        tt = make_inputs(B, H, W, heads, HEAD_DIM, device="cpu", qk_scale=wl["qk_scale"])
+        tt = [make_inputs(st["B"], st["H"], st["W"], st["heads"], HEAD_DIM, device="cpu", qk_scale=st["qk_scale"])
+              for st in stages_of(wl)]
         cpu = cpu_baseline(tt, wl)
         cpu.pop("seconds", None)
 
     if rank == 0:
+        nlaunch = sum(1 + (2 if st["M"] * st["M"] < 128 else 5) for st, _ in blocks)
         line = {
             "metric": METRIC, "value": main_res["tflops"], "unit": "TFLOP/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": main_res["ms"], "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": {"workload": args.workload, "B_per_gpu": B, "H": H, "W": W, "heads": heads, "d": HEAD_DIM,
-                       "M": M, "shifts": list(wl["shifts"]), "qk_scale": wl["qk_scale"],
-                       "step": "fwd+bwd at every shift", "parallelism": f"dp{world}",
-                       "l2": "inputs larger than L2 (each tensor > 126 MB)"},
+            "config": dict(workload_config(args.workload, wl, world),
+                           l2="inputs larger than L2 (the largest stage's tensors > 126 MB each)"),
             "pct_bf16_peak": 100 * main_res["tflops"] / peaks["bf16_tflops"] / world,
             "tokens_per_s": main_res["tokens_per_s"], "peak_gb": main_res["peak_gb"],
-            # per shift: the forward, then the one-tile backward and the d theta sum (windows
-            # inside one tile) or prep, main, post and the d theta sum
-            "gpu_launches": args.steps * nshift * (1 + (2 if M * M < 128 else 4)),
+            # per block: the forward, then the one-tile backward and the d theta sum (windows
+            # inside one tile) or prep, scale, main, post and the d theta sum
+            "gpu_launches": args.steps * nlaunch,
             "roofline": roof, "clocks": main_res["clocks"], "e2e": e2e, "cpu_baseline": cpu,
             "per_config": per_config, "peaks": peaks,
         }

@@ -59,3 +59,48 @@ def test_cpu_baseline_samples_every_unit_of_a_small_workload():
     assert f"{n_units} of {n_units} at s=0" in res["sample"] and f"{n_units} of {n_units} at s=4" in res["sample"]
     assert res["units_per_s"] == pytest.approx(2 * n_units / res["seconds"])
     assert res["full_step_s_extrapolated"] == pytest.approx(res["seconds"])
+
+
+def test_four_stage_workload_counts_every_block():
+    """The headline step: FlashSwin-T's four stages at p=2, an unshifted and a
+    shifted block per stage (stage 4 twice unshifted), flops from the brute-force
+    pair count of every block."""
+    wl = bench.WORKLOADS["flashswin_t_p2_4stage"]
+    blocks = bench.blocks_of(wl)
+    assert [(st["H"], st["heads"], st["M"], s) for st, s in blocks] == [
+        (128, 3, 32, 0), (128, 3, 32, 16), (64, 6, 32, 0), (64, 6, 32, 16),
+        (32, 12, 32, 0), (32, 12, 32, 16), (16, 24, 16, 0), (16, 24, 16, 0)]
+    # the pair count of a block is per image and head: brute force on one image, one head
+    pairs = sum(_brute_pairs(1, st["H"], st["W"], 1, st["M"], s) * st["B"] * st["heads"] for st, s in blocks)
+    fwd, bwd = bench.workload_flops(wl)
+    assert fwd == 4 * 32 * pairs and bwd == 10 * 32 * pairs
+    assert bench.workload_tokens(wl) == 128 * 2 * (128 ** 2 + 64 ** 2 + 32 ** 2 + 16 ** 2)
+
+
+def test_roofline_of_the_dominant_kernel():
+    wl = dict(stages=[dict(B=1, H=64, W=64, heads=2, M=32, shifts=(0, 16)),
+                      dict(B=1, H=16, W=16, heads=4, M=16, shifts=(0,))], qk_scale=1.0)
+    blocks = bench.blocks_of(wl)
+    peaks = {"hbm_gbs": 6000.0, "bf16_tflops": 1600.0, "bf16_tflops_sustained": 1400.0, "source": "measured"}
+    res = {"phase_ms_per_step": {"fwd": 1.0, "bwd_prep": 0.2, "bwd_main": 2.0, "bwd_post": 0.1, "bwd_dtheta": 0.01}}
+    roof = bench.roofline(wl, res, peaks, sm_mhz=1900.0)
+    fl = sum(10 * 32 * bench.unmasked_pairs(st["B"], st["H"], st["W"], st["heads"], st["M"], s) for st, s in blocks)
+    assert roof["kernel"] == "bwd_main" and roof["bound"] == "tensor"
+    assert roof["achieved"] == pytest.approx(fl / 2e-3 / 1e12)
+    assert roof["frac"] == pytest.approx(roof["achieved"] / 1400.0)
+    assert roof["mufu_ceiling_tflops"] == pytest.approx(320 * 16 * 148 * 1900e6 / 1e12)
+    # windows inside one tile: HBM-bound, 520 bytes per token-head row for the one-tile backward
+    wl8 = dict(B=2, H=16, W=16, heads=3, M=8, shifts=(0, 4), qk_scale=1.0)
+    roof8 = bench.roofline(wl8, res, peaks)
+    assert roof8["bound"] == "hbm" and roof8["kernel"] == "bwd_main"
+    assert roof8["achieved"] == pytest.approx(2 * 520 * 2 * 16 * 16 * 3 / 2e-3 / 1e9)
+
+
+def test_cpu_baseline_samples_every_stage():
+    wl = dict(stages=[dict(B=1, H=16, W=16, heads=2, M=8, shifts=(0, 4)),
+                      dict(B=1, H=16, W=16, heads=1, M=16, shifts=(0,))], qk_scale=1.0)
+    t = [make_inputs(1, 16, 16, 2, 32), make_inputs(1, 16, 16, 1, 32)]
+    res = bench.cpu_baseline(t, wl, seconds=2.0)
+    assert "8 of 8 at 16x16/M=8 s=0" in res["sample"] and "8 of 8 at 16x16/M=8 s=4" in res["sample"]
+    assert "1 of 1 at 16x16/M=16 s=0" in res["sample"]
+    assert res["units_per_s"] == pytest.approx(17 / res["seconds"])
