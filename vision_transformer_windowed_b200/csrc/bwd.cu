@@ -519,7 +519,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         bool ok = true;
         for (long long item = blockIdx.x; item < prm.items && ok; item += gridDim.x) {
             const Item I = item_of(g, item);
-            const uint32_t keyseg = seg_at(d_tile_segs(g, I.u, I.win), r >> g.lBT);
+            const uint32_t keyseg = I.masked ? seg_at(d_tile_segs(g, I.u, I.win), r >> g.lBT) : 0u;
             for (int n = 0; n < I.nq && ok; ++n) {
                 if (!q_active(g, I, n)) continue;
                 const int st = qc % kQStages;
@@ -528,7 +528,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const float* dvec = lse2 + kTile;
                 uint8_t* ds = smem + kDSOff + (j & 1) * kDSBytes;
                 // bit c: query columns [16 c, 16 c + 16) attend this key row
-                const uint32_t a16 = d_allow16(g, keyseg, I.q0 + n, I.win);
+                // every 16-column group attends unless the window is cut by the mask
+                const uint32_t a16 = I.masked ? d_allow16(g, keyseg, I.q0 + n, I.win) : 0xFFu;
                 for (int h = 0; h < 2; ++h, ++hc) {
                     const uint32_t b = hc & 1u;
                     const int col0 = 64 * h + 32 * cw;  // this thread's 32 query columns

@@ -9,7 +9,7 @@
 //                     memory (bf16 in, fp16 out)
 //   warp 8 + w        TMA producer (window boxes at shifted addresses)
 //   warp 10 + w       tcgen05 MMA issuer: S = Q'K'^T and O_tile = P V in TMEM
-// plus its own Q slots, K/V ring, output staging tile, RoPE table and 224 TMEM
+// plus its own Q slots, K/V ring, output staging tile, RoPE table and 256 TMEM
 // columns.  The workers share nothing but the SM, so neither ever waits for
 // the other.
 //
@@ -46,7 +46,6 @@ __device__ __forceinline__ int kv_off(int w) { return w * kWorkerBytes + kQBytes
 __device__ __forceinline__ int ost_off(int w) { return w * kWorkerBytes + kQBytes + kKVBytes; }
 __device__ __forceinline__ int tab_off(int w) { return w * kWorkerBytes + kQBytes + kKVBytes + kTileBytes; }
 
-// TMEM columns per worker: S [128 cols], P (bf16) [64], O tile [32]
 // TMEM columns per worker: two S buffers of 128 columns, used by alternate
 // tiles.  A tile's P (bf16) is written over the first 64 columns of its S
 // buffer as the softmax consumes them, and the tile's P V product goes to
@@ -331,7 +330,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 if (!group_sync(0x407)) return false;
             }
-            myseg = seg_at(d_tile_segs(g, I.X, I.win), r >> g.lBT);
+            myseg = I.masked ? seg_at(d_tile_segs(g, I.X, I.win), r >> g.lBT) : 0u;
             unext = __ffs(I.act) - 1;
             const int qi = jt & 1;
             if (!wwait(&B.q_full[qi], (jt >> 1) & 1, 0x401)) return false;
@@ -351,7 +350,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (!((I.act >> u) & 1u)) continue;
                 // rotate the following K tile while this tile's S is computed
                 if (!rotate_next()) { ok = false; break; }
-                const uint32_t a16 = d_allow16(g, myseg, I.kv0 + u, I.win);
+                // every 16-column group attends unless the window is cut by the mask
+                const uint32_t a16 = I.masked ? d_allow16(g, myseg, I.kv0 + u, I.win) : 0xFFu;
                 const bool full = a16 == 0xFFu;
                 const uint32_t b = tcs & 1u;
                 const uint32_t t_s = t_row + col_s(wk, b);

@@ -19,6 +19,7 @@ struct FwdItem {
     long long kv0;    // first key/value tile of the group
     int nkv;          // key/value tiles in the group (<= 32)
     uint32_t act;     // bit u: tile kv0 + u holds keys that query tile X attends
+    bool masked;      // some pairs of the group do not attend (the shift-region mask, or several windows per tile)
     Win win;          // the window (>= 128 tokens) or the first window of tile X
 };
 
@@ -36,7 +37,8 @@ __host__ __device__ inline FwdItem fwd_item(const Geo& g, long long it) {
         I.nkv = g.tpw;
         I.win = win_of(g, gw);
         I.act = low_bits(g.tpw);
-        if (g.s && (I.win.wr == g.Hp / g.M - 1 || I.win.wc == g.nWw - 1)) {
+        I.masked = g.s && (I.win.wr == g.Hp / g.M - 1 || I.win.wc == g.nWw - 1);
+        if (I.masked) {
             const uint64_t sx = tile_segs(g, I.X, I.win);
             I.act = 0;
             for (int u = 0; u < g.tpw; ++u)
@@ -47,6 +49,7 @@ __host__ __device__ inline FwdItem fwd_item(const Geo& g, long long it) {
         I.nkv = 1;
         I.win = tile_win(g, I.X);
         I.act = 1u;
+        I.masked = true;
     }
     return I;
 }
@@ -59,6 +62,7 @@ struct BwdItem {
     int nq;         // candidate query tiles (<= 32)
     bool paired;    // small windows: the only query tile is u
     uint32_t act;   // bit n: query tile q0 + n attends to u
+    bool masked;    // some pairs of the group do not attend (the shift-region mask, or several windows per tile)
     Win win;        // the window (>= 256 tokens) or the first window of tile u
 };
 
@@ -80,7 +84,8 @@ __host__ __device__ inline BwdItem bwd_item(const Geo& g, long long it) {
         I.paired = false;
         I.win = win_of(g, gw);
         I.act = low_bits(g.tpw);
-        if (g.s && (I.win.wr == g.Hp / g.M - 1 || I.win.wc == g.nWw - 1)) {
+        I.masked = g.s && (I.win.wr == g.Hp / g.M - 1 || I.win.wc == g.nWw - 1);
+        if (I.masked) {
             const uint64_t su = tile_segs(g, I.u, I.win);
             I.act = 0;
             for (int n = 0; n < g.tpw; ++n)
@@ -95,6 +100,7 @@ __host__ __device__ inline BwdItem bwd_item(const Geo& g, long long it) {
         I.paired = true;
         I.win = tile_win(g, T);
         I.act = 1u;
+        I.masked = true;
     }
     return I;
 }
