@@ -120,18 +120,21 @@ def kernel_sources_sha256(tu: str) -> str:
     return h.hexdigest()
 
 
-def measured_traffic(kernel: str, workload: str):
-    """DRAM bytes per launch of `kernel` from the committed ncu capture, or None when
-    there is none for this workload or the kernel sources changed since."""
+def measured_traffic(phase: str, workload: str):
+    """DRAM bytes per step of the workload's `phase` kernel from the committed ncu capture, or None
+    when there is none for this workload or the kernel's sources changed since."""
     path = os.path.join(os.path.dirname(os.path.abspath(__file__)), "profiles", "traffic.json")
     try:
         with open(path) as fh:
-            rec = json.load(fh).get(kernel)
+            recs = json.load(fh).get("records", [])
     except (OSError, ValueError):
         return None
-    if not rec or rec.get("workload") != workload or rec.get("sources_sha256") != kernel_sources_sha256(rec["source"]):
-        return None
-    return rec["bytes_per_launch"]
+    for rec in recs:
+        if rec.get("phase") == phase and rec.get("workload") == workload:
+            if rec.get("sources_sha256") != kernel_sources_sha256(rec["source"]):
+                return None
+            return rec["bytes_per_step"]
+    return None
 
 
 def stages_of(wl) -> list:
@@ -212,7 +215,7 @@ def roofline(wl, res, peaks, sm_mhz=None) -> dict:
         peak = peaks["bf16_tflops_sustained"]
         roof = {"kernel": dom, "bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                 "frac": achieved / peak, "frac_of_burst": achieved / peaks["bf16_tflops"], "traffic": None,
-                "algorithmic_flops_per_step": fl,
+                "algorithmic_flops_per_step": fl, "algorithmic_bytes_per_step": sum(w["bytes"][dom] for w in work),
                 "peak_note": f"cuBLAS bf16 sustained (burst {peaks['bf16_tflops']:.1f}), {peaks['source']}"}
         per_exp = (4.0 if dom == "fwd" else 10.0) * HEAD_DIM
         mhz = sm_mhz or 1965.0
@@ -337,7 +340,7 @@ def cpu_baseline(tensors, wl, seconds: float = 12.0):
             "seconds": total_dt}
 
 
-def config_entry(wl, r, peaks, world) -> dict:
+def config_entry(wl, r, peaks, world, name=None) -> dict:
     """Per-workload figures: fwd+bwd and forward-alone throughput, the no-recompute count of
     the backward (8 d per pair instead of 10 d), % of the measured and of the spec bf16 peak,
     the forward's algorithmic HBM rate, peak memory and the backward workspace."""
@@ -360,6 +363,8 @@ def config_entry(wl, r, peaks, world) -> dict:
         e["bwd_workspace_gb"] = r["ws_bytes"] / 1e9
     if "phase_ms_per_step" in r:
         e["roofline"] = roofline(wl, r, peaks)
+        if name is not None:
+            e["roofline"]["traffic"] = measured_traffic(e["roofline"]["kernel"], name)
     return e
 
 
@@ -611,7 +616,7 @@ def main():
     blocks = blocks_of(wl)
     sm_mhz = main_res["clocks"]["sm_mhz"] if main_res["clocks"] else None
     roof = roofline(wl, main_res, peaks, sm_mhz)
-    roof["traffic"] = measured_traffic(roof["kernel"], args.workload)
+    roof["traffic"] = measured_traffic(roof["kernel"], args.workload)  # bytes per step, like "achieved"
 
     # end to end through the public API with host buffers (pinned), copies inside the timed region
     host = [{k: t[k].cpu().pin_memory() for k in ("q", "k", "v", "dout", "theta")} for _, t, _, _ in main_res["data"]]
@@ -652,7 +657,7 @@ def main():
     e2e = {"value": fl * world / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s", "ms_per_step": e2e_ms,
            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
 
-    per_config = {args.workload: config_entry(wl, main_res, peaks, world)}
+    per_config = {args.workload: config_entry(wl, main_res, peaks, world, args.workload)}
     del main_res["data"], host, res_host
     if not args.no_extra:
         for name in WORKLOADS:
@@ -661,7 +666,7 @@ def main():
             torch.cuda.empty_cache()
             r = run_workload(name, max(3, args.steps // 2), 3, phase=True, clocks=False)
             del r["data"]
-            per_config[name] = config_entry(WORKLOADS[name], r, peaks, world)
+            per_config[name] = config_entry(WORKLOADS[name], r, peaks, world, name)
 
     if not args.no_extra:
         for name, wl_b in BLOCK_WORKLOADS.items():

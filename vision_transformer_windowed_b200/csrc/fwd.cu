@@ -357,24 +357,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const uint32_t t_s = t_row + col_s(wk, b);
                 if (!wwait(&B.s_full[b], (tcs >> 1) & 1u, 0x403)) { ok = false; break; }
                 tc_fence_after();
-                // pass 1: row maximum of the attended raw scores
-                float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-#pragma unroll 1
-                for (int c = 0; c < 4; ++c) {  // rolled: keeps live ranges (registers) short
-                    uint32_t v[32];
-                    tmem_ld32(t_s + 32 * c, v);
-                    tmem_wait_ld();
-                    if (!full) {
-#pragma unroll
-                        for (int e = 0; e < 32; ++e)
-                            if (!((a16 >> (2 * c + (e >> 4))) & 1u)) v[e] = __float_as_uint(-INFINITY);
-                    }
-#pragma unroll
-                    for (int e = 0; e < 32; e += 2)
-                        mx4[(e >> 1) & 3] = fmax3(mx4[(e >> 1) & 3], __uint_as_float(v[e]), __uint_as_float(v[e + 1]));
-                }
-                const float mx = fmaxf(fmax3(mx4[0], mx4[1], mx4[2]), mx4[3]);
-                const float m_tile = mx * sl2;
                 if (!first) {  // the previous tile's P V product, in the other S buffer
                     if (!wwait(&B.o_full, oph, 0x404)) { ok = false; break; }
                     oph ^= 1;
@@ -388,25 +370,79 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                     for (int e = 0; e < 32; e += 2)
                         fadd2(o[e], o[e + 1], o[e], o[e + 1], __uint_as_float(v[e]), __uint_as_float(v[e + 1]));
-                }
-                if (m_tile > m + 8.f) {
-                    const float alpha = ex2_approx(m - m_tile);
+                } else {
+                    // the item's first tile: its row maximum in a pass of its own
+                    float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll 1
+                    for (int c = 0; c < 4; ++c) {  // rolled: keeps live ranges (registers) short
+                        uint32_t v[32];
+                        tmem_ld32(t_s + 32 * c, v);
+                        tmem_wait_ld();
+                        if (!full) {
 #pragma unroll
-                    for (int e = 0; e < 32; e += 2) fmul2(o[e], o[e + 1], o[e], o[e + 1], alpha, alpha);
-                    l *= alpha;
-                    m = m_tile;
+                            for (int e = 0; e < 32; ++e)
+                                if (!((a16 >> (2 * c + (e >> 4))) & 1u)) v[e] = __float_as_uint(-INFINITY);
+                        }
+#pragma unroll
+                        for (int e = 0; e < 32; e += 2)
+                            mx4[(e >> 1) & 3] =
+                                fmax3(mx4[(e >> 1) & 3], __uint_as_float(v[e]), __uint_as_float(v[e + 1]));
+                    }
+                    m = fmaxf(fmax3(mx4[0], mx4[1], mx4[2]), mx4[3]) * sl2;  // O and l are zero
                 }
-                const float mu = (m == -INFINITY) ? 0.f : m;
-                // pass 2: probabilities, row sum, bf16 P into TMEM.  A masked
-                // 16-column group gets the addend -inf: exp2(-inf) = 0 for free.
+                // Probabilities, row sum, bf16 P into TMEM.  A masked 16-column group
+                // gets the addend -inf: exp2(-inf) = 0 for free.  After an item's first
+                // tile the running maximum m is known, so one pass suffices: each
+                // chunk's maximum is checked first, and only when it exceeds m by more
+                // than 2^64 (or m is still -inf) are m, l, O and the tile's P chunks
+                // already written rescaled.  (P up to 2^64 stays far inside the range of
+                // bf16 and of the fp32 sums; the result is the same softmax.)
                 float l4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll 1
                 for (int c = 0; c < 4; ++c) {
                     uint32_t v[32];
                     tmem_ld32(t_s + 32 * c, v);
                     tmem_wait_ld();
-                    const float add0 = ((a16 >> (2 * c)) & 1u) ? -mu : -INFINITY;
-                    const float add1 = ((a16 >> (2 * c + 1)) & 1u) ? -mu : -INFINITY;
+                    const bool ok0 = (a16 >> (2 * c)) & 1u, ok1 = (a16 >> (2 * c + 1)) & 1u;
+                    if (!first) {
+                        float c4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+                        if (ok0) {
+#pragma unroll
+                            for (int e = 0; e < 16; e += 2)
+                                c4[(e >> 1) & 1] = fmax3(c4[(e >> 1) & 1], __uint_as_float(v[e]), __uint_as_float(v[e + 1]));
+                        }
+                        if (ok1) {
+#pragma unroll
+                            for (int e = 16; e < 32; e += 2)
+                                c4[2 + ((e >> 1) & 1)] =
+                                    fmax3(c4[2 + ((e >> 1) & 1)], __uint_as_float(v[e]), __uint_as_float(v[e + 1]));
+                        }
+                        const float cm = fmaxf(fmaxf(c4[0], c4[1]), fmaxf(c4[2], c4[3])) * sl2;
+                        const bool grow = cm > m + 64.f;
+                        if (__any_sync(0xFFFFFFFFu, grow)) {
+                            const float alpha = grow ? ex2_approx(m - cm) : 1.f;
+                            if (grow) m = cm;
+#pragma unroll
+                            for (int e = 0; e < 32; e += 2) fmul2(o[e], o[e + 1], o[e], o[e + 1], alpha, alpha);
+                            l *= alpha;
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) l4[e] *= alpha;
+                            if (c > 0) tmem_wait_st();
+#pragma unroll 1
+                            for (int k = 0; k < c; ++k) {  // this tile's P chunks already in TMEM
+                                uint32_t pw[16];
+                                tmem_ld16(t_s + kColP + 16 * k, pw);
+                                tmem_wait_ld();
+#pragma unroll
+                                for (int e = 0; e < 16; ++e)
+                                    pw[e] = pack_bf16x2(bf16lo_to_f32(pw[e]) * alpha, bf16hi_to_f32(pw[e]) * alpha);
+                                tmem_st16(t_s + kColP + 16 * k, pw);
+                            }
+                        }
+                    }
+                    const float mu = (m == -INFINITY) ? 0.f : m;
+                    const float add0 = ok0 ? -mu : -INFINITY;
+                    const float add1 = ok1 ? -mu : -INFINITY;
                     uint32_t w[16];
 #pragma unroll
                     for (int e = 0; e < 16; ++e) {
