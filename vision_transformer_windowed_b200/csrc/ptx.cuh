@@ -311,44 +311,6 @@ __device__ __forceinline__ void fmul2(float& dx, float& dy, float ax, float ay, 
         : "f"(ax), "f"(ay), "f"(bx), "f"(by));
 }
 
-__device__ __forceinline__ void fsub2(float& dx, float& dy, float ax, float ay, float bx, float by) {
-    asm("{\n\t.reg .b64 a, b, d;\n\tmov.b64 a, {%2, %3};\n\tmov.b64 b, {%4, %5};\n\t"
-        "sub.rn.f32x2 d, a, b;\n\tmov.b64 {%0, %1}, d;\n\t}"
-        : "=f"(dx), "=f"(dy)
-        : "f"(ax), "f"(ay), "f"(bx), "f"(by));
-}
-
-// 2^x for a pair of values on the FMA and integer pipes (no MUFU), to take part
-// of a softmax's exponentials off the MUFU unit.  Method: Cody-Waite style
-// range reduction (W. J. Cody and W. Waite, "Software Manual for the
-// Elementary Functions", 1980) x = j + f with j = floor(x), f in [0, 1): one
-// add rounded toward minus infinity against 1.5 * 2^23 leaves j in the low
-// mantissa bits; 2^f by a cubic in f whose coefficients were fitted for this
-// library by linear programming (smallest maximum relative error over [0, 1]
-// with the constant term fixed at 1, so that 2^0 is exact): maximum relative
-// error 8.6e-5, below half a bf16 ulp; 2^j is then added to the exponent field.
-// x is clamped at -127 (the result there is below 2^-126, about 1e-38), and
-// must stay below 128.
-__device__ __forceinline__ void ex2_fma2(float& y0, float& y1, float x0, float x1) {
-    constexpr float kRound = 12582912.0f;  // 1.5 * 2^23
-    x0 = fmaxf(x0, -127.f);
-    x1 = fmaxf(x1, -127.f);
-    float t0, t1, j0, j1, f0, f1, p0, p1;
-    asm("{\n\t.reg .b64 a, b, d;\n\tmov.b64 a, {%2, %3};\n\tmov.b64 b, {%4, %4};\n\t"
-        "add.rm.f32x2 d, a, b;\n\tmov.b64 {%0, %1}, d;\n\t}"
-        : "=f"(t0), "=f"(t1)
-        : "f"(x0), "f"(x1), "f"(kRound));
-    fsub2(j0, j1, t0, t1, kRound, kRound);  // floor(x), exact
-    fsub2(f0, f1, x0, x1, j0, j1);          // x - floor(x), exact
-    ffma2(p0, p1, f0, f1, 0.07706724107265472f, 0.07706724107265472f, 0.22764497995376587f, 0.22764497995376587f);
-    ffma2(p0, p1, p0, p1, f0, f1, 0.6951166391372681f, 0.6951166391372681f);
-    ffma2(p0, p1, p0, p1, f0, f1, 1.0f, 1.0f);
-    // the low bits of t hold floor(x) in two's complement; shifted into the exponent
-    // field they add floor(x) to p's exponent (1.5 * 2^23 has zeros there)
-    y0 = __uint_as_float(__float_as_uint(p0) + (__float_as_uint(t0) << 23));
-    y1 = __uint_as_float(__float_as_uint(p1) + (__float_as_uint(t1) << 23));
-}
-
 // Packs two floats into f16x2 with `lo` in the low half (round to nearest even).
 __device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
     uint32_t r;
