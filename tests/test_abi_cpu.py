@@ -38,8 +38,10 @@ GOOD = [(1, 16, 16, 2, 32, 8, 0), (128, 64, 64, 3, 32, 8, 4), (128, 128, 128, 3,
         (2, 8, 24, 1, 32, 4, 0), (1, 32, 32, 1, 32, 32, 0),
         # H or W not a multiple of M: padded to the next multiple
         (1, 20, 16, 2, 32, 8, 0), (1, 16, 20, 2, 32, 8, 4), (2, 200, 334, 3, 32, 8, 4),
-        (1, 33, 17, 1, 32, 16, 8), (1, 65, 100, 1, 32, 64, 32)]
-BAD = [(1, 16, 16, 2, 64, 8, 0),    # d != 32
+        (1, 33, 17, 1, 32, 16, 8), (1, 65, 100, 1, 32, 64, 32),
+        (1, 16, 16, 2, 64, 8, 4), (1, 64, 64, 1, 64, 32, 16), (1, 20, 13, 2, 64, 8, 4)]
+BAD = [(1, 16, 16, 2, 48, 8, 0),    # d not 32 or 64
+       (1, 16, 16, 2, 16, 8, 0),
        (1, 16, 16, 2, 32, 12, 0),   # M not supported
        (1, 7, 16, 2, 32, 8, 0),     # H < M
        (1, 16, 15, 2, 32, 16, 0),   # W < M
@@ -128,3 +130,11 @@ def test_block_forward_rejects_before_launch():
     assert call((1, 16, 16, 4, 32, 8, 0), *ok) == _lib.FS_ERR_SHAPE    # four heads
     assert call((1, 16, 16, 3, 32, 8, 0), 0, *ok[1:]) == _lib.FS_ERR_NULL
     assert call((1, 16, 16, 3, 32, 8, 0), 24, *ok[1:]) == _lib.FS_ERR_ALIGN
+
+
+def test_workspace_flat_in_window_size_at_d64():
+    """64-channel heads: the backward scratch depends on the token count only."""
+    a = _lib.fs_winattn_bwd_workspace_bytes(_lib.make_shape(16, 256, 256, 3, 64, 32, 16))
+    b = _lib.fs_winattn_bwd_workspace_bytes(_lib.make_shape(16, 256, 256, 3, 64, 64, 32))
+    c = _lib.fs_winattn_bwd_workspace_bytes(_lib.make_shape(16, 256, 256, 3, 64, 8, 4))
+    assert a == b == c > 0

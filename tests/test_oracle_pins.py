@@ -38,6 +38,8 @@ SHAPES = [  # (B, H, W, heads, d, M, s)
     (1, 6, 6, 1, 4, 3, 1),
     (1, 16, 16, 2, 32, 8, 4),
     (1, 16, 8, 3, 32, 8, 0),
+    (1, 8, 8, 1, 64, 4, 2),      # 64-channel heads (16 RoPE pairs per axis)
+    (1, 16, 16, 2, 64, 8, 4),
 ]
 
 
@@ -170,10 +172,10 @@ def test_shift_consistency_interior_windows():
     assert not np.allclose(r["o"][0, (H - 1 + s) % H], o_back[0, (H - 1 + s) % H], atol=1e-6)
 
 
-@pytest.mark.parametrize("s", [0, 2])
-def test_finite_difference_gradients(s):
+@pytest.mark.parametrize("s,d", [(0, 8), (2, 8), (2, 64)])
+def test_finite_difference_gradients(s, d):
     """Central differences of L = sum(O * dO) in fp64 (rel. err <= 1e-6)."""
-    B, H, W, h, d, M = 1, 8, 8, 2, 8, 4
+    B, H, W, h, M = 1, 8, 8, 2, 4
     inp = _f64(make_inputs(B, H, W, h, d))
     inp["theta"] = inp["theta"] * 3.0
     r = oracle.full(inp["q"], inp["k"], inp["v"], inp["theta"], M, s, dout=inp["dout"])

@@ -149,6 +149,16 @@ fs_status fs_winattn_fwd(const fs_winattn_shape* shape, const void* q, const voi
     unsigned int* status = nullptr;
     int sms = 0;
     if ((st = device_state(&status, &sms)) != FS_OK) return st;
+    if (g.d == 64) {  // heads of 64 channels: the wide kernels (no tensor maps)
+        unsigned long long lim;
+        {
+            std::lock_guard<std::mutex> lk(g_mu);
+            lim = g_limit_ns;
+        }
+        const cudaError_t e = launch_wide_fwd(g, q, k, v, theta, o, lse, status, lim, sms,
+                                              reinterpret_cast<cudaStream_t>(stream));
+        return e == cudaSuccess ? FS_OK : FS_ERR_CUDA;
+    }
     CUtensorMap mq, mk, mv, mo;
     if (encode_box_map(&mq, q, g) || encode_box_map(&mk, k, g) || encode_box_map(&mv, v, g) ||
         encode_box_map(&mo, o, g))
@@ -170,7 +180,7 @@ fs_status fs_winattn_block_fwd(const fs_winattn_shape* shape, const void* x, con
     Geo g;
     fs_status st = make_geo(shape, &g);
     if (st != FS_OK) return st;
-    if (g.N >= kTile || g.heads > 3) return FS_ERR_SHAPE;  // windows inside one tile, C <= 96
+    if (g.N >= kTile || g.heads > 3 || g.d != 32) return FS_ERR_SHAPE;  // windows inside one tile, C <= 96
     if (g.B == 0) return FS_OK;
     if (!x || !w_qkv || !b_qkv || !w_o || !b_o || !theta || !y) return FS_ERR_NULL;
     if (!aligned16(x) || !aligned16(w_qkv) || !aligned16(w_o) || !aligned16(y) ||
@@ -193,7 +203,7 @@ fs_status fs_winattn_block_fwd(const fs_winattn_shape* shape, const void* x, con
 size_t fs_winattn_bwd_workspace_bytes(const fs_winattn_shape* shape) {
     Geo g;
     if (make_geo(shape, &g) != FS_OK) return 0;
-    return bwd_workspace_bytes(g);
+    return g.d == 64 ? wide_bwd_workspace_bytes(g) : bwd_workspace_bytes(g);
 }
 
 fs_status fs_winattn_bwd(const fs_winattn_shape* shape, const void* q, const void* k, const void* v,
@@ -209,7 +219,7 @@ fs_status fs_winattn_bwd(const fs_winattn_shape* shape, const void* q, const voi
     if (g.B == 0) {
         // Empty batch: gradients of theta are zero.
         if ((st = device_state(&status, &sms)) != FS_OK) return st;
-        const int n = g.heads * 2 * (kHeadDim / 4);
+        const int n = g.heads * 2 * (g.d / 4);
         zero_f32_kernel<<<(n + 255) / 256, 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(dtheta, n);
         return cudaGetLastError() == cudaSuccess ? FS_OK : FS_ERR_CUDA;
     }
@@ -218,9 +228,20 @@ fs_status fs_winattn_bwd(const fs_winattn_shape* shape, const void* q, const voi
         !aligned16(dk) || !aligned16(dv) || (reinterpret_cast<uintptr_t>(lse) & 3u) ||
         (reinterpret_cast<uintptr_t>(theta) & 3u) || (reinterpret_cast<uintptr_t>(dtheta) & 3u))
         return FS_ERR_ALIGN;
-    if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) || workspace_bytes < bwd_workspace_bytes(g))
+    const size_t need = g.d == 64 ? wide_bwd_workspace_bytes(g) : bwd_workspace_bytes(g);
+    if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) || workspace_bytes < need)
         return FS_ERR_WORKSPACE;
     if ((st = device_state(&status, &sms)) != FS_OK) return st;
+    if (g.d == 64) {  // heads of 64 channels: the wide kernels
+        unsigned long long lim;
+        {
+            std::lock_guard<std::mutex> lk(g_mu);
+            lim = g_limit_ns;
+        }
+        BwdPtrs p{q, k, v, o, dout, lse, theta, dq, dk, dv, dtheta, static_cast<uint8_t*>(workspace)};
+        const cudaError_t e = launch_wide_bwd(g, p, status, lim, sms, reinterpret_cast<cudaStream_t>(stream));
+        return e == cudaSuccess ? FS_OK : FS_ERR_CUDA;
+    }
     BwdMaps maps;
     if (encode_box_map(&maps.q, q, g) || encode_box_map(&maps.k, k, g) || encode_box_map(&maps.v, v, g) ||
         encode_box_map(&maps.o, o, g) || encode_box_map(&maps.dout, dout, g) || encode_box_map(&maps.dq, dq, g) ||

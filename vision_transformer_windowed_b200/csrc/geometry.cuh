@@ -54,7 +54,7 @@ __host__ __device__ inline uint32_t fdiv(const FastDiv& f, uint32_t n) {
 }
 
 constexpr int kTile = 128;                  // token rows per tile
-constexpr int kHeadDim = 32;                // supported head dimension
+constexpr int kHeadDim = 32;                // channels of one tile row (a d = 64 head takes two)
 constexpr int kRowBytes = kHeadDim * 2;     // one 16-bit token row
 constexpr int kTileBytes = kTile * kRowBytes;
 
@@ -73,6 +73,7 @@ struct Geo {
     long long tiles;    // tiles per head
     float scale_log2;   // log2(e) / sqrt(d)
     FastDiv fd_nW, fd_nWw, fd_tiles, fd_heads;  // window, tile and item indices fit 32 bits
+    int d;              // head dimension: 32, or 64 (the wide kernels)
 };
 
 __host__ __device__ inline int ilog2_exact(int x) {
@@ -84,7 +85,7 @@ __host__ __device__ inline int ilog2_exact(int x) {
 // Builds the geometry of a problem.  Returns 0 on success, 2 for an
 // unsupported shape (the FS_ERR_SHAPE code of the C ABI).
 inline int geo_init(Geo* g, int B, int H, int W, int heads, int d, int M, int s) {
-    if (d != kHeadDim) return 2;
+    if (d != 32 && d != 64) return 2;
     if (!(M == 4 || M == 8 || M == 16 || M == 32 || M == 64)) return 2;
     if (B < 0 || heads < 1 || H < M || W < M) return 2;
     if (s < 0 || s >= M || s % 4) return 2;
@@ -107,6 +108,7 @@ inline int geo_init(Geo* g, int B, int H, int W, int heads, int d, int M, int s)
     x.Hp = Hp;
     x.Wp = Wp;
     x.heads = heads;
+    x.d = d;
     x.M = M;
     x.s = s;
     x.nWw = Wp / M;
@@ -130,7 +132,7 @@ inline int geo_init(Geo* g, int B, int H, int W, int heads, int d, int M, int s)
     x.lwpt = x.wpt ? ilog2_exact(x.wpt) : 0;
     x.wins = static_cast<long long>(B) * x.nW;
     x.tiles = (x.wins * x.N + kTile - 1) / kTile;
-    x.scale_log2 = 1.4426950408889634f / 5.656854249492380195f;  // log2(e) / sqrt(32)
+    x.scale_log2 = 1.4426950408889634f / (d == 64 ? 8.0f : 5.656854249492380195f);  // log2(e) / sqrt(d)
     x.fd_nW = make_fastdiv(static_cast<uint32_t>(x.nW));
     x.fd_nWw = make_fastdiv(static_cast<uint32_t>(x.nWw));
     x.fd_tiles = make_fastdiv(static_cast<uint32_t>(x.tiles > 0 ? x.tiles : 1));

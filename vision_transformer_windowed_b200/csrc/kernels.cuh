@@ -79,6 +79,23 @@ cudaError_t launch_small_fwd(const Geo& g, const void* q, const void* k, const v
                              float* lse, unsigned int* status, unsigned long long limit_ns, int num_sms,
                              cudaStream_t stream);
 
+// Heads of d = 64 channels, every window size (plain one-tile pipelines).  The
+// backward's workspace holds an fp32 dQ' accumulator of 256 bytes per
+// token-head row and the d theta partials.
+size_t wide_bwd_workspace_bytes(const Geo& g);
+cudaError_t launch_wide_fwd(const Geo& g, const void* q, const void* k, const void* v, const float* theta, void* o,
+                            float* lse, unsigned int* status, unsigned long long limit_ns, int num_sms,
+                            cudaStream_t stream);
+cudaError_t launch_wide_bwd(const Geo& g, const BwdPtrs& p, unsigned int* status, unsigned long long limit_ns,
+                            int num_sms, cudaStream_t stream);
+
+// Fixed-order d theta sum: part [heads][per_head][16] -> dtheta [heads][16] (one
+// launch; cnt: heads counters that are zero when it starts).
+namespace bwdk {
+cudaError_t launch_dtheta(const float* part, long long per_head, int heads, float* scratch, unsigned int* cnt,
+                          float* dtheta, cudaStream_t stream);
+}
+
 // The attention block with its projections (inference), windows of fewer than
 // 128 tokens, at most three heads: y = attention(x W_qkv^T + b_qkv) W_o^T + b_o.
 struct BlockPtrs {
