@@ -57,6 +57,9 @@ WORKLOADS = {
     # padded with zero tokens (200 x 336 at window 8; 224 x 352 at window 32), batch 16
     "swin_t_det_stage1_p4_m8": dict(B=16, H=200, W=334, heads=3, M=8, shifts=(0, 4), qk_scale=1.0),
     "flashswin_t_det_stage1_p4_m32": dict(B=16, H=200, W=334, heads=3, M=32, shifts=(0, 16), qk_scale=1.0),
+    # heads of 64 channels (the wide kernels): the FlashSwin-T stage-1 grid at p=2 with 3 heads of d=64,
+    # window 32, shifted block; batch 64 keeps each tensor at the size of the d=32 workload's
+    "flashswin_stage1_p2_m32_d64": dict(B=64, H=128, W=128, heads=3, M=32, shifts=(16,), qk_scale=1.0, d=64),
 }
 HEADLINE = "flashswin_t_p2_4stage"
 SPEC_BF16_TFLOPS = 2250.0  # NVIDIA's dense bf16 figure for one B200: a spec value, not a measurement
@@ -138,11 +141,13 @@ def measured_traffic(phase: str, workload: str):
 
 
 def stages_of(wl) -> list:
-    """A workload as a list of stages: one grid shape each, with the shifts of its blocks."""
+    """A workload as a list of stages: one grid shape each, with the shifts of its blocks (and its
+    head dimension, 32 unless given)."""
     if "stages" in wl:
-        return [dict(st, qk_scale=st.get("qk_scale", wl.get("qk_scale", 1.0)), infer=wl.get("infer", False))
+        return [dict(st, qk_scale=st.get("qk_scale", wl.get("qk_scale", 1.0)), infer=wl.get("infer", False),
+                     d=st.get("d", wl.get("d", HEAD_DIM)))
                 for st in wl["stages"]]
-    return [wl]
+    return [dict(wl, d=wl.get("d", HEAD_DIM))]
 
 
 def blocks_of(wl) -> list:
@@ -152,8 +157,9 @@ def blocks_of(wl) -> list:
 
 def workload_flops(wl) -> tuple[float, float]:
     """Useful forward and backward FLOPs of one step (fwd 4*d per pair, bwd 10*d per pair)."""
-    pairs = sum(unmasked_pairs(st["B"], st["H"], st["W"], st["heads"], st["M"], s) for st, s in blocks_of(wl))
-    return 4.0 * HEAD_DIM * pairs, 10.0 * HEAD_DIM * pairs
+    dpairs = sum(st["d"] * unmasked_pairs(st["B"], st["H"], st["W"], st["heads"], st["M"], s)
+                 for st, s in blocks_of(wl))
+    return 4.0 * dpairs, 10.0 * dpairs
 
 
 def workload_tokens(wl) -> int:
@@ -172,15 +178,21 @@ def phase_work(st, s) -> dict:
     the zeroed dQ' accumulator out, 588 B, and the per-window scale pass over lse2, 8 B, timed with
     it; main: the images, dO, v, lse2, D in, dk, dv out, 392 B; post: the dQ' accumulator and q in, dq
     out, 256 B)."""
-    B, H, W, heads, M = st["B"], st["H"], st["W"], st["heads"], st["M"]
+    B, H, W, heads, M, d = st["B"], st["H"], st["W"], st["heads"], st["M"], st.get("d", HEAD_DIM)
     rows = B * H * W * heads
     pairs = unmasked_pairs(B, H, W, heads, M, s)
     small = M * M < 128
-    nbytes = {"fwd": (256 if st.get("infer") else 260) * rows, "bwd_prep": 0 if small else 596 * rows,
-              "bwd_main": (520 if small else 392) * rows, "bwd_post": 0 if small else 256 * rows,
-              "bwd_dtheta": 0}
-    flops = {"fwd": 4.0 * HEAD_DIM * pairs, "bwd_main": 10.0 * HEAD_DIM * pairs}
-    return {"bytes": nbytes, "flops": flops, "hbm_bound": small}
+    if d == 64:  # the wide kernels: prep reads dO, v and zeroes the fp32 dQ' accumulator; main reads
+        # q, k, v, o, dO and lse, writes dk, dv (the dQ' additions resolve in L2); post reads the
+        # accumulator and q, writes dq
+        nbytes = {"fwd": (512 if st.get("infer") else 516) * rows, "bwd_prep": 512 * rows,
+                  "bwd_main": 900 * rows, "bwd_post": 512 * rows, "bwd_dtheta": 0}
+    else:
+        nbytes = {"fwd": (256 if st.get("infer") else 260) * rows, "bwd_prep": 0 if small else 596 * rows,
+                  "bwd_main": (520 if small else 392) * rows, "bwd_post": 0 if small else 256 * rows,
+                  "bwd_dtheta": 0}
+    flops = {"fwd": 4.0 * d * pairs, "bwd_main": 10.0 * d * pairs}
+    return {"bytes": nbytes, "flops": flops, "hbm_bound": small and d == 32}
 
 
 def mufu_ceiling_tflops(flops_per_exp: float, sm_mhz: float, sms: int = 148) -> float:
@@ -217,7 +229,7 @@ def roofline(wl, res, peaks, sm_mhz=None) -> dict:
                 "frac": achieved / peak, "frac_of_burst": achieved / peaks["bf16_tflops"], "traffic": None,
                 "algorithmic_flops_per_step": fl, "algorithmic_bytes_per_step": sum(w["bytes"][dom] for w in work),
                 "peak_note": f"cuBLAS bf16 sustained (burst {peaks['bf16_tflops']:.1f}), {peaks['source']}"}
-        per_exp = (4.0 if dom == "fwd" else 10.0) * HEAD_DIM
+        per_exp = (4.0 if dom == "fwd" else 10.0) * blocks[0][0]["d"]
         mhz = sm_mhz or 1965.0
         roof["mufu_ceiling_tflops"] = mufu_ceiling_tflops(per_exp, mhz)
         roof["mufu_note"] = (f"one MUFU exp2 per score element: 16/clk/SM x 148 SMs x {mhz:.0f} MHz x "
@@ -327,7 +339,7 @@ def cpu_baseline(tensors, wl, seconds: float = 12.0):
             oracle.units(t["q"], t["k"], t["v"], t["theta"], M, s, ids, dout=t["dout"], nthreads=cores)
             dt = time.perf_counter() - t0
             # useful flops of the sampled units (pairs that attend)
-            flops += 14.0 * HEAD_DIM * unmasked_pairs(B, H, W, heads, M, s) * (n / n_units)
+            flops += 14.0 * st.get("d", HEAD_DIM) * unmasked_pairs(B, H, W, heads, M, s) * (n / n_units)
             total_dt += dt
             done += n
             full_s += dt * n_units / n
@@ -347,6 +359,7 @@ def config_entry(wl, r, peaks, world, name=None) -> dict:
     blocks = blocks_of(wl)
     fwd_ms = r["phase_ms"]["fwd"] * len(blocks)  # per step
     infer = wl.get("infer", False)
+    row_bytes = {32: (256 if infer else 260), 64: (512 if infer else 516)}
     e = {"tflops": r["tflops"], "ms_per_step": r["ms"],
          "pct_bf16_peak": 100 * r["tflops"] / peaks["bf16_tflops"] / world,
          "pct_bf16_spec": 100 * r["tflops"] / SPEC_BF16_TFLOPS / world,
@@ -354,8 +367,8 @@ def config_entry(wl, r, peaks, world, name=None) -> dict:
          "tokens_per_s": r["tokens_per_s"], "peak_gb": r["peak_gb"], "phase_ms": r["phase_ms"]}
     e["fwd_pct_bf16_peak"] = 100 * e["fwd_tflops"] / peaks["bf16_tflops"] / world
     # q, k, v read and o written (bf16), plus the fp32 lse of a training forward
-    rows = sum(st["B"] * st["H"] * st["W"] * st["heads"] for st, _ in blocks)
-    e["fwd_gbs"] = (256 if infer else 260) * rows / (fwd_ms * 1e-3) / 1e9
+    e["fwd_gbs"] = sum(row_bytes[st["d"]] * st["B"] * st["H"] * st["W"] * st["heads"] for st, _ in blocks) / (
+        fwd_ms * 1e-3) / 1e9
     if infer:
         e["step"] = "inference forward (no LSE) at every shift"
     else:
@@ -426,7 +439,7 @@ def workload_config(name, wl, world) -> dict:
     def shape(st):
         return {"B_per_gpu": st["B"], "H": st["H"], "W": st["W"], "heads": st["heads"], "M": st["M"],
                 "shifts": list(st["shifts"])}
-    cfg = {"workload": name, "d": HEAD_DIM}
+    cfg = {"workload": name, "d": stages_of(wl)[0]["d"]}
     if "stages" in wl:
         cfg["stages"] = [shape(st) for st in stages_of(wl)]
     else:
@@ -445,7 +458,7 @@ def run_reference(args):
 
     from vision_transformer_windowed_b200.inputs import make_inputs
     wl = WORKLOADS[args.workload]
-    t = [make_inputs(st["B"], st["H"], st["W"], st["heads"], HEAD_DIM, device="cpu", qk_scale=st["qk_scale"])
+    t = [make_inputs(st["B"], st["H"], st["W"], st["heads"], st["d"], device="cpu", qk_scale=st["qk_scale"])
          for st in stages_of(wl)]
     per_step = max(1.0, args.reference_seconds / max(1, args.steps + args.warmup))
     for _ in range(args.warmup):
@@ -520,7 +533,7 @@ def main():
         data = []
         for st in stages_of(wl):
             B, H, W, heads, M = st["B"], st["H"], st["W"], st["heads"], st["M"]
-            t = dp.rank_inputs(B, H, W, heads, HEAD_DIM, rank, dev, qk_scale=st["qk_scale"])
+            t = dp.rank_inputs(B, H, W, heads, st["d"], rank, dev, qk_scale=st["qk_scale"])
             blocks = []
             for s in st["shifts"]:
                 o = torch.empty_like(t["q"])
@@ -618,44 +631,75 @@ def main():
     roof = roofline(wl, main_res, peaks, sm_mhz)
     roof["traffic"] = measured_traffic(roof["kernel"], args.workload)  # bytes per step, like "achieved"
 
-    # end to end through the public API with host buffers (pinned), copies inside the timed region
+    # End to end through the public API with host buffers (pinned), copies inside the timed
+    # region.  e2e: every block's inputs (q, k, v, dO, theta) come from pinned host memory on a
+    # copy stream, a stage's compute waits only for its own inputs (so the next stage's upload
+    # overlaps the current stage's kernels), and each block's d theta (the parameter gradient, the
+    # step's result for an optimizer) is read back; O, dQ, dK, dV stay on the device, as they do
+    # inside a model.  e2e_all_outputs: the same with O, dQ, dK, dV and d theta all read back and
+    # every copy on the compute stream.
     host = [{k: t[k].cpu().pin_memory() for k in ("q", "k", "v", "dout", "theta")} for _, t, _, _ in main_res["data"]]
     res_host = {}
     e2e_steps = max(1, min(args.steps, 5))
     torch.cuda.synchronize()
     h2d = sum(x.numel() * x.element_size() for hs in host for x in hs.values())
-    d2h = 0
+    copy_stream = torch.cuda.Stream(device=dev)
+    d2h = {"result": 0, "all": 0}
 
-    def e2e_step():
-        nonlocal d2h
-        d2h = 0
-        for si, (st, hs) in enumerate(zip(stages_of(wl), host)):
+    def e2e_step(read_all: bool):
+        main = torch.cuda.current_stream(dev)
+        nbytes = 0
+        staged = []
+        if read_all:
+            staged = [({k: x.to(dev, non_blocking=True) for k, x in hs.items()}, None) for hs in host]
+        else:
+            with torch.cuda.stream(copy_stream):
+                for hs in host:
+                    dvi = {k: x.to(dev, non_blocking=True) for k, x in hs.items()}
+                    ev = torch.cuda.Event()
+                    ev.record(copy_stream)
+                    staged.append((dvi, ev))
+        for si, (st, (dvi, ev)) in enumerate(zip(stages_of(wl), staged)):
+            if ev is not None:
+                main.wait_event(ev)
+                for x in dvi.values():
+                    x.record_stream(main)  # allocated on the copy stream, used on this one
             M = st["M"]
-            dv = {k: x.to(dev, non_blocking=True) for k, x in hs.items()}
             for bi, s in enumerate(st["shifts"]):
-                o, lse = ops.winattn_fwd(dv["q"], dv["k"], dv["v"], dv["theta"], M, s)
-                dq, dk, dvv, dth = ops.winattn_bwd(dv["q"], dv["k"], dv["v"], o, dv["dout"], lse, dv["theta"], M, s)
+                o, lse = ops.winattn_fwd(dvi["q"], dvi["k"], dvi["v"], dvi["theta"], M, s)
+                dq, dk, dvv, dth = ops.winattn_bwd(dvi["q"], dvi["k"], dvi["v"], o, dvi["dout"], lse, dvi["theta"], M, s)
                 dp.allreduce_dtheta(dth)
-                for name, x in (("o", o), ("dq", dq), ("dk", dk), ("dv", dvv), ("dtheta", dth)):
+                outs = (("o", o), ("dq", dq), ("dk", dk), ("dv", dvv), ("dtheta", dth)) if read_all else (("dtheta", dth),)
+                for name, x in outs:
                     key = (si, bi, name)
                     if key not in res_host:
                         res_host[key] = torch.empty(x.shape, dtype=x.dtype, pin_memory=True)
                     res_host[key].copy_(x, non_blocking=True)
-                    d2h += x.numel() * x.element_size()
+                    nbytes += x.numel() * x.element_size()
+        d2h["all" if read_all else "result"] = nbytes
 
-    e2e_step()
-    torch.cuda.synchronize()
-    barrier()
-    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    a.record()
-    for _ in range(e2e_steps):
-        e2e_step()
-    b.record()
-    torch.cuda.synchronize()
-    e2e_ms = dp.max_over_ranks(a.elapsed_time(b) / e2e_steps, dev)
+    def e2e_time(read_all: bool) -> float:
+        e2e_step(read_all)
+        torch.cuda.synchronize()
+        barrier()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        for _ in range(e2e_steps):
+            e2e_step(read_all)
+        b.record()
+        torch.cuda.synchronize()
+        return dp.max_over_ranks(a.elapsed_time(b) / e2e_steps, dev)
+
     fl = main_res["fwd_flops"] + main_res["bwd_flops"]
+    e2e_ms = e2e_time(False)
     e2e = {"value": fl * world / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s", "ms_per_step": e2e_ms,
-           "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+           "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h["result"],
+           "step": "inputs from pinned host memory (uploads overlapped with the previous stage's kernels), "
+                   "d theta of every block read back"}
+    e2e_all_ms = e2e_time(True)
+    e2e_all = {"value": fl * world / (e2e_all_ms * 1e-3) / 1e12, "unit": "TFLOP/s", "ms_per_step": e2e_all_ms,
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h["all"],
+               "step": "inputs from pinned host memory; O, dQ, dK, dV and d theta of every block read back; one stream"}
 
     per_config = {args.workload: config_entry(wl, main_res, peaks, world, args.workload)}
     del main_res["data"], host, res_host
@@ -675,13 +719,13 @@ def main():
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        tt = [make_inputs(st["B"], st["H"], st["W"], st["heads"], HEAD_DIM, device="cpu", qk_scale=st["qk_scale"])
+        tt = [make_inputs(st["B"], st["H"], st["W"], st["heads"], st["d"], device="cpu", qk_scale=st["qk_scale"])
               for st in stages_of(wl)]
         cpu = cpu_baseline(tt, wl)
         cpu.pop("seconds", None)
 
     if rank == 0:
-        nlaunch = sum(1 + (2 if st["M"] * st["M"] < 128 else 5) for st, _ in blocks)
+        nlaunch = sum(1 + (4 if st["d"] == 64 else (2 if st["M"] * st["M"] < 128 else 5)) for st, _ in blocks)
         line = {
             "metric": METRIC, "value": main_res["tflops"], "unit": "TFLOP/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": main_res["ms"], "higher_is_better": True,
@@ -693,7 +737,7 @@ def main():
             # per block: the forward, then the one-tile backward and the d theta sum (windows
             # inside one tile) or prep, scale, main, post and the d theta sum
             "gpu_launches": args.steps * nlaunch,
-            "roofline": roof, "clocks": main_res["clocks"], "e2e": e2e, "cpu_baseline": cpu,
+            "roofline": roof, "clocks": main_res["clocks"], "e2e": e2e, "e2e_all_outputs": e2e_all, "cpu_baseline": cpu,
             "per_config": per_config, "peaks": peaks,
         }
         a, b = per_config.get("highres_p2_m32"), per_config.get("highres_p2_m64")

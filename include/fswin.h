@@ -12,7 +12,7 @@
  *
  * Conventions (readings of the paper where it is silent):
  *  - tensors q, k, v, o, dout, dq, dk, dv are bf16, contiguous [B, H, W, heads, d]
- *    (d = 32), 16-byte aligned, in DEVICE memory;
+ *    (d = 32 or 64), 16-byte aligned, in DEVICE memory;
  *  - theta and dtheta are fp32 [heads, 2, d/4]; axis 0 (x) rotates channel pairs
  *    (2k, 2k+1) of the first d/2 channels by j * theta[h][0][k], axis 1 (y) the pairs
  *    of the last d/2 channels by i * theta[h][1][k], where (i, j) is the token's
@@ -72,11 +72,14 @@ typedef enum {
 } fs_status;
 
 /*
- * Problem shape.  Supported: d == 32; M in {4, 8, 16, 32, 64}; H >= M and W >= M
+ * Problem shape.  Supported: d == 32 or d == 64; M in {4, 8, 16, 32, 64}; H >= M and W >= M
  * (not necessarily multiples of M: the grid is then padded, see above; a grid
  * smaller than the window is the caller's to clamp, as Swin clamps the window);
  * 0 <= s < M with s a multiple of 4; heads >= 1; B >= 0 (B == 0 is a valid empty
  * problem).  Anything else returns FS_ERR_SHAPE.
+ * Heads of d = 64 (16 RoPE pairs per axis) run their own kernels, plain
+ * one-tile pipelines; their backward's workspace holds an fp32 dQ accumulator
+ * (256 bytes per token-head) besides the d theta partials.
  */
 typedef struct {
     int B, H, W, heads, d, M, s;
@@ -108,7 +111,7 @@ FS_API fs_status fs_winattn_fwd(const fs_winattn_shape* shape, const void* q, co
  *   y = o W_o^T + b_o, o taken as [B,H,W,C].
  * In: x bf16 [B,H,W,C] with C = heads * d; w_qkv bf16 [3C, C] (output channels
  * q of every head, then k, then v); b_qkv fp32 [3C]; w_o bf16 [C, C]; b_o
- * fp32 [C]; theta fp32 [heads,2,d/4].  Out: y bf16 [B,H,W,C], overwritten.
+ * fp32 [C]; theta fp32 [heads,2,d/4].  Out: y bf16 [B,H,W,C], overwritten.  d == 32 only.
  * q, k, v and o never reach device memory.  Supported: the shapes of
  * fs_winattn_check_shape with M*M < 128 (windows inside one 128-token tile)
  * and heads <= 3; anything else returns FS_ERR_SHAPE.  On a padded grid (H or W

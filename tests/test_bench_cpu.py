@@ -104,3 +104,13 @@ def test_cpu_baseline_samples_every_stage():
     assert "8 of 8 at 16x16/M=8 s=0" in res["sample"] and "8 of 8 at 16x16/M=8 s=4" in res["sample"]
     assert "1 of 1 at 16x16/M=16 s=0" in res["sample"]
     assert res["units_per_s"] == pytest.approx(17 / res["seconds"])
+
+
+def test_flops_and_bytes_scale_with_the_head_dimension():
+    wl = dict(B=1, H=16, W=16, heads=2, M=8, shifts=(4,), qk_scale=1.0, d=64)
+    pairs = _brute_pairs(1, 16, 16, 2, 8, 4)
+    fwd, bwd = bench.workload_flops(wl)
+    assert fwd == 4 * 64 * pairs and bwd == 10 * 64 * pairs
+    w = bench.phase_work(bench.stages_of(wl)[0], 4)
+    assert w["flops"]["bwd_main"] == 10 * 64 * pairs and not w["hbm_bound"]
+    assert w["bytes"]["fwd"] == 516 * 16 * 16 * 2

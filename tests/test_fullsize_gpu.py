@@ -70,12 +70,28 @@ def _sample_units(B, H, W, heads, M, n_random=6, seed=7):
     return np.array(sorted(set(units)), dtype=np.int64)
 
 
+# heads of 64 channels (the wide kernels) at the benchmark's d = 64 workload and a
+# detection-sized padded grid: (name, B, H, W, heads, M, s, qk_scale)
+FULL64 = [
+    ("flashswin_stage1_p2_m32_d64", 64, 128, 128, 3, 32, 16, 1.0),
+    ("det_stage1_p4_m8_d64_s4", 16, 200, 334, 3, 8, 4, 1.0),
+]
+
+
 @pytest.mark.gpu
 @pytest.mark.parametrize("cfg", FULL, ids=[c[0] for c in FULL])
 def test_full_size_sampled_windows(cfg):
-    name, B, H, W, heads, M, s, qk = cfg[:8]
-    dscale = cfg[8] if len(cfg) > 8 else 1.0
-    inp = make_inputs(B, H, W, heads, 32, qk_scale=qk)
+    _full_size(*cfg[:8], dscale=cfg[8] if len(cfg) > 8 else 1.0)
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("cfg", FULL64, ids=[c[0] for c in FULL64])
+def test_full_size_sampled_windows_d64(cfg):
+    _full_size(*cfg, d=64)
+
+
+def _full_size(name, B, H, W, heads, M, s, qk, dscale=1.0, d=32):
+    inp = make_inputs(B, H, W, heads, d, qk_scale=qk)
     units = _sample_units(B, H, W, heads, M)
     pos = []
     for u in units:  # real tokens of each unit, and their window-local slots
@@ -109,7 +125,7 @@ def test_full_size_sampled_windows(cfg):
     for key in ("dq", "dk", "dv"):
         _check(f"{name} {key}", cat(got[key]), cat(want[key]), GRAD_TOL)
     # dθ: only the sampled units carry dO, so the total is their sum
-    want_th = np.zeros((heads, 2, 8))
+    want_th = np.zeros((heads, 2, d // 4))
     for u, share in zip(units, ref["dtheta"]):
         want_th[int(u) % heads] += share
     _check(f"{name} dtheta", dth.float().cpu().numpy(), want_th, GRAD_TOL)

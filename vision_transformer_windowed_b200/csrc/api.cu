@@ -156,7 +156,8 @@ fs_status fs_winattn_fwd(const fs_winattn_shape* shape, const void* q, const voi
             lim = g_limit_ns;
         }
         const cudaError_t e = launch_wide_fwd(g, q, k, v, theta, o, lse, status, lim, sms,
-                                              reinterpret_cast<cudaStream_t>(stream));
+                                              reinterpret_cast<cudaStream_t>(stream),
+                                              g_phase_n >= 2 ? g_phase_events : nullptr);
         return e == cudaSuccess ? FS_OK : FS_ERR_CUDA;
     }
     CUtensorMap mq, mk, mv, mo;
@@ -239,7 +240,8 @@ fs_status fs_winattn_bwd(const fs_winattn_shape* shape, const void* q, const voi
             lim = g_limit_ns;
         }
         BwdPtrs p{q, k, v, o, dout, lse, theta, dq, dk, dv, dtheta, static_cast<uint8_t*>(workspace)};
-        const cudaError_t e = launch_wide_bwd(g, p, status, lim, sms, reinterpret_cast<cudaStream_t>(stream));
+        const cudaError_t e = launch_wide_bwd(g, p, status, lim, sms, reinterpret_cast<cudaStream_t>(stream),
+                                              g_phase_n >= 5 ? g_phase_events : nullptr);
         return e == cudaSuccess ? FS_OK : FS_ERR_CUDA;
     }
     BwdMaps maps;

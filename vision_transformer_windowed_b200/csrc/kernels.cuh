@@ -83,11 +83,14 @@ cudaError_t launch_small_fwd(const Geo& g, const void* q, const void* k, const v
 // backward's workspace holds an fp32 dQ' accumulator of 256 bytes per
 // token-head row and the d theta partials.
 size_t wide_bwd_workspace_bytes(const Geo& g);
+// events: NULL, or (forward) 2 events recorded before and after the kernel,
+// (backward) 5 events recorded before the first and after each of prep, main,
+// post and the d theta sum.
 cudaError_t launch_wide_fwd(const Geo& g, const void* q, const void* k, const void* v, const float* theta, void* o,
                             float* lse, unsigned int* status, unsigned long long limit_ns, int num_sms,
-                            cudaStream_t stream);
+                            cudaStream_t stream, cudaEvent_t const* events);
 cudaError_t launch_wide_bwd(const Geo& g, const BwdPtrs& p, unsigned int* status, unsigned long long limit_ns,
-                            int num_sms, cudaStream_t stream);
+                            int num_sms, cudaStream_t stream, cudaEvent_t const* events);
 
 // Fixed-order d theta sum: part [heads][per_head][16] -> dtheta [heads][16] (one
 // launch; cnt: heads counters that are zero when it starts).

@@ -140,6 +140,12 @@ __device__ __forceinline__ void bulk_reduce_add_f32(void* dst, const void* src, 
                  "r"(smem_u32(src)), "r"(bytes)
                  : "memory");
 }
+// p[0..3] += v (one 16-byte vector reduction in L2; p 16-byte aligned).
+__device__ __forceinline__ void red_add_v4(float* p, float a, float b, float c, float d) {
+    asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(reinterpret_cast<uint64_t>(p)), "f"(a), "f"(b),
+                 "f"(c), "f"(d)
+                 : "memory");
+}
 __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 __device__ __forceinline__ void bulk_wait_read_all() {
     asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");

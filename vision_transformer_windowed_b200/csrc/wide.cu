@@ -15,8 +15,9 @@
 //   backward: prep (per tile and head: the largest |dO row| and |v row| for the
 //             gradient scaling, zeroed dQ' accumulator), main (item = (key tile,
 //             head); the query tiles of its group in turn: S^T, dP^T, P'^T and
-//             dS'^T, dV and dK' accumulated in TMEM, dQ' reduce-added with fp32
-//             atomics; dk, dv and the key side of d theta at the item's end),
+//             dS'^T, dV and dK' accumulated in TMEM, dQ' added with 16-byte
+//             fp32 vector reductions; dk, dv and the key side of d theta at the
+//             item's end),
 //             post (dq and the query side of d theta), and the fixed-order
 //             d theta sum of the d = 32 backward.
 #include <cuda.h>
@@ -691,7 +692,9 @@ __global__ void __launch_bounds__(kThreads, 1) main_kernel(const __grid_constant
                     tmem_wait_ld();
                     if (qvalid) {
 #pragma unroll
-                        for (int e = 0; e < 32; ++e) atomicAdd(accrow + 32 * hf + e, __uint_as_float(v[e]) * sc);
+                        for (int e = 0; e < 32; e += 4)
+                            red_add_v4(accrow + 32 * hf + e, __uint_as_float(v[e]) * sc, __uint_as_float(v[e + 1]) * sc,
+                                       __uint_as_float(v[e + 2]) * sc, __uint_as_float(v[e + 3]) * sc);
                     }
                 }
             }
@@ -772,7 +775,13 @@ __global__ void __launch_bounds__(128) post_kernel(const Params p) {
         for (int hf = 0; hf < kHalves; ++hf) {
             float dx[32];
 #pragma unroll
-            for (int e = 0; e < 32; ++e) dx[e] = __ldcg(acc + 32 * hf + e);
+            for (int e = 0; e < 32; e += 4) {
+                const float4 a4 = *reinterpret_cast<const float4*>(acc + 32 * hf + e);
+                dx[e] = a4.x;
+                dx[e + 1] = a4.y;
+                dx[e + 2] = a4.z;
+                dx[e + 3] = a4.w;
+            }
             rope_half(dx, hf ? pi : pj, tab + hf * kPairs * 64, true);
             dtheta_terms(part, dx, hf ? q1 : q0, static_cast<float>(hf ? pi : pj), hf);
 #pragma unroll
@@ -790,7 +799,7 @@ size_t wide_bwd_workspace_bytes(const Geo& g) { return widek::bwd::ws_layout(g).
 
 cudaError_t launch_wide_fwd(const Geo& g, const void* q, const void* k, const void* v, const float* theta, void* o,
                             float* lse, unsigned int* status, unsigned long long limit_ns, int num_sms,
-                            cudaStream_t stream) {
+                            cudaStream_t stream, cudaEvent_t const* events) {
     using namespace widek;
     static SmemOptIn optin;
     if (cudaError_t e = optin.ensure(reinterpret_cast<const void*>(fwd::fwd_kernel), fwd::kSmemBytes)) return e;
@@ -807,12 +816,16 @@ cudaError_t launch_wide_fwd(const Geo& g, const void* q, const void* k, const vo
     prm.items = fwd_item_count(g);
     if (prm.items == 0) return cudaSuccess;
     const long long grid = prm.items < 2ll * num_sms ? prm.items : 2ll * num_sms;  // two CTAs per SM (TMEM)
+    cudaError_t e = events ? cudaEventRecord(events[0], stream) : cudaSuccess;
+    if (e != cudaSuccess) return e;
     fwd::fwd_kernel<<<static_cast<unsigned>(grid), fwd::kThreads, fwd::kSmemBytes, stream>>>(prm);
-    return cudaGetLastError();
+    e = cudaGetLastError();
+    if (e == cudaSuccess && events) e = cudaEventRecord(events[1], stream);
+    return e;
 }
 
 cudaError_t launch_wide_bwd(const Geo& g, const BwdPtrs& p, unsigned int* status, unsigned long long limit_ns,
-                            int num_sms, cudaStream_t stream) {
+                            int num_sms, cudaStream_t stream, cudaEvent_t const* events) {
     using namespace widek;
     static SmemOptIn optin;
     if (cudaError_t e = optin.ensure(reinterpret_cast<const void*>(bwd::main_kernel), bwd::kSmemBytes)) return e;
@@ -836,18 +849,28 @@ cudaError_t launch_wide_bwd(const Geo& g, const BwdPtrs& p, unsigned int* status
     prm.items = bwd_item_count(g);
     prm.scale = 0.125f;  // 1/sqrt(64)
     const long long ht = static_cast<long long>(g.heads) * g.tiles;
+    cudaError_t e = cudaSuccess;
+    auto mark = [&](int i) {
+        if (events && e == cudaSuccess) e = cudaEventRecord(events[i], stream);
+    };
+    mark(0);
     bwd::prep_kernel<<<static_cast<unsigned>(ht), 128, 0, stream>>>(prm);
-    cudaError_t e = cudaGetLastError();
-    if (e != cudaSuccess) return e;
+    if (e == cudaSuccess) e = cudaGetLastError();
+    mark(1);
     const long long grid = prm.items < num_sms ? prm.items : num_sms;
     bwd::main_kernel<<<static_cast<unsigned>(grid), bwd::kThreads, bwd::kSmemBytes, stream>>>(prm);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    if (e == cudaSuccess) e = cudaGetLastError();
+    mark(2);
     bwd::post_kernel<<<static_cast<unsigned>(ht), 128, 0, stream>>>(prm);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    if (e == cudaSuccess) e = cudaGetLastError();
+    mark(3);
     // d theta: [heads][2 axes] sums of [tiles * 8][16] partials, as heads * 2 rows of 16
-    return bwdk::launch_dtheta(reinterpret_cast<const float*>(p.ws + L.part), g.tiles * 8, 2 * g.heads,
-                         reinterpret_cast<float*>(p.ws + L.part2), reinterpret_cast<unsigned int*>(p.ws + L.cnt),
-                         p.dtheta, stream);
+    if (e == cudaSuccess)
+        e = bwdk::launch_dtheta(reinterpret_cast<const float*>(p.ws + L.part), g.tiles * 8, 2 * g.heads,
+                                reinterpret_cast<float*>(p.ws + L.part2), reinterpret_cast<unsigned int*>(p.ws + L.cnt),
+                                p.dtheta, stream);
+    mark(4);
+    return e;
 }
 
 }  // namespace fswin

@@ -8,7 +8,7 @@ Vision Transformers with Memory Efficient Attention", thelatestinai.com/papers/
 learnable 2D RoPE, the fused FlashAttention-style kernel replacing Swin's
 materialised score matrix.
 
-Shapes: q, k, v [B, H, W, heads, 32] bf16, with H >= M and W >= M.  H or W
+Shapes: q, k, v [B, H, W, heads, d] bf16 with d = 32 or 64, H >= M and W >= M.  H or W
 need not be a multiple of the window M: the grid is then worked on padded at
 the bottom and right with zero tokens to the next multiple (the Swin layer's
 padding), and only the H x W real tokens are read and written.
