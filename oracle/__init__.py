@@ -14,6 +14,12 @@ Two independent restatements of the same definition live here:
   the mask built from the Swin slice rule) and autograd for the gradients.  It
   exists to pin the C oracle, on tiny grids only.
 
+Both also take an optional low-rank additive bias (the FlashBias-T variant of
+the same pages: thelatestinai.com/papers/2610.04664, Table 2 and Table S1
+captions, a trainable rank-16 bias factorization): per head, factors U, W of
+shape [M*M, rank] over window-local positions t = i*M + j, and S_tu = scale
+q'_t.k'_u + U_t.W_u for every window.
+
 Both follow "FLASHSWIN: Unlocking Large Windows and Dense Tokens in Swin Vision
 Transformers with Memory Efficient Attention" (arxivdaily.com/papers/2610.04664,
 English abstract: exact softmax attention per M x M window, window-local
@@ -45,6 +51,10 @@ class _In(ctypes.Structure):
     _fields_ = [("p", ctypes.c_void_p), ("dtype", ctypes.c_int)]
 
 
+class _Bias(ctypes.Structure):
+    _fields_ = [("u", ctypes.c_void_p), ("w", ctypes.c_void_p), ("rank", ctypes.c_int)]
+
+
 _BF16, _F64 = 0, 1
 
 
@@ -66,9 +76,9 @@ def _load():
             lib = ctypes.CDLL(build())
             vp, P = ctypes.c_void_p, ctypes.POINTER(_Shape)
             lib.fso_units.restype = ctypes.c_int
-            lib.fso_units.argtypes = [P, _In, _In, _In, _In, vp, vp, ctypes.c_int64] + [vp] * 6 + [ctypes.c_int]
+            lib.fso_units.argtypes = [P, _In, _In, _In, _In, vp, _Bias, vp, ctypes.c_int64] + [vp] * 8 + [ctypes.c_int]
             lib.fso_full.restype = ctypes.c_int
-            lib.fso_full.argtypes = [P, _In, _In, _In, _In, vp] + [vp] * 6 + [ctypes.c_int]
+            lib.fso_full.argtypes = [P, _In, _In, _In, _In, vp, _Bias] + [vp] * 8 + [ctypes.c_int]
             lib.fso_labels.restype = ctypes.c_int
             lib.fso_labels.argtypes = [ctypes.c_int] * 4 + [vp]
             _lib = lib
@@ -117,6 +127,15 @@ def _dptr(a):
     return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
 
 
+def _bias_arg(bias, heads: int, N: int):
+    """(kept-alive arrays, _Bias) for optional factors (u, w), each [heads, N, rank]."""
+    if bias is None:
+        return (), _Bias(None, None, 0), 0
+    u, w = (_theta64(x) for x in bias)
+    assert u.ndim == 3 and u.shape == w.shape and u.shape[:2] == (heads, N), (u.shape, w.shape)
+    return (u, w), _Bias(u.ctypes.data, w.ctypes.data, u.shape[2]), u.shape[2]
+
+
 def labels(H: int, W: int, M: int, s: int) -> np.ndarray:
     """Region label of every rolled token, [H, W] (0 everywhere when s == 0)."""
     out = np.zeros((H, W), dtype=np.int32)
@@ -124,7 +143,7 @@ def labels(H: int, W: int, M: int, s: int) -> np.ndarray:
     return out
 
 
-def full(q, k, v, theta, M: int, s: int, dout=None, nthreads: int | None = None) -> dict:
+def full(q, k, v, theta, M: int, s: int, dout=None, nthreads: int | None = None, bias=None) -> dict:
     """Whole-tensor forward (and backward when ``dout`` is given).
 
     q, k, v, dout: [B, H, W, heads, d] (bf16 torch tensors or bit arrays are
@@ -133,7 +152,9 @@ def full(q, k, v, theta, M: int, s: int, dout=None, nthreads: int | None = None)
     and, with dout, dq, dk, dv and dtheta [heads, 2, d/4].  H or W that is not
     a multiple of M is padded with zero tokens up to the next multiple (the
     Swin layer's padding); the windows, the shift and its mask then refer to
-    the padded grid.
+    the padded grid.  ``bias = (u, w)``, each [heads, M*M, rank], adds the
+    low-rank bias u_t.w_u to every window's scores; the backward then also
+    returns du and dw [heads, M*M, rank].
     """
     qa, qi = _as_input(q)
     ka, ki = _as_input(k)
@@ -142,32 +163,39 @@ def full(q, k, v, theta, M: int, s: int, dout=None, nthreads: int | None = None)
     th = _theta64(theta)
     assert th.shape == (heads, 2, d // 4), th.shape
     sh = _Shape(B, H, W, heads, d, M, s)
+    keep, bi, rank = _bias_arg(bias, heads, M * M)
     o = np.zeros((B, H, W, heads, d))
     lse = np.zeros((B, H, W, heads))
     res = {"o": o, "lse": lse}
     di = _In(None, 0)
     da = None
-    grads = [None] * 4
+    grads = [None] * 6
     if dout is not None:
         da, di = _as_input(dout)
         grads = [np.zeros((B, H, W, heads, d)) for _ in range(3)] + [np.zeros((heads, 2, d // 4))]
         res.update(dq=grads[0], dk=grads[1], dv=grads[2], dtheta=grads[3])
-    st = _load().fso_full(ctypes.byref(sh), qi, ki, vi, di, _dptr(th), _dptr(o), _dptr(lse),
+        if rank:
+            grads += [np.zeros((heads, M * M, rank)) for _ in range(2)]
+            res.update(du=grads[4], dw=grads[5])
+        else:
+            grads += [None, None]
+    st = _load().fso_full(ctypes.byref(sh), qi, ki, vi, di, _dptr(th), bi, _dptr(o), _dptr(lse),
                           *[_dptr(g) for g in grads], int(nthreads or default_threads()))
     if st:
         raise ValueError(f"oracle rejected the problem (status {st})")
-    del qa, ka, va, da
+    del qa, ka, va, da, keep
     return res
 
 
-def units(q, k, v, theta, M: int, s: int, unit_ids, dout=None, nthreads: int | None = None) -> dict:
+def units(q, k, v, theta, M: int, s: int, unit_ids, dout=None, nthreads: int | None = None, bias=None) -> dict:
     """Forward (and backward with ``dout``) for selected (batch, window, head) units.
 
     unit = (b * nW + w) * heads + h, windows w = wr * (Wp/M) + wc in the rolled
     frame of the padded grid (Hp, Wp = H, W rounded up to multiples of M).
     Outputs are per unit in window-local token order t = i*M + j, padded tokens
     included:
-    o, dq, dk, dv [n, M*M, d]; lse [n, M*M]; dtheta [n, 2, d/4] (the unit's share).
+    o, dq, dk, dv [n, M*M, d]; lse [n, M*M]; dtheta [n, 2, d/4] (the unit's share);
+    with ``bias = (u, w)`` also du, dw [n, M*M, rank] (the unit's shares).
     """
     qa, qi = _as_input(q)
     ka, ki = _as_input(k)
@@ -178,22 +206,28 @@ def units(q, k, v, theta, M: int, s: int, unit_ids, dout=None, nthreads: int | N
     n = uid.shape[0]
     N = M * M
     sh = _Shape(B, H, W, heads, d, M, s)
+    keep, bi, rank = _bias_arg(bias, heads, N)
     o = np.zeros((n, N, d))
     lse = np.zeros((n, N))
     res = {"o": o, "lse": lse}
     di = _In(None, 0)
     da = None
-    grads = [None] * 4
+    grads = [None] * 6
     if dout is not None:
         da, di = _as_input(dout)
         grads = [np.zeros((n, N, d)) for _ in range(3)] + [np.zeros((n, 2, d // 4))]
         res.update(dq=grads[0], dk=grads[1], dv=grads[2], dtheta=grads[3])
-    st = _load().fso_units(ctypes.byref(sh), qi, ki, vi, di, _dptr(th), _dptr(uid), ctypes.c_int64(n),
+        if rank:
+            grads += [np.zeros((n, N, rank)) for _ in range(2)]
+            res.update(du=grads[4], dw=grads[5])
+        else:
+            grads += [None, None]
+    st = _load().fso_units(ctypes.byref(sh), qi, ki, vi, di, _dptr(th), bi, _dptr(uid), ctypes.c_int64(n),
                            _dptr(o), _dptr(lse), *[_dptr(g) for g in grads],
                            int(nthreads or default_threads()))
     if st:
         raise ValueError(f"oracle rejected the problem (status {st})")
-    del qa, ka, va, da
+    del qa, ka, va, da, keep
     return res
 
 

@@ -36,6 +36,18 @@
  *    and only the H x W real positions are written back.
  *
  * Gradients are those of L = sum(O * dO) for the upstream gradient dO.
+ *
+ * Optional low-rank additive bias (the FlashBias-T variant of the same pages:
+ * thelatestinai.com/papers/2610.04664, Table 2 and Table S1 captions, "a
+ * trainable rank-16 bias factorization" whose parameters grow with M).  Reading
+ * where the pages are silent: per head h the bias of the window's N x N
+ * (query position, key position) pairs is U_h W_h^T with U_h, W_h of shape
+ * [N][rank], N = M*M, positions t = i*M + j in the rolled frame, shared by every
+ * window of the batch like Swin's relative position bias; it is added to the
+ * scaled score before the shift mask, so S_tu = scale q'_t.k'_u + U_t.W_u.  Its
+ * gradients are dU_t = sum dS_tu W_u and dW_u = sum dS_tu U_t, summed over every
+ * window of the batch (padded tokens of a padded grid included, as in the
+ * softmax).
  */
 #include <math.h>
 #include <pthread.h>
@@ -106,13 +118,20 @@ static void rope_rotate(double* x, int d, int pos_x, int pos_y, const double* th
     }
 }
 
+/* Low-rank bias factors: u, w [heads][M*M][rank]; u == NULL: no bias. */
+typedef struct {
+    const double *u, *w;
+    int rank;
+} fso_bias;
+
 typedef struct {
     const fso_shape* sh;
     fso_in q, k, v, dout;
     const double* theta;
+    fso_bias bias;
     const int64_t* units;
     int64_t n_units;
-    double *o, *lse, *dq, *dk, *dv, *dth;
+    double *o, *lse, *dq, *dk, *dv, *dth, *du, *dw;
     int tid, nthreads;
     int status;
 } fso_job;
@@ -123,7 +142,7 @@ static int fso_padded(int X, int M) { return (X + M - 1) / M * M; }
 /* One (batch, window, head) unit.  Outputs are in window-local token order
  * t = i*M + j (padded tokens included). */
 static int fso_one_unit(const fso_job* jb, int64_t unit, double* o, double* lse, double* dq, double* dk,
-                        double* dv, double* dth) {
+                        double* dv, double* dth, double* du, double* dw) {
     const fso_shape* sh = jb->sh;
     const int H = sh->H, W = sh->W, heads = sh->heads, d = sh->d, M = sh->M, s = sh->s;
     const int Hp = fso_padded(H, M), Wp = fso_padded(W, M);
@@ -136,6 +155,9 @@ static int fso_one_unit(const fso_job* jb, int64_t unit, double* o, double* lse,
     const double* th = jb->theta + (int64_t)h * 2 * (d / 4);
     const double scale = 1.0 / sqrt((double)d);
     const int bwd = jb->dout.p != NULL && dq != NULL;
+    const int rank = jb->bias.u ? jb->bias.rank : 0;
+    const double* ub = rank ? jb->bias.u + (int64_t)h * N * rank : NULL; /* this head's factors */
+    const double* wb = rank ? jb->bias.w + (int64_t)h * N * rank : NULL;
 
     double* buf = (double*)calloc((size_t)N * d * 6 + (size_t)N * 3, sizeof(double));
     if (!buf) return 4;
@@ -144,6 +166,10 @@ static int fso_one_unit(const fso_job* jb, int64_t unit, double* o, double* lse,
     double *srow = dkr + (size_t)N * d, *prow = srow + N;
     int* lab = (int*)(prow + N);
     if (bwd) memset(dv, 0, sizeof(double) * (size_t)N * d);
+    if (bwd && rank) {
+        memset(du, 0, sizeof(double) * (size_t)N * rank);
+        memset(dw, 0, sizeof(double) * (size_t)N * rank);
+    }
 
     /* Step 1: roll and partition; step 2: rotate q and k. */
     for (int t = 0; t < N; ++t) {
@@ -172,9 +198,10 @@ static int fso_one_unit(const fso_job* jb, int64_t unit, double* o, double* lse,
                 srow[u] = -INFINITY;
                 continue;
             }
-            double acc = 0.0;
+            double acc = 0.0, bias = 0.0;
             for (int e = 0; e < d; ++e) acc += qr[(size_t)t * d + e] * kr[(size_t)u * d + e];
-            srow[u] = scale * acc;
+            for (int x = 0; x < rank; ++x) bias += ub[(size_t)t * rank + x] * wb[(size_t)u * rank + x];
+            srow[u] = scale * acc + bias;
             if (srow[u] > mx) mx = srow[u];
         }
         double sum = 0.0;
@@ -199,6 +226,10 @@ static int fso_one_unit(const fso_job* jb, int64_t unit, double* o, double* lse,
                 dqr[(size_t)t * d + e] += scale * ds * kr[(size_t)u * d + e];
                 dkr[(size_t)u * d + e] += scale * ds * qr[(size_t)t * d + e];
                 dv[(size_t)u * d + e] += prow[u] * go[(size_t)t * d + e];
+            }
+            for (int x = 0; x < rank; ++x) {
+                du[(size_t)t * rank + x] += ds * wb[(size_t)u * rank + x];
+                dw[(size_t)u * rank + x] += ds * ub[(size_t)t * rank + x];
             }
         }
     }
@@ -234,10 +265,12 @@ static void* fso_worker(void* arg) {
     fso_job* jb = (fso_job*)arg;
     const fso_shape* sh = jb->sh;
     const size_t N = (size_t)sh->M * sh->M, d = (size_t)sh->d, q = (size_t)sh->d / 4;
+    const size_t rk = jb->bias.u ? (size_t)jb->bias.rank : 0;
     for (int64_t n = jb->tid; n < jb->n_units; n += jb->nthreads) {
         int st = fso_one_unit(jb, jb->units[n], jb->o + n * N * d, jb->lse + n * N,
                               jb->dq ? jb->dq + n * N * d : NULL, jb->dk ? jb->dk + n * N * d : NULL,
-                              jb->dv ? jb->dv + n * N * d : NULL, jb->dth ? jb->dth + n * 2 * q : NULL);
+                              jb->dv ? jb->dv + n * N * d : NULL, jb->dth ? jb->dth + n * 2 * q : NULL,
+                              jb->du ? jb->du + n * N * rk : NULL, jb->dw ? jb->dw + n * N * rk : NULL);
         if (st) {
             jb->status = st;
             break;
@@ -251,19 +284,22 @@ static void* fso_worker(void* arg) {
  * of units.  unit = (b*nW + w)*heads + h with windows w = wr*(Wp/M) + wc in the
  * rolled frame of the padded grid.  Per unit outputs, window-local token order t = i*M + j:
  *   o, dq, dk, dv: [n_units][M*M][d];  lse: [n_units][M*M];
- *   dth: [n_units][2][d/4], this unit's share of d theta for its head.
+ *   dth: [n_units][2][d/4], this unit's share of d theta for its head;
+ *   du, dw: [n_units][M*M][rank], the unit's shares of the bias gradients (with a bias).
  */
 int fso_units(const fso_shape* sh, fso_in q, fso_in k, fso_in v, fso_in dout, const double* theta,
-              const int64_t* units, int64_t n_units, double* o, double* lse, double* dq, double* dk, double* dv,
-              double* dth, int nthreads) {
+              fso_bias bias, const int64_t* units, int64_t n_units, double* o, double* lse, double* dq, double* dk,
+              double* dv, double* dth, double* du, double* dw, int nthreads) {
     int st = fso_check_shape(sh);
     if (st) return st;
+    if (bias.u && (!bias.w || bias.rank < 1)) return 2;
+    if (bias.u && dq && (!du || !dw)) return 1;
     if (nthreads < 1) nthreads = 1;
     if (nthreads > 256) nthreads = 256;
     pthread_t tids[256];
     fso_job jobs[256];
     for (int t = 0; t < nthreads; ++t) {
-        fso_job jb = {sh, q, k, v, dout, theta, units, n_units, o, lse, dq, dk, dv, dth, t, nthreads, 0};
+        fso_job jb = {sh, q, k, v, dout, theta, bias, units, n_units, o, lse, dq, dk, dv, dth, du, dw, t, nthreads, 0};
         jobs[t] = jb;
     }
     if (nthreads == 1) {
@@ -281,22 +317,34 @@ int fso_units(const fso_shape* sh, fso_in q, fso_in k, fso_in v, fso_in dout, co
  * Whole-tensor forward/backward.  Outputs at original token positions (padded
  * tokens are dropped):
  *   o, dq, dk, dv: [B][H][W][heads][d];  lse: [B][H][W][heads];
- *   dtheta: [heads][2][d/4], summed over units in increasing unit order.
+ *   dtheta: [heads][2][d/4], summed over units in increasing unit order;
+ *   du, dw: [heads][M*M][rank] with a bias, summed over units in the same order.
  * Backward outputs may be NULL (forward only).
  */
-int fso_full(const fso_shape* sh, fso_in q, fso_in k, fso_in v, fso_in dout, const double* theta, double* o,
-             double* lse, double* dq, double* dk, double* dv, double* dtheta, int nthreads) {
+int fso_full(const fso_shape* sh, fso_in q, fso_in k, fso_in v, fso_in dout, const double* theta, fso_bias bias,
+             double* o, double* lse, double* dq, double* dk, double* dv, double* dtheta, double* du, double* dw,
+             int nthreads) {
     int st = fso_check_shape(sh);
     if (st) return st;
+    if (bias.u && (!bias.w || bias.rank < 1)) return 2;
     const int H = sh->H, W = sh->W, heads = sh->heads, d = sh->d, M = sh->M, s = sh->s;
     const int Hp = fso_padded(H, M), Wp = fso_padded(W, M);
     const int nWw = Wp / M, nW = (Hp / M) * nWw, N = M * M, qq = d / 4;
     const int64_t n_units = (int64_t)sh->B * nW * heads;
-    const int bwd = dout.p != NULL && dq && dk && dv && dtheta;
+    const int bwd = dout.p != NULL && dq && dk && dv && dtheta && (!bias.u || (du && dw));
+    const int rk = bias.u ? bias.rank : 0;
     int64_t* units = (int64_t*)malloc(sizeof(int64_t) * (size_t)(n_units > 0 ? n_units : 1));
     double* uo = (double*)calloc((size_t)(n_units > 0 ? n_units : 1) * N * d, sizeof(double));
     double* ul = (double*)calloc((size_t)(n_units > 0 ? n_units : 1) * N, sizeof(double));
-    double *udq = NULL, *udk = NULL, *udv = NULL, *uth = NULL;
+    double *udq = NULL, *udk = NULL, *udv = NULL, *uth = NULL, *udu = NULL, *udw = NULL;
+    if (bwd && rk) {
+        udu = (double*)calloc((size_t)(n_units > 0 ? n_units : 1) * N * rk, sizeof(double));
+        udw = (double*)calloc((size_t)(n_units > 0 ? n_units : 1) * N * rk, sizeof(double));
+        if (!udu || !udw) {
+            st = 4;
+            goto done;
+        }
+    }
     if (bwd) {
         udq = (double*)calloc((size_t)(n_units > 0 ? n_units : 1) * N * d, sizeof(double));
         udk = (double*)calloc((size_t)(n_units > 0 ? n_units : 1) * N * d, sizeof(double));
@@ -308,8 +356,8 @@ int fso_full(const fso_shape* sh, fso_in q, fso_in k, fso_in v, fso_in dout, con
         goto done;
     }
     for (int64_t n = 0; n < n_units; ++n) units[n] = n;
-    st = fso_units(sh, q, k, v, bwd ? dout : (fso_in){NULL, 0}, theta, units, n_units, uo, ul, udq, udk, udv,
-                   uth, nthreads);
+    st = fso_units(sh, q, k, v, bwd ? dout : (fso_in){NULL, 0}, theta, bias, units, n_units, uo, ul, udq, udk, udv,
+                   uth, udu, udw, nthreads);
     if (st) goto done;
     for (int64_t n = 0; n < n_units; ++n) {
         int64_t b = n / ((int64_t)nW * heads), rem = n % ((int64_t)nW * heads);
@@ -338,6 +386,16 @@ int fso_full(const fso_shape* sh, fso_in q, fso_in k, fso_in v, fso_in dout, con
             for (int x = 0; x < 2 * qq; ++x) dtheta[h * 2 * qq + x] += uth[(size_t)n * 2 * qq + x];
         }
     }
+    if (bwd && rk) {
+        for (int64_t x = 0; x < (int64_t)heads * N * rk; ++x) du[x] = dw[x] = 0.0;
+        for (int64_t n = 0; n < n_units; ++n) {
+            int h = (int)((n % ((int64_t)nW * heads)) % heads);
+            for (int64_t x = 0; x < (int64_t)N * rk; ++x) {
+                du[(int64_t)h * N * rk + x] += udu[(size_t)n * N * rk + x];
+                dw[(int64_t)h * N * rk + x] += udw[(size_t)n * N * rk + x];
+            }
+        }
+    }
 done:
     free(units);
     free(uo);
@@ -346,5 +404,7 @@ done:
     free(udk);
     free(udv);
     free(uth);
+    free(udu);
+    free(udw);
     return st;
 }

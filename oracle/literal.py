@@ -9,6 +9,11 @@ A grid that is not a multiple of M is zero-padded with
 ``torch.nn.functional.pad`` before the roll and cropped after it, as a Swin
 layer does.
 
+The optional low-rank bias (FlashBias-T, thelatestinai.com/papers/2610.04664,
+Table 2 and Table S1 captions) is the per-head matrix product U_h W_h^T over
+window-local positions, broadcast to every window and added to the scaled
+scores before the mask.
+
 Method: "FLASHSWIN ..." (arxivdaily.com/papers/2610.04664, English abstract:
 exact softmax attention inside each M x M window, window-local learnable 2D
 RoPE); the mask slices [0, H-M), [H-M, H-s), [H-s, H) are the Swin shifted-
@@ -65,8 +70,9 @@ def rope(x: torch.Tensor, theta: torch.Tensor, pos_i: torch.Tensor, pos_j: torch
     return torch.cat(out, dim=-1)
 
 
-def forward(q, k, v, theta, M: int, s: int):
-    """Returns (o [B,H,W,h,d], lse [B,H,W,h]) in float64."""
+def forward(q, k, v, theta, M: int, s: int, bias=None):
+    """Returns (o [B,H,W,h,d], lse [B,H,W,h]) in float64; bias = (u, w), each
+    [h, M*M, rank], adds u @ w^T to every window's scores."""
     B, H0, W0, h, d = q.shape
     H, W = -(-H0 // M) * M, -(-W0 // M) * M
     q, k, v = (F.pad(t, (0, 0, 0, 0, 0, W - W0, 0, H - H0)) for t in (q, k, v))
@@ -77,6 +83,8 @@ def forward(q, k, v, theta, M: int, s: int):
     qr = rope(qw, theta, pos_i, pos_j)
     kr = rope(kw, theta, pos_i, pos_j)
     scores = (qr @ kr.transpose(-1, -2)) / math.sqrt(d)          # [B,nh,nw,h,N,N]
+    if bias is not None:
+        scores = scores + bias[0] @ bias[1].transpose(-1, -2)     # [h,N,N] broadcast over windows
     lab = _windows(region_labels(H, W, M, s)[None, :, :, None, None], M)[..., 0]  # [1,nh,nw,1,N]
     allowed = lab[..., :, None] == lab[..., None, :]
     scores = scores.masked_fill(~allowed, float("-inf"))
@@ -87,10 +95,15 @@ def forward(q, k, v, theta, M: int, s: int):
     return o[:, :H0, :W0], lse[:, :H0, :W0]
 
 
-def forward_backward(q, k, v, theta, M: int, s: int, dout):
-    """Forward plus autograd gradients of sum(o * dout) w.r.t. q, k, v, theta."""
-    leaves = [t.detach().to(torch.float64).clone().requires_grad_(True) for t in (q, k, v, theta)]
-    o, lse = forward(*leaves, M, s)
+def forward_backward(q, k, v, theta, M: int, s: int, dout, bias=None):
+    """Forward plus autograd gradients of sum(o * dout) w.r.t. q, k, v, theta
+    (and the bias factors u, w when given)."""
+    tensors = (q, k, v, theta) + (tuple(bias) if bias is not None else ())
+    leaves = [torch.as_tensor(t).detach().to(torch.float64).clone().requires_grad_(True) for t in tensors]
+    o, lse = forward(*leaves[:4], M, s, bias=leaves[4:] if bias is not None else None)
     (o * dout.to(torch.float64)).sum().backward()
-    dq, dk, dv, dth = (t.grad for t in leaves)
-    return {"o": o.detach(), "lse": lse.detach(), "dq": dq, "dk": dk, "dv": dv, "dtheta": dth}
+    dq, dk, dv, dth = (t.grad for t in leaves[:4])
+    res = {"o": o.detach(), "lse": lse.detach(), "dq": dq, "dk": dk, "dv": dv, "dtheta": dth}
+    if bias is not None:
+        res.update(du=leaves[4].grad, dw=leaves[5].grad)
+    return res

@@ -17,6 +17,11 @@ For the attention block with its projections (Figure 1B): x bf16 N(0, 1) on a
 N(0, 1/C), the variance of a linear layer's initialisation, so that q, k, v
 are near N(0, 1) like the attention workloads' (seeds 6 and 8); b_qkv and b_o
 fp32 N(0, 0.02^2) (seeds 7 and 9); theta as above.
+
+For the low-rank additive bias (the FlashBias-T variant, Table 2 and Table S1:
+a trainable rank-16 bias factorization): factors U, W fp32 [heads, M*M, rank]
+drawn N(0, 0.5^2) (seeds 10 and 11), so that every bias entry U_t.W_u of rank
+16 has unit variance, the spread of the scores themselves.
 """
 from __future__ import annotations
 
@@ -24,6 +29,7 @@ import torch
 
 SEED_Q, SEED_K, SEED_V, SEED_DO, SEED_THETA = 0, 1, 2, 3, 4
 SEED_X, SEED_WQKV, SEED_BQKV, SEED_WO, SEED_BO = 5, 6, 7, 8, 9
+SEED_U, SEED_W = 10, 11
 
 
 def _normal(shape, seed: int, device, scale: float = 1.0) -> torch.Tensor:
@@ -81,3 +87,14 @@ def make_block_inputs(B: int, H: int, W: int, heads: int, d: int, device="cpu") 
         "b_o": draw((C,), SEED_BO, 0.02, torch.float32),
         "theta": theta_init(heads, d, device),
     }
+
+
+def make_bias(heads: int, M: int, rank: int = 16, device="cpu", std: float = 0.5) -> dict:
+    """Low-rank bias factors u, w: fp32 [heads, M*M, rank]."""
+
+    def draw(seed):
+        g = torch.Generator(device="cpu")
+        g.manual_seed(seed)
+        return (torch.randn((heads, M * M, rank), generator=g, dtype=torch.float32) * std).to(device)
+
+    return {"u": draw(SEED_U), "w": draw(SEED_W)}
