@@ -142,6 +142,41 @@ FS_API fs_status fs_winattn_bwd(const fs_winattn_shape* shape, const void* q, co
                          void* dk, void* dv, float* dtheta, void* workspace, size_t workspace_bytes,
                          fs_stream_t stream);
 
+/*
+ * Windowed attention with a low-rank additive bias (the FlashBias-T variant of
+ * the same pages: thelatestinai.com 2610.04664, Table 2 and Table S1 captions,
+ * a trainable rank-16 factorization of an additive attention bias whose
+ * parameters grow with M).  Reading where the pages are silent: per head h the
+ * bias of a window's (query position t, key position u) pair is
+ * U[h][t] . W[h][u], t = i*M + j the window-local position in the rolled frame,
+ * the same for every window of the batch, added to the scaled score before the
+ * shift mask:  S_tu = q'_t . k'_u / sqrt(d) + U[h][t] . W[h][u].
+ *
+ * Shapes: those of fs_winattn_check_shape with d == 32 (else FS_ERR_SHAPE);
+ * rank == 16 (else FS_ERR_SHAPE).  u, w: fp32 [heads][M*M][16], 16-byte aligned.
+ * theta may be NULL: no rotation (q' = q, k' = k), and the backward then takes
+ * dtheta == NULL too; with theta the RoPE of fs_winattn_fwd applies.  Other
+ * arguments, layouts, ownership and errors as fs_winattn_fwd / fs_winattn_bwd.
+ *
+ * Forward: o and lse (lse may be NULL: inference), overwritten.
+ * Backward: dq, dk, dv, dtheta (when theta is given), du and dw (fp32
+ * [heads][M*M][16], the gradients summed over every window of the batch, in a
+ * fixed order), all overwritten.  dq, du and the query side of dtheta are
+ * accumulated in fp32 with vector reductions whose order varies from run to
+ * run; dk, dv and dw do not vary.  workspace: at least fs_winattn_lrbias_bwd_workspace_bytes(shape)
+ * bytes, 256-byte aligned (about 268 bytes per token-head on the padded grid,
+ * plus a few KB per head).  The kernels are plain one-tile pipelines.
+ */
+FS_API fs_status fs_winattn_lrbias_fwd(const fs_winattn_shape* shape, const void* q, const void* k, const void* v,
+                                       const float* theta, const float* u, const float* w, int rank, void* o,
+                                       float* lse, fs_stream_t stream);
+FS_API size_t fs_winattn_lrbias_bwd_workspace_bytes(const fs_winattn_shape* shape);
+FS_API fs_status fs_winattn_lrbias_bwd(const fs_winattn_shape* shape, const void* q, const void* k, const void* v,
+                                       const void* o, const void* dout, const float* lse, const float* theta,
+                                       const float* u, const float* w, int rank, void* dq, void* dk, void* dv,
+                                       float* dtheta, float* du, float* dw, void* workspace, size_t workspace_bytes,
+                                       fs_stream_t stream);
+
 /* Human-readable name of a status. */
 FS_API const char* fs_status_string(fs_status status);
 
@@ -192,7 +227,9 @@ FS_API size_t fs_winattn_bwd_noalloc_max_bytes(void);
  * n == 0 to switch the hook off.  While set, fs_winattn_fwd records events[0]
  * before and events[1] after its kernel (n >= 2), and fs_winattn_bwd records
  * events[0] before its first kernel and events[1 + i] after its kernel i
- * (prep, main, post, dtheta reduction; n >= 5), on the call's stream.  The
+ * (prep, main, post, dtheta reduction; n >= 5), on the call's stream; the
+ * low-rank-bias entry points record the same marks (the backward's last one
+ * after the dtheta, du and dw sums).  The
  * handles are kept by value; the hook is process-wide and not thread-safe.
  */
 FS_API fs_status fs_set_phase_events(void* const* events, int n);

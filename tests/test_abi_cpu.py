@@ -138,3 +138,53 @@ def test_workspace_flat_in_window_size_at_d64():
     b = _lib.fs_winattn_bwd_workspace_bytes(_lib.make_shape(16, 256, 256, 3, 64, 64, 32))
     c = _lib.fs_winattn_bwd_workspace_bytes(_lib.make_shape(16, 256, 256, 3, 64, 8, 4))
     assert a == b == c > 0
+
+
+def test_lrbias_entry_points_reject_before_launch():
+    """Low-rank bias: d = 32 and rank 16 only; NULL factors, gradients and
+    misaligned pointers; theta without dtheta; a short workspace."""
+    good = _lib.make_shape(1, 16, 16, 2, 32, 8, 4)
+    n = _lib.fs_winattn_lrbias_bwd_workspace_bytes(good)
+    assert n > 0
+    assert _lib.fs_winattn_lrbias_bwd_workspace_bytes(_lib.make_shape(1, 16, 16, 2, 64, 8, 4)) == 0
+
+    def fwd(shape, *a):
+        with pytest.raises(_lib.FswinError) as e:
+            _lib.fs_winattn_lrbias_fwd(shape, *a, 0)
+        return e.value.status
+
+    p = 256
+    #              q  k  v  theta u  w  rank o  lse
+    assert fwd(_lib.make_shape(1, 16, 16, 2, 64, 8, 4), p, p, p, p, p, p, 16, p, p) == _lib.FS_ERR_SHAPE
+    assert fwd(good, p, p, p, p, p, p, 8, p, p) == _lib.FS_ERR_SHAPE
+    assert fwd(good, p, p, p, p, 0, p, 16, p, p) == _lib.FS_ERR_NULL
+    assert fwd(good, p, p, p, p, p + 4, p, 16, p, p) == _lib.FS_ERR_ALIGN
+
+    def bwd(shape, dtheta=p, du=p, ws=p, nbytes=n, theta=p, rank=16):
+        with pytest.raises(_lib.FswinError) as e:
+            _lib.fs_winattn_lrbias_bwd(shape, p, p, p, p, p, p, theta, p, p, rank, p, p, p, dtheta, du, p, ws,
+                                       nbytes, 0)
+        return e.value.status
+
+    assert bwd(good, rank=32) == _lib.FS_ERR_SHAPE
+    assert bwd(good, dtheta=0) == _lib.FS_ERR_NULL      # theta given, dtheta NULL
+    assert bwd(good, du=0) == _lib.FS_ERR_NULL
+    assert bwd(good, du=p + 8) == _lib.FS_ERR_ALIGN
+    assert bwd(good, nbytes=n - 1) == _lib.FS_ERR_WORKSPACE
+    assert bwd(good, ws=p + 16) == _lib.FS_ERR_WORKSPACE
+
+
+def test_lrbias_workspace_size():
+    """The bias backward's scratch: 256 B of accumulator rows per token-head (on
+    the padded grid), 8 x 16 fp32 d theta partials and the norms per (head,
+    tile), a fixed d theta part, and one [head][window slot][32] fp32 block per
+    16 windows for the first level of the dU / dW sum."""
+    B, H, W, heads, M = 4, 64, 64, 3, 16
+    n = _lib.fs_winattn_lrbias_bwd_workspace_bytes(_lib.make_shape(B, H, W, heads, 32, M, 8))
+    tokens = B * H * W * heads
+    wins = B * (H // M) * (W // M)
+    chunks = -(-wins // 16)
+    tiles = B * H * W // 128
+    expect = tokens * 256 + heads * tiles * 8 + heads * tiles * 8 * 16 * 4 + heads * 64 * 16 * 4 + heads * 4 + \
+        chunks * heads * M * M * 32 * 4
+    assert expect <= n <= expect + 6 * 256

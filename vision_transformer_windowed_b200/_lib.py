@@ -71,6 +71,12 @@ def load(build_if_missing: bool = True):
         lib.fs_winattn_bwd_noalloc.restype = st
         lib.fs_winattn_bwd_noalloc_max_bytes.argtypes = []
         lib.fs_winattn_bwd_noalloc_max_bytes.restype = ctypes.c_size_t
+        lib.fs_winattn_lrbias_fwd.argtypes = [P] + [vp] * 6 + [ctypes.c_int, vp, vp, vp]
+        lib.fs_winattn_lrbias_fwd.restype = st
+        lib.fs_winattn_lrbias_bwd_workspace_bytes.argtypes = [P]
+        lib.fs_winattn_lrbias_bwd_workspace_bytes.restype = ctypes.c_size_t
+        lib.fs_winattn_lrbias_bwd.argtypes = [P] + [vp] * 9 + [ctypes.c_int] + [vp] * 7 + [ctypes.c_size_t, vp]
+        lib.fs_winattn_lrbias_bwd.restype = st
         _lib = lib
         return lib
 
@@ -122,6 +128,24 @@ def fs_winattn_bwd_noalloc(shape: Shape, q: int, k: int, v: int, o: int, dout: i
 
 def fs_winattn_bwd_noalloc_max_bytes() -> int:
     return int(load().fs_winattn_bwd_noalloc_max_bytes())
+
+
+def fs_winattn_lrbias_fwd(shape: Shape, q: int, k: int, v: int, theta: int, u: int, w: int, rank: int, o: int,
+                          lse: int, stream: int) -> None:
+    _check(load().fs_winattn_lrbias_fwd(ctypes.byref(shape), q, k, v, theta, u, w, int(rank), o, lse, stream),
+           "fs_winattn_lrbias_fwd")
+
+
+def fs_winattn_lrbias_bwd_workspace_bytes(shape: Shape) -> int:
+    return int(load().fs_winattn_lrbias_bwd_workspace_bytes(ctypes.byref(shape)))
+
+
+def fs_winattn_lrbias_bwd(shape: Shape, q: int, k: int, v: int, o: int, dout: int, lse: int, theta: int, u: int,
+                          w: int, rank: int, dq: int, dk: int, dv: int, dtheta: int, du: int, dw: int,
+                          workspace: int, workspace_bytes: int, stream: int) -> None:
+    _check(load().fs_winattn_lrbias_bwd(ctypes.byref(shape), q, k, v, o, dout, lse, theta, u, w, int(rank), dq, dk,
+                                        dv, dtheta, du, dw, workspace, workspace_bytes, stream),
+           "fs_winattn_lrbias_bwd")
 
 
 def fs_device_status() -> int:

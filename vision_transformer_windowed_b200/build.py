@@ -10,7 +10,7 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 BUILD = os.path.join(HERE, "_build")
 LIB = os.path.join(BUILD, "libfswin.so")
-SOURCES = ["api.cu", "fwd.cu", "bwd.cu", "small.cu", "block.cu", "noalloc.cu", "wide.cu"]
+SOURCES = ["api.cu", "fwd.cu", "bwd.cu", "small.cu", "block.cu", "noalloc.cu", "wide.cu", "lrbias.cu"]
 HEADERS = ["dgeo.cuh", "geometry.cuh", "kernels.cuh", "ptx.cuh", "rows.cuh", "schedule.cuh", "tile_io.cuh"]
 
 

@@ -260,6 +260,104 @@ fs_status fs_winattn_bwd(const fs_winattn_shape* shape, const void* q, const voi
     return e == cudaSuccess ? FS_OK : FS_ERR_CUDA;
 }
 
+fs_status fs_winattn_lrbias_fwd(const fs_winattn_shape* shape, const void* q, const void* k, const void* v,
+                                const float* theta, const float* u, const float* w, int rank, void* o, float* lse,
+                                fs_stream_t stream) {
+    Geo g;
+    fs_status st = make_geo(shape, &g);
+    if (st != FS_OK) return st;
+    if (g.d != 32 || rank != 16) return FS_ERR_SHAPE;
+    if (g.B == 0) return FS_OK;
+    if (!q || !k || !v || !u || !w || !o) return FS_ERR_NULL;  // theta and lse may be NULL
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(u) || !aligned16(w) ||
+        (reinterpret_cast<uintptr_t>(theta) & 3u) || (reinterpret_cast<uintptr_t>(lse) & 3u))
+        return FS_ERR_ALIGN;
+    unsigned int* status = nullptr;
+    int sms = 0;
+    if ((st = device_state(&status, &sms)) != FS_OK) return st;
+    unsigned long long lim;
+    {
+        std::lock_guard<std::mutex> lk(g_mu);
+        lim = g_limit_ns;
+    }
+    LrbPtrs p{};
+    p.q = q;
+    p.k = k;
+    p.v = v;
+    p.theta = theta;
+    p.u = u;
+    p.w = w;
+    p.o_out = o;
+    p.lse_out = lse;
+    const cudaError_t e = launch_lrbias_fwd(g, p, status, lim, sms, reinterpret_cast<cudaStream_t>(stream),
+                                            g_phase_n >= 2 ? g_phase_events : nullptr);
+    return e == cudaSuccess ? FS_OK : FS_ERR_CUDA;
+}
+
+size_t fs_winattn_lrbias_bwd_workspace_bytes(const fs_winattn_shape* shape) {
+    Geo g;
+    if (make_geo(shape, &g) != FS_OK || g.d != 32) return 0;
+    return lrbias_bwd_workspace_bytes(g);
+}
+
+fs_status fs_winattn_lrbias_bwd(const fs_winattn_shape* shape, const void* q, const void* k, const void* v,
+                                const void* o, const void* dout, const float* lse, const float* theta,
+                                const float* u, const float* w, int rank, void* dq, void* dk, void* dv,
+                                float* dtheta, float* du, float* dw, void* workspace, size_t workspace_bytes,
+                                fs_stream_t stream) {
+    Geo g;
+    fs_status st = make_geo(shape, &g);
+    if (st != FS_OK) return st;
+    if (g.d != 32 || rank != 16) return FS_ERR_SHAPE;
+    if (!du || !dw || (theta && !dtheta)) return FS_ERR_NULL;
+    if (!aligned16(du) || !aligned16(dw) || (reinterpret_cast<uintptr_t>(dtheta) & 3u)) return FS_ERR_ALIGN;
+    unsigned int* status = nullptr;
+    int sms = 0;
+    const cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+    if (g.B == 0) {
+        // Empty batch: the parameter gradients are empty sums.
+        if ((st = device_state(&status, &sms)) != FS_OK) return st;
+        const int nb = g.heads * g.N * 16;
+        zero_f32_kernel<<<(nb + 255) / 256, 256, 0, cs>>>(du, nb);
+        zero_f32_kernel<<<(nb + 255) / 256, 256, 0, cs>>>(dw, nb);
+        if (theta) zero_f32_kernel<<<(g.heads * 16 + 255) / 256, 256, 0, cs>>>(dtheta, g.heads * 16);
+        return cudaGetLastError() == cudaSuccess ? FS_OK : FS_ERR_CUDA;
+    }
+    if (!q || !k || !v || !o || !dout || !lse || !u || !w || !dq || !dk || !dv) return FS_ERR_NULL;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(dout) || !aligned16(dq) ||
+        !aligned16(dk) || !aligned16(dv) || !aligned16(u) || !aligned16(w) ||
+        (reinterpret_cast<uintptr_t>(lse) & 3u) || (reinterpret_cast<uintptr_t>(theta) & 3u))
+        return FS_ERR_ALIGN;
+    if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) ||
+        workspace_bytes < lrbias_bwd_workspace_bytes(g))
+        return FS_ERR_WORKSPACE;
+    if ((st = device_state(&status, &sms)) != FS_OK) return st;
+    unsigned long long lim;
+    {
+        std::lock_guard<std::mutex> lk(g_mu);
+        lim = g_limit_ns;
+    }
+    LrbPtrs p{};
+    p.q = q;
+    p.k = k;
+    p.v = v;
+    p.o = o;
+    p.dout = dout;
+    p.lse = lse;
+    p.theta = theta;
+    p.u = u;
+    p.w = w;
+    p.dq = dq;
+    p.dk = dk;
+    p.dv = dv;
+    p.dtheta = theta ? dtheta : nullptr;
+    p.du = du;
+    p.dw = dw;
+    p.ws = static_cast<uint8_t*>(workspace);
+    const cudaError_t e = launch_lrbias_bwd(g, p, status, lim, sms, cs, g_phase_n >= 5 ? g_phase_events : nullptr);
+    return e == cudaSuccess ? FS_OK : FS_ERR_CUDA;
+}
+
 fs_status fs_device_status(unsigned int* code) {
     if (!code) return FS_ERR_NULL;
     unsigned int* status = nullptr;

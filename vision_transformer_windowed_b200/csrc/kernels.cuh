@@ -92,6 +92,24 @@ cudaError_t launch_wide_fwd(const Geo& g, const void* q, const void* k, const vo
 cudaError_t launch_wide_bwd(const Geo& g, const BwdPtrs& p, unsigned int* status, unsigned long long limit_ns,
                             int num_sms, cudaStream_t stream, cudaEvent_t const* events);
 
+// Windowed attention with a low-rank additive bias U_h W_h^T (heads of 32
+// channels, every window size; theta may be null: no rotation, no d theta).
+struct LrbPtrs {
+    const void *q, *k, *v, *o, *dout;  // bf16 [B, H, W, heads, 32]
+    const float *lse, *theta;           // theta: [heads][2][8] or null
+    const float *u, *w;                 // [heads][M*M][16]
+    void *o_out, *dq, *dk, *dv;         // o_out: the forward's O
+    float *lse_out, *dtheta, *du, *dw;
+    uint8_t* ws;
+};
+size_t lrbias_bwd_workspace_bytes(const Geo& g);
+// events as for the 64-channel kernels (the backward's last mark follows the
+// d theta and dU / dW sums).
+cudaError_t launch_lrbias_fwd(const Geo& g, const LrbPtrs& p, unsigned int* status, unsigned long long limit_ns,
+                              int num_sms, cudaStream_t stream, cudaEvent_t const* events);
+cudaError_t launch_lrbias_bwd(const Geo& g, const LrbPtrs& p, unsigned int* status, unsigned long long limit_ns,
+                              int num_sms, cudaStream_t stream, cudaEvent_t const* events);
+
 // Fixed-order d theta sum: part [heads][per_head][16] -> dtheta [heads][16] (one
 // launch; cnt: heads counters that are zero when it starts).
 namespace bwdk {

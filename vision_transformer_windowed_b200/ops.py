@@ -139,3 +139,91 @@ class WindowAttentionRoPE(torch.autograd.Function):
 
 def window_attention(q, k, v, theta, M: int, s: int):
     return WindowAttentionRoPE.apply(q, k, v, theta, M, s)
+
+
+# ------------------------------------------------------------ low-rank bias
+# The FlashBias-T variant of the same pages (thelatestinai.com/papers/2610.04664,
+# Table 2 and Table S1 captions): a trainable rank-16 factorization U_h W_h^T of
+# an additive bias over window-local positions, shared by every window and added
+# to the scaled scores before the shift mask.  Heads of 32 channels; theta may be
+# None (no rotation).
+LRBIAS_RANK = 16
+
+
+def _check_factors(q, u, w, M: int) -> None:
+    heads = q.shape[3]
+    for name, t in (("u", u), ("w", w)):
+        _check_tensor(name, t, (heads, M * M, LRBIAS_RANK), torch.float32)
+
+
+def winattn_lrbias_fwd(q, k, v, theta, u, w, M: int, s: int, o=None, lse=None, need_lse: bool = True):
+    """O, LSE of windowed attention with the low-rank bias u_t . w_u (bf16 in/out, fp32 LSE)."""
+    sh = _shape(q, M, s)
+    B, H, W, heads, d = q.shape
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        _check_tensor(name, t, q.shape, torch.bfloat16)
+    if theta is not None:
+        _check_tensor("theta", theta, (heads, 2, d // 4), torch.float32)
+    _check_factors(q, u, w, M)
+    if o is None:
+        o = torch.empty_like(q)
+    if lse is None and need_lse:
+        lse = torch.empty((B, H, W, heads), device=q.device, dtype=torch.float32)
+    _check_tensor("o", o, q.shape, torch.bfloat16)
+    if lse is not None:
+        _check_tensor("lse", lse, (B, H, W, heads), torch.float32)
+    _lib.fs_winattn_lrbias_fwd(sh, q.data_ptr(), k.data_ptr(), v.data_ptr(),
+                               theta.data_ptr() if theta is not None else 0, u.data_ptr(), w.data_ptr(),
+                               LRBIAS_RANK, o.data_ptr(), lse.data_ptr() if lse is not None else 0,
+                               _stream(q.device))
+    return o, lse
+
+
+def alloc_lrbias_workspace(q: torch.Tensor, M: int, s: int) -> torch.Tensor:
+    n = _lib.fs_winattn_lrbias_bwd_workspace_bytes(_shape(q, M, s))
+    return torch.empty(max(n, 256), device=q.device, dtype=torch.uint8)
+
+
+def winattn_lrbias_bwd(q, k, v, o, dout, lse, theta, u, w, M: int, s: int, workspace=None):
+    """dQ, dK, dV, dtheta (None without theta), dU, dW of sum(O * dout)."""
+    sh = _shape(q, M, s)
+    B, H, W, heads, d = q.shape
+    for name, t in (("q", q), ("k", k), ("v", v), ("o", o), ("dout", dout)):
+        _check_tensor(name, t, q.shape, torch.bfloat16)
+    _check_tensor("lse", lse, (B, H, W, heads), torch.float32)
+    if theta is not None:
+        _check_tensor("theta", theta, (heads, 2, d // 4), torch.float32)
+    _check_factors(q, u, w, M)
+    dq, dk, dv = (torch.empty_like(q) for _ in range(3))
+    dtheta = torch.empty_like(theta) if theta is not None else None
+    du, dw = torch.empty_like(u), torch.empty_like(w)
+    if workspace is None:
+        workspace = alloc_lrbias_workspace(q, M, s)
+    _lib.fs_winattn_lrbias_bwd(sh, q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), dout.data_ptr(),
+                               lse.data_ptr(), theta.data_ptr() if theta is not None else 0, u.data_ptr(),
+                               w.data_ptr(), LRBIAS_RANK, dq.data_ptr(), dk.data_ptr(), dv.data_ptr(),
+                               dtheta.data_ptr() if dtheta is not None else 0, du.data_ptr(), dw.data_ptr(),
+                               workspace.data_ptr(), workspace.numel(), _stream(q.device))
+    return dq, dk, dv, dtheta, du, dw
+
+
+class WindowAttentionLowRankBias(torch.autograd.Function):
+    """Autograd wrapper of the low-rank-bias attention (forward and backward in libfswin.so)."""
+
+    @staticmethod
+    def forward(ctx, q, k, v, theta, u, w, M: int, s: int):
+        o, lse = winattn_lrbias_fwd(q, k, v, theta, u, w, M, s)
+        ctx.save_for_backward(q, k, v, o, lse, u, w, *(() if theta is None else (theta,)))
+        ctx.M, ctx.s, ctx.has_theta = M, s, theta is not None
+        return o
+
+    @staticmethod
+    def backward(ctx, dout):
+        q, k, v, o, lse, u, w, *rest = ctx.saved_tensors
+        theta = rest[0] if ctx.has_theta else None
+        dq, dk, dv, dth, du, dw = winattn_lrbias_bwd(q, k, v, o, dout.contiguous(), lse, theta, u, w, ctx.M, ctx.s)
+        return dq, dk, dv, dth, du, dw, None, None
+
+
+def window_attention_lrbias(q, k, v, theta, u, w, M: int, s: int):
+    return WindowAttentionLowRankBias.apply(q, k, v, theta, u, w, M, s)
