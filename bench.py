@@ -60,7 +60,12 @@ WORKLOADS = {
     # heads of 64 channels (the wide kernels): the FlashSwin-T stage-1 grid at p=2 with 3 heads of d=64,
     # window 32, shifted block; batch 64 keeps each tensor at the size of the d=32 workload's
     "flashswin_stage1_p2_m32_d64": dict(B=64, H=128, W=128, heads=3, M=32, shifts=(16,), qk_scale=1.0, d=64),
+    # the low-rank additive bias variant (FlashBias-T: a trainable rank-16 bias factorization, with RoPE
+    # here) at the FlashSwin-T stage-1 shapes, p=2 window 32 and p=4 window 8
+    "flashbias_t_stage1_p2_m32": dict(B=128, H=128, W=128, heads=3, M=32, shifts=(0, 16), qk_scale=1.0, lrbias=True),
+    "flashbias_t_stage1_p4_m8": dict(B=128, H=64, W=64, heads=3, M=8, shifts=(0, 4), qk_scale=1.0, lrbias=True),
 }
+LRBIAS_RANK = 16
 HEADLINE = "flashswin_t_p2_4stage"
 SPEC_BF16_TFLOPS = 2250.0  # NVIDIA's dense bf16 figure for one B200: a spec value, not a measurement
 
@@ -145,9 +150,9 @@ def stages_of(wl) -> list:
     head dimension, 32 unless given)."""
     if "stages" in wl:
         return [dict(st, qk_scale=st.get("qk_scale", wl.get("qk_scale", 1.0)), infer=wl.get("infer", False),
-                     d=st.get("d", wl.get("d", HEAD_DIM)))
+                     d=st.get("d", wl.get("d", HEAD_DIM)), lrbias=wl.get("lrbias", False))
                 for st in wl["stages"]]
-    return [dict(wl, d=wl.get("d", HEAD_DIM))]
+    return [dict(wl, d=wl.get("d", HEAD_DIM), lrbias=wl.get("lrbias", False))]
 
 
 def blocks_of(wl) -> list:
@@ -155,11 +160,25 @@ def blocks_of(wl) -> list:
     return [(st, s) for st in stages_of(wl) for s in st["shifts"]]
 
 
+def pair_flops(st) -> tuple[float, float]:
+    """FLOPs per attending pair of the forward and the backward products: 4 d forward (S and P V)
+    and 10 d backward (S again, dP, dV, dK, dQ); with the rank-r low-rank bias the score product
+    and the two gradient products that carry the factors contract over d + r channels, so
+    4 d + 2 r and 10 d + 6 r."""
+    d = st.get("d", HEAD_DIM)
+    r = LRBIAS_RANK if st.get("lrbias") else 0
+    return 4.0 * d + 2.0 * r, 10.0 * d + 6.0 * r
+
+
 def workload_flops(wl) -> tuple[float, float]:
-    """Useful forward and backward FLOPs of one step (fwd 4*d per pair, bwd 10*d per pair)."""
-    dpairs = sum(st["d"] * unmasked_pairs(st["B"], st["H"], st["W"], st["heads"], st["M"], s)
-                 for st, s in blocks_of(wl))
-    return 4.0 * dpairs, 10.0 * dpairs
+    """Useful forward and backward FLOPs of one step (per attending pair: `pair_flops`)."""
+    fwd = bwd = 0.0
+    for st, s in blocks_of(wl):
+        pairs = unmasked_pairs(st["B"], st["H"], st["W"], st["heads"], st["M"], s)
+        pf, pb = pair_flops(st)
+        fwd += pf * pairs
+        bwd += pb * pairs
+    return fwd, bwd
 
 
 def workload_tokens(wl) -> int:
@@ -182,6 +201,14 @@ def phase_work(st, s) -> dict:
     rows = B * H * W * heads
     pairs = unmasked_pairs(B, H, W, heads, M, s)
     small = M * M < 128
+    pf, pb = pair_flops(st)
+    if st.get("lrbias"):  # the bias kernels (plain pipelines at every window size): prep reads dO, v
+        # and zeroes the fp32 accumulator rows (256 B); main reads q, k, v, o, dO, lse and writes dk,
+        # dv; post reads the accumulator's dQ' part and q and writes dq; the window sums read the
+        # accumulator's dU / dW part (the factors themselves stay in L2)
+        nbytes = {"fwd": (256 if st.get("infer") else 260) * rows, "bwd_prep": 384 * rows,
+                  "bwd_main": 452 * rows, "bwd_post": 256 * rows, "bwd_dtheta": 128 * rows}
+        return {"bytes": nbytes, "flops": {"fwd": pf * pairs, "bwd_main": pb * pairs}, "hbm_bound": False}
     if d == 64:  # the wide kernels: prep reads dO, v and zeroes the fp32 dQ' accumulator; main reads
         # q, k, v, o, dO and lse, writes dk, dv (the dQ' additions resolve in L2); post reads the
         # accumulator and q, writes dq
@@ -191,7 +218,7 @@ def phase_work(st, s) -> dict:
         nbytes = {"fwd": (256 if st.get("infer") else 260) * rows, "bwd_prep": 0 if small else 596 * rows,
                   "bwd_main": (520 if small else 392) * rows, "bwd_post": 0 if small else 256 * rows,
                   "bwd_dtheta": 0}
-    flops = {"fwd": 4.0 * d * pairs, "bwd_main": 10.0 * d * pairs}
+    flops = {"fwd": pf * pairs, "bwd_main": pb * pairs}
     return {"bytes": nbytes, "flops": flops, "hbm_bound": small and d == 32}
 
 
@@ -229,7 +256,7 @@ def roofline(wl, res, peaks, sm_mhz=None) -> dict:
                 "frac": achieved / peak, "frac_of_burst": achieved / peaks["bf16_tflops"], "traffic": None,
                 "algorithmic_flops_per_step": fl, "algorithmic_bytes_per_step": sum(w["bytes"][dom] for w in work),
                 "peak_note": f"cuBLAS bf16 sustained (burst {peaks['bf16_tflops']:.1f}), {peaks['source']}"}
-        per_exp = (4.0 if dom == "fwd" else 10.0) * blocks[0][0]["d"]
+        per_exp = pair_flops(blocks[0][0])[0 if dom == "fwd" else 1]
         mhz = sm_mhz or 1965.0
         roof["mufu_ceiling_tflops"] = mufu_ceiling_tflops(per_exp, mhz)
         roof["mufu_note"] = (f"one MUFU exp2 per score element: 16/clk/SM x 148 SMs x {mhz:.0f} MHz x "
@@ -330,16 +357,17 @@ def cpu_baseline(tensors, wl, seconds: float = 12.0):
             # units spread over the batch, including windows of the last row/column
             t0 = time.perf_counter()
             probe = np.arange(0, min(n_units, 4 * cores))
-            oracle.units(t["q"], t["k"], t["v"], t["theta"], M, s, probe, dout=t["dout"], nthreads=cores)
+            bias = (t["u"], t["w"]) if st.get("lrbias") else None
+            oracle.units(t["q"], t["k"], t["v"], t["theta"], M, s, probe, dout=t["dout"], nthreads=cores, bias=bias)
             dt = max(time.perf_counter() - t0, 1e-6)
             budget = seconds / nblocks
             n = int(min(n_units, max(len(probe), len(probe) * budget / dt)))
             ids = np.linspace(0, n_units - 1, n).astype(np.int64)
             t0 = time.perf_counter()
-            oracle.units(t["q"], t["k"], t["v"], t["theta"], M, s, ids, dout=t["dout"], nthreads=cores)
+            oracle.units(t["q"], t["k"], t["v"], t["theta"], M, s, ids, dout=t["dout"], nthreads=cores, bias=bias)
             dt = time.perf_counter() - t0
             # useful flops of the sampled units (pairs that attend)
-            flops += 14.0 * st.get("d", HEAD_DIM) * unmasked_pairs(B, H, W, heads, M, s) * (n / n_units)
+            flops += sum(pair_flops(st)) * unmasked_pairs(B, H, W, heads, M, s) * (n / n_units)
             total_dt += dt
             done += n
             full_s += dt * n_units / n
@@ -350,6 +378,18 @@ def cpu_baseline(tensors, wl, seconds: float = 12.0):
             "units_per_s": done / total_dt,
             "full_step_s_extrapolated": full_s,  # equal to the measured time when every unit was sampled
             "seconds": total_dt}
+
+
+def cpu_stage_inputs(wl) -> list:
+    """Seeded CPU inputs of every stage of a workload (with the bias factors when it has them)."""
+    from vision_transformer_windowed_b200.inputs import make_bias, make_inputs
+    out = []
+    for st in stages_of(wl):
+        t = make_inputs(st["B"], st["H"], st["W"], st["heads"], st["d"], device="cpu", qk_scale=st["qk_scale"])
+        if st.get("lrbias"):
+            t.update(make_bias(st["heads"], st["M"], LRBIAS_RANK))
+        out.append(t)
+    return out
 
 
 def config_entry(wl, r, peaks, world, name=None) -> dict:
@@ -456,10 +496,8 @@ def run_reference(args):
         return
     import torch
 
-    from vision_transformer_windowed_b200.inputs import make_inputs
     wl = WORKLOADS[args.workload]
-    t = [make_inputs(st["B"], st["H"], st["W"], st["heads"], st["d"], device="cpu", qk_scale=st["qk_scale"])
-         for st in stages_of(wl)]
+    t = cpu_stage_inputs(wl)
     per_step = max(1.0, args.reference_seconds / max(1, args.steps + args.warmup))
     for _ in range(args.warmup):
         cpu_baseline(t, wl, seconds=per_step)
@@ -509,7 +547,7 @@ def main():
     import torch.distributed as dist
 
     from vision_transformer_windowed_b200 import _lib, dp, ops
-    from vision_transformer_windowed_b200.inputs import make_inputs
+    from vision_transformer_windowed_b200.inputs import make_bias
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -529,19 +567,29 @@ def main():
     def run_workload(name, steps, warmup, phase=True, clocks=False):
         wl = WORKLOADS[name]
         infer = wl.get("infer", False)
+        lrb = wl.get("lrbias", False)
         # per stage: inputs, a backward workspace, and the outputs of each of its blocks
         data = []
         for st in stages_of(wl):
             B, H, W, heads, M = st["B"], st["H"], st["W"], st["heads"], st["M"]
             t = dp.rank_inputs(B, H, W, heads, st["d"], rank, dev, qk_scale=st["qk_scale"])
+            if lrb:
+                t.update(make_bias(heads, M, LRBIAS_RANK, device=dev))
             blocks = []
             for s in st["shifts"]:
                 o = torch.empty_like(t["q"])
                 lse = None if infer else torch.empty((B, H, W, heads), device=dev, dtype=torch.float32)
                 g = None if infer else (torch.empty_like(t["q"]), torch.empty_like(t["q"]), torch.empty_like(t["q"]),
                                         torch.empty_like(t["theta"]))
+                if lrb:
+                    g = g + (torch.empty_like(t["u"]), torch.empty_like(t["w"]))
                 blocks.append((s, o, lse, g))
-            ws = torch.empty(0, dtype=torch.uint8) if infer else ops.alloc_workspace(t["q"], M, st["shifts"][0])
+            if infer:
+                ws = torch.empty(0, dtype=torch.uint8)
+            elif lrb:
+                ws = ops.alloc_lrbias_workspace(t["q"], M, st["shifts"][0])
+            else:
+                ws = ops.alloc_workspace(t["q"], M, st["shifts"][0])
             data.append((st, t, blocks, ws))
 
         def step(evs=None):
@@ -554,6 +602,14 @@ def main():
                         _lib.fs_set_phase_events([e.cuda_event for e in evs[i][0]])
                     if infer:  # forward only, O only
                         ops.winattn_fwd(q, k, v, th, M, s, o=o, need_lse=False)
+                    elif lrb:  # the low-rank bias variant: theta, U and W are shared by the batch
+                        ops.winattn_lrbias_fwd(q, k, v, th, t["u"], t["w"], M, s, o=o, lse=lse)
+                        if evs is not None:
+                            _lib.fs_set_phase_events([e.cuda_event for e in evs[i][1]])
+                        dq, dk, dv, dth, du, dw = g
+                        ops.winattn_lrbias_bwd(q, k, v, o, do, lse, th, t["u"], t["w"], M, s, workspace=ws, dq=dq,
+                                               dk=dk, dv=dv, dtheta=dth, du=du, dw=dw)
+                        dp.allreduce_param_grads(dth, du, dw)
                     else:
                         ops.winattn_fwd(q, k, v, th, M, s, o=o, lse=lse)
                         if evs is not None:
@@ -638,7 +694,9 @@ def main():
     # step's result for an optimizer) is read back; O, dQ, dK, dV stay on the device, as they do
     # inside a model.  e2e_all_outputs: the same with O, dQ, dK, dV and d theta all read back and
     # every copy on the compute stream.
-    host = [{k: t[k].cpu().pin_memory() for k in ("q", "k", "v", "dout", "theta")} for _, t, _, _ in main_res["data"]]
+    lrb = wl.get("lrbias", False)
+    in_keys = ("q", "k", "v", "dout", "theta") + (("u", "w") if lrb else ())
+    host = [{k: t[k].cpu().pin_memory() for k in in_keys} for _, t, _, _ in main_res["data"]]
     res_host = {}
     e2e_steps = max(1, min(args.steps, 5))
     torch.cuda.synchronize()
@@ -666,10 +724,19 @@ def main():
                     x.record_stream(main)  # allocated on the copy stream, used on this one
             M = st["M"]
             for bi, s in enumerate(st["shifts"]):
-                o, lse = ops.winattn_fwd(dvi["q"], dvi["k"], dvi["v"], dvi["theta"], M, s)
-                dq, dk, dvv, dth = ops.winattn_bwd(dvi["q"], dvi["k"], dvi["v"], o, dvi["dout"], lse, dvi["theta"], M, s)
-                dp.allreduce_dtheta(dth)
-                outs = (("o", o), ("dq", dq), ("dk", dk), ("dv", dvv), ("dtheta", dth)) if read_all else (("dtheta", dth),)
+                if lrb:
+                    o, lse = ops.winattn_lrbias_fwd(dvi["q"], dvi["k"], dvi["v"], dvi["theta"], dvi["u"], dvi["w"], M, s)
+                    dq, dk, dvv, dth, du, dw = ops.winattn_lrbias_bwd(dvi["q"], dvi["k"], dvi["v"], o, dvi["dout"], lse,
+                                                                      dvi["theta"], dvi["u"], dvi["w"], M, s)
+                    dp.allreduce_param_grads(dth, du, dw)
+                    params = (("dtheta", dth), ("du", du), ("dw", dw))
+                else:
+                    o, lse = ops.winattn_fwd(dvi["q"], dvi["k"], dvi["v"], dvi["theta"], M, s)
+                    dq, dk, dvv, dth = ops.winattn_bwd(dvi["q"], dvi["k"], dvi["v"], o, dvi["dout"], lse, dvi["theta"],
+                                                       M, s)
+                    dp.allreduce_dtheta(dth)
+                    params = (("dtheta", dth),)
+                outs = (("o", o), ("dq", dq), ("dk", dk), ("dv", dvv)) + params if read_all else params
                 for name, x in outs:
                     key = (si, bi, name)
                     if key not in res_host:
@@ -695,7 +762,7 @@ def main():
     e2e = {"value": fl * world / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s", "ms_per_step": e2e_ms,
            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h["result"],
            "step": "inputs from pinned host memory (uploads overlapped with the previous stage's kernels), "
-                   "d theta of every block read back"}
+                   "the parameter gradients (d theta; dU, dW with the bias) of every block read back"}
     e2e_all_ms = e2e_time(True)
     e2e_all = {"value": fl * world / (e2e_all_ms * 1e-3) / 1e12, "unit": "TFLOP/s", "ms_per_step": e2e_all_ms,
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h["all"],
@@ -719,13 +786,15 @@ def main():
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        tt = [make_inputs(st["B"], st["H"], st["W"], st["heads"], st["d"], device="cpu", qk_scale=st["qk_scale"])
-              for st in stages_of(wl)]
-        cpu = cpu_baseline(tt, wl)
+        cpu = cpu_baseline(cpu_stage_inputs(wl), wl)
         cpu.pop("seconds", None)
 
     if rank == 0:
-        nlaunch = sum(1 + (4 if st["d"] == 64 else (2 if st["M"] * st["M"] < 128 else 5)) for st, _ in blocks)
+        def launches(st):  # kernels of one block: the forward, then the backward's
+            if st.get("lrbias"):
+                return 1 + 6  # prep, main, post, d theta sum, two dU / dW sum levels
+            return 1 + (4 if st["d"] == 64 else (2 if st["M"] * st["M"] < 128 else 5))
+        nlaunch = sum(launches(st) for st, _ in blocks)
         line = {
             "metric": METRIC, "value": main_res["tflops"], "unit": "TFLOP/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": main_res["ms"], "higher_is_better": True,

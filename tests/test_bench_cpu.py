@@ -114,3 +114,26 @@ def test_flops_and_bytes_scale_with_the_head_dimension():
     w = bench.phase_work(bench.stages_of(wl)[0], 4)
     assert w["flops"]["bwd_main"] == 10 * 64 * pairs and not w["hbm_bound"]
     assert w["bytes"]["fwd"] == 516 * 16 * 16 * 2
+
+
+def test_lrbias_flops_count_the_factor_channels():
+    """The bias variant's products contract over d + 16 channels where the factors
+    ride along: 4 d + 32 forward and 10 d + 96 backward flops per attending pair."""
+    wl = bench.WORKLOADS["flashbias_t_stage1_p2_m32"]
+    assert wl["lrbias"]
+    pairs = sum(bench.unmasked_pairs(wl["B"], wl["H"], wl["W"], wl["heads"], wl["M"], s) for s in wl["shifts"])
+    fwd, bwd = bench.workload_flops(wl)
+    assert fwd == 160 * pairs and bwd == 416 * pairs
+    st = bench.stages_of(wl)[0]
+    w = bench.phase_work(st, 16)
+    assert not w["hbm_bound"] and w["flops"]["bwd_main"] == 416 * bench.unmasked_pairs(128, 128, 128, 3, 32, 16)
+    peaks = {"hbm_gbs": 6000.0, "bf16_tflops": 1600.0, "bf16_tflops_sustained": 1400.0, "source": "measured"}
+    res = {"phase_ms_per_step": {"fwd": 1.0, "bwd_prep": 0.2, "bwd_main": 2.0, "bwd_post": 0.1, "bwd_dtheta": 0.01}}
+    roof = bench.roofline(wl, res, peaks, sm_mhz=1900.0)
+    assert roof["mufu_ceiling_tflops"] == pytest.approx(416 * 16 * 148 * 1900e6 / 1e12)
+
+
+def test_cpu_baseline_runs_the_bias_oracle():
+    wl = dict(B=1, H=16, W=16, heads=2, M=8, shifts=(4,), qk_scale=1.0, lrbias=True)
+    res = bench.cpu_baseline(bench.cpu_stage_inputs(wl), wl, seconds=1.0)
+    assert res["value"] > 0 and "8 of 8 at s=4" in res["sample"]

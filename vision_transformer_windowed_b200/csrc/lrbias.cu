@@ -480,11 +480,11 @@ __global__ void __launch_bounds__(128) prep_kernel(const Params p) {
 constexpr int kThreads = 128;
 constexpr int kKOff = 0;                           // K~ half tiles: k' and W
 constexpr int kVOff = kKOff + 2 * kTileBytes;      // V tile
-constexpr int kQOff = kVOff + kTileBytes;          // Q~ half tiles: q' and sqrt(d) U
-constexpr int kDOOff = kQOff + 2 * kTileBytes;     // dO tile
-constexpr int kDSOff = kDOOff + kTileBytes;        // dS', MN-major 128-byte swizzle (1024-aligned)
-constexpr int kVecOff = kDSOff + 4 * kTileBytes;   // lse2[128], D[128]
-constexpr int kTabOff = kVecOff + 2 * kTile * 4;
+constexpr int kBufOff = kVOff + kTileBytes;        // two query buffers: Q~ half tiles (q', sqrt(d) U), dO tile
+constexpr int kBufBytes = 3 * kTileBytes;
+constexpr int kDSOff = kBufOff + 2 * kBufBytes;    // dS', MN-major 128-byte swizzle (1024-aligned)
+constexpr int kVecOff = kDSOff + 4 * kTileBytes;   // per buffer: lse2[128], D[128]
+constexpr int kTabOff = kVecOff + 2 * 2 * kTile * 4;
 constexpr int kBarOff = kTabOff + kTabBytes;
 constexpr int kSmemBytes = kBarOff + 256 + 1024;
 static_assert(kDSOff % 1024 == 0, "128-byte swizzled operand must be 1024-byte aligned");
@@ -538,13 +538,10 @@ __global__ void __launch_bounds__(kThreads, 1) main_kernel(const __grid_constant
     const float sl2 = g.scale_log2;
     float2* tab = reinterpret_cast<float2*>(smem + kTabOff);
     const float2* rtab = prm.theta ? tab : nullptr;
-    float* lse2v = reinterpret_cast<float*>(smem + kVecOff);
-    float* dvec = lse2v + kTile;
+    float* vec = reinterpret_cast<float*>(smem + kVecOff);  // buffer b: lse2 at [256 b], D at [256 b + 128]
     uint8_t* ds = smem + kDSOff;
     uint8_t* kh[2] = {smem + kKOff, smem + kKOff + kTileBytes};
     uint8_t* vt = smem + kVOff;
-    uint8_t* qh[2] = {smem + kQOff, smem + kQOff + kTileBytes};
-    uint8_t* dot = smem + kDOOff;
     float* acc_all = reinterpret_cast<float*>(prm.ws + prm.L.acc);
     uint32_t gph = 0, sph = 0, mph = 0;
     int tab_head = -1;
@@ -596,42 +593,61 @@ __global__ void __launch_bounds__(kThreads, 1) main_kernel(const __grid_constant
         __syncwarp();
         prep_row(kh[0], r, ki, kj, rtab);
         bool first = true;
-        for (int n = 0; n < I.nq && ok; ++n) {
-            if (!bwd_active(g, I, n)) continue;
-            const long long T = I.q0 + n;
-            // this thread's query row: Q, dO rows, Q rotated, the query factors, D and lse2 - e
-            int qi, qj;
+        // Query steps, double-buffered: the copies, factors, D and lse2 of the next
+        // active query tile are issued while the current step's products run.
+        auto stage = [&](int n, int b, int& qi, int& qj, bool& qvalid) {
             long long qtok;
-            const bool qvalid = slot_token(g, T, r, I.h, &qi, &qj, &qtok);
-            copy_rows(qh[0], prm.q, qtok, qvalid, warp, lane);
-            copy_rows(dot, prm.dout, qtok, qvalid, warp, lane);
+            qvalid = slot_token(g, I.q0 + n, r, I.h, &qi, &qj, &qtok);
+            uint8_t* qb = smem + kBufOff + b * kBufBytes;
+            copy_rows(qb, prm.q, qtok, qvalid, warp, lane);
+            copy_rows(qb + 2 * kTileBytes, prm.dout, qtok, qvalid, warp, lane);
             cp_async_commit();
-            fill_factor(qh[1], r, uh + (qi * g.M + qj) * 16, kSqrtD);
+            fill_factor(qb + kTileBytes, r, uh + (qi * g.M + qj) * 16, kSqrtD);
             float D = 0.f;
             if (qvalid) {
-                float a[32], b[32];
+                float a[32], c[32];
                 load_row32(prm.o, qtok, a);
-                load_row32(prm.dout, qtok, b);
+                load_row32(prm.dout, qtok, c);
 #pragma unroll
-                for (int e = 0; e < 32; ++e) D = fmaf(a[e], b[e], D);
+                for (int e = 0; e < 32; ++e) D = fmaf(a[e], c[e], D);
             }
-            dvec[r] = D;
-            lse2v[r] = qvalid ? __ldg(prm.lse + qtok) * 1.4426950408889634f - static_cast<float>(gexp) : INFINITY;
+            vec[256 * b + kTile + r] = D;
+            vec[256 * b + r] = qvalid ? __ldg(prm.lse + qtok) * 1.4426950408889634f - static_cast<float>(gexp)
+                                      : INFINITY;
+        };
+        auto next_active = [&](int n) {
+            while (n < I.nq && !bwd_active(g, I, n)) ++n;
+            return n;
+        };
+        int n = next_active(0), b = 0, qi = 0, qj = 0;
+        bool qvalid = false;
+        if (n < I.nq) stage(n, 0, qi, qj, qvalid);
+        while (n < I.nq && ok) {
+            const long long T = I.q0 + n;
+            const int nn = next_active(n + 1);
+            const int qoff = kBufOff + b * kBufBytes, dooff = qoff + 2 * kTileBytes;
+            const float* lse2v = vec + 256 * b;
+            const float* dvec = lse2v + kTile;
             cp_async_wait<0>();
             __syncwarp();
-            prep_row(qh[0], r, qi, qj, rtab);
+            prep_row(smem + qoff, r, qi, qj, rtab);
             fence_proxy_async_smem();
             if (!group_sync(0x6404)) { ok = false; break; }  // rows staged and rotated
             if (r == 0) {
                 tc_fence_after();
 #pragma unroll
                 for (int k = 0; k < kHeadDim / 16; ++k) {
-                    umma_ss(tmem + kColS, dK0 + u16(kKOff) + 2 * k, dK0 + u16(kQOff) + 2 * k, id_s, k > 0);
-                    umma_ss(tmem + kColDP, dK0 + u16(kVOff) + 2 * k, dK0 + u16(kDOOff) + 2 * k, id_dp, k > 0);
+                    umma_ss(tmem + kColS, dK0 + u16(kKOff) + 2 * k, dK0 + u16(qoff) + 2 * k, id_s, k > 0);
+                    umma_ss(tmem + kColDP, dK0 + u16(kVOff) + 2 * k, dK0 + u16(dooff) + 2 * k, id_dp, k > 0);
                 }
-                umma_ss(tmem + kColS, dK0 + u16(kKOff + kTileBytes), dK0 + u16(kQOff + kTileBytes), id_s, 1u);
+                umma_ss(tmem + kColS, dK0 + u16(kKOff + kTileBytes), dK0 + u16(qoff + kTileBytes), id_s, 1u);
                 umma_commit(&bars->s_full);
             }
+            // the next step's rows go to the other buffer, whose products (the previous
+            // step's) have completed
+            int nqi = 0, nqj = 0;
+            bool nqvalid = false;
+            if (nn < I.nq) stage(nn, b ^ 1, nqi, nqj, nqvalid);
             const uint32_t a16 = I.masked ? d_allow16(g, keyseg, T, I.win) : 0xFFu;
             if (!wwait(&bars->s_full, sph, 0x6405)) { ok = false; break; }
             sph ^= 1;
@@ -684,14 +700,14 @@ __global__ void __launch_bounds__(kThreads, 1) main_kernel(const __grid_constant
                 const uint32_t acc = first ? 0u : 1u;
 #pragma unroll
                 for (int k = 0; k < kTile / 16; ++k)
-                    umma_ts(tmem + kColDV, tmem + kColP + 8 * k, dMN0 + u16(kDOOff) + 64 * k, id_dv,
+                    umma_ts(tmem + kColDV, tmem + kColP + 8 * k, dMN0 + u16(dooff) + 64 * k, id_dv,
                             k > 0 ? 1u : acc);
 #pragma unroll
                 for (int hf = 0; hf < 2; ++hf) {
 #pragma unroll
                     for (int k = 0; k < kTile / 16; ++k)
                         umma_ts(tmem + kColDK + kHeadDim * hf, tmem + kColDS + 8 * k,
-                                dMN0 + u16(kQOff + hf * kTileBytes) + 64 * k, id_dk, k > 0 ? 1u : acc);
+                                dMN0 + u16(qoff + hf * kTileBytes) + 64 * k, id_dk, k > 0 ? 1u : acc);
 #pragma unroll
                     for (int k = 0; k < kTile / 16; ++k)
                         umma_ss(tmem + kColDQ + kHeadDim * hf, dDS + 128 * k,
@@ -728,6 +744,11 @@ __global__ void __launch_bounds__(kThreads, 1) main_kernel(const __grid_constant
                                __uint_as_float(v16[e + 2]) * down, __uint_as_float(v16[e + 3]) * down);
             }
             tc_fence_before();  // ordered before the next step's products by its group barrier
+            n = nn;
+            b ^= 1;
+            qi = nqi;
+            qj = nqj;
+            qvalid = nqvalid;
         }
         if (!ok) break;
         // item end: dk (dK' un-rotated) and dv of this key row, the key side of
@@ -779,6 +800,7 @@ __global__ void __launch_bounds__(kThreads, 1) main_kernel(const __grid_constant
         store_rows(prm.dv, vt, ktok, kvalid, warp, lane);
         if (rtab) write_partials(part, reinterpret_cast<float*>(prm.ws + prm.L.part), g, I.h, I.u, 4 + warp, lane);
     }
+    cp_async_wait<0>();  // a step staged before a failed wait: its copies land before the CTA exits
     if (r == 0) {
         umma_commit(&bars->done);
         mbar_wait(&bars->done, 0, ctl, 0x64ff);
@@ -855,23 +877,35 @@ __global__ void __launch_bounds__(256) bias_sum1_kernel(const Params p) {
     }
 }
 
-// Level 2: thread (head, slot sigma, quarter) sums the chunks in order and writes
-// dU (quarters 0-3) or dW (4-7) at the slot's window position t = i M + j.
+// Level 2: warp (head, slot sigma, quarter) sums the chunks, lane l those with
+// c = l mod 32 in increasing order, then the 32 lane sums in a fixed butterfly,
+// and writes dU (quarters 0-3) or dW (4-7) at the slot's window position
+// t = i M + j.
 __global__ void __launch_bounds__(256) bias_sum2_kernel(const Params p) {
     const Geo& g = p.g;
-    const int h = blockIdx.y;
-    const int idx = blockIdx.x * blockDim.x + threadIdx.x;
-    if (idx >= g.N * 8) return;
+    const int lane = threadIdx.x & 31;
+    const long long gw = static_cast<long long>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
+    if (gw >= static_cast<long long>(g.heads) * g.N * 8) return;  // whole warps leave together
+    const int h = static_cast<int>(gw / (g.N * 8));
+    const int idx = static_cast<int>(gw - static_cast<long long>(h) * g.N * 8);
     const int sigma = idx >> 3, qd = idx & 7;
     const float4* red = reinterpret_cast<const float4*>(p.ws + p.L.red);
     float4 s = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (long long c = 0; c < p.L.chunks; ++c) {
+    for (long long c = lane; c < p.L.chunks; c += 32) {
         const float4 a = __ldcg(red + (c * g.heads + h) * static_cast<long long>(g.N) * 8 + idx);
         s.x += a.x;
         s.y += a.y;
         s.z += a.z;
         s.w += a.w;
     }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        s.x += __shfl_xor_sync(0xffffffffu, s.x, o);
+        s.y += __shfl_xor_sync(0xffffffffu, s.y, o);
+        s.z += __shfl_xor_sync(0xffffffffu, s.z, o);
+        s.w += __shfl_xor_sync(0xffffffffu, s.w, o);
+    }
+    if (lane) return;
     int i, j;
     tile_row_pos(g, sigma >> 7, sigma & (kTile - 1), &i, &j);
     float* dst = qd < 4 ? p.du : p.dw;
@@ -967,9 +1001,9 @@ cudaError_t launch_lrbias_bwd(const Geo& g, const LrbPtrs& p, unsigned int* stat
             prm);
         e = cudaGetLastError();
     }
-    if (e == cudaSuccess) {
-        bwd::bias_sum2_kernel<<<dim3(static_cast<unsigned>((g.N * 8 + 255) / 256), static_cast<unsigned>(g.heads)), 256,
-                                0, stream>>>(prm);
+    if (e == cudaSuccess) {  // one warp per (head, slot, quarter), eight warps per block
+        const long long warps = static_cast<long long>(g.heads) * g.N * 8;
+        bwd::bias_sum2_kernel<<<static_cast<unsigned>((warps + 7) / 8), 256, 0, stream>>>(prm);
         e = cudaGetLastError();
     }
     mark(4);

@@ -27,6 +27,15 @@ def allreduce_dtheta(dtheta: torch.Tensor, group=None) -> torch.Tensor:
     return dtheta
 
 
+def allreduce_param_grads(*grads, group=None):
+    """Sum each rank's gradients of parameters shared by the whole batch (theta,
+    the low-rank bias factors) in place."""
+    for g in grads:
+        if g is not None:
+            allreduce_dtheta(g, group)
+    return grads
+
+
 def max_over_ranks(value: float, device, group=None) -> float:
     """The largest value over all ranks (the job's time is its slowest rank's)."""
     if not (dist.is_available() and dist.is_initialized() and dist.get_world_size(group) > 1):

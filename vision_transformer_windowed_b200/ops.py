@@ -184,7 +184,8 @@ def alloc_lrbias_workspace(q: torch.Tensor, M: int, s: int) -> torch.Tensor:
     return torch.empty(max(n, 256), device=q.device, dtype=torch.uint8)
 
 
-def winattn_lrbias_bwd(q, k, v, o, dout, lse, theta, u, w, M: int, s: int, workspace=None):
+def winattn_lrbias_bwd(q, k, v, o, dout, lse, theta, u, w, M: int, s: int, workspace=None, dq=None, dk=None,
+                       dv=None, dtheta=None, du=None, dw=None):
     """dQ, dK, dV, dtheta (None without theta), dU, dW of sum(O * dout)."""
     sh = _shape(q, M, s)
     B, H, W, heads, d = q.shape
@@ -194,9 +195,16 @@ def winattn_lrbias_bwd(q, k, v, o, dout, lse, theta, u, w, M: int, s: int, works
     if theta is not None:
         _check_tensor("theta", theta, (heads, 2, d // 4), torch.float32)
     _check_factors(q, u, w, M)
-    dq, dk, dv = (torch.empty_like(q) for _ in range(3))
-    dtheta = torch.empty_like(theta) if theta is not None else None
-    du, dw = torch.empty_like(u), torch.empty_like(w)
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(q) if dk is None else dk
+    dv = torch.empty_like(q) if dv is None else dv
+    dtheta = (torch.empty_like(theta) if dtheta is None else dtheta) if theta is not None else None
+    du = torch.empty_like(u) if du is None else du
+    dw = torch.empty_like(w) if dw is None else dw
+    for name, t, ref in (("dq", dq, q), ("dk", dk, q), ("dv", dv, q), ("du", du, u), ("dw", dw, w)):
+        _check_tensor(name, t, ref.shape, ref.dtype)
+    if dtheta is not None:
+        _check_tensor("dtheta", dtheta, theta.shape, torch.float32)
     if workspace is None:
         workspace = alloc_lrbias_workspace(q, M, s)
     _lib.fs_winattn_lrbias_bwd(sh, q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), dout.data_ptr(),
