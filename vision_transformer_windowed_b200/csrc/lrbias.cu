@@ -477,7 +477,13 @@ __global__ void __launch_bounds__(128) prep_kernel(const Params p) {
                         fmaxf(fmaxf(nrm_w[0].y, nrm_w[1].y), fmaxf(nrm_w[2].y, nrm_w[3].y)));
 }
 
-constexpr int kThreads = 128;
+// Main kernel: two warpgroups of four warps; warp w serves TMEM lanes (key rows)
+// 32 (w & 3) .. + 31, and the warpgroups split each step's work: the column
+// halves of S^T and dP^T, the staging of rows (q and the U factors, k and its
+// rotation: group 0; dO, D and lse2, v and the W factors: group 1), the dQ' and
+// dU parts of the accumulator rows, and the item's end (dk and the key side of
+// d theta: group 0; dv and the dW share: group 1).
+constexpr int kThreads = 256;
 constexpr int kKOff = 0;                           // K~ half tiles: k' and W
 constexpr int kVOff = kKOff + 2 * kTileBytes;      // V tile
 constexpr int kBufOff = kVOff + kTileBytes;        // two query buffers: Q~ half tiles (q', sqrt(d) U), dO tile
@@ -489,9 +495,11 @@ constexpr int kBarOff = kTabOff + kTabBytes;
 constexpr int kSmemBytes = kBarOff + 256 + 1024;
 static_assert(kDSOff % 1024 == 0, "128-byte swizzled operand must be 1024-byte aligned");
 constexpr uint32_t kTmemCols = 512;
-// S^T [0,128) with P'^T (bf16) over [0,64); dP^T [128,256) with dS'^T (fp16) over
-// [128,192); dQ~ over the consumed [64,128); dV [256,288), dK~ [320,384).
-constexpr uint32_t kColS = 0, kColDP = 128, kColP = 0, kColDS = 128, kColDQ = 64, kColDV = 256, kColDK = 320;
+// S^T [0,128), dP^T [128,256); P'^T (bf16) [384,448) and dS'^T (fp16) [448,512),
+// apart from S^T and dP^T because the two warpgroups read and write different
+// column halves at once; dQ~ over S^T's consumed [64,128); dV [256,288),
+// dK~ [320,384).
+constexpr uint32_t kColS = 0, kColDP = 128, kColP = 384, kColDS = 448, kColDQ = 64, kColDV = 256, kColDK = 320;
 
 struct Bars {
     uint64_t s_full, mma_done, grp, done;
@@ -505,12 +513,12 @@ __global__ void __launch_bounds__(kThreads, 1) main_kernel(const __grid_constant
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     Bars* bars = reinterpret_cast<Bars*>(smem + kBarOff);
     const Geo& g = prm.g;
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, r = tid;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
     if (tid == 0) {
         mbar_init(&bars->s_full, 1);
         mbar_init(&bars->mma_done, 1);
-        mbar_init(&bars->grp, 4);
+        mbar_init(&bars->grp, 8);
         mbar_init(&bars->done, 1);
         bars->abort_flag = 0;
         fence_mbar_init();
@@ -522,14 +530,19 @@ __global__ void __launch_bounds__(kThreads, 1) main_kernel(const __grid_constant
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
+    const int wg = warp >> 2, quad = warp & 3;
+    const int r = tid & (kTile - 1);  // this thread's row (TMEM lane)
     const uint32_t tmem = bars->tmem_base;
-    const uint32_t trow = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+    const uint32_t trow = tmem + (static_cast<uint32_t>(quad * 32) << 16);
     const Ctl ctl{prm.status, &bars->abort_flag, prm.limit_ns};
     const uint32_t id_s = make_idesc(kTile, kTile, false, false, true);     // fp16 K~, Q~
     const uint32_t id_dp = make_idesc(kTile, kTile, false, false, false);   // bf16 V, dO
     const uint32_t id_dv = make_idesc(kTile, kHeadDim, false, true, false); // P'^T (TMEM) x dO
-    const uint32_t id_dk = make_idesc(kTile, kHeadDim, false, true, true);  // dS'^T (TMEM) x Q~ half
-    const uint32_t id_dq = make_idesc(kTile, kHeadDim, true, true, true);   // dS' (smem) x K~ half
+    // dK~ and dQ~ take both half tiles in one N = 64 product: the MN-major B
+    // operand's 64-byte swizzle atoms (32 channels) follow each other at the
+    // descriptor's leading byte offset, one half tile apart
+    const uint32_t id_dk = make_idesc(kTile, 2 * kHeadDim, false, true, true);  // dS'^T (TMEM) x Q~
+    const uint32_t id_dq = make_idesc(kTile, 2 * kHeadDim, true, true, true);   // dS' (smem) x K~
     const uint32_t sbase = smem_u32(smem);
     const uint64_t dK0 = make_sdesc(sbase, 16, 512, kSw64);
     const uint64_t dMN0 = make_sdesc(sbase, 8192, 512, kSw64);
@@ -561,7 +574,7 @@ __global__ void __launch_bounds__(kThreads, 1) main_kernel(const __grid_constant
         const BwdItem I = d_bwd_item(g, it);
         if (rtab && I.h != tab_head) {
             if (!group_sync(0x6401)) break;
-            build_table(tab, prm.theta + I.h * 2 * kPairs, g.M, r, kThreads);
+            build_table(tab, prm.theta + I.h * 2 * kPairs, g.M, tid, kThreads);
             if (!group_sync(0x6402)) break;
             tab_head = I.h;
         }
@@ -579,19 +592,23 @@ __global__ void __launch_bounds__(kThreads, 1) main_kernel(const __grid_constant
             }
         }
         const int gexp = grad_scale_exp(mdo, mv);
-        // this thread's key row: K, V rows, K rotated, the key factors
+        // this thread's key row: K rotated (group 0), V and the key factors (group 1)
         int ki, kj;
         long long ktok;
         const bool kvalid = slot_token(g, I.u, r, I.h, &ki, &kj, &ktok);
         const uint32_t keyseg = I.masked ? seg_at(d_tile_segs(g, I.u, I.win), r >> g.lBT) : 0u;
         if (!group_sync(0x6403)) break;  // the previous item's K~, V rows are read by every thread
-        copy_rows(kh[0], prm.k, ktok, kvalid, warp, lane);
-        copy_rows(vt, prm.v, ktok, kvalid, warp, lane);
-        cp_async_commit();
-        fill_factor(kh[1], r, wh + (ki * g.M + kj) * 16, 1.f);
-        cp_async_wait<0>();
-        __syncwarp();
-        prep_row(kh[0], r, ki, kj, rtab);
+        if (wg == 0) {
+            copy_rows(kh[0], prm.k, ktok, kvalid, quad, lane);
+            cp_async_commit();
+            cp_async_wait<0>();
+            __syncwarp();
+            prep_row(kh[0], r, ki, kj, rtab);
+        } else {
+            copy_rows(vt, prm.v, ktok, kvalid, quad, lane);
+            cp_async_commit();
+            fill_factor(kh[1], r, wh + (ki * g.M + kj) * 16, 1.f);
+        }
         bool first = true;
         // Query steps, double-buffered: the copies, factors, D and lse2 of the next
         // active query tile are issued while the current step's products run.
@@ -599,21 +616,25 @@ __global__ void __launch_bounds__(kThreads, 1) main_kernel(const __grid_constant
             long long qtok;
             qvalid = slot_token(g, I.q0 + n, r, I.h, &qi, &qj, &qtok);
             uint8_t* qb = smem + kBufOff + b * kBufBytes;
-            copy_rows(qb, prm.q, qtok, qvalid, warp, lane);
-            copy_rows(qb + 2 * kTileBytes, prm.dout, qtok, qvalid, warp, lane);
-            cp_async_commit();
-            fill_factor(qb + kTileBytes, r, uh + (qi * g.M + qj) * 16, kSqrtD);
-            float D = 0.f;
-            if (qvalid) {
-                float a[32], c[32];
-                load_row32(prm.o, qtok, a);
-                load_row32(prm.dout, qtok, c);
+            if (wg == 0) {
+                copy_rows(qb, prm.q, qtok, qvalid, quad, lane);
+                cp_async_commit();
+                fill_factor(qb + kTileBytes, r, uh + (qi * g.M + qj) * 16, kSqrtD);
+            } else {
+                copy_rows(qb + 2 * kTileBytes, prm.dout, qtok, qvalid, quad, lane);
+                cp_async_commit();
+                float D = 0.f;
+                if (qvalid) {
+                    float a[32], c[32];
+                    load_row32(prm.o, qtok, a);
+                    load_row32(prm.dout, qtok, c);
 #pragma unroll
-                for (int e = 0; e < 32; ++e) D = fmaf(a[e], c[e], D);
+                    for (int e = 0; e < 32; ++e) D = fmaf(a[e], c[e], D);
+                }
+                vec[256 * b + kTile + r] = D;
+                vec[256 * b + r] = qvalid ? __ldg(prm.lse + qtok) * 1.4426950408889634f - static_cast<float>(gexp)
+                                          : INFINITY;
             }
-            vec[256 * b + kTile + r] = D;
-            vec[256 * b + r] = qvalid ? __ldg(prm.lse + qtok) * 1.4426950408889634f - static_cast<float>(gexp)
-                                      : INFINITY;
         };
         auto next_active = [&](int n) {
             while (n < I.nq && !bwd_active(g, I, n)) ++n;
@@ -630,10 +651,10 @@ __global__ void __launch_bounds__(kThreads, 1) main_kernel(const __grid_constant
             const float* dvec = lse2v + kTile;
             cp_async_wait<0>();
             __syncwarp();
-            prep_row(smem + qoff, r, qi, qj, rtab);
+            if (wg == 0) prep_row(smem + qoff, r, qi, qj, rtab);
             fence_proxy_async_smem();
             if (!group_sync(0x6404)) { ok = false; break; }  // rows staged and rotated
-            if (r == 0) {
+            if (tid == 0) {
                 tc_fence_after();
 #pragma unroll
                 for (int k = 0; k < kHeadDim / 16; ++k) {
@@ -652,9 +673,9 @@ __global__ void __launch_bounds__(kThreads, 1) main_kernel(const __grid_constant
             if (!wwait(&bars->s_full, sph, 0x6405)) { ok = false; break; }
             sph ^= 1;
             tc_fence_after();
-            // this key row of P'^T and dS'^T, 32 query columns at a time
+            // this key row of P'^T and dS'^T: the group's 64 query columns, 32 at a time
 #pragma unroll 1
-            for (int c = 0; c < 4; ++c) {
+            for (int c = 2 * wg; c < 2 * wg + 2; ++c) {
                 uint8_t* base = ds + (c >> 1) * 16384 + (r >> 3) * 1024 + (r & 7) * 128;
                 uint32_t sv[32], pv[32];
                 tmem_ld32(trow + kColS + 32 * c, sv);
@@ -695,7 +716,7 @@ __global__ void __launch_bounds__(kThreads, 1) main_kernel(const __grid_constant
             fence_proxy_async_smem();
             tc_fence_before();
             if (!group_sync(0x6406)) { ok = false; break; }  // every row's P'^T, dS'^T and dS' written
-            if (r == 0) {
+            if (tid == 0) {
                 tc_fence_after();
                 const uint32_t acc = first ? 0u : 1u;
 #pragma unroll
@@ -703,45 +724,45 @@ __global__ void __launch_bounds__(kThreads, 1) main_kernel(const __grid_constant
                     umma_ts(tmem + kColDV, tmem + kColP + 8 * k, dMN0 + u16(dooff) + 64 * k, id_dv,
                             k > 0 ? 1u : acc);
 #pragma unroll
-                for (int hf = 0; hf < 2; ++hf) {
+                for (int k = 0; k < kTile / 16; ++k)
+                    umma_ts(tmem + kColDK, tmem + kColDS + 8 * k, dMN0 + u16(qoff) + 64 * k, id_dk,
+                            k > 0 ? 1u : acc);
 #pragma unroll
-                    for (int k = 0; k < kTile / 16; ++k)
-                        umma_ts(tmem + kColDK + kHeadDim * hf, tmem + kColDS + 8 * k,
-                                dMN0 + u16(qoff + hf * kTileBytes) + 64 * k, id_dk, k > 0 ? 1u : acc);
-#pragma unroll
-                    for (int k = 0; k < kTile / 16; ++k)
-                        umma_ss(tmem + kColDQ + kHeadDim * hf, dDS + 128 * k,
-                                dMN0 + u16(kKOff + hf * kTileBytes) + 64 * k, id_dq, k > 0);
-                }
+                for (int k = 0; k < kTile / 16; ++k)
+                    umma_ss(tmem + kColDQ, dDS + 128 * k, dMN0 + u16(kKOff) + 64 * k, id_dq, k > 0);
                 umma_commit(&bars->mma_done);
             }
             first = false;
             if (!wwait(&bars->mma_done, mph, 0x6407)) { ok = false; break; }
             mph ^= 1;
             tc_fence_after();
-            // this query row's dQ' (softmax scale and 2^-e) and dU share (2^-e),
-            // added into its accumulator row
+            // this query row's dQ' (group 0: softmax scale and 2^-e) and dU share
+            // (group 1: 2^-e), added into its accumulator row
             {
                 const float down = exp2i(-gexp);
-                const float sc = prm.scale * down;
                 float* accrow = acc_all + ((static_cast<long long>(I.h) * g.tiles + T) * kTile + r) * 64;
-                uint32_t v[32];
-                tmem_ld32(trow + kColDQ, v);
-                tmem_wait_ld();
-                if (qvalid) {
+                if (wg == 0) {
+                    const float sc = prm.scale * down;
+                    uint32_t v[32];
+                    tmem_ld32(trow + kColDQ, v);
+                    tmem_wait_ld();
+                    if (qvalid) {
 #pragma unroll
-                    for (int e = 0; e < 32; e += 4)
-                        red_add_v4(accrow + e, __uint_as_float(v[e]) * sc, __uint_as_float(v[e + 1]) * sc,
-                                   __uint_as_float(v[e + 2]) * sc, __uint_as_float(v[e + 3]) * sc);
+                        for (int e = 0; e < 32; e += 4)
+                            red_add_v4(accrow + e, __uint_as_float(v[e]) * sc, __uint_as_float(v[e + 1]) * sc,
+                                       __uint_as_float(v[e + 2]) * sc, __uint_as_float(v[e + 3]) * sc);
+                    }
+                } else {
+                    uint32_t v16[16];
+                    tmem_ld16(trow + kColDQ + kHeadDim, v16);
+                    tmem_wait_ld();
+                    // a padded token's row adds nothing: its dS' row is zero (lse2 = +inf)
+#pragma unroll
+                    for (int e = 0; e < 16; e += 4)
+                        red_add_v4(accrow + 32 + e, __uint_as_float(v16[e]) * down,
+                                   __uint_as_float(v16[e + 1]) * down, __uint_as_float(v16[e + 2]) * down,
+                                   __uint_as_float(v16[e + 3]) * down);
                 }
-                uint32_t v16[16];
-                tmem_ld16(trow + kColDQ + kHeadDim, v16);
-                tmem_wait_ld();
-                // a padded token's row adds nothing: its dS' row is zero (lse2 = +inf)
-#pragma unroll
-                for (int e = 0; e < 16; e += 4)
-                    red_add_v4(accrow + 32 + e, __uint_as_float(v16[e]) * down, __uint_as_float(v16[e + 1]) * down,
-                               __uint_as_float(v16[e + 2]) * down, __uint_as_float(v16[e + 3]) * down);
             }
             tc_fence_before();  // ordered before the next step's products by its group barrier
             n = nn;
@@ -751,13 +772,18 @@ __global__ void __launch_bounds__(kThreads, 1) main_kernel(const __grid_constant
             qvalid = nqvalid;
         }
         if (!ok) break;
-        // item end: dk (dK' un-rotated) and dv of this key row, the key side of
-        // d theta, and the row's dW share
+        // item end: group 0 dk (dK' un-rotated) and the key side of d theta, group 1
+        // dv and the row's dW share
         const float down = exp2i(-gexp);
         float part[16];
 #pragma unroll
         for (int e = 0; e < 16; ++e) part[e] = 0.f;
-        if (!first) {
+        if (first) {  // no query tile attends these keys (cannot happen: a key attends itself)
+            float z[32];
+#pragma unroll
+            for (int e = 0; e < 32; ++e) z[e] = 0.f;
+            store_row_swz(wg == 0 ? kh[0] : vt, r, z);
+        } else if (wg == 0) {
             uint32_t t[32];
             float dx[32], x[32];
             tmem_ld32(trow + kColDK, t);
@@ -770,38 +796,36 @@ __global__ void __launch_bounds__(kThreads, 1) main_kernel(const __grid_constant
                 rope_row(dx, ki, kj, rtab, true);
             }
             store_row_swz(kh[0], r, dx);  // dk (bf16), staged over k'
-            {
-                uint32_t t16[16];
-                tmem_ld16(trow + kColDK + kHeadDim, t16);
-                tmem_wait_ld();
-                float4* dst = reinterpret_cast<float4*>(
-                    acc_all + ((static_cast<long long>(I.h) * g.tiles + I.u) * kTile + r) * 64 + 48);
-                const float f = prm.scale * down;
+        } else {
+            uint32_t t16[16];
+            tmem_ld16(trow + kColDK + kHeadDim, t16);
+            tmem_wait_ld();
+            float4* dst = reinterpret_cast<float4*>(
+                acc_all + ((static_cast<long long>(I.h) * g.tiles + I.u) * kTile + r) * 64 + 48);
+            const float f = prm.scale * down;
 #pragma unroll
-                for (int c = 0; c < 4; ++c)
-                    dst[c] = make_float4(__uint_as_float(t16[4 * c]) * f, __uint_as_float(t16[4 * c + 1]) * f,
-                                         __uint_as_float(t16[4 * c + 2]) * f, __uint_as_float(t16[4 * c + 3]) * f);
-            }
+            for (int c = 0; c < 4; ++c)
+                dst[c] = make_float4(__uint_as_float(t16[4 * c]) * f, __uint_as_float(t16[4 * c + 1]) * f,
+                                     __uint_as_float(t16[4 * c + 2]) * f, __uint_as_float(t16[4 * c + 3]) * f);
+            uint32_t t[32];
+            float x[32];
             tmem_ld32(trow + kColDV, t);
             tmem_wait_ld();
 #pragma unroll
             for (int e = 0; e < 32; ++e) x[e] = __uint_as_float(t[e]) * down;
             store_row_swz(vt, r, x);  // dv, staged over v
-        } else {  // no query tile attends these keys (cannot happen: a key attends itself)
-            float z[32];
-#pragma unroll
-            for (int e = 0; e < 32; ++e) z[e] = 0.f;
-            store_row_swz(kh[0], r, z);
-            store_row_swz(vt, r, z);
         }
         tc_fence_before();
         __syncwarp();
-        store_rows(prm.dk, kh[0], ktok, kvalid, warp, lane);
-        store_rows(prm.dv, vt, ktok, kvalid, warp, lane);
-        if (rtab) write_partials(part, reinterpret_cast<float*>(prm.ws + prm.L.part), g, I.h, I.u, 4 + warp, lane);
+        if (wg == 0) {
+            store_rows(prm.dk, kh[0], ktok, kvalid, quad, lane);
+            if (rtab) write_partials(part, reinterpret_cast<float*>(prm.ws + prm.L.part), g, I.h, I.u, 4 + quad, lane);
+        } else {
+            store_rows(prm.dv, vt, ktok, kvalid, quad, lane);
+        }
     }
     cp_async_wait<0>();  // a step staged before a failed wait: its copies land before the CTA exits
-    if (r == 0) {
+    if (tid == 0) {
         umma_commit(&bars->done);
         mbar_wait(&bars->done, 0, ctl, 0x64ff);
     }
