@@ -13,8 +13,9 @@
 // A fixed-order two-level sum over the windows of the batch turns the shares
 // into dU and dW.
 //
-// Kernels (plain one-tile pipelines: one CTA of four row warps walks its work
-// items, thread 0 issues the MMAs):
+// Kernels (plain one-tile pipelines: one CTA of row warps walks its work items,
+// four in the forward, eight in the backward's main kernel; thread 0 issues the
+// MMAs):
 //   forward:  item = (query tile, head); the key tiles of its group in turn,
 //             online softmax with O in registers;
 //   backward: prep (per tile and head: the largest |dO row| and |v row| for the

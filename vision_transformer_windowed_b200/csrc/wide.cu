@@ -7,17 +7,18 @@
 // position j with theta[h][0][k], those of the second half by the row position i
 // with theta[h][1][k], k = 0 .. 15.
 //
-// The kernels are plain one-tile pipelines (one CTA of four row warps walks its
-// work items; thread 0 issues the MMAs): copies, rotation, products and softmax
-// follow each other without overlap across items.
+// The kernels are plain one-tile pipelines (one CTA of row warps walks its work
+// items, four in the forward, eight in the backward's main kernel; thread 0
+// issues the MMAs): copies, rotation, products and softmax follow each other
+// without overlap across items.
 //   forward:  item = (query tile, head); the key tiles of its group in turn,
 //             online softmax with O in registers;
 //   backward: prep (per tile and head: the largest |dO row| and |v row| for the
-//             gradient scaling, zeroed dQ' accumulator), main (item = (key tile,
-//             head); the query tiles of its group in turn: S^T, dP^T, P'^T and
-//             dS'^T, dV and dK' accumulated in TMEM, dQ' added with 16-byte
-//             fp32 vector reductions; dk, dv and the key side of d theta at the
-//             item's end),
+//             gradient scaling, zeroed dQ' accumulator), main (eight warps in two
+//             warpgroups; item = (key tile, head); the query tiles of its group
+//             in turn, double-buffered: S^T, dP^T, P'^T and dS'^T, dV and dK'
+//             accumulated in TMEM, dQ' added with 16-byte fp32 vector
+//             reductions; dk, dv and the key side of d theta at the item's end),
 //             post (dq and the query side of d theta), and the fixed-order
 //             d theta sum of the d = 32 backward.
 #include <cuda.h>
@@ -148,7 +149,9 @@ __global__ void __launch_bounds__(kThreads, 2) fwd_kernel(const __grid_constant_
     const uint32_t trow = tmem + (static_cast<uint32_t>(warp * 32) << 16);
     const Ctl ctl{prm.status, &bars->abort_flag, prm.limit_ns};
     const uint32_t id_s = make_idesc(kTile, kTile, false, false, true);    // fp16 Q', K'
-    const uint32_t id_pv = make_idesc_bf16(kTile, kHeadDim, false, true);  // P (TMEM) x V half
+    // P (TMEM) x V over both half tiles in one N = 64 product (the MN-major
+    // operand's two swizzle atoms one half tile apart)
+    const uint32_t id_pv = make_idesc_bf16(kTile, 2 * kHeadDim, false, true);
     const uint32_t sbase = smem_u32(smem);
     const uint64_t dK0 = make_sdesc(sbase, 16, 512, kSw64);     // K-major, 64-byte rows
     const uint64_t dMN0 = make_sdesc(sbase, 8192, 512, kSw64);  // MN-major, 64-byte rows
@@ -287,11 +290,8 @@ __global__ void __launch_bounds__(kThreads, 2) fwd_kernel(const __grid_constant_
             if (r == 0) {
                 tc_fence_after();
 #pragma unroll
-                for (int hf = 0; hf < kHalves; ++hf)
-#pragma unroll
-                    for (int k = 0; k < kTile / 16; ++k)
-                        umma_ts(tmem + kColO + kHeadDim * hf, tmem + kColP + 8 * k,
-                                dMN0 + ((kVOff + hf * kTileBytes) >> 4) + 64 * k, id_pv, k > 0);
+                for (int k = 0; k < kTile / 16; ++k)
+                    umma_ts(tmem + kColO, tmem + kColP + 8 * k, dMN0 + (kVOff >> 4) + 64 * k, id_pv, k > 0);
                 umma_commit(&bars->o_full);
             }
             if (!wwait(&bars->o_full, oph, 0x6107)) { ok = false; break; }
@@ -448,21 +448,28 @@ __global__ void __launch_bounds__(128) prep_kernel(const Params p) {
                         fmaxf(fmaxf(nrm_w[0].y, nrm_w[1].y), fmaxf(nrm_w[2].y, nrm_w[3].y)));
 }
 
-constexpr int kThreads = 128;
-constexpr int kKOff = 0;                             // K' half tiles
-constexpr int kVOff = kKOff + kHalves * kTileBytes;  // V half tiles
-constexpr int kQOff = kVOff + kHalves * kTileBytes;  // Q' half tiles
-constexpr int kDOOff = kQOff + kHalves * kTileBytes; // dO half tiles
-constexpr int kDSOff = kDOOff + kHalves * kTileBytes;  // dS, MN-major 128-byte swizzle (1024-aligned)
-constexpr int kVecOff = kDSOff + 4 * kTileBytes;       // lse2[128], D[128]
-constexpr int kTabOff = kVecOff + 2 * kTile * 4;
+// Main kernel: two warpgroups of four warps; warp w serves TMEM lanes (key rows)
+// 32 (w & 3) .. + 31, and the warpgroups split each step's work: the column
+// halves of S^T and dP^T, the row staging (k and q with their rotation: group
+// 0; v, dO, D and lse2: group 1), the two 32-channel halves of dQ', and the
+// item's end (dk and d theta: group 0; dv: group 1).
+constexpr int kThreads = 256;
+constexpr int kKOff = 0;                               // K' half tiles
+constexpr int kVOff = kKOff + kHalves * kTileBytes;    // V half tiles
+constexpr int kBufOff = kVOff + kHalves * kTileBytes;  // two query buffers: Q' half tiles, dO half tiles
+constexpr int kBufBytes = 2 * kHalves * kTileBytes;
+constexpr int kDSOff = kBufOff + 2 * kBufBytes;        // dS', MN-major 128-byte swizzle (1024-aligned)
+constexpr int kVecOff = kDSOff + 4 * kTileBytes;       // per buffer: lse2[128], D[128]
+constexpr int kTabOff = kVecOff + 2 * 2 * kTile * 4;
 constexpr int kBarOff = kTabOff + kTabBytes;
 constexpr int kSmemBytes = kBarOff + 256 + 1024;
 static_assert(kDSOff % 1024 == 0, "128-byte swizzled operand must be 1024-byte aligned");
 constexpr uint32_t kTmemCols = 512;
-// S^T [0,128) with P'^T (bf16) over [0,64); dP^T [128,256) with dS'^T (fp16) over
-// [128,192); dQ' over the consumed [64,128); dV [256,320), dK' [320,384).
-constexpr uint32_t kColS = 0, kColDP = 128, kColP = 0, kColDS = 128, kColDQ = 64, kColDV = 256, kColDK = 320;
+// S^T [0,128), dP^T [128,256); dV [256,320), dK' [320,384); P'^T (bf16) [384,448)
+// and dS'^T (fp16) [448,512), apart from S^T and dP^T because the two
+// warpgroups read and write different column halves at once; dQ' over S^T's
+// consumed [64,128).
+constexpr uint32_t kColS = 0, kColDP = 128, kColDV = 256, kColDK = 320, kColP = 384, kColDS = 448, kColDQ = 64;
 
 struct Bars {
     uint64_t s_full, mma_done, grp, done;
@@ -476,12 +483,12 @@ __global__ void __launch_bounds__(kThreads, 1) main_kernel(const __grid_constant
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     Bars* bars = reinterpret_cast<Bars*>(smem + kBarOff);
     const Geo& g = prm.g;
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, r = tid;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
     if (tid == 0) {
         mbar_init(&bars->s_full, 1);
         mbar_init(&bars->mma_done, 1);
-        mbar_init(&bars->grp, 4);
+        mbar_init(&bars->grp, 8);
         mbar_init(&bars->done, 1);
         bars->abort_flag = 0;
         fence_mbar_init();
@@ -493,14 +500,19 @@ __global__ void __launch_bounds__(kThreads, 1) main_kernel(const __grid_constant
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
+    const int wg = warp >> 2, quad = warp & 3;
+    const int r = tid & (kTile - 1);  // this thread's row (TMEM lane)
     const uint32_t tmem = bars->tmem_base;
-    const uint32_t trow = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+    const uint32_t trow = tmem + (static_cast<uint32_t>(quad * 32) << 16);
     const Ctl ctl{prm.status, &bars->abort_flag, prm.limit_ns};
-    const uint32_t id_s = make_idesc(kTile, kTile, false, false, true);     // fp16 K', Q'
-    const uint32_t id_dp = make_idesc(kTile, kTile, false, false, false);   // bf16 V, dO
-    const uint32_t id_dv = make_idesc(kTile, kHeadDim, false, true, false); // P'^T (TMEM) x dO half
-    const uint32_t id_dk = make_idesc(kTile, kHeadDim, false, true, true);  // dS'^T (TMEM) x Q' half
-    const uint32_t id_dq = make_idesc(kTile, kHeadDim, true, true, true);   // dS' (smem) x K' half
+    const uint32_t id_s = make_idesc(kTile, kTile, false, false, true);    // fp16 K', Q'
+    const uint32_t id_dp = make_idesc(kTile, kTile, false, false, false);  // bf16 V, dO
+    // the gradient products take both half tiles in one N = 64 product: the
+    // MN-major B operand's 64-byte swizzle atoms (32 channels) follow each other
+    // at the descriptor's leading byte offset, one half tile apart
+    const uint32_t id_dv = make_idesc(kTile, 64, false, true, false);  // P'^T (TMEM) x dO
+    const uint32_t id_dk = make_idesc(kTile, 64, false, true, true);   // dS'^T (TMEM) x Q'
+    const uint32_t id_dq = make_idesc(kTile, 64, true, true, true);    // dS' (smem) x K'
     const uint32_t sbase = smem_u32(smem);
     const uint64_t dK0 = make_sdesc(sbase, 16, 512, kSw64);
     const uint64_t dMN0 = make_sdesc(sbase, 8192, 512, kSw64);
@@ -508,13 +520,11 @@ __global__ void __launch_bounds__(kThreads, 1) main_kernel(const __grid_constant
     auto u16 = [](int bytes) { return static_cast<uint64_t>(bytes >> 4); };
     const float sl2 = g.scale_log2;
     float2* tab = reinterpret_cast<float2*>(smem + kTabOff);
-    float* lse2v = reinterpret_cast<float*>(smem + kVecOff);
-    float* dvec = lse2v + kTile;
+    float* vec = reinterpret_cast<float*>(smem + kVecOff);  // buffer b: lse2 at [256 b], D at [256 b + 128]
     uint8_t* ds = smem + kDSOff;
     uint8_t* kh[2] = {smem + kKOff, smem + kKOff + kTileBytes};
     uint8_t* vh[2] = {smem + kVOff, smem + kVOff + kTileBytes};
-    uint8_t* qh[2] = {smem + kQOff, smem + kQOff + kTileBytes};
-    uint8_t* doh[2] = {smem + kDOOff, smem + kDOOff + kTileBytes};
+    float* dqacc = reinterpret_cast<float*>(prm.ws + prm.L.dqacc);
     uint32_t gph = 0, sph = 0, mph = 0;
     int tab_head = -1;
     bool ok = true;
@@ -528,21 +538,21 @@ __global__ void __launch_bounds__(kThreads, 1) main_kernel(const __grid_constant
         gph ^= 1;
         return passed;
     };
-    auto rotate_row = [&](uint8_t* const* h2, int pi, int pj) {
+    auto rotate_row = [&](uint8_t* h0, uint8_t* h1, int pi, int pj) {
         float x[32];
-        load_row_swz(h2[0], r, x, false);
+        load_row_swz(h0, r, x, false);
         rope_half(x, pj, tab, false);
-        store_row_swz(h2[0], r, x, true);
-        load_row_swz(h2[1], r, x, false);
+        store_row_swz(h0, r, x, true);
+        load_row_swz(h1, r, x, false);
         rope_half(x, pi, tab + kPairs * 64, false);
-        store_row_swz(h2[1], r, x, true);
+        store_row_swz(h1, r, x, true);
     };
 
     for (long long it = blockIdx.x; it < prm.items && ok; it += gridDim.x) {
         const BwdItem I = d_bwd_item(g, it);
         if (I.h != tab_head) {
             if (!group_sync(0x6201)) break;
-            build_table(tab, prm.theta + I.h * 2 * kPairs, g.M, r, kThreads);
+            build_table(tab, prm.theta + I.h * 2 * kPairs, g.M, tid, kThreads);
             if (!group_sync(0x6202)) break;
             tab_head = I.h;
         }
@@ -558,64 +568,91 @@ __global__ void __launch_bounds__(kThreads, 1) main_kernel(const __grid_constant
             }
         }
         const int gexp = grad_scale_exp(mdo, mv);
-        // this thread's key row: K, V rows, K rotated
+        // this thread's key row: K rotated (group 0), V (group 1)
         int ki, kj;
         long long ktok;
         const bool kvalid = slot_token(g, I.u, r, I.h, &ki, &kj, &ktok);
         const uint32_t keyseg = I.masked ? seg_at(d_tile_segs(g, I.u, I.win), r >> g.lBT) : 0u;
         if (!group_sync(0x6203)) break;  // the previous item's K', V rows are read by every thread
-        copy_rows(kh[0], kh[1], prm.k, ktok, kvalid, warp, lane);
-        copy_rows(vh[0], vh[1], prm.v, ktok, kvalid, warp, lane);
-        cp_async_commit();
-        cp_async_wait<0>();
-        __syncwarp();
-        rotate_row(kh, ki, kj);
-        bool first = true;
-        for (int n = 0; n < I.nq && ok; ++n) {
-            if (!bwd_active(g, I, n)) continue;
-            const long long T = I.q0 + n;
-            // this thread's query row: Q, dO rows, Q rotated, D and lse2 - e
-            int qi, qj;
-            long long qtok;
-            const bool qvalid = slot_token(g, T, r, I.h, &qi, &qj, &qtok);
-            copy_rows(qh[0], qh[1], prm.q, qtok, qvalid, warp, lane);
-            copy_rows(doh[0], doh[1], prm.dout, qtok, qvalid, warp, lane);
+        if (wg == 0) {
+            copy_rows(kh[0], kh[1], prm.k, ktok, kvalid, quad, lane);
             cp_async_commit();
-            float D = 0.f;
-            if (qvalid) {
-                float a0[32], a1[32], b0[32], b1[32];
-                load_row64(prm.o, qtok, a0, a1);
-                load_row64(prm.dout, qtok, b0, b1);
-#pragma unroll
-                for (int e = 0; e < 32; ++e) D = fmaf(a0[e], b0[e], fmaf(a1[e], b1[e], D));
-            }
-            dvec[r] = D;
-            lse2v[r] = qvalid ? __ldg(prm.lse + qtok) * 1.4426950408889634f - static_cast<float>(gexp) : INFINITY;
             cp_async_wait<0>();
             __syncwarp();
-            rotate_row(qh, qi, qj);
+            rotate_row(kh[0], kh[1], ki, kj);
+        } else {
+            copy_rows(vh[0], vh[1], prm.v, ktok, kvalid, quad, lane);
+            cp_async_commit();
+        }
+        bool first = true;
+        // Query steps, double-buffered: the copies, D and lse2 of the next active
+        // query tile are issued while the current step's products run.
+        auto stage = [&](int n, int b, int& qi, int& qj, bool& qvalid) {
+            long long qtok;
+            qvalid = slot_token(g, I.q0 + n, r, I.h, &qi, &qj, &qtok);
+            uint8_t* qb = smem + kBufOff + b * kBufBytes;
+            if (wg == 0) {
+                copy_rows(qb, qb + kTileBytes, prm.q, qtok, qvalid, quad, lane);
+                cp_async_commit();
+            } else {
+                copy_rows(qb + 2 * kTileBytes, qb + 3 * kTileBytes, prm.dout, qtok, qvalid, quad, lane);
+                cp_async_commit();
+                float D = 0.f;
+                if (qvalid) {
+                    float a0[32], a1[32], b0[32], b1[32];
+                    load_row64(prm.o, qtok, a0, a1);
+                    load_row64(prm.dout, qtok, b0, b1);
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) D = fmaf(a0[e], b0[e], fmaf(a1[e], b1[e], D));
+                }
+                vec[256 * b + kTile + r] = D;
+                vec[256 * b + r] = qvalid ? __ldg(prm.lse + qtok) * 1.4426950408889634f - static_cast<float>(gexp)
+                                          : INFINITY;
+            }
+        };
+        auto next_active = [&](int n) {
+            while (n < I.nq && !bwd_active(g, I, n)) ++n;
+            return n;
+        };
+        int n = next_active(0), b = 0, qi = 0, qj = 0;
+        bool qvalid = false;
+        if (n < I.nq) stage(n, 0, qi, qj, qvalid);
+        while (n < I.nq && ok) {
+            const long long T = I.q0 + n;
+            const int nn = next_active(n + 1);
+            const int qoff = kBufOff + b * kBufBytes, dooff = qoff + 2 * kTileBytes;
+            const float* lse2v = vec + 256 * b;
+            const float* dvec = lse2v + kTile;
+            cp_async_wait<0>();
+            __syncwarp();
+            if (wg == 0) rotate_row(smem + qoff, smem + qoff + kTileBytes, qi, qj);
             fence_proxy_async_smem();
             if (!group_sync(0x6204)) { ok = false; break; }  // rows staged and rotated
-            if (r == 0) {
+            if (tid == 0) {
                 tc_fence_after();
 #pragma unroll
                 for (int hf = 0; hf < kHalves; ++hf)
 #pragma unroll
                     for (int k = 0; k < kHeadDim / 16; ++k) {
                         umma_ss(tmem + kColS, dK0 + u16(kKOff + hf * kTileBytes) + 2 * k,
-                                dK0 + u16(kQOff + hf * kTileBytes) + 2 * k, id_s, (hf | k) != 0);
+                                dK0 + u16(qoff + hf * kTileBytes) + 2 * k, id_s, (hf | k) != 0);
                         umma_ss(tmem + kColDP, dK0 + u16(kVOff + hf * kTileBytes) + 2 * k,
-                                dK0 + u16(kDOOff + hf * kTileBytes) + 2 * k, id_dp, (hf | k) != 0);
+                                dK0 + u16(dooff + hf * kTileBytes) + 2 * k, id_dp, (hf | k) != 0);
                     }
                 umma_commit(&bars->s_full);
             }
+            // the next step's rows go to the other buffer, whose products (the previous
+            // step's) have completed
+            int nqi = 0, nqj = 0;
+            bool nqvalid = false;
+            if (nn < I.nq) stage(nn, b ^ 1, nqi, nqj, nqvalid);
             const uint32_t a16 = I.masked ? d_allow16(g, keyseg, T, I.win) : 0xFFu;
             if (!wwait(&bars->s_full, sph, 0x6205)) { ok = false; break; }
             sph ^= 1;
             tc_fence_after();
-            // this key row of P'^T and dS'^T, 32 query columns at a time
+            // this key row of P'^T and dS'^T: the group's 64 query columns, 32 at a time
 #pragma unroll 1
-            for (int c = 0; c < 4; ++c) {
+            for (int c = 2 * wg; c < 2 * wg + 2; ++c) {
                 uint8_t* base = ds + (c >> 1) * 16384 + (r >> 3) * 1024 + (r & 7) * 128;
                 uint32_t sv[32], pv[32];
                 tmem_ld32(trow + kColS + 32 * c, sv);
@@ -656,91 +693,90 @@ __global__ void __launch_bounds__(kThreads, 1) main_kernel(const __grid_constant
             fence_proxy_async_smem();
             tc_fence_before();
             if (!group_sync(0x6206)) { ok = false; break; }  // every row's P'^T, dS'^T and dS' written
-            if (r == 0) {
+            if (tid == 0) {
                 tc_fence_after();
                 const uint32_t acc = first ? 0u : 1u;
 #pragma unroll
-                for (int hf = 0; hf < kHalves; ++hf) {
+                for (int k = 0; k < kTile / 16; ++k)
+                    umma_ts(tmem + kColDV, tmem + kColP + 8 * k, dMN0 + u16(dooff) + 64 * k, id_dv,
+                            k > 0 ? 1u : acc);
 #pragma unroll
-                    for (int k = 0; k < kTile / 16; ++k)
-                        umma_ts(tmem + kColDV + kHeadDim * hf, tmem + kColP + 8 * k,
-                                dMN0 + u16(kDOOff + hf * kTileBytes) + 64 * k, id_dv, k > 0 ? 1u : acc);
+                for (int k = 0; k < kTile / 16; ++k)
+                    umma_ts(tmem + kColDK, tmem + kColDS + 8 * k, dMN0 + u16(qoff) + 64 * k, id_dk,
+                            k > 0 ? 1u : acc);
 #pragma unroll
-                    for (int k = 0; k < kTile / 16; ++k)
-                        umma_ts(tmem + kColDK + kHeadDim * hf, tmem + kColDS + 8 * k,
-                                dMN0 + u16(kQOff + hf * kTileBytes) + 64 * k, id_dk, k > 0 ? 1u : acc);
-#pragma unroll
-                    for (int k = 0; k < kTile / 16; ++k)
-                        umma_ss(tmem + kColDQ + kHeadDim * hf, dDS + 128 * k,
-                                dMN0 + u16(kKOff + hf * kTileBytes) + 64 * k, id_dq, k > 0);
-                }
+                for (int k = 0; k < kTile / 16; ++k)
+                    umma_ss(tmem + kColDQ, dDS + 128 * k, dMN0 + u16(kKOff) + 64 * k, id_dq, k > 0);
                 umma_commit(&bars->mma_done);
             }
             first = false;
             if (!wwait(&bars->mma_done, mph, 0x6207)) { ok = false; break; }
             mph ^= 1;
             tc_fence_after();
-            // this query row's dQ', softmax scale and 2^-e applied, added into the accumulator
+            // this query row's dQ' half (the group's 32 channels), softmax scale and
+            // 2^-e applied, added into the accumulator
             {
                 const float sc = prm.scale * exp2i(-gexp);
-                float* accrow = reinterpret_cast<float*>(prm.ws + prm.L.dqacc) +
-                                ((static_cast<long long>(I.h) * g.tiles + T) * kTile + r) * 64;
+                float* accrow = dqacc + ((static_cast<long long>(I.h) * g.tiles + T) * kTile + r) * 64 + 32 * wg;
+                uint32_t v[32];
+                tmem_ld32(trow + kColDQ + kHeadDim * wg, v);
+                tmem_wait_ld();
+                if (qvalid) {
 #pragma unroll
-                for (int hf = 0; hf < kHalves; ++hf) {
-                    uint32_t v[32];
-                    tmem_ld32(trow + kColDQ + kHeadDim * hf, v);
-                    tmem_wait_ld();
-                    if (qvalid) {
-#pragma unroll
-                        for (int e = 0; e < 32; e += 4)
-                            red_add_v4(accrow + 32 * hf + e, __uint_as_float(v[e]) * sc, __uint_as_float(v[e + 1]) * sc,
-                                       __uint_as_float(v[e + 2]) * sc, __uint_as_float(v[e + 3]) * sc);
-                    }
+                    for (int e = 0; e < 32; e += 4)
+                        red_add_v4(accrow + e, __uint_as_float(v[e]) * sc, __uint_as_float(v[e + 1]) * sc,
+                                   __uint_as_float(v[e + 2]) * sc, __uint_as_float(v[e + 3]) * sc);
                 }
             }
             tc_fence_before();  // ordered before the next step's products by its group barrier
+            n = nn;
+            b ^= 1;
+            qi = nqi;
+            qj = nqj;
+            qvalid = nqvalid;
         }
         if (!ok) break;
-        // item end: dk (dK' un-rotated) and dv of this key row, the key side of d theta
+        // item end: group 0 dk (dK' un-rotated) and the key side of d theta, group 1 dv
         const float down = exp2i(-gexp);
         float part[32];
 #pragma unroll
         for (int e = 0; e < 32; ++e) part[e] = 0.f;
-        if (!first) {
-#pragma unroll 1
-            for (int hf = 0; hf < kHalves; ++hf) {
-                uint32_t t[32];
-                tmem_ld32(trow + kColDK + kHeadDim * hf, t);
-                tmem_wait_ld();
-                float dx[32], x[32];
-#pragma unroll
-                for (int e = 0; e < 32; ++e) dx[e] = __uint_as_float(t[e]) * (prm.scale * down);
-                load_row_swz(kh[hf], r, x, true);  // rotated k' (fp16)
-                if (kvalid) dtheta_terms(part, dx, x, static_cast<float>(hf ? ki : kj), hf);
-                rope_half(dx, hf ? ki : kj, tab + hf * kPairs * 64, true);
-                store_row_swz(kh[hf], r, dx);  // dk (bf16), staged over k'
-                tmem_ld32(trow + kColDV + kHeadDim * hf, t);
-                tmem_wait_ld();
-#pragma unroll
-                for (int e = 0; e < 32; ++e) x[e] = __uint_as_float(t[e]) * down;
-                store_row_swz(vh[hf], r, x);  // dv, staged over v
-            }
-        } else {  // no query tile attends these keys (cannot happen: a key attends itself)
+        uint8_t* const* st = wg == 0 ? kh : vh;
+        if (first) {  // no query tile attends these keys (cannot happen: a key attends itself)
             float z[32];
 #pragma unroll
             for (int e = 0; e < 32; ++e) z[e] = 0.f;
-            store_row_swz(kh[0], r, z);
-            store_row_swz(kh[1], r, z);
-            store_row_swz(vh[0], r, z);
-            store_row_swz(vh[1], r, z);
+            store_row_swz(st[0], r, z);
+            store_row_swz(st[1], r, z);
+        } else {
+#pragma unroll 1
+            for (int hf = 0; hf < kHalves; ++hf) {
+                uint32_t t[32];
+                float dx[32];
+                tmem_ld32(trow + (wg == 0 ? kColDK : kColDV) + kHeadDim * hf, t);
+                tmem_wait_ld();
+                if (wg == 0) {
+                    float x[32];
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) dx[e] = __uint_as_float(t[e]) * (prm.scale * down);
+                    load_row_swz(kh[hf], r, x, true);  // rotated k' (fp16)
+                    if (kvalid) dtheta_terms(part, dx, x, static_cast<float>(hf ? ki : kj), hf);
+                    rope_half(dx, hf ? ki : kj, tab + hf * kPairs * 64, true);
+                } else {
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) dx[e] = __uint_as_float(t[e]) * down;
+                }
+                store_row_swz(st[hf], r, dx);  // dk staged over k', dv over v (bf16)
+            }
         }
         tc_fence_before();
         __syncwarp();
-        store_rows(prm.dk, kh[0], kh[1], ktok, kvalid, warp, lane);
-        store_rows(prm.dv, vh[0], vh[1], ktok, kvalid, warp, lane);
-        write_partials(part, reinterpret_cast<float*>(prm.ws + prm.L.part), g, I.h, I.u, 4 + warp, lane);
+        store_rows(wg == 0 ? prm.dk : prm.dv, st[0], st[1], ktok, kvalid, quad, lane);
+        if (wg == 0)
+            write_partials(part, reinterpret_cast<float*>(prm.ws + prm.L.part), g, I.h, I.u, 4 + quad, lane);
     }
-    if (r == 0) {
+    cp_async_wait<0>();  // a step staged before a failed wait: its copies land before the CTA exits
+    if (tid == 0) {
         umma_commit(&bars->done);
         mbar_wait(&bars->done, 0, ctl, 0x62ff);
     }
