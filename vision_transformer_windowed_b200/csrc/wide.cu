@@ -96,10 +96,10 @@ __device__ __forceinline__ void store_rows(uint8_t* dst, const uint8_t* half0, c
 namespace fwd {
 
 constexpr int kThreads = 128;
-constexpr int kQOff = 0;                          // Q' half tiles (then the staged O)
-constexpr int kKOff = kQOff + kHalves * kTileBytes;  // K' half tiles
-constexpr int kVOff = kKOff + kHalves * kTileBytes;  // V half tiles
-constexpr int kTabOff = kVOff + kHalves * kTileBytes;
+constexpr int kQOff = 0;                             // Q' half tiles (then the staged O)
+constexpr int kKVOff = kQOff + kHalves * kTileBytes;  // two key buffers: K' half tiles, V half tiles
+constexpr int kKVBytes = 2 * kHalves * kTileBytes;
+constexpr int kTabOff = kKVOff + 2 * kKVBytes;
 constexpr int kBarOff = kTabOff + kTabBytes;
 constexpr int kSmemBytes = kBarOff + 256 + 1024;  // + alignment of the base
 constexpr uint32_t kTmemCols = 256;
@@ -159,10 +159,6 @@ __global__ void __launch_bounds__(kThreads, 2) fwd_kernel(const __grid_constant_
     float2* tab = reinterpret_cast<float2*>(smem + kTabOff);
     uint8_t* q0 = smem + kQOff;
     uint8_t* q1 = q0 + kTileBytes;
-    uint8_t* k0 = smem + kKOff;
-    uint8_t* k1 = k0 + kTileBytes;
-    uint8_t* v0 = smem + kVOff;
-    uint8_t* v1 = v0 + kTileBytes;
     uint32_t gph = 0, sph = 0, oph = 0;
     int tab_head = -1;
     bool ok = true;
@@ -201,8 +197,24 @@ __global__ void __launch_bounds__(kThreads, 2) fwd_kernel(const __grid_constant_
         const bool qvalid = slot_token(g, I.X, r, I.h, &pi, &pj, &qtok);
         const uint32_t myseg = I.masked ? seg_at(d_tile_segs(g, I.X, I.win), r >> g.lBT) : 0u;
         if (!group_sync(0x6103)) break;  // the previous item's staged O rows are stored
+        // Key tiles, double-buffered: the next active tile's K, V rows are copied
+        // while the current tile's softmax runs.
+        auto kv_stage = [&](int u, int b, int& ki, int& kj) {
+            long long ktok;
+            const bool kvalid = slot_token(g, I.kv0 + u, r, I.h, &ki, &kj, &ktok);
+            uint8_t* kb = smem + kKVOff + b * kKVBytes;
+            copy_rows(kb, kb + kTileBytes, prm.k, ktok, kvalid, warp, lane);
+            copy_rows(kb + 2 * kTileBytes, kb + 3 * kTileBytes, prm.v, ktok, kvalid, warp, lane);
+            cp_async_commit();
+        };
+        auto next_kv = [&](int u) {
+            while (u < I.nkv && !((I.act >> u) & 1u)) ++u;
+            return u;
+        };
         copy_rows(q0, q1, prm.q, qtok, qvalid, warp, lane);
         cp_async_commit();
+        int u = next_kv(0), b = 0, ki = 0, kj = 0;
+        if (u < I.nkv) kv_stage(u, 0, ki, kj);
         cp_async_wait<0>();
         __syncwarp();
         rotate_row(q0, q1, pi, pj);
@@ -210,19 +222,13 @@ __global__ void __launch_bounds__(kThreads, 2) fwd_kernel(const __grid_constant_
 #pragma unroll
         for (int e = 0; e < 64; ++e) o[e] = 0.f;
         float m = -INFINITY, l = 0.f;
-        for (int u = 0; u < I.nkv && ok; ++u) {
-            if (!((I.act >> u) & 1u)) continue;
+        while (u < I.nkv && ok) {
             const long long kt = I.kv0 + u;
-            int ki, kj;
-            long long ktok;
-            const bool kvalid = slot_token(g, kt, r, I.h, &ki, &kj, &ktok);
-            // K, V rows (the previous tile's products have completed: o_full was waited)
-            copy_rows(k0, k1, prm.k, ktok, kvalid, warp, lane);
-            copy_rows(v0, v1, prm.v, ktok, kvalid, warp, lane);
-            cp_async_commit();
+            const int un = next_kv(u + 1);
+            const int koff = kKVOff + b * kKVBytes;
             cp_async_wait<0>();
             __syncwarp();
-            rotate_row(k0, k1, ki, kj);
+            rotate_row(smem + koff, smem + koff + kTileBytes, ki, kj);
             fence_proxy_async_smem();
             if (!group_sync(0x6104)) { ok = false; break; }  // every Q' and K' row rotated
             if (r == 0) {
@@ -232,9 +238,13 @@ __global__ void __launch_bounds__(kThreads, 2) fwd_kernel(const __grid_constant_
 #pragma unroll
                     for (int k = 0; k < kHeadDim / 16; ++k)
                         umma_ss(tmem + kColS, dK0 + ((kQOff + hf * kTileBytes) >> 4) + 2 * k,
-                                dK0 + ((kKOff + hf * kTileBytes) >> 4) + 2 * k, id_s, (hf | k) != 0);
+                                dK0 + ((koff + hf * kTileBytes) >> 4) + 2 * k, id_s, (hf | k) != 0);
                 umma_commit(&bars->s_full);
             }
+            // the next tile's rows go to the other buffer, whose products (the
+            // previous tile's) have completed
+            int nki = 0, nkj = 0;
+            if (un < I.nkv) kv_stage(un, b ^ 1, nki, nkj);
             const uint32_t a16 = I.masked ? d_allow16(g, myseg, kt, I.win) : 0xFFu;
             if (!wwait(&bars->s_full, sph, 0x6105)) { ok = false; break; }
             sph ^= 1;
@@ -291,7 +301,8 @@ __global__ void __launch_bounds__(kThreads, 2) fwd_kernel(const __grid_constant_
                 tc_fence_after();
 #pragma unroll
                 for (int k = 0; k < kTile / 16; ++k)
-                    umma_ts(tmem + kColO, tmem + kColP + 8 * k, dMN0 + (kVOff >> 4) + 64 * k, id_pv, k > 0);
+                    umma_ts(tmem + kColO, tmem + kColP + 8 * k, dMN0 + ((koff + 2 * kTileBytes) >> 4) + 64 * k, id_pv,
+                            k > 0);
                 umma_commit(&bars->o_full);
             }
             if (!wwait(&bars->o_full, oph, 0x6107)) { ok = false; break; }
@@ -306,6 +317,10 @@ __global__ void __launch_bounds__(kThreads, 2) fwd_kernel(const __grid_constant_
                 for (int e = 0; e < 32; ++e) o[32 * hf + e] += __uint_as_float(v[e]);
             }
             tc_fence_before();  // ordered before the next tile's products by its group barrier
+            u = un;
+            b ^= 1;
+            ki = nki;
+            kj = nkj;
         }
         if (!ok) break;
         // epilogue: O / l staged over Q', coalesced stores, log-sum-exp
@@ -323,6 +338,7 @@ __global__ void __launch_bounds__(kThreads, 2) fwd_kernel(const __grid_constant_
         store_rows(prm.o, q0, q1, qtok, qvalid, warp, lane);
         if (qvalid && prm.lse != nullptr) prm.lse[qtok] = (m + lg2_approx(l)) * 0.69314718055994530942f;
     }
+    cp_async_wait<0>();  // a tile staged before a failed wait: its copies land before the CTA exits
     if (r == 0) {  // every MMA issued here has completed before the columns are freed
         umma_commit(&bars->done);
         mbar_wait(&bars->done, 0, ctl, 0x61ff);
