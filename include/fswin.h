@@ -208,7 +208,7 @@ FS_API fs_status fs_selftest_bounded_wait(uint64_t limit_ns, fs_stream_t stream)
  * launch nothing.  Arguments and results are those of fs_winattn_bwd.
  *
  * The first call on a device looks up the array's device address (once per
- * device, synchronously).  All calls on a device share the array: calls whose kernels may overlap on the GPU (other
+ * device).  All calls on a device share the array: calls whose kernels may overlap on the GPU (other
  * streams or host threads without ordering between them) race on it.
  * The address is kept for the life of the process: do not use this entry point
  * (or any other of this library, whose device status word is looked up the same
