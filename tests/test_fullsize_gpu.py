@@ -25,7 +25,7 @@ GRAD_TOL = (3e-2, 5e-3)
 # and the FlashSwin-T stage shapes at 256 x 256 input with patch 2; with a
 # dout_scale (a power of two) the GPU gets dO times it, and its gradients,
 # divided by it, are compared with the oracle's at scale 1 (upstream gradients
-# at the magnitudes of bf16 training, judged at their unit scale)
+# at the magnitudes of bf16 training, compared at their unit scale)
 FULL = [
     ("swin_t_stage1_p4_m8_s0", 128, 64, 64, 3, 8, 0, 1.0),
     ("swin_t_stage1_p4_m8_s4", 128, 64, 64, 3, 8, 4, 1.0),

@@ -5,7 +5,7 @@ Table 2 and Table S1 captions: a trainable rank-16 bias factorization).  The
 small shape lists of the 32-channel parity tests run element by element (every
 window size, shifted and not, ragged tiles, padded grids), with RoPE and
 without it (theta = None on the GPU, theta = 0 for the oracle: the identity
-rotation), plus upstream gradients at training magnitudes judged at unit scale,
+rotation), plus upstream gradients at training magnitudes compared at unit scale,
 a sharpened softmax, and full-size FlashBias-T stage shapes on sampled windows
 (du and dw through dO kept on the sampled windows only: the other windows'
 shares are then zero, so the totals are the sampled units' sums).

@@ -40,7 +40,7 @@ def run_both(B, H, W, h, M, s, qk_scale=1.0, dout_scale=1.0):
     """The CUDA path and the oracle on the same seeded inputs.  With dout_scale
     (a power of two) the CUDA path gets dO * dout_scale, its gradients are
     divided by dout_scale (both exact in binary floating point), and the oracle
-    runs at scale 1: the comparison is then judged at the gradients' unit scale,
+    runs at scale 1: the comparison is then made at the gradients' unit scale,
     so the absolute term of the tolerance cannot hide an underflow."""
     inp = make_inputs(B, H, W, h, 32, qk_scale=qk_scale)
     dev = {k: v.cuda() for k, v in inp.items()}

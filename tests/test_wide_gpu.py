@@ -2,7 +2,7 @@
 
 The same shape lists as the 32-channel parity tests (every window size, shifted
 and not, ragged tiles, padded grids), element by element, with the same
-tolerances; plus upstream gradients at training magnitudes judged at their unit
+tolerances; plus upstream gradients at training magnitudes compared at their unit
 scale, and a sharpened softmax.
 """
 import numpy as np
