@@ -189,7 +189,8 @@ def _sample_units(B, H, W, heads, M, n_random=5, seed=11):
     rng = np.random.default_rng(seed)
     for _ in range(n_random):
         picks.add((int(rng.integers(B)), int(rng.integers(nWh)), int(rng.integers(nWw))))
-    return np.array(sorted((b * nW + wr * nWw + wc) * heads + h for b, wr, wc in picks for h in range(heads)),
+    hs = range(heads) if heads <= 3 else (0, heads // 2, heads - 1)
+    return np.array(sorted((b * nW + wr * nWw + wc) * heads + h for b, wr, wc in picks for h in hs),
                     dtype=np.int64)
 
 
@@ -199,6 +200,9 @@ FULL = [
     ("flashbias_t_stage1_p2_m32_s16", 128, 128, 128, 3, 32, 16),
     ("flashbias_t_stage1_p2_m32_s0", 128, 128, 128, 3, 32, 0),
     ("flashbias_t_stage1_p4_m8_s4", 128, 64, 64, 3, 8, 4),
+    # the later FlashSwin-T stages at p = 2: more heads, the window covering the grid
+    ("flashbias_t_stage3_p2_m32_s16", 128, 32, 32, 12, 32, 16),
+    ("flashbias_t_stage4_p2_m16_s0", 128, 16, 16, 24, 16, 0),
 ]
 
 
