@@ -192,11 +192,13 @@ PHASES = ["fwd", "bwd_prep", "bwd_main", "bwd_post", "bwd_dtheta"]
 def phase_work(st, s) -> dict:
     """Algorithmic work of one block per kernel phase: flops of its products and the bytes it must
     move.  Windows inside one tile run the whole backward as one kernel (Q, K, V, O, dO read, dQ, dK,
-    dV written, LSE and D: 520 B per token-head row, recorded as bwd_main); larger windows run prep /
-    main / post with workspace round trips (prep: q, k, v, o, dO, lse in, q', k' images, lse2, D and
-    the zeroed dQ' accumulator out, 588 B, and the per-window scale pass over lse2, 8 B, timed with
-    it; main: the images, dO, v, lse2, D in, dk, dv out, 392 B; post: the dQ' accumulator and q in, dq
-    out, 256 B)."""
+    dV written, LSE and D: 520 B per token-head row, recorded as bwd_main); larger windows run the
+    training pair: the forward phase writes the rotated q', k' images (q, k in, images out, 256 B)
+    and runs the forward on them (images, v in, o, lse out, 260 B); the backward runs prep / main /
+    post with workspace round trips (prep: v, o, dO, lse in, lse2, D and the zeroed dQ' accumulator
+    out, 332 B, and the per-window scale pass over lse2, 8 B, timed with it; main: the images, dO, v,
+    lse2, D in, dk, dv out, 392 B; post: the dQ' accumulator and q in, dq out, 256 B).  An inference
+    forward reads q, k, v and writes o (256 B)."""
     B, H, W, heads, M, d = st["B"], st["H"], st["W"], st["heads"], st["M"], st.get("d", HEAD_DIM)
     rows = B * H * W * heads
     pairs = unmasked_pairs(B, H, W, heads, M, s)
@@ -215,7 +217,8 @@ def phase_work(st, s) -> dict:
         nbytes = {"fwd": (512 if st.get("infer") else 516) * rows, "bwd_prep": 512 * rows,
                   "bwd_main": 900 * rows, "bwd_post": 512 * rows, "bwd_dtheta": 0}
     else:
-        nbytes = {"fwd": (256 if st.get("infer") else 260) * rows, "bwd_prep": 0 if small else 596 * rows,
+        fwd_row = 256 if st.get("infer") else (260 if small else 516)
+        nbytes = {"fwd": fwd_row * rows, "bwd_prep": 0 if small else 340 * rows,
                   "bwd_main": (520 if small else 392) * rows, "bwd_post": 0 if small else 256 * rows,
                   "bwd_dtheta": 0}
     flops = {"fwd": pf * pairs, "bwd_main": pb * pairs}
@@ -399,16 +402,14 @@ def config_entry(wl, r, peaks, world, name=None) -> dict:
     blocks = blocks_of(wl)
     fwd_ms = r["phase_ms"]["fwd"] * len(blocks)  # per step
     infer = wl.get("infer", False)
-    row_bytes = {32: (256 if infer else 260), 64: (512 if infer else 516)}
     e = {"tflops": r["tflops"], "ms_per_step": r["ms"],
          "pct_bf16_peak": 100 * r["tflops"] / peaks["bf16_tflops"] / world,
          "pct_bf16_spec": 100 * r["tflops"] / SPEC_BF16_TFLOPS / world,
          "fwd_tflops": r["fwd_flops"] * world / (fwd_ms * 1e-3) / 1e12,
          "tokens_per_s": r["tokens_per_s"], "peak_gb": r["peak_gb"], "phase_ms": r["phase_ms"]}
     e["fwd_pct_bf16_peak"] = 100 * e["fwd_tflops"] / peaks["bf16_tflops"] / world
-    # q, k, v read and o written (bf16), plus the fp32 lse of a training forward
-    e["fwd_gbs"] = sum(row_bytes[st["d"]] * st["B"] * st["H"] * st["W"] * st["heads"] for st, _ in blocks) / (
-        fwd_ms * 1e-3) / 1e9
+    # the forward phase's algorithmic bytes (phase_work) over its time
+    e["fwd_gbs"] = sum(phase_work(st, s)["bytes"]["fwd"] for st, s in blocks) / (fwd_ms * 1e-3) / 1e9
     if infer:
         e["step"] = "inference forward (no LSE) at every shift"
     else:
@@ -610,12 +611,13 @@ def main():
                         ops.winattn_lrbias_bwd(q, k, v, o, do, lse, th, t["u"], t["w"], M, s, workspace=ws, dq=dq,
                                                dk=dk, dv=dv, dtheta=dth, du=du, dw=dw)
                         dp.allreduce_param_grads(dth, du, dw)
-                    else:
-                        ops.winattn_fwd(q, k, v, th, M, s, o=o, lse=lse)
+                    else:  # the training pair: the forward leaves the rotated q', k' tiles in ws
+                        ops.winattn_fwd(q, k, v, th, M, s, o=o, lse=lse, workspace=ws)
                         if evs is not None:
                             _lib.fs_set_phase_events([e.cuda_event for e in evs[i][1]])
                         dq, dk, dv, dth = g
-                        ops.winattn_bwd(q, k, v, o, do, lse, th, M, s, workspace=ws, dq=dq, dk=dk, dv=dv, dtheta=dth)
+                        ops.winattn_bwd(q, k, v, o, do, lse, th, M, s, workspace=ws, dq=dq, dk=dk, dv=dv, dtheta=dth,
+                                        after_train_fwd=True)
                         dp.allreduce_dtheta(dth)  # theta is shared by the whole data-parallel batch
                     i += 1
             if evs is not None:
@@ -730,10 +732,11 @@ def main():
                                                                       dvi["theta"], dvi["u"], dvi["w"], M, s)
                     dp.allreduce_param_grads(dth, du, dw)
                     params = (("dtheta", dth), ("du", du), ("dw", dw))
-                else:
-                    o, lse = ops.winattn_fwd(dvi["q"], dvi["k"], dvi["v"], dvi["theta"], M, s)
+                else:  # the training pair, as the autograd wrapper calls it
+                    ws = ops.alloc_workspace(dvi["q"], M, s)
+                    o, lse = ops.winattn_fwd(dvi["q"], dvi["k"], dvi["v"], dvi["theta"], M, s, workspace=ws)
                     dq, dk, dvv, dth = ops.winattn_bwd(dvi["q"], dvi["k"], dvi["v"], o, dvi["dout"], lse, dvi["theta"],
-                                                       M, s)
+                                                       M, s, workspace=ws, after_train_fwd=True)
                     dp.allreduce_dtheta(dth)
                     params = (("dtheta", dth),)
                 outs = (("o", o), ("dq", dq), ("dk", dk), ("dv", dvv)) + params if read_all else params
@@ -790,10 +793,14 @@ def main():
         cpu.pop("seconds", None)
 
     if rank == 0:
-        def launches(st):  # kernels of one block: the forward, then the backward's
+        def launches(st):  # kernels of one block: the forward's, then the backward's
             if st.get("lrbias"):
                 return 1 + 6  # prep, main, post, d theta sum, two dU / dW sum levels
-            return 1 + (4 if st["d"] == 64 else (2 if st["M"] * st["M"] < 128 else 5))
+            if st["d"] == 64:
+                return 1 + 4  # prep, main, post, d theta sum
+            if st["M"] * st["M"] < 128:
+                return 1 + 2  # the one-tile backward, d theta sum
+            return 2 + 5  # q', k' images and the forward; prep, scale, main, post, d theta sum
         nlaunch = sum(launches(st) for st, _ in blocks)
         line = {
             "metric": METRIC, "value": main_res["tflops"], "unit": "TFLOP/s", "n_gpus": world,
@@ -803,8 +810,8 @@ def main():
                            l2="inputs larger than L2 (the largest stage's tensors > 126 MB each)"),
             "pct_bf16_peak": 100 * main_res["tflops"] / peaks["bf16_tflops"] / world,
             "tokens_per_s": main_res["tokens_per_s"], "peak_gb": main_res["peak_gb"],
-            # per block: the forward, then the one-tile backward and the d theta sum (windows
-            # inside one tile) or prep, scale, main, post and the d theta sum
+            # per block: the forward (windows of >= 128 tokens: the rotated q', k' images,
+            # then the forward), then the backward's kernels
             "gpu_launches": args.steps * nlaunch,
             "roofline": roof, "clocks": main_res["clocks"], "e2e": e2e, "e2e_all_outputs": e2e_all, "cpu_baseline": cpu,
             "per_config": per_config, "peaks": peaks,

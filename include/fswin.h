@@ -177,6 +177,30 @@ FS_API fs_status fs_winattn_lrbias_bwd(const fs_winattn_shape* shape, const void
                                        float* dtheta, float* du, float* dw, void* workspace, size_t workspace_bytes,
                                        fs_stream_t stream);
 
+/*
+ * Training pair.  fs_winattn_fwd_train is fs_winattn_fwd (lse required) that
+ * also leaves, in `workspace` (the backward's: at least
+ * fs_winattn_bwd_workspace_bytes(shape) bytes, 256-byte aligned), the rotated
+ * q', k' tiles the backward needs; fs_winattn_bwd_train is fs_winattn_bwd that
+ * takes them from there instead of rotating q and k again.  The forward of
+ * windows of >= 128 tokens (d == 32) then reads its Q', K' tiles from those
+ * images, rotating each row once instead of once per query tile of the window.
+ * Same results as fs_winattn_fwd / fs_winattn_bwd.  Contract: the backward gets
+ * the workspace of the training forward of the same shape, q, k and theta,
+ * unchanged in between (otherwise its gradients are wrong; nothing checks it).
+ * For windows of fewer than 128 tokens and for d == 64 the pair behaves as
+ * fs_winattn_fwd / fs_winattn_bwd (the forward writes nothing to the workspace).
+ * Errors as those of fs_winattn_fwd and fs_winattn_bwd; the forward also
+ * returns FS_ERR_WORKSPACE for a missing, misaligned or short workspace.
+ */
+FS_API fs_status fs_winattn_fwd_train(const fs_winattn_shape* shape, const void* q, const void* k, const void* v,
+                                      const float* theta, void* o, float* lse, void* workspace,
+                                      size_t workspace_bytes, fs_stream_t stream);
+FS_API fs_status fs_winattn_bwd_train(const fs_winattn_shape* shape, const void* q, const void* k, const void* v,
+                                      const void* o, const void* dout, const float* lse, const float* theta,
+                                      void* dq, void* dk, void* dv, float* dtheta, void* workspace,
+                                      size_t workspace_bytes, fs_stream_t stream);
+
 /* Human-readable name of a status. */
 FS_API const char* fs_status_string(fs_status status);
 

@@ -188,3 +188,23 @@ def test_lrbias_workspace_size():
     expect = tokens * 256 + heads * tiles * 8 + heads * tiles * 8 * 16 * 4 + heads * 64 * 16 * 4 + heads * 4 + \
         chunks * heads * M * M * 32 * 4
     assert expect <= n <= expect + 6 * 256
+
+
+def test_train_pair_rejects_before_launch():
+    """The training forward needs lse and the backward's workspace."""
+    sh = _lib.make_shape(1, 64, 64, 2, 32, 32, 16)
+    n = _lib.fs_winattn_bwd_workspace_bytes(sh)
+    p = 256
+
+    def fwd(lse=p, ws=p, nbytes=n):
+        with pytest.raises(_lib.FswinError) as e:
+            _lib.fs_winattn_fwd_train(sh, p, p, p, p, p, lse, ws, nbytes, 0)
+        return e.value.status
+
+    assert fwd(lse=0) == _lib.FS_ERR_NULL
+    assert fwd(ws=0) == _lib.FS_ERR_WORKSPACE
+    assert fwd(ws=p + 16) == _lib.FS_ERR_WORKSPACE
+    assert fwd(nbytes=n - 1) == _lib.FS_ERR_WORKSPACE
+    with pytest.raises(_lib.FswinError) as e:
+        _lib.fs_winattn_bwd_train(sh, *([p] * 11), p, n - 1, 0)
+    assert e.value.status == _lib.FS_ERR_WORKSPACE

@@ -71,6 +71,10 @@ def load(build_if_missing: bool = True):
         lib.fs_winattn_bwd_noalloc.restype = st
         lib.fs_winattn_bwd_noalloc_max_bytes.argtypes = []
         lib.fs_winattn_bwd_noalloc_max_bytes.restype = ctypes.c_size_t
+        lib.fs_winattn_fwd_train.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, ctypes.c_size_t, vp]
+        lib.fs_winattn_fwd_train.restype = st
+        lib.fs_winattn_bwd_train.argtypes = [P] + [vp] * 12 + [ctypes.c_size_t, vp]
+        lib.fs_winattn_bwd_train.restype = st
         lib.fs_winattn_lrbias_fwd.argtypes = [P] + [vp] * 6 + [ctypes.c_int, vp, vp, vp]
         lib.fs_winattn_lrbias_fwd.restype = st
         lib.fs_winattn_lrbias_bwd_workspace_bytes.argtypes = [P]
@@ -116,6 +120,18 @@ def fs_winattn_bwd(shape: Shape, q: int, k: int, v: int, o: int, dout: int, lse:
                    dv: int, dtheta: int, workspace: int, workspace_bytes: int, stream: int) -> None:
     _check(load().fs_winattn_bwd(ctypes.byref(shape), q, k, v, o, dout, lse, theta, dq, dk, dv, dtheta, workspace,
                                  workspace_bytes, stream), "fs_winattn_bwd")
+
+
+def fs_winattn_fwd_train(shape: Shape, q: int, k: int, v: int, theta: int, o: int, lse: int, workspace: int,
+                         workspace_bytes: int, stream: int) -> None:
+    _check(load().fs_winattn_fwd_train(ctypes.byref(shape), q, k, v, theta, o, lse, workspace, workspace_bytes,
+                                       stream), "fs_winattn_fwd_train")
+
+
+def fs_winattn_bwd_train(shape: Shape, q: int, k: int, v: int, o: int, dout: int, lse: int, theta: int, dq: int,
+                         dk: int, dv: int, dtheta: int, workspace: int, workspace_bytes: int, stream: int) -> None:
+    _check(load().fs_winattn_bwd_train(ctypes.byref(shape), q, k, v, o, dout, lse, theta, dq, dk, dv, dtheta,
+                                       workspace, workspace_bytes, stream), "fs_winattn_bwd_train")
 
 
 def fs_winattn_bwd_noalloc(shape: Shape, q: int, k: int, v: int, o: int, dout: int, lse: int, theta: int, dq: int,

@@ -136,8 +136,14 @@ const char* fs_status_string(fs_status st) {
     return "unknown fs_status";
 }
 
-fs_status fs_winattn_fwd(const fs_winattn_shape* shape, const void* q, const void* k, const void* v,
-                         const float* theta, void* o, float* lse, fs_stream_t stream) {
+}  // extern "C"
+
+namespace {
+
+// The forward; train_ws: NULL, or the backward's workspace (already checked),
+// which then receives the rotated q', k' images for the training backward.
+fs_status forward(const fs_winattn_shape* shape, const void* q, const void* k, const void* v, const float* theta,
+                  void* o, float* lse, uint8_t* train_ws, fs_stream_t stream) {
     Geo g;
     fs_status st = make_geo(shape, &g);
     if (st != FS_OK) return st;
@@ -171,8 +177,31 @@ fs_status fs_winattn_fwd(const fs_winattn_shape* shape, const void* q, const voi
     }
     cudaError_t e = launch_fwd(g, mq, mk, mv, mo, q, k, v, o, theta, lse, status, lim, sms,
                                reinterpret_cast<cudaStream_t>(stream),
-                               g_phase_n >= 2 ? g_phase_events : nullptr);
+                               g_phase_n >= 2 ? g_phase_events : nullptr, g.N >= kTile ? train_ws : nullptr);
     return e == cudaSuccess ? FS_OK : FS_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+fs_status fs_winattn_fwd(const fs_winattn_shape* shape, const void* q, const void* k, const void* v,
+                         const float* theta, void* o, float* lse, fs_stream_t stream) {
+    return forward(shape, q, k, v, theta, o, lse, nullptr, stream);
+}
+
+fs_status fs_winattn_fwd_train(const fs_winattn_shape* shape, const void* q, const void* k, const void* v,
+                               const float* theta, void* o, float* lse, void* workspace, size_t workspace_bytes,
+                               fs_stream_t stream) {
+    Geo g;
+    fs_status st = make_geo(shape, &g);
+    if (st != FS_OK) return st;
+    if (g.B == 0) return FS_OK;
+    if (!lse) return FS_ERR_NULL;  // the backward needs it
+    const size_t need = g.d == 64 ? wide_bwd_workspace_bytes(g) : bwd_workspace_bytes(g);
+    if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) || workspace_bytes < need)
+        return FS_ERR_WORKSPACE;
+    return forward(shape, q, k, v, theta, o, lse, g.d == 32 ? static_cast<uint8_t*>(workspace) : nullptr, stream);
 }
 
 fs_status fs_winattn_block_fwd(const fs_winattn_shape* shape, const void* x, const void* w_qkv,
@@ -207,10 +236,13 @@ size_t fs_winattn_bwd_workspace_bytes(const fs_winattn_shape* shape) {
     return g.d == 64 ? wide_bwd_workspace_bytes(g) : bwd_workspace_bytes(g);
 }
 
-fs_status fs_winattn_bwd(const fs_winattn_shape* shape, const void* q, const void* k, const void* v,
-                         const void* o, const void* dout, const float* lse, const float* theta, void* dq,
-                         void* dk, void* dv, float* dtheta, void* workspace, size_t workspace_bytes,
-                         fs_stream_t stream) {
+}  // extern "C"
+
+namespace {
+
+fs_status backward(const fs_winattn_shape* shape, const void* q, const void* k, const void* v, const void* o,
+                   const void* dout, const float* lse, const float* theta, void* dq, void* dk, void* dv,
+                   float* dtheta, void* workspace, size_t workspace_bytes, bool images_ready, fs_stream_t stream) {
     Geo g;
     fs_status st = make_geo(shape, &g);
     if (st != FS_OK) return st;
@@ -256,8 +288,28 @@ fs_status fs_winattn_bwd(const fs_winattn_shape* shape, const void* q, const voi
     }
     BwdPtrs p{q, k, v, o, dout, lse, theta, dq, dk, dv, dtheta, static_cast<uint8_t*>(workspace)};
     cudaError_t e = launch_bwd(g, p, maps, status, lim, sms, reinterpret_cast<cudaStream_t>(stream),
-                               g_phase_n >= 5 ? g_phase_events : nullptr);
+                               g_phase_n >= 5 ? g_phase_events : nullptr, images_ready);
     return e == cudaSuccess ? FS_OK : FS_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+fs_status fs_winattn_bwd(const fs_winattn_shape* shape, const void* q, const void* k, const void* v,
+                         const void* o, const void* dout, const float* lse, const float* theta, void* dq,
+                         void* dk, void* dv, float* dtheta, void* workspace, size_t workspace_bytes,
+                         fs_stream_t stream) {
+    return backward(shape, q, k, v, o, dout, lse, theta, dq, dk, dv, dtheta, workspace, workspace_bytes, false,
+                    stream);
+}
+
+fs_status fs_winattn_bwd_train(const fs_winattn_shape* shape, const void* q, const void* k, const void* v,
+                               const void* o, const void* dout, const float* lse, const float* theta, void* dq,
+                               void* dk, void* dv, float* dtheta, void* workspace, size_t workspace_bytes,
+                               fs_stream_t stream) {
+    return backward(shape, q, k, v, o, dout, lse, theta, dq, dk, dv, dtheta, workspace, workspace_bytes, true,
+                    stream);
 }
 
 fs_status fs_winattn_lrbias_fwd(const fs_winattn_shape* shape, const void* q, const void* k, const void* v,

@@ -61,12 +61,19 @@ __host__ __device__ inline WsLayout ws_layout(const Geo& g) {
     return L;
 }
 
+// What a prep launch does: everything (the backward on its own); only the
+// rotated q', k' images (the training forward, which reads them); everything
+// but the images (the backward after such a forward, whose images are still
+// in the workspace).
+enum PrepMode : int { kPrepFull = 0, kPrepImages = 1, kPrepReuse = 2 };
+
 struct PrepParams {
     Geo g;
     const uint4 *q, *k, *v, *o, *dout;
     const float *lse, *theta;
     uint8_t* ws;
     WsLayout L;
+    int mode;
 };
 
 struct PostParams {
@@ -125,48 +132,58 @@ __global__ void __launch_bounds__(128) prep_kernel(const PrepParams p) {
     __shared__ float2 tab[2 * 64 * 8];
     __shared__ float2 nrm_w[4];
     const Geo& g = p.g;
+    const bool images = p.mode != kPrepReuse, extras = p.mode != kPrepImages;  // uniform over the launch
     // blocks take the heads of a tile in turn (a token's heads share memory
     // lines); ht indexes the workspace images, [head][tile]
     const long long T = blockIdx.x / g.heads;
     const int h = static_cast<int>(blockIdx.x - T * g.heads);
     const long long ht = static_cast<long long>(h) * g.tiles + T;
-    if (blockIdx.x == 0)  // the d theta reduction's counters, for its launch after this one
+    if (extras && blockIdx.x == 0)  // the d theta reduction's counters, for its launch after this one
         for (int i = threadIdx.x; i < g.heads; i += blockDim.x) reinterpret_cast<unsigned int*>(p.ws + p.L.cnt)[i] = 0u;
-    build_table(tab, p.theta + h * 16, g.M, threadIdx.x, blockDim.x);
-    __syncthreads();
+    if (images) {
+        build_table(tab, p.theta + h * 16, g.M, threadIdx.x, blockDim.x);
+        __syncthreads();
+    }
     const int r = threadIdx.x;
     const Slot sl = slot_of(g, T, r);
     float q[32], k[32], dO[32], o[32];
     float D = 0.f, lse2 = INFINITY, ndo = 0.f, nv = 0.f;
     if (sl.valid) {
         const long long tok = ((static_cast<long long>(sl.box.b) * g.H + sl.row) * g.W + sl.col) * g.heads + h;
-        load_row_bf16(p.q + tok * 4, q);
-        load_row_bf16(p.k + tok * 4, k);
-        load_row_bf16(p.dout + tok * 4, dO);
-        load_row_bf16(p.o + tok * 4, o);
-        float acc[4] = {0.f, 0.f, 0.f, 0.f}, n4[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-        for (int e = 0; e < 32; ++e) {
-            acc[e & 3] = fmaf(dO[e], o[e], acc[e & 3]);
-            n4[e & 3] = fmaf(dO[e], dO[e], n4[e & 3]);
+        if (images) {
+            load_row_bf16(p.q + tok * 4, q);
+            load_row_bf16(p.k + tok * 4, k);
+            rope32(q, sl.i, sl.j, tab, false);
+            rope32(k, sl.i, sl.j, tab, false);
         }
-        D = (acc[0] + acc[1]) + (acc[2] + acc[3]);
-        ndo = (n4[0] + n4[1]) + (n4[2] + n4[3]);
-        load_row_bf16(p.v + tok * 4, o);  // o is done with: v's row
+        if (extras) {
+            load_row_bf16(p.dout + tok * 4, dO);
+            load_row_bf16(p.o + tok * 4, o);
+            float acc[4] = {0.f, 0.f, 0.f, 0.f}, n4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-        for (int e = 0; e < 4; ++e) n4[e] = 0.f;
+            for (int e = 0; e < 32; ++e) {
+                acc[e & 3] = fmaf(dO[e], o[e], acc[e & 3]);
+                n4[e & 3] = fmaf(dO[e], dO[e], n4[e & 3]);
+            }
+            D = (acc[0] + acc[1]) + (acc[2] + acc[3]);
+            ndo = (n4[0] + n4[1]) + (n4[2] + n4[3]);
+            load_row_bf16(p.v + tok * 4, o);  // o is done with: v's row
 #pragma unroll
-        for (int e = 0; e < 32; ++e) n4[e & 3] = fmaf(o[e], o[e], n4[e & 3]);
-        nv = (n4[0] + n4[1]) + (n4[2] + n4[3]);
-        lse2 = p.lse[tok] * 1.4426950408889634f;
-        rope32(q, sl.i, sl.j, tab, false);
-        rope32(k, sl.i, sl.j, tab, false);
+            for (int e = 0; e < 4; ++e) n4[e] = 0.f;
+#pragma unroll
+            for (int e = 0; e < 32; ++e) n4[e & 3] = fmaf(o[e], o[e], n4[e & 3]);
+            nv = (n4[0] + n4[1]) + (n4[2] + n4[3]);
+            lse2 = p.lse[tok] * 1.4426950408889634f;
+        }
     } else {
 #pragma unroll
-        for (int e = 0; e < 32; ++e) q[e] = k[e] = dO[e] = 0.f;
+        for (int e = 0; e < 32; ++e) q[e] = k[e] = 0.f;
     }
-    store_row_swz(p.ws + p.L.qimg + ht * kTileBytes, r, q, true);
-    store_row_swz(p.ws + p.L.kimg + ht * kTileBytes, r, k, true);
+    if (images) {
+        store_row_swz(p.ws + p.L.qimg + ht * kTileBytes, r, q, true);
+        store_row_swz(p.ws + p.L.kimg + ht * kTileBytes, r, k, true);
+    }
+    if (!extras) return;
     reinterpret_cast<float*>(p.ws + p.L.lse2)[ht * kTile + r] = lse2;
     reinterpret_cast<float*>(p.ws + p.L.dvec)[ht * kTile + r] = D;
     uint4* acc = reinterpret_cast<uint4*>(p.ws + p.L.dqacc + (ht * kTile + r) * kHeadDim * 4);
@@ -846,11 +863,28 @@ cudaError_t launch_dtheta(const float* part, long long per_head, int heads, floa
 
 size_t bwd_workspace_bytes(const Geo& g) { return bwdk::ws_layout(g).total; }
 
+void bwd_image_offsets(const Geo& g, size_t* qimg, size_t* kimg) {
+    const bwdk::WsLayout L = bwdk::ws_layout(g);
+    *qimg = L.qimg;
+    *kimg = L.kimg;
+}
+
+cudaError_t launch_rope_images(const Geo& g, const void* q, const void* k, const float* theta, uint8_t* ws,
+                               cudaStream_t stream) {
+    using namespace bwdk;
+    const long long ht = static_cast<long long>(g.heads) * g.tiles;
+    PrepParams pp{g, static_cast<const uint4*>(q), static_cast<const uint4*>(k), nullptr, nullptr, nullptr,
+                  nullptr, theta, ws, ws_layout(g), kPrepImages};
+    prep_kernel<<<static_cast<unsigned>(ht), 128, 0, stream>>>(pp);
+    return cudaGetLastError();
+}
+
 long long bwd_items(const Geo& g) { return bwd_item_count(g); }
 
 
 cudaError_t launch_bwd(const Geo& g, const BwdPtrs& p, const BwdMaps& maps, unsigned int* status,
-                       unsigned long long limit_ns, int num_sms, cudaStream_t stream, cudaEvent_t const* events) {
+                       unsigned long long limit_ns, int num_sms, cudaStream_t stream, cudaEvent_t const* events,
+                       bool images_ready) {
     using namespace bwdk;
     const WsLayout L = ws_layout(g);
     const long long ht = static_cast<long long>(g.heads) * g.tiles;
@@ -888,7 +922,8 @@ cudaError_t launch_bwd(const Geo& g, const BwdPtrs& p, const BwdMaps& maps, unsi
                   p.lse,
                   p.theta,
                   p.ws,
-                  L};
+                  L,
+                  images_ready ? kPrepReuse : kPrepFull};
     prep_kernel<<<static_cast<unsigned>(ht), 128, 0, stream>>>(pp);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     scale_kernel<<<static_cast<unsigned>(g.heads * g.wins), 128, 0, stream>>>(g, p.ws, L);

@@ -72,6 +72,9 @@ struct Params {
     Geo g;
     const float* theta;  // [heads][2][8]
     float* lse;          // [B,H,W,heads], or null (inference: not written)
+    // null, or the rotated fp16 q', k' tile images [heads][tiles][128 rows]
+    // (64-byte swizzle): Q', K' are then bulk copies of them, not rotated here
+    const uint8_t *qimg, *kimg;
     unsigned int* status;
     unsigned long long limit_ns;
     long long items;
@@ -111,14 +114,17 @@ __device__ __forceinline__ void rope_row(uint8_t* __restrict__ tile, int r, int 
     for (int c = 0; c < 4; ++c) *reinterpret_cast<uint4*>(row + ((c ^ sw) << 4)) = v[c];
 }
 
-// Rotates this thread's row of one tile and signals the MMA issuer (one arrival
-// per warp): the tile's generic-proxy writes are fenced for the tensor core.
+// Rotates this thread's row of one tile (unless the tile arrived rotated) and
+// signals the MMA issuer (one arrival per warp): the tile's generic-proxy
+// writes are fenced for the tensor core.
 __device__ __forceinline__ void rotate_and_signal(uint8_t* tile, int r, long long tile_idx, const Geo& g,
-                                                  const float2* tab, uint64_t* bar, int lane) {
-    int pi, pj;
-    tile_row_pos(g, tile_idx, r, &pi, &pj);
-    rope_row(tile, r, pi, pj, tab);
-    fence_proxy_async_smem();
+                                                  const float2* tab, uint64_t* bar, int lane, bool rotate) {
+    if (rotate) {
+        int pi, pj;
+        tile_row_pos(g, tile_idx, r, &pi, &pj);
+        rope_row(tile, r, pi, pj, tab);
+        fence_proxy_async_smem();
+    }
     __syncwarp();
     if (lane == 0) mbar_arrive(bar);
 }
@@ -187,7 +193,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const int qi = it & 1;
                 if (!mbar_wait(&B.q_empty[qi], ((it >> 1) & 1) ^ 1, ctl, 0x101)) break;
                 mbar_arrive_expect_tx(&B.q_full[qi], kTileBytes);
-                tile_tma(g, &map_q, smem + q_off(wk) + qi * kTileBytes, &B.q_full[qi], I.X, I.h, false);
+                if (prm.qimg)
+                    bulk_load(smem + q_off(wk) + qi * kTileBytes,
+                              prm.qimg + (static_cast<size_t>(I.h) * g.tiles + static_cast<size_t>(I.X)) * kTileBytes,
+                              kTileBytes, &B.q_full[qi]);
+                else
+                    tile_tma(g, &map_q, smem + q_off(wk) + qi * kTileBytes, &B.q_full[qi], I.X, I.h, false);
                 for (int u = 0; u < I.nkv; ++u) {
                     if (!((I.act >> u) & 1u)) continue;
                     const int st = kvc % kStages;
@@ -196,7 +207,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                     if (!mbar_wait(&B.kv_empty[st], ph ^ 1, ctl, 0x102)) { ok = false; break; }
                     uint8_t* ks = smem + kv_off(wk) + st * 2 * kTileBytes;
                     mbar_arrive_expect_tx(&B.kv_full[st], 2 * kTileBytes);
-                    tile_tma(g, &map_k, ks, &B.kv_full[st], I.kv0 + u, I.h, false);
+                    if (prm.kimg)
+                        bulk_load(ks,
+                                  prm.kimg + (static_cast<size_t>(I.h) * g.tiles + static_cast<size_t>(I.kv0 + u)) *
+                                                 kTileBytes,
+                                  kTileBytes, &B.kv_full[st]);
+                    else
+                        tile_tma(g, &map_k, ks, &B.kv_full[st], I.kv0 + u, I.h, false);
                     tile_tma(g, &map_v, ks + kTileBytes, &B.kv_full[st], I.kv0 + u, I.h, false);
                 }
             }
@@ -278,6 +295,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint8_t* ost = smem + ost_off(wk);
         float2* tab = reinterpret_cast<float2*>(smem + tab_off(wk));
         const bool leader = (quarter == 0 && lane == 0);
+        const bool rotate = prm.qimg == nullptr;  // Q', K' arrive rotated from the images otherwise
         const float sl2 = g.scale_log2;
         uint32_t oph = 0, gph = 0, kvc_rot = 0;
         int tab_head = -1;
@@ -308,7 +326,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             ++kvc_rot;
             if (!wwait(&B.kv_full[st], ph, 0x402)) return false;
             rotate_and_signal(smem + kv_off(wk) + st * 2 * kTileBytes, r, I.kv0 + unext, g, tab, &B.kv_ready[st],
-                              lane);
+                              lane, rotate);
             const uint32_t rest = unext + 1 < 32 ? (I.act >> (unext + 1)) : 0u;
             unext = rest ? unext + __ffs(rest) : -1;
             return true;
@@ -318,7 +336,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // that the item's first S = Q K^T can start.
         auto start_item = [&](long long item, int jt) -> bool {
             I = d_fwd_item(g, item);
-            if (I.h != tab_head) {
+            if (rotate && I.h != tab_head) {
                 if (!group_sync(0x406)) return false;  // rotations with the old table done
                 tab_head = I.h;
                 const float* th = prm.theta + I.h * 16;
@@ -334,7 +352,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             unext = __ffs(I.act) - 1;
             const int qi = jt & 1;
             if (!wwait(&B.q_full[qi], (jt >> 1) & 1, 0x401)) return false;
-            rotate_and_signal(smem + q_off(wk) + qi * kTileBytes, r, I.X, g, tab, &B.q_ready[qi], lane);
+            rotate_and_signal(smem + q_off(wk) + qi * kTileBytes, r, I.X, g, tab, &B.q_ready[qi], lane, rotate);
             return rotate_next();
         };
 
@@ -545,11 +563,13 @@ long long fwd_items(const Geo& g) { return fwd_item_count(g); }
 cudaError_t launch_fwd(const Geo& g, const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                        const CUtensorMap& mo, const void* q, const void* k, const void* v, void* o,
                        const float* theta, float* lse, unsigned int* status,
-                       unsigned long long limit_ns, int num_sms, cudaStream_t stream, cudaEvent_t const* events) {
+                       unsigned long long limit_ns, int num_sms, cudaStream_t stream, cudaEvent_t const* events,
+                       uint8_t* train_ws) {
     fwdk::Params prm;
     prm.g = g;
     prm.theta = theta;
     prm.lse = lse;
+    prm.qimg = prm.kimg = nullptr;
     prm.status = status;
     prm.limit_ns = limit_ns;
     prm.items = fwd_items(g);
@@ -571,6 +591,13 @@ cudaError_t launch_fwd(const Geo& g, const CUtensorMap& mq, const CUtensorMap& m
     if (events) {
         cudaError_t e = cudaEventRecord(events[0], stream);
         if (e != cudaSuccess) return e;
+    }
+    if (train_ws) {  // rotated q', k' images first, once per row, into the backward's workspace
+        if (cudaError_t e = launch_rope_images(g, q, k, theta, train_ws, stream)) return e;
+        size_t qo = 0, ko = 0;
+        bwd_image_offsets(g, &qo, &ko);
+        prm.qimg = train_ws + qo;
+        prm.kimg = train_ws + ko;
     }
     fwdk::fwd_kernel<<<static_cast<unsigned>(grid), fwdk::kThreads, fwdk::kSmemBytes, stream>>>(mq, mk, mv, mo, prm);
     cudaError_t e = cudaGetLastError();

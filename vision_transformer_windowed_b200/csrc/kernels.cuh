@@ -44,10 +44,15 @@ class SmemOptIn {
 int device_ready();
 
 long long fwd_items(const Geo& g);
+// train_ws: NULL, or the backward's workspace (windows of >= 128 tokens): the
+// forward then first writes the rotated q', k' tile images there (the images
+// the backward's prep would write) and reads Q', K' from them, instead of
+// rotating every K tile again for each query tile of its window.
 cudaError_t launch_fwd(const Geo& g, const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                        const CUtensorMap& mo, const void* q, const void* k, const void* v, void* o,
                        const float* theta, float* lse, unsigned int* status,
-                       unsigned long long limit_ns, int num_sms, cudaStream_t stream, cudaEvent_t const* events);
+                       unsigned long long limit_ns, int num_sms, cudaStream_t stream, cudaEvent_t const* events,
+                       uint8_t* train_ws = nullptr);
 
 struct BwdPtrs {
     const void *q, *k, *v, *o, *dout;
@@ -64,11 +69,19 @@ struct BwdMaps {
 
 long long bwd_items(const Geo& g);
 size_t bwd_workspace_bytes(const Geo& g);
+// Offsets of the rotated q', k' tile images in the backward's workspace, and
+// the launch that writes them (windows of >= 128 tokens).
+void bwd_image_offsets(const Geo& g, size_t* qimg, size_t* kimg);
+cudaError_t launch_rope_images(const Geo& g, const void* q, const void* k, const float* theta, uint8_t* ws,
+                               cudaStream_t stream);
 // events: NULL, or 5 events recorded before the first and after each of the
 // four launches (prep, main, post, d theta; windows of fewer than 128 tokens
 // run one kernel in the place of the first three).
+// images_ready: the workspace already holds the q', k' images of these inputs
+// (written by a training forward, windows of >= 128 tokens): prep skips them.
 cudaError_t launch_bwd(const Geo& g, const BwdPtrs& p, const BwdMaps& maps, unsigned int* status,
-                       unsigned long long limit_ns, int num_sms, cudaStream_t stream, cudaEvent_t const* events);
+                       unsigned long long limit_ns, int num_sms, cudaStream_t stream, cudaEvent_t const* events,
+                       bool images_ready = false);
 
 // Windows of fewer than 128 tokens (the tile holds whole windows): the whole
 // backward of a tile in one kernel (d theta partials, 4 x 16 per (head, tile),

@@ -44,10 +44,12 @@ def _stream(device) -> int:
     return torch.cuda.current_stream(device).cuda_stream
 
 
-def winattn_fwd(q, k, v, theta, M: int, s: int, o=None, lse=None, need_lse: bool = True):
+def winattn_fwd(q, k, v, theta, M: int, s: int, o=None, lse=None, need_lse: bool = True, workspace=None):
     """O, LSE = fused windowed-RoPE attention forward (bf16 in/out, fp32 LSE).
 
-    need_lse=False (and no lse buffer): inference forward, O only; LSE is returned as None."""
+    need_lse=False (and no lse buffer): inference forward, O only; LSE is returned as None.
+    workspace (the backward's, from alloc_workspace): the training forward, which
+    also leaves the rotated q', k' tiles there for winattn_bwd(..., after_train_fwd=True)."""
     sh = _shape(q, M, s)
     B, H, W, heads, d = q.shape
     for name, t in (("q", q), ("k", k), ("v", v)):
@@ -60,6 +62,12 @@ def winattn_fwd(q, k, v, theta, M: int, s: int, o=None, lse=None, need_lse: bool
     _check_tensor("o", o, q.shape, torch.bfloat16)
     if lse is not None:
         _check_tensor("lse", lse, (B, H, W, heads), torch.float32)
+    if workspace is not None:
+        if lse is None:
+            raise ValueError("the training forward writes lse")
+        _lib.fs_winattn_fwd_train(sh, q.data_ptr(), k.data_ptr(), v.data_ptr(), theta.data_ptr(), o.data_ptr(),
+                                  lse.data_ptr(), workspace.data_ptr(), workspace.numel(), _stream(q.device))
+        return o, lse
     _lib.fs_winattn_fwd(sh, q.data_ptr(), k.data_ptr(), v.data_ptr(), theta.data_ptr(), o.data_ptr(),
                         lse.data_ptr() if lse is not None else 0, _stream(q.device))
     return o, lse
@@ -95,8 +103,12 @@ def alloc_workspace(q: torch.Tensor, M: int, s: int) -> torch.Tensor:
 
 
 def winattn_bwd(q, k, v, o, dout, lse, theta, M: int, s: int, workspace=None, dq=None, dk=None, dv=None,
-                dtheta=None):
-    """dQ, dK, dV, dtheta of sum(O * dout) (recompute-based backward)."""
+                dtheta=None, after_train_fwd: bool = False):
+    """dQ, dK, dV, dtheta of sum(O * dout) (recompute-based backward).
+
+    after_train_fwd: `workspace` is the one a training forward (winattn_fwd with
+    that workspace) of the same q, k, theta filled, unchanged since; its rotated
+    q', k' tiles are reused."""
     sh = _shape(q, M, s)
     B, H, W, heads, d = q.shape
     for name, t in (("q", q), ("k", k), ("v", v), ("o", o), ("dout", dout)):
@@ -108,10 +120,13 @@ def winattn_bwd(q, k, v, o, dout, lse, theta, M: int, s: int, workspace=None, dq
     dv = torch.empty_like(q) if dv is None else dv
     dtheta = torch.empty_like(theta) if dtheta is None else dtheta
     if workspace is None:
+        if after_train_fwd:
+            raise ValueError("after_train_fwd needs the training forward's workspace")
         workspace = alloc_workspace(q, M, s)
-    _lib.fs_winattn_bwd(sh, q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), dout.data_ptr(), lse.data_ptr(),
-                        theta.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), dtheta.data_ptr(),
-                        workspace.data_ptr(), workspace.numel(), _stream(q.device))
+    call = _lib.fs_winattn_bwd_train if after_train_fwd else _lib.fs_winattn_bwd
+    call(sh, q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), dout.data_ptr(), lse.data_ptr(),
+         theta.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), dtheta.data_ptr(),
+         workspace.data_ptr(), workspace.numel(), _stream(q.device))
     return dq, dk, dv, dtheta
 
 
@@ -125,15 +140,19 @@ class WindowAttentionRoPE(torch.autograd.Function):
 
     @staticmethod
     def forward(ctx, q, k, v, theta, M: int, s: int):
-        o, lse = winattn_fwd(q, k, v, theta, M, s)
-        ctx.save_for_backward(q, k, v, o, lse, theta)
+        # the training pair: the forward leaves the rotated q', k' tiles in the
+        # backward's workspace
+        ws = alloc_workspace(q, M, s)
+        o, lse = winattn_fwd(q, k, v, theta, M, s, workspace=ws)
+        ctx.save_for_backward(q, k, v, o, lse, theta, ws)
         ctx.M, ctx.s = M, s
         return o
 
     @staticmethod
     def backward(ctx, dout):
-        q, k, v, o, lse, theta = ctx.saved_tensors
-        dq, dk, dv, dth = winattn_bwd(q, k, v, o, dout.contiguous(), lse, theta, ctx.M, ctx.s)
+        q, k, v, o, lse, theta, ws = ctx.saved_tensors
+        dq, dk, dv, dth = winattn_bwd(q, k, v, o, dout.contiguous(), lse, theta, ctx.M, ctx.s, workspace=ws,
+                                      after_train_fwd=True)
         return dq, dk, dv, dth, None, None
 
 
