@@ -90,7 +90,18 @@ def test_full_size_sampled_windows_d64(cfg):
     _full_size(*cfg, d=64)
 
 
-def _full_size(name, B, H, W, heads, M, s, qk, dscale=1.0, d=32):
+# the four-stage step's blocks through the training pair, as the benchmark runs them
+# (the forward reads the rotated q', k' tiles it left in the backward's workspace)
+TRAIN = [c for c in FULL if c[0].startswith("flashswin_t_stage")]
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("cfg", TRAIN, ids=[c[0] + "_train" for c in TRAIN])
+def test_full_size_sampled_windows_training_pair(cfg):
+    _full_size(*cfg[:8], dscale=cfg[8] if len(cfg) > 8 else 1.0, train=True)
+
+
+def _full_size(name, B, H, W, heads, M, s, qk, dscale=1.0, d=32, train=False):
     inp = make_inputs(B, H, W, heads, d, qk_scale=qk)
     units = _sample_units(B, H, W, heads, M)
     pos = []
@@ -105,8 +116,10 @@ def _full_size(name, B, H, W, heads, M, s, qk, dscale=1.0, d=32):
     dout = torch.where(keep[..., None], inp["dout"], torch.zeros((), dtype=inp["dout"].dtype))
 
     dev = {k: v.cuda() for k, v in inp.items() if k != "dout"}
-    o, lse = ops.winattn_fwd(dev["q"], dev["k"], dev["v"], dev["theta"], M, s)
-    dq, dk, dv, dth = ops.winattn_bwd(dev["q"], dev["k"], dev["v"], o, dout.cuda() * dscale, lse, dev["theta"], M, s)
+    ws = ops.alloc_workspace(dev["q"], M, s) if train else None
+    o, lse = ops.winattn_fwd(dev["q"], dev["k"], dev["v"], dev["theta"], M, s, workspace=ws)
+    dq, dk, dv, dth = ops.winattn_bwd(dev["q"], dev["k"], dev["v"], o, dout.cuda() * dscale, lse, dev["theta"], M, s,
+                                      workspace=ws, after_train_fwd=train)
     torch.cuda.synchronize()
     if dscale != 1.0:
         dq, dk, dv, dth = (t.double() / dscale for t in (dq, dk, dv, dth))
