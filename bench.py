@@ -732,7 +732,7 @@ def main():
                                                                       dvi["theta"], dvi["u"], dvi["w"], M, s)
                     dp.allreduce_param_grads(dth, du, dw)
                     params = (("dtheta", dth), ("du", du), ("dw", dw))
-                else:  # the training pair, as the autograd wrapper calls it
+                else:  # the training pair (ops.window_attention(..., reuse_rotated=True) calls it so)
                     ws = ops.alloc_workspace(dvi["q"], M, s)
                     o, lse = ops.winattn_fwd(dvi["q"], dvi["k"], dvi["v"], dvi["theta"], M, s, workspace=ws)
                     dq, dk, dvv, dth = ops.winattn_bwd(dvi["q"], dvi["k"], dvi["v"], o, dvi["dout"], lse, dvi["theta"],

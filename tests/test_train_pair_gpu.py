@@ -6,7 +6,7 @@ workspace and, for windows of >= 128 tokens, reads its own Q', K' tiles from
 them; the backward then reuses them.  Same shape lists and tolerances as the
 stand-alone calls, plus a check that the backward's results equal those of the
 stand-alone backward bit for bit where that one is deterministic (dk, dv), and
-the autograd wrapper (which uses the pair).
+the autograd wrapper with reuse_rotated=True (which uses the pair).
 """
 import numpy as np
 import pytest
@@ -95,10 +95,10 @@ def test_train_backward_matches_standalone_backward(cfg):
 
 
 @pytest.mark.gpu
-def test_autograd_uses_the_pair():
+def test_autograd_with_the_pair():
     inp = make_inputs(1, 64, 64, 2, 32)
     leaves = {k: v.cuda().requires_grad_(k != "dout") for k, v in inp.items()}
-    o = ops.window_attention(leaves["q"], leaves["k"], leaves["v"], leaves["theta"], 32, 16)
+    o = ops.window_attention(leaves["q"], leaves["k"], leaves["v"], leaves["theta"], 32, 16, reuse_rotated=True)
     (o.float() * leaves["dout"].float()).sum().backward()
     ref = oracle.full(inp["q"], inp["k"], inp["v"], inp["theta"], 32, 16, dout=inp["dout"])
     check("o", o, ref["o"], FWD_TOL)

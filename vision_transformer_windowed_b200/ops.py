@@ -139,25 +139,30 @@ class WindowAttentionRoPE(torch.autograd.Function):
     """
 
     @staticmethod
-    def forward(ctx, q, k, v, theta, M: int, s: int):
-        # the training pair: the forward leaves the rotated q', k' tiles in the
-        # backward's workspace
-        ws = alloc_workspace(q, M, s)
+    def forward(ctx, q, k, v, theta, M: int, s: int, reuse_rotated: bool = False):
+        # reuse_rotated: the training pair, whose forward leaves the rotated q', k'
+        # tiles in the backward's workspace; the workspace (about 262 bytes per
+        # token-head) then stays allocated until the backward, beside the saved
+        # q, k, v, o (256 bytes per token-head)
+        ws = alloc_workspace(q, M, s) if reuse_rotated else None
         o, lse = winattn_fwd(q, k, v, theta, M, s, workspace=ws)
-        ctx.save_for_backward(q, k, v, o, lse, theta, ws)
-        ctx.M, ctx.s = M, s
+        ctx.save_for_backward(q, k, v, o, lse, theta, *(() if ws is None else (ws,)))
+        ctx.M, ctx.s, ctx.reuse = M, s, reuse_rotated
         return o
 
     @staticmethod
     def backward(ctx, dout):
-        q, k, v, o, lse, theta, ws = ctx.saved_tensors
-        dq, dk, dv, dth = winattn_bwd(q, k, v, o, dout.contiguous(), lse, theta, ctx.M, ctx.s, workspace=ws,
-                                      after_train_fwd=True)
-        return dq, dk, dv, dth, None, None
+        q, k, v, o, lse, theta, *ws = ctx.saved_tensors
+        dq, dk, dv, dth = winattn_bwd(q, k, v, o, dout.contiguous(), lse, theta, ctx.M, ctx.s,
+                                      workspace=ws[0] if ctx.reuse else None, after_train_fwd=ctx.reuse)
+        return dq, dk, dv, dth, None, None, None
 
 
-def window_attention(q, k, v, theta, M: int, s: int):
-    return WindowAttentionRoPE.apply(q, k, v, theta, M, s)
+def window_attention(q, k, v, theta, M: int, s: int, reuse_rotated: bool = False):
+    """Autograd windowed-RoPE attention.  reuse_rotated=True runs the training
+    pair (faster at windows of >= 128 tokens; keeps the backward's workspace
+    from the forward to the backward)."""
+    return WindowAttentionRoPE.apply(q, k, v, theta, M, s, reuse_rotated)
 
 
 # ------------------------------------------------------------ low-rank bias
