@@ -392,7 +392,7 @@ __global__ void __launch_bounds__(kThreads, 2) fwd_kernel(const __grid_constant_
 namespace bwd {
 
 struct WsLayout {
-    size_t acc, nrm, part, part2, cnt, red, total;
+    size_t acc, nrm, rowv, fac, part, part2, cnt, red, total;
     long long chunks;  // first-level dU / dW sums
 };
 
@@ -405,6 +405,8 @@ __host__ __device__ inline WsLayout ws_layout(const Geo& g) {
     size_t o = 0;
     L.acc = o;   o += round256(ht * kTile * 64 * 4);  // fp32 [heads][tiles][128][64]
     L.nrm = o;   o += round256(ht * 8);               // max |dO row|^2, max |v row|^2 per (head, tile)
+    L.rowv = o;  o += round256(ht * kTile * 8);       // per slot row: lse log2(e), D
+    L.fac = o;   o += round256(static_cast<size_t>(g.heads) * g.N * 2 * 32);  // [h][pos]: sqrt(d) U, W (fp16)
     L.part = o;  o += round256(ht * 8 * 16 * 4);      // d theta partials [heads][tiles][8][16]
     L.part2 = o; o += round256(static_cast<size_t>(g.heads) * 64 * 16 * 4);
     L.cnt = o;   o += round256(static_cast<size_t>(g.heads) * 4);
@@ -470,18 +472,42 @@ __global__ void __launch_bounds__(128) prep_kernel(const Params p) {
     const int r = threadIdx.x;
     if (blockIdx.x == 0)
         for (int i = r; i < g.heads; i += blockDim.x) reinterpret_cast<unsigned int*>(p.ws + p.L.cnt)[i] = 0u;
+    // the head's factor rows in fp16 (sqrt(d) U and W; 32 bytes each), written by
+    // the blocks of its first tiles, one position per thread
+    const long long pos = T * kTile + r;
+    if (pos < g.N) {
+        uint8_t* f = p.ws + p.L.fac + (static_cast<size_t>(h) * g.N + static_cast<size_t>(pos)) * 64;
+        const float4* u4 = reinterpret_cast<const float4*>(p.u + (static_cast<long long>(h) * g.N + pos) * 16);
+        const float4* w4 = reinterpret_cast<const float4*>(p.w + (static_cast<long long>(h) * g.N + pos) * 16);
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+            const float4 a0 = __ldg(u4 + 2 * c), a1 = __ldg(u4 + 2 * c + 1);
+            const float4 b0 = __ldg(w4 + 2 * c), b1 = __ldg(w4 + 2 * c + 1);
+            reinterpret_cast<uint4*>(f)[c] =
+                make_uint4(pack_f16x2(a0.x * kSqrtD, a0.y * kSqrtD), pack_f16x2(a0.z * kSqrtD, a0.w * kSqrtD),
+                           pack_f16x2(a1.x * kSqrtD, a1.y * kSqrtD), pack_f16x2(a1.z * kSqrtD, a1.w * kSqrtD));
+            reinterpret_cast<uint4*>(f + 32)[c] = make_uint4(pack_f16x2(b0.x, b0.y), pack_f16x2(b0.z, b0.w),
+                                                             pack_f16x2(b1.x, b1.y), pack_f16x2(b1.z, b1.w));
+        }
+    }
     int pi, pj;
     long long tok;
-    float ndo = 0.f, nv = 0.f;
+    float ndo = 0.f, nv = 0.f, D = 0.f, lse2 = INFINITY;
     if (slot_token(g, T, r, h, &pi, &pj, &tok)) {
-        float a[32];
+        float a[32], c[32];
         load_row32(p.dout, tok, a);
+        load_row32(p.o, tok, c);
 #pragma unroll
-        for (int e = 0; e < 32; ++e) ndo = fmaf(a[e], a[e], ndo);
+        for (int e = 0; e < 32; ++e) {
+            ndo = fmaf(a[e], a[e], ndo);
+            D = fmaf(a[e], c[e], D);
+        }
         load_row32(p.v, tok, a);
 #pragma unroll
         for (int e = 0; e < 32; ++e) nv = fmaf(a[e], a[e], nv);
+        lse2 = __ldg(p.lse + tok) * 1.4426950408889634f;
     }
+    reinterpret_cast<float2*>(p.ws + p.L.rowv)[ht * kTile + r] = make_float2(lse2, D);
     uint4* acc = reinterpret_cast<uint4*>(p.ws + p.L.acc + (ht * kTile + r) * 64 * 4);
 #pragma unroll
     for (int c = 0; c < 16; ++c) acc[c] = make_uint4(0, 0, 0, 0);
@@ -493,6 +519,15 @@ __global__ void __launch_bounds__(128) prep_kernel(const Params p) {
         reinterpret_cast<float2*>(p.ws + p.L.nrm)[ht] =
             make_float2(fmaxf(fmaxf(nrm_w[0].x, nrm_w[1].x), fmaxf(nrm_w[2].x, nrm_w[3].x)),
                         fmaxf(fmaxf(nrm_w[0].y, nrm_w[1].y), fmaxf(nrm_w[2].y, nrm_w[3].y)));
+}
+
+// cp.async copy of a factor row (32 bytes, fp16) into row r of a factor half
+// tile, channels 16..31 zero-filled.
+__device__ __forceinline__ void copy_factor(uint8_t* tile, int r, const uint8_t* src) {
+    uint8_t* row = tile + r * kRowBytes;
+    const int sw = (r >> 1) & 3;
+#pragma unroll
+    for (int c = 0; c < 4; ++c) cp_async16(smem_u32(row + ((c ^ sw) << 4)), src + 16 * (c & 1), c < 2 ? 16u : 0u);
 }
 
 // Main kernel: two warpgroups of four warps; warp w serves TMEM lanes (key rows)
@@ -574,6 +609,8 @@ __global__ void __launch_bounds__(kThreads, 1) main_kernel(const __grid_constant
     uint8_t* kh[2] = {smem + kKOff, smem + kKOff + kTileBytes};
     uint8_t* vt = smem + kVOff;
     float* acc_all = reinterpret_cast<float*>(prm.ws + prm.L.acc);
+    const uint8_t* fac = prm.ws + prm.L.fac;                                // [h][pos]: sqrt(d) U, W (fp16)
+    const float2* rowv = reinterpret_cast<const float2*>(prm.ws + prm.L.rowv);  // per slot row: lse2, D
     uint32_t gph = 0, sph = 0, mph = 0;
     int tab_head = -1;
     bool ok = true;
@@ -596,8 +633,6 @@ __global__ void __launch_bounds__(kThreads, 1) main_kernel(const __grid_constant
             if (!group_sync(0x6402)) break;
             tab_head = I.h;
         }
-        const float* uh = prm.u + static_cast<long long>(I.h) * g.N * 16;
-        const float* wh = prm.w + static_cast<long long>(I.h) * g.N * 16;
         // the gradient scaling 2^e of the item: the largest |dO| and |v| rows of its
         // window (or tile, for windows inside one tile), from the prep kernel
         float mdo = 0.f, mv = 0.f;
@@ -624,8 +659,8 @@ __global__ void __launch_bounds__(kThreads, 1) main_kernel(const __grid_constant
             prep_row(kh[0], r, ki, kj, rtab);
         } else {
             copy_rows(vt, prm.v, ktok, kvalid, quad, lane);
+            copy_factor(kh[1], r, fac + (static_cast<size_t>(I.h) * g.N + ki * g.M + kj) * 64 + 32);
             cp_async_commit();
-            fill_factor(kh[1], r, wh + (ki * g.M + kj) * 16, 1.f);
         }
         bool first = true;
         // Query steps, double-buffered: the copies, factors, D and lse2 of the next
@@ -636,22 +671,15 @@ __global__ void __launch_bounds__(kThreads, 1) main_kernel(const __grid_constant
             uint8_t* qb = smem + kBufOff + b * kBufBytes;
             if (wg == 0) {
                 copy_rows(qb, prm.q, qtok, qvalid, quad, lane);
+                copy_factor(qb + kTileBytes, r, fac + (static_cast<size_t>(I.h) * g.N + qi * g.M + qj) * 64);
                 cp_async_commit();
-                fill_factor(qb + kTileBytes, r, uh + (qi * g.M + qj) * 16, kSqrtD);
             } else {
                 copy_rows(qb + 2 * kTileBytes, prm.dout, qtok, qvalid, quad, lane);
                 cp_async_commit();
-                float D = 0.f;
-                if (qvalid) {
-                    float a[32], c[32];
-                    load_row32(prm.o, qtok, a);
-                    load_row32(prm.dout, qtok, c);
-#pragma unroll
-                    for (int e = 0; e < 32; ++e) D = fmaf(a[e], c[e], D);
-                }
-                vec[256 * b + kTile + r] = D;
-                vec[256 * b + r] = qvalid ? __ldg(prm.lse + qtok) * 1.4426950408889634f - static_cast<float>(gexp)
-                                          : INFINITY;
+                // lse2 and D of the row, from the prep kernel (lse2 = +inf for a padded row)
+                const float2 ld = __ldcg(rowv + ((static_cast<long long>(I.h) * g.tiles + I.q0 + n) * kTile + r));
+                vec[256 * b + kTile + r] = ld.y;
+                vec[256 * b + r] = ld.x - static_cast<float>(gexp);
             }
         };
         auto next_active = [&](int n) {
