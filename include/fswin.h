@@ -164,7 +164,7 @@ FS_API fs_status fs_winattn_bwd(const fs_winattn_shape* shape, const void* q, co
  * fixed order), all overwritten.  dq, du and the query side of dtheta are
  * accumulated in fp32 with vector reductions whose order varies from run to
  * run; dk, dv and dw do not vary.  workspace: at least fs_winattn_lrbias_bwd_workspace_bytes(shape)
- * bytes, 256-byte aligned (about 268 bytes per token-head on the padded grid,
+ * bytes, 256-byte aligned (about 276 bytes per token-head on the padded grid,
  * plus a few KB per head).  The kernels are plain one-tile pipelines.
  */
 FS_API fs_status fs_winattn_lrbias_fwd(const fs_winattn_shape* shape, const void* q, const void* k, const void* v,

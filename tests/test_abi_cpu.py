@@ -175,8 +175,9 @@ def test_lrbias_entry_points_reject_before_launch():
 
 
 def test_lrbias_workspace_size():
-    """The bias backward's scratch: 256 B of accumulator rows per token-head (on
-    the padded grid), 8 x 16 fp32 d theta partials and the norms per (head,
+    """The bias backward's scratch: 256 B of accumulator rows and 8 B of lse2 and
+    D per token-head (on the padded grid), the fp16 factor rows (64 B per head
+    and window position), 8 x 16 fp32 d theta partials and the norms per (head,
     tile), a fixed d theta part, and one [head][window slot][32] fp32 block per
     16 windows for the first level of the dU / dW sum."""
     B, H, W, heads, M = 4, 64, 64, 3, 16
@@ -185,9 +186,10 @@ def test_lrbias_workspace_size():
     wins = B * (H // M) * (W // M)
     chunks = -(-wins // 16)
     tiles = B * H * W // 128
-    expect = tokens * 256 + heads * tiles * 8 + heads * tiles * 8 * 16 * 4 + heads * 64 * 16 * 4 + heads * 4 + \
+    expect = tokens * (256 + 8) + heads * M * M * 64 + heads * tiles * 8 + heads * tiles * 8 * 16 * 4 + \
+        heads * 64 * 16 * 4 + heads * 4 + \
         chunks * heads * M * M * 32 * 4
-    assert expect <= n <= expect + 6 * 256
+    assert expect <= n <= expect + 8 * 256
 
 
 def test_train_pair_rejects_before_launch():
