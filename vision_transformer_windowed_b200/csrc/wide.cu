@@ -356,7 +356,7 @@ namespace bwd {
 
 // workspace: the dQ' accumulator, per-tile norms, d theta partials and scratch
 struct WsLayout {
-    size_t dqacc, nrm, part, part2, cnt, total;
+    size_t dqacc, nrm, rowv, part, part2, cnt, total;
 };
 
 __host__ __device__ inline size_t round256(size_t x) { return (x + 255) & ~size_t(255); }
@@ -367,6 +367,7 @@ __host__ __device__ inline WsLayout ws_layout(const Geo& g) {
     size_t o = 0;
     L.dqacc = o; o += round256(ht * kTile * 64 * 4);   // fp32 [heads][tiles][128][64]
     L.nrm = o;   o += round256(ht * 8);                // max |dO row|^2, max |v row|^2 per (head, tile)
+    L.rowv = o;  o += round256(ht * kTile * 8);        // per slot row: lse log2(e), D
     L.part = o;  o += round256(ht * 2 * 8 * 16 * 4);   // [heads][2 axes][tiles][8][16]
     L.part2 = o; o += round256(static_cast<size_t>(g.heads) * 2 * 64 * 16 * 4);
     L.cnt = o;   o += round256(static_cast<size_t>(g.heads) * 2 * 4);
@@ -441,16 +442,23 @@ __global__ void __launch_bounds__(128) prep_kernel(const Params p) {
         for (int i = r; i < 2 * g.heads; i += blockDim.x) reinterpret_cast<unsigned int*>(p.ws + p.L.cnt)[i] = 0u;
     int pi, pj;
     long long tok;
-    float ndo = 0.f, nv = 0.f;
+    float ndo = 0.f, nv = 0.f, D = 0.f, lse2 = INFINITY;
     if (slot_token(g, T, r, h, &pi, &pj, &tok)) {
-        float a[32], b[32];
+        float a[32], b[32], c[32], d[32];
         load_row64(p.dout, tok, a, b);
+        load_row64(p.o, tok, c, d);
 #pragma unroll
-        for (int e = 0; e < 32; ++e) ndo = fmaf(a[e], a[e], fmaf(b[e], b[e], ndo));
+        for (int e = 0; e < 32; ++e) {
+            ndo = fmaf(a[e], a[e], fmaf(b[e], b[e], ndo));
+            D = fmaf(a[e], c[e], fmaf(b[e], d[e], D));
+        }
         load_row64(p.v, tok, a, b);
 #pragma unroll
         for (int e = 0; e < 32; ++e) nv = fmaf(a[e], a[e], fmaf(b[e], b[e], nv));
+        lse2 = __ldg(p.lse + tok) * 1.4426950408889634f;
     }
+    // D = dO . O and lse in log2 units per slot row, staged by the main kernel
+    reinterpret_cast<float2*>(p.ws + p.L.rowv)[ht * kTile + r] = make_float2(lse2, D);
     uint4* acc = reinterpret_cast<uint4*>(p.ws + p.L.dqacc + (ht * kTile + r) * 64 * 4);
 #pragma unroll
     for (int c = 0; c < 16; ++c) acc[c] = make_uint4(0, 0, 0, 0);
@@ -613,17 +621,11 @@ __global__ void __launch_bounds__(kThreads, 1) main_kernel(const __grid_constant
             } else {
                 copy_rows(qb + 2 * kTileBytes, qb + 3 * kTileBytes, prm.dout, qtok, qvalid, quad, lane);
                 cp_async_commit();
-                float D = 0.f;
-                if (qvalid) {
-                    float a0[32], a1[32], b0[32], b1[32];
-                    load_row64(prm.o, qtok, a0, a1);
-                    load_row64(prm.dout, qtok, b0, b1);
-#pragma unroll
-                    for (int e = 0; e < 32; ++e) D = fmaf(a0[e], b0[e], fmaf(a1[e], b1[e], D));
-                }
-                vec[256 * b + kTile + r] = D;
-                vec[256 * b + r] = qvalid ? __ldg(prm.lse + qtok) * 1.4426950408889634f - static_cast<float>(gexp)
-                                          : INFINITY;
+                // lse2 and D of the row, from the prep kernel (lse2 = +inf for a padded row)
+                const float2 ld = __ldcg(reinterpret_cast<const float2*>(prm.ws + prm.L.rowv) +
+                                         ((static_cast<long long>(I.h) * g.tiles + I.q0 + n) * kTile + r));
+                vec[256 * b + kTile + r] = ld.y;
+                vec[256 * b + r] = ld.x - static_cast<float>(gexp);
             }
         };
         auto next_active = [&](int n) {
