@@ -508,6 +508,9 @@ __global__ void __launch_bounds__(128) prep_kernel(const Params p) {
         lse2 = __ldg(p.lse + tok) * 1.4426950408889634f;
     }
     reinterpret_cast<float2*>(p.ws + p.L.rowv)[ht * kTile + r] = make_float2(lse2, D);
+    // the key side of d theta: the main kernel writes one slot per run of items of a
+    // head in a CTA, the other slots 4..7 of the head's tiles must read zero
+    if (r < 64) reinterpret_cast<float*>(p.ws + p.L.part)[(ht * 8 + 4) * 16 + r] = 0.f;
     uint4* acc = reinterpret_cast<uint4*>(p.ws + p.L.acc + (ht * kTile + r) * 64 * 4);
 #pragma unroll
     for (int c = 0; c < 16; ++c) acc[c] = make_uint4(0, 0, 0, 0);
@@ -614,6 +617,20 @@ __global__ void __launch_bounds__(kThreads, 1) main_kernel(const __grid_constant
     uint32_t gph = 0, sph = 0, mph = 0;
     int tab_head = -1;
     bool ok = true;
+    // key side of d theta, summed over this CTA's run of items of one head (items
+    // go head by head) and written once per run, to slot 4 + quad of the run's
+    // first key tile
+    float part[16];
+#pragma unroll
+    for (int e = 0; e < 16; ++e) part[e] = 0.f;
+    int run_head = -1;
+    long long run_tile = 0;
+    auto flush_partials = [&]() {
+        if (rtab && wg == 0 && run_head >= 0)
+            write_partials(part, reinterpret_cast<float*>(prm.ws + prm.L.part), g, run_head, run_tile, 4 + quad, lane);
+#pragma unroll
+        for (int e = 0; e < 16; ++e) part[e] = 0.f;
+    };
     auto wwait = [&](uint64_t* bar, uint32_t ph, unsigned int where) -> bool {
         return __all_sync(0xFFFFFFFFu, mbar_wait(bar, ph, ctl, where));
     };
@@ -627,6 +644,11 @@ __global__ void __launch_bounds__(kThreads, 1) main_kernel(const __grid_constant
 
     for (long long it = blockIdx.x; it < prm.items && ok; it += gridDim.x) {
         const BwdItem I = d_bwd_item(g, it);
+        if (I.h != run_head) {  // a new run of items of one head
+            flush_partials();
+            run_head = I.h;
+            run_tile = I.u;
+        }
         if (rtab && I.h != tab_head) {
             if (!group_sync(0x6401)) break;
             build_table(tab, prm.theta + I.h * 2 * kPairs, g.M, tid, kThreads);
@@ -821,9 +843,6 @@ __global__ void __launch_bounds__(kThreads, 1) main_kernel(const __grid_constant
         // item end: group 0 dk (dK' un-rotated) and the key side of d theta, group 1
         // dv and the row's dW share
         const float down = exp2i(-gexp);
-        float part[16];
-#pragma unroll
-        for (int e = 0; e < 16; ++e) part[e] = 0.f;
         if (first) {  // no query tile attends these keys (cannot happen: a key attends itself)
             float z[32];
 #pragma unroll
@@ -865,11 +884,11 @@ __global__ void __launch_bounds__(kThreads, 1) main_kernel(const __grid_constant
         __syncwarp();
         if (wg == 0) {
             store_rows(prm.dk, kh[0], ktok, kvalid, quad, lane);
-            if (rtab) write_partials(part, reinterpret_cast<float*>(prm.ws + prm.L.part), g, I.h, I.u, 4 + quad, lane);
         } else {
             store_rows(prm.dv, vt, ktok, kvalid, quad, lane);
         }
     }
+    flush_partials();
     cp_async_wait<0>();  // a step staged before a failed wait: its copies land before the CTA exits
     if (tid == 0) {
         umma_commit(&bars->done);
