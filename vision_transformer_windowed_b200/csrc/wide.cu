@@ -410,7 +410,7 @@ __device__ __forceinline__ void dtheta_terms(float (&part)[32], const float (&dx
                                              int axis) {
 #pragma unroll
     for (int k = 0; k < kPairs; ++k)
-        part[axis * kPairs + k] = pos * (dx[2 * k + 1] * x[2 * k] - dx[2 * k] * x[2 * k + 1]);
+        part[axis * kPairs + k] += pos * (dx[2 * k + 1] * x[2 * k] - dx[2 * k] * x[2 * k + 1]);
 }
 
 // The warp's 32 d theta partials, summed over the warp in a fixed order, to
@@ -459,6 +459,13 @@ __global__ void __launch_bounds__(128) prep_kernel(const Params p) {
     }
     // D = dO . O and lse in log2 units per slot row, staged by the main kernel
     reinterpret_cast<float2*>(p.ws + p.L.rowv)[ht * kTile + r] = make_float2(lse2, D);
+    // the key side of d theta: the main kernel writes one slot per run of items of a
+    // head in a CTA, the other slots 4..7 of the head's tiles must read zero
+    {
+        const int axis = r >> 6, i = r & 63;
+        reinterpret_cast<float*>(p.ws + p.L.part)[(((static_cast<long long>(h) * 2 + axis) * g.tiles + T) * 8 + 4) * 16 + i] =
+            0.f;
+    }
     uint4* acc = reinterpret_cast<uint4*>(p.ws + p.L.dqacc + (ht * kTile + r) * 64 * 4);
 #pragma unroll
     for (int c = 0; c < 16; ++c) acc[c] = make_uint4(0, 0, 0, 0);
@@ -571,9 +578,28 @@ __global__ void __launch_bounds__(kThreads, 1) main_kernel(const __grid_constant
         rope_half(x, pi, tab + kPairs * 64, false);
         store_row_swz(h1, r, x, true);
     };
+    // key side of d theta, summed over this CTA's run of items of one head (items
+    // go head by head) and written once per run, to slot 4 + quad of the run's
+    // first key tile
+    float part[32];
+#pragma unroll
+    for (int e = 0; e < 32; ++e) part[e] = 0.f;
+    int run_head = -1;
+    long long run_tile = 0;
+    auto flush_partials = [&]() {
+        if (wg == 0 && run_head >= 0)
+            write_partials(part, reinterpret_cast<float*>(prm.ws + prm.L.part), g, run_head, run_tile, 4 + quad, lane);
+#pragma unroll
+        for (int e = 0; e < 32; ++e) part[e] = 0.f;
+    };
 
     for (long long it = blockIdx.x; it < prm.items && ok; it += gridDim.x) {
         const BwdItem I = d_bwd_item(g, it);
+        if (I.h != run_head) {  // a new run of items of one head
+            flush_partials();
+            run_head = I.h;
+            run_tile = I.u;
+        }
         if (I.h != tab_head) {
             if (!group_sync(0x6201)) break;
             build_table(tab, prm.theta + I.h * 2 * kPairs, g.M, tid, kThreads);
@@ -756,9 +782,6 @@ __global__ void __launch_bounds__(kThreads, 1) main_kernel(const __grid_constant
         if (!ok) break;
         // item end: group 0 dk (dK' un-rotated) and the key side of d theta, group 1 dv
         const float down = exp2i(-gexp);
-        float part[32];
-#pragma unroll
-        for (int e = 0; e < 32; ++e) part[e] = 0.f;
         uint8_t* const* st = wg == 0 ? kh : vh;
         if (first) {  // no query tile attends these keys (cannot happen: a key attends itself)
             float z[32];
@@ -790,9 +813,8 @@ __global__ void __launch_bounds__(kThreads, 1) main_kernel(const __grid_constant
         tc_fence_before();
         __syncwarp();
         store_rows(wg == 0 ? prm.dk : prm.dv, st[0], st[1], ktok, kvalid, quad, lane);
-        if (wg == 0)
-            write_partials(part, reinterpret_cast<float*>(prm.ws + prm.L.part), g, I.h, I.u, 4 + quad, lane);
     }
+    flush_partials();
     cp_async_wait<0>();  // a step staged before a failed wait: its copies land before the CTA exits
     if (tid == 0) {
         umma_commit(&bars->done);
