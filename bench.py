@@ -204,18 +204,18 @@ def phase_work(st, s) -> dict:
     pairs = unmasked_pairs(B, H, W, heads, M, s)
     small = M * M < 128
     pf, pb = pair_flops(st)
-    if st.get("lrbias"):  # the bias kernels (plain pipelines at every window size): prep reads dO, v
-        # and zeroes the fp32 accumulator rows (256 B); main reads q, k, v, o, dO, lse and writes dk,
-        # dv; post reads the accumulator's dQ' part and q and writes dq; the window sums read the
-        # accumulator's dU / dW part (the factors themselves stay in L2)
-        nbytes = {"fwd": (256 if st.get("infer") else 260) * rows, "bwd_prep": 384 * rows,
-                  "bwd_main": 452 * rows, "bwd_post": 256 * rows, "bwd_dtheta": 128 * rows}
+    if st.get("lrbias"):  # the bias kernels (plain pipelines at every window size): prep reads dO, o,
+        # v and lse, writes lse2 and D and zeroes the fp32 accumulator rows (256 B); main reads q, k, v,
+        # dO, lse2 and D and writes dk, dv; post reads the accumulator's dQ' part and q and writes dq;
+        # the window sums read the dU / dW shares (the factors themselves stay in L2)
+        nbytes = {"fwd": (256 if st.get("infer") else 260) * rows, "bwd_prep": 460 * rows,
+                  "bwd_main": 392 * rows, "bwd_post": 256 * rows, "bwd_dtheta": 128 * rows}
         return {"bytes": nbytes, "flops": {"fwd": pf * pairs, "bwd_main": pb * pairs}, "hbm_bound": False}
-    if d == 64:  # the wide kernels: prep reads dO, v and zeroes the fp32 dQ' accumulator; main reads
-        # q, k, v, o, dO and lse, writes dk, dv (the dQ' additions resolve in L2); post reads the
-        # accumulator and q, writes dq
-        nbytes = {"fwd": (512 if st.get("infer") else 516) * rows, "bwd_prep": 512 * rows,
-                  "bwd_main": 900 * rows, "bwd_post": 512 * rows, "bwd_dtheta": 0}
+    if d == 64:  # the wide kernels: prep reads dO, o, v and lse, writes lse2 and D and zeroes the fp32
+        # dQ' accumulator; main reads q, k, v, dO, lse2 and D, writes dk, dv (the dQ' additions
+        # resolve in L2); post reads the accumulator and q, writes dq
+        nbytes = {"fwd": (512 if st.get("infer") else 516) * rows, "bwd_prep": 652 * rows,
+                  "bwd_main": 776 * rows, "bwd_post": 512 * rows, "bwd_dtheta": 0}
     else:
         fwd_row = 256 if st.get("infer") else (260 if small else 516)
         nbytes = {"fwd": fwd_row * rows, "bwd_prep": 0 if small else 340 * rows,
