@@ -104,17 +104,22 @@ __device__ __forceinline__ void store_rows(uint8_t* dst, const uint8_t* tile, lo
     }
 }
 
-// Row r of a factor half tile: mul * f[0..15] as fp16 in channels 0..15, zeros in 16..31.
-__device__ __forceinline__ void fill_factor(uint8_t* tile, int r, const float* f, float mul) {
+// A factor row's 16 fp32 values, loaded into registers (no wait here).
+__device__ __forceinline__ void load_factor(float4 (&f)[4], const float* src) {
+    const float4* p = reinterpret_cast<const float4*>(src);
+#pragma unroll
+    for (int c = 0; c < 4; ++c) f[c] = __ldg(p + c);
+}
+
+// Row r of a factor half tile: mul * f as fp16 in channels 0..15, zeros in 16..31.
+__device__ __forceinline__ void put_factor(uint8_t* tile, int r, const float4 (&f)[4], float mul) {
     float x[32];
-    const float4* p = reinterpret_cast<const float4*>(f);
 #pragma unroll
     for (int c = 0; c < 4; ++c) {
-        const float4 a = __ldg(p + c);
-        x[4 * c] = a.x * mul;
-        x[4 * c + 1] = a.y * mul;
-        x[4 * c + 2] = a.z * mul;
-        x[4 * c + 3] = a.w * mul;
+        x[4 * c] = f[c].x * mul;
+        x[4 * c + 1] = f[c].y * mul;
+        x[4 * c + 2] = f[c].z * mul;
+        x[4 * c + 3] = f[c].w * mul;
     }
 #pragma unroll
     for (int e = 16; e < 32; ++e) x[e] = 0.f;
@@ -147,14 +152,16 @@ __device__ __forceinline__ void load_row32(const uint8_t* base, long long tok, f
 namespace fwd {
 
 constexpr int kThreads = 128;
+constexpr int kKVBufs = 3;                        // key buffers: staged, in the score product, in P V
 constexpr int kQOff = 0;                          // Q~ half tiles: q' and sqrt(d) U (then the staged O)
-constexpr int kKVOff = kQOff + 2 * kTileBytes;    // two key buffers: K~ half tiles (k', W), V tile
+constexpr int kKVOff = kQOff + 2 * kTileBytes;    // key buffers: K~ half tiles (k', W), V tile
 constexpr int kKVBytes = 3 * kTileBytes;
-constexpr int kTabOff = kKVOff + 2 * kKVBytes;
+constexpr int kTabOff = kKVOff + kKVBufs * kKVBytes;
 constexpr int kBarOff = kTabOff + kTabBytes;
 constexpr int kSmemBytes = kBarOff + 256 + 1024;  // + alignment of the base
 constexpr uint32_t kTmemCols = 256;
-constexpr uint32_t kColS = 0, kColP = 0, kColO = 128;
+constexpr uint32_t kSBuf = 128;                   // two S buffers, at columns 0 and 128
+constexpr uint32_t kColP = 0, kColO = 64;         // within an S buffer: bf16 P, then the tile's P V
 
 struct Bars {
     uint64_t s_full, o_full, grp, done;
@@ -175,6 +182,14 @@ struct Params {
     long long items;
 };
 
+// The loop over an item's key tiles keeps one product in flight behind the
+// softmax: tile u's P V goes to the spare columns of u's S buffer, and the next
+// tile's S goes to the other buffer.  Thread 0 issues both in order, so when the
+// softmax sees tile u+1's S complete, tile u's P V is complete too (a commit
+// covers every earlier product of its thread) and is added to the O registers
+// then; only an item's last P V has a barrier of its own.  The key buffers
+// rotate over three: while tile u's S is computed, tile u+1's rows are copied
+// into the buffer of tile u-2, whose P V completed before tile u-1's softmax.
 __global__ void __launch_bounds__(kThreads, 2) fwd_kernel(const __grid_constant__ Params prm) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -210,7 +225,7 @@ __global__ void __launch_bounds__(kThreads, 2) fwd_kernel(const __grid_constant_
     const float2* rtab = prm.theta ? tab : nullptr;
     uint8_t* q0 = smem + kQOff;
     uint8_t* q1 = q0 + kTileBytes;
-    uint32_t gph = 0, sph = 0, oph = 0;
+    uint32_t gph = 0, sph = 0, oph = 0, tcs = 0;  // tcs: tiles whose S was issued; S buffer tcs & 1
     int tab_head = -1;
     bool ok = true;
     auto wwait = [&](uint64_t* bar, uint32_t ph, unsigned int where) -> bool {
@@ -240,16 +255,16 @@ __global__ void __launch_bounds__(kThreads, 2) fwd_kernel(const __grid_constant_
         const bool qvalid = slot_token(g, I.X, r, I.h, &pi, &pj, &qtok);
         const uint32_t myseg = I.masked ? seg_at(d_tile_segs(g, I.X, I.win), r >> g.lBT) : 0u;
         if (!group_sync(0x6303)) break;  // the previous item's staged O rows are stored
-        // Key tiles, double-buffered: the next active tile's K, V rows and key
-        // factors are copied while the current tile's softmax runs.
-        auto kv_stage = [&](int u, int b, int& ki, int& kj) {
+        // A key tile's K, V rows (copies) and key factor row (loads into
+        // registers, written to the tile when the tile is prepared).
+        auto kv_stage = [&](int u, int b, int& ki, int& kj, float4 (&f)[4]) {
             long long ktok;
             const bool kvalid = slot_token(g, I.kv0 + u, r, I.h, &ki, &kj, &ktok);
             uint8_t* kb = smem + kKVOff + b * kKVBytes;
             copy_rows(kb, prm.k, ktok, kvalid, warp, lane);
             copy_rows(kb + 2 * kTileBytes, prm.v, ktok, kvalid, warp, lane);
             cp_async_commit();
-            fill_factor(kb + kTileBytes, r, wh + (ki * g.M + kj) * 16, 1.f);
+            load_factor(f, wh + (ki * g.M + kj) * 16);
         };
         auto next_kv = [&](int u) {
             while (u < I.nkv && !((I.act >> u) & 1u)) ++u;
@@ -257,9 +272,11 @@ __global__ void __launch_bounds__(kThreads, 2) fwd_kernel(const __grid_constant_
         };
         copy_rows(q0, prm.q, qtok, qvalid, warp, lane);
         cp_async_commit();
-        fill_factor(q1, r, uh + (pi * g.M + pj) * 16, kSqrtD);
+        float4 fq[4], fk[4];
+        load_factor(fq, uh + (pi * g.M + pj) * 16);
         int u = next_kv(0), b = 0, ki = 0, kj = 0;
-        if (u < I.nkv) kv_stage(u, 0, ki, kj);
+        if (u < I.nkv) kv_stage(u, 0, ki, kj, fk);
+        put_factor(q1, r, fq, kSqrtD);
         cp_async_wait<0>();
         __syncwarp();
         prep_row(q0, r, pi, pj, rtab);
@@ -267,63 +284,111 @@ __global__ void __launch_bounds__(kThreads, 2) fwd_kernel(const __grid_constant_
 #pragma unroll
         for (int e = 0; e < 32; ++e) o[e] = 0.f;
         float m = -INFINITY, l = 0.f;
+        bool first = true;
         while (u < I.nkv && ok) {
             const long long kt = I.kv0 + u;
             const int un = next_kv(u + 1);
             const int koff = kKVOff + b * kKVBytes;
+            const uint32_t sb = (tcs & 1u) * kSBuf;
             cp_async_wait<0>();
             __syncwarp();
             prep_row(smem + koff, r, ki, kj, rtab);
+            put_factor(smem + koff + kTileBytes, r, fk, 1.f);
             fence_proxy_async_smem();
-            if (!group_sync(0x6304)) { ok = false; break; }  // every Q~ and K~ row staged
+            if (!group_sync(0x6304)) { ok = false; break; }  // every Q~ and K~ row staged, P V rows read
             if (r == 0) {
                 tc_fence_after();
 #pragma unroll
                 for (int k = 0; k < kHeadDim / 16; ++k)  // q'.k'
-                    umma_ss(tmem + kColS, dK0 + (kQOff >> 4) + 2 * k, dK0 + (koff >> 4) + 2 * k, id_s, k > 0);
+                    umma_ss(tmem + sb, dK0 + (kQOff >> 4) + 2 * k, dK0 + (koff >> 4) + 2 * k, id_s, k > 0);
                 // sqrt(d) U.W: the 16 factor channels only
-                umma_ss(tmem + kColS, dK0 + ((kQOff + kTileBytes) >> 4), dK0 + ((koff + kTileBytes) >> 4), id_s, 1u);
+                umma_ss(tmem + sb, dK0 + ((kQOff + kTileBytes) >> 4), dK0 + ((koff + kTileBytes) >> 4), id_s, 1u);
                 umma_commit(&bars->s_full);
             }
-            // the next tile's rows go to the other buffer, whose products (the
-            // previous tile's) have completed
             int nki = 0, nkj = 0;
-            if (un < I.nkv) kv_stage(un, b ^ 1, nki, nkj);
+            const int nb = b == kKVBufs - 1 ? 0 : b + 1;
+            if (un < I.nkv) kv_stage(un, nb, nki, nkj, fk);
             const uint32_t a16 = I.masked ? d_allow16(g, myseg, kt, I.win) : 0xFFu;
             if (!wwait(&bars->s_full, sph, 0x6305)) { ok = false; break; }
             sph ^= 1;
             tc_fence_after();
-            // row maximum of the attended raw scores
-            float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-#pragma unroll 1
-            for (int c = 0; c < 4; ++c) {
+            const uint32_t t_s = trow + sb;
+            if (!first) {  // the previous tile's P V, complete with this S
                 uint32_t v[32];
-                tmem_ld32(trow + kColS + 32 * c, v);
+                tmem_ld32(trow + (sb ^ kSBuf) + kColO, v);
                 tmem_wait_ld();
 #pragma unroll
-                for (int e = 0; e < 32; ++e)
-                    if (!((a16 >> (2 * c + (e >> 4))) & 1u)) v[e] = __float_as_uint(-INFINITY);
-#pragma unroll
                 for (int e = 0; e < 32; e += 2)
-                    mx4[(e >> 1) & 3] = fmax3(mx4[(e >> 1) & 3], __uint_as_float(v[e]), __uint_as_float(v[e + 1]));
-            }
-            const float m_tile = fmaxf(fmax3(mx4[0], mx4[1], mx4[2]), mx4[3]) * sl2;
-            if (m_tile > m + 8.f) {  // conditional rescale: exact, P stays below 2^8
-                const float alpha = ex2_approx(m - m_tile);
+                    fadd2(o[e], o[e + 1], o[e], o[e + 1], __uint_as_float(v[e]), __uint_as_float(v[e + 1]));
+            } else {
+                // the item's first tile: its row maximum in a pass of its own
+                float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll 1
+                for (int c = 0; c < 4; ++c) {
+                    uint32_t v[32];
+                    tmem_ld32(t_s + 32 * c, v);
+                    tmem_wait_ld();
 #pragma unroll
-                for (int e = 0; e < 32; ++e) o[e] *= alpha;
-                l *= alpha;
-                m = m_tile;
+                    for (int e = 0; e < 32; ++e)
+                        if (!((a16 >> (2 * c + (e >> 4))) & 1u)) v[e] = __float_as_uint(-INFINITY);
+#pragma unroll
+                    for (int e = 0; e < 32; e += 2)
+                        mx4[(e >> 1) & 3] = fmax3(mx4[(e >> 1) & 3], __uint_as_float(v[e]), __uint_as_float(v[e + 1]));
+                }
+                m = fmaxf(fmax3(mx4[0], mx4[1], mx4[2]), mx4[3]) * sl2;  // O and l are zero
             }
-            const float mu = (m == -INFINITY) ? 0.f : m;
+            // Probabilities, row sum and bf16 P in one pass.  After the first tile
+            // each chunk's maximum is checked against the running maximum m; only
+            // when it exceeds m by more than 64 (in log2 units), or m is still
+            // -inf, are m, l, O and the chunks of P already written rescaled.  P
+            // up to 2^64 stays far inside the range of bf16 and of the fp32 sums,
+            // and the softmax is the same.
             float l4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll 1
             for (int c = 0; c < 4; ++c) {
                 uint32_t v[32];
-                tmem_ld32(trow + kColS + 32 * c, v);
+                tmem_ld32(t_s + 32 * c, v);
                 tmem_wait_ld();
-                const float add0 = ((a16 >> (2 * c)) & 1u) ? -mu : -INFINITY;
-                const float add1 = ((a16 >> (2 * c + 1)) & 1u) ? -mu : -INFINITY;
+                const bool ok0 = (a16 >> (2 * c)) & 1u, ok1 = (a16 >> (2 * c + 1)) & 1u;
+                if (!first) {
+                    float c4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+                    if (ok0) {
+#pragma unroll
+                        for (int e = 0; e < 16; e += 2)
+                            c4[(e >> 1) & 1] = fmax3(c4[(e >> 1) & 1], __uint_as_float(v[e]), __uint_as_float(v[e + 1]));
+                    }
+                    if (ok1) {
+#pragma unroll
+                        for (int e = 16; e < 32; e += 2)
+                            c4[2 + ((e >> 1) & 1)] =
+                                fmax3(c4[2 + ((e >> 1) & 1)], __uint_as_float(v[e]), __uint_as_float(v[e + 1]));
+                    }
+                    const float cm = fmaxf(fmaxf(c4[0], c4[1]), fmaxf(c4[2], c4[3])) * sl2;
+                    const bool grow = cm > m + 64.f;
+                    if (__any_sync(0xFFFFFFFFu, grow)) {
+                        const float alpha = grow ? ex2_approx(m - cm) : 1.f;
+                        if (grow) m = cm;
+#pragma unroll
+                        for (int e = 0; e < 32; e += 2) fmul2(o[e], o[e + 1], o[e], o[e + 1], alpha, alpha);
+                        l *= alpha;
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) l4[e] *= alpha;
+                        if (c > 0) tmem_wait_st();
+#pragma unroll 1
+                        for (int k = 0; k < c; ++k) {  // this tile's P chunks already in TMEM
+                            uint32_t pw[16];
+                            tmem_ld16(t_s + kColP + 16 * k, pw);
+                            tmem_wait_ld();
+#pragma unroll
+                            for (int e = 0; e < 16; ++e)
+                                pw[e] = pack_bf16x2(bf16lo_to_f32(pw[e]) * alpha, bf16hi_to_f32(pw[e]) * alpha);
+                            tmem_st16(t_s + kColP + 16 * k, pw);
+                        }
+                    }
+                }
+                const float mu = (m == -INFINITY) ? 0.f : m;
+                const float add0 = ok0 ? -mu : -INFINITY;
+                const float add1 = ok1 ? -mu : -INFINITY;
                 uint32_t w[16];
 #pragma unroll
                 for (int e = 0; e < 16; ++e) {
@@ -335,7 +400,7 @@ __global__ void __launch_bounds__(kThreads, 2) fwd_kernel(const __grid_constant_
                     fadd2(l4[a], l4[a + 1], l4[a], l4[a + 1], p0, p1);
                     w[e] = pack_bf16x2(p0, p1);
                 }
-                tmem_st16(trow + kColP + 16 * c, w);  // over columns of S already read
+                tmem_st16(t_s + kColP + 16 * c, w);  // over columns of S already read
             }
             l += (l4[0] + l4[1]) + (l4[2] + l4[3]);
             tmem_wait_st();
@@ -345,27 +410,30 @@ __global__ void __launch_bounds__(kThreads, 2) fwd_kernel(const __grid_constant_
                 tc_fence_after();
 #pragma unroll
                 for (int k = 0; k < kTile / 16; ++k)
-                    umma_ts(tmem + kColO, tmem + kColP + 8 * k, dMN0 + ((koff + 2 * kTileBytes) >> 4) + 64 * k, id_pv,
-                            k > 0);
-                umma_commit(&bars->o_full);
+                    umma_ts(tmem + sb + kColO, tmem + sb + kColP + 8 * k, dMN0 + ((koff + 2 * kTileBytes) >> 4) + 64 * k,
+                            id_pv, k > 0);
+                if (un >= I.nkv) umma_commit(&bars->o_full);  // the item's last product
             }
-            if (!wwait(&bars->o_full, oph, 0x6307)) { ok = false; break; }
-            oph ^= 1;
-            tc_fence_after();
-            {
-                uint32_t v[32];
-                tmem_ld32(trow + kColO, v);
-                tmem_wait_ld();
-#pragma unroll
-                for (int e = 0; e < 32; ++e) o[e] += __uint_as_float(v[e]);
-            }
-            tc_fence_before();  // ordered before the next tile's products by its group barrier
+            first = false;
+            ++tcs;
             u = un;
-            b ^= 1;
+            b = nb;
             ki = nki;
             kj = nkj;
         }
         if (!ok) break;
+        if (!first) {  // the last tile's P V
+            if (!wwait(&bars->o_full, oph, 0x6307)) break;
+            oph ^= 1;
+            tc_fence_after();
+            uint32_t v[32];
+            tmem_ld32(trow + ((tcs - 1u) & 1u) * kSBuf + kColO, v);
+            tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 32; e += 2)
+                fadd2(o[e], o[e + 1], o[e], o[e + 1], __uint_as_float(v[e]), __uint_as_float(v[e + 1]));
+            tc_fence_before();  // ordered before the next item's products by its group barriers
+        }
         // epilogue: O / l staged over q', coalesced stores, log-sum-exp
         const float inv = 1.f / l;
 #pragma unroll
