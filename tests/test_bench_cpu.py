@@ -137,3 +137,25 @@ def test_cpu_baseline_runs_the_bias_oracle():
     wl = dict(B=1, H=16, W=16, heads=2, M=8, shifts=(4,), qk_scale=1.0, lrbias=True)
     res = bench.cpu_baseline(bench.cpu_stage_inputs(wl), wl, seconds=1.0)
     assert res["value"] > 0 and "8 of 8 at s=4" in res["sample"]
+
+
+def test_traffic_records_are_reported_only_for_the_sources_they_were_taken_on(monkeypatch):
+    """Every stored DRAM-traffic record names a benchmarked workload, an existing
+    kernel source and its ncu summary; bench reports its bytes while the
+    kernel's sources hash to the stored value and null once they differ."""
+    import json
+    import os
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    with open(os.path.join(root, "profiles", "traffic.json")) as fh:
+        recs = json.load(fh)["records"]
+    assert recs
+    for rec in recs:
+        assert rec["workload"] in bench.WORKLOADS
+        assert os.path.exists(os.path.join(root, "vision_transformer_windowed_b200", "csrc", rec["source"]))
+        assert os.path.exists(os.path.join(root, "profiles", rec["summary"]))
+        assert rec["bytes_per_step"] > 0 and len(rec["sources_sha256"]) == 64
+        monkeypatch.setattr(bench, "kernel_sources_sha256", lambda tu, h=rec["sources_sha256"]: h)
+        assert bench.measured_traffic(rec["phase"], rec["workload"]) == rec["bytes_per_step"]
+        monkeypatch.setattr(bench, "kernel_sources_sha256", lambda tu: "0" * 64)
+        assert bench.measured_traffic(rec["phase"], rec["workload"]) is None
+    assert bench.measured_traffic("bwd_main", "no_such_workload") is None
