@@ -159,3 +159,33 @@ def test_traffic_records_are_reported_only_for_the_sources_they_were_taken_on(mo
         monkeypatch.setattr(bench, "kernel_sources_sha256", lambda tu: "0" * 64)
         assert bench.measured_traffic(rec["phase"], rec["workload"]) is None
     assert bench.measured_traffic("bwd_main", "no_such_workload") is None
+
+
+def _run_reference_arm(rank: int, world: int):
+    import json
+    import os
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    env = dict(os.environ, RANK=str(rank), WORLD_SIZE=str(world), LOCAL_RANK=str(rank))
+    out = subprocess.run([sys.executable, os.path.join(root, "bench.py"), "--impl", "reference", "--gpus", str(world),
+                          "--workload", "swin_t_stage1_p4_m8", "--steps", "1", "--warmup", "3",
+                          "--reference-seconds", "4"], capture_output=True, text=True, env=env, cwd=root, timeout=300)
+    assert out.returncode == 0, out.stderr[-2000:]
+    return [json.loads(l) for l in out.stdout.splitlines() if l.strip()]
+
+
+def test_reference_arm_prints_one_line_on_rank_zero_only():
+    """The reference arm (the oracle on the host cores) keeps the bench line's
+    contract: rank 0 prints one JSON line with the same metric and workload as
+    the kernels' arm; the other ranks of a multi-process launch exit 0 silently."""
+    assert _run_reference_arm(1, 2) == []
+    lines = _run_reference_arm(0, 2)
+    assert len(lines) == 1
+    line = lines[0]
+    assert line["impl"] == "reference" and line["metric"] == bench.METRIC and line["n_gpus"] == 2
+    assert line["config"]["workload"] == "swin_t_stage1_p4_m8" and line["steps"] == 1 and line["warmup"] == 3
+    assert line["value"] > 0 and line["cpu_baseline"]["value"] == line["value"]
+    assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["cores"] >= 1
+    assert line["e2e"] == {"value": line["value"], "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                           "d2h_bytes_per_step": 0}
