@@ -58,3 +58,41 @@ def block_forward(x, w_qkv, b_qkv, w_o, b_o, theta, M: int, s: int, heads: int, 
     o = full(q, k, v, theta, M, s, nthreads=nthreads)["o"][:, :H, :W]  # [B, H, W, heads, d]
     of = o.reshape(B, H, W, -1)
     return of @ _f64(w_o).T + _f64(b_o), o
+
+
+def block_backward(x, w_qkv, b_qkv, w_o, b_o, theta, M: int, s: int, heads: int, dy, nthreads: int | None = None):
+    """Gradients of sum(y * dy) for the block's output y, dy [B, H, W, C]:
+    dict of dx [B, H, W, C], dw_qkv [3C, C], db_qkv [3C], dw_o [C, C], db_o [C]
+    and dtheta [heads, 2, d/4], all float64.
+
+    The chain rule through the block's three steps in reverse order: the output
+    map (dW_o = sum over tokens of dy^T o, db_o = sum of dy, do = dy W_o), the
+    attention backward of ``oracle.full`` with do as its upstream gradient, and
+    the qkv map (dqkv = [dq, dk, dv] in the channel order of the forward split,
+    dW_qkv = sum over tokens of dqkv^T x, db_qkv = sum of dqkv, dx = dqkv W_qkv).
+    On a padded grid the padding tokens' outputs are cropped, so their dy is 0;
+    their q, k, v (the bias) still take part in the attention, so their dqkv
+    reaches db_qkv, while x is 0 there and dx is cropped.
+    """
+    x, dy = _f64(x), _f64(dy)
+    w_qkv, w_o = _f64(w_qkv), _f64(w_o)
+    B, H, W, C = x.shape
+    d = C // heads
+    Hp, Wp = -(-H // M) * M, -(-W // M) * M
+    xp = np.zeros((B, Hp, Wp, C))
+    xp[:, :H, :W] = x
+    dyp = np.zeros((B, Hp, Wp, C))
+    dyp[:, :H, :W] = dy
+    q, k, v = project_qkv(xp, w_qkv, b_qkv, heads)
+    dop = (dyp @ w_o).reshape(B, Hp, Wp, heads, d)
+    att = full(q, k, v, theta, M, s, dout=dop, nthreads=nthreads)
+    o = att["o"].reshape(B, Hp, Wp, C)
+    dqkv = np.stack([att["dq"], att["dk"], att["dv"]], axis=3).reshape(B, Hp, Wp, 3 * C)
+    return {
+        "dx": (dqkv @ w_qkv)[:, :H, :W],
+        "dw_qkv": dqkv.reshape(-1, 3 * C).T @ xp.reshape(-1, C),
+        "db_qkv": dqkv.reshape(-1, 3 * C).sum(axis=0),
+        "dw_o": dyp.reshape(-1, C).T @ o.reshape(-1, C),
+        "db_o": dyp.reshape(-1, C).sum(axis=0),
+        "dtheta": att["dtheta"],
+    }
